@@ -1,0 +1,273 @@
+"""fp64 CPU oracle for the Wan-style causal Conv3D and residual block.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product library imports this
+package; only the tests, the smoke check and the benchmark's CPU-baseline leg
+use it.  It shares no code with the CUDA library.
+
+The arithmetic lives in ``cc3d_oracle.c`` (plain C, fp64, OpenMP).  This
+module compiles it with gcc on first use (or from ``build()``) and marshals
+numpy / torch CPU arrays into it.  All tensors use the pages' logical layout
+[B, C, T, H, W] ("Cosmos3 Wan VAE -- engine size vs context memory",
+§10.1); a caller holding channels-last data passes a permuted view and the
+strides carry the layout.
+
+Functions (each cites the passage it follows in the C source):
+  causal_conv3d         -- §10.3 WanCausalConv3d, bias once
+  causal_conv3d_points  -- the same definition at chosen output voxels
+  rms_norm              -- §10.2 WanRMS_norm (+ optional SiLU, §10.4)
+  resblock              -- §10.4 WanResidualBlock, identity shortcut
+  resblock_points       -- the same definition at chosen output voxels
+  round_bf16            -- bfloat16 round-to-nearest-even of one double
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "cc3d_oracle.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD_DIR, "libcc3d_oracle.so")
+
+_lock = threading.Lock()
+_lib = None
+
+F64, F32, BF16 = 0, 1, 2
+
+
+class _Tensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int),
+                ("stride", ctypes.c_longlong * 5)]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into oracle/_build/libcc3d_oracle.so."""
+    os.makedirs(_BUILD_DIR, exist_ok=True)
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+           "-Wall", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.POINTER
+            T = P(_Tensor)
+            dp = P(ctypes.c_double)
+            ip = P(ctypes.c_int)
+            i = ctypes.c_int
+            lib.orc_causal_conv3d.argtypes = [T, T, i, i, i, i, i, T, i, i, i, i, i, i, dp, dp]
+            lib.orc_causal_conv3d_points.argtypes = [T, T, i, i, i, i, i, T, i, i, i, i, i, i, dp,
+                                                     i, ip, dp]
+            lib.orc_rms_norm.argtypes = [T, i, i, i, i, i, dp, dp, i, dp]
+            lib.orc_resblock.argtypes = [T, T, T, i, i, i, i, i, T, dp, dp, T, dp, dp, i, dp, dp, dp]
+            lib.orc_resblock_points.argtypes = [T, T, T, i, i, i, i, i, T, dp, dp, T, dp, dp, i,
+                                                i, ip, dp]
+            lib.orc_round_bf16.argtypes = [ctypes.c_double]
+            lib.orc_round_bf16.restype = ctypes.c_double
+            lib.orc_silu.argtypes = [ctypes.c_double]
+            lib.orc_silu.restype = ctypes.c_double
+            for name in ("orc_causal_conv3d", "orc_causal_conv3d_points", "orc_rms_norm",
+                         "orc_resblock", "orc_resblock_points"):
+                getattr(lib, name).restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _view(a, keep):
+    """Describe a 5-D array (numpy, or torch CPU tensor of float64/float32/
+    bfloat16) as an oracle tensor.  Logical dims are (n, c, t, h, w); the
+    array's own strides carry the memory layout."""
+    if a is None:
+        return None
+    try:
+        import torch
+    except ImportError:  # pragma: no cover
+        torch = None
+    if torch is not None and isinstance(a, torch.Tensor):
+        assert a.device.type == "cpu", "oracle inputs live in host memory"
+        assert a.dim() == 5
+        if a.dtype == torch.bfloat16:
+            dt = BF16
+        elif a.dtype == torch.float32:
+            dt = F32
+        elif a.dtype == torch.float64:
+            dt = F64
+        else:
+            raise TypeError(f"unsupported dtype {a.dtype}")
+        keep.append(a)
+        st = _Tensor()
+        st.data = a.data_ptr()
+        st.dtype = dt
+        for k in range(5):
+            st.stride[k] = a.stride(k)
+        return st
+    a = np.asarray(a)
+    assert a.ndim == 5
+    if a.dtype == np.float64:
+        dt = F64
+    elif a.dtype == np.float32:
+        dt = F32
+    elif a.dtype == np.uint16:
+        dt = BF16
+    else:
+        raise TypeError(f"unsupported dtype {a.dtype}")
+    keep.append(a)
+    st = _Tensor()
+    st.data = a.ctypes.data
+    st.dtype = dt
+    for k in range(5):
+        st.stride[k] = a.strides[k] // a.itemsize
+    return st
+
+
+def _ptr(st):
+    return ctypes.byref(st) if st is not None else None
+
+
+def _dvec(v, keep):
+    if v is None:
+        return None
+    v = np.ascontiguousarray(np.asarray(v, dtype=np.float64).reshape(-1))
+    keep.append(v)
+    return v.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _shape5(a):
+    return tuple(int(s) for s in a.shape)
+
+
+def causal_conv3d(x, weight, bias=None, cache=None, pad=(1, 1)):
+    """y[n,co,t,h,w] = b[co] + sum_{ci,kt,kh,kw} W[co,ci,kt,kh,kw] *
+    xt[n,ci,t+kt,h+kh-pad_h,w+kw-pad_w], xt = concat(cache or zeros, x) on t.
+    x: [N,Cin,T,H,W]; weight: [Cout,Cin,KT,KH,KW]; cache: [N,Cin,KT-1,H,W]
+    or None.  Returns float64 [N,Cout,T,H,W]."""
+    lib = _load()
+    keep = []
+    N, Cin, T, H, W = _shape5(x)
+    Cout, Cin2, KT, KH, KW = _shape5(weight)
+    assert Cin2 == Cin
+    if cache is not None:
+        assert _shape5(cache) == (N, Cin, KT - 1, H, W)
+    tx, tc, tw = _view(x, keep), _view(cache, keep), _view(weight, keep)
+    y = np.empty((N, Cout, T, H, W), dtype=np.float64)
+    rc = lib.orc_causal_conv3d(_ptr(tx), _ptr(tc), N, Cin, T, H, W, _ptr(tw), Cout, KT, KH, KW,
+                               pad[0], pad[1], _dvec(bias, keep),
+                               y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc != 0:
+        raise ValueError(f"orc_causal_conv3d failed ({rc})")
+    return y
+
+
+def _pts(points, keep):
+    p = np.ascontiguousarray(np.asarray(points, dtype=np.int32).reshape(-1, 4))
+    keep.append(p)
+    return p.shape[0], p.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+
+
+def causal_conv3d_points(x, weight, bias, cache, points, pad=(1, 1)):
+    """The causal Conv3D at the output voxels in ``points`` (rows n,t,h,w).
+    Returns float64 [P, Cout]."""
+    lib = _load()
+    keep = []
+    N, Cin, T, H, W = _shape5(x)
+    Cout, _, KT, KH, KW = _shape5(weight)
+    tx, tc, tw = _view(x, keep), _view(cache, keep), _view(weight, keep)
+    P, pp = _pts(points, keep)
+    y = np.empty((P, Cout), dtype=np.float64)
+    rc = lib.orc_causal_conv3d_points(_ptr(tx), _ptr(tc), N, Cin, T, H, W, _ptr(tw), Cout, KT, KH,
+                                      KW, pad[0], pad[1], _dvec(bias, keep), P, pp,
+                                      y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc != 0:
+        raise ValueError(f"orc_causal_conv3d_points failed ({rc})")
+    return y
+
+
+def rms_norm(x, gamma, beta=None, silu=False):
+    """Channel RMS_norm over C (+ SiLU).  Returns float64 [N,C,T,H,W]."""
+    lib = _load()
+    keep = []
+    N, C, T, H, W = _shape5(x)
+    tx = _view(x, keep)
+    y = np.empty((N, C, T, H, W), dtype=np.float64)
+    rc = lib.orc_rms_norm(_ptr(tx), N, C, T, H, W, _dvec(gamma, keep), _dvec(beta, keep),
+                          1 if silu else 0, y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc != 0:
+        raise ValueError(f"orc_rms_norm failed ({rc})")
+    return y
+
+
+def resblock(x, w1, b1, g1, w2, b2, g2, cache1=None, cache2=None, round_bf16=True,
+             return_acts=False):
+    """WanResidualBlock (identity shortcut).  Returns y float64 [N,C,T,H,W]
+    (and a0, a1 when return_acts)."""
+    lib = _load()
+    keep = []
+    N, C, T, H, W = _shape5(x)
+    tx, t1, t2 = _view(x, keep), _view(cache1, keep), _view(cache2, keep)
+    tw1, tw2 = _view(w1, keep), _view(w2, keep)
+    y = np.empty((N, C, T, H, W), dtype=np.float64)
+    a0 = np.empty_like(y) if return_acts else None
+    a1 = np.empty_like(y) if return_acts else None
+    dp = ctypes.POINTER(ctypes.c_double)
+    rc = lib.orc_resblock(_ptr(tx), _ptr(t1), _ptr(t2), N, C, T, H, W,
+                          _ptr(tw1), _dvec(b1, keep), _dvec(g1, keep),
+                          _ptr(tw2), _dvec(b2, keep), _dvec(g2, keep),
+                          1 if round_bf16 else 0, y.ctypes.data_as(dp),
+                          a0.ctypes.data_as(dp) if a0 is not None else None,
+                          a1.ctypes.data_as(dp) if a1 is not None else None)
+    if rc != 0:
+        raise ValueError(f"orc_resblock failed ({rc})")
+    return (y, a0, a1) if return_acts else y
+
+
+def resblock_points(x, w1, b1, g1, w2, b2, g2, points, cache1=None, cache2=None,
+                    round_bf16=True):
+    """The residual block at chosen output voxels.  Returns float64 [P, C]."""
+    lib = _load()
+    keep = []
+    N, C, T, H, W = _shape5(x)
+    tx, t1, t2 = _view(x, keep), _view(cache1, keep), _view(cache2, keep)
+    tw1, tw2 = _view(w1, keep), _view(w2, keep)
+    P, pp = _pts(points, keep)
+    y = np.empty((P, C), dtype=np.float64)
+    rc = lib.orc_resblock_points(_ptr(tx), _ptr(t1), _ptr(t2), N, C, T, H, W,
+                                 _ptr(tw1), _dvec(b1, keep), _dvec(g1, keep),
+                                 _ptr(tw2), _dvec(b2, keep), _dvec(g2, keep),
+                                 1 if round_bf16 else 0, P, pp,
+                                 y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc != 0:
+        raise ValueError(f"orc_resblock_points failed ({rc})")
+    return y
+
+
+def round_bf16(v: float) -> float:
+    return _load().orc_round_bf16(float(v))
+
+
+def silu(z: float) -> float:
+    return _load().orc_silu(float(z))
+
+
+def round_bf16_array(a):
+    """Elementwise bfloat16 RNE of a float64 array (loops over round_bf16;
+    meant for small arrays)."""
+    lib = _load()
+    a = np.asarray(a, dtype=np.float64)
+    out = np.empty_like(a)
+    flat_in, flat_out = a.reshape(-1), out.reshape(-1)
+    for k in range(flat_in.size):
+        flat_out[k] = lib.orc_round_bf16(float(flat_in[k]))
+    return out

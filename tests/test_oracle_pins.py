@@ -1,0 +1,404 @@
+"""Pins for the fp64 CPU oracle (no GPU).
+
+The oracle is checked against things other than itself:
+  * a library special case: torch's float64 conv3d on an explicitly padded
+    input (zero frames or the cache in front of t, spatial zeros);
+  * a second brute force written here: explicit padded copy, then a dense
+    3-D correlation with numpy windows;
+  * the per-temporal-slice algebra of the "cache-aware video decoder
+    lowering" summary (one Conv2D per kernel time slice, summed, bias once);
+  * k_t = 1 reducing to a per-frame Conv2D;
+  * the impulse response (pins orientation and the causal time shift);
+  * the invariants the pages state: causality, chunked streaming with a
+    2-frame cache equal to whole-sequence evaluation, bias added once,
+    linearity in x;
+  * closed forms for RMS_norm, SiLU and bf16 rounding;
+  * a hand-worked example under tests/golden/.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from video_vae_causal_implicit_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rnd(shape, seed, scale=1.0):
+    g = np.random.default_rng(seed)
+    return g.standard_normal(shape) * scale
+
+
+def torch_causal_conv3d(x, w, b, cache=None, pad=(1, 1)):
+    """Library special case: F.pad + conv3d in float64."""
+    x = torch.from_numpy(np.ascontiguousarray(x))
+    w = torch.from_numpy(np.ascontiguousarray(w))
+    kt = w.shape[2]
+    if cache is not None:
+        xt = torch.cat([torch.from_numpy(np.ascontiguousarray(cache)), x], dim=2)
+        xt = F.pad(xt, (pad[1], pad[1], pad[0], pad[0], 0, 0))
+    else:
+        xt = F.pad(x, (pad[1], pad[1], pad[0], pad[0], kt - 1, 0))
+    bb = torch.from_numpy(np.asarray(b)) if b is not None else None
+    return F.conv3d(xt, w, bb).numpy()
+
+
+def numpy_padded_correlation(x, w, b, cache=None):
+    """Brute force 2: materialise the padded input, then correlate."""
+    N, Ci, T, H, W = x.shape
+    Co, _, KT, KH, KW = w.shape
+    front = cache if cache is not None else np.zeros((N, Ci, KT - 1, H, W))
+    xt = np.concatenate([front, x], axis=2)
+    xt = np.pad(xt, ((0, 0), (0, 0), (0, 0), (KH // 2, KH // 2), (KW // 2, KW // 2)))
+    y = np.zeros((N, Co, T, H, W))
+    for t in range(T):
+        for h in range(H):
+            for ww in range(W):
+                patch = xt[:, :, t:t + KT, h:h + KH, ww:ww + KW]  # N,Ci,KT,KH,KW
+                y[:, :, t, h, ww] = np.einsum("nijkl,oijkl->no", patch, w)
+    return y + (0 if b is None else np.asarray(b)[None, :, None, None, None])
+
+
+def per_slice_conv2d(x, w, b):
+    """Per-temporal-slice lowering: for each kernel time slice kt, one Conv2D
+    over the frames it reads (tau = t + kt - 2; frames before 0 are zero and
+    contribute nothing), summed over kt; bias once at the end."""
+    N, Ci, T, H, W = x.shape
+    Co, _, KT, KH, KW = w.shape
+    y = torch.zeros((N, Co, T, H, W), dtype=torch.float64)
+    xt = torch.from_numpy(x)
+    for kt in range(KT):
+        shift = KT - 1 - kt  # output t reads frame t - shift
+        if shift >= T:
+            continue
+        frames = xt[:, :, : T - shift]  # frames 0 .. T-shift-1 feed outputs shift .. T-1
+        batch = frames.permute(0, 2, 1, 3, 4).reshape(-1, Ci, H, W)
+        out = F.conv2d(batch, torch.from_numpy(w[:, :, kt]), padding=(KH // 2, KW // 2))
+        out = out.reshape(N, T - shift, Co, H, W).permute(0, 2, 1, 3, 4)
+        y[:, :, shift:] += out
+    return (y + torch.from_numpy(np.asarray(b))[None, :, None, None, None]).numpy()
+
+
+SHAPES = [
+    (1, 3, 4, 2, 5, 6),
+    (2, 4, 3, 3, 4, 3),
+    (1, 8, 8, 4, 6, 6),
+    (1, 2, 5, 1, 1, 1),
+    (1, 5, 2, 6, 3, 7),
+]
+
+
+@pytest.mark.parametrize("N,Ci,Co,T,H,W", SHAPES)
+def test_conv_matches_torch_fp64(N, Ci, Co, T, H, W):
+    x = rnd((N, Ci, T, H, W), 1)
+    w = rnd((Co, Ci, 3, 3, 3), 2, 0.3)
+    b = rnd((Co,), 3, 0.1)
+    y = oracle.causal_conv3d(x, w, b)
+    ref = torch_causal_conv3d(x, w, b)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("N,Ci,Co,T,H,W", SHAPES[:3])
+def test_conv_with_cache_matches_torch_fp64(N, Ci, Co, T, H, W):
+    x = rnd((N, Ci, T, H, W), 4)
+    cache = rnd((N, Ci, 2, H, W), 5)
+    w = rnd((Co, Ci, 3, 3, 3), 6, 0.3)
+    b = rnd((Co,), 7, 0.1)
+    y = oracle.causal_conv3d(x, w, b, cache=cache)
+    np.testing.assert_allclose(y, torch_causal_conv3d(x, w, b, cache=cache), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(y, numpy_padded_correlation(x, w, b, cache), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("N,Ci,Co,T,H,W", SHAPES)
+def test_conv_matches_padded_copy_and_per_slice(N, Ci, Co, T, H, W):
+    x = rnd((N, Ci, T, H, W), 8)
+    w = rnd((Co, Ci, 3, 3, 3), 9, 0.3)
+    b = rnd((Co,), 10, 0.1)
+    y = oracle.causal_conv3d(x, w, b)
+    np.testing.assert_allclose(y, numpy_padded_correlation(x, w, b), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(y, per_slice_conv2d(x, w, b), rtol=1e-12, atol=1e-12)
+
+
+def test_kt1_is_per_frame_conv2d():
+    x = rnd((1, 4, 3, 5, 6), 11)
+    w = rnd((6, 4, 1, 3, 3), 12, 0.3)
+    b = rnd((6,), 13)
+    y = oracle.causal_conv3d(x, w, b)
+    for t in range(3):
+        ref = F.conv2d(torch.from_numpy(x[:, :, t]), torch.from_numpy(w[:, :, 0]),
+                       torch.from_numpy(b), padding=1).numpy()
+        np.testing.assert_allclose(y[:, :, t], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_impulse_response_pins_orientation_and_causal_shift():
+    Ci, Co, T, H, W = 2, 3, 5, 5, 5
+    w = rnd((Co, Ci, 3, 3, 3), 14)
+    b = rnd((Co,), 15)
+    ci, t0, h0, w0 = 1, 1, 2, 2
+    x = np.zeros((1, Ci, T, H, W))
+    x[0, ci, t0, h0, w0] = 1.0
+    y = oracle.causal_conv3d(x, w, None)
+    yb = oracle.causal_conv3d(x, w, b)
+    np.testing.assert_allclose(yb - y, np.broadcast_to(b[None, :, None, None, None], y.shape),
+                               rtol=0, atol=1e-15)
+    for kt in range(3):
+        for kh in range(3):
+            for kw in range(3):
+                # y[t] reads frame t + kt - 2, so the impulse at t0 reaches
+                # output t0 + 2 - kt; rows/cols likewise with pad 1.
+                t, h, ww = t0 + 2 - kt, h0 + 1 - kh, w0 + 1 - kw
+                if t < T:
+                    np.testing.assert_array_equal(y[0, :, t, h, ww], w[:, ci, kt, kh, kw])
+    # nothing before t0, nothing beyond t0 + 2
+    assert np.all(y[0, :, :t0] == 0.0)
+    assert np.all(y[0, :, t0 + 3:] == 0.0)
+
+
+def test_causality_future_frames_do_not_leak():
+    x = rnd((1, 3, 6, 4, 5), 16)
+    w = rnd((4, 3, 3, 3, 3), 17)
+    b = rnd((4,), 18)
+    y = oracle.causal_conv3d(x, w, b)
+    for t0 in range(6):
+        x2 = x.copy()
+        x2[:, :, t0] += rnd((1, 3, 4, 5), 100 + t0)
+        y2 = oracle.causal_conv3d(x2, w, b)
+        np.testing.assert_array_equal(y2[:, :, :t0], y[:, :, :t0])
+        assert np.any(y2[:, :, t0] != y[:, :, t0])
+
+
+@pytest.mark.parametrize("chunk", [1, 2, 3])
+def test_streaming_equals_whole_sequence_bitwise(chunk):
+    T = 7
+    x = rnd((1, 3, T, 4, 5), 19)
+    w = rnd((4, 3, 3, 3, 3), 20)
+    b = rnd((4,), 21)
+    whole = oracle.causal_conv3d(x, w, b)
+    cache = None
+    outs = []
+    for s in range(0, T, chunk):
+        xc = x[:, :, s:s + chunk]
+        outs.append(oracle.causal_conv3d(xc, w, b, cache=cache))
+        # next cache: last 2 frames of concat(cache or zeros, chunk)
+        prev = cache if cache is not None else np.zeros((1, 3, 2, 4, 5))
+        cache = np.ascontiguousarray(np.concatenate([prev, xc], axis=2)[:, :, -2:])
+    np.testing.assert_array_equal(np.concatenate(outs, axis=2), whole)
+
+
+def test_zero_cache_equals_no_cache_bitwise():
+    x = rnd((1, 3, 3, 4, 4), 22)
+    w = rnd((2, 3, 3, 3, 3), 23)
+    b = rnd((2,), 24)
+    np.testing.assert_array_equal(oracle.causal_conv3d(x, w, b),
+                                  oracle.causal_conv3d(x, w, b, cache=np.zeros((1, 3, 2, 4, 4))))
+
+
+def test_bias_added_once_and_linearity():
+    x1 = rnd((1, 3, 4, 4, 5), 25)
+    x2 = rnd((1, 3, 4, 4, 5), 26)
+    w = rnd((4, 3, 3, 3, 3), 27)
+    b = rnd((4,), 28)
+    y0 = oracle.causal_conv3d(np.zeros_like(x1), w, b)
+    np.testing.assert_array_equal(y0, np.broadcast_to(b[None, :, None, None, None], y0.shape))
+    f = lambda x: oracle.causal_conv3d(x, w, b) - y0  # noqa: E731
+    a, c = 0.7, -1.9
+    np.testing.assert_allclose(f(a * x1 + c * x2), a * f(x1) + c * f(x2), rtol=1e-12, atol=1e-12)
+    # bias twice (once per temporal slice) would break this:
+    np.testing.assert_allclose(oracle.causal_conv3d(x1, w, None) + b[None, :, None, None, None],
+                               oracle.causal_conv3d(x1, w, b), rtol=0, atol=1e-13)
+
+
+def test_points_equal_full_conv_bitwise():
+    x = rnd((2, 3, 4, 5, 6), 29)
+    cache = rnd((2, 3, 2, 5, 6), 30)
+    w = rnd((4, 3, 3, 3, 3), 31)
+    b = rnd((4,), 32)
+    y = oracle.causal_conv3d(x, w, b, cache=cache)
+    pts = np.array([[0, 0, 0, 0], [1, 3, 4, 5], [0, 1, 2, 3], [1, 0, 4, 0], [0, 2, 0, 5]])
+    yp = oracle.causal_conv3d_points(x, w, b, cache, pts)
+    for k, (n, t, h, ww) in enumerate(pts):
+        np.testing.assert_array_equal(yp[k], y[n, :, t, h, ww])
+
+
+def test_strided_bf16_view_reads_channels_last():
+    """The oracle reads a channels-last bf16 buffer through a permuted view
+    exactly as it reads the same values in NCTHW float64."""
+    case = synth.conv_case(4, 5, 3, 4, 6)
+    x_cl = synth.ndhwc(case["x"])
+    y_view = oracle.causal_conv3d(synth.ncthw_view(x_cl), case["w"], case["b"].double().numpy())
+    y_f64 = oracle.causal_conv3d(case["x"].double().numpy(), case["w"].double().numpy(),
+                                 case["b"].double().numpy())
+    np.testing.assert_array_equal(y_view, y_f64)
+
+
+# ---- RMS_norm, SiLU, bf16 rounding -------------------------------------------
+
+def test_rms_norm_closed_forms():
+    C = 6
+    g = np.linspace(0.5, 1.5, C)
+    x = rnd((1, C, 2, 3, 4), 33)
+    r = oracle.rms_norm(x, g)
+    # || r / gamma ||_2 = sqrt(C) at every voxel
+    nrm = np.sqrt(((r / g[None, :, None, None, None]) ** 2).sum(axis=1))
+    np.testing.assert_allclose(nrm, math.sqrt(C), rtol=1e-13)
+    # invariant to positive scaling of the channel vector
+    np.testing.assert_allclose(oracle.rms_norm(3.7 * x, g), r, rtol=1e-13, atol=1e-15)
+    # one-hot v = a e_k  ->  r = sqrt(C) gamma_k e_k (sign of a)
+    oh = np.zeros((1, C, 1, 1, 1))
+    oh[0, 2] = -4.0
+    ro = oracle.rms_norm(oh, g)[0, :, 0, 0, 0]
+    exp = np.zeros(C)
+    exp[2] = -math.sqrt(C) * g[2]
+    np.testing.assert_allclose(ro, exp, rtol=1e-15, atol=0)
+    # zero vector -> 0 (denominator floored at 1e-12), SiLU(0) = 0
+    z = oracle.rms_norm(np.zeros((1, C, 1, 1, 1)), g, silu=True)
+    assert np.all(z == 0.0)
+    # beta is added after the scale
+    beta = np.arange(C) * 0.25
+    np.testing.assert_allclose(oracle.rms_norm(x, g, beta), r + beta[None, :, None, None, None],
+                               rtol=1e-14, atol=1e-14)
+
+
+def test_rms_norm_matches_torch_normalize():
+    C = 8
+    x = rnd((2, C, 3, 2, 2), 34)
+    g = rnd((C,), 35)
+    ref = F.normalize(torch.from_numpy(x), dim=1).numpy() * math.sqrt(C) * g[None, :, None, None, None]
+    np.testing.assert_allclose(oracle.rms_norm(x, g), ref, rtol=1e-13, atol=1e-14)
+    ref_silu = F.silu(torch.from_numpy(ref)).numpy()
+    np.testing.assert_allclose(oracle.rms_norm(x, g, silu=True), ref_silu, rtol=1e-13, atol=1e-14)
+
+
+def test_silu_closed_forms():
+    assert oracle.silu(0.0) == 0.0
+    assert abs(oracle.silu(1.0) - 1.0 / (1.0 + math.exp(-1.0))) < 1e-16
+    for z in (-7.5, -1.0, -1e-3, 0.25, 3.0, 20.0):
+        assert abs((oracle.silu(z) - oracle.silu(-z)) - z) < 1e-14 * max(1.0, abs(z))
+    assert abs(oracle.silu(-40.0)) < 1e-15
+
+
+def test_round_bf16_ties_and_library_case():
+    r = oracle.round_bf16
+    assert r(1.0) == 1.0
+    assert r(1.0 + 2.0 ** -8) == 1.0                      # tie -> even (mantissa 0)
+    assert r(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6      # tie -> even (mantissa 2)
+    assert r(1.0 + 2.0 ** -8 + 2.0 ** -30) == 1.0 + 2.0 ** -7
+    assert r(-3.0) == -3.0
+    assert r(2.0 ** -140) == 0.0
+    assert r(2.0 ** -133) == 2.0 ** -133
+    assert math.isinf(r(3.5e38))
+    # library special case: torch's fp32 -> bf16 cast is RNE too
+    v = torch.randn(4096, dtype=torch.float64, generator=torch.Generator().manual_seed(5)) * 10
+    v32 = v.float()
+    ref = v32.to(torch.bfloat16).double().numpy()
+    got = oracle.round_bf16_array(v32.double().numpy())
+    np.testing.assert_array_equal(got, ref)
+
+
+# ---- residual block -----------------------------------------------------------
+
+def _block_small(C=8, T=4, H=5, W=6, seed=0):
+    return synth.block_case(C, T, H, W, seed_base=seed)
+
+
+def _np(t):
+    return t.double().numpy()
+
+
+def test_block_is_composition_of_pinned_parts():
+    c = _block_small()
+    y, a0, a1 = oracle.resblock(c["x"], c["w1"], _np(c["b1"]), _np(c["g1"]), c["w2"], _np(c["b2"]),
+                                _np(c["g2"]), return_acts=True)
+    # rebuild with torch fp64 ops: normalize*sqrt(C)*gamma, silu, bf16 RNE, conv
+    x = c["x"].double()
+    C = x.shape[1]
+
+    def rs(v, g):
+        return F.silu(F.normalize(v, dim=1) * math.sqrt(C) * g.double()[None, :, None, None, None])
+
+    a0_ref = rs(x, c["g1"]).float().to(torch.bfloat16).double()
+    # double->float->bf16 can double-round; compare with tolerance of 1 bf16 ulp
+    np.testing.assert_allclose(a0, a0_ref.numpy(), rtol=2 ** -7, atol=1e-30)
+    a0t = torch.from_numpy(a0)
+    h1 = torch.from_numpy(torch_causal_conv3d(a0t.numpy(), _np(c["w1"]), _np(c["b1"])))
+    a1_ref = rs(h1, c["g2"]).numpy()
+    np.testing.assert_allclose(a1, oracle.round_bf16_array(a1_ref), rtol=0, atol=0)
+    y_ref = torch_causal_conv3d(a1, _np(c["w2"]), _np(c["b2"])) + x.numpy()
+    np.testing.assert_allclose(y, y_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_block_identity_when_conv2_is_zero():
+    c = _block_small(seed=3)
+    y = oracle.resblock(c["x"], c["w1"], _np(c["b1"]), _np(c["g1"]), torch.zeros_like(c["w2"]),
+                        np.zeros(8), _np(c["g2"]))
+    np.testing.assert_array_equal(y, _np(c["x"]))
+
+
+def test_block_points_equal_full_block_bitwise():
+    c = _block_small(C=6, T=4, H=5, W=5, seed=7)
+    cache1 = synth.normal((1, 6, 2, 5, 5), 90)
+    cache2 = synth.normal((1, 6, 2, 5, 5), 91)
+    args = (c["x"], c["w1"], _np(c["b1"]), _np(c["g1"]), c["w2"], _np(c["b2"]), _np(c["g2"]))
+    for c1, c2 in ((None, None), (cache1, cache2)):
+        y = oracle.resblock(*args, cache1=c1, cache2=c2)
+        pts = np.array([[0, 0, 0, 0], [0, 3, 4, 4], [0, 1, 2, 3], [0, 2, 0, 4], [0, 0, 4, 1]])
+        yp = oracle.resblock_points(*args, pts, cache1=c1, cache2=c2)
+        for k, (n, t, h, w) in enumerate(pts):
+            np.testing.assert_array_equal(yp[k], y[n, :, t, h, w])
+
+
+def test_block_streaming_equals_whole():
+    """Chunked block with per-conv 2-frame caches (a0 history for conv1, a1
+    history for conv2) equals the whole-sequence block, bitwise."""
+    C, T, H, W = 4, 5, 4, 4
+    c = _block_small(C=C, T=T, H=H, W=W, seed=11)
+    args = (_np(c["w1"]), _np(c["b1"]), _np(c["g1"]), _np(c["w2"]), _np(c["b2"]), _np(c["g2"]))
+    x = _np(c["x"])
+    whole, a0, a1 = oracle.resblock(x, *args[:3], *args[3:], return_acts=True)
+    outs = []
+    c1 = c2 = None
+    for s in range(T):
+        xc = np.ascontiguousarray(x[:, :, s:s + 1])
+        outs.append(oracle.resblock(xc, *args, cache1=c1, cache2=c2))
+        c1 = np.ascontiguousarray(a0[:, :, max(0, s - 1):s + 1]) if s >= 1 else np.concatenate(
+            [np.zeros((1, C, 1, H, W)), a0[:, :, :1]], axis=2)
+        c2 = np.ascontiguousarray(a1[:, :, max(0, s - 1):s + 1]) if s >= 1 else np.concatenate(
+            [np.zeros((1, C, 1, H, W)), a1[:, :, :1]], axis=2)
+    np.testing.assert_array_equal(np.concatenate(outs, axis=2), whole)
+
+
+# ---- hand-worked example --------------------------------------------------------
+
+def _read_golden(name):
+    vals = {}
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            key, val = line.split("=")
+            vals[key.strip()] = [float(v) for v in val.split()]
+    return vals
+
+
+def test_golden_hand_worked_ones():
+    g = _read_golden("causal_ones_T3_H2_W3.txt")
+    T, H, W = 3, 2, 3
+    x = np.ones((1, 1, T, H, W))
+    w = np.ones((1, 1, 3, 3, 3))
+    y = oracle.causal_conv3d(x, w, np.array([0.5]))
+    np.testing.assert_array_equal(y.reshape(-1), np.array(g["y"]))
+
+
+def test_golden_hand_worked_ramp_kernel():
+    g = _read_golden("causal_timeramp_T4.txt")
+    x = np.array(g["x"]).reshape(1, 1, 4, 1, 1)
+    w = np.zeros((1, 1, 3, 3, 3))
+    w[0, 0, :, 1, 1] = g["w_t"]
+    y = oracle.causal_conv3d(x, w, np.array(g["b"]))
+    np.testing.assert_array_equal(y.reshape(-1), np.array(g["y"]))
