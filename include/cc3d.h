@@ -1,0 +1,195 @@
+/*
+ * cc3d.h -- C ABI of libcc3d.so: the Wan-style causal Conv3D
+ * (WanCausalConv3d) and the residual block built around it, for NVIDIA
+ * B200 (sm_100a).
+ *
+ * What is computed
+ * ----------------
+ * Causal Conv3D ("Cosmos3 Wan VAE -- engine size vs context memory",
+ * §10.3, WanCausalConv3d, "causal padding"):
+ *
+ *   y[n,t,h,w,co] = b[co] + sum_{ci,kt,kh,kw} W[co,ci,kt,kh,kw] *
+ *                   xt[n, t+kt, h+kh-pad_h, w+kw-pad_w, ci]
+ *
+ * where xt = concat(cache_in, x) along t and cache_in holds the kt-1 frames
+ * before this chunk (zeros when cache_in is NULL: the causal front pad).
+ * Spatially out-of-range reads are zero.  Stride 1, dilation 1, one group.
+ * The bias is added once, after all taps ("cache-aware video decoder
+ * lowering" summary, the section on per-slice Conv2D: bias after the sum).
+ * Chunked evaluation that carries cache_out into the next call's cache_in
+ * gives the same outputs as one whole-sequence call (§10.3, cache_x
+ * concatenated in front of t; §8.5, CACHE_T = 2).
+ *
+ * RMS_norm + SiLU (§10.2 WanRMS_norm, §10.4 SiLU):
+ *   a[v,c] = SiLU( x[v,c] / max(||x[v,:]||_2, 1e-12) * sqrt(C) * gamma[c]
+ *                  (+ beta[c]) ),  computed in fp32, rounded once to bf16.
+ *
+ * Residual block (§10.4 WanResidualBlock, C_in == C_out, identity
+ * shortcut, dropout = identity at inference):
+ *   a0 = RMS_SiLU(x; g1);  a1 = RMS_SiLU(conv1(a0) + b1; g2);
+ *   y  = conv2(a1) + b2 + x.
+ *
+ * Layout
+ * ------
+ * Activations are channels-last NDHWC ([N][T][H][W][C], C fastest), bf16
+ * (fp32 for CC3D_FP32 plans).  Caches are [N][kt-1][H][W][C] in the same
+ * dtype.  A caller holding NCTHW tensors permutes them first.
+ *
+ * Conventions
+ * -----------
+ *  - Every pointer argument named x, y, cache*, residual, weight, bias,
+ *    gamma, beta is a DEVICE pointer on the current device.  The caller owns
+ *    all of them; plans and blocks copy what they keep.
+ *  - Calls are stream-ordered and asynchronous.  A validation error returns
+ *    before anything is launched.  Device-side waits are bounded: a wait
+ *    that runs out sets a device status word that cc3d_sync_status()
+ *    reports as CC3D_ERR_TIMEOUT (kernels never trap).
+ *  - Activation pointers must be 16-byte aligned.  cache_out must not
+ *    overlap cache_in, x or y (CC3D_ERR_ALIAS); callers ping-pong two cache
+ *    buffers.
+ *  - There is no CPU fallback.  A descriptor the kernels do not cover
+ *    returns CC3D_ERR_UNSUPPORTED, and the plan's counters record which
+ *    kernel served each call.
+ */
+#ifndef CC3D_H_
+#define CC3D_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CC3D_OK = 0,
+  CC3D_ERR_INVALID_ARG = 1,  /* null pointer, bad size, t out of [1, max_t] */
+  CC3D_ERR_UNSUPPORTED = 2,  /* stride/dilation/groups != 1, channel counts or
+                                kernel sizes no kernel covers, no sm_100 GPU */
+  CC3D_ERR_ALIGNMENT = 3,    /* pointer not 16-byte aligned */
+  CC3D_ERR_ALIAS = 4,        /* cache_out overlaps cache_in, x or y */
+  CC3D_ERR_OOM = 5,          /* device allocation failed in a create call */
+  CC3D_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed */
+  CC3D_ERR_TIMEOUT = 7       /* a device-side bounded wait ran out */
+} cc3d_status;
+
+typedef enum { CC3D_BF16 = 0, CC3D_FP32 = 1 } cc3d_dtype;
+
+/* Epilogue fused into the conv (§10.4: bias, residual add, next RMS+SiLU). */
+typedef enum {
+  CC3D_EPI_BIAS = 0,          /* y = conv + b                                  */
+  CC3D_EPI_BIAS_RESIDUAL = 1, /* y = conv + b + residual                       */
+  CC3D_EPI_BIAS_RMS_SILU = 2  /* y = SiLU(RMS(conv + b; gamma) (+ beta)),
+                                 needs c_out <= 256 so one CTA owns a row      */
+} cc3d_epilogue;
+
+/* Kernel that served a call (the plan's route counters). */
+typedef enum {
+  CC3D_VARIANT_NONE = 0,
+  CC3D_VARIANT_UMMA = 1,     /* tcgen05 implicit GEMM, TMA halo tiles       */
+  CC3D_VARIANT_THIN = 2,     /* c_in = 3 first layer, tcgen05, gathered A   */
+  CC3D_VARIANT_FP32 = 3      /* fp32 SIMT direct convolution               */
+} cc3d_variant;
+
+typedef struct {
+  int n, c_in, c_out, h, w, max_t;   /* max_t: largest frame count per call  */
+  int kt, kh, kw;                    /* kernel size; causal front pad = kt-1 */
+  int pad_h, pad_w;                  /* spatial zero padding (kh/2, kw/2)    */
+  int stride_t, stride_h, stride_w;  /* must be 1                            */
+  int dil_t, dil_h, dil_w;           /* must be 1                            */
+  int groups;                        /* must be 1                            */
+  cc3d_dtype dtype;
+  const void *weight;  /* device [c_out][c_in][kt][kh][kw] (PyTorch order),
+                          dtype; copied (and re-tiled) at create             */
+  const float *bias;   /* device [c_out] fp32, nullable (= 0); copied        */
+  cc3d_epilogue epi;
+  const float *gamma;  /* device [c_out] fp32, EPI_BIAS_RMS_SILU only; copied */
+  const float *beta;   /* device [c_out] fp32, nullable; copied               */
+} cc3d_desc;
+
+typedef struct {
+  uint64_t calls;          /* successful cc3d_forward launches               */
+  uint64_t rejected;       /* calls refused by validation                    */
+  uint64_t tiles;          /* output tiles launched in total                 */
+  int variant;             /* cc3d_variant chosen at create                  */
+  int tile_h, tile_w;      /* output tile (rows x cols of one frame)         */
+  int n_tile;              /* output channels per CTA                        */
+  int k_chunk;             /* input channels per pipeline stage              */
+} cc3d_stats;
+
+typedef struct cc3d_plan cc3d_plan;
+typedef struct cc3d_block cc3d_block;
+
+/* Validate desc, pick a kernel, copy and re-tile the weights (and bias,
+ * gamma, beta) into plan-owned device memory.  Synchronous.  Returns
+ * CC3D_ERR_UNSUPPORTED for stride/dilation/groups != 1, even kernel sizes,
+ * or channel counts no kernel covers (bf16: c_in == 3, or c_in % 32 == 0;
+ * c_out % 16 == 0; fp32: any).  *out is set only on CC3D_OK. */
+cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out);
+cc3d_status cc3d_plan_destroy(cc3d_plan *plan);
+
+/* One causal conv over a chunk of t frames (1 <= t <= max_t).
+ *   x         [n][t][h][w][c_in]       input chunk
+ *   cache_in  [n][kt-1][h][w][c_in]    frames before the chunk, oldest
+ *                                      first; NULL = zero frames
+ *   y         [n][t][h][w][c_out]      output
+ *   cache_out [n][kt-1][h][w][c_in]    nullable: the last kt-1 frames of
+ *                                      concat(cache_in, x), for the next call
+ *   residual  [n][t][h][w][c_out]      EPI_BIAS_RESIDUAL only, else NULL
+ *   next_cache_in / next_cache_out     EPI_BIAS_RMS_SILU only, nullable:
+ *                                      [n][2][h][w][c_out]; next_cache_out
+ *                                      receives the last 2 frames of
+ *                                      concat(next_cache_in, y) -- the cache
+ *                                      of the conv that consumes y.
+ *   stream    a cudaStream_t (NULL = legacy default stream). */
+cc3d_status cc3d_forward(cc3d_plan *plan, const void *x, int t,
+                         const void *cache_in, void *y, void *cache_out,
+                         const void *residual, const void *next_cache_in,
+                         void *next_cache_out, void *stream);
+
+/* Stand-alone channel RMS_norm + SiLU (§10.2, §10.4), bf16 in / bf16 out.
+ *   x, y      [n][t][h][w][c]; gamma [c] fp32; beta [c] fp32 nullable
+ *   cache_in / cache_out  nullable, [n][2][h][w][c]: cache_out receives the
+ *             last 2 frames of concat(cache_in (or zeros), y).
+ * c must be a multiple of 8 and at most 1024. */
+cc3d_status rmsnorm_silu(const void *x, const float *gamma, const float *beta,
+                         int n, int t, int h, int w, int c, void *y,
+                         const void *cache_in, void *cache_out, void *stream);
+
+/* Residual block with c channels (§10.4).  Weights w1, w2 are device
+ * [c][c][3][3][3] bf16; b1, b2, g1, g2 device [c] fp32.  All are copied.
+ * The block owns two activation buffers of max_t frames (a0, a1).
+ * c % 32 == 0 and 32 <= c <= 256. */
+cc3d_status cc3d_block_create(int n, int c, int h, int w, int max_t,
+                              const void *w1, const float *b1, const float *g1,
+                              const void *w2, const float *b2, const float *g2,
+                              cc3d_block **out);
+cc3d_status cc3d_block_destroy(cc3d_block *block);
+
+/* y = block(x) for a chunk of t frames.  cache1_* is conv1's history (a0
+ * frames), cache2_* conv2's (a1 frames); *_in nullable (zeros), *_out
+ * nullable.  All [n][2][h][w][c] bf16. */
+cc3d_status cc3d_resblock_forward(cc3d_block *block, const void *x, int t,
+                                  const void *cache1_in, const void *cache2_in,
+                                  void *y, void *cache1_out, void *cache2_out,
+                                  void *stream);
+
+/* Synchronise `stream` and report (then clear) the device status word:
+ * CC3D_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
+ * CC3D_ERR_CUDA on a CUDA error, else CC3D_OK. */
+cc3d_status cc3d_sync_status(void *stream);
+
+/* Copy the plan's counters. */
+cc3d_status cc3d_get_stats(const cc3d_plan *plan, cc3d_stats *out);
+
+/* Static description of a status code. */
+const char *cc3d_status_string(cc3d_status s);
+
+/* Number of kernel launches made by this library in this process (all
+ * entry points).  Lets callers count device work. */
+uint64_t cc3d_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CC3D_H_ */

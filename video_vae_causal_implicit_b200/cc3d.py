@@ -1,0 +1,242 @@
+"""ctypes binding of libcc3d.so (the C ABI in include/cc3d.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  The raw entry points keep the C names (``cc3d_plan_create``,
+``cc3d_forward``, ``rmsnorm_silu``, ``cc3d_block_create``,
+``cc3d_resblock_forward``, ...).  ``Plan`` and ``Block`` wrap them for
+torch tensors: they pass ``data_ptr()`` and the current CUDA stream, nothing
+else.  Loading fails loudly when the library is missing -- there is no CPU
+path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libcc3d.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_ALIAS, ERR_OOM, ERR_CUDA, ERR_TIMEOUT = \
+    range(8)
+BF16, FP32 = 0, 1
+EPI_BIAS, EPI_BIAS_RESIDUAL, EPI_BIAS_RMS_SILU = 0, 1, 2
+VARIANT_NONE, VARIANT_UMMA, VARIANT_THIN, VARIANT_FP32 = 0, 1, 2, 3
+
+_STATUS_NAMES = {0: "CC3D_OK", 1: "CC3D_ERR_INVALID_ARG", 2: "CC3D_ERR_UNSUPPORTED",
+                 3: "CC3D_ERR_ALIGNMENT", 4: "CC3D_ERR_ALIAS", 5: "CC3D_ERR_OOM",
+                 6: "CC3D_ERR_CUDA", 7: "CC3D_ERR_TIMEOUT"}
+
+
+class Cc3dError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS_NAMES.get(status, status)} "
+                         f"({lib().cc3d_status_string(status).decode()})")
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "n", "c_in", "c_out", "h", "w", "max_t", "kt", "kh", "kw", "pad_h", "pad_w",
+        "stride_t", "stride_h", "stride_w", "dil_t", "dil_h", "dil_w", "groups", "dtype")] + [
+        ("weight", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("epi", ctypes.c_int),
+        ("gamma", ctypes.c_void_p), ("beta", ctypes.c_void_p)]
+
+
+class Stats(ctypes.Structure):
+    _fields_ = [("calls", ctypes.c_uint64), ("rejected", ctypes.c_uint64),
+                ("tiles", ctypes.c_uint64), ("variant", ctypes.c_int), ("tile_h", ctypes.c_int),
+                ("tile_w", ctypes.c_int), ("n_tile", ctypes.c_int), ("k_chunk", ctypes.c_int)]
+
+
+# name -> (restype, argtypes)
+_VP, _I = ctypes.c_void_p, ctypes.c_int
+SIGNATURES = {
+    "cc3d_plan_create": (_I, [ctypes.POINTER(Desc), ctypes.POINTER(_VP)]),
+    "cc3d_plan_destroy": (_I, [_VP]),
+    "cc3d_forward": (_I, [_VP, _VP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "rmsnorm_silu": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP]),
+    "cc3d_block_create": (_I, [_I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP,
+                               ctypes.POINTER(_VP)]),
+    "cc3d_block_destroy": (_I, [_VP]),
+    "cc3d_resblock_forward": (_I, [_VP, _VP, _I, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "cc3d_sync_status": (_I, [_VP]),
+    "cc3d_get_stats": (_I, [_VP, ctypes.POINTER(Stats)]),
+    "cc3d_status_string": (ctypes.c_char_p, [_I]),
+    "cc3d_launch_count": (ctypes.c_uint64, []),
+}
+
+_lib = None
+
+
+def lib():
+    """Load libcc3d.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m video_vae_causal_implicit_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def check(status, where):
+    if status != OK:
+        raise Cc3dError(status, where)
+
+
+# Raw C entry points, same names as the header.
+def cc3d_plan_create(desc, out):
+    return lib().cc3d_plan_create(ctypes.byref(desc), ctypes.byref(out))
+
+
+def cc3d_plan_destroy(plan):
+    return lib().cc3d_plan_destroy(plan)
+
+
+def cc3d_forward(plan, x, t, cache_in, y, cache_out, residual, next_cache_in, next_cache_out,
+                 stream):
+    return lib().cc3d_forward(plan, x, t, cache_in, y, cache_out, residual, next_cache_in,
+                              next_cache_out, stream)
+
+
+def rmsnorm_silu(x, gamma, beta, n, t, h, w, c, y, cache_in, cache_out, stream):
+    return lib().rmsnorm_silu(x, gamma, beta, n, t, h, w, c, y, cache_in, cache_out, stream)
+
+
+def cc3d_block_create(n, c, h, w, max_t, w1, b1, g1, w2, b2, g2, out):
+    return lib().cc3d_block_create(n, c, h, w, max_t, w1, b1, g1, w2, b2, g2, ctypes.byref(out))
+
+
+def cc3d_block_destroy(block):
+    return lib().cc3d_block_destroy(block)
+
+
+def cc3d_resblock_forward(block, x, t, cache1_in, cache2_in, y, cache1_out, cache2_out, stream):
+    return lib().cc3d_resblock_forward(block, x, t, cache1_in, cache2_in, y, cache1_out,
+                                       cache2_out, stream)
+
+
+def cc3d_sync_status(stream):
+    return lib().cc3d_sync_status(stream)
+
+
+def cc3d_get_stats(plan, out):
+    return lib().cc3d_get_stats(plan, ctypes.byref(out))
+
+
+def cc3d_status_string(status):
+    return lib().cc3d_status_string(status).decode()
+
+
+def cc3d_launch_count():
+    return int(lib().cc3d_launch_count())
+
+
+# ---- torch conveniences (pointers + current stream only) --------------------------
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class Plan:
+    """A causal conv plan.  ``weight`` is [C_out, C_in, kt, kh, kw] on the
+    device (bf16, or fp32 for dtype=FP32); bias/gamma/beta fp32 [C_out]."""
+
+    def __init__(self, weight, bias=None, *, n=1, h, w, max_t, epi=EPI_BIAS, gamma=None,
+                 beta=None, dtype=BF16, pad=None):
+        co, ci, kt, kh, kw = (int(s) for s in weight.shape)
+        d = Desc()
+        d.n, d.c_in, d.c_out, d.h, d.w, d.max_t = n, ci, co, h, w, max_t
+        d.kt, d.kh, d.kw = kt, kh, kw
+        d.pad_h, d.pad_w = pad if pad is not None else (kh // 2, kw // 2)
+        d.stride_t = d.stride_h = d.stride_w = 1
+        d.dil_t = d.dil_h = d.dil_w = 1
+        d.groups = 1
+        d.dtype = dtype
+        weight = weight.contiguous()
+        d.weight = weight.data_ptr()
+        d.bias = bias.data_ptr() if bias is not None else None
+        d.epi = epi
+        d.gamma = gamma.data_ptr() if gamma is not None else None
+        d.beta = beta.data_ptr() if beta is not None else None
+        self.desc = d
+        self.handle = ctypes.c_void_p()
+        check(cc3d_plan_create(d, self.handle), "cc3d_plan_create")
+
+    def forward(self, x, y, t=None, cache_in=None, cache_out=None, residual=None,
+                next_cache_in=None, next_cache_out=None, stream=None):
+        t = int(x.shape[1]) if t is None else t
+        check(cc3d_forward(self.handle, _ptr(x), t, _ptr(cache_in), _ptr(y), _ptr(cache_out),
+                           _ptr(residual), _ptr(next_cache_in), _ptr(next_cache_out),
+                           _stream(stream)), "cc3d_forward")
+        return y
+
+    def stats(self):
+        s = Stats()
+        check(cc3d_get_stats(self.handle, s), "cc3d_get_stats")
+        return s
+
+    def close(self):
+        if self.handle:
+            cc3d_plan_destroy(self.handle)
+            self.handle = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class Block:
+    """Residual block (C_in == C_out, 3x3x3 convs)."""
+
+    def __init__(self, w1, b1, g1, w2, b2, g2, *, n=1, h, w, max_t):
+        c = int(w1.shape[0])
+        self.c = c
+        self._keep = [t.contiguous() for t in (w1, b1, g1, w2, b2, g2)]
+        self.handle = ctypes.c_void_p()
+        check(cc3d_block_create(n, c, h, w, max_t, *(_ptr(t) for t in self._keep), self.handle),
+              "cc3d_block_create")
+        self._keep = None
+
+    def forward(self, x, y, t=None, cache1_in=None, cache2_in=None, cache1_out=None,
+                cache2_out=None, stream=None):
+        t = int(x.shape[1]) if t is None else t
+        check(cc3d_resblock_forward(self.handle, _ptr(x), t, _ptr(cache1_in), _ptr(cache2_in),
+                                    _ptr(y), _ptr(cache1_out), _ptr(cache2_out), _stream(stream)),
+              "cc3d_resblock_forward")
+        return y
+
+    def close(self):
+        if self.handle:
+            cc3d_block_destroy(self.handle)
+            self.handle = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def rms_silu(x, gamma, y, beta=None, cache_in=None, cache_out=None, stream=None):
+    n, t, h, w, c = (int(s) for s in x.shape)
+    check(rmsnorm_silu(_ptr(x), _ptr(gamma), _ptr(beta), n, t, h, w, c, _ptr(y), _ptr(cache_in),
+                       _ptr(cache_out), _stream(stream)), "rmsnorm_silu")
+    return y
+
+
+def sync_status(stream=None):
+    check(cc3d_sync_status(_stream(stream)), "cc3d_sync_status")

@@ -1,0 +1,489 @@
+// cc3d_api.cu -- the C ABI of libcc3d.so (declared in include/cc3d.h):
+// descriptor validation, plan-time weight re-tiling, TMA tensor-map
+// encoding, kernel selection and launch, the residual block, route
+// counters and the device status word.
+//
+// Gating mirrors the fast-path rule of the "cache-aware video decoder
+// lowering" summary (5-D tensors, temporal stride 1, one group): anything
+// else is refused with CC3D_ERR_UNSUPPORTED -- there is no fallback path.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "cc3d.h"
+#include "internal.h"
+
+namespace cc3d {
+
+// Device status word: non-zero after a bounded device wait ran out.
+__device__ int g_status_word;
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+unsigned long long wait_limit_ns() {
+  static unsigned long long v = [] {
+    const char *s = std::getenv("CC3D_WAIT_LIMIT_MS");
+    unsigned long long ms = s ? std::strtoull(s, nullptr, 10) : 2000ull;
+    if (ms == 0) ms = 2000ull;
+    return ms * 1000000ull;
+  }();
+  return v;
+}
+
+std::mutex g_mu;
+int *g_status_ptr[64] = {nullptr};
+
+int *status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int *>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+bool is_sm100() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return false;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return false;
+  return major == 10 && minor == 0;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// 5-D bf16 tensor map over an NDHWC buffer: dims (C, W, H, T, N), a box of
+// 8 channels x box_w x box_h x 1 x 1, no swizzle, zero fill out of bounds.
+bool encode_act_map(CUtensorMap *m, const void *base, int c, int w, int h, int t, int n,
+                    int box_w, int box_h) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[5] = {(cuuint64_t)c, (cuuint64_t)w, (cuuint64_t)h, (cuuint64_t)t,
+                        (cuuint64_t)n};
+  cuuint64_t strides[4] = {(cuuint64_t)c * 2, (cuuint64_t)c * 2 * w, (cuuint64_t)c * 2 * w * h,
+                           (cuuint64_t)c * 2 * w * h * t};
+  cuuint32_t box[5] = {8, (cuuint32_t)box_w, (cuuint32_t)box_h, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+}  // namespace cc3d
+
+using namespace cc3d;
+
+struct cc3d_plan {
+  cc3d_desc d;
+  int variant;
+  int device;
+  // UMMA
+  int kc, nt, n_ntiles, na, nb, tmem_cols;
+  uint8_t *wimg;
+  // fp32 / thin
+  void *wraw;
+  int kpad;
+  float *bias, *gamma, *beta;
+  cc3d_stats st;
+  std::mutex mu;
+};
+
+struct cc3d_block {
+  int n, c, h, w, max_t;
+  cc3d_plan *conv1, *conv2;
+  float *g1;
+  __nv_bfloat16 *a0, *a1;
+};
+
+namespace {
+
+cc3d_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return CC3D_OK;
+  if (e == cudaErrorMemoryAllocation) return CC3D_ERR_OOM;
+  return CC3D_ERR_CUDA;
+}
+
+void free_plan(cc3d_plan *p) {
+  if (!p) return;
+  cudaFree(p->wimg);
+  cudaFree(p->wraw);
+  cudaFree(p->bias);
+  cudaFree(p->gamma);
+  cudaFree(p->beta);
+  delete p;
+}
+
+cc3d_status copy_vec(float **dst, const float *src, int c, bool zero_if_null) {
+  *dst = nullptr;
+  if (!src && !zero_if_null) return CC3D_OK;
+  cudaError_t e = cudaMalloc(dst, sizeof(float) * c);
+  if (e != cudaSuccess) return CC3D_ERR_OOM;
+  if (src)
+    e = cudaMemcpy(*dst, src, sizeof(float) * c, cudaMemcpyDeviceToDevice);
+  else
+    e = cudaMemset(*dst, 0, sizeof(float) * c);
+  return from_cuda(e);
+}
+
+// Validation that needs no GPU: returns CC3D_OK when a kernel covers desc.
+cc3d_status check_desc(const cc3d_desc *d, int *variant) {
+  if (!d || !d->weight) return CC3D_ERR_INVALID_ARG;
+  if (d->n < 1 || d->c_in < 1 || d->c_out < 1 || d->h < 1 || d->w < 1 || d->max_t < 1)
+    return CC3D_ERR_INVALID_ARG;
+  if (d->kt < 1 || d->kh < 1 || d->kw < 1) return CC3D_ERR_INVALID_ARG;
+  if (d->stride_t != 1 || d->stride_h != 1 || d->stride_w != 1 || d->dil_t != 1 ||
+      d->dil_h != 1 || d->dil_w != 1 || d->groups != 1)
+    return CC3D_ERR_UNSUPPORTED;
+  if (d->kh % 2 == 0 || d->kw % 2 == 0 || d->pad_h != d->kh / 2 || d->pad_w != d->kw / 2)
+    return CC3D_ERR_UNSUPPORTED;
+  if (d->kt > 3 || d->kh > 3 || d->kw > 3) return CC3D_ERR_UNSUPPORTED;
+  if (d->epi < CC3D_EPI_BIAS || d->epi > CC3D_EPI_BIAS_RMS_SILU) return CC3D_ERR_INVALID_ARG;
+  if (d->epi == CC3D_EPI_BIAS_RMS_SILU && !d->gamma) return CC3D_ERR_INVALID_ARG;
+  if (d->dtype == CC3D_FP32) {
+    if (d->epi != CC3D_EPI_BIAS) return CC3D_ERR_UNSUPPORTED;
+    *variant = CC3D_VARIANT_FP32;
+    return CC3D_OK;
+  }
+  if (d->dtype != CC3D_BF16) return CC3D_ERR_INVALID_ARG;
+  if (d->c_out % 16 != 0) return CC3D_ERR_UNSUPPORTED;
+  if (d->c_in % 32 == 0) {
+    if (d->epi == CC3D_EPI_BIAS_RMS_SILU && d->c_out > 256) return CC3D_ERR_UNSUPPORTED;
+    *variant = CC3D_VARIANT_UMMA;
+    return CC3D_OK;
+  }
+  return CC3D_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *cc3d_status_string(cc3d_status s) {
+  switch (s) {
+    case CC3D_OK: return "ok";
+    case CC3D_ERR_INVALID_ARG: return "invalid argument";
+    case CC3D_ERR_UNSUPPORTED: return "unsupported descriptor (no kernel covers it)";
+    case CC3D_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case CC3D_ERR_ALIAS: return "cache_out overlaps cache_in, x or y";
+    case CC3D_ERR_OOM: return "device allocation failed";
+    case CC3D_ERR_CUDA: return "CUDA error";
+    case CC3D_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+uint64_t cc3d_launch_count(void) { return g_launches.load(); }
+
+cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
+  if (!out) return CC3D_ERR_INVALID_ARG;
+  int variant = 0;
+  cc3d_status s = check_desc(desc, &variant);
+  if (s != CC3D_OK) return s;
+  if (!is_sm100()) return CC3D_ERR_UNSUPPORTED;
+  cc3d_plan *p = new cc3d_plan();
+  p->d = *desc;
+  p->d.weight = nullptr;
+  p->d.bias = p->d.gamma = p->d.beta = nullptr;
+  p->variant = variant;
+  cudaGetDevice(&p->device);
+  std::memset(&p->st, 0, sizeof(p->st));
+  p->st.variant = variant;
+  const int taps = desc->kt * desc->kh * desc->kw;
+  cudaError_t e = cudaSuccess;
+  if ((s = copy_vec(&p->bias, desc->bias, desc->c_out, true)) != CC3D_OK) goto fail;
+  if ((s = copy_vec(&p->gamma, desc->gamma, desc->c_out, false)) != CC3D_OK) goto fail;
+  if ((s = copy_vec(&p->beta, desc->beta, desc->c_out, false)) != CC3D_OK) goto fail;
+  if (variant == CC3D_VARIANT_FP32) {
+    const size_t bytes = sizeof(float) * desc->c_out * desc->c_in * taps;
+    if (cudaMalloc(&p->wraw, bytes) != cudaSuccess) { s = CC3D_ERR_OOM; goto fail; }
+    e = cudaMemcpy(p->wraw, desc->weight, bytes, cudaMemcpyDeviceToDevice);
+    if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
+  } else {
+    if (!encode_fn()) { s = CC3D_ERR_CUDA; goto fail; }
+    e = umma_prepare();
+    if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
+    if (!status_ptr()) { s = CC3D_ERR_CUDA; goto fail; }
+    p->kc = (desc->c_in % 64 == 0) ? 64 : 32;
+    int split = 1;
+    while (desc->c_out / split > 256 || (desc->c_out % split) != 0 ||
+           ((desc->c_out / split) % 16) != 0)
+      ++split;
+    p->nt = desc->c_out / split;
+    p->n_ntiles = split;
+    int cols = 32;
+    while (cols < p->nt) cols *= 2;
+    p->tmem_cols = cols;
+    // Pipeline depths: two halo stages, as many weight stages as fit.
+    p->na = 2;
+    const size_t budget = 200 * 1024;
+    int nb = 8;
+    while (nb > 2 && umma_smem_bytes(p->kc, p->nt, desc->kh, desc->kw, p->na, nb) > budget) --nb;
+    p->nb = nb;
+    p->st.tile_h = umma_tile_h();
+    p->st.tile_w = umma_tile_w();
+    p->st.n_tile = p->nt;
+    p->st.k_chunk = p->kc;
+    const size_t bytes = sizeof(__nv_bfloat16) * desc->c_out * desc->c_in * taps;
+    if (cudaMalloc(&p->wimg, bytes) != cudaSuccess) { s = CC3D_ERR_OOM; goto fail; }
+    e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(desc->weight), p->wimg,
+                           desc->c_out, desc->c_in, taps, p->nt, p->kc, 0);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
+  }
+  *out = p;
+  return CC3D_OK;
+fail:
+  free_plan(p);
+  return s;
+}
+
+cc3d_status cc3d_plan_destroy(cc3d_plan *plan) {
+  if (!plan) return CC3D_ERR_INVALID_ARG;
+  free_plan(plan);
+  return CC3D_OK;
+}
+
+cc3d_status cc3d_get_stats(const cc3d_plan *plan, cc3d_stats *out) {
+  if (!plan || !out) return CC3D_ERR_INVALID_ARG;
+  *out = plan->st;
+  return CC3D_OK;
+}
+
+cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_in, void *y,
+                         void *cache_out, const void *residual, const void *next_cache_in,
+                         void *next_cache_out, void *stream_v) {
+  if (!p) return CC3D_ERR_INVALID_ARG;
+  const cc3d_desc &d = p->d;
+  auto reject = [&](cc3d_status s) {
+    std::lock_guard<std::mutex> lk(p->mu);
+    p->st.rejected++;
+    return s;
+  };
+  if (!x || !y || t < 1 || t > d.max_t) return reject(CC3D_ERR_INVALID_ARG);
+  if ((d.epi == CC3D_EPI_BIAS_RESIDUAL) != (residual != nullptr))
+    return reject(CC3D_ERR_INVALID_ARG);
+  if (d.epi != CC3D_EPI_BIAS_RMS_SILU && (next_cache_in || next_cache_out))
+    return reject(CC3D_ERR_INVALID_ARG);
+  if (!aligned16(x) || !aligned16(y) || !aligned16(cache_in) || !aligned16(cache_out) ||
+      !aligned16(residual) || !aligned16(next_cache_in) || !aligned16(next_cache_out))
+    return reject(CC3D_ERR_ALIGNMENT);
+  const size_t esz = d.dtype == CC3D_FP32 ? 4 : 2;
+  const int front = d.kt - 1;
+  const size_t in_frame = static_cast<size_t>(d.h) * d.w * d.c_in * esz;
+  const size_t out_frame = static_cast<size_t>(d.h) * d.w * d.c_out * esz;
+  const size_t x_bytes = in_frame * d.n * t, y_bytes = out_frame * d.n * t;
+  const size_t c_bytes = in_frame * d.n * front;
+  const size_t nc_bytes = out_frame * d.n * 2;
+  if (overlaps(cache_out, c_bytes, cache_in, c_bytes) || overlaps(cache_out, c_bytes, x, x_bytes) ||
+      overlaps(cache_out, c_bytes, y, y_bytes) ||
+      overlaps(next_cache_out, nc_bytes, next_cache_in, nc_bytes) ||
+      overlaps(next_cache_out, nc_bytes, y, y_bytes) ||
+      overlaps(next_cache_out, nc_bytes, x, x_bytes) || overlaps(y, y_bytes, x, x_bytes))
+    return reject(CC3D_ERR_ALIAS);
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (dev != p->device) return reject(CC3D_ERR_INVALID_ARG);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  int *status = status_ptr();
+  if (!status) return reject(CC3D_ERR_CUDA);
+  cudaError_t e = cudaSuccess;
+  uint64_t tiles = 0;
+  if (p->variant == CC3D_VARIANT_FP32) {
+    Fp32Args a;
+    a.x = static_cast<const float *>(x);
+    a.cache = static_cast<const float *>(cache_in);
+    a.w = static_cast<const float *>(p->wraw);
+    a.bias = p->bias;
+    a.y = static_cast<float *>(y);
+    a.n = d.n; a.t = t; a.h = d.h; a.w_ = d.w; a.c_in = d.c_in; a.c_out = d.c_out;
+    a.kt = d.kt; a.kh = d.kh; a.kw = d.kw; a.pad_h = d.pad_h; a.pad_w = d.pad_w;
+    e = launch_conv_fp32(a, stream);
+    tiles = 1;
+  } else {
+    CUtensorMap mx, mc;
+    const int box_w = umma_tile_w() + d.kw - 1, box_h = umma_tile_h() + d.kh - 1;
+    if (!encode_act_map(&mx, x, d.c_in, d.w, d.h, t, d.n, box_w, box_h))
+      return reject(CC3D_ERR_CUDA);
+    if (cache_in && front > 0) {
+      if (!encode_act_map(&mc, cache_in, d.c_in, d.w, d.h, front, d.n, box_w, box_h))
+        return reject(CC3D_ERR_CUDA);
+    } else {
+      mc = mx;
+    }
+    UmmaArgs a;
+    a.wimg = p->wimg;
+    a.bias = p->bias;
+    a.gamma = p->gamma;
+    a.beta = p->beta;
+    a.residual = static_cast<const __nv_bfloat16 *>(residual);
+    a.y = static_cast<__nv_bfloat16 *>(y);
+    a.status = status;
+    a.wait_limit_ns = wait_limit_ns();
+    a.n = d.n; a.t = t; a.h = d.h; a.w = d.w; a.c_in = d.c_in; a.c_out = d.c_out;
+    a.kt = d.kt; a.kh = d.kh; a.kw = d.kw; a.pad_h = d.pad_h; a.pad_w = d.pad_w;
+    a.nt = p->nt; a.n_ntiles = p->n_ntiles;
+    a.tiles_w = (d.w + umma_tile_w() - 1) / umma_tile_w();
+    a.tiles_h = (d.h + umma_tile_h() - 1) / umma_tile_h();
+    a.na = p->na; a.nb = p->nb; a.tmem_cols = p->tmem_cols;
+    a.epi = static_cast<int>(d.epi);
+    a.has_cache = (cache_in && front > 0) ? 1 : 0;
+    tiles = static_cast<uint64_t>(d.n) * t * a.tiles_h * a.tiles_w * a.n_ntiles;
+    e = launch_conv_umma(mx, mc, a, p->kc, static_cast<unsigned>(tiles), stream);
+    count_launch();
+  }
+  if (e == cudaSuccess && cache_out && front > 0)
+    e = launch_cache_update(cache_in, x, cache_out, d.n, t, front, in_frame, stream);
+  if (e == cudaSuccess && next_cache_out)
+    e = launch_cache_update(next_cache_in, y, next_cache_out, d.n, t, 2, out_frame, stream);
+  if (e != cudaSuccess) return reject(from_cuda(e));
+  std::lock_guard<std::mutex> lk(p->mu);
+  p->st.calls++;
+  p->st.tiles += tiles;
+  return CC3D_OK;
+}
+
+cc3d_status rmsnorm_silu(const void *x, const float *gamma, const float *beta, int n, int t,
+                         int h, int w, int c, void *y, const void *cache_in, void *cache_out,
+                         void *stream_v) {
+  if (!x || !gamma || !y || n < 1 || t < 1 || h < 1 || w < 1 || c < 8) return CC3D_ERR_INVALID_ARG;
+  if (c % 8 != 0 || c > 1024) return CC3D_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(cache_in) || !aligned16(cache_out))
+    return CC3D_ERR_ALIGNMENT;
+  const size_t frame = static_cast<size_t>(h) * w * c * 2;
+  const size_t xb = frame * n * t, cb = frame * n * 2;
+  if (overlaps(cache_out, cb, cache_in, cb) || overlaps(cache_out, cb, y, xb) ||
+      overlaps(cache_out, cb, x, xb))
+    return CC3D_ERR_ALIAS;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  const long long voxels = static_cast<long long>(n) * t * h * w;
+  cudaError_t e = launch_rmsnorm_silu(static_cast<const __nv_bfloat16 *>(x), gamma, beta, voxels,
+                                      c, static_cast<__nv_bfloat16 *>(y), stream);
+  if (e == cudaSuccess && cache_out)
+    e = launch_cache_update(cache_in, y, cache_out, n, t, 2, frame, stream);
+  return from_cuda(e);
+}
+
+cc3d_status cc3d_block_create(int n, int c, int h, int w, int max_t, const void *w1,
+                              const float *b1, const float *g1, const void *w2, const float *b2,
+                              const float *g2, cc3d_block **out) {
+  if (!out || !w1 || !w2 || !g1 || !g2 || n < 1 || h < 1 || w < 1 || max_t < 1)
+    return CC3D_ERR_INVALID_ARG;
+  if (c < 32 || c > 256 || c % 32 != 0) return CC3D_ERR_UNSUPPORTED;
+  cc3d_desc d;
+  std::memset(&d, 0, sizeof d);
+  d.n = n; d.c_in = c; d.c_out = c; d.h = h; d.w = w; d.max_t = max_t;
+  d.kt = d.kh = d.kw = 3; d.pad_h = d.pad_w = 1;
+  d.stride_t = d.stride_h = d.stride_w = 1; d.dil_t = d.dil_h = d.dil_w = 1; d.groups = 1;
+  d.dtype = CC3D_BF16;
+  cc3d_block *b = new cc3d_block();
+  std::memset(b, 0, sizeof *b);
+  b->n = n; b->c = c; b->h = h; b->w = w; b->max_t = max_t;
+  cc3d_status s;
+  d.weight = w1; d.bias = b1; d.epi = CC3D_EPI_BIAS_RMS_SILU; d.gamma = g2; d.beta = nullptr;
+  if ((s = cc3d_plan_create(&d, &b->conv1)) != CC3D_OK) goto fail;
+  d.weight = w2; d.bias = b2; d.epi = CC3D_EPI_BIAS_RESIDUAL; d.gamma = nullptr;
+  if ((s = cc3d_plan_create(&d, &b->conv2)) != CC3D_OK) goto fail;
+  if ((s = copy_vec(&b->g1, g1, c, false)) != CC3D_OK) goto fail;
+  {
+    const size_t bytes = sizeof(__nv_bfloat16) * static_cast<size_t>(n) * max_t * h * w * c;
+    if (cudaMalloc(&b->a0, bytes) != cudaSuccess || cudaMalloc(&b->a1, bytes) != cudaSuccess) {
+      s = CC3D_ERR_OOM;
+      goto fail;
+    }
+  }
+  *out = b;
+  return CC3D_OK;
+fail:
+  cc3d_block_destroy(b);
+  return s;
+}
+
+cc3d_status cc3d_block_destroy(cc3d_block *b) {
+  if (!b) return CC3D_ERR_INVALID_ARG;
+  if (b->conv1) cc3d_plan_destroy(b->conv1);
+  if (b->conv2) cc3d_plan_destroy(b->conv2);
+  cudaFree(b->g1);
+  cudaFree(b->a0);
+  cudaFree(b->a1);
+  delete b;
+  return CC3D_OK;
+}
+
+cc3d_status cc3d_resblock_forward(cc3d_block *b, const void *x, int t, const void *cache1_in,
+                                  const void *cache2_in, void *y, void *cache1_out,
+                                  void *cache2_out, void *stream) {
+  if (!b || !x || !y || t < 1 || t > b->max_t) return CC3D_ERR_INVALID_ARG;
+  const size_t frame = static_cast<size_t>(b->h) * b->w * b->c * 2;
+  const size_t xb = frame * b->n * t, cb = frame * b->n * 2;
+  if (overlaps(x, xb, y, xb)) return CC3D_ERR_ALIAS;
+  if (overlaps(cache1_out, cb, cache1_in, cb) || overlaps(cache2_out, cb, cache2_in, cb) ||
+      overlaps(cache1_out, cb, x, xb) || overlaps(cache1_out, cb, y, xb) ||
+      overlaps(cache2_out, cb, x, xb) || overlaps(cache2_out, cb, y, xb) ||
+      overlaps(cache1_out, cb, cache2_out, cb) || overlaps(cache1_out, cb, cache2_in, cb) ||
+      overlaps(cache2_out, cb, cache1_in, cb))
+    return CC3D_ERR_ALIAS;
+  // a0 = SiLU(RMS(x; g1)); conv1's cache is a0's history.
+  cc3d_status s = rmsnorm_silu(x, b->g1, nullptr, b->n, t, b->h, b->w, b->c, b->a0, cache1_in,
+                               cache1_out, stream);
+  if (s != CC3D_OK) return s;
+  // a1 = SiLU(RMS(conv1(a0) + b1; g2)), fused epilogue; conv2's cache is a1's history.
+  s = cc3d_forward(b->conv1, b->a0, t, cache1_in, b->a1, nullptr, nullptr, cache2_in, cache2_out,
+                   stream);
+  if (s != CC3D_OK) return s;
+  // y = conv2(a1) + b2 + x, fused epilogue.
+  return cc3d_forward(b->conv2, b->a1, t, cache2_in, y, nullptr, x, nullptr, nullptr, stream);
+}
+
+cc3d_status cc3d_sync_status(void *stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return CC3D_ERR_CUDA;
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status_word, sizeof v);
+  if (e != cudaSuccess) return CC3D_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(g_status_word, &zero, sizeof zero);
+    return CC3D_ERR_TIMEOUT;
+  }
+  return CC3D_OK;
+}
+
+}  // extern "C"

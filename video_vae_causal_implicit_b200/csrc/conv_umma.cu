@@ -1,0 +1,335 @@
+// conv_umma.cu -- bf16 implicit-GEMM causal Conv3D on tcgen05 tensor cores.
+//
+// Operation ("Cosmos3 Wan VAE -- engine size vs context memory", §10.3
+// WanCausalConv3d and its implicit-GEMM view): M = output voxels,
+// N = C_out, K = C_in * kt * kh * kw; every tap is summed into one fp32
+// accumulator held in tensor memory; bias is added once in the epilogue
+// ("cache-aware video decoder lowering" summary: bias after the sum).
+//
+// Tiling.  A CTA owns one output tile of TW = 8 columns x TH = 16 rows of
+// one frame (M = 128 rows of the GEMM, row m = 8 * r + c) and NT output
+// channels.  The K loop runs over (kt, channel chunk of KC, kh, kw).
+//
+// A operand: for each (kt, channel chunk) one TMA box brings the input
+// halo of the tile -- (TH + kh - 1) x (TW + kw - 1) pixels x KC channels --
+// from the current chunk x (frame tau = t + kt - (kt_size - 1) >= 0) or the
+// frame cache (tau < 0).  Spatial padding and absent caches are TMA
+// out-of-bounds zero fill, so no padded copy exists anywhere.  The halo is
+// stored as "interleaved" core matrices without swizzle,
+//     [KC/8 slabs][halo rows][halo cols][8 channels],
+// so the A matrix of spatial tap (kh, kw) is the same buffer seen from a
+// start address shifted by (kh * halo_cols + kw) * 16 bytes: one load
+// serves all kh * kw taps.
+//
+// B operand: the weights, re-tiled at plan time into the exact shared
+// memory image of each (N tile, tap, channel chunk) stage
+//     [KC/8][NT][8 channels]   (K-major core matrices),
+// fetched with one 1-D bulk copy per stage.
+//
+// Warp roles (192 threads): warp 0 issues the loads, warp 1 owns tensor
+// memory and issues tcgen05.mma from one thread, warps 2..5 run the
+// epilogue (tensor memory -> registers -> bias / residual / RMS+SiLU ->
+// bf16 -> global).  Stages are handed over with mbarriers; every wait is
+// bounded and reports through the status word instead of hanging.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace cc3d {
+
+namespace {
+
+constexpr int kTW = 8;    // tile columns (one core matrix of rows)
+constexpr int kTH = 16;   // tile rows -> M = 128
+constexpr int kM = kTW * kTH;
+constexpr int kThreads = 192;
+
+struct SmemLayout {
+  uint32_t a_off, a_stage, slab, b_off, b_stage, bar_off, total;
+  int na, nb;
+};
+
+__host__ __device__ inline uint32_t round_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+
+__host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw, int na, int nb) {
+  SmemLayout L;
+  const uint32_t hh = kTH + kh - 1, hw = kTW + kw - 1;
+  L.slab = round_up(hh * hw * 16u, 128u);
+  L.a_stage = (kc / 8) * L.slab;
+  L.b_stage = static_cast<uint32_t>(nt) * kc * 2u;
+  L.na = na;
+  L.nb = nb;
+  L.a_off = 0;
+  L.b_off = round_up(L.a_off + na * L.a_stage, 1024u);
+  L.bar_off = round_up(L.b_off + nb * L.b_stage, 64u);
+  // full_a, empty_a, full_b, empty_b, acc_full, tmem slot
+  L.total = L.bar_off + 8u * (2 * na + 2 * nb + 1) + 16u;
+  return L;
+}
+
+template <int KC>
+__global__ void __launch_bounds__(kThreads, 1)
+    conv_umma_kernel(const __grid_constant__ CUtensorMap map_x,
+                     const __grid_constant__ CUtensorMap map_cache, UmmaArgs p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // Align the dynamic shared window to 1 KiB ourselves (the attribute is a
+  // request, not a guarantee).
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const SmemLayout L = make_layout(KC, p.nt, p.kh, p.kw, p.na, p.nb);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
+  uint64_t *full_a = bars;
+  uint64_t *empty_a = full_a + L.na;
+  uint64_t *full_b = empty_a + L.na;
+  uint64_t *empty_b = full_b + L.nb;
+  uint64_t *acc_full = empty_b + L.nb;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  // ---- tile coordinates --------------------------------------------------------
+  const int ntile = blockIdx.x % p.n_ntiles;
+  int mt = blockIdx.x / p.n_ntiles;
+  const int tw_i = mt % p.tiles_w;
+  mt /= p.tiles_w;
+  const int th_i = mt % p.tiles_h;
+  mt /= p.tiles_h;
+  const int t_out = mt % p.t;
+  const int n_img = mt / p.t;
+  const int w0 = tw_i * kTW, h0 = th_i * kTH;
+
+  const int n_cc = p.c_in / KC;          // channel chunks
+  const int taps_sp = p.kh * p.kw;       // spatial taps per kt
+  const int n_a = p.kt * n_cc;           // A stages per tile
+  const uint32_t halo_w = kTW + p.kw - 1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L.na; ++i) {
+      mbar_init(&full_a[i], 1);
+      mbar_init(&empty_a[i], 1);
+    }
+    for (int i = 0; i < L.nb; ++i) {
+      mbar_init(&full_b[i], 1);
+      mbar_init(&empty_b[i], 1);
+    }
+    mbar_init(acc_full, 1);
+    fence_mbar_init();
+    prefetch_tmap(&map_x);
+    if (p.has_cache) prefetch_tmap(&map_cache);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t smem_base = smem_u32(smem);
+  bool ok = true;
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------------
+    if (lane == 0) {
+      const uint32_t a_bytes = (KC / 8) * (8u * 2u * halo_w * (kTH + p.kh - 1));
+      for (int ia = 0; ia < n_a && ok; ++ia) {
+        const int kt = ia / n_cc, cc = ia % n_cc;
+        const int sa = ia % L.na;
+        if (!mbar_wait_bounded(&empty_a[sa], ((ia / L.na) & 1) ^ 1, p.wait_limit_ns, p.status, 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full_a[sa], a_bytes);
+        const int tau = t_out + kt - (p.kt - 1);
+        const bool from_cache = tau < 0 && p.has_cache;
+        const CUtensorMap *map = from_cache ? &map_cache : &map_x;
+        const int tc = from_cache ? tau + (p.kt - 1) : tau;  // negative: zero fill
+        const uint32_t dst = smem_base + L.a_off + sa * L.a_stage;
+#pragma unroll
+        for (int s = 0; s < KC / 8; ++s)
+          tma_load_5d(dst + s * L.slab, map, &full_a[sa], cc * KC + s * 8, w0 - p.pad_w,
+                      h0 - p.pad_h, tc, n_img);
+        for (int ts = 0; ts < taps_sp; ++ts) {
+          const int ib = ia * taps_sp + ts;
+          const int sb = ib % L.nb;
+          if (!mbar_wait_bounded(&empty_b[sb], ((ib / L.nb) & 1) ^ 1, p.wait_limit_ns, p.status,
+                                 2)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full_b[sb], L.b_stage);
+          const size_t stage_idx =
+              (static_cast<size_t>(ntile) * p.kt * taps_sp + kt * taps_sp + ts) * n_cc + cc;
+          bulk_load(smem_base + L.b_off + sb * L.b_stage, p.wimg + stage_idx * L.b_stage,
+                    L.b_stage, &full_b[sb]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ----------------------------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kM, p.nt);
+      const uint32_t a_sbo = halo_w * 16u;
+      const uint32_t b_lbo = static_cast<uint32_t>(p.nt) * 16u;
+      uint32_t accumulate = 0;
+      for (int ia = 0; ia < n_a && ok; ++ia) {
+        const int sa = ia % L.na;
+        if (!mbar_wait_bounded(&full_a[sa], (ia / L.na) & 1, p.wait_limit_ns, p.status, 3)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_stage = smem_base + L.a_off + sa * L.a_stage;
+        for (int ts = 0; ts < taps_sp; ++ts) {
+          const int ib = ia * taps_sp + ts;
+          const int sb = ib % L.nb;
+          if (!mbar_wait_bounded(&full_b[sb], (ib / L.nb) & 1, p.wait_limit_ns, p.status, 4)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int kh = ts / p.kw, kw = ts % p.kw;
+          const uint32_t a_tap = a_stage + (kh * halo_w + kw) * 16u;
+          const uint32_t b_stage = smem_base + L.b_off + sb * L.b_stage;
+#pragma unroll
+          for (int j = 0; j < KC / 16; ++j) {
+            const uint64_t ad = smem_desc_noswizzle(a_tap + 2 * j * L.slab, L.slab, a_sbo);
+            const uint64_t bd = smem_desc_noswizzle(b_stage + 2 * j * b_lbo, b_lbo, 128u);
+            umma_bf16(tmem_base, ad, bd, idesc, accumulate);
+            accumulate = 1;
+          }
+          umma_commit(&empty_b[sb]);  // frees the B stage when these MMAs finish
+        }
+        umma_commit(&empty_a[sa]);
+      }
+      umma_commit(acc_full);
+    }
+  } else {
+    // ------------------------------ epilogue ------------------------------------
+    const int q = warp % 4;  // tensor-memory lane quarter this warp may read
+    const int m = q * 32 + lane;
+    const int r = m / kTW, c = m % kTW;
+    const int h = h0 + r, w = w0 + c;
+    const bool valid = (h < p.h) && (w < p.w);
+    uint32_t got = 0;
+    if (lane == 0) got = mbar_wait_bounded(acc_full, 0, p.wait_limit_ns, p.status, 5) ? 1u : 0u;
+    got = __shfl_sync(0xffffffffu, got, 0);
+    if (got) {
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      const int n0 = ntile * p.nt;
+      const size_t pix = ((static_cast<size_t>(n_img) * p.t + t_out) * p.h + h) * p.w + w;
+      __nv_bfloat16 *yrow = p.y + pix * p.c_out + n0;
+      const __nv_bfloat16 *rrow = p.residual ? p.residual + pix * p.c_out + n0 : nullptr;
+      float inv = 1.0f;
+      if (p.epi == 2) {
+        float ss = 0.f;
+        for (int j = 0; j < p.nt; j += 16) {
+          float v[16];
+          __syncwarp();
+          tmem_ld16(taddr + j, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float hv = v[i] + p.bias[n0 + j + i];
+            ss = fmaf(hv, hv, ss);
+          }
+        }
+        inv = sqrtf(static_cast<float>(p.c_out)) / fmaxf(sqrtf(ss), 1e-12f);
+      }
+      for (int j = 0; j < p.nt; j += 16) {
+        float v[16];
+        __syncwarp();
+        tmem_ld16(taddr + j, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] += p.bias[n0 + j + i];
+        if (p.epi == 1 && valid) {
+          const uint4 *rr = reinterpret_cast<const uint4 *>(rrow + j);
+          uint4 r0 = rr[0], r1 = rr[1];
+          const __nv_bfloat16 *rb0 = reinterpret_cast<const __nv_bfloat16 *>(&r0);
+          const __nv_bfloat16 *rb1 = reinterpret_cast<const __nv_bfloat16 *>(&r1);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            v[i] += __bfloat162float(rb0[i]);
+            v[8 + i] += __bfloat162float(rb1[i]);
+          }
+        } else if (p.epi == 2) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float a = v[i] * inv * p.gamma[n0 + j + i];
+            if (p.beta) a += p.beta[n0 + j + i];
+            v[i] = a / (1.0f + __expf(-a));
+          }
+        }
+        if (valid) {
+          uint4 o0, o1;
+          o0.x = pack_bf16x2(v[0], v[1]);
+          o0.y = pack_bf16x2(v[2], v[3]);
+          o0.z = pack_bf16x2(v[4], v[5]);
+          o0.w = pack_bf16x2(v[6], v[7]);
+          o1.x = pack_bf16x2(v[8], v[9]);
+          o1.y = pack_bf16x2(v[10], v[11]);
+          o1.z = pack_bf16x2(v[12], v[13]);
+          o1.w = pack_bf16x2(v[14], v[15]);
+          uint4 *dst = reinterpret_cast<uint4 *>(yrow + j);
+          dst[0] = o0;
+          dst[1] = o1;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+  if (!ok && threadIdx.x == 0) {
+    // A wait ran out: give copies already issued time to land before the
+    // CTA's shared memory is handed to another block.
+    __nanosleep(100000);
+  }
+}
+
+}  // namespace
+
+size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb) {
+  return make_layout(kc, nt, kh, kw, na, nb).total + 1024;  // + alignment slack
+}
+
+int umma_tile_w() { return kTW; }
+int umma_tile_h() { return kTH; }
+
+cudaError_t umma_prepare() {
+  // Opt in to the largest dynamic shared memory window once per process.
+  constexpr int kMaxSmem = 227 * 1024;
+  cudaError_t e = cudaFuncSetAttribute(conv_umma_kernel<64>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(conv_umma_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kMaxSmem);
+  return e;
+}
+
+cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_cache,
+                             const UmmaArgs &args, int kc, unsigned grid, cudaStream_t stream) {
+  const size_t smem = umma_smem_bytes(kc, args.nt, args.kh, args.kw, args.na, args.nb);
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  if (kc == 64) {
+    conv_umma_kernel<64><<<grid, kThreads, smem, stream>>>(map_x, map_cache, args);
+  } else if (kc == 32) {
+    conv_umma_kernel<32><<<grid, kThreads, smem, stream>>>(map_x, map_cache, args);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace cc3d

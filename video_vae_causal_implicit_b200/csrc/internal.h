@@ -1,0 +1,83 @@
+// internal.h -- declarations shared by the kernels and the C-ABI layer of
+// libcc3d.so (not part of the public interface).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace cc3d {
+
+// Arguments of the tcgen05 implicit-GEMM conv kernel.
+struct UmmaArgs {
+  const uint8_t *wimg;            // re-tiled weights, [ntile][tap][cchunk][KC/8][NT][8] bf16
+  const float *bias;              // [c_out] fp32 (never null; zeros when absent)
+  const float *gamma;             // [c_out] (RMS epilogue)
+  const float *beta;              // [c_out] or null
+  const __nv_bfloat16 *residual;  // [n][t][h][w][c_out] or null
+  __nv_bfloat16 *y;               // [n][t][h][w][c_out]
+  int *status;                    // device status word
+  unsigned long long wait_limit_ns;
+  int n, t, h, w, c_in, c_out;
+  int kt, kh, kw, pad_h, pad_w;
+  int nt, n_ntiles, tiles_w, tiles_h;
+  int na, nb;                     // pipeline depths (A halo stages, B weight stages)
+  int tmem_cols;
+  int epi;                        // 0 bias, 1 bias + residual, 2 bias + RMS + SiLU
+  int has_cache;
+};
+
+size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb);
+cudaError_t umma_prepare();
+int umma_tile_w();
+int umma_tile_h();
+cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_cache,
+                             const UmmaArgs &args, int kc, unsigned grid, cudaStream_t stream);
+
+// Weight re-tiling for the UMMA kernel (plan time):
+// W[c_out][c_in][kt][kh][kw] (bf16) -> image[ntile][tap][cchunk][kc/8][nt][8].
+cudaError_t launch_repack_umma(const __nv_bfloat16 *w, uint8_t *img, int c_out, int c_in,
+                               int taps, int nt, int kc, cudaStream_t stream);
+
+// Thin first-layer conv (c_in small): weights to [tap*c_in padded to kpad][c_out]
+// image and the kernel itself.
+struct ThinArgs {
+  const __nv_bfloat16 *x;         // [n][t][h][w][c_in]
+  const __nv_bfloat16 *cache;     // [n][kt-1][h][w][c_in] or null
+  const uint8_t *wimg;            // [kpad/8][c_out][8] bf16 core-matrix image
+  const float *bias;              // [c_out]
+  __nv_bfloat16 *y;               // [n][t][h][w][c_out]
+  int *status;
+  unsigned long long wait_limit_ns;
+  int n, t, h, w, c_in, c_out, kt, kh, kw, pad_h, pad_w;
+  int kpad;                       // K padded to a multiple of 16
+  int tiles_w, tiles_h, n_tiles;
+  int tmem_cols;
+};
+cudaError_t launch_repack_thin(const __nv_bfloat16 *w, uint8_t *img, int c_out, int c_in,
+                               int taps, int kpad, cudaStream_t stream);
+size_t thin_smem_bytes(const ThinArgs &a);
+cudaError_t launch_conv_thin(const ThinArgs &args, unsigned grid, cudaStream_t stream);
+
+// fp32 SIMT direct convolution.
+struct Fp32Args {
+  const float *x, *cache, *w, *bias;
+  float *y;
+  int n, t, h, w_, c_in, c_out, kt, kh, kw, pad_h, pad_w;
+};
+cudaError_t launch_conv_fp32(const Fp32Args &a, cudaStream_t stream);
+
+// cache_out = last (kt-1) frames of concat(cache_in or zeros, src[0..t)).
+cudaError_t launch_cache_update(const void *cache_in, const void *src, void *cache_out, int n,
+                                int t, int frames, size_t frame_bytes, cudaStream_t stream);
+
+// RMS_norm + SiLU over channels, bf16 in/out.
+cudaError_t launch_rmsnorm_silu(const __nv_bfloat16 *x, const float *gamma, const float *beta,
+                                long long voxels, int c, __nv_bfloat16 *y, cudaStream_t stream);
+
+// Host-side launch counter (all kernels of this library).
+void count_launch();
+
+}  // namespace cc3d
