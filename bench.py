@@ -1,0 +1,462 @@
+"""Benchmark of the causal Conv3D hot path (libcc3d.so) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cc3d|reference] [--sweep]
+
+Workload (one "step"): the decoder latent-resolution causal conv,
+bf16, C_in = C_out = 384 on x[1, 384, 5, 30, 52], 3x3x3, run once over the
+whole sequence and once as 5 one-frame chunks that carry a 2-frame cache
+(the outputs of the two are bitwise identical; the tests check that).
+FLOP per step = 2 * (2 * C_out * C_in * 27 * T * H * W).  Inputs are 1.2 MB,
+smaller than L2, so L2 is flushed (a 512 MiB buffer is rewritten) before
+every timed step and the flush is outside the timed events.
+
+The same JSON line carries the residual block (x[1, 192, 9, 240, 416]:
+RMS_norm+SiLU -> conv -> RMS_norm+SiLU (fused) -> conv + x (fused)) as
+``resblock`` with its latency, and with ``--sweep`` the encoder convs
+(3 -> 96, 96 -> 96 at 17 x 480 x 832) and the streaming channel/resolution
+sweep (21 one-frame chunks, CUDA-graph captured).
+
+Multi-GPU: the path runs as independent replicas (one process per GPU, no
+data-path collective); ``value`` is the FLOP all ranks processed divided by
+the slowest rank's time ("scaling": "weak").
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload (the only other place this script runs the oracle besides the
+``cpu_baseline`` leg).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "causal Conv3D effective TFLOP/s and % of bf16 tensor roofline; resblock latency"
+WORKLOAD = ("decoder latent-res causal conv bf16 384->384 k3x3x3, x[1,384,5,30,52], "
+            "whole sequence + 5 one-frame chunks with 2-frame cache per step")
+C2 = dict(c=384, t=5, h=30, w=52)
+C4 = dict(c=192, t=9, h=240, w=416)
+
+
+def conv_flop(n, cin, cout, t, h, w, taps=27):
+    return 2.0 * n * cout * cin * taps * t * h * w
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ---- clocks sampled during the timed region ---------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="cc3d_clocks_", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        under_load = [s for s in sm if smax and s > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(under_load) if under_load else None,
+                "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---- the reference arm: the fp64 oracle on a bounded sample -----------------------
+
+def oracle_sample_rate(points_count, seed=11):
+    """Time the oracle on `points_count` output voxels of the workload; returns
+    (TFLOP/s, seconds, flop)."""
+    import oracle
+    from video_vae_causal_implicit_b200 import synth
+    case = synth.conv_case(C2["c"], C2["c"], C2["t"], C2["h"], C2["w"])
+    x = synth.ndhwc(case["x"])
+    pts = synth.sample_points(1, C2["t"], C2["h"], C2["w"], points_count, seed)
+    t0 = time.perf_counter()
+    oracle.causal_conv3d_points(synth.ncthw_view(x), case["w"], case["b"].double().numpy(), None,
+                                pts)
+    dt = time.perf_counter() - t0
+    flop = 2.0 * points_count * C2["c"] * C2["c"] * 27
+    return flop / dt / 1e12, dt, flop
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    cores = len(os.sched_getaffinity(0))
+    pts = 256  # about 2 GFLOP of fp64 work per step
+    for _ in range(args.warmup):
+        oracle_sample_rate(pts, seed=1)
+    times, flops = [], 0.0
+    for k in range(args.steps):
+        _, dt, fl = oracle_sample_rate(pts, seed=100 + k)
+        times.append(dt)
+        flops += fl
+    total = sum(times)
+    value = flops / total / 1e12
+    sample = (f"{pts} seeded output voxels (all 384 channels each) of the 384->384 conv on "
+              f"[1,384,5,30,52] per step, fp64")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "l2": "n/a (host)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---- the CUDA arm ------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cc3d", choices=["cc3d", "reference"])
+    ap.add_argument("--sweep", action="store_true", help="also time configs 3 and 5")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from video_vae_causal_implicit_b200 import cc3d, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks = load_peaks()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def flush_l2(k):
+        flush.fill_(k & 0xFF)
+
+    # --- workload: config 2 ---
+    c, T, H, W = C2["c"], C2["t"], C2["h"], C2["w"]
+    case = synth.conv_case(c, c, T, H, W)
+    x = synth.ndhwc(case["x"]).to(dev)
+    plan = cc3d.Plan(case["w"].to(dev), case["b"].to(dev), h=H, w=W, max_t=T)
+    y_whole = torch.empty((1, T, H, W, c), dtype=torch.bfloat16, device=dev)
+    xs = [x[:, k:k + 1].contiguous() for k in range(T)]
+    ys = [torch.empty((1, 1, H, W, c), dtype=torch.bfloat16, device=dev) for _ in range(T)]
+    caches = [torch.empty((1, 2, H, W, c), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    flop_step = 2 * conv_flop(1, c, c, T, H, W)
+
+    def step(xin=None):
+        src = x if xin is None else xin
+        plan.forward(src, y_whole)
+        cache = None
+        for k in range(T):
+            xk = xs[k] if xin is None else src[:, k:k + 1]
+            plan.forward(xk, ys[k], t=1, cache_in=cache, cache_out=caches[k % 2])
+            cache = caches[k % 2]
+
+    for k in range(args.warmup):
+        flush_l2(k)
+        step()
+    cc3d.sync_status()
+
+    sampler = ClockSampler(local)
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    launches0 = cc3d.cc3d_launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for k in range(args.steps):
+        flush_l2(k)
+        ev0[k].record(stream)
+        step()
+        ev1[k].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    launches = cc3d.cc3d_launch_count() - launches0
+    cc3d.sync_status()
+    step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
+    ms_local = sum(step_ms) / len(step_ms)
+    ms = max_over_ranks(ms_local)
+    value = world * flop_step / (ms * 1e-3) / 1e12
+
+    # --- roofline of the dominant kernel: the whole-sequence conv launch ---
+    ew0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ew1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for k in range(args.steps):
+        flush_l2(k)
+        ew0[k].record(stream)
+        plan.forward(x, y_whole)
+        ew1[k].record(stream)
+    torch.cuda.synchronize()
+    whole_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ew0, ew1))
+    achieved = conv_flop(1, c, c, T, H, W) / (whole_ms * 1e-3) / 1e12
+    # chunk (streaming) launch time for context
+    chunk_ms = (ms_local - whole_ms) / T
+
+    # --- end to end through the public API with host buffers ---
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty((2,) + tuple(y_whole.shape), dtype=torch.bfloat16).pin_memory()
+    x_dev2 = torch.empty_like(x)
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for k in range(args.warmup + args.steps):
+        flush_l2(k)
+        i = k - args.warmup
+        if i >= 0:
+            e0[i].record(stream)
+        x_dev2.copy_(x_host, non_blocking=True)
+        step(x_dev2)
+        y_host[0].copy_(y_whole, non_blocking=True)
+        for kk in range(T):
+            y_host[1][:, kk:kk + 1].copy_(ys[kk], non_blocking=True)
+        if i >= 0:
+            e1[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(e0, e1)))
+    e2e = {"value": world * flop_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": 2 * y_whole.numel() * 2,
+           "ms_per_step": e2e_ms}
+
+    # --- residual block (config 4): latency ---
+    resblock = None
+    cb, Tb, Hb, Wb = C4["c"], C4["t"], C4["h"], C4["w"]
+    bc = synth.block_case(cb, Tb, Hb, Wb)
+    blk = cc3d.Block(*(bc[k].to(dev) for k in ("w1", "b1", "g1", "w2", "b2", "g2")), h=Hb, w=Wb,
+                     max_t=Tb)
+    xb = synth.ndhwc(bc["x"]).to(dev)
+    yb = torch.empty_like(xb)
+    for _ in range(args.warmup):
+        blk.forward(xb, yb)
+    torch.cuda.synchronize()
+    b0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    b1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for k in range(args.steps):
+        b0[k].record(stream)
+        blk.forward(xb, yb)
+        b1[k].record(stream)
+    torch.cuda.synchronize()
+    cc3d.sync_status()
+    blk_ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in zip(b0, b1)))
+    blk_flop = 2 * conv_flop(1, cb, cb, Tb, Hb, Wb)
+    act_bytes = Tb * Hb * Wb * cb * 2
+    blk_bytes = 7 * act_bytes  # x r, a0 w, a0 r, a1 w, a1 r, x r (residual), y w
+    roof_ms = max(blk_flop / (peaks["bf16_tflops_sustained"] * 1e12),
+                  blk_bytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    resblock = {"workload": "Wan residual block bf16 192ch x[1,192,9,240,416]",
+                "ms": blk_ms, "tflops": blk_flop / (blk_ms * 1e-3) / 1e12,
+                "roofline_ms": roof_ms, "frac": roof_ms / blk_ms,
+                "peak_basis": "sustained bf16 (" + peaks["source"] + ")"}
+    del blk, xb, yb
+
+    sweep = run_sweep(args, dev, stream, peaks, flush_l2) if args.sweep else None
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        pts = 2048
+        rate, dt, fl = oracle_sample_rate(pts)
+        cpu = {"value": rate, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
+               "kind": "oracle", "seconds": dt,
+               "sample": f"{pts} seeded output voxels x 384 channels of the 384->384 conv "
+                         f"on [1,384,5,30,52] ({fl / 1e9:.1f} GFLOP fp64)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) activations, Kaiming-uniform weights)",
+            "config": {"workload": WORKLOAD, "global_batch": world, "parallelism": f"replicas{world}",
+                       "l2": "flushed before every timed step (512 MiB rewrite, untimed)",
+                       "flop_per_step": flop_step},
+            "roofline": {"bound": "tensor", "achieved": achieved,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                         "kernel": "conv_umma_kernel (whole-sequence launch)",
+                         "launch_ms": whole_ms, "peak_basis": "burst bf16 (" + peaks["source"] + ")"},
+            "streaming_chunk_ms": chunk_ms,
+            "resblock": resblock,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        if sweep is not None:
+            line["sweep"] = sweep
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_sweep(args, dev, stream, peaks, flush_l2):
+    """Configs 3 (encoder full-res convs) and 5 (streaming sweep)."""
+    import torch
+
+    from video_vae_causal_implicit_b200 import cc3d, synth
+    out = {}
+    reps = max(3, min(args.steps, 10))
+
+    def timed(fn, flush=False):
+        for k in range(2):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for k in range(reps):
+            if flush:
+                flush_l2(k)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    # config 3b: 96 -> 96 at 17 x 480 x 832
+    T, H, W = 17, 480, 832
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    x96 = torch.randn((1, T, H, W, 96), generator=g, device=dev).to(torch.bfloat16)
+    w96 = synth.kaiming_uniform(96, 96, (3, 3, 3), 1).to(dev)
+    b96 = synth.uniform((96,), -0.1, 0.1, 2).to(dev)
+    p96 = cc3d.Plan(w96, b96, h=H, w=W, max_t=T)
+    y96 = torch.empty_like(x96)
+    ms = timed(lambda: p96.forward(x96, y96))
+    fl = conv_flop(1, 96, 96, T, H, W)
+    out["cfg3b_96to96_17x480x832"] = {"ms": ms, "tflops": fl / ms / 1e9,
+                                      "frac": fl / ms / 1e9 / peaks["bf16_tflops"]}
+    del p96, x96, y96
+    # config 5: C x resolution, 21 one-frame chunks, graph-captured
+    for cc in (96, 192, 384):
+        for (H, W) in ((90, 160), (180, 320), (360, 640)):
+            T = 21
+            x5 = torch.randn((1, T, H, W, cc), generator=g, device=dev).to(torch.bfloat16)
+            w5 = synth.kaiming_uniform(cc, cc, (3, 3, 3), 1).to(dev)
+            b5 = synth.uniform((cc,), -0.1, 0.1, 2).to(dev)
+            p5 = cc3d.Plan(w5, b5, h=H, w=W, max_t=1)
+            y5 = torch.empty_like(x5)
+            xsl = [x5[:, k:k + 1] for k in range(T)]
+            ysl = [y5[:, k:k + 1] for k in range(T)]
+            cbuf = [torch.empty((1, 2, H, W, cc), dtype=torch.bfloat16, device=dev)
+                    for _ in range(2)]
+
+            def run():
+                cache = None
+                for k in range(T):
+                    p5.forward(xsl[k], ysl[k], t=1, cache_in=cache, cache_out=cbuf[k % 2])
+                    cache = cbuf[k % 2]
+
+            run()
+            torch.cuda.synchronize()
+            gs = torch.cuda.Stream(device=dev)
+            graph = torch.cuda.CUDAGraph()
+            gs.wait_stream(stream)
+            with torch.cuda.stream(gs):
+                graph.capture_begin()
+                cache = None
+                for k in range(T):
+                    p5.forward(xsl[k], ysl[k], t=1, cache_in=cache, cache_out=cbuf[k % 2],
+                               stream=gs)
+                    cache = cbuf[k % 2]
+                graph.capture_end()
+            stream.wait_stream(gs)
+            ms = timed(graph.replay, flush=True)
+            fl = conv_flop(1, cc, cc, T, H, W)
+            out[f"cfg5_c{cc}_{H}x{W}_21x1frame"] = {"ms": ms, "tflops": fl / ms / 1e9,
+                                                    "frac": fl / ms / 1e9 / peaks["bf16_tflops"]}
+            del graph, p5, x5, y5, cbuf
+            torch.cuda.synchronize()
+    cc3d.sync_status()
+    return out
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -185,6 +185,7 @@ cc3d_status check_desc(const cc3d_desc *d, int *variant) {
   if (d->dtype != CC3D_BF16) return CC3D_ERR_INVALID_ARG;
   if (d->c_out % 16 != 0) return CC3D_ERR_UNSUPPORTED;
   if (d->c_in % 32 == 0) {
+    if (d->kh != d->kw) return CC3D_ERR_UNSUPPORTED;
     if (d->epi == CC3D_EPI_BIAS_RMS_SILU && d->c_out > 256) return CC3D_ERR_UNSUPPORTED;
     *variant = CC3D_VARIANT_UMMA;
     return CC3D_OK;

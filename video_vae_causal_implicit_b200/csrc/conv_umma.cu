@@ -72,7 +72,7 @@ __host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw
   return L;
 }
 
-template <int KC>
+template <int KC, int KS>
 __global__ void __launch_bounds__(kThreads, 1)
     conv_umma_kernel(const __grid_constant__ CUtensorMap map_x,
                      const __grid_constant__ CUtensorMap map_cache, UmmaArgs p) {
@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // request, not a guarantee).
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const SmemLayout L = make_layout(KC, p.nt, p.kh, p.kw, p.na, p.nb);
+  const SmemLayout L = make_layout(KC, p.nt, KS, KS, p.na, p.nb);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
   uint64_t *full_a = bars;
   uint64_t *empty_a = full_a + L.na;
@@ -105,9 +105,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int w0 = tw_i * kTW, h0 = th_i * kTH;
 
   const int n_cc = p.c_in / KC;          // channel chunks
-  const int taps_sp = p.kh * p.kw;       // spatial taps per kt
   const int n_a = p.kt * n_cc;           // A stages per tile
-  const uint32_t halo_w = kTW + p.kw - 1;
+  const uint32_t halo_w = kTW + KS - 1;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L.na; ++i) {
@@ -137,11 +136,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------ producer ------------------------------------
     if (lane == 0) {
-      const uint32_t a_bytes = (KC / 8) * (8u * 2u * halo_w * (kTH + p.kh - 1));
+      const uint32_t a_bytes = (KC / 8) * (8u * 2u * halo_w * (kTH + KS - 1));
+      int sa = 0, sb = 0;
+      uint32_t pa = 0, pb = 0;
+      const uint8_t *wsrc = p.wimg + static_cast<size_t>(ntile) * p.kt * KS * KS * n_cc * L.b_stage;
       for (int ia = 0; ia < n_a && ok; ++ia) {
         const int kt = ia / n_cc, cc = ia % n_cc;
-        const int sa = ia % L.na;
-        if (!mbar_wait_bounded(&empty_a[sa], ((ia / L.na) & 1) ^ 1, p.wait_limit_ns, p.status, 1)) {
+        if (!mbar_wait_bounded(&empty_a[sa], pa ^ 1, p.wait_limit_ns, p.status, 1)) {
           ok = false;
           break;
         }
@@ -153,21 +154,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t dst = smem_base + L.a_off + sa * L.a_stage;
 #pragma unroll
         for (int s = 0; s < KC / 8; ++s)
-          tma_load_5d(dst + s * L.slab, map, &full_a[sa], cc * KC + s * 8, w0 - p.pad_w,
-                      h0 - p.pad_h, tc, n_img);
-        for (int ts = 0; ts < taps_sp; ++ts) {
-          const int ib = ia * taps_sp + ts;
-          const int sb = ib % L.nb;
-          if (!mbar_wait_bounded(&empty_b[sb], ((ib / L.nb) & 1) ^ 1, p.wait_limit_ns, p.status,
-                                 2)) {
+          tma_load_5d(dst + s * L.slab, map, &full_a[sa], cc * KC + s * 8, w0 - KS / 2,
+                      h0 - KS / 2, tc, n_img);
+        if (++sa == L.na) { sa = 0; pa ^= 1; }
+#pragma unroll 1
+        for (int ts = 0; ts < KS * KS; ++ts) {
+          if (!mbar_wait_bounded(&empty_b[sb], pb ^ 1, p.wait_limit_ns, p.status, 2)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&full_b[sb], L.b_stage);
-          const size_t stage_idx =
-              (static_cast<size_t>(ntile) * p.kt * taps_sp + kt * taps_sp + ts) * n_cc + cc;
-          bulk_load(smem_base + L.b_off + sb * L.b_stage, p.wimg + stage_idx * L.b_stage,
+          const size_t stage_idx = static_cast<size_t>(kt * KS * KS + ts) * n_cc + cc;
+          bulk_load(smem_base + L.b_off + sb * L.b_stage, wsrc + stage_idx * L.b_stage,
                     L.b_stage, &full_b[sb]);
+          if (++sb == L.nb) { sb = 0; pb ^= 1; }
         }
       }
     }
@@ -177,36 +177,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = idesc_bf16_f32(kM, p.nt);
       const uint32_t a_sbo = halo_w * 16u;
       const uint32_t b_lbo = static_cast<uint32_t>(p.nt) * 16u;
+      // Descriptors of stage 0; other stages, taps and K steps only move the
+      // start address (low 14 bits, 16-byte units), so they are additions.
+      const uint64_t adesc0 = smem_desc_noswizzle(smem_base + L.a_off, L.slab, a_sbo);
+      const uint64_t bdesc0 = smem_desc_noswizzle(smem_base + L.b_off, b_lbo, 128u);
+      const uint32_t slab16 = L.slab >> 4, blbo16 = b_lbo >> 4;
       uint32_t accumulate = 0;
+      int sa = 0, sb = 0;
+      uint32_t pa = 0, pb = 0;
       for (int ia = 0; ia < n_a && ok; ++ia) {
-        const int sa = ia % L.na;
-        if (!mbar_wait_bounded(&full_a[sa], (ia / L.na) & 1, p.wait_limit_ns, p.status, 3)) {
+        if (!mbar_wait_bounded(&full_a[sa], pa, p.wait_limit_ns, p.status, 3)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a_stage = smem_base + L.a_off + sa * L.a_stage;
-        for (int ts = 0; ts < taps_sp; ++ts) {
-          const int ib = ia * taps_sp + ts;
-          const int sb = ib % L.nb;
-          if (!mbar_wait_bounded(&full_b[sb], (ib / L.nb) & 1, p.wait_limit_ns, p.status, 4)) {
+        const uint64_t a_st = adesc0 + ((sa * L.a_stage) >> 4);
+#pragma unroll
+        for (int ts = 0; ts < KS * KS; ++ts) {
+          if (!mbar_wait_bounded(&full_b[sb], pb, p.wait_limit_ns, p.status, 4)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const int kh = ts / p.kw, kw = ts % p.kw;
-          const uint32_t a_tap = a_stage + (kh * halo_w + kw) * 16u;
-          const uint32_t b_stage = smem_base + L.b_off + sb * L.b_stage;
+          const uint64_t a_tap = a_st + ((ts / KS) * halo_w + (ts % KS));
+          const uint64_t b_st = bdesc0 + ((sb * L.b_stage) >> 4);
 #pragma unroll
           for (int j = 0; j < KC / 16; ++j) {
-            const uint64_t ad = smem_desc_noswizzle(a_tap + 2 * j * L.slab, L.slab, a_sbo);
-            const uint64_t bd = smem_desc_noswizzle(b_stage + 2 * j * b_lbo, b_lbo, 128u);
-            umma_bf16(tmem_base, ad, bd, idesc, accumulate);
+            umma_bf16(tmem_base, a_tap + 2 * j * slab16, b_st + 2 * j * blbo16, idesc, accumulate);
             accumulate = 1;
           }
           umma_commit(&empty_b[sb]);  // frees the B stage when these MMAs finish
+          if (++sb == L.nb) { sb = 0; pb ^= 1; }
         }
         umma_commit(&empty_a[sa]);
+        if (++sa == L.na) { sa = 0; pa ^= 1; }
       }
       umma_commit(acc_full);
     }
@@ -307,28 +311,36 @@ size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb) {
 int umma_tile_w() { return kTW; }
 int umma_tile_h() { return kTH; }
 
+template <int KC, int KS>
+cudaError_t set_smem_attr() {
+  return cudaFuncSetAttribute(conv_umma_kernel<KC, KS>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+}
+
 cudaError_t umma_prepare() {
   // Opt in to the largest dynamic shared memory window once per process.
-  constexpr int kMaxSmem = 227 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(conv_umma_kernel<64>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(conv_umma_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kMaxSmem);
+  cudaError_t e = set_smem_attr<64, 3>();
+  if (e == cudaSuccess) e = set_smem_attr<32, 3>();
+  if (e == cudaSuccess) e = set_smem_attr<64, 1>();
+  if (e == cudaSuccess) e = set_smem_attr<32, 1>();
   return e;
 }
 
 cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_cache,
                              const UmmaArgs &args, int kc, unsigned grid, cudaStream_t stream) {
   const size_t smem = umma_smem_bytes(kc, args.nt, args.kh, args.kw, args.na, args.nb);
-  if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  if (kc == 64) {
-    conv_umma_kernel<64><<<grid, kThreads, smem, stream>>>(map_x, map_cache, args);
-  } else if (kc == 32) {
-    conv_umma_kernel<32><<<grid, kThreads, smem, stream>>>(map_x, map_cache, args);
-  } else {
+  if (smem > 227 * 1024 || args.kh != args.kw || (args.kh != 1 && args.kh != 3))
     return cudaErrorInvalidValue;
-  }
+  if (kc == 64 && args.kh == 3)
+    conv_umma_kernel<64, 3><<<grid, kThreads, smem, stream>>>(map_x, map_cache, args);
+  else if (kc == 32 && args.kh == 3)
+    conv_umma_kernel<32, 3><<<grid, kThreads, smem, stream>>>(map_x, map_cache, args);
+  else if (kc == 64 && args.kh == 1)
+    conv_umma_kernel<64, 1><<<grid, kThreads, smem, stream>>>(map_x, map_cache, args);
+  else if (kc == 32 && args.kh == 1)
+    conv_umma_kernel<32, 1><<<grid, kThreads, smem, stream>>>(map_x, map_cache, args);
+  else
+    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 

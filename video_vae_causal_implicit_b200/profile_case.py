@@ -1,0 +1,90 @@
+"""Run one named workload a few times, for profiler captures (ncu).
+
+    python -m video_vae_causal_implicit_b200.profile_case --case NAME [--reps R]
+
+Cases (seeded synthetic inputs, generated on the device):
+  c2      384 -> 384 causal conv, whole sequence, x[1,384,5,30,52]
+  c2s     the same as 5 one-frame chunks with a 2-frame cache
+  c3a     3 -> 96 causal conv on x[1,3,17,480,832]
+  c3b     96 -> 96 causal conv on x[1,96,17,480,832]
+  c4      the residual block on x[1,192,9,240,416]
+  c4s     the residual block on a 3-frame slice x[1,192,3,240,416]
+  c5big   384 -> 384, one frame of 360 x 640 with a 2-frame cache
+Prints nothing but a final "ok"; timing comes from the profiler.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import cc3d, synth
+
+
+def _rand(shape, dev, seed=0):
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    return torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+
+
+def build_case(name, dev):
+    if name in ("c2", "c2s"):
+        c, T, H, W = 384, 5, 30, 52
+    elif name == "c3a":
+        c, T, H, W = 3, 17, 480, 832
+    elif name == "c3b":
+        c, T, H, W = 96, 17, 480, 832
+    elif name in ("c4", "c4s"):
+        c, T, H, W = 192, (9 if name == "c4" else 3), 240, 416
+    elif name == "c5big":
+        c, T, H, W = 384, 1, 360, 640
+    else:
+        raise SystemExit(f"unknown case {name}")
+    x = _rand((1, T, H, W, c), dev)
+    if name in ("c4", "c4s"):
+        w1 = synth.kaiming_uniform(c, c, (3, 3, 3), 1).to(dev)
+        w2 = synth.kaiming_uniform(c, c, (3, 3, 3), 4).to(dev)
+        b1 = synth.uniform((c,), -0.1, 0.1, 2).to(dev)
+        b2 = synth.uniform((c,), -0.1, 0.1, 5).to(dev)
+        g1 = synth.uniform((c,), 0.5, 1.5, 3).to(dev)
+        g2 = synth.uniform((c,), 0.5, 1.5, 6).to(dev)
+        blk = cc3d.Block(w1, b1, g1, w2, b2, g2, h=H, w=W, max_t=T)
+        y = torch.empty_like(x)
+        return lambda: blk.forward(x, y), [blk]
+    cout = 96 if name == "c3a" else c
+    wt = synth.kaiming_uniform(cout, c, (3, 3, 3), 1).to(dev)
+    b = synth.uniform((cout,), -0.1, 0.1, 2).to(dev)
+    if name == "c2s":
+        plan = cc3d.Plan(wt, b, h=H, w=W, max_t=1)
+        ys = [torch.empty((1, 1, H, W, cout), dtype=torch.bfloat16, device=dev) for _ in range(T)]
+        cb = [torch.empty((1, 2, H, W, c), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+
+        def run():
+            cache = None
+            for k in range(T):
+                plan.forward(x[:, k:k + 1], ys[k], t=1, cache_in=cache, cache_out=cb[k % 2])
+                cache = cb[k % 2]
+        return run, [plan]
+    plan = cc3d.Plan(wt, b, h=H, w=W, max_t=T)
+    y = torch.empty((1, T, H, W, cout), dtype=torch.bfloat16, device=dev)
+    cache = _rand((1, 2, H, W, c), dev, 9) if name == "c5big" else None
+    return (lambda: plan.forward(x, y, cache_in=cache)), [plan]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--case", required=True)
+    ap.add_argument("--reps", type=int, default=3)
+    args = ap.parse_args()
+    dev = torch.device("cuda", 0)
+    run, keep = build_case(args.case, dev)
+    for _ in range(args.reps):
+        run()
+    torch.cuda.synchronize()
+    cc3d.sync_status()
+    del keep
+    print("ok")
+
+
+if __name__ == "__main__":
+    main()
