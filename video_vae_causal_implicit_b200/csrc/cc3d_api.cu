@@ -116,7 +116,7 @@ struct cc3d_plan {
   int variant;
   int device;
   // UMMA
-  int kc, nt, n_ntiles, na, nb, tmem_cols;
+  int kc, nt, n_ntiles, na, nb, tmem_cols, sm_count, ctas_per_sm;
   uint8_t *wimg;
   // fp32 / thin
   void *wraw;
@@ -242,22 +242,48 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
     e = umma_prepare();
     if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
     if (!status_ptr()) { s = CC3D_ERR_CUDA; goto fail; }
-    p->kc = (desc->c_in % 64 == 0) ? 64 : 32;
-    int split = 1;
-    while (desc->c_out / split > 256 || (desc->c_out % split) != 0 ||
-           ((desc->c_out / split) % 16) != 0)
-      ++split;
-    p->nt = desc->c_out / split;
-    p->n_ntiles = split;
-    int cols = 32;
-    while (cols < p->nt) cols *= 2;
-    p->tmem_cols = cols;
+    p->kc = (desc->c_in % 64 == 0) ? 64 : (desc->c_in % 96 == 0) ? 96 : 32;
+    if (cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, p->device) !=
+        cudaSuccess)
+      p->sm_count = 148;
+    // N tile: the largest channel split that divides c_out (a multiple of
+    // 16, at most 256: the tcgen05 N limit).  Measured on B200: the time of
+    // one 128 x N x 16 MMA has a floor of ~130 cycles for N <= 192, so
+    // smaller N tiles only add CTAs that each run at lower efficiency.  The
+    // choice depends on c_out only, never on t, so a streamed sequence and a
+    // whole-sequence call run identical arithmetic.
+    {
+      int best_nt = 0;
+      for (int nt = 256; nt >= 16 && !best_nt; nt -= 16) {
+        if (desc->c_out % nt) continue;
+        if (desc->epi == CC3D_EPI_BIAS_RMS_SILU && nt != desc->c_out) continue;
+        best_nt = nt;
+      }
+      if (!best_nt) { s = CC3D_ERR_UNSUPPORTED; goto fail; }
+      p->nt = best_nt;
+      p->n_ntiles = desc->c_out / best_nt;
+    }
+    {
+      int cols = 32;
+      while (cols < 2 * p->nt) cols *= 2;  // two accumulators (double buffer)
+      p->tmem_cols = cols;
+    }
     // Pipeline depths: two halo stages, as many weight stages as fit.
     p->na = 2;
-    const size_t budget = 200 * 1024;
-    int nb = 8;
-    while (nb > 2 && umma_smem_bytes(p->kc, p->nt, desc->kh, desc->kw, p->na, nb) > budget) --nb;
-    p->nb = nb;
+    {
+      const size_t budget = 200 * 1024;
+      int nb = 8;
+      while (nb > 2 && umma_smem_bytes(p->kc, p->nt, desc->kh, desc->kw, p->na, nb) > budget)
+        --nb;
+      p->nb = nb;
+      const size_t smem =
+          umma_launch_smem(p->kc, p->nt, desc->kh, p->na, p->nb, p->tmem_cols) + 1024;
+      int per_sm = static_cast<int>((228 * 1024) / smem);
+      if (per_sm > 512 / p->tmem_cols) per_sm = 512 / p->tmem_cols;
+      if (per_sm > 2) per_sm = 2;
+      if (per_sm < 1) per_sm = 1;
+      p->ctas_per_sm = per_sm;
+    }
     p->st.tile_h = umma_tile_h();
     p->st.tile_w = umma_tile_w();
     p->st.n_tile = p->nt;
@@ -367,7 +393,9 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
     a.epi = static_cast<int>(d.epi);
     a.has_cache = (cache_in && front > 0) ? 1 : 0;
     tiles = static_cast<uint64_t>(d.n) * t * a.tiles_h * a.tiles_w * a.n_ntiles;
-    e = launch_conv_umma(mx, mc, a, p->kc, static_cast<unsigned>(tiles), stream);
+    const uint64_t slots = static_cast<uint64_t>(p->sm_count) * p->ctas_per_sm;
+    const uint64_t grid = tiles < slots ? tiles : slots;
+    e = launch_conv_umma(mx, mc, a, p->kc, static_cast<unsigned>(grid), stream);
     count_launch();
   }
   if (e == cudaSuccess && cache_out && front > 0)

@@ -6,9 +6,10 @@
 // accumulator held in tensor memory; bias is added once in the epilogue
 // ("cache-aware video decoder lowering" summary: bias after the sum).
 //
-// Tiling.  A CTA owns one output tile of TW = 8 columns x TH = 16 rows of
-// one frame (M = 128 rows of the GEMM, row m = 8 * r + c) and NT output
-// channels.  The K loop runs over (kt, channel chunk of KC, kh, kw).
+// Tiling.  An output tile is TW = 8 columns x TH = 16 rows of one frame
+// (M = 128 rows of the GEMM, row m = 8 * r + c) by NT output channels.  The
+// kernel is persistent: one CTA per SM walks the tiles round-robin.  The K
+// loop of a tile runs over (kt, channel chunk of KC, kh, kw).
 //
 // A operand: for each (kt, channel chunk) one TMA box brings the input
 // halo of the tile -- (TH + kh - 1) x (TW + kw - 1) pixels x KC channels --
@@ -29,8 +30,10 @@
 // Warp roles (192 threads): warp 0 issues the loads, warp 1 owns tensor
 // memory and issues tcgen05.mma from one thread, warps 2..5 run the
 // epilogue (tensor memory -> registers -> bias / residual / RMS+SiLU ->
-// bf16 -> global).  Stages are handed over with mbarriers; every wait is
-// bounded and reports through the status word instead of hanging.
+// bf16 -> global).  Two accumulators live in tensor memory, so the
+// epilogue of one tile overlaps the MMAs of the next.  Stages are handed
+// over with mbarriers; every wait is bounded and reports through the status
+// word instead of hanging.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -48,6 +51,7 @@ constexpr int kTW = 8;    // tile columns (one core matrix of rows)
 constexpr int kTH = 16;   // tile rows -> M = 128
 constexpr int kM = kTW * kTH;
 constexpr int kThreads = 192;
+constexpr int kEpiWarps = 4;
 
 struct SmemLayout {
   uint32_t a_off, a_stage, slab, b_off, b_stage, bar_off, total;
@@ -67,9 +71,30 @@ __host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw
   L.a_off = 0;
   L.b_off = round_up(L.a_off + na * L.a_stage, 1024u);
   L.bar_off = round_up(L.b_off + nb * L.b_stage, 64u);
-  // full_a, empty_a, full_b, empty_b, acc_full, tmem slot
-  L.total = L.bar_off + 8u * (2 * na + 2 * nb + 1) + 16u;
+  // full_a, empty_a, full_b, empty_b, acc_full[2], acc_empty[2], tmem slot
+  L.total = L.bar_off + 8u * (2 * na + 2 * nb + 4) + 16u;
   return L;
+}
+
+struct TileCoord {
+  int ntile, n, t, h0, w0;
+};
+
+// Tile order: N tile fastest (CTAs sharing an input halo run together),
+// then tile column, tile row, frame, batch image.
+__device__ __forceinline__ TileCoord decode_tile(int tile, const UmmaArgs &p) {
+  TileCoord c;
+  c.ntile = tile % p.n_ntiles;
+  int mt = tile / p.n_ntiles;
+  const int tw = mt % p.tiles_w;
+  mt /= p.tiles_w;
+  const int th = mt % p.tiles_h;
+  mt /= p.tiles_h;
+  c.t = mt % p.t;
+  c.n = mt / p.t;
+  c.w0 = tw * kTW;
+  c.h0 = th * kTH;
+  return c;
 }
 
 template <int KC, int KS>
@@ -87,26 +112,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *empty_a = full_a + L.na;
   uint64_t *full_b = empty_a + L.na;
   uint64_t *empty_b = full_b + L.nb;
-  uint64_t *acc_full = empty_b + L.nb;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+  uint64_t *acc_full = empty_b + L.nb;   // [2]
+  uint64_t *acc_empty = acc_full + 2;    // [2]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
-  // ---- tile coordinates --------------------------------------------------------
-  const int ntile = blockIdx.x % p.n_ntiles;
-  int mt = blockIdx.x / p.n_ntiles;
-  const int tw_i = mt % p.tiles_w;
-  mt /= p.tiles_w;
-  const int th_i = mt % p.tiles_h;
-  mt /= p.tiles_h;
-  const int t_out = mt % p.t;
-  const int n_img = mt / p.t;
-  const int w0 = tw_i * kTW, h0 = th_i * kTH;
-
-  const int n_cc = p.c_in / KC;          // channel chunks
-  const int n_a = p.kt * n_cc;           // A stages per tile
+  const int n_cc = p.c_in / KC;   // channel chunks
+  const int n_a = p.kt * n_cc;    // A stages per tile
   const uint32_t halo_w = kTW + KS - 1;
+  const int n_tiles = p.n * p.t * p.tiles_h * p.tiles_w * p.n_ntiles;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L.na; ++i) {
@@ -117,7 +133,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full_b[i], 1);
       mbar_init(&empty_b[i], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], kEpiWarps);
+    }
     fence_mbar_init();
     prefetch_tmap(&map_x);
     if (p.has_cache) prefetch_tmap(&map_cache);
@@ -139,35 +158,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t a_bytes = (KC / 8) * (8u * 2u * halo_w * (kTH + KS - 1));
       int sa = 0, sb = 0;
       uint32_t pa = 0, pb = 0;
-      const uint8_t *wsrc = p.wimg + static_cast<size_t>(ntile) * p.kt * KS * KS * n_cc * L.b_stage;
-      for (int ia = 0; ia < n_a && ok; ++ia) {
-        const int kt = ia / n_cc, cc = ia % n_cc;
-        if (!mbar_wait_bounded(&empty_a[sa], pa ^ 1, p.wait_limit_ns, p.status, 1)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&full_a[sa], a_bytes);
-        const int tau = t_out + kt - (p.kt - 1);
-        const bool from_cache = tau < 0 && p.has_cache;
-        const CUtensorMap *map = from_cache ? &map_cache : &map_x;
-        const int tc = from_cache ? tau + (p.kt - 1) : tau;  // negative: zero fill
-        const uint32_t dst = smem_base + L.a_off + sa * L.a_stage;
-#pragma unroll
-        for (int s = 0; s < KC / 8; ++s)
-          tma_load_5d(dst + s * L.slab, map, &full_a[sa], cc * KC + s * 8, w0 - KS / 2,
-                      h0 - KS / 2, tc, n_img);
-        if (++sa == L.na) { sa = 0; pa ^= 1; }
-#pragma unroll 1
-        for (int ts = 0; ts < KS * KS; ++ts) {
-          if (!mbar_wait_bounded(&empty_b[sb], pb ^ 1, p.wait_limit_ns, p.status, 2)) {
+      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+        const TileCoord tc0 = decode_tile(tile, p);
+        const uint8_t *wsrc =
+            p.wimg + static_cast<size_t>(tc0.ntile) * p.kt * KS * KS * n_cc * L.b_stage;
+        for (int ia = 0; ia < n_a && ok; ++ia) {
+          const int kt = ia / n_cc, cc = ia % n_cc;
+          if (!mbar_wait_bounded(&empty_a[sa], pa ^ 1, p.wait_limit_ns, p.status, 1)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full_b[sb], L.b_stage);
-          const size_t stage_idx = static_cast<size_t>(kt * KS * KS + ts) * n_cc + cc;
-          bulk_load(smem_base + L.b_off + sb * L.b_stage, wsrc + stage_idx * L.b_stage,
-                    L.b_stage, &full_b[sb]);
-          if (++sb == L.nb) { sb = 0; pb ^= 1; }
+          mbar_arrive_expect_tx(&full_a[sa], a_bytes);
+          const int tau = tc0.t + kt - (p.kt - 1);
+          const bool from_cache = tau < 0 && p.has_cache;
+          const CUtensorMap *map = from_cache ? &map_cache : &map_x;
+          const int tcoord = from_cache ? tau + (p.kt - 1) : tau;  // negative: zero fill
+          const uint32_t dst = smem_base + L.a_off + sa * L.a_stage;
+#pragma unroll
+          for (int s = 0; s < KC / 8; ++s)
+            tma_load_5d(dst + s * L.slab, map, &full_a[sa], cc * KC + s * 8, tc0.w0 - KS / 2,
+                        tc0.h0 - KS / 2, tcoord, tc0.n);
+          if (++sa == L.na) { sa = 0; pa ^= 1; }
+#pragma unroll 1
+          for (int ts = 0; ts < KS * KS; ++ts) {
+            if (!mbar_wait_bounded(&empty_b[sb], pb ^ 1, p.wait_limit_ns, p.status, 2)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full_b[sb], L.b_stage);
+            const size_t stage_idx = static_cast<size_t>(kt * KS * KS + ts) * n_cc + cc;
+            bulk_load(smem_base + L.b_off + sb * L.b_stage, wsrc + stage_idx * L.b_stage,
+                      L.b_stage, &full_b[sb]);
+            if (++sb == L.nb) { sb = 0; pb ^= 1; }
+          }
         }
       }
     }
@@ -182,53 +205,73 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t adesc0 = smem_desc_noswizzle(smem_base + L.a_off, L.slab, a_sbo);
       const uint64_t bdesc0 = smem_desc_noswizzle(smem_base + L.b_off, b_lbo, 128u);
       const uint32_t slab16 = L.slab >> 4, blbo16 = b_lbo >> 4;
-      uint32_t accumulate = 0;
       int sa = 0, sb = 0;
       uint32_t pa = 0, pb = 0;
-      for (int ia = 0; ia < n_a && ok; ++ia) {
-        if (!mbar_wait_bounded(&full_a[sa], pa, p.wait_limit_ns, p.status, 3)) {
+      int it = 0;
+      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++it) {
+        const int buf = it & 1;
+        // wait until the epilogue has drained this accumulator buffer
+        if (!mbar_wait_bounded(&acc_empty[buf], ((it >> 1) & 1) ^ 1, p.wait_limit_ns, p.status,
+                               6)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t a_st = adesc0 + ((sa * L.a_stage) >> 4);
-#pragma unroll
-        for (int ts = 0; ts < KS * KS; ++ts) {
-          if (!mbar_wait_bounded(&full_b[sb], pb, p.wait_limit_ns, p.status, 4)) {
+        const uint32_t d_tmem = tmem_base + buf * p.nt;
+        uint32_t accumulate = 0;
+        for (int ia = 0; ia < n_a && ok; ++ia) {
+          if (!mbar_wait_bounded(&full_a[sa], pa, p.wait_limit_ns, p.status, 3)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t a_tap = a_st + ((ts / KS) * halo_w + (ts % KS));
-          const uint64_t b_st = bdesc0 + ((sb * L.b_stage) >> 4);
+          const uint64_t a_st = adesc0 + ((sa * L.a_stage) >> 4);
 #pragma unroll
-          for (int j = 0; j < KC / 16; ++j) {
-            umma_bf16(tmem_base, a_tap + 2 * j * slab16, b_st + 2 * j * blbo16, idesc, accumulate);
-            accumulate = 1;
+          for (int ts = 0; ts < KS * KS; ++ts) {
+            if (!mbar_wait_bounded(&full_b[sb], pb, p.wait_limit_ns, p.status, 4)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t a_tap = a_st + ((ts / KS) * halo_w + (ts % KS));
+            const uint64_t b_st = bdesc0 + ((sb * L.b_stage) >> 4);
+#pragma unroll
+            for (int j = 0; j < KC / 16; ++j) {
+              umma_bf16(d_tmem, a_tap + 2 * j * slab16, b_st + 2 * j * blbo16, idesc, accumulate);
+              accumulate = 1;
+            }
+            umma_commit(&empty_b[sb]);  // frees the B stage when these MMAs finish
+            if (++sb == L.nb) { sb = 0; pb ^= 1; }
           }
-          umma_commit(&empty_b[sb]);  // frees the B stage when these MMAs finish
-          if (++sb == L.nb) { sb = 0; pb ^= 1; }
+          umma_commit(&empty_a[sa]);
+          if (++sa == L.na) { sa = 0; pa ^= 1; }
         }
-        umma_commit(&empty_a[sa]);
-        if (++sa == L.na) { sa = 0; pa ^= 1; }
+        umma_commit(&acc_full[buf]);  // accumulator ready for the epilogue
       }
-      umma_commit(acc_full);
     }
   } else {
     // ------------------------------ epilogue ------------------------------------
     const int q = warp % 4;  // tensor-memory lane quarter this warp may read
     const int m = q * 32 + lane;
     const int r = m / kTW, c = m % kTW;
-    const int h = h0 + r, w = w0 + c;
-    const bool valid = (h < p.h) && (w < p.w);
-    uint32_t got = 0;
-    if (lane == 0) got = mbar_wait_bounded(acc_full, 0, p.wait_limit_ns, p.status, 5) ? 1u : 0u;
-    got = __shfl_sync(0xffffffffu, got, 0);
-    if (got) {
+    int it = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+      const int buf = it & 1;
+      const TileCoord tc0 = decode_tile(tile, p);
+      const int h = tc0.h0 + r, w = tc0.w0 + c;
+      const bool valid = (h < p.h) && (w < p.w);
+      uint32_t got = 0;
+      if (lane == 0)
+        got = mbar_wait_bounded(&acc_full[buf], (it >> 1) & 1, p.wait_limit_ns, p.status, 5)
+                  ? 1u
+                  : 0u;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-      const int n0 = ntile * p.nt;
-      const size_t pix = ((static_cast<size_t>(n_img) * p.t + t_out) * p.h + h) * p.w + w;
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * p.nt);
+      const int n0 = tc0.ntile * p.nt;
+      const size_t pix = ((static_cast<size_t>(tc0.n) * p.t + tc0.t) * p.h + h) * p.w + w;
       __nv_bfloat16 *yrow = p.y + pix * p.c_out + n0;
       const __nv_bfloat16 *rrow = p.residual ? p.residual + pix * p.c_out + n0 : nullptr;
       float inv = 1.0f;
@@ -250,6 +293,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         float v[16];
         __syncwarp();
         tmem_ld16(taddr + j, v);
+        if (j + 16 >= p.nt) {
+          // last read of this accumulator: hand the buffer back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] += p.bias[n0 + j + i];
         if (p.epi == 1 && valid) {
@@ -321,27 +370,39 @@ cudaError_t umma_prepare() {
   // Opt in to the largest dynamic shared memory window once per process.
   cudaError_t e = set_smem_attr<64, 3>();
   if (e == cudaSuccess) e = set_smem_attr<32, 3>();
+  if (e == cudaSuccess) e = set_smem_attr<96, 3>();
   if (e == cudaSuccess) e = set_smem_attr<64, 1>();
   if (e == cudaSuccess) e = set_smem_attr<32, 1>();
+  if (e == cudaSuccess) e = set_smem_attr<96, 1>();
   return e;
+}
+
+size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols) {
+  size_t smem = umma_smem_bytes(kc, nt, ks, ks, na, nb);
+  // A CTA that holds more than half of tensor memory must have its SM to
+  // itself; asking for more than half the shared memory guarantees that.
+  if (tmem_cols > 256 && smem < 116 * 1024) smem = 116 * 1024;
+  return smem;
 }
 
 cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_cache,
                              const UmmaArgs &args, int kc, unsigned grid, cudaStream_t stream) {
-  const size_t smem = umma_smem_bytes(kc, args.nt, args.kh, args.kw, args.na, args.nb);
-  if (smem > 227 * 1024 || args.kh != args.kw || (args.kh != 1 && args.kh != 3))
-    return cudaErrorInvalidValue;
-  if (kc == 64 && args.kh == 3)
-    conv_umma_kernel<64, 3><<<grid, kThreads, smem, stream>>>(map_x, map_cache, args);
-  else if (kc == 32 && args.kh == 3)
-    conv_umma_kernel<32, 3><<<grid, kThreads, smem, stream>>>(map_x, map_cache, args);
-  else if (kc == 64 && args.kh == 1)
-    conv_umma_kernel<64, 1><<<grid, kThreads, smem, stream>>>(map_x, map_cache, args);
-  else if (kc == 32 && args.kh == 1)
-    conv_umma_kernel<32, 1><<<grid, kThreads, smem, stream>>>(map_x, map_cache, args);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  if (args.kh != args.kw || (args.kh != 1 && args.kh != 3)) return cudaErrorInvalidValue;
+  const size_t smem = umma_launch_smem(kc, args.nt, args.kh, args.na, args.nb, args.tmem_cols);
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+#define CC3D_LAUNCH(KC_, KS_)                                                              \
+  if (kc == KC_ && args.kh == KS_) {                                                       \
+    conv_umma_kernel<KC_, KS_><<<grid, kThreads, smem, stream>>>(map_x, map_cache, args); \
+    return cudaGetLastError();                                                             \
+  }
+  CC3D_LAUNCH(64, 3)
+  CC3D_LAUNCH(32, 3)
+  CC3D_LAUNCH(96, 3)
+  CC3D_LAUNCH(64, 1)
+  CC3D_LAUNCH(32, 1)
+  CC3D_LAUNCH(96, 1)
+#undef CC3D_LAUNCH
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace cc3d

@@ -31,6 +31,8 @@ struct UmmaArgs {
 
 size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb);
 cudaError_t umma_prepare();
+// Dynamic shared memory a launch requests (with the one-CTA-per-SM rule).
+size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols);
 int umma_tile_w();
 int umma_tile_h();
 cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_cache,
