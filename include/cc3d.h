@@ -70,7 +70,9 @@ typedef enum {
   CC3D_ERR_ALIAS = 4,        /* cache_out overlaps cache_in, x or y */
   CC3D_ERR_OOM = 5,          /* device allocation failed in a create call */
   CC3D_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed */
-  CC3D_ERR_TIMEOUT = 7       /* a device-side bounded wait ran out */
+  CC3D_ERR_TIMEOUT = 7,      /* a device-side bounded wait ran out */
+  CC3D_ERR_TOO_LARGE = 8     /* cc3d_forward_noalloc: weights exceed its
+                                fixed scratch                              */
 } cc3d_status;
 
 typedef enum { CC3D_BF16 = 0, CC3D_FP32 = 1 } cc3d_dtype;
@@ -188,6 +190,35 @@ const char *cc3d_status_string(cc3d_status s);
 /* Number of kernel launches made by this library in this process (all
  * entry points).  Lets callers count device work. */
 uint64_t cc3d_launch_count(void);
+
+/* cc3d_forward without a plan and without any device allocation.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot call cudaMalloc: code that must hand all device memory out of
+ * its own fixed pool (a serving process that reserves its budget up front,
+ * a framework whose allocator owns the device), and latency-critical loops
+ * where an allocation's implicit synchronisation is not acceptable.
+ *
+ * It computes exactly what cc3d_plan_create(desc) + cc3d_forward(...) would
+ * (same kernel, same tiles), for bf16 descriptors that the tensor-core path
+ * covers.  desc->weight / bias / gamma / beta are read on every call (bias
+ * and gamma/beta directly, the weights after re-tiling); desc->max_t bounds
+ * t as usual.  The re-tiled weights live in one fixed, file-scope device
+ * array of 8 MiB + 16 KiB that every GPU which loads the library holds until
+ * the process exits.  A descriptor whose weights need more than 8 MiB
+ * (c_out * c_in * kt * kh * kw * 2 bytes; 384 x 384 x 3 x 3 x 3 fits)
+ * returns CC3D_ERR_TOO_LARGE before anything is launched.
+ *
+ * All calls on a device share that array and it keeps the last call's
+ * contents; calls that overlap on the GPU (different streams, no ordering
+ * between them) race on it and give wrong results.  Serialise them.
+ * The first call on a device looks the array's device address up (and
+ * prepares the kernels); make that first call before any stream capture.
+ * Arguments and errors are those of cc3d_forward. */
+cc3d_status cc3d_forward_noalloc(const cc3d_desc *desc, const void *x, int t,
+                                 const void *cache_in, void *y, void *cache_out,
+                                 const void *residual, const void *next_cache_in,
+                                 void *next_cache_out, void *stream);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,88 @@
+"""cc3d_forward_noalloc: the conv entry point for callers that cannot call
+cudaMalloc (their device memory comes from a fixed pool they manage, or an
+allocation's implicit synchronisation is not acceptable where they call).
+Its output must match the planned entry point (cc3d_plan_create +
+cc3d_forward) on the same inputs, call after call, although all its calls
+share one fixed scratch array inside the library.
+
+This file is named so that pytest collects it last."""
+import ctypes
+
+import pytest
+import torch
+
+from tests.parity import assert_close_bf16, ncthw_np, to_dev
+from video_vae_causal_implicit_b200 import cc3d, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _desc_for(plan_kwargs, weight, bias, gamma=None):
+    """Same descriptor a Plan builds, pointing at the caller's tensors."""
+    co, ci, kt, kh, kw = (int(s) for s in weight.shape)
+    d = cc3d.Desc()
+    d.n, d.c_in, d.c_out = 1, ci, co
+    d.h, d.w, d.max_t = plan_kwargs["h"], plan_kwargs["w"], plan_kwargs["max_t"]
+    d.kt, d.kh, d.kw, d.pad_h, d.pad_w = kt, kh, kw, kh // 2, kw // 2
+    d.stride_t = d.stride_h = d.stride_w = d.dil_t = d.dil_h = d.dil_w = d.groups = 1
+    d.dtype = cc3d.BF16
+    d.weight = weight.data_ptr()
+    d.bias = bias.data_ptr() if bias is not None else None
+    d.epi = plan_kwargs.get("epi", cc3d.EPI_BIAS)
+    d.gamma = gamma.data_ptr() if gamma is not None else None
+    d.beta = None
+    return d
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def test_noalloc_matches_planned_conv_on_two_calls_in_a_row():
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    # call 1: 384 -> 384 with a bias and a cache; call 2: different weights,
+    # no bias (the scratch's zero bias must be cleared), 96 -> 192.
+    cases = [
+        dict(cin=384, cout=384, t=2, h=30, w=52, bias=True, cache=True, seed=1),
+        dict(cin=96, cout=192, t=3, h=21, w=17, bias=False, cache=False, seed=2),
+    ]
+    outs = []
+    for cs in cases:
+        case = synth.conv_case(cs["cin"], cs["cout"], cs["t"], cs["h"], cs["w"],
+                               seed_base=cs["seed"])
+        x = to_dev(synth.ndhwc(case["x"]))
+        w = to_dev(case["w"])
+        b = to_dev(case["b"]) if cs["bias"] else None
+        cache = (to_dev(synth.ndhwc(synth.normal((1, cs["cin"], 2, cs["h"], cs["w"]), 40)))
+                 if cs["cache"] else None)
+        kw = dict(h=cs["h"], w=cs["w"], max_t=cs["t"])
+        plan = cc3d.Plan(w, b, **kw)
+        y_ref = torch.empty((1, cs["t"], cs["h"], cs["w"], cs["cout"]), dtype=torch.bfloat16,
+                            device="cuda")
+        plan.forward(x, y_ref, cache_in=cache)
+        y = torch.full_like(y_ref, float("nan"))
+        cache_out = torch.empty((1, 2, cs["h"], cs["w"], cs["cin"]), dtype=torch.bfloat16,
+                                device="cuda")
+        d = _desc_for(kw, w, b)
+        st = cc3d.cc3d_forward_noalloc(d, _p(x), cs["t"], _p(cache), _p(y), _p(cache_out), None,
+                                       None, None, stream)
+        assert st == cc3d.OK, cc3d.cc3d_status_string(st)
+        cc3d.sync_status()
+        assert_close_bf16(ncthw_np(y), ncthw_np(y_ref), f"noalloc call {cs}")
+        assert torch.equal(y.cpu(), y_ref.cpu())  # same kernel and tiles: same bytes
+        assert torch.equal(cache_out[:, -2:].cpu(), x[:, -2:].cpu())
+        outs.append(y)
+        plan.close()
+    torch.cuda.synchronize()
+
+
+def test_noalloc_refuses_weights_beyond_its_scratch():
+    big = torch.empty((512, 512, 3, 3, 3), dtype=torch.bfloat16, device="cuda")  # 14 MB
+    d = _desc_for(dict(h=8, w=8, max_t=1), big, None)
+    x = torch.zeros((1, 1, 8, 8, 512), dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros((1, 1, 8, 8, 512), dtype=torch.bfloat16, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    launches = cc3d.cc3d_launch_count()
+    st = cc3d.cc3d_forward_noalloc(d, _p(x), 1, None, _p(y), None, None, None, None, stream)
+    assert st == cc3d.ERR_TOO_LARGE
+    assert cc3d.cc3d_launch_count() == launches

@@ -16,15 +16,15 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libcc3d.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_ALIAS, ERR_OOM, ERR_CUDA, ERR_TIMEOUT = \
-    range(8)
+(OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_ALIAS, ERR_OOM, ERR_CUDA, ERR_TIMEOUT,
+ ERR_TOO_LARGE) = range(9)
 BF16, FP32 = 0, 1
 EPI_BIAS, EPI_BIAS_RESIDUAL, EPI_BIAS_RMS_SILU = 0, 1, 2
 VARIANT_NONE, VARIANT_UMMA, VARIANT_THIN, VARIANT_FP32 = 0, 1, 2, 3
 
 _STATUS_NAMES = {0: "CC3D_OK", 1: "CC3D_ERR_INVALID_ARG", 2: "CC3D_ERR_UNSUPPORTED",
                  3: "CC3D_ERR_ALIGNMENT", 4: "CC3D_ERR_ALIAS", 5: "CC3D_ERR_OOM",
-                 6: "CC3D_ERR_CUDA", 7: "CC3D_ERR_TIMEOUT"}
+                 6: "CC3D_ERR_CUDA", 7: "CC3D_ERR_TIMEOUT", 8: "CC3D_ERR_TOO_LARGE"}
 
 
 class Cc3dError(RuntimeError):
@@ -63,6 +63,8 @@ SIGNATURES = {
     "cc3d_get_stats": (_I, [_VP, ctypes.POINTER(Stats)]),
     "cc3d_status_string": (ctypes.c_char_p, [_I]),
     "cc3d_launch_count": (ctypes.c_uint64, []),
+    "cc3d_forward_noalloc": (_I, [ctypes.POINTER(Desc), _VP, _I, _VP, _VP, _VP, _VP, _VP, _VP,
+                                  _VP]),
 }
 
 _lib = None
@@ -135,6 +137,14 @@ def cc3d_status_string(status):
 
 def cc3d_launch_count():
     return int(lib().cc3d_launch_count())
+
+
+def cc3d_forward_noalloc(desc, x, t, cache_in, y, cache_out, residual, next_cache_in,
+                         next_cache_out, stream):
+    """The conv without a plan and without device allocation (scratch is a
+    fixed array inside the library; see include/cc3d.h)."""
+    return lib().cc3d_forward_noalloc(ctypes.byref(desc), x, t, cache_in, y, cache_out, residual,
+                                      next_cache_in, next_cache_out, stream)
 
 
 # ---- torch conveniences (pointers + current stream only) --------------------------

@@ -107,6 +107,13 @@ bool encode_act_map(CUtensorMap *m, const void *base, int c, int w, int h, int t
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+int *device_status_word() { return status_ptr(); }
+
+bool encode_activation_map(CUtensorMap *m, const void *base, int c, int w, int h, int t, int n,
+                           int box_w, int box_h) {
+  return encode_act_map(m, base, c, w, h, t, n, box_w, box_h);
+}
+
 }  // namespace cc3d
 
 using namespace cc3d;
@@ -207,6 +214,7 @@ const char *cc3d_status_string(cc3d_status s) {
     case CC3D_ERR_OOM: return "device allocation failed";
     case CC3D_ERR_CUDA: return "CUDA error";
     case CC3D_ERR_TIMEOUT: return "device wait timed out";
+    case CC3D_ERR_TOO_LARGE: return "problem exceeds the fixed no-allocation scratch";
   }
   return "unknown status";
 }

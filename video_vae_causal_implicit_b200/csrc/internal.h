@@ -82,4 +82,10 @@ cudaError_t launch_rmsnorm_silu(const __nv_bfloat16 *x, const float *gamma, cons
 // Host-side launch counter (all kernels of this library).
 void count_launch();
 
+// Device address of the status word on the current device (null on error).
+int *device_status_word();
+// 5-D bf16 activation tensor map (dims C, W, H, T, N; 8-channel boxes).
+bool encode_activation_map(CUtensorMap *m, const void *base, int c, int w, int h, int t, int n,
+                           int box_w, int box_h);
+
 }  // namespace cc3d
