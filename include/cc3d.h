@@ -125,8 +125,11 @@ typedef struct cc3d_block cc3d_block;
 /* Validate desc, pick a kernel, copy and re-tile the weights (and bias,
  * gamma, beta) into plan-owned device memory.  Synchronous.  Returns
  * CC3D_ERR_UNSUPPORTED for stride/dilation/groups != 1, even kernel sizes,
- * or channel counts no kernel covers (bf16: c_in == 3, or c_in % 32 == 0;
- * c_out % 16 == 0; fp32: any).  *out is set only on CC3D_OK. */
+ * or channel counts no kernel covers.  bf16 covers c_out % 16 == 0 with
+ * either c_in % 32 == 0 (kh == kw in {1, 3}, kt <= 3; N tiles of at most
+ * 256 channels) or c_in <= 8 (the thin first-layer path: bias epilogue,
+ * c_out <= 256, kt*kh*kw*c_in <= 256); fp32 covers any channel count with
+ * the bias epilogue.  *out is set only on CC3D_OK. */
 cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out);
 cc3d_status cc3d_plan_destroy(cc3d_plan *plan);
 

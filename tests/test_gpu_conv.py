@@ -210,3 +210,55 @@ def test_sampled_points_config3b_shape():
                                       None, pts)
     got = gather_points(y.cpu(), pts)
     assert_close_bf16(got, ref, "config 3b sampled")
+
+
+# ---- thin first layer (C_in <= 8) --------------------------------------------------
+
+@pytest.mark.parametrize("cin,cout,t,h,w", [(3, 96, 3, 20, 13), (3, 32, 2, 17, 9), (1, 16, 2, 9, 8),
+                                            (8, 64, 2, 16, 11)])
+def test_thin_conv_matches_oracle(cin, cout, t, h, w):
+    case = synth.conv_case(cin, cout, t, h, w, seed_base=30 + cin, x_dist="uniform")
+    plan, x, y = run_conv(case)
+    assert plan.stats().variant == cc3d.VARIANT_THIN
+    ref = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], _bias64(case["b"]))
+    assert_close_bf16(ncthw_np(y), ref, f"thin conv {cin}->{cout}")
+
+
+def test_thin_conv_with_cache_and_streaming_bitwise():
+    cin, cout, t, h, w = 3, 96, 4, 19, 10
+    case = synth.conv_case(cin, cout, t, h, w, seed_base=44, x_dist="uniform")
+    plan, x, y = run_conv(case)
+    ys = _stream_chunks(plan, x, 1, cin)
+    assert torch.equal(ys.cpu(), y.cpu())
+    cache = to_dev(synth.ndhwc(synth.uniform((1, cin, 2, h, w), -1, 1, 45, torch.bfloat16)))
+    y2 = torch.empty_like(y)
+    plan.forward(x, y2, cache_in=cache)
+    cc3d.sync_status()
+    ref = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], _bias64(case["b"]),
+                               cache=synth.ncthw_view(cache.cpu()))
+    assert_close_bf16(ncthw_np(y2), ref, "thin conv with cache")
+
+
+def test_config3_encoder_chain_sampled():
+    """Video x[1,3,17,480,832] ~ U(-1,1) -> causal conv 3 -> 96 -> causal conv
+    96 -> 96, full size.  Each layer is checked on sampled voxels with the
+    oracle fed the same inputs that layer saw (layer 2 gets the GPU's bf16
+    output of layer 1)."""
+    t, h, w = 17, 480, 832
+    c1 = synth.conv_case(3, 96, t, h, w, x_dist="uniform")
+    plan1, x, y1 = run_conv(c1)
+    assert plan1.stats().variant == cc3d.VARIANT_THIN
+    w2 = synth.kaiming_uniform(96, 96, (3, 3, 3), 11)
+    b2 = synth.uniform((96,), -0.1, 0.1, 12)
+    plan2 = cc3d.Plan(to_dev(w2), to_dev(b2), h=h, w=w, max_t=t)
+    y2 = torch.empty_like(y1)
+    plan2.forward(y1, y2)
+    cc3d.sync_status()
+    pts = torch.cat([synth.sample_points(1, t, h, w, 3000, 77),
+                     synth.sample_points(1, t, h, w, 0, 0, frames=[0, t - 1])[::2011]])
+    x_cpu, y1_cpu, y2_cpu = x.cpu(), y1.cpu(), y2.cpu()
+    ref1 = oracle.causal_conv3d_points(synth.ncthw_view(x_cpu), c1["w"], _bias64(c1["b"]), None,
+                                       pts)
+    assert_close_bf16(gather_points(y1_cpu, pts), ref1, "config 3a sampled")
+    ref2 = oracle.causal_conv3d_points(synth.ncthw_view(y1_cpu), w2, _bias64(b2), None, pts)
+    assert_close_bf16(gather_points(y2_cpu, pts), ref2, "config 3b (chained) sampled")

@@ -103,6 +103,23 @@ bool encode_act_map(CUtensorMap *m, const void *base, int c, int w, int h, int t
   return r == CUDA_SUCCESS;
 }
 
+// 4-D bf16 tensor map over an NDHWC buffer with few channels: dims
+// (W*C, H, T, N), a box of `row` elements x `box_h` rows x 1 x 1.
+bool encode_thin_map(CUtensorMap *m, const void *base, int c, int w, int h, int t, int n,
+                     int row, int box_h) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t wc = static_cast<cuuint64_t>(w) * c;
+  cuuint64_t dims[4] = {wc, (cuuint64_t)h, (cuuint64_t)t, (cuuint64_t)n};
+  cuuint64_t strides[3] = {wc * 2, wc * 2 * h, wc * 2 * h * t};
+  cuuint32_t box[4] = {(cuuint32_t)row, (cuuint32_t)box_h, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
@@ -191,6 +208,13 @@ cc3d_status check_desc(const cc3d_desc *d, int *variant) {
   }
   if (d->dtype != CC3D_BF16) return CC3D_ERR_INVALID_ARG;
   if (d->c_out % 16 != 0) return CC3D_ERR_UNSUPPORTED;
+  if (d->c_in <= 8) {
+    // thin path: whole K gathered per pixel, one N tile, bias epilogue
+    if (d->epi != CC3D_EPI_BIAS || d->c_out > 256) return CC3D_ERR_UNSUPPORTED;
+    if (d->kt * d->kh * d->kw * d->c_in > 256) return CC3D_ERR_UNSUPPORTED;
+    *variant = CC3D_VARIANT_THIN;
+    return CC3D_OK;
+  }
   if (d->c_in % 32 == 0) {
     if (d->kh != d->kw) return CC3D_ERR_UNSUPPORTED;
     if (d->epi == CC3D_EPI_BIAS_RMS_SILU && d->c_out > 256) return CC3D_ERR_UNSUPPORTED;
@@ -240,7 +264,40 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
   if ((s = copy_vec(&p->bias, desc->bias, desc->c_out, true)) != CC3D_OK) goto fail;
   if ((s = copy_vec(&p->gamma, desc->gamma, desc->c_out, false)) != CC3D_OK) goto fail;
   if ((s = copy_vec(&p->beta, desc->beta, desc->c_out, false)) != CC3D_OK) goto fail;
-  if (variant == CC3D_VARIANT_FP32) {
+  if (variant == CC3D_VARIANT_THIN) {
+    if (!status_ptr()) { s = CC3D_ERR_CUDA; goto fail; }
+    if (cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, p->device) !=
+        cudaSuccess)
+      p->sm_count = 148;
+    p->kpad = (taps * desc->c_in + 15) / 16 * 16;
+    p->nt = desc->c_out;
+    p->n_ntiles = 1;
+    int cols = 32;
+    while (cols < 2 * desc->c_out) cols *= 2;
+    p->tmem_cols = cols;
+    {
+      ThinArgs probe;
+      std::memset(&probe, 0, sizeof probe);
+      probe.kpad = p->kpad; probe.c_out = desc->c_out; probe.kt = desc->kt;
+      probe.kh = desc->kh; probe.kw = desc->kw; probe.c_in = desc->c_in;
+      probe.pad_w = desc->pad_w; probe.use_tma = 1; probe.spec_rgb333 = 0;
+      int per_sm = static_cast<int>((228 * 1024) / (thin_smem_bytes(probe) + 1024));
+      if (per_sm > 512 / cols) per_sm = 512 / cols;
+      if (per_sm > 2) per_sm = 2;
+      p->ctas_per_sm = per_sm < 1 ? 1 : per_sm;
+    }
+    p->st.tile_h = umma_tile_h();
+    p->st.tile_w = umma_tile_w();
+    p->st.n_tile = p->nt;
+    p->st.k_chunk = p->kpad;
+    const size_t bytes = sizeof(__nv_bfloat16) * p->kpad * desc->c_out;
+    if (cudaMalloc(&p->wraw, bytes) != cudaSuccess) { s = CC3D_ERR_OOM; goto fail; }
+    e = launch_repack_thin(static_cast<const __nv_bfloat16 *>(desc->weight),
+                           static_cast<uint8_t *>(p->wraw), desc->c_out, desc->c_in, taps,
+                           p->kpad, 0);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
+  } else if (variant == CC3D_VARIANT_FP32) {
     const size_t bytes = sizeof(float) * desc->c_out * desc->c_in * taps;
     if (cudaMalloc(&p->wraw, bytes) != cudaSuccess) { s = CC3D_ERR_OOM; goto fail; }
     e = cudaMemcpy(p->wraw, desc->weight, bytes, cudaMemcpyDeviceToDevice);
@@ -337,7 +394,14 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
     return reject(CC3D_ERR_INVALID_ARG);
   if (d.epi != CC3D_EPI_BIAS_RMS_SILU && (next_cache_in || next_cache_out))
     return reject(CC3D_ERR_INVALID_ARG);
-  if (!aligned16(x) || !aligned16(y) || !aligned16(cache_in) || !aligned16(cache_out) ||
+  // The thin path reads x and the caches with 2-byte loads (or TMA when they
+  // happen to be 16-byte aligned), so a chunk of a 3-channel video may start
+  // anywhere on a bf16 boundary; everything else needs 16 bytes.
+  const bool thin = p->variant == CC3D_VARIANT_THIN;
+  auto in_ok = [&](const void *q) {
+    return thin ? (reinterpret_cast<uintptr_t>(q) & 1u) == 0 : aligned16(q);
+  };
+  if (!in_ok(x) || !aligned16(y) || !in_ok(cache_in) || !in_ok(cache_out) ||
       !aligned16(residual) || !aligned16(next_cache_in) || !aligned16(next_cache_out))
     return reject(CC3D_ERR_ALIGNMENT);
   const size_t esz = d.dtype == CC3D_FP32 ? 4 : 2;
@@ -372,6 +436,49 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
     a.kt = d.kt; a.kh = d.kh; a.kw = d.kw; a.pad_h = d.pad_h; a.pad_w = d.pad_w;
     e = launch_conv_fp32(a, stream);
     tiles = 1;
+  } else if (p->variant == CC3D_VARIANT_THIN) {
+    ThinArgs a;
+    a.x = static_cast<const uint16_t *>(x);
+    a.cache = static_cast<const uint16_t *>(cache_in);
+    a.wimg = static_cast<const uint8_t *>(p->wraw);
+    a.bias = p->bias;
+    a.y = static_cast<__nv_bfloat16 *>(y);
+    a.status = status;
+    a.wait_limit_ns = wait_limit_ns();
+    a.n = d.n; a.t = t; a.h = d.h; a.w = d.w; a.c_in = d.c_in; a.c_out = d.c_out;
+    a.kt = d.kt; a.kh = d.kh; a.kw = d.kw; a.pad_h = d.pad_h; a.pad_w = d.pad_w;
+    a.kpad = p->kpad;
+    a.tiles_w = (d.w + umma_tile_w() - 1) / umma_tile_w();
+    a.tiles_h = (d.h + umma_tile_h() - 1) / umma_tile_h();
+    a.n_tiles = d.n * t * a.tiles_h * a.tiles_w;
+    a.tmem_cols = p->tmem_cols;
+    // TMA halo when both inputs can be described by a tensor map
+    a.use_tma = (static_cast<long long>(d.w) * d.c_in % 8 == 0 && aligned16(x) &&
+                 (!cache_in || aligned16(cache_in)))
+                    ? 1
+                    : 0;
+    CUtensorMap mx, mc;
+    std::memset(&mx, 0, sizeof mx);
+    std::memset(&mc, 0, sizeof mc);
+    if (a.use_tma) {
+      const int row = thin_tma_row(a), box_h = umma_tile_h() + d.kh - 1;
+      if (row > 256 || !encode_thin_map(&mx, x, d.c_in, d.w, d.h, t, d.n, row, box_h))
+        a.use_tma = 0;
+      else if (cache_in && front > 0 &&
+               !encode_thin_map(&mc, cache_in, d.c_in, d.w, d.h, front, d.n, row, box_h))
+        a.use_tma = 0;
+      else if (!(cache_in && front > 0))
+        mc = mx;
+    }
+    // the specialised im2col assumes the TMA halo geometry of RGB 3x3x3:
+    // rows of 40 elements, frames 768 elements apart
+    a.spec_rgb333 = (a.use_tma && d.c_in == 3 && d.kt == 3 && d.kh == 3 && d.kw == 3 &&
+                     thin_tma_row(a) == 40 && p->kpad == 96)
+                        ? 1
+                        : 0;
+    tiles = static_cast<uint64_t>(a.n_tiles);
+    const uint64_t slots = static_cast<uint64_t>(p->sm_count) * p->ctas_per_sm;
+    e = launch_conv_thin(mx, mc, a, static_cast<unsigned>(tiles < slots ? tiles : slots), stream);
   } else {
     CUtensorMap mx, mc;
     const int box_w = umma_tile_w() + d.kw - 1, box_h = umma_tile_h() + d.kh - 1;

@@ -1,0 +1,473 @@
+// conv_thin.cu -- causal Conv3D for inputs with very few channels (the
+// encoder's first layer, RGB video: C_in = 3), on tcgen05 tensor cores.
+//
+// Operation: the same causal conv as conv_umma.cu ("Cosmos3 Wan VAE --
+// engine size vs context memory", §10.3), but with C_in so small that one
+// pixel is 6 bytes: TMA boxes cannot start on such pixels and one tap holds
+// only C_in useful K values.  The whole K = kt * kh * kw * C_in (81 for a
+// 3x3x3 kernel on RGB) is instead gathered per output pixel ("im2col" in
+// shared memory), zero-padded to a multiple of 16, and multiplied in
+// K / 16 MMAs.  The layer moves ~40 MB in and writes C_out values per input
+// pixel (1.3 GB at 17 x 480 x 832 x 96), so it is bound by the HBM write of
+// y; the design keeps every other step off that critical path.
+//
+// Persistent CTAs (one or two per SM), 320 threads:
+//   warp  5    halo loader: one TMA box per frame brings the tile's input
+//              halo (kt frames x (16 + kh - 1) rows x a 16-byte aligned
+//              run of (8 + kw - 1) * C_in elements) into a double-buffered
+//              shared buffer -- from the cache when the frame precedes the
+//              chunk; out-of-image and absent-cache reads are TMA zero fill;
+//   warps 0-3  builders: write the 128 x K_pad A tile from the halo as
+//              K-major core matrices (A double buffered).  When the input
+//              cannot be described by a tensor map (unaligned chunk start,
+//              W * C_in not a multiple of 8) they stage the halo themselves
+//              with plain loads;
+//   warp  4    tensor memory owner and MMA issuer (one thread);
+//   warps 6-9  epilogue: tensor memory -> +bias -> bf16 -> global.
+// The weights ([K_pad/8][C_out][8] core matrices) stay in shared memory for
+// the life of the CTA; two accumulators in tensor memory let the epilogue
+// of one tile overlap the build and MMAs of the next.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace cc3d {
+namespace {
+
+constexpr int kTW = 8, kTH = 16, kM = kTW * kTH;
+constexpr int kBuilders = 128;  // warps 0-3
+constexpr int kMmaWarp = 4;
+constexpr int kLoadWarp = 5;    // halo TMA producer
+constexpr int kThreads = 320;   // + epilogue warps 6-9
+constexpr int kNH = 4;          // halo ring depth (loader runs ahead)
+
+// Halo geometry of one tile.  Frames are [kt] slabs of `kt_stride`
+// elements; a slab holds (16 + kh - 1) rows of `row` elements; the pixel
+// (w0 - pad_w) starts at element `rem` of each row.
+struct HaloGeom {
+  int row, rem, kt_stride;
+};
+
+__host__ __device__ inline uint32_t rup(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+
+__host__ __device__ inline HaloGeom halo_geom(const ThinArgs &a) {
+  HaloGeom g;
+  const int hh = kTH + a.kh - 1, hw = kTW + a.kw - 1;
+  if (a.use_tma) {
+    // rows start on a 16-byte boundary: round the first element down to a
+    // multiple of 8 (w0 is a multiple of 8, so the remainder is constant)
+    g.rem = ((-a.pad_w * a.c_in) % 8 + 8) % 8;
+    g.row = static_cast<int>(rup(g.rem + hw * a.c_in, 8));
+    g.kt_stride = static_cast<int>(rup(g.row * hh * 2, 128) / 2);
+  } else {
+    g.rem = 0;
+    g.row = hw * a.c_in;
+    g.kt_stride = g.row * hh;
+  }
+  return g;
+}
+
+struct ThinLayout {
+  uint32_t b_off, a_off, a_bytes, halo_off, halo_bytes, koff_off, bias_off, bar_off, total;
+};
+
+__host__ __device__ inline ThinLayout thin_layout(const ThinArgs &a) {
+  ThinLayout L;
+  const HaloGeom g = halo_geom(a);
+  L.b_off = 0;
+  const uint32_t b_bytes = static_cast<uint32_t>(a.kpad) * a.c_out * 2u;
+  L.a_off = rup(b_bytes, 1024u);
+  L.a_bytes = rup(static_cast<uint32_t>(a.kpad) * kM * 2u, 1024u);
+  L.halo_off = L.a_off + 2 * L.a_bytes;
+  L.halo_bytes = rup(static_cast<uint32_t>(a.kt) * g.kt_stride * 2u, 128u);  // per buffer
+  L.koff_off = L.halo_off + kNH * L.halo_bytes;  // int32 halo offset per K index
+  L.bias_off = L.koff_off + 4u * a.kpad;           // fp32 bias copy
+  L.bar_off = rup(L.bias_off + 4u * a.c_out, 64u);
+  // b_full, a_full[2], a_empty[2], acc_full[2], acc_empty[2],
+  // halo_full[kNH], halo_empty[kNH], tmem slot + flag
+  L.total = L.bar_off + 8u * (9 + 2 * kNH) + 16u;
+  return L;
+}
+
+struct Tile {
+  int n, t, h0, w0;
+};
+
+__device__ __forceinline__ Tile thin_tile(int tile, const ThinArgs &p) {
+  Tile c;
+  const int tw = tile % p.tiles_w;
+  int r = tile / p.tiles_w;
+  const int th = r % p.tiles_h;
+  r /= p.tiles_h;
+  c.t = r % p.t;
+  c.n = r / p.t;
+  c.w0 = tw * kTW;
+  c.h0 = th * kTH;
+  return c;
+}
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, uint64_t *bar,
+                                            int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Row of A for C_in = 3 and a 3x3x3 kernel read from the TMA halo
+// (rows of 40 elements, frames 768 elements apart): K index
+// k = ((kt * 3 + ih) * 3 + iw) * 3 + ci sits at halo offset
+// kt * 768 + ih * 40 + iw * 3 + ci, all compile-time; K 81..95 is zero.
+__device__ __forceinline__ void build_row_rgb333(const uint16_t *hbits, uint8_t *a_row) {
+#pragma unroll
+  for (int k8 = 0; k8 < 12; ++k8) {
+    uint32_t packed[4];
+#pragma unroll
+    for (int e2 = 0; e2 < 4; ++e2) {
+      uint32_t v2[2];
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        const int k = k8 * 8 + e2 * 2 + s;
+        const int ci = k % 3, iw = (k / 3) % 3, ih = (k / 9) % 3, kt = k / 27;
+        v2[s] = k < 81 ? static_cast<uint32_t>(hbits[kt * 768 + ih * 40 + iw * 3 + ci]) : 0u;
+      }
+      packed[e2] = v2[0] | (v2[1] << 16);
+    }
+    *reinterpret_cast<uint4 *>(a_row + k8 * (kM * 16)) =
+        make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    conv_thin_kernel(const __grid_constant__ CUtensorMap map_x,
+                     const __grid_constant__ CUtensorMap map_cache, ThinArgs p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const ThinLayout L = thin_layout(p);
+  const HaloGeom G = halo_geom(p);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
+  uint64_t *b_full = bars;
+  uint64_t *a_full = bars + 1;       // [2]
+  uint64_t *a_empty = bars + 3;      // [2]
+  uint64_t *acc_full = bars + 5;     // [2]
+  uint64_t *acc_empty = bars + 7;    // [2]
+  uint64_t *halo_full = bars + 9;          // [kNH]
+  uint64_t *halo_empty = bars + 9 + kNH;   // [kNH]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9 + 2 * kNH);
+  float *sbias = reinterpret_cast<float *>(smem + L.bias_off);
+  volatile uint32_t *go_flag = tmem_slot + 1;
+  int *koff = reinterpret_cast<int *>(smem + L.koff_off);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n_tiles = p.n * p.t * p.tiles_h * p.tiles_w;
+  const int hh = kTH + p.kh - 1, hw = kTW + p.kw - 1;
+  const int K = p.kt * p.kh * p.kw * p.c_in;
+  const uint32_t smem_base = smem_u32(smem);
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&a_full[i], kBuilders);
+      mbar_init(&a_empty[i], 1);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    for (int i = 0; i < kNH; ++i) {
+      mbar_init(&halo_full[i], 1);
+      mbar_init(&halo_empty[i], 1);
+    }
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < p.c_out; i += kThreads) sbias[i] = p.bias[i];
+  // halo offset of each K index k = ((kt * kh + ih) * kw + iw) * c_in + ci,
+  // relative to the output pixel's own halo position; -1 pads K to kpad
+  for (int k = threadIdx.x; k < p.kpad; k += kThreads) {
+    int off = -1;
+    if (k < K) {
+      int q = k;
+      const int ci = q % p.c_in;
+      q /= p.c_in;
+      const int iw = q % p.kw;
+      q /= p.kw;
+      const int ih = q % p.kh;
+      const int kt = q / p.kh;
+      off = kt * G.kt_stride + ih * G.row + iw * p.c_in + ci;
+    }
+    koff[k] = off;
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  bool ok = true;
+
+  if (warp < 4) {
+    // ------------------------------ builders -----------------------------------
+    const int m = threadIdx.x;  // A row built by this thread
+    const int r = m / kTW, c = m % kTW;
+    if (threadIdx.x == 0) {
+      // weights: one bulk copy for the life of the CTA
+      const uint32_t wbytes = static_cast<uint32_t>(p.kpad) * p.c_out * 2u;
+      mbar_arrive_expect_tx(b_full, wbytes);
+      bulk_load(smem_base + L.b_off, p.wimg, wbytes, b_full);
+    }
+    int it = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+      const int buf = it & 1;
+      const int hb = p.use_tma ? it % kNH : 0;
+      const uint32_t hph = static_cast<uint32_t>((it / kNH) & 1);
+      uint16_t *halo = reinterpret_cast<uint16_t *>(smem + L.halo_off + hb * L.halo_bytes);
+      if (!p.use_tma) {
+        // stage the halo with plain loads: issue a batch of loads, then store
+        const Tile tc = thin_tile(tile, p);
+        const int helems = p.kt * hh * hw * p.c_in;
+        for (int i0 = 0; i0 < helems; i0 += 8 * kBuilders) {
+          uint16_t v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kBuilders + threadIdx.x;
+            v[u] = 0;
+            if (i < helems) {
+              int q = i;
+              const int ci = q % p.c_in;
+              q /= p.c_in;
+              const int cc = q % hw;
+              q /= hw;
+              const int rr = q % hh;
+              const int kt = q / hh;
+              const int tau = tc.t + kt - (p.kt - 1);
+              const int h = tc.h0 - p.pad_h + rr, w = tc.w0 - p.pad_w + cc;
+              if (h >= 0 && h < p.h && w >= 0 && w < p.w) {
+                const size_t pix = (static_cast<size_t>(h) * p.w + w) * p.c_in + ci;
+                const uint16_t *src = nullptr;
+                if (tau >= 0)
+                  src = p.x + ((static_cast<size_t>(tc.n) * p.t + tau) * p.h * p.w) * p.c_in;
+                else if (p.cache)
+                  src = p.cache + ((static_cast<size_t>(tc.n) * (p.kt - 1) + tau + (p.kt - 1)) *
+                                   p.h * p.w) * p.c_in;
+                if (src) v[u] = src[pix];
+              }
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kBuilders + threadIdx.x;
+            if (i < helems) halo[i] = v[u];  // row = hw * c_in, kt_stride = row * hh
+          }
+        }
+      }
+      // thread 0 waits for: this A buffer free (MMAs of two tiles ago done)
+      // and, with TMA, this tile's halo landed
+      if (threadIdx.x == 0) {
+        bool g = mbar_wait_bounded(&a_empty[buf], ((it >> 1) & 1) ^ 1, p.wait_limit_ns, p.status,
+                                   11);
+        if (g && p.use_tma)
+          g = mbar_wait_bounded(&halo_full[hb], hph, p.wait_limit_ns, p.status, 16);
+        *go_flag = g ? 1u : 0u;
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kBuilders) : "memory");
+      if (!*go_flag) {  // every builder reads the same flag: all leave together
+        ok = false;
+        break;
+      }
+      uint8_t *a_row = smem + L.a_off + buf * L.a_bytes + (m / 8) * 128 + (m % 8) * 16;
+      const uint16_t *hbits = halo + r * G.row + G.rem + c * p.c_in;
+      if (p.spec_rgb333) {
+        build_row_rgb333(hbits, a_row);
+      } else {
+        // build row m of A (zero where koff is -1)
+        for (int k8 = 0; k8 < p.kpad / 8; ++k8) {
+          uint32_t packed[4];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const int o0 = koff[k8 * 8 + e2 * 2], o1 = koff[k8 * 8 + e2 * 2 + 1];
+            const uint32_t lo = o0 >= 0 ? hbits[o0] : 0u;
+            const uint32_t hi = o1 >= 0 ? hbits[o1] : 0u;
+            packed[e2] = lo | (hi << 16);
+          }
+          *reinterpret_cast<uint4 *>(a_row + k8 * (kM * 16)) =
+              make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        }
+      }
+      // make the generic-proxy writes visible to the tensor core, then signal
+      fence_proxy_async_smem();
+      mbar_arrive(&a_full[buf]);
+      asm volatile("bar.sync 1, %0;" ::"n"(kBuilders) : "memory");  // halo fully read
+      if (p.use_tma && threadIdx.x == 0) mbar_arrive(&halo_empty[hb]);
+    }
+  } else if (warp == kLoadWarp) {
+    // ------------------------------ halo loader (TMA) ----------------------------
+    if (p.use_tma && lane == 0) {
+      const uint32_t box_bytes = static_cast<uint32_t>(G.row) * hh * 2u;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+        const int hb = it % kNH;
+        if (!mbar_wait_bounded(&halo_empty[hb], ((it / kNH) & 1) ^ 1, p.wait_limit_ns, p.status,
+                               17)) {
+          ok = false;
+          break;
+        }
+        const Tile tc = thin_tile(tile, p);
+        mbar_arrive_expect_tx(&halo_full[hb], box_bytes * p.kt);
+        const uint32_t dst = smem_base + L.halo_off + hb * L.halo_bytes;
+        const int x0 = (tc.w0 - p.pad_w) * p.c_in - G.rem;  // multiple of 8 elements
+        for (int kt = 0; kt < p.kt; ++kt) {
+          const int tau = tc.t + kt - (p.kt - 1);
+          const bool from_cache = tau < 0 && p.cache;
+          tma_load_4d(dst + kt * G.kt_stride * 2, from_cache ? &map_cache : &map_x,
+                      &halo_full[hb], x0, tc.h0 - p.pad_h, from_cache ? tau + (p.kt - 1) : tau,
+                      tc.n);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------ MMA issuer ----------------------------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kM, p.c_out);
+      // A: [kpad/8][16 row groups][8 rows][8]: K step 16*128 B, M step 128 B
+      const uint64_t adesc0 = smem_desc_noswizzle(smem_base + L.a_off, kM * 16u, 128u);
+      // B: [kpad/8][c_out][8]: K step c_out*16 B, N step 128 B
+      const uint32_t b_lbo = static_cast<uint32_t>(p.c_out) * 16u;
+      const uint64_t bdesc0 = smem_desc_noswizzle(smem_base + L.b_off, b_lbo, 128u);
+      if (!mbar_wait_bounded(b_full, 0, p.wait_limit_ns, p.status, 12)) ok = false;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++it) {
+        const int buf = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        if (!mbar_wait_bounded(&acc_empty[buf], ph ^ 1, p.wait_limit_ns, p.status, 13) ||
+            !mbar_wait_bounded(&a_full[buf], ph, p.wait_limit_ns, p.status, 14)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t a_st = adesc0 + ((buf * L.a_bytes) >> 4);
+        for (int j = 0; j < p.kpad / 16; ++j)
+          umma_bf16(tmem_base + buf * p.c_out, a_st + 2 * j * (kM * 16 / 16),
+                    bdesc0 + 2 * j * (b_lbo >> 4), idesc, j > 0 ? 1u : 0u);
+        umma_commit(&a_empty[buf]);
+        umma_commit(&acc_full[buf]);
+      }
+    }
+  } else {
+    // ------------------------------ epilogue (warps 6-9) -------------------------
+    const int q = warp % 4;
+    const int m = q * 32 + lane;
+    const int r = m / kTW, c = m % kTW;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+      const int buf = it & 1;
+      const Tile tc = thin_tile(tile, p);
+      uint32_t got = 0;
+      if (lane == 0)
+        got = mbar_wait_bounded(&acc_full[buf], (it >> 1) & 1, p.wait_limit_ns, p.status, 15)
+                  ? 1u
+                  : 0u;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) break;
+      tc_fence_after();
+      const int h = tc.h0 + r, w = tc.w0 + c;
+      const bool valid = h < p.h && w < p.w;
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * p.c_out);
+      __nv_bfloat16 *yrow =
+          p.y + (((static_cast<size_t>(tc.n) * p.t + tc.t) * p.h + h) * p.w + w) * p.c_out;
+      for (int j = 0; j < p.c_out; j += 16) {
+        float v[16];
+        __syncwarp();
+        tmem_ld16(taddr + j, v);
+        if (j + 16 >= p.c_out) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+        if (valid) {
+          uint4 o0, o1;
+          o0.x = pack_bf16x2(v[0] + sbias[j + 0], v[1] + sbias[j + 1]);
+          o0.y = pack_bf16x2(v[2] + sbias[j + 2], v[3] + sbias[j + 3]);
+          o0.z = pack_bf16x2(v[4] + sbias[j + 4], v[5] + sbias[j + 5]);
+          o0.w = pack_bf16x2(v[6] + sbias[j + 6], v[7] + sbias[j + 7]);
+          o1.x = pack_bf16x2(v[8] + sbias[j + 8], v[9] + sbias[j + 9]);
+          o1.y = pack_bf16x2(v[10] + sbias[j + 10], v[11] + sbias[j + 11]);
+          o1.z = pack_bf16x2(v[12] + sbias[j + 12], v[13] + sbias[j + 13]);
+          o1.w = pack_bf16x2(v[14] + sbias[j + 14], v[15] + sbias[j + 15]);
+          uint4 *dst = reinterpret_cast<uint4 *>(yrow + j);
+          dst[0] = o0;
+          dst[1] = o1;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+  if (!ok && threadIdx.x == 0) __nanosleep(100000);
+}
+
+__global__ void repack_thin_kernel(const __nv_bfloat16 *__restrict__ w, __nv_bfloat16 *img,
+                                   int c_out, int c_in, int taps, int kpad) {
+  // img[k8][co][e] = W[co][ci][tap] with k = tap * c_in + ci = k8 * 8 + e; 0 past K
+  const int total = kpad * c_out;
+  const int K = taps * c_in;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const int e = i % 8;
+    const int co = (i / 8) % c_out;
+    const int k8 = i / (8 * c_out);
+    const int k = k8 * 8 + e;
+    __nv_bfloat16 v = __float2bfloat16_rn(0.f);
+    if (k < K) {
+      const int tap = k / c_in, ci = k % c_in;
+      v = w[(static_cast<size_t>(co) * c_in + ci) * taps + tap];
+    }
+    img[i] = v;
+  }
+}
+
+}  // namespace
+
+size_t thin_smem_bytes(const ThinArgs &a) { return thin_layout(a).total + 1024; }
+
+int thin_tma_row(const ThinArgs &a) { return halo_geom(a).row; }
+
+cudaError_t launch_repack_thin(const __nv_bfloat16 *w, uint8_t *img, int c_out, int c_in,
+                               int taps, int kpad, cudaStream_t stream) {
+  const int total = kpad * c_out;
+  repack_thin_kernel<<<(total + 255) / 256, 256, 0, stream>>>(
+      w, reinterpret_cast<__nv_bfloat16 *>(img), c_out, c_in, taps, kpad);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_conv_thin(const CUtensorMap &map_x, const CUtensorMap &map_cache,
+                             const ThinArgs &args, unsigned grid, cudaStream_t stream) {
+  const size_t smem = thin_smem_bytes(args);
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(conv_thin_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  conv_thin_kernel<<<grid, kThreads, smem, stream>>>(map_x, map_cache, args);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace cc3d

@@ -46,8 +46,8 @@ cudaError_t launch_repack_umma(const __nv_bfloat16 *w, uint8_t *img, int c_out, 
 // Thin first-layer conv (c_in small): weights to [tap*c_in padded to kpad][c_out]
 // image and the kernel itself.
 struct ThinArgs {
-  const __nv_bfloat16 *x;         // [n][t][h][w][c_in]
-  const __nv_bfloat16 *cache;     // [n][kt-1][h][w][c_in] or null
+  const uint16_t *x;              // [n][t][h][w][c_in] bf16 bits
+  const uint16_t *cache;          // [n][kt-1][h][w][c_in] or null
   const uint8_t *wimg;            // [kpad/8][c_out][8] bf16 core-matrix image
   const float *bias;              // [c_out]
   __nv_bfloat16 *y;               // [n][t][h][w][c_out]
@@ -57,11 +57,16 @@ struct ThinArgs {
   int kpad;                       // K padded to a multiple of 16
   int tiles_w, tiles_h, n_tiles;
   int tmem_cols;
+  int use_tma;                    // halo by TMA (x and cache 16-byte aligned, w*c_in % 8 == 0)
+  int spec_rgb333;                // compile-time im2col (c_in 3, 3x3x3, pad 1, TMA halo)
 };
 cudaError_t launch_repack_thin(const __nv_bfloat16 *w, uint8_t *img, int c_out, int c_in,
                                int taps, int kpad, cudaStream_t stream);
 size_t thin_smem_bytes(const ThinArgs &a);
-cudaError_t launch_conv_thin(const ThinArgs &args, unsigned grid, cudaStream_t stream);
+// Elements per halo row of the TMA box (the box's inner extent).
+int thin_tma_row(const ThinArgs &a);
+cudaError_t launch_conv_thin(const CUtensorMap &map_x, const CUtensorMap &map_cache,
+                             const ThinArgs &args, unsigned grid, cudaStream_t stream);
 
 // fp32 SIMT direct convolution.
 struct Fp32Args {
