@@ -45,6 +45,12 @@ C2 = dict(c=384, t=5, h=30, w=52)
 C4 = dict(c=192, t=9, h=240, w=416)
 
 
+# DRAM bytes (read + write) per launch of the conv kernel on this workload,
+# from one ncu capture of the current kernel (profiles/ holds the summaries
+# and commands); None until captured.
+NCU_TRAFFIC = {"whole": 14.006272e6, "chunk": 11.61e6}
+
+
 def conv_flop(n, cin, cout, t, h, w, taps=27):
     return 2.0 * n * cout * cin * taps * t * h * w
 
@@ -215,14 +221,22 @@ def main():
     caches = [torch.empty((1, 2, H, W, c), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     flop_step = 2 * conv_flop(1, c, c, T, H, W)
 
-    def step(xin=None):
+    def step(xin=None, marks=None):
+        """One pass: the whole sequence, then 5 one-frame chunks carrying the
+        cache.  `marks` (T + 2 events) bracket each forward call."""
         src = x if xin is None else xin
+        if marks:
+            marks[0].record(stream)
         plan.forward(src, y_whole)
+        if marks:
+            marks[1].record(stream)
         cache = None
         for k in range(T):
             xk = xs[k] if xin is None else src[:, k:k + 1]
             plan.forward(xk, ys[k], t=1, cache_in=cache, cache_out=caches[k % 2])
             cache = caches[k % 2]
+            if marks:
+                marks[2 + k].record(stream)
 
     for k in range(args.warmup):
         flush_l2(k)
@@ -230,40 +244,35 @@ def main():
     cc3d.sync_status()
 
     sampler = ClockSampler(local)
-    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(T + 2)]
+             for _ in range(args.steps)]
     launches0 = cc3d.cc3d_launch_count()
     barrier()
     torch.cuda.synchronize()
     sampler.start()
     for k in range(args.steps):
         flush_l2(k)
-        ev0[k].record(stream)
-        step()
-        ev1[k].record(stream)
+        step(marks=marks[k])
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
     launches = cc3d.cc3d_launch_count() - launches0
     cc3d.sync_status()
-    step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
+    step_ms = [m[0].elapsed_time(m[-1]) for m in marks]
+    whole_ms = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
+    chunk_ms = statistics.mean(m[1 + i].elapsed_time(m[2 + i]) for m in marks for i in range(T))
     ms_local = sum(step_ms) / len(step_ms)
     ms = max_over_ranks(ms_local)
     value = world * flop_step / (ms * 1e-3) / 1e12
-
-    # --- roofline of the dominant kernel: the whole-sequence conv launch ---
-    ew0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ew1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    for k in range(args.steps):
-        flush_l2(k)
-        ew0[k].record(stream)
-        plan.forward(x, y_whole)
-        ew1[k].record(stream)
-    torch.cuda.synchronize()
-    whole_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ew0, ew1))
-    achieved = conv_flop(1, c, c, T, H, W) / (whole_ms * 1e-3) / 1e12
-    # chunk (streaming) launch time for context
-    chunk_ms = (ms_local - whole_ms) / T
+    # the conv kernel over the timed region: 6 forward calls per step (each
+    # is the conv launch plus its small cache-update copy)
+    flop_whole = conv_flop(1, c, c, T, H, W)
+    flop_chunk = conv_flop(1, c, c, 1, H, W)
+    avg_launch_ms = (whole_ms + T * chunk_ms) / (T + 1)
+    achieved = (flop_step / (T + 1)) / (avg_launch_ms * 1e-3) / 1e12
+    traffic_avg = None
+    if NCU_TRAFFIC["whole"] is not None and NCU_TRAFFIC["chunk"] is not None:
+        traffic_avg = (NCU_TRAFFIC["whole"] + T * NCU_TRAFFIC["chunk"]) / (T + 1)
 
     # --- end to end through the public API with host buffers ---
     x_host = x.cpu().pin_memory()
@@ -344,10 +353,18 @@ def main():
                        "flop_per_step": flop_step},
             "roofline": {"bound": "tensor", "achieved": achieved,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": achieved / peaks["bf16_tflops"], "traffic": None,
-                         "kernel": "conv_umma_kernel (whole-sequence launch)",
-                         "launch_ms": whole_ms, "peak_basis": "burst bf16 (" + peaks["source"] + ")"},
-            "streaming_chunk_ms": chunk_ms,
+                         "frac": achieved / peaks["bf16_tflops"], "traffic": traffic_avg,
+                         "kernel": "conv_umma_kernel, average over the 6 launches of a step",
+                         "peak_basis": "burst bf16 (" + peaks["source"] + ")",
+                         "per_launch": {
+                             "whole_sequence": {"ms": whole_ms, "gflop": flop_whole / 1e9,
+                                                "tflops": flop_whole / whole_ms / 1e9,
+                                                "frac": flop_whole / whole_ms / 1e9 / peaks["bf16_tflops"],
+                                                "traffic": NCU_TRAFFIC["whole"]},
+                             "one_frame_chunk": {"ms": chunk_ms, "gflop": flop_chunk / 1e9,
+                                                 "tflops": flop_chunk / chunk_ms / 1e9,
+                                                 "frac": flop_chunk / chunk_ms / 1e9 / peaks["bf16_tflops"],
+                                                 "traffic": NCU_TRAFFIC["chunk"]}}},
             "resblock": resblock,
             "e2e": e2e,
             "gpu_launches": launches,

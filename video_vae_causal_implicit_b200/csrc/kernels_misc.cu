@@ -16,6 +16,11 @@ namespace cc3d {
 
 namespace {
 
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&p);
+}
+
 __global__ void repack_umma_kernel(const __nv_bfloat16 *__restrict__ w, __nv_bfloat16 *img,
                                    int c_out, int c_in, int taps, int nt, int kc) {
   const long long total = static_cast<long long>(c_out) * c_in * taps;
@@ -70,10 +75,12 @@ __global__ void copy_frames_kernel(const uint8_t *__restrict__ cache_in,
   }
 }
 
-// One warp per voxel; lane l owns channel groups l, l+32, ... of 8 channels
-// (16 bytes).  Sum of squares reduced with a fixed xor butterfly, so the
-// result does not depend on scheduling.
-template <int CPL>
+// A warp normalises VPW voxels per iteration; lane l owns channel groups
+// l, l+32, ... of 8 channels (16 bytes) of each.  All loads of the VPW
+// voxels are issued before any reduction so enough bytes are in flight to
+// keep HBM busy.  The sum of squares is reduced with a fixed xor butterfly,
+// so the result does not depend on scheduling.
+template <int CPL, int VPW>
 __global__ void rmsnorm_silu_kernel(const __nv_bfloat16 *__restrict__ x,
                                     const float *__restrict__ gamma,
                                     const float *__restrict__ beta, long long voxels, int c,
@@ -83,51 +90,57 @@ __global__ void rmsnorm_silu_kernel(const __nv_bfloat16 *__restrict__ x,
   const long long nwarps = static_cast<long long>(gridDim.x) * blockDim.x / 32;
   const int groups = c / 8;
   const float scale = sqrtf(static_cast<float>(c));
-  for (long long v = warp0; v < voxels; v += nwarps) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + v * c);
-    float vals[CPL][8];
-    float ss = 0.f;
+  for (long long v0 = warp0 * VPW; v0 < voxels; v0 += nwarps * VPW) {
+    uint4 raw[VPW][CPL];
 #pragma unroll
-    for (int k = 0; k < CPL; ++k) {
-      const int g = lane + 32 * k;
-      if (g < groups) {
-        uint4 u = src[g];
-        const __nv_bfloat16 *b = reinterpret_cast<const __nv_bfloat16 *>(&u);
+    for (int u = 0; u < VPW; ++u)
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) {
+        const int g = lane + 32 * k;
+        raw[u][k] = make_uint4(0, 0, 0, 0);
+        if (v0 + u < voxels && g < groups)
+          raw[u][k] = __ldcs(reinterpret_cast<const uint4 *>(x + (v0 + u) * c) + g);
+      }
+    float inv[VPW];
+#pragma unroll
+    for (int u = 0; u < VPW; ++u) {
+      float ss = 0.f;
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) {
+        const __nv_bfloat16 *b = reinterpret_cast<const __nv_bfloat16 *>(&raw[u][k]);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          vals[k][e] = __bfloat162float(b[e]);
-          ss = fmaf(vals[k][e], vals[k][e], ss);
+          const float f = __bfloat162float(b[e]);
+          ss = fmaf(f, f, ss);
         }
       }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      inv[u] = scale / fmaxf(sqrtf(ss), 1e-12f);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float inv = scale / fmaxf(sqrtf(ss), 1e-12f);
-    uint4 *dst = reinterpret_cast<uint4 *>(y + v * c);
+    for (int u = 0; u < VPW; ++u)
 #pragma unroll
-    for (int k = 0; k < CPL; ++k) {
-      const int g = lane + 32 * k;
-      if (g < groups) {
-        float o[8];
+      for (int k = 0; k < CPL; ++k) {
+        const int g = lane + 32 * k;
+        if (v0 + u < voxels && g < groups) {
+          const __nv_bfloat16 *b = reinterpret_cast<const __nv_bfloat16 *>(&raw[u][k]);
+          float o[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int ch = g * 8 + e;
-          float a = vals[k][e] * inv * gamma[ch];
-          if (beta) a += beta[ch];
-          o[e] = a / (1.0f + __expf(-a));
+          for (int e = 0; e < 8; ++e) {
+            const int ch = g * 8 + e;
+            float a = __bfloat162float(b[e]) * inv[u] * __ldg(gamma + ch);
+            if (beta) a += __ldg(beta + ch);
+            o[e] = a / (1.0f + __expf(-a));
+          }
+          uint4 w;
+          w.x = pack2(o[0], o[1]);
+          w.y = pack2(o[2], o[3]);
+          w.z = pack2(o[4], o[5]);
+          w.w = pack2(o[6], o[7]);
+          __stcs(reinterpret_cast<uint4 *>(y + (v0 + u) * c) + g, w);
         }
-        uint4 u;
-        __nv_bfloat162 p0 = __floats2bfloat162_rn(o[0], o[1]);
-        __nv_bfloat162 p1 = __floats2bfloat162_rn(o[2], o[3]);
-        __nv_bfloat162 p2 = __floats2bfloat162_rn(o[4], o[5]);
-        __nv_bfloat162 p3 = __floats2bfloat162_rn(o[6], o[7]);
-        u.x = *reinterpret_cast<uint32_t *>(&p0);
-        u.y = *reinterpret_cast<uint32_t *>(&p1);
-        u.z = *reinterpret_cast<uint32_t *>(&p2);
-        u.w = *reinterpret_cast<uint32_t *>(&p3);
-        dst[g] = u;
       }
-    }
   }
 }
 
@@ -216,15 +229,18 @@ cudaError_t launch_rmsnorm_silu(const __nv_bfloat16 *x, const float *gamma, cons
                                 long long voxels, int c, __nv_bfloat16 *y, cudaStream_t stream) {
   const int groups = c / 8;
   const int cpl = (groups + 31) / 32;
+  constexpr int kVpw = 4;
   const int block = 256;
-  long long g = (voxels * 32 + block - 1) / block;
-  if (g > 148LL * 64) g = 148LL * 64;
+  long long warps = (voxels + kVpw - 1) / kVpw;
+  long long g = (warps * 32 + block - 1) / block;
+  if (g > 148LL * 16) g = 148LL * 16;
   if (g < 1) g = 1;
+  const int grid = static_cast<int>(g);
   switch (cpl) {
-    case 1: rmsnorm_silu_kernel<1><<<static_cast<int>(g), block, 0, stream>>>(x, gamma, beta, voxels, c, y); break;
-    case 2: rmsnorm_silu_kernel<2><<<static_cast<int>(g), block, 0, stream>>>(x, gamma, beta, voxels, c, y); break;
-    case 3: rmsnorm_silu_kernel<3><<<static_cast<int>(g), block, 0, stream>>>(x, gamma, beta, voxels, c, y); break;
-    case 4: rmsnorm_silu_kernel<4><<<static_cast<int>(g), block, 0, stream>>>(x, gamma, beta, voxels, c, y); break;
+    case 1: rmsnorm_silu_kernel<1, kVpw><<<grid, block, 0, stream>>>(x, gamma, beta, voxels, c, y); break;
+    case 2: rmsnorm_silu_kernel<2, kVpw><<<grid, block, 0, stream>>>(x, gamma, beta, voxels, c, y); break;
+    case 3: rmsnorm_silu_kernel<3, kVpw><<<grid, block, 0, stream>>>(x, gamma, beta, voxels, c, y); break;
+    case 4: rmsnorm_silu_kernel<4, kVpw><<<grid, block, 0, stream>>>(x, gamma, beta, voxels, c, y); break;
     default: return cudaErrorInvalidValue;
   }
   count_launch();
