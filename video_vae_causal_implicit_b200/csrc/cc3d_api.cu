@@ -120,6 +120,23 @@ bool encode_thin_map(CUtensorMap *m, const void *base, int c, int w, int h, int 
   return r == CUDA_SUCCESS;
 }
 
+// Store map over y (NDHWC bf16): dims (C, W, H, T, N), a box of 32 channels
+// x 8 columns x 16 rows with the 64-byte swizzle.
+bool encode_store_map(CUtensorMap *m, const void *base, int c, int w, int h, int t, int n) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[5] = {(cuuint64_t)c, (cuuint64_t)w, (cuuint64_t)h, (cuuint64_t)t,
+                        (cuuint64_t)n};
+  cuuint64_t strides[4] = {(cuuint64_t)c * 2, (cuuint64_t)c * 2 * w, (cuuint64_t)c * 2 * w * h,
+                           (cuuint64_t)c * 2 * w * h * t};
+  cuuint32_t box[5] = {32, 8, 16, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
@@ -144,7 +161,7 @@ struct cc3d_plan {
   uint8_t *wimg;
   // fp32 / thin
   void *wraw;
-  int kpad;
+  int kpad, thin_spec;
   float *bias, *gamma, *beta;
   cc3d_stats st;
   std::mutex mu;
@@ -270,6 +287,11 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
         cudaSuccess)
       p->sm_count = 148;
     p->kpad = (taps * desc->c_in + 15) / 16 * 16;
+    // RGB input with a 3x3x3 kernel: segment-ordered K (see conv_thin.cu)
+    p->thin_spec = (desc->c_in == 3 && desc->kt == 3 && desc->kh == 3 && desc->kw == 3 &&
+                    desc->pad_h == 1 && desc->pad_w == 1 && p->kpad == 96)
+                       ? 1
+                       : 0;
     p->nt = desc->c_out;
     p->n_ntiles = 1;
     int cols = 32;
@@ -280,7 +302,7 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
       std::memset(&probe, 0, sizeof probe);
       probe.kpad = p->kpad; probe.c_out = desc->c_out; probe.kt = desc->kt;
       probe.kh = desc->kh; probe.kw = desc->kw; probe.c_in = desc->c_in;
-      probe.pad_w = desc->pad_w; probe.use_tma = 1; probe.spec_rgb333 = 0;
+      probe.pad_w = desc->pad_w; probe.use_tma = 1; probe.spec_rgb333 = 0; probe.store_boxes = 1;
       int per_sm = static_cast<int>((228 * 1024) / (thin_smem_bytes(probe) + 1024));
       if (per_sm > 512 / cols) per_sm = 512 / cols;
       if (per_sm > 2) per_sm = 2;
@@ -294,7 +316,7 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
     if (cudaMalloc(&p->wraw, bytes) != cudaSuccess) { s = CC3D_ERR_OOM; goto fail; }
     e = launch_repack_thin(static_cast<const __nv_bfloat16 *>(desc->weight),
                            static_cast<uint8_t *>(p->wraw), desc->c_out, desc->c_in, taps,
-                           p->kpad, 0);
+                           p->kpad, p->thin_spec, 0);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
   } else if (variant == CC3D_VARIANT_FP32) {
@@ -470,15 +492,17 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
       else if (!(cache_in && front > 0))
         mc = mx;
     }
-    // the specialised im2col assumes the TMA halo geometry of RGB 3x3x3:
-    // rows of 40 elements, frames 768 elements apart
-    a.spec_rgb333 = (a.use_tma && d.c_in == 3 && d.kt == 3 && d.kh == 3 && d.kw == 3 &&
-                     thin_tma_row(a) == 40 && p->kpad == 96)
+    a.spec_rgb333 = p->thin_spec;
+    CUtensorMap my_map;
+    std::memset(&my_map, 0, sizeof my_map);
+    a.store_boxes = (d.c_out % 32 == 0 && umma_tile_w() == 8 && umma_tile_h() == 16 &&
+                     encode_store_map(&my_map, y, d.c_out, d.w, d.h, t, d.n))
                         ? 1
                         : 0;
     tiles = static_cast<uint64_t>(a.n_tiles);
     const uint64_t slots = static_cast<uint64_t>(p->sm_count) * p->ctas_per_sm;
-    e = launch_conv_thin(mx, mc, a, static_cast<unsigned>(tiles < slots ? tiles : slots), stream);
+    e = launch_conv_thin(mx, mc, my_map, a, static_cast<unsigned>(tiles < slots ? tiles : slots),
+                         stream);
   } else {
     CUtensorMap mx, mc;
     const int box_w = umma_tile_w() + d.kw - 1, box_h = umma_tile_h() + d.kh - 1;

@@ -44,7 +44,7 @@ constexpr int kBuilders = 128;  // warps 0-3
 constexpr int kMmaWarp = 4;
 constexpr int kLoadWarp = 5;    // halo TMA producer
 constexpr int kThreads = 320;   // + epilogue warps 6-9
-constexpr int kNH = 4;          // halo ring depth (loader runs ahead)
+constexpr int kNH = 3;          // halo ring depth (loader runs ahead)
 
 // Halo geometry of one tile.  Frames are [kt] slabs of `kt_stride`
 // elements; a slab holds (16 + kh - 1) rows of `row` elements; the pixel
@@ -56,24 +56,22 @@ struct HaloGeom {
 __host__ __device__ inline uint32_t rup(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
 __host__ __device__ inline HaloGeom halo_geom(const ThinArgs &a) {
+  // One halo row is a run of the flattened (W * C_in) image row that starts
+  // on a 16-byte boundary: the first element, (w0 - pad_w) * C_in, is
+  // rounded down to a multiple of 8 (w0 is a multiple of 8, so the
+  // remainder `rem` is the same for every tile).  The TMA box and the
+  // plain-load staging fill exactly this shape, zero outside the image.
   HaloGeom g;
   const int hh = kTH + a.kh - 1, hw = kTW + a.kw - 1;
-  if (a.use_tma) {
-    // rows start on a 16-byte boundary: round the first element down to a
-    // multiple of 8 (w0 is a multiple of 8, so the remainder is constant)
-    g.rem = ((-a.pad_w * a.c_in) % 8 + 8) % 8;
-    g.row = static_cast<int>(rup(g.rem + hw * a.c_in, 8));
-    g.kt_stride = static_cast<int>(rup(g.row * hh * 2, 128) / 2);
-  } else {
-    g.rem = 0;
-    g.row = hw * a.c_in;
-    g.kt_stride = g.row * hh;
-  }
+  g.rem = ((-a.pad_w * a.c_in) % 8 + 8) % 8;
+  g.row = static_cast<int>(rup(g.rem + hw * a.c_in, 8));
+  g.kt_stride = static_cast<int>(rup(g.row * hh * 2, 128) / 2);
   return g;
 }
 
 struct ThinLayout {
-  uint32_t b_off, a_off, a_bytes, halo_off, halo_bytes, koff_off, bias_off, bar_off, total;
+  uint32_t b_off, a_off, a_bytes, halo_off, halo_bytes, koff_off, bias_off, stage_off,
+      stage_pitch, bar_off, total;
 };
 
 __host__ __device__ inline ThinLayout thin_layout(const ThinArgs &a) {
@@ -86,8 +84,12 @@ __host__ __device__ inline ThinLayout thin_layout(const ThinArgs &a) {
   L.halo_off = L.a_off + 2 * L.a_bytes;
   L.halo_bytes = rup(static_cast<uint32_t>(a.kt) * g.kt_stride * 2u, 128u);  // per buffer
   L.koff_off = L.halo_off + kNH * L.halo_bytes;  // int32 halo offset per K index
-  L.bias_off = L.koff_off + 4u * a.kpad;           // fp32 bias copy
-  L.bar_off = rup(L.bias_off + 4u * a.c_out, 64u);
+  L.bias_off = rup(L.koff_off + 4u * a.kpad, 16u);  // fp32 bias copy
+  // output staging: 128 pixels, each c_out * 2 bytes plus one spare 16-byte
+  // chunk so eight consecutive pixels start in eight different bank quads
+  L.stage_pitch = static_cast<uint32_t>(a.c_out) * 2u + 16u;
+  L.stage_off = rup(L.bias_off + 4u * a.c_out, 1024u);
+  L.bar_off = rup(L.stage_off + kM * L.stage_pitch, 64u);
   // b_full, a_full[2], a_empty[2], acc_full[2], acc_empty[2],
   // halo_full[kNH], halo_empty[kNH], tmem slot + flag
   L.total = L.bar_off + 8u * (9 + 2 * kNH) + 16u;
@@ -121,33 +123,37 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
-// Row of A for C_in = 3 and a 3x3x3 kernel read from the TMA halo
-// (rows of 40 elements, frames 768 elements apart): K index
-// k = ((kt * 3 + ih) * 3 + iw) * 3 + ci sits at halo offset
-// kt * 768 + ih * 40 + iw * 3 + ci, all compile-time; K 81..95 is zero.
+// Row of A for C_in = 3 and a 3x3x3 kernel, read from the halo (rows of 40
+// elements, frames 768 elements apart).  K is ordered as nine segments
+// (kt, kh) of ten: k = ((kt * 3 + kh) * 10) + kw * 3 + ci, the tenth element
+// of each segment (the next pixel's first channel) meeting a zero weight,
+// and K 90..95 zero.  A segment is ten consecutive halo elements, so it is
+// read as six aligned 32-bit words and realigned with funnel shifts.
 __device__ __forceinline__ void build_row_rgb333(const uint16_t *hbits, uint8_t *a_row) {
+  const uintptr_t e0 = reinterpret_cast<uintptr_t>(hbits);
+  const uint32_t *w32 = reinterpret_cast<const uint32_t *>(e0 & ~static_cast<uintptr_t>(3));
+  const uint32_t sh = (e0 & 2) ? 16u : 0u;
+  uint32_t pairs[48];
 #pragma unroll
-  for (int k8 = 0; k8 < 12; ++k8) {
-    uint32_t packed[4];
+  for (int seg = 0; seg < 9; ++seg) {
+    const int off = ((seg / 3) * 768 + (seg % 3) * 40) / 2;  // even element offsets
+    uint32_t w[6];
 #pragma unroll
-    for (int e2 = 0; e2 < 4; ++e2) {
-      uint32_t v2[2];
+    for (int i = 0; i < 6; ++i) w[i] = w32[off + i];
 #pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        const int k = k8 * 8 + e2 * 2 + s;
-        const int ci = k % 3, iw = (k / 3) % 3, ih = (k / 9) % 3, kt = k / 27;
-        v2[s] = k < 81 ? static_cast<uint32_t>(hbits[kt * 768 + ih * 40 + iw * 3 + ci]) : 0u;
-      }
-      packed[e2] = v2[0] | (v2[1] << 16);
-    }
-    *reinterpret_cast<uint4 *>(a_row + k8 * (kM * 16)) =
-        make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    for (int i = 0; i < 5; ++i) pairs[seg * 5 + i] = __funnelshift_r(w[i], w[i + 1], sh);
   }
+  pairs[45] = pairs[46] = pairs[47] = 0u;
+#pragma unroll
+  for (int k8 = 0; k8 < 12; ++k8)
+    *reinterpret_cast<uint4 *>(a_row + k8 * (kM * 16)) =
+        make_uint4(pairs[4 * k8], pairs[4 * k8 + 1], pairs[4 * k8 + 2], pairs[4 * k8 + 3]);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     conv_thin_kernel(const __grid_constant__ CUtensorMap map_x,
-                     const __grid_constant__ CUtensorMap map_cache, ThinArgs p) {
+                     const __grid_constant__ CUtensorMap map_cache,
+                     const __grid_constant__ CUtensorMap map_y, ThinArgs p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -164,6 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9 + 2 * kNH);
   float *sbias = reinterpret_cast<float *>(smem + L.bias_off);
   volatile uint32_t *go_flag = tmem_slot + 1;
+  volatile uint32_t *epi_flag = tmem_slot + 2;
   int *koff = reinterpret_cast<int *>(smem + L.koff_off);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -230,42 +237,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t hph = static_cast<uint32_t>((it / kNH) & 1);
       uint16_t *halo = reinterpret_cast<uint16_t *>(smem + L.halo_off + hb * L.halo_bytes);
       if (!p.use_tma) {
-        // stage the halo with plain loads: issue a batch of loads, then store
+        // stage the halo box with plain loads (zero outside the image): the
+        // same shape the TMA box has; batches of loads are issued together
         const Tile tc = thin_tile(tile, p);
-        const int helems = p.kt * hh * hw * p.c_in;
+        const int helems = p.kt * hh * G.row;
+        const long long wc = static_cast<long long>(p.w) * p.c_in;
+        const long long x0 = static_cast<long long>(tc.w0 - p.pad_w) * p.c_in - G.rem;
         for (int i0 = 0; i0 < helems; i0 += 8 * kBuilders) {
           uint16_t v[8];
+          int dst[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const int i = i0 + u * kBuilders + threadIdx.x;
             v[u] = 0;
+            dst[u] = -1;
             if (i < helems) {
-              int q = i;
-              const int ci = q % p.c_in;
-              q /= p.c_in;
-              const int cc = q % hw;
-              q /= hw;
+              const int pos = i % G.row;
+              const int q = i / G.row;
               const int rr = q % hh;
               const int kt = q / hh;
+              dst[u] = kt * G.kt_stride + rr * G.row + pos;
               const int tau = tc.t + kt - (p.kt - 1);
-              const int h = tc.h0 - p.pad_h + rr, w = tc.w0 - p.pad_w + cc;
-              if (h >= 0 && h < p.h && w >= 0 && w < p.w) {
-                const size_t pix = (static_cast<size_t>(h) * p.w + w) * p.c_in + ci;
+              const int h = tc.h0 - p.pad_h + rr;
+              const long long e = x0 + pos;
+              if (h >= 0 && h < p.h && e >= 0 && e < wc) {
                 const uint16_t *src = nullptr;
                 if (tau >= 0)
-                  src = p.x + ((static_cast<size_t>(tc.n) * p.t + tau) * p.h * p.w) * p.c_in;
+                  src = p.x + (static_cast<size_t>(tc.n) * p.t + tau) * p.h * wc;
                 else if (p.cache)
-                  src = p.cache + ((static_cast<size_t>(tc.n) * (p.kt - 1) + tau + (p.kt - 1)) *
-                                   p.h * p.w) * p.c_in;
-                if (src) v[u] = src[pix];
+                  src = p.cache + (static_cast<size_t>(tc.n) * (p.kt - 1) + tau + (p.kt - 1)) *
+                                      p.h * wc;
+                if (src) v[u] = src[static_cast<size_t>(h) * wc + e];
               }
             }
           }
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * kBuilders + threadIdx.x;
-            if (i < helems) halo[i] = v[u];  // row = hw * c_in, kt_stride = row * hh
-          }
+          for (int u = 0; u < 8; ++u)
+            if (dst[u] >= 0) halo[dst[u]] = v[u];
         }
       }
       // thread 0 waits for: this A buffer free (MMAs of two tiles ago done)
@@ -362,52 +370,110 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------ epilogue (warps 6-9) -------------------------
+    // Each thread owns one output pixel (its tensor-memory lane): TMEM ->
+    // +bias -> bf16 -> shared staging -> global through the TMA engine.
+    //  * store_boxes (c_out % 32 == 0): the tile is staged as c_out / 32
+    //    boxes of [128 pixels][32 channels] with the 64-byte swizzle (eight
+    //    consecutive pixels write eight different bank quads), and one thread
+    //    stores each box with a TMA tensor store, which also clips the tile
+    //    at the image edge;
+    //  * otherwise each thread bulk-copies its own pixel from a padded slot.
     const int q = warp % 4;
     const int m = q * 32 + lane;
     const int r = m / kTW, c = m % kTW;
+    const int et = threadIdx.x - 6 * 32;  // 0..127
+    uint8_t *stage = smem + L.stage_off;
+    uint8_t *my = stage + m * L.stage_pitch;
+    const uint32_t pix_bytes = static_cast<uint32_t>(p.c_out) * 2u;
     int it = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
       const int buf = it & 1;
       const Tile tc = thin_tile(tile, p);
-      uint32_t got = 0;
-      if (lane == 0)
-        got = mbar_wait_bounded(&acc_full[buf], (it >> 1) & 1, p.wait_limit_ns, p.status, 15)
-                  ? 1u
-                  : 0u;
-      got = __shfl_sync(0xffffffffu, got, 0);
-      if (!got) break;
+      // one thread waits (and, with box stores, lets its previous stores
+      // finish reading the staging); the four warps agree through shared
+      // memory so all of them take the named barriers or all leave
+      if (et == 0) {
+        if (p.store_boxes) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        *epi_flag =
+            mbar_wait_bounded(&acc_full[buf], (it >> 1) & 1, p.wait_limit_ns, p.status, 15) ? 1u
+                                                                                            : 0u;
+      }
+      asm volatile("bar.sync 2, %0;" ::"n"(128) : "memory");
+      if (!*epi_flag) break;
       tc_fence_after();
-      const int h = tc.h0 + r, w = tc.w0 + c;
-      const bool valid = h < p.h && w < p.w;
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * p.c_out);
-      __nv_bfloat16 *yrow =
-          p.y + (((static_cast<size_t>(tc.n) * p.t + tc.t) * p.h + h) * p.w + w) * p.c_out;
-      for (int j = 0; j < p.c_out; j += 16) {
-        float v[16];
+      if (!p.store_boxes) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      for (int j0 = 0; j0 < p.c_out; j0 += 48) {
+        // up to three 16-column loads in flight, one wait
+        const int nld = (p.c_out - j0) >= 48 ? 3 : (p.c_out - j0) / 16;
+        uint32_t raw[48];
         __syncwarp();
-        tmem_ld16(taddr + j, v);
-        if (j + 16 >= p.c_out) {
+#pragma unroll
+        for (int u = 0; u < 3; ++u)
+          if (u < nld) tmem_ld16_nowait(taddr + j0 + 16 * u, raw + 16 * u);
+        tmem_wait_ld();
+        tmem_regs_after_wait<48>(raw);
+        if (j0 + 48 >= p.c_out) {
+          // last read of this accumulator: hand the buffer back to the MMA warp
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
-        if (valid) {
-          uint4 o0, o1;
-          o0.x = pack_bf16x2(v[0] + sbias[j + 0], v[1] + sbias[j + 1]);
-          o0.y = pack_bf16x2(v[2] + sbias[j + 2], v[3] + sbias[j + 3]);
-          o0.z = pack_bf16x2(v[4] + sbias[j + 4], v[5] + sbias[j + 5]);
-          o0.w = pack_bf16x2(v[6] + sbias[j + 6], v[7] + sbias[j + 7]);
-          o1.x = pack_bf16x2(v[8] + sbias[j + 8], v[9] + sbias[j + 9]);
-          o1.y = pack_bf16x2(v[10] + sbias[j + 10], v[11] + sbias[j + 11]);
-          o1.z = pack_bf16x2(v[12] + sbias[j + 12], v[13] + sbias[j + 13]);
-          o1.w = pack_bf16x2(v[14] + sbias[j + 14], v[15] + sbias[j + 15]);
-          uint4 *dst = reinterpret_cast<uint4 *>(yrow + j);
-          dst[0] = o0;
-          dst[1] = o1;
+#pragma unroll
+        for (int u = 0; u < 3; ++u) {
+          if (u >= nld) continue;
+          const int j = j0 + 16 * u;
+          const float4 *b4 = reinterpret_cast<const float4 *>(sbias + j);
+          uint32_t o[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 t4 = b4[i];
+            o[2 * i] = pack_bf16x2(__uint_as_float(raw[16 * u + 4 * i]) + t4.x,
+                                   __uint_as_float(raw[16 * u + 4 * i + 1]) + t4.y);
+            o[2 * i + 1] = pack_bf16x2(__uint_as_float(raw[16 * u + 4 * i + 2]) + t4.z,
+                                       __uint_as_float(raw[16 * u + 4 * i + 3]) + t4.w);
+          }
+          if (p.store_boxes) {
+            // channels j..j+15 = chunks (j % 32) / 8 and +1 of box j / 32
+            uint8_t *box = stage + (j / 32) * (kM * 64) + m * 64;
+            const int ch0 = (j % 32) / 8, sw = (m >> 1) & 3;
+            *reinterpret_cast<uint4 *>(box + ((ch0 ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4 *>(box + (((ch0 + 1) ^ sw) << 4)) =
+                make_uint4(o[4], o[5], o[6], o[7]);
+          } else {
+            reinterpret_cast<uint4 *>(my + j * 2)[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            reinterpret_cast<uint4 *>(my + j * 2)[1] = make_uint4(o[4], o[5], o[6], o[7]);
+          }
+        }
+      }
+      fence_proxy_async_smem();  // staged bytes, written by this thread, to the TMA engine
+      if (p.store_boxes) {
+        asm volatile("bar.sync 2, %0;" ::"n"(128) : "memory");
+        if (et == 0) {
+          for (int bx = 0; bx < p.c_out / 32; ++bx)
+            asm volatile(
+                "cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group"
+                " [%0, {%1, %2, %3, %4, %5}], [%6];" ::"l"(reinterpret_cast<uint64_t>(&map_y)),
+                "r"(bx * 32), "r"(tc.w0), "r"(tc.h0), "r"(tc.t), "r"(tc.n),
+                "r"(smem_u32(stage + bx * (kM * 64)))
+                : "memory");
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+      } else {
+        const int h = tc.h0 + r, w = tc.w0 + c;
+        if (h < p.h && w < p.w) {
+          __nv_bfloat16 *dst =
+              p.y + (((static_cast<size_t>(tc.n) * p.t + tc.t) * p.h + h) * p.w + w) * p.c_out;
+          asm volatile(
+              "cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+              "r"(smem_u32(my)), "r"(pix_bytes)
+              : "memory");
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
         }
       }
     }
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
 
   tc_fence_before();
@@ -421,8 +487,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 __global__ void repack_thin_kernel(const __nv_bfloat16 *__restrict__ w, __nv_bfloat16 *img,
-                                   int c_out, int c_in, int taps, int kpad) {
-  // img[k8][co][e] = W[co][ci][tap] with k = tap * c_in + ci = k8 * 8 + e; 0 past K
+                                   int c_out, int c_in, int taps, int kpad, int spec) {
+  // img[k8][co][e] = W[co][ci][tap] at K index k = k8 * 8 + e; 0 past K.
+  // Generic order: k = tap * c_in + ci.  RGB 3x3x3 order (spec): nine
+  // segments of ten, k = (kt * 3 + kh) * 10 + kw * 3 + ci, the tenth zero.
   const int total = kpad * c_out;
   const int K = taps * c_in;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
@@ -431,7 +499,13 @@ __global__ void repack_thin_kernel(const __nv_bfloat16 *__restrict__ w, __nv_bfl
     const int k8 = i / (8 * c_out);
     const int k = k8 * 8 + e;
     __nv_bfloat16 v = __float2bfloat16_rn(0.f);
-    if (k < K) {
+    if (spec) {
+      const int seg = k / 10, j = k % 10;
+      if (seg < 9 && j < 9) {
+        const int tap = seg * 3 + j / 3, ci = j % 3;
+        v = w[(static_cast<size_t>(co) * 3 + ci) * 27 + tap];
+      }
+    } else if (k < K) {
       const int tap = k / c_in, ci = k % c_in;
       v = w[(static_cast<size_t>(co) * c_in + ci) * taps + tap];
     }
@@ -446,16 +520,17 @@ size_t thin_smem_bytes(const ThinArgs &a) { return thin_layout(a).total + 1024; 
 int thin_tma_row(const ThinArgs &a) { return halo_geom(a).row; }
 
 cudaError_t launch_repack_thin(const __nv_bfloat16 *w, uint8_t *img, int c_out, int c_in,
-                               int taps, int kpad, cudaStream_t stream) {
+                               int taps, int kpad, int spec, cudaStream_t stream) {
   const int total = kpad * c_out;
   repack_thin_kernel<<<(total + 255) / 256, 256, 0, stream>>>(
-      w, reinterpret_cast<__nv_bfloat16 *>(img), c_out, c_in, taps, kpad);
+      w, reinterpret_cast<__nv_bfloat16 *>(img), c_out, c_in, taps, kpad, spec);
   count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_conv_thin(const CUtensorMap &map_x, const CUtensorMap &map_cache,
-                             const ThinArgs &args, unsigned grid, cudaStream_t stream) {
+                             const CUtensorMap &map_y, const ThinArgs &args, unsigned grid,
+                             cudaStream_t stream) {
   const size_t smem = thin_smem_bytes(args);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   static bool attr_set = false;
@@ -465,7 +540,7 @@ cudaError_t launch_conv_thin(const CUtensorMap &map_x, const CUtensorMap &map_ca
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  conv_thin_kernel<<<grid, kThreads, smem, stream>>>(map_x, map_cache, args);
+  conv_thin_kernel<<<grid, kThreads, smem, stream>>>(map_x, map_cache, map_y, args);
   count_launch();
   return cudaGetLastError();
 }

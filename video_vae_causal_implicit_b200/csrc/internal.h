@@ -58,15 +58,17 @@ struct ThinArgs {
   int tiles_w, tiles_h, n_tiles;
   int tmem_cols;
   int use_tma;                    // halo by TMA (x and cache 16-byte aligned, w*c_in % 8 == 0)
-  int spec_rgb333;                // compile-time im2col (c_in 3, 3x3x3, pad 1, TMA halo)
+  int spec_rgb333;                // RGB 3x3x3 pad 1: segment-ordered K (set at plan time)
+  int store_boxes;                // y written by TMA tensor stores (c_out % 32 == 0)
 };
 cudaError_t launch_repack_thin(const __nv_bfloat16 *w, uint8_t *img, int c_out, int c_in,
-                               int taps, int kpad, cudaStream_t stream);
+                               int taps, int kpad, int spec, cudaStream_t stream);
 size_t thin_smem_bytes(const ThinArgs &a);
 // Elements per halo row of the TMA box (the box's inner extent).
 int thin_tma_row(const ThinArgs &a);
 cudaError_t launch_conv_thin(const CUtensorMap &map_x, const CUtensorMap &map_cache,
-                             const ThinArgs &args, unsigned grid, cudaStream_t stream);
+                             const CUtensorMap &map_y, const ThinArgs &args, unsigned grid,
+                             cudaStream_t stream);
 
 // fp32 SIMT direct convolution.
 struct Fp32Args {
