@@ -29,12 +29,14 @@ namespace {
 
 std::atomic<uint64_t> g_launches{0};
 
+// Bound of every device-side wait, read once per process from
+// CC3D_WAIT_LIMIT_US (microseconds; default 2 s).
 unsigned long long wait_limit_ns() {
   static unsigned long long v = [] {
-    const char *s = std::getenv("CC3D_WAIT_LIMIT_MS");
-    unsigned long long ms = s ? std::strtoull(s, nullptr, 10) : 2000ull;
-    if (ms == 0) ms = 2000ull;
-    return ms * 1000000ull;
+    const char *s = std::getenv("CC3D_WAIT_LIMIT_US");
+    unsigned long long us = s ? std::strtoull(s, nullptr, 10) : 0ull;
+    if (us == 0) us = 2000000ull;
+    return us * 1000ull;
   }();
   return v;
 }

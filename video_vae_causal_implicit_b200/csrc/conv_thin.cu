@@ -45,6 +45,9 @@ constexpr int kMmaWarp = 4;
 constexpr int kLoadWarp = 5;    // halo TMA producer
 constexpr int kThreads = 320;   // + epilogue warps 6-9
 constexpr int kNH = 3;          // halo ring depth (loader runs ahead)
+// Bound of the drain waits at exit (copies / MMAs already issued finish in
+// microseconds; this only guards against a broken pipeline).
+constexpr unsigned long long kDrainLimitNs = 100ull * 1000000ull;
 
 // Halo geometry of one tile.  Frames are [kt] slabs of `kt_stride`
 // elements; a slab holds (16 + kh - 1) rows of `row` elements; the pixel
@@ -91,8 +94,8 @@ __host__ __device__ inline ThinLayout thin_layout(const ThinArgs &a) {
   L.stage_off = rup(L.bias_off + 4u * a.c_out, 1024u);
   L.bar_off = rup(L.stage_off + kM * L.stage_pitch, 64u);
   // b_full, a_full[2], a_empty[2], acc_full[2], acc_empty[2],
-  // halo_full[kNH], halo_empty[kNH], tmem slot + flag
-  L.total = L.bar_off + 8u * (9 + 2 * kNH) + 16u;
+  // halo_full[kNH], halo_empty[kNH], drain, tmem slot + flags
+  L.total = L.bar_off + 8u * (10 + 2 * kNH) + 16u;
   return L;
 }
 
@@ -167,7 +170,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint64_t *acc_empty = bars + 7;    // [2]
   uint64_t *halo_full = bars + 9;          // [kNH]
   uint64_t *halo_empty = bars + 9 + kNH;   // [kNH]
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9 + 2 * kNH);
+  uint64_t *drain = bars + 9 + 2 * kNH;    // MMA completion before TMEM is freed
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10 + 2 * kNH);
   float *sbias = reinterpret_cast<float *>(smem + L.bias_off);
   volatile uint32_t *go_flag = tmem_slot + 1;
   volatile uint32_t *epi_flag = tmem_slot + 2;
@@ -175,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_tiles = p.n * p.t * p.tiles_h * p.tiles_w;
-  const int hh = kTH + p.kh - 1, hw = kTW + p.kw - 1;
+  const int hh = kTH + p.kh - 1;
   const int K = p.kt * p.kh * p.kw * p.c_in;
   const uint32_t smem_base = smem_u32(smem);
 
@@ -191,6 +195,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&halo_full[i], 1);
       mbar_init(&halo_empty[i], 1);
     }
+    mbar_init(drain, 1);
     fence_mbar_init();
   }
   for (int i = threadIdx.x; i < p.c_out; i += kThreads) sbias[i] = p.bias[i];
@@ -315,10 +320,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       asm volatile("bar.sync 1, %0;" ::"n"(kBuilders) : "memory");  // halo fully read
       if (p.use_tma && threadIdx.x == 0) mbar_arrive(&halo_empty[hb]);
     }
+    // Drain: the weight copy issued by thread 0 lands before the CTA may exit.
+    if (threadIdx.x == 0) mbar_wait_bounded(b_full, 0, kDrainLimitNs, nullptr, 0);
   } else if (warp == kLoadWarp) {
     // ------------------------------ halo loader (TMA) ----------------------------
     if (p.use_tma && lane == 0) {
       const uint32_t box_bytes = static_cast<uint32_t>(G.row) * hh * 2u;
+      uint32_t h_used = 0, h_par = 0;  // ring slots issued, parity of their last issue
       int it = 0;
       for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
         const int hb = it % kNH;
@@ -329,6 +337,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         const Tile tc = thin_tile(tile, p);
         mbar_arrive_expect_tx(&halo_full[hb], box_bytes * p.kt);
+        h_used |= 1u << hb;
+        h_par = (h_par & ~(1u << hb)) | (static_cast<uint32_t>((it / kNH) & 1) << hb);
         const uint32_t dst = smem_base + L.halo_off + hb * L.halo_bytes;
         const int x0 = (tc.w0 - p.pad_w) * p.c_in - G.rem;  // multiple of 8 elements
         for (int kt = 0; kt < p.kt; ++kt) {
@@ -339,6 +349,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                       tc.n);
         }
       }
+      // Drain: every halo load issued here lands before the CTA may exit.
+      for (int i = 0; i < kNH; ++i)
+        if (h_used >> i & 1u)
+          mbar_wait_bounded(&halo_full[i], h_par >> i & 1u, kDrainLimitNs, nullptr, 0);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------ MMA issuer ----------------------------------
@@ -367,6 +381,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         umma_commit(&a_empty[buf]);
         umma_commit(&acc_full[buf]);
       }
+      // Drain: all MMAs issued here are complete before tensor memory is freed.
+      umma_commit(drain);
+      mbar_wait_bounded(drain, 0, kDrainLimitNs, nullptr, 0);
     }
   } else {
     // ------------------------------ epilogue (warps 6-9) -------------------------
@@ -483,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
     tmem_dealloc(tmem_base, p.tmem_cols);
   }
-  if (!ok && threadIdx.x == 0) __nanosleep(100000);
+  (void)ok;
 }
 
 __global__ void repack_thin_kernel(const __nv_bfloat16 *__restrict__ w, __nv_bfloat16 *img,

@@ -52,6 +52,9 @@ constexpr int kTH = 16;   // tile rows -> M = 128
 constexpr int kM = kTW * kTH;
 constexpr int kThreads = 192;
 constexpr int kEpiWarps = 4;
+// Bound of the drain waits at exit (loads / MMAs already issued finish in
+// microseconds; this only guards against a broken pipeline).
+constexpr unsigned long long kDrainLimitNs = 100ull * 1000000ull;
 
 struct SmemLayout {
   uint32_t a_off, a_stage, slab, b_off, b_stage, bar_off, total;
@@ -71,8 +74,8 @@ __host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw
   L.a_off = 0;
   L.b_off = round_up(L.a_off + na * L.a_stage, 1024u);
   L.bar_off = round_up(L.b_off + nb * L.b_stage, 64u);
-  // full_a, empty_a, full_b, empty_b, acc_full[2], acc_empty[2], tmem slot
-  L.total = L.bar_off + 8u * (2 * na + 2 * nb + 4) + 16u;
+  // full_a, empty_a, full_b, empty_b, acc_full[2], acc_empty[2], drain, tmem slot
+  L.total = L.bar_off + 8u * (2 * na + 2 * nb + 5) + 16u;
   return L;
 }
 
@@ -114,7 +117,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *empty_b = full_b + L.nb;
   uint64_t *acc_full = empty_b + L.nb;   // [2]
   uint64_t *acc_empty = acc_full + 2;    // [2]
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+  uint64_t *drain = acc_empty + 2;       // MMA completion before TMEM is freed
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -137,6 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], kEpiWarps);
     }
+    mbar_init(drain, 1);
     fence_mbar_init();
     prefetch_tmap(&map_x);
     if (p.has_cache) prefetch_tmap(&map_cache);
@@ -158,6 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t a_bytes = (KC / 8) * (8u * 2u * halo_w * (kTH + KS - 1));
       int sa = 0, sb = 0;
       uint32_t pa = 0, pb = 0;
+      // stages issued at least once, and the phase parity of their last issue
+      uint32_t a_used = 0, a_par = 0, b_used = 0, b_par = 0;
       for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
         const TileCoord tc0 = decode_tile(tile, p);
         const uint8_t *wsrc =
@@ -169,6 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full_a[sa], a_bytes);
+          a_used |= 1u << sa;
+          a_par = (a_par & ~(1u << sa)) | (pa << sa);
           const int tau = tc0.t + kt - (p.kt - 1);
           const bool from_cache = tau < 0 && p.has_cache;
           const CUtensorMap *map = from_cache ? &map_cache : &map_x;
@@ -186,6 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             mbar_arrive_expect_tx(&full_b[sb], L.b_stage);
+            b_used |= 1u << sb;
+            b_par = (b_par & ~(1u << sb)) | (pb << sb);
             const size_t stage_idx = static_cast<size_t>(kt * KS * KS + ts) * n_cc + cc;
             bulk_load(smem_base + L.b_off + sb * L.b_stage, wsrc + stage_idx * L.b_stage,
                       L.b_stage, &full_b[sb]);
@@ -193,6 +204,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // Drain: every load this thread issued lands before the CTA may exit
+      // (after a timeout elsewhere the consumer may not have waited for it).
+      for (int i = 0; i < L.na; ++i)
+        if (a_used >> i & 1u)
+          mbar_wait_bounded(&full_a[i], a_par >> i & 1u, kDrainLimitNs, nullptr, 0);
+      for (int i = 0; i < L.nb; ++i)
+        if (b_used >> i & 1u)
+          mbar_wait_bounded(&full_b[i], b_par >> i & 1u, kDrainLimitNs, nullptr, 0);
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ----------------------------------
@@ -248,6 +267,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma_commit(&acc_full[buf]);  // accumulator ready for the epilogue
       }
+      // Drain: all MMAs issued here are complete before tensor memory is freed.
+      umma_commit(drain);
+      mbar_wait_bounded(drain, 0, kDrainLimitNs, nullptr, 0);
     }
   } else {
     // ------------------------------ epilogue ------------------------------------
@@ -343,11 +365,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, p.tmem_cols);
-  }
-  if (!ok && threadIdx.x == 0) {
-    // A wait ran out: give copies already issued time to land before the
-    // CTA's shared memory is handed to another block.
-    __nanosleep(100000);
   }
 }
 
