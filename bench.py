@@ -323,10 +323,42 @@ def main():
     blk_bytes = 7 * act_bytes  # x r, a0 w, a0 r, a1 w, a1 r, x r (residual), y w
     roof_ms = max(blk_flop / (peaks["bf16_tflops_sustained"] * 1e12),
                   blk_bytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    # the block's three kernels, timed one by one through the public API
+    dv = {k: bc[k].to(dev) for k in ("w1", "b1", "g1", "w2", "b2", "g2")}
+    conv1 = cc3d.Plan(dv["w1"], dv["b1"], h=Hb, w=Wb, max_t=Tb, epi=cc3d.EPI_BIAS_RMS_SILU,
+                      gamma=dv["g2"])
+    conv2 = cc3d.Plan(dv["w2"], dv["b2"], h=Hb, w=Wb, max_t=Tb, epi=cc3d.EPI_BIAS_RESIDUAL)
+    a0 = torch.empty_like(xb)
+    a1 = torch.empty_like(xb)
+    parts = {"rmsnorm_silu": lambda: cc3d.rms_silu(xb, dv["g1"], a0),
+             "conv1_rms_silu_epilogue": lambda: conv1.forward(a0, a1),
+             "conv2_residual_epilogue": lambda: conv2.forward(a1, yb, residual=xb)}
+    breakdown = {}
+    for name, fn in parts.items():
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        ea = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        eb = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for k in range(args.steps):
+            ea[k].record(stream)
+            fn()
+            eb[k].record(stream)
+        torch.cuda.synchronize()
+        pms = statistics.median(a.elapsed_time(b) for a, b in zip(ea, eb))
+        if name == "rmsnorm_silu":
+            gbs = 2 * act_bytes / pms / 1e6
+            breakdown[name] = {"ms": pms, "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"]}
+        else:
+            tf = conv_flop(1, cb, cb, Tb, Hb, Wb) / pms / 1e9
+            breakdown[name] = {"ms": pms, "tflops": tf, "frac": tf / peaks["bf16_tflops"]}
+    cc3d.sync_status()
     resblock = {"workload": "Wan residual block bf16 192ch x[1,192,9,240,416]",
                 "ms": blk_ms, "tflops": blk_flop / (blk_ms * 1e-3) / 1e12,
                 "roofline_ms": roof_ms, "frac": roof_ms / blk_ms,
-                "peak_basis": "sustained bf16 (" + peaks["source"] + ")"}
+                "peak_basis": "sustained bf16 (" + peaks["source"] + ")",
+                "kernels": breakdown}
+    del conv1, conv2, a0, a1
     del blk, xb, yb
 
     sweep = run_sweep(args, dev, stream, peaks, flush_l2) if args.sweep else None

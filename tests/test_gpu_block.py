@@ -11,7 +11,7 @@ from video_vae_causal_implicit_b200 import cc3d, synth
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("c", [8, 96, 192, 384, 1024])
+@pytest.mark.parametrize("c", [8, 40, 96, 192, 200, 384, 1024])
 def test_rmsnorm_silu_matches_oracle(c):
     x = synth.normal((1, c, 3, 7, 9), 21)
     g = synth.uniform((c,), 0.5, 1.5, 22)

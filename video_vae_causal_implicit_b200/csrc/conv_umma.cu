@@ -298,62 +298,93 @@ __global__ void __launch_bounds__(kThreads, 1)
       const __nv_bfloat16 *rrow = p.residual ? p.residual + pix * p.c_out + n0 : nullptr;
       float inv = 1.0f;
       if (p.epi == 2) {
+        // pass 1: sum of squares of the biased row (three loads in flight)
         float ss = 0.f;
-        for (int j = 0; j < p.nt; j += 16) {
-          float v[16];
+        for (int j0 = 0; j0 < p.nt; j0 += 48) {
+          const int nld = (p.nt - j0) >= 48 ? 3 : (p.nt - j0) / 16;
+          uint32_t raw[48];
           __syncwarp();
-          tmem_ld16(taddr + j, v);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float hv = v[i] + p.bias[n0 + j + i];
-            ss = fmaf(hv, hv, ss);
+          for (int u = 0; u < 3; ++u)
+            if (u < nld) tmem_ld16_nowait(taddr + j0 + 16 * u, raw + 16 * u);
+          tmem_wait_ld();
+          tmem_regs_after_wait<48>(raw);
+#pragma unroll
+          for (int u = 0; u < 3; ++u) {
+            if (u >= nld) continue;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float hv = __uint_as_float(raw[16 * u + i]) + p.bias[n0 + j0 + 16 * u + i];
+              ss = fmaf(hv, hv, ss);
+            }
           }
         }
         inv = sqrtf(static_cast<float>(p.c_out)) / fmaxf(sqrtf(ss), 1e-12f);
       }
-      for (int j = 0; j < p.nt; j += 16) {
-        float v[16];
+      // pass 2: bias (+ residual | RMS scale + SiLU) -> bf16 -> global
+      for (int j0 = 0; j0 < p.nt; j0 += 48) {
+        const int nld = (p.nt - j0) >= 48 ? 3 : (p.nt - j0) / 16;
+        uint4 res[6];
+        if (p.epi == 1 && valid) {
+          // residual loads first, so their latency overlaps the TMEM reads
+#pragma unroll
+          for (int u = 0; u < 3; ++u)
+            if (u < nld) {
+              const uint4 *rr = reinterpret_cast<const uint4 *>(rrow + j0 + 16 * u);
+              res[2 * u] = rr[0];
+              res[2 * u + 1] = rr[1];
+            }
+        }
+        uint32_t raw[48];
         __syncwarp();
-        tmem_ld16(taddr + j, v);
-        if (j + 16 >= p.nt) {
+#pragma unroll
+        for (int u = 0; u < 3; ++u)
+          if (u < nld) tmem_ld16_nowait(taddr + j0 + 16 * u, raw + 16 * u);
+        tmem_wait_ld();
+        tmem_regs_after_wait<48>(raw);
+        if (j0 + 48 >= p.nt) {
           // last read of this accumulator: hand the buffer back to the MMA warp
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] += p.bias[n0 + j + i];
-        if (p.epi == 1 && valid) {
-          const uint4 *rr = reinterpret_cast<const uint4 *>(rrow + j);
-          uint4 r0 = rr[0], r1 = rr[1];
-          const __nv_bfloat16 *rb0 = reinterpret_cast<const __nv_bfloat16 *>(&r0);
-          const __nv_bfloat16 *rb1 = reinterpret_cast<const __nv_bfloat16 *>(&r1);
+        for (int u = 0; u < 3; ++u) {
+          if (u >= nld) continue;
+          const int j = j0 + 16 * u;
+          float v[16];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            v[i] += __bfloat162float(rb0[i]);
-            v[8 + i] += __bfloat162float(rb1[i]);
-          }
-        } else if (p.epi == 2) {
+          for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(raw[16 * u + i]) + p.bias[n0 + j + i];
+          if (p.epi == 1 && valid) {
+            const __nv_bfloat16 *rb0 = reinterpret_cast<const __nv_bfloat16 *>(&res[2 * u]);
+            const __nv_bfloat16 *rb1 = reinterpret_cast<const __nv_bfloat16 *>(&res[2 * u + 1]);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float a = v[i] * inv * p.gamma[n0 + j + i];
-            if (p.beta) a += p.beta[n0 + j + i];
-            v[i] = a / (1.0f + __expf(-a));
+            for (int i = 0; i < 8; ++i) {
+              v[i] += __bfloat162float(rb0[i]);
+              v[8 + i] += __bfloat162float(rb1[i]);
+            }
+          } else if (p.epi == 2) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float a = v[i] * inv * p.gamma[n0 + j + i];
+              if (p.beta) a += p.beta[n0 + j + i];
+              v[i] = silu_fast(a);
+            }
           }
-        }
-        if (valid) {
-          uint4 o0, o1;
-          o0.x = pack_bf16x2(v[0], v[1]);
-          o0.y = pack_bf16x2(v[2], v[3]);
-          o0.z = pack_bf16x2(v[4], v[5]);
-          o0.w = pack_bf16x2(v[6], v[7]);
-          o1.x = pack_bf16x2(v[8], v[9]);
-          o1.y = pack_bf16x2(v[10], v[11]);
-          o1.z = pack_bf16x2(v[12], v[13]);
-          o1.w = pack_bf16x2(v[14], v[15]);
-          uint4 *dst = reinterpret_cast<uint4 *>(yrow + j);
-          dst[0] = o0;
-          dst[1] = o1;
+          if (valid) {
+            uint4 o0, o1;
+            o0.x = pack_bf16x2(v[0], v[1]);
+            o0.y = pack_bf16x2(v[2], v[3]);
+            o0.z = pack_bf16x2(v[4], v[5]);
+            o0.w = pack_bf16x2(v[6], v[7]);
+            o1.x = pack_bf16x2(v[8], v[9]);
+            o1.y = pack_bf16x2(v[10], v[11]);
+            o1.z = pack_bf16x2(v[12], v[13]);
+            o1.w = pack_bf16x2(v[14], v[15]);
+            uint4 *dst = reinterpret_cast<uint4 *>(yrow + j);
+            dst[0] = o0;
+            dst[1] = o1;
+          }
         }
       }
     }

@@ -11,6 +11,7 @@
 #include <cstdint>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace cc3d {
 
@@ -75,38 +76,44 @@ __global__ void copy_frames_kernel(const uint8_t *__restrict__ cache_in,
   }
 }
 
-// A warp normalises VPW voxels per iteration; lane l owns channel groups
-// l, l+32, ... of 8 channels (16 bytes) of each.  All loads of the VPW
-// voxels are issued before any reduction so enough bytes are in flight to
-// keep HBM busy.  The sum of squares is reduced with a fixed xor butterfly,
-// so the result does not depend on scheduling.
-template <int CPL, int VPW>
-__global__ void rmsnorm_silu_kernel(const __nv_bfloat16 *__restrict__ x,
-                                    const float *__restrict__ gamma,
-                                    const float *__restrict__ beta, long long voxels, int c,
-                                    __nv_bfloat16 *__restrict__ y) {
+// Lane-mapped RMS_norm + SiLU for channel counts whose 8-channel groups
+// split evenly over a power-of-two number of lanes: LPV lanes share a voxel,
+// each lane owning GPL groups (GPL = c / 8 / LPV, e.g. C = 192: 8 lanes x 3
+// groups, four voxels per warp).  A warp's loads cover 32 * GPL consecutive
+// 16-byte chunks (fully coalesced, every lane busy); UNR warp passes are
+// loaded before any is used.  The sum of squares is reduced with a fixed
+// xor butterfly over the LPV lanes, so the result does not depend on
+// scheduling.
+template <int GPL, int UNR>
+__global__ void __launch_bounds__(256, 2)
+    rmsnorm_silu_lanes_kernel(const __nv_bfloat16 *__restrict__ x,
+                              const float *__restrict__ gamma, const float *__restrict__ beta,
+                              long long voxels, int c, int lpv,
+                              __nv_bfloat16 *__restrict__ y) {
   const int lane = threadIdx.x % 32;
+  const int vpw = 32 / lpv;                 // voxels per warp pass
+  const int sub = lane % lpv, vloc = lane / lpv;
   const long long warp0 = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) / 32;
   const long long nwarps = static_cast<long long>(gridDim.x) * blockDim.x / 32;
-  const int groups = c / 8;
   const float scale = sqrtf(static_cast<float>(c));
-  for (long long v0 = warp0 * VPW; v0 < voxels; v0 += nwarps * VPW) {
-    uint4 raw[VPW][CPL];
+  const int groups = c / 8;
+  for (long long vb = warp0 * vpw * UNR; vb < voxels; vb += nwarps * vpw * UNR) {
+    uint4 raw[UNR][GPL];
 #pragma unroll
-    for (int u = 0; u < VPW; ++u)
+    for (int u = 0; u < UNR; ++u) {
+      const long long v = vb + u * vpw + vloc;
 #pragma unroll
-      for (int k = 0; k < CPL; ++k) {
-        const int g = lane + 32 * k;
-        raw[u][k] = make_uint4(0, 0, 0, 0);
-        if (v0 + u < voxels && g < groups)
-          raw[u][k] = __ldcs(reinterpret_cast<const uint4 *>(x + (v0 + u) * c) + g);
-      }
-    float inv[VPW];
+      for (int k = 0; k < GPL; ++k)
+        raw[u][k] = v < voxels
+                        ? __ldcs(reinterpret_cast<const uint4 *>(x + v * c) + sub + k * lpv)
+                        : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-    for (int u = 0; u < VPW; ++u) {
+    for (int u = 0; u < UNR; ++u) {
+      const long long v = vb + u * vpw + vloc;
       float ss = 0.f;
 #pragma unroll
-      for (int k = 0; k < CPL; ++k) {
+      for (int k = 0; k < GPL; ++k) {
         const __nv_bfloat16 *b = reinterpret_cast<const __nv_bfloat16 *>(&raw[u][k]);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -114,33 +121,108 @@ __global__ void rmsnorm_silu_kernel(const __nv_bfloat16 *__restrict__ x,
           ss = fmaf(f, f, ss);
         }
       }
+      for (int o = lpv / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float inv = scale / fmaxf(sqrtf(ss), 1e-12f);
+      if (v >= voxels) continue;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      inv[u] = scale / fmaxf(sqrtf(ss), 1e-12f);
+      for (int k = 0; k < GPL; ++k) {
+        const int g = sub + k * lpv;
+        const float4 g0 = __ldg(reinterpret_cast<const float4 *>(gamma + g * 8));
+        const float4 g1 = __ldg(reinterpret_cast<const float4 *>(gamma + g * 8) + 1);
+        const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        const __nv_bfloat16 *b = reinterpret_cast<const __nv_bfloat16 *>(&raw[u][k]);
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float a = __bfloat162float(b[e]) * inv * gm[e];
+          if (beta) a += __ldg(beta + g * 8 + e);
+          o[e] = silu_fast(a);
+        }
+        uint4 w;
+        w.x = pack2(o[0], o[1]);
+        w.y = pack2(o[2], o[3]);
+        w.z = pack2(o[4], o[5]);
+        w.w = pack2(o[6], o[7]);
+        __stcs(reinterpret_cast<uint4 *>(y + v * c) + g, w);
+      }
+    }
+    (void)groups;
+  }
+}
+
+// A CTA normalises a contiguous run of voxels: its 256 threads load the
+// run's consecutive 16-byte chunks (8 channels each, CPT per thread, all
+// issued before any use), write each chunk's sum of squares to shared
+// memory, then one thread per voxel adds its chunks' partial sums in
+// channel order (a fixed order: the result does not depend on scheduling),
+// and every thread scales, applies SiLU and stores its chunks.
+template <int CPT>
+__global__ void __launch_bounds__(256)
+    rmsnorm_silu_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ gamma,
+                        const float *__restrict__ beta, long long voxels, int c,
+                        __nv_bfloat16 *__restrict__ y) {
+  __shared__ float partial[256 * CPT];
+  __shared__ float inv_s[256 * CPT];
+  const int groups = c / 8;
+  const int vpb = (256 * CPT) / groups;  // voxels per CTA pass
+  const float scale = sqrtf(static_cast<float>(c));
+  for (long long v0 = static_cast<long long>(blockIdx.x) * vpb; v0 < voxels;
+       v0 += static_cast<long long>(gridDim.x) * vpb) {
+    const int nv = static_cast<int>(voxels - v0 < vpb ? voxels - v0 : vpb);
+    const int nch = nv * groups;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + v0 * c);
+    uint4 raw[CPT];
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) {
+      const int idx = threadIdx.x + 256 * k;
+      raw[k] = idx < nch ? __ldcs(src + idx) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int u = 0; u < VPW; ++u)
+    for (int k = 0; k < CPT; ++k) {
+      const int idx = threadIdx.x + 256 * k;
+      const __nv_bfloat16 *b = reinterpret_cast<const __nv_bfloat16 *>(&raw[k]);
+      float ss = 0.f;
 #pragma unroll
-      for (int k = 0; k < CPL; ++k) {
-        const int g = lane + 32 * k;
-        if (v0 + u < voxels && g < groups) {
-          const __nv_bfloat16 *b = reinterpret_cast<const __nv_bfloat16 *>(&raw[u][k]);
-          float o[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int ch = g * 8 + e;
-            float a = __bfloat162float(b[e]) * inv[u] * __ldg(gamma + ch);
-            if (beta) a += __ldg(beta + ch);
-            o[e] = a / (1.0f + __expf(-a));
-          }
-          uint4 w;
-          w.x = pack2(o[0], o[1]);
-          w.y = pack2(o[2], o[3]);
-          w.z = pack2(o[4], o[5]);
-          w.w = pack2(o[6], o[7]);
-          __stcs(reinterpret_cast<uint4 *>(y + (v0 + u) * c) + g, w);
-        }
+      for (int e = 0; e < 8; ++e) {
+        const float f = __bfloat162float(b[e]);
+        ss = fmaf(f, f, ss);
       }
+      if (idx < nch) partial[idx] = ss;
+    }
+    __syncthreads();
+    for (int v = threadIdx.x; v < nv; v += 256) {
+      float ss = 0.f;
+      for (int g = 0; g < groups; ++g) ss += partial[v * groups + g];
+      inv_s[v] = scale / fmaxf(sqrtf(ss), 1e-12f);
+    }
+    __syncthreads();
+    uint4 *dst = reinterpret_cast<uint4 *>(y + v0 * c);
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) {
+      const int idx = threadIdx.x + 256 * k;
+      if (idx < nch) {
+        const int v = idx / groups, g = idx - (idx / groups) * groups;
+        const float inv = inv_s[v];
+        const float4 g0 = __ldg(reinterpret_cast<const float4 *>(gamma + g * 8));
+        const float4 g1 = __ldg(reinterpret_cast<const float4 *>(gamma + g * 8) + 1);
+        const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        const __nv_bfloat16 *b = reinterpret_cast<const __nv_bfloat16 *>(&raw[k]);
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float a = __bfloat162float(b[e]) * inv * gm[e];
+          if (beta) a += __ldg(beta + g * 8 + e);
+          o[e] = silu_fast(a);
+        }
+        uint4 w;
+        w.x = pack2(o[0], o[1]);
+        w.y = pack2(o[2], o[3]);
+        w.z = pack2(o[4], o[5]);
+        w.w = pack2(o[6], o[7]);
+        __stcs(dst + idx, w);
+      }
+    }
+    __syncthreads();  // partial / inv_s are rewritten by the next pass
   }
 }
 
@@ -228,20 +310,34 @@ cudaError_t launch_cache_update(const void *cache_in, const void *src, void *cac
 cudaError_t launch_rmsnorm_silu(const __nv_bfloat16 *x, const float *gamma, const float *beta,
                                 long long voxels, int c, __nv_bfloat16 *y, cudaStream_t stream) {
   const int groups = c / 8;
-  const int cpl = (groups + 31) / 32;
-  constexpr int kVpw = 4;
-  const int block = 256;
-  long long warps = (voxels + kVpw - 1) / kVpw;
-  long long g = (warps * 32 + block - 1) / block;
-  if (g > 148LL * 16) g = 148LL * 16;
-  if (g < 1) g = 1;
-  const int grid = static_cast<int>(g);
-  switch (cpl) {
-    case 1: rmsnorm_silu_kernel<1, kVpw><<<grid, block, 0, stream>>>(x, gamma, beta, voxels, c, y); break;
-    case 2: rmsnorm_silu_kernel<2, kVpw><<<grid, block, 0, stream>>>(x, gamma, beta, voxels, c, y); break;
-    case 3: rmsnorm_silu_kernel<3, kVpw><<<grid, block, 0, stream>>>(x, gamma, beta, voxels, c, y); break;
-    case 4: rmsnorm_silu_kernel<4, kVpw><<<grid, block, 0, stream>>>(x, gamma, beta, voxels, c, y); break;
-    default: return cudaErrorInvalidValue;
+  if (groups < 1) return cudaErrorInvalidValue;
+  // lanes per voxel: the largest power of two (<= 32) dividing the groups
+  int lpv = 1;
+  while (lpv < 32 && groups % (lpv * 2) == 0) lpv *= 2;
+  const int gpl = groups / lpv;
+  if (gpl <= 4) {
+    constexpr int kUnr = 2;
+    const long long per_warp = static_cast<long long>(32 / lpv) * kUnr;
+    long long warps = (voxels + per_warp - 1) / per_warp;
+    long long g = (warps * 32 + 255) / 256;
+    if (g > 148LL * 8) g = 148LL * 8;
+    if (g < 1) g = 1;
+    const int grid = static_cast<int>(g);
+    switch (gpl) {
+      case 1: rmsnorm_silu_lanes_kernel<1, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y); break;
+      case 2: rmsnorm_silu_lanes_kernel<2, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y); break;
+      case 3: rmsnorm_silu_lanes_kernel<3, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y); break;
+      default: rmsnorm_silu_lanes_kernel<4, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y); break;
+    }
+  } else {
+    constexpr int kCpt = 12;  // 16-byte chunks per thread and pass
+    if (groups > 256 * kCpt) return cudaErrorInvalidValue;
+    const int vpb = (256 * kCpt) / groups;
+    long long g = (voxels + vpb - 1) / vpb;
+    if (g > 148LL * 8) g = 148LL * 8;
+    if (g < 1) g = 1;
+    rmsnorm_silu_kernel<kCpt><<<static_cast<int>(g), 256, 0, stream>>>(x, gamma, beta, voxels,
+                                                                       c, y);
   }
   count_launch();
   return cudaGetLastError();
