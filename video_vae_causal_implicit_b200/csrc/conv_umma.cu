@@ -14,13 +14,18 @@
 // A operand: for each (kt, channel chunk) one TMA box brings the input
 // halo of the tile -- (TH + kh - 1) x (TW + kw - 1) pixels x KC channels --
 // from the current chunk x (frame tau = t + kt - (kt_size - 1) >= 0) or the
-// frame cache (tau < 0).  Spatial padding and absent caches are TMA
-// out-of-bounds zero fill, so no padded copy exists anywhere.  The halo is
-// stored as "interleaved" core matrices without swizzle,
+// frame cache (tau < 0).  Spatial padding is TMA out-of-bounds zero fill,
+// and a frame before the chunk with no cache (all zeros) is skipped: its
+// stage is neither loaded nor multiplied.  No padded copy exists anywhere.  For 64-channel
+// chunks the halo is one TMA box with the 128-byte swizzle,
+//     [halo rows][halo cols][64 channels = 128 bytes],
+// and the A matrix of spatial tap (kh, kw) is the same buffer seen from a
+// start address shifted by (kh * halo_cols + kw) whole 128-byte rows: the
+// tensor core un-swizzles by absolute shared-memory address, so a row-shifted
+// view reads correctly (checked on B200).  One load serves all kh * kw taps.
+// 32- and 96-channel chunks use no-swizzle core matrices instead,
 //     [KC/8 slabs][halo rows][halo cols][8 channels],
-// so the A matrix of spatial tap (kh, kw) is the same buffer seen from a
-// start address shifted by (kh * halo_cols + kw) * 16 bytes: one load
-// serves all kh * kw taps.
+// loaded as one 8-channel box per slab, where a pixel shift is 16 bytes.
 //
 // B operand: the weights, re-tiled at plan time into the exact shared
 // memory image of each (N tile, tap, channel chunk) stage
@@ -171,6 +176,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             p.wimg + static_cast<size_t>(tc0.ntile) * p.kt * KS * KS * n_cc * L.b_stage;
         for (int ia = 0; ia < n_a && ok; ++ia) {
           const int kt = ia / n_cc, cc = ia % n_cc;
+          // A frame before the chunk with no cache is all zeros: its stage
+          // (and its taps' weights) is skipped here and by the MMA issuer.
+          if (tc0.t + kt - (p.kt - 1) < 0 && !p.has_cache) continue;
           if (!mbar_wait_bounded(&empty_a[sa], pa ^ 1, p.wait_limit_ns, p.status, 1)) {
             ok = false;
             break;
@@ -179,9 +187,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           a_used |= 1u << sa;
           a_par = (a_par & ~(1u << sa)) | (pa << sa);
           const int tau = tc0.t + kt - (p.kt - 1);
-          const bool from_cache = tau < 0 && p.has_cache;
+          const bool from_cache = tau < 0;  // (zero frames were skipped above)
           const CUtensorMap *map = from_cache ? &map_cache : &map_x;
-          const int tcoord = from_cache ? tau + (p.kt - 1) : tau;  // negative: zero fill
+          const int tcoord = from_cache ? tau + (p.kt - 1) : tau;
           const uint32_t dst = smem_base + L.a_off + sa * L.a_stage;
 #pragma unroll
           for (int s = 0; s < KC / 8; ++s)
@@ -221,9 +229,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t b_lbo = static_cast<uint32_t>(p.nt) * 16u;
       // Descriptors of stage 0; other stages, taps and K steps only move the
       // start address (low 14 bits, 16-byte units), so they are additions.
+      // A 16-element K step is two 8-channel slabs (A) or two core-matrix
+      // columns (B) further on; a halo pixel is 16 bytes.
       const uint64_t adesc0 = smem_desc_noswizzle(smem_base + L.a_off, L.slab, a_sbo);
       const uint64_t bdesc0 = smem_desc_noswizzle(smem_base + L.b_off, b_lbo, 128u);
-      const uint32_t slab16 = L.slab >> 4, blbo16 = b_lbo >> 4;
+      const uint32_t astep16 = 2u * (L.slab >> 4);
+      const uint32_t bstep16 = 2u * (b_lbo >> 4);
+      const uint32_t pix16 = 1u;
       int sa = 0, sb = 0;
       uint32_t pa = 0, pb = 0;
       int it = 0;
@@ -237,8 +249,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * p.nt;
+        const TileCoord tcm = decode_tile(tile, p);
         uint32_t accumulate = 0;
         for (int ia = 0; ia < n_a && ok; ++ia) {
+          // the same zero-frame stages the producer skipped; adding their
+          // exact zeros would not change the accumulator
+          if (tcm.t + ia / n_cc - (p.kt - 1) < 0 && !p.has_cache) continue;
           if (!mbar_wait_bounded(&full_a[sa], pa, p.wait_limit_ns, p.status, 3)) {
             ok = false;
             break;
@@ -252,11 +268,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            const uint64_t a_tap = a_st + ((ts / KS) * halo_w + (ts % KS));
+            const uint64_t a_tap = a_st + ((ts / KS) * halo_w + (ts % KS)) * pix16;
             const uint64_t b_st = bdesc0 + ((sb * L.b_stage) >> 4);
 #pragma unroll
             for (int j = 0; j < KC / 16; ++j) {
-              umma_bf16(d_tmem, a_tap + 2 * j * slab16, b_st + 2 * j * blbo16, idesc, accumulate);
+              umma_bf16(d_tmem, a_tap + j * astep16, b_st + j * bstep16, idesc, accumulate);
               accumulate = 1;
             }
             umma_commit(&empty_b[sb]);  // frees the B stage when these MMAs finish

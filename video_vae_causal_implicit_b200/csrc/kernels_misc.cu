@@ -46,11 +46,53 @@ __global__ void repack_umma_kernel(const __nv_bfloat16 *__restrict__ w, __nv_bfl
   }
 }
 
-__global__ void copy_frames_kernel(const uint8_t *__restrict__ cache_in,
-                                   const uint8_t *__restrict__ src, uint8_t *__restrict__ out,
-                                   int n, int t, int frames, size_t frame_bytes, int vec16) {
-  // out[b][i] = concat(cache_in[b] (frames), src[b] (t))[t + i], i < frames
-  const size_t per_frame = vec16 ? frame_bytes / 16 : frame_bytes / 2;
+// out[b][i] = concat(cache_in[b] (frames), src[b] (t))[t + i], i < frames.
+// 16-byte path: each thread moves U chunks per pass, all loads issued before
+// the stores, so enough bytes are in flight to stream at HBM speed.
+template <int U>
+__global__ void copy_frames16_kernel(const uint8_t *__restrict__ cache_in,
+                                     const uint8_t *__restrict__ src, uint8_t *__restrict__ out,
+                                     int n, int t, int frames, size_t frame_bytes) {
+  const size_t per_frame = frame_bytes / 16;
+  const size_t total = static_cast<size_t>(n) * frames * per_frame;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t k0 = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; k0 < total;
+       k0 += stride * U) {
+    uint4 v[U];
+    uint4 *to[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const size_t k = k0 + u * stride;
+      to[u] = nullptr;
+      v[u] = make_uint4(0, 0, 0, 0);
+      if (k < total) {
+        const size_t off = k % per_frame;
+        const size_t fi = k / per_frame;
+        const int i = static_cast<int>(fi % frames);
+        const int b = static_cast<int>(fi / frames);
+        const int ci = t + i;  // index into concat
+        const uint8_t *from = nullptr;
+        if (ci < frames) {
+          if (cache_in) from = cache_in + (static_cast<size_t>(b) * frames + ci) * frame_bytes;
+        } else {
+          from = src + (static_cast<size_t>(b) * t + (ci - frames)) * frame_bytes;
+        }
+        if (from) v[u] = __ldcs(reinterpret_cast<const uint4 *>(from) + off);
+        to[u] = reinterpret_cast<uint4 *>(out + (static_cast<size_t>(b) * frames + i) * frame_bytes) +
+                off;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (to[u]) *to[u] = v[u];
+  }
+}
+
+// 2-byte path for frames whose size or start is not 16-byte aligned.
+__global__ void copy_frames2_kernel(const uint8_t *__restrict__ cache_in,
+                                    const uint8_t *__restrict__ src, uint8_t *__restrict__ out,
+                                    int n, int t, int frames, size_t frame_bytes) {
+  const size_t per_frame = frame_bytes / 2;
   const size_t total = static_cast<size_t>(n) * frames * per_frame;
   for (size_t k = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; k < total;
        k += static_cast<size_t>(gridDim.x) * blockDim.x) {
@@ -58,7 +100,7 @@ __global__ void copy_frames_kernel(const uint8_t *__restrict__ cache_in,
     const size_t fi = k / per_frame;
     const int i = static_cast<int>(fi % frames);
     const int b = static_cast<int>(fi / frames);
-    const int ci = t + i;  // index into concat
+    const int ci = t + i;
     const uint8_t *from = nullptr;
     if (ci < frames) {
       if (cache_in) from = cache_in + (static_cast<size_t>(b) * frames + ci) * frame_bytes;
@@ -66,13 +108,8 @@ __global__ void copy_frames_kernel(const uint8_t *__restrict__ cache_in,
       from = src + (static_cast<size_t>(b) * t + (ci - frames)) * frame_bytes;
     }
     uint8_t *to = out + (static_cast<size_t>(b) * frames + i) * frame_bytes;
-    if (vec16) {
-      uint4 v = from ? reinterpret_cast<const uint4 *>(from)[off] : make_uint4(0, 0, 0, 0);
-      reinterpret_cast<uint4 *>(to)[off] = v;
-    } else {
-      uint16_t v = from ? reinterpret_cast<const uint16_t *>(from)[off] : 0;
-      reinterpret_cast<uint16_t *>(to)[off] = v;
-    }
+    const uint16_t v = from ? reinterpret_cast<const uint16_t *>(from)[off] : 0;
+    reinterpret_cast<uint16_t *>(to)[off] = v;
   }
 }
 
@@ -293,16 +330,25 @@ cudaError_t launch_repack_umma(const __nv_bfloat16 *w, uint8_t *img, int c_out, 
 cudaError_t launch_cache_update(const void *cache_in, const void *src, void *cache_out, int n,
                                 int t, int frames, size_t frame_bytes, cudaStream_t stream) {
   if (frames <= 0) return cudaSuccess;
-  const int vec16 = (frame_bytes % 16 == 0 && (reinterpret_cast<uintptr_t>(src) % 16) == 0 &&
+  const bool vec16 = frame_bytes % 16 == 0 && (reinterpret_cast<uintptr_t>(src) % 16) == 0 &&
                      (reinterpret_cast<uintptr_t>(cache_out) % 16) == 0 &&
-                     (reinterpret_cast<uintptr_t>(cache_in) % 16) == 0)
-                        ? 1
-                        : 0;
-  const long long work =
-      static_cast<long long>(n) * frames * (vec16 ? frame_bytes / 16 : frame_bytes / 2);
-  copy_frames_kernel<<<grid_for(work, 256), 256, 0, stream>>>(
-      static_cast<const uint8_t *>(cache_in), static_cast<const uint8_t *>(src),
-      static_cast<uint8_t *>(cache_out), n, t, frames, frame_bytes, vec16);
+                     (reinterpret_cast<uintptr_t>(cache_in) % 16) == 0;
+  const auto *ci = static_cast<const uint8_t *>(cache_in);
+  const auto *sr = static_cast<const uint8_t *>(src);
+  auto *co = static_cast<uint8_t *>(cache_out);
+  if (vec16) {
+    constexpr int kU = 4;
+    const long long work = static_cast<long long>(n) * frames * (frame_bytes / 16);
+    long long g = (work / kU + 255) / 256;
+    if (g > 148LL * 8) g = 148LL * 8;
+    if (g < 1) g = 1;
+    copy_frames16_kernel<kU><<<static_cast<int>(g), 256, 0, stream>>>(ci, sr, co, n, t, frames,
+                                                                        frame_bytes);
+  } else {
+    const long long work = static_cast<long long>(n) * frames * (frame_bytes / 2);
+    copy_frames2_kernel<<<grid_for(work, 256), 256, 0, stream>>>(ci, sr, co, n, t, frames,
+                                                                 frame_bytes);
+  }
   count_launch();
   return cudaGetLastError();
 }
