@@ -117,6 +117,9 @@ typedef struct {
   int tile_h, tile_w;      /* output tile (rows x cols of one frame)         */
   int n_tile;              /* output channels per CTA                        */
   int k_chunk;             /* input channels per pipeline stage              */
+  int k_split;             /* CTAs sharing one output tile, one temporal tap
+                              each, summed in one of them: 1, or kt for
+                              frames too small to occupy the GPU            */
 } cc3d_stats;
 
 typedef struct cc3d_plan cc3d_plan;

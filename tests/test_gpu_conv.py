@@ -108,6 +108,7 @@ def test_config2_whole_and_streaming_bitwise_and_oracle():
     both against the full fp64 oracle."""
     case = synth.conv_case(384, 384, 5, 30, 52)
     plan, x, y = run_conv(case)
+    assert plan.stats().k_split == 3  # 28 tiles a frame: one temporal tap per CTA
     ys = _stream_chunks(plan, x, 1, 384)
     assert torch.equal(ys.cpu(), y.cpu()), "streaming != whole sequence"
     ref = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], _bias64(case["b"]))

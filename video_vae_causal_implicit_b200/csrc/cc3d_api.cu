@@ -88,19 +88,22 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 }
 
 // 5-D bf16 tensor map over an NDHWC buffer: dims (C, W, H, T, N), a box of
-// 8 channels x box_w x box_h x 1 x 1, no swizzle, zero fill out of bounds.
+// box_c channels x box_w x box_h x 1 x 1, zero fill out of bounds; 64-channel
+// boxes (128-byte pixel rows) land 128-byte swizzled, 8-channel boxes plain.
 bool encode_act_map(CUtensorMap *m, const void *base, int c, int w, int h, int t, int n,
-                    int box_w, int box_h) {
+                    int box_w, int box_h, int box_c) {
+  if (box_c != 8 && box_c != 64) return false;
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[5] = {(cuuint64_t)c, (cuuint64_t)w, (cuuint64_t)h, (cuuint64_t)t,
                         (cuuint64_t)n};
   cuuint64_t strides[4] = {(cuuint64_t)c * 2, (cuuint64_t)c * 2 * w, (cuuint64_t)c * 2 * w * h,
                            (cuuint64_t)c * 2 * w * h * t};
-  cuuint32_t box[5] = {8, (cuuint32_t)box_w, (cuuint32_t)box_h, 1, 1};
+  cuuint32_t box[5] = {(cuuint32_t)box_c, (cuuint32_t)box_w, (cuuint32_t)box_h, 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  box_c == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -146,8 +149,8 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 int *device_status_word() { return status_ptr(); }
 
 bool encode_activation_map(CUtensorMap *m, const void *base, int c, int w, int h, int t, int n,
-                           int box_w, int box_h) {
-  return encode_act_map(m, base, c, w, h, t, n, box_w, box_h);
+                           int box_w, int box_h, int box_c) {
+  return encode_act_map(m, base, c, w, h, t, n, box_w, box_h, box_c);
 }
 
 }  // namespace cc3d
@@ -159,7 +162,7 @@ struct cc3d_plan {
   int variant;
   int device;
   // UMMA
-  int kc, nt, n_ntiles, na, nb, tmem_cols, sm_count, ctas_per_sm;
+  int kc, nt, n_ntiles, na, nb, tmem_cols, sm_count, ctas_per_sm, sub, nbuf, split, max_clusters;
   uint8_t *wimg;
   // fp32 / thin
   void *wraw;
@@ -278,6 +281,7 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
   cudaGetDevice(&p->device);
   std::memset(&p->st, 0, sizeof(p->st));
   p->st.variant = variant;
+  p->st.k_split = 1;
   const int taps = desc->kt * desc->kh * desc->kw;
   cudaError_t e = cudaSuccess;
   if ((s = copy_vec(&p->bias, desc->bias, desc->c_out, true)) != CC3D_OK) goto fail;
@@ -331,52 +335,33 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
     e = umma_prepare();
     if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
     if (!status_ptr()) { s = CC3D_ERR_CUDA; goto fail; }
-    p->kc = (desc->c_in % 64 == 0) ? 64 : (desc->c_in % 96 == 0) ? 96 : 32;
     if (cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, p->device) !=
         cudaSuccess)
       p->sm_count = 148;
-    // N tile: the largest channel split that divides c_out (a multiple of
-    // 16, at most 256: the tcgen05 N limit).  Measured on B200: the time of
-    // one 128 x N x 16 MMA has a floor of ~130 cycles for N <= 192, so
-    // smaller N tiles only add CTAs that each run at lower efficiency.  The
-    // choice depends on c_out only, never on t, so a streamed sequence and a
-    // whole-sequence call run identical arithmetic.
+    // Tile configuration (N split, sub-tiles, pipeline depths): a function
+    // of (n, c_in, c_out, h, w, epilogue), never of t, so a streamed
+    // sequence and a whole-sequence call run identical arithmetic.
     {
-      int best_nt = 0;
-      for (int nt = 256; nt >= 16 && !best_nt; nt -= 16) {
-        if (desc->c_out % nt) continue;
-        if (desc->epi == CC3D_EPI_BIAS_RMS_SILU && nt != desc->c_out) continue;
-        best_nt = nt;
+      UmmaConfig cfg;
+      if (!choose_umma_config(desc->n, desc->c_in, desc->c_out, desc->h, desc->w, desc->kt,
+                              desc->kh, desc->epi == CC3D_EPI_BIAS_RMS_SILU, p->sm_count, &cfg)) {
+        s = CC3D_ERR_UNSUPPORTED;
+        goto fail;
       }
-      if (!best_nt) { s = CC3D_ERR_UNSUPPORTED; goto fail; }
-      p->nt = best_nt;
-      p->n_ntiles = desc->c_out / best_nt;
-    }
-    {
-      int cols = 32;
-      while (cols < 2 * p->nt) cols *= 2;  // two accumulators (double buffer)
-      p->tmem_cols = cols;
-    }
-    // Pipeline depths: two halo stages, as many weight stages as fit.
-    p->na = 2;
-    {
-      const size_t budget = 200 * 1024;
-      int nb = 8;
-      while (nb > 2 && umma_smem_bytes(p->kc, p->nt, desc->kh, desc->kw, p->na, nb) > budget)
-        --nb;
-      p->nb = nb;
-      const size_t smem =
-          umma_launch_smem(p->kc, p->nt, desc->kh, p->na, p->nb, p->tmem_cols) + 1024;
-      int per_sm = static_cast<int>((228 * 1024) / smem);
-      if (per_sm > 512 / p->tmem_cols) per_sm = 512 / p->tmem_cols;
-      if (per_sm > 2) per_sm = 2;
-      if (per_sm < 1) per_sm = 1;
-      p->ctas_per_sm = per_sm;
+      p->kc = cfg.kc; p->nt = cfg.nt; p->n_ntiles = cfg.n_ntiles; p->sub = cfg.sub;
+      p->nbuf = cfg.nbuf; p->na = cfg.na; p->nb = cfg.nb; p->tmem_cols = cfg.tmem_cols;
+      p->ctas_per_sm = cfg.ctas_per_sm; p->split = cfg.split;
+      p->max_clusters = 0;
+      if (cfg.split > 1) {
+        p->max_clusters = umma_max_clusters(cfg, desc->kh);
+        if (p->max_clusters < 1) { s = CC3D_ERR_CUDA; goto fail; }
+      }
     }
     p->st.tile_h = umma_tile_h();
-    p->st.tile_w = umma_tile_w();
+    p->st.tile_w = umma_tile_w() * p->sub;
     p->st.n_tile = p->nt;
     p->st.k_chunk = p->kc;
+    p->st.k_split = p->split;
     const size_t bytes = sizeof(__nv_bfloat16) * desc->c_out * desc->c_in * taps;
     if (cudaMalloc(&p->wimg, bytes) != cudaSuccess) { s = CC3D_ERR_OOM; goto fail; }
     e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(desc->weight), p->wimg,
@@ -507,11 +492,13 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
                          stream);
   } else {
     CUtensorMap mx, mc;
-    const int box_w = umma_tile_w() + d.kw - 1, box_h = umma_tile_h() + d.kh - 1;
-    if (!encode_act_map(&mx, x, d.c_in, d.w, d.h, t, d.n, box_w, box_h))
+    const int tile_w = umma_tile_w() * p->sub;
+    const int box_w = umma_halo_box_w(p->kc, p->sub, d.kw), box_h = umma_tile_h() + d.kh - 1;
+    const int box_c = umma_halo_box_c(p->kc);
+    if (!encode_act_map(&mx, x, d.c_in, d.w, d.h, t, d.n, box_w, box_h, box_c))
       return reject(CC3D_ERR_CUDA);
     if (cache_in && front > 0) {
-      if (!encode_act_map(&mc, cache_in, d.c_in, d.w, d.h, front, d.n, box_w, box_h))
+      if (!encode_act_map(&mc, cache_in, d.c_in, d.w, d.h, front, d.n, box_w, box_h, box_c))
         return reject(CC3D_ERR_CUDA);
     } else {
       mc = mx;
@@ -528,14 +515,22 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
     a.n = d.n; a.t = t; a.h = d.h; a.w = d.w; a.c_in = d.c_in; a.c_out = d.c_out;
     a.kt = d.kt; a.kh = d.kh; a.kw = d.kw; a.pad_h = d.pad_h; a.pad_w = d.pad_w;
     a.nt = p->nt; a.n_ntiles = p->n_ntiles;
-    a.tiles_w = (d.w + umma_tile_w() - 1) / umma_tile_w();
+    a.sub = p->sub; a.nbuf = p->nbuf; a.split = p->split;
+    a.tiles_w = (d.w + tile_w - 1) / tile_w;
     a.tiles_h = (d.h + umma_tile_h() - 1) / umma_tile_h();
     a.na = p->na; a.nb = p->nb; a.tmem_cols = p->tmem_cols;
     a.epi = static_cast<int>(d.epi);
     a.has_cache = (cache_in && front > 0) ? 1 : 0;
     tiles = static_cast<uint64_t>(d.n) * t * a.tiles_h * a.tiles_w * a.n_ntiles;
-    const uint64_t slots = static_cast<uint64_t>(p->sm_count) * p->ctas_per_sm;
-    const uint64_t grid = tiles < slots ? tiles : slots;
+    uint64_t grid;
+    if (p->split > 1) {
+      // one cluster of `split` CTAs per tile, at most as many as fit at once
+      const uint64_t clusters = static_cast<uint64_t>(p->max_clusters);
+      grid = (tiles < clusters ? tiles : clusters) * p->split;
+    } else {
+      const uint64_t slots = static_cast<uint64_t>(p->sm_count) * p->ctas_per_sm;
+      grid = tiles < slots ? tiles : slots;
+    }
     e = launch_conv_umma(mx, mc, a, p->kc, static_cast<unsigned>(grid), stream);
     count_launch();
   }

@@ -6,31 +6,36 @@
 // accumulator held in tensor memory; bias is added once in the epilogue
 // ("cache-aware video decoder lowering" summary: bias after the sum).
 //
-// Tiling.  An output tile is TW = 8 columns x TH = 16 rows of one frame
-// (M = 128 rows of the GEMM, row m = 8 * r + c) by NT output channels.  The
-// kernel is persistent: one CTA per SM walks the tiles round-robin.  The K
-// loop of a tile runs over (kt, channel chunk of KC, kh, kw).
+// Tiling.  An MMA tile is TW = 8 columns x TH = 16 rows of one frame
+// (M = 128 rows of the GEMM, row m = 8 * r + c) by NT output channels.  A
+// CTA tile is SUB = 1 or 2 such MMA tiles side by side (8 or 16 columns);
+// with two, every weight stage feeds two MMAs.  The kernel is persistent:
+// one CTA per SM walks the tiles round-robin.  The K loop of a tile runs
+// over (kt, channel chunk of KC, kh, kw).
 //
-// A operand: for each (kt, channel chunk) one TMA box brings the input
-// halo of the tile -- (TH + kh - 1) x (TW + kw - 1) pixels x KC channels --
+// A operand: for each (kt, channel chunk) the input halo of the tile --
+// (TH + kh - 1) x (SUB * TW + kw - 1) pixels x KC channels -- arrives by TMA
 // from the current chunk x (frame tau = t + kt - (kt_size - 1) >= 0) or the
-// frame cache (tau < 0).  Spatial padding is TMA out-of-bounds zero fill,
-// and a frame before the chunk with no cache (all zeros) is skipped: its
-// stage is neither loaded nor multiplied.  No padded copy exists anywhere.  For 64-channel
-// chunks the halo is one TMA box with the 128-byte swizzle,
-//     [halo rows][halo cols][64 channels = 128 bytes],
-// and the A matrix of spatial tap (kh, kw) is the same buffer seen from a
-// start address shifted by (kh * halo_cols + kw) whole 128-byte rows: the
-// tensor core un-swizzles by absolute shared-memory address, so a row-shifted
-// view reads correctly (checked on B200).  One load serves all kh * kw taps.
-// 32- and 96-channel chunks use no-swizzle core matrices instead,
+// frame cache (tau < 0), as no-swizzle core matrices,
 //     [KC/8 slabs][halo rows][halo cols][8 channels],
-// loaded as one 8-channel box per slab, where a pixel shift is 16 bytes.
+// one 8-channel box per slab.  Spatial padding is TMA out-of-bounds zero
+// fill, and a frame before the chunk with no cache (all zeros) is skipped:
+// its stage is neither loaded nor multiplied.  No padded copy exists.  The
+// A matrix of spatial tap (kh, kw) and of sub-tile s is the same buffer seen
+// from a start address shifted by (kh * halo_cols + kw + 8 s) pixels of 16
+// bytes, so one load serves every tap.
 //
 // B operand: the weights, re-tiled at plan time into the exact shared
 // memory image of each (N tile, tap, channel chunk) stage
 //     [KC/8][NT][8 channels]   (K-major core matrices),
 // fetched with one 1-D bulk copy per stage.
+//
+// Temporal split.  When a frame has too few tiles to occupy the GPU, the
+// kernel runs as clusters of kt CTAs that all take the same tile: CTA r
+// multiplies temporal tap r only, the senders (r < kt - 1) stage their fp32
+// partial sums in their own shared memory, and the last CTA reads them
+// through distributed shared memory, adds them to its own accumulator in a
+// fixed order and runs the epilogue.
 //
 // Warp roles (192 threads): warp 0 issues the loads, warp 1 owns tensor
 // memory and issues tcgen05.mma from one thread, warps 2..5 run the
@@ -60,27 +65,56 @@ constexpr int kEpiWarps = 4;
 // Bound of the drain waits at exit (loads / MMAs already issued finish in
 // microseconds; this only guards against a broken pipeline).
 constexpr unsigned long long kDrainLimitNs = 100ull * 1000000ull;
+// Temporal split: partial sums cross from the sender CTAs to the leader CTA
+// of the cluster in rounds of kXC accumulator columns.  Each epilogue warp of
+// the leader owns kXSlots receive slots, each holding one kXC-column piece
+// (32 lanes x kXC fp32 = kXPieceBytes) per sender.
+constexpr int kXC = 16;
+constexpr int kXSlots = 2;
+constexpr uint32_t kXPieceBytes = 32u * kXC * 4u;
+__host__ __device__ constexpr uint32_t x_bytes(int split) {
+  return split > 1 ? kEpiWarps * kXSlots * static_cast<uint32_t>(split - 1) * kXPieceBytes : 0u;
+}
 
 struct SmemLayout {
-  uint32_t a_off, a_stage, slab, b_off, b_stage, bar_off, total;
+  uint32_t a_off, a_stage, slab, b_off, b_stage, x_off, bar_off, total;
   int na, nb;
 };
 
 __host__ __device__ inline uint32_t round_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-__host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw, int na, int nb) {
+// 64-channel chunks stage the A halo with the 128-byte swizzle: one TMA box
+// of 128-byte pixel rows, its columns padded to a multiple of 8 so that an
+// image row of the halo spans whole 1024-byte swizzle atoms.  Other chunk
+// widths use 8-channel no-swizzle slabs (16-byte rows, 8 boxes for 64
+// channels: many more TMA requests per stage).
+__host__ __device__ constexpr bool uses_sw128(int kc) { return kc == 64; }
+__host__ __device__ inline int halo_cols(int kc, int sub, int kw) {
+  const int hw = kTW * sub + kw - 1;
+  return uses_sw128(kc) ? (hw + 7) / 8 * 8 : hw;
+}
+
+__host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw, int na, int nb,
+                                                  int sub, int split) {
   SmemLayout L;
-  const uint32_t hh = kTH + kh - 1, hw = kTW + kw - 1;
-  L.slab = round_up(hh * hw * 16u, 128u);
-  L.a_stage = (kc / 8) * L.slab;
+  const uint32_t hh = kTH + kh - 1, hw = static_cast<uint32_t>(halo_cols(kc, sub, kw));
+  if (uses_sw128(kc)) {
+    L.slab = hh * hw * 128u;  // the whole halo; a multiple of 1024
+    L.a_stage = L.slab;
+  } else {
+    L.slab = round_up(hh * hw * 16u, 128u);
+    L.a_stage = (kc / 8) * L.slab;
+  }
   L.b_stage = static_cast<uint32_t>(nt) * kc * 2u;
   L.na = na;
   L.nb = nb;
   L.a_off = 0;
   L.b_off = round_up(L.a_off + na * L.a_stage, 1024u);
-  L.bar_off = round_up(L.b_off + nb * L.b_stage, 64u);
-  // full_a, empty_a, full_b, empty_b, acc_full[2], acc_empty[2], drain, tmem slot
-  L.total = L.bar_off + 8u * (2 * na + 2 * nb + 5) + 16u;
+  L.x_off = round_up(L.b_off + nb * L.b_stage, 128u);
+  L.bar_off = round_up(L.x_off + x_bytes(split), 64u);
+  // full_a, empty_a, full_b, empty_b, acc_full[2], acc_empty[2], drain,
+  // (split: x_ready[4][2], x_free[4][2]), tmem slot
+  L.total = L.bar_off + 8u * (2 * na + 2 * nb + 5 + (split > 1 ? 4 * kEpiWarps : 0)) + 16u;
   return L;
 }
 
@@ -100,12 +134,12 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, const UmmaArgs &p) {
   mt /= p.tiles_h;
   c.t = mt % p.t;
   c.n = mt / p.t;
-  c.w0 = tw * kTW;
+  c.w0 = tw * kTW * p.sub;
   c.h0 = th * kTH;
   return c;
 }
 
-template <int KC, int KS>
+template <int KC, int KS, int SUB>
 __global__ void __launch_bounds__(kThreads, 1)
     conv_umma_kernel(const __grid_constant__ CUtensorMap map_x,
                      const __grid_constant__ CUtensorMap map_cache, UmmaArgs p) {
@@ -114,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // request, not a guarantee).
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const SmemLayout L = make_layout(KC, p.nt, KS, KS, p.na, p.nb);
+  const SmemLayout L = make_layout(KC, p.nt, KS, KS, p.na, p.nb, SUB, p.split);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
   uint64_t *full_a = bars;
   uint64_t *empty_a = full_a + L.na;
@@ -123,14 +157,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *acc_full = empty_b + L.nb;   // [2]
   uint64_t *acc_empty = acc_full + 2;    // [2]
   uint64_t *drain = acc_empty + 2;       // MMA completion before TMEM is freed
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  const bool split = p.split > 1;
+  // split: x_ready[q][slot] (leader: its own arrival plus the senders'
+  // bytes) and x_free[q][slot] (each sender: one arrival from the leader)
+  uint64_t *x_ready = drain + 1;
+  uint64_t *x_free = x_ready + (split ? kEpiWarps * kXSlots : 0);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(x_free + (split ? kEpiWarps * kXSlots : 0));
+
+  // Cluster geometry.  Without a split every CTA is its own cluster.  With
+  // one, the CTAs of a cluster walk the same tiles; CTA `rank` multiplies
+  // temporal tap kt = rank only, and the last CTA (tap kt - 1: the current
+  // frame, never a causal zero frame) sums the partial results and runs the
+  // epilogue.
+  const int rank = split ? static_cast<int>(cluster_ctarank()) : 0;
+  const int cid = split ? static_cast<int>(blockIdx.x) / p.split : static_cast<int>(blockIdx.x);
+  const int ncl = split ? static_cast<int>(gridDim.x) / p.split : static_cast<int>(gridDim.x);
+  const int kt_lo = split ? rank : 0;
+  const int n_kt = split ? 1 : p.kt;
+  const int leader = p.split - 1;
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
   const int n_cc = p.c_in / KC;   // channel chunks
-  const int n_a = p.kt * n_cc;    // A stages per tile
-  const uint32_t halo_w = kTW + KS - 1;
+  const int n_a = n_kt * n_cc;    // A stages per tile (of this CTA)
+  constexpr bool kSw = uses_sw128(KC);
+  const uint32_t halo_w = static_cast<uint32_t>(halo_cols(KC, SUB, KS));
   const int n_tiles = p.n * p.t * p.tiles_h * p.tiles_w * p.n_ntiles;
 
   if (threadIdx.x == 0) {
@@ -147,6 +199,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[i], kEpiWarps);
     }
     mbar_init(drain, 1);
+    if (split)
+      for (int i = 0; i < kEpiWarps * kXSlots; ++i) {
+        mbar_init(&x_ready[i], 1);
+        mbar_init(&x_free[i], 1);
+      }
     fence_mbar_init();
     prefetch_tmap(&map_x);
     if (p.has_cache) prefetch_tmap(&map_cache);
@@ -156,7 +213,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  // (with a split, no CTA may arrive on a peer's barriers before the peer
+  // has initialised them)
+  if (split)
+    cluster_sync();
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t smem_base = smem_u32(smem);
@@ -165,17 +227,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------ producer ------------------------------------
     if (lane == 0) {
-      const uint32_t a_bytes = (KC / 8) * (8u * 2u * halo_w * (kTH + KS - 1));
+      const uint32_t a_tx = kSw ? L.a_stage : (KC / 8) * (16u * halo_w * (kTH + KS - 1));
       int sa = 0, sb = 0;
       uint32_t pa = 0, pb = 0;
       // stages issued at least once, and the phase parity of their last issue
       uint32_t a_used = 0, a_par = 0, b_used = 0, b_par = 0;
-      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+      for (int tile = cid; tile < n_tiles && ok; tile += ncl) {
         const TileCoord tc0 = decode_tile(tile, p);
         const uint8_t *wsrc =
             p.wimg + static_cast<size_t>(tc0.ntile) * p.kt * KS * KS * n_cc * L.b_stage;
         for (int ia = 0; ia < n_a && ok; ++ia) {
-          const int kt = ia / n_cc, cc = ia % n_cc;
+          const int kt = kt_lo + ia / n_cc, cc = ia % n_cc;
           // A frame before the chunk with no cache is all zeros: its stage
           // (and its taps' weights) is skipped here and by the MMA issuer.
           if (tc0.t + kt - (p.kt - 1) < 0 && !p.has_cache) continue;
@@ -183,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full_a[sa], a_bytes);
+          mbar_arrive_expect_tx(&full_a[sa], a_tx);
           a_used |= 1u << sa;
           a_par = (a_par & ~(1u << sa)) | (pa << sa);
           const int tau = tc0.t + kt - (p.kt - 1);
@@ -191,10 +253,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const CUtensorMap *map = from_cache ? &map_cache : &map_x;
           const int tcoord = from_cache ? tau + (p.kt - 1) : tau;
           const uint32_t dst = smem_base + L.a_off + sa * L.a_stage;
+          if constexpr (kSw) {
+            tma_load_5d(dst, map, &full_a[sa], cc * KC, tc0.w0 - KS / 2, tc0.h0 - KS / 2, tcoord,
+                        tc0.n);
+          } else {
 #pragma unroll
-          for (int s = 0; s < KC / 8; ++s)
-            tma_load_5d(dst + s * L.slab, map, &full_a[sa], cc * KC + s * 8, tc0.w0 - KS / 2,
-                        tc0.h0 - KS / 2, tcoord, tc0.n);
+            for (int s = 0; s < KC / 8; ++s)
+              tma_load_5d(dst + s * L.slab, map, &full_a[sa], cc * KC + s * 8, tc0.w0 - KS / 2,
+                          tc0.h0 - KS / 2, tcoord, tc0.n);
+          }
           if (++sa == L.na) { sa = 0; pa ^= 1; }
 #pragma unroll 1
           for (int ts = 0; ts < KS * KS; ++ts) {
@@ -225,36 +292,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------ MMA issuer ----------------------------------
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kM, p.nt);
-      const uint32_t a_sbo = halo_w * 16u;
       const uint32_t b_lbo = static_cast<uint32_t>(p.nt) * 16u;
-      // Descriptors of stage 0; other stages, taps and K steps only move the
-      // start address (low 14 bits, 16-byte units), so they are additions.
-      // A 16-element K step is two 8-channel slabs (A) or two core-matrix
-      // columns (B) further on; a halo pixel is 16 bytes.
-      const uint64_t adesc0 = smem_desc_noswizzle(smem_base + L.a_off, L.slab, a_sbo);
+      // Descriptors of stage 0; other stages, taps, sub-tiles and K steps
+      // only move the start address (low 14 bits, 16-byte units), so they
+      // are additions.  A halo pixel is 128 bytes (swizzled) or 16 bytes (an
+      // 8-channel slab); a 16-element K step is 32 bytes along the swizzled
+      // row, or two slabs / two B core-matrix columns further on.
+      const uint64_t adesc0 =
+          kSw ? smem_desc_sw128(smem_base + L.a_off, halo_w * 128u)
+              : smem_desc_noswizzle(smem_base + L.a_off, L.slab, halo_w * 16u);
       const uint64_t bdesc0 = smem_desc_noswizzle(smem_base + L.b_off, b_lbo, 128u);
-      const uint32_t astep16 = 2u * (L.slab >> 4);
+      const uint32_t astep16 = kSw ? 2u : 2u * (L.slab >> 4);
       const uint32_t bstep16 = 2u * (b_lbo >> 4);
-      const uint32_t pix16 = 1u;
+      const uint32_t pix16 = kSw ? 8u : 1u;
       int sa = 0, sb = 0;
       uint32_t pa = 0, pb = 0;
       int it = 0;
-      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++it) {
-        const int buf = it & 1;
+      for (int tile = cid; tile < n_tiles && ok; tile += ncl, ++it) {
+        const int buf = it % p.nbuf;
+        const uint32_t use_par = static_cast<uint32_t>((it / p.nbuf) & 1);
         // wait until the epilogue has drained this accumulator buffer
-        if (!mbar_wait_bounded(&acc_empty[buf], ((it >> 1) & 1) ^ 1, p.wait_limit_ns, p.status,
-                               6)) {
+        if (!mbar_wait_bounded(&acc_empty[buf], use_par ^ 1, p.wait_limit_ns, p.status, 6)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + buf * p.nt;
+        // sub-tile s of this buffer accumulates at columns (buf * SUB + s) * nt
+        const uint32_t d_tmem = tmem_base + buf * SUB * p.nt;
         const TileCoord tcm = decode_tile(tile, p);
         uint32_t accumulate = 0;
         for (int ia = 0; ia < n_a && ok; ++ia) {
           // the same zero-frame stages the producer skipped; adding their
           // exact zeros would not change the accumulator
-          if (tcm.t + ia / n_cc - (p.kt - 1) < 0 && !p.has_cache) continue;
+          if (tcm.t + kt_lo + ia / n_cc - (p.kt - 1) < 0 && !p.has_cache) continue;
           if (!mbar_wait_bounded(&full_a[sa], pa, p.wait_limit_ns, p.status, 3)) {
             ok = false;
             break;
@@ -272,7 +342,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t b_st = bdesc0 + ((sb * L.b_stage) >> 4);
 #pragma unroll
             for (int j = 0; j < KC / 16; ++j) {
-              umma_bf16(d_tmem, a_tap + j * astep16, b_st + j * bstep16, idesc, accumulate);
+              // every sub-tile (8 pixels further along the halo row) reuses
+              // this weight stage
+#pragma unroll
+              for (int sbt = 0; sbt < SUB; ++sbt)
+                umma_bf16(d_tmem + sbt * p.nt, a_tap + sbt * kTW * pix16 + j * astep16,
+                          b_st + j * bstep16, idesc, accumulate);
               accumulate = 1;
             }
             umma_commit(&empty_b[sb]);  // frees the B stage when these MMAs finish
@@ -293,31 +368,185 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int m = q * 32 + lane;
     const int r = m / kTW, c = m % kTW;
     int it = 0;
-    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
-      const int buf = it & 1;
+    uint32_t xk = 0;  // exchange rounds of this warp so far (split)
+    // the leader's receive slots of this warp: [slot][sender][quad of 4
+    // columns][lane][4 fp32]; x_lane(slot, sender) is this lane's quad 0
+    const int n_send = p.split - 1;
+    auto x_lane = [&](uint32_t slot, int sender) -> uint32_t {
+      return smem_base + L.x_off +
+             ((static_cast<uint32_t>(q) * kXSlots + slot) * static_cast<uint32_t>(n_send) +
+              static_cast<uint32_t>(sender)) * kXPieceBytes +
+             static_cast<uint32_t>(lane) * 16u;
+    };
+    for (int tile = cid; tile < n_tiles; tile += ncl, ++it) {
+      const int buf = it % p.nbuf;
+      const uint32_t use_par = static_cast<uint32_t>((it / p.nbuf) & 1);
       const TileCoord tc0 = decode_tile(tile, p);
-      const int h = tc0.h0 + r, w = tc0.w0 + c;
-      const bool valid = (h < p.h) && (w < p.w);
       uint32_t got = 0;
       if (lane == 0)
-        got = mbar_wait_bounded(&acc_full[buf], (it >> 1) & 1, p.wait_limit_ns, p.status, 5)
-                  ? 1u
-                  : 0u;
+        got = mbar_wait_bounded(&acc_full[buf], use_par, p.wait_limit_ns, p.status, 5) ? 1u : 0u;
       got = __shfl_sync(0xffffffffu, got, 0);
       if (!got) break;
       tc_fence_after();
-      const uint32_t taddr =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * p.nt);
-      const int n0 = tc0.ntile * p.nt;
-      const size_t pix = ((static_cast<size_t>(tc0.n) * p.t + tc0.t) * p.h + h) * p.w + w;
-      __nv_bfloat16 *yrow = p.y + pix * p.c_out + n0;
-      const __nv_bfloat16 *rrow = p.residual ? p.residual + pix * p.c_out + n0 : nullptr;
-      float inv = 1.0f;
-      if (p.epi == 2) {
-        // pass 1: sum of squares of the biased row (three loads in flight)
-        float ss = 0.f;
+      if (split && rank != leader) {
+        // ---- sender: hand this CTA's partial sums to the leader, kXC
+        // columns per round, written straight into the leader's receive slot
+        // with st.async (the leader's x_ready counts the bytes).  A tile
+        // whose only frame is a causal zero frame has no partial (its MMAs
+        // were skipped): its rounds send nothing but still take their turn.
+        const bool zero = !p.has_cache && tc0.t + rank - (p.kt - 1) < 0;
+        bool xok = true;
+        for (int sbt = 0; sbt < SUB && xok; ++sbt) {
+          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                 static_cast<uint32_t>((buf * SUB + sbt) * p.nt);
+          for (int j0 = 0; j0 < p.nt; j0 += kXC, ++xk) {
+            uint32_t raw[kXC];
+            if (!zero) {
+              __syncwarp();
+              tmem_ld16_nowait(taddr + j0, raw);
+              tmem_wait_ld();
+              tmem_regs_after_wait<kXC>(raw);
+            }
+            if (sbt == SUB - 1 && j0 + kXC >= p.nt) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            }
+            const uint32_t slot = xk % kXSlots, ph = (xk / kXSlots) & 1u;
+            uint32_t free_ok = 0;
+            if (lane == 0)
+              free_ok = mbar_wait_bounded_cluster(&x_free[q * kXSlots + slot], ph ^ 1u,
+                                                  p.wait_limit_ns, p.status, 7)
+                            ? 1u
+                            : 0u;
+            free_ok = __shfl_sync(0xffffffffu, free_ok, 0);
+            if (!free_ok) {
+              xok = false;
+              break;
+            }
+            if (!zero) {
+              const uint32_t dst = mapa_shared(x_lane(slot, rank), static_cast<uint32_t>(leader));
+              const uint32_t bar = mapa_shared(smem_u32(&x_ready[q * kXSlots + slot]),
+                                               static_cast<uint32_t>(leader));
+#pragma unroll
+              for (int u = 0; u < kXC / 4; ++u) st_async_v4(dst + u * 512u, raw + 4 * u, bar);
+            }
+          }
+        }
+        if (!xok) break;
+        continue;
+      }
+      if (split) {
+        // ---- leader: fold the senders' partial sums into this accumulator,
+        // in a fixed order (own tap, then taps kt-2 .. 0), so that every call
+        // over the same frames gives the same bits.
+        int n_live = 0;  // senders whose tap is not a causal zero frame
+        for (int sr = 0; sr < n_send; ++sr)
+          n_live += (!p.has_cache && tc0.t + sr - (p.kt - 1) < 0) ? 0 : 1;
+        bool xok = true;
+        for (int sbt = 0; sbt < SUB && xok; ++sbt) {
+          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                 static_cast<uint32_t>((buf * SUB + sbt) * p.nt);
+          for (int j0 = 0; j0 < p.nt; j0 += kXC, ++xk) {
+            const uint32_t slot = xk % kXSlots, ph = (xk / kXSlots) & 1u;
+            uint32_t raw[kXC];
+            __syncwarp();
+            tmem_ld16_nowait(taddr + j0, raw);
+            uint32_t ready = 0;
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&x_ready[q * kXSlots + slot],
+                                    static_cast<uint32_t>(n_live) * kXPieceBytes);
+              ready = mbar_wait_bounded_cluster(&x_ready[q * kXSlots + slot], ph, p.wait_limit_ns,
+                                                p.status, 8)
+                          ? 1u
+                          : 0u;
+            }
+            ready = __shfl_sync(0xffffffffu, ready, 0);
+            tmem_wait_ld();
+            tmem_regs_after_wait<kXC>(raw);
+            if (!ready) {
+              xok = false;
+              break;
+            }
+            for (int src_rank = leader - 1; src_rank >= 0; --src_rank) {
+              if (!p.has_cache && tc0.t + src_rank - (p.kt - 1) < 0) continue;  // no partial
+              const uint32_t src = x_lane(slot, src_rank);
+#pragma unroll
+              for (int u = 0; u < kXC / 4; ++u) {
+                float4 f;
+                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                             : "=f"(f.x), "=f"(f.y), "=f"(f.z), "=f"(f.w)
+                             : "r"(src + u * 512u)
+                             : "memory");
+                raw[4 * u] = __float_as_uint(__uint_as_float(raw[4 * u]) + f.x);
+                raw[4 * u + 1] = __float_as_uint(__uint_as_float(raw[4 * u + 1]) + f.y);
+                raw[4 * u + 2] = __float_as_uint(__uint_as_float(raw[4 * u + 2]) + f.z);
+                raw[4 * u + 3] = __float_as_uint(__uint_as_float(raw[4 * u + 3]) + f.w);
+              }
+            }
+            // the slot's values are in registers: the senders may refill it
+            __syncwarp();
+            if (lane == 0)
+              for (int dst_rank = 0; dst_rank < leader; ++dst_rank)
+                mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&x_free[q * kXSlots + slot]),
+                                                       static_cast<uint32_t>(dst_rank)));
+            __syncwarp();
+            tmem_st16(taddr + j0, raw);
+          }
+        }
+        __syncwarp();
+        tmem_wait_st();
+        if (!xok) break;
+      }
+      for (int sbt = 0; sbt < SUB; ++sbt) {
+        const int h = tc0.h0 + r, w = tc0.w0 + sbt * kTW + c;
+        const bool valid = (h < p.h) && (w < p.w);
+        const bool last_sub = sbt == SUB - 1;
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>((buf * SUB + sbt) * p.nt);
+        const int n0 = tc0.ntile * p.nt;
+        const size_t pix = ((static_cast<size_t>(tc0.n) * p.t + tc0.t) * p.h + h) * p.w + w;
+        __nv_bfloat16 *yrow = p.y + pix * p.c_out + n0;
+        const __nv_bfloat16 *rrow = p.residual ? p.residual + pix * p.c_out + n0 : nullptr;
+        float inv = 1.0f;
+        if (p.epi == 2) {
+          // pass 1: sum of squares of the biased row (three loads in flight)
+          float ss = 0.f;
+          for (int j0 = 0; j0 < p.nt; j0 += 48) {
+            const int nld = (p.nt - j0) >= 48 ? 3 : (p.nt - j0) / 16;
+            uint32_t raw[48];
+            __syncwarp();
+#pragma unroll
+            for (int u = 0; u < 3; ++u)
+              if (u < nld) tmem_ld16_nowait(taddr + j0 + 16 * u, raw + 16 * u);
+            tmem_wait_ld();
+            tmem_regs_after_wait<48>(raw);
+#pragma unroll
+            for (int u = 0; u < 3; ++u) {
+              if (u >= nld) continue;
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float hv = __uint_as_float(raw[16 * u + i]) + p.bias[n0 + j0 + 16 * u + i];
+                ss = fmaf(hv, hv, ss);
+              }
+            }
+          }
+          inv = sqrtf(static_cast<float>(p.c_out)) / fmaxf(sqrtf(ss), 1e-12f);
+        }
+        // pass 2: bias (+ residual | RMS scale + SiLU) -> bf16 -> global
         for (int j0 = 0; j0 < p.nt; j0 += 48) {
           const int nld = (p.nt - j0) >= 48 ? 3 : (p.nt - j0) / 16;
+          uint4 res[6];
+          if (p.epi == 1 && valid) {
+            // residual loads first, so their latency overlaps the TMEM reads
+#pragma unroll
+            for (int u = 0; u < 3; ++u)
+              if (u < nld) {
+                const uint4 *rr = reinterpret_cast<const uint4 *>(rrow + j0 + 16 * u);
+                res[2 * u] = rr[0];
+                res[2 * u + 1] = rr[1];
+              }
+          }
           uint32_t raw[48];
           __syncwarp();
 #pragma unroll
@@ -325,89 +554,60 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (u < nld) tmem_ld16_nowait(taddr + j0 + 16 * u, raw + 16 * u);
           tmem_wait_ld();
           tmem_regs_after_wait<48>(raw);
+          if (last_sub && j0 + 48 >= p.nt) {
+            // last read of this accumulator buffer: hand it back to the MMA warp
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+          }
 #pragma unroll
           for (int u = 0; u < 3; ++u) {
             if (u >= nld) continue;
+            const int j = j0 + 16 * u;
+            float v[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float hv = __uint_as_float(raw[16 * u + i]) + p.bias[n0 + j0 + 16 * u + i];
-              ss = fmaf(hv, hv, ss);
+            for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(raw[16 * u + i]) + p.bias[n0 + j + i];
+            if (p.epi == 1 && valid) {
+              const __nv_bfloat16 *rb0 = reinterpret_cast<const __nv_bfloat16 *>(&res[2 * u]);
+              const __nv_bfloat16 *rb1 = reinterpret_cast<const __nv_bfloat16 *>(&res[2 * u + 1]);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                v[i] += __bfloat162float(rb0[i]);
+                v[8 + i] += __bfloat162float(rb1[i]);
+              }
+            } else if (p.epi == 2) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                float a = v[i] * inv * p.gamma[n0 + j + i];
+                if (p.beta) a += p.beta[n0 + j + i];
+                v[i] = silu_fast(a);
+              }
+            }
+            if (valid) {
+              uint4 o0, o1;
+              o0.x = pack_bf16x2(v[0], v[1]);
+              o0.y = pack_bf16x2(v[2], v[3]);
+              o0.z = pack_bf16x2(v[4], v[5]);
+              o0.w = pack_bf16x2(v[6], v[7]);
+              o1.x = pack_bf16x2(v[8], v[9]);
+              o1.y = pack_bf16x2(v[10], v[11]);
+              o1.z = pack_bf16x2(v[12], v[13]);
+              o1.w = pack_bf16x2(v[14], v[15]);
+              uint4 *dst = reinterpret_cast<uint4 *>(yrow + j);
+              dst[0] = o0;
+              dst[1] = o1;
             }
           }
         }
-        inv = sqrtf(static_cast<float>(p.c_out)) / fmaxf(sqrtf(ss), 1e-12f);
-      }
-      // pass 2: bias (+ residual | RMS scale + SiLU) -> bf16 -> global
-      for (int j0 = 0; j0 < p.nt; j0 += 48) {
-        const int nld = (p.nt - j0) >= 48 ? 3 : (p.nt - j0) / 16;
-        uint4 res[6];
-        if (p.epi == 1 && valid) {
-          // residual loads first, so their latency overlaps the TMEM reads
-#pragma unroll
-          for (int u = 0; u < 3; ++u)
-            if (u < nld) {
-              const uint4 *rr = reinterpret_cast<const uint4 *>(rrow + j0 + 16 * u);
-              res[2 * u] = rr[0];
-              res[2 * u + 1] = rr[1];
-            }
-        }
-        uint32_t raw[48];
-        __syncwarp();
-#pragma unroll
-        for (int u = 0; u < 3; ++u)
-          if (u < nld) tmem_ld16_nowait(taddr + j0 + 16 * u, raw + 16 * u);
-        tmem_wait_ld();
-        tmem_regs_after_wait<48>(raw);
-        if (j0 + 48 >= p.nt) {
-          // last read of this accumulator: hand the buffer back to the MMA warp
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[buf]);
-        }
-#pragma unroll
-        for (int u = 0; u < 3; ++u) {
-          if (u >= nld) continue;
-          const int j = j0 + 16 * u;
-          float v[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(raw[16 * u + i]) + p.bias[n0 + j + i];
-          if (p.epi == 1 && valid) {
-            const __nv_bfloat16 *rb0 = reinterpret_cast<const __nv_bfloat16 *>(&res[2 * u]);
-            const __nv_bfloat16 *rb1 = reinterpret_cast<const __nv_bfloat16 *>(&res[2 * u + 1]);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              v[i] += __bfloat162float(rb0[i]);
-              v[8 + i] += __bfloat162float(rb1[i]);
-            }
-          } else if (p.epi == 2) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float a = v[i] * inv * p.gamma[n0 + j + i];
-              if (p.beta) a += p.beta[n0 + j + i];
-              v[i] = silu_fast(a);
-            }
-          }
-          if (valid) {
-            uint4 o0, o1;
-            o0.x = pack_bf16x2(v[0], v[1]);
-            o0.y = pack_bf16x2(v[2], v[3]);
-            o0.z = pack_bf16x2(v[4], v[5]);
-            o0.w = pack_bf16x2(v[6], v[7]);
-            o1.x = pack_bf16x2(v[8], v[9]);
-            o1.y = pack_bf16x2(v[10], v[11]);
-            o1.z = pack_bf16x2(v[12], v[13]);
-            o1.w = pack_bf16x2(v[14], v[15]);
-            uint4 *dst = reinterpret_cast<uint4 *>(yrow + j);
-            dst[0] = o0;
-            dst[1] = o1;
-          }
-        }
-      }
+      }  // sub-tiles
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  // no CTA leaves while a peer may still read its staging or arrive on its
+  // barriers
+  if (split) cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -417,17 +617,113 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb) {
-  return make_layout(kc, nt, kh, kw, na, nb).total + 1024;  // + alignment slack
+size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb, int sub, int split) {
+  return make_layout(kc, nt, kh, kw, na, nb, sub, split).total + 1024;  // + alignment slack
+}
+
+namespace {
+// Buffers, pipeline depths and residency of one (sub, nt) tile shape.
+bool finish_config(int ks, UmmaConfig &c) {
+  c.nbuf = (2 * c.sub * c.nt <= 512) ? 2 : 1;  // double-buffered accumulators when they fit
+  c.tmem_cols = 32;
+  while (c.tmem_cols < c.nbuf * c.sub * c.nt) c.tmem_cols *= 2;
+  if (c.tmem_cols > 512) return false;
+  c.na = 2;
+  c.nb = 8;
+  // (a split's exchange staging gets room of its own above the usual budget)
+  const size_t budget = (c.split > 1 ? 216 : 200) * 1024;
+  while (c.nb > 2 && umma_smem_bytes(c.kc, c.nt, ks, ks, c.na, c.nb, c.sub, c.split) > budget)
+    --c.nb;
+  int per_sm = static_cast<int>(
+      (228 * 1024) /
+      (umma_launch_smem(c.kc, c.nt, ks, c.na, c.nb, c.tmem_cols, c.sub, c.split) + 1024));
+  if (per_sm > 512 / c.tmem_cols) per_sm = 512 / c.tmem_cols;
+  if (per_sm > 2) per_sm = 2;
+  c.ctas_per_sm = per_sm < 1 ? 1 : per_sm;
+  return true;
+}
+
+// Relative time of one frame of n images: whole waves of CTA tiles, each
+// wave as long as one tile's MMAs -- sub MMAs of 128 x nt x 16 per K step,
+// at the issue times measured on B200 (48 cycles up to N = 64, 56 up to
+// N = 96, N / 2 beyond) -- times the CTAs that share an SM's tensor core
+// once the tiles outnumber the SMs.
+long long frame_cost(const UmmaConfig &c, int n, int h, int w, int sm_count) {
+  const long long tiles = static_cast<long long>(n) * ((h + kTH - 1) / kTH) *
+                          ((w + c.sub * kTW - 1) / (c.sub * kTW)) * c.n_ntiles;
+  const long long slots = static_cast<long long>(sm_count) * c.ctas_per_sm;
+  const long long cyc = c.nt <= 64 ? 48 : c.nt <= 96 ? 56 : c.nt / 2;
+  const long long share = tiles > sm_count ? c.ctas_per_sm : 1;
+  return (tiles + slots - 1) / slots * share * c.sub * cyc;
+}
+}  // namespace
+
+bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
+                        int sm_count, UmmaConfig *cfg) {
+  // N tile: the largest split of c_out that is a multiple of 16 and at most
+  // `cap` (256 is the tcgen05 N limit); the RMS epilogue needs the whole row
+  // in one CTA.
+  auto largest_nt = [&](int cap) {
+    for (int nt = cap; nt >= 16; nt -= 16)
+      if (c_out % nt == 0 && (!rms_epi || nt == c_out)) return nt;
+    return 0;
+  };
+  UmmaConfig one;
+  one.kc = (c_in % 64 == 0) ? 64 : (c_in % 96 == 0) ? 96 : 32;
+  one.sub = 1;
+  one.split = 1;
+  one.nt = largest_nt(256);
+  if (!one.nt) return false;
+  one.n_ntiles = c_out / one.nt;
+  if (!finish_config(ks, one)) return false;
+  *cfg = one;
+  // Two sub-tiles (a 16 x 16 pixel CTA tile, two 8 x 16 MMA tiles) share
+  // every weight stage, halving the weight bytes that each MMA waits for.
+  // Only with N <= 128, where both sub-tiles still fit two accumulator
+  // buffers (a single buffer stalls the MMAs behind the epilogue), and only
+  // when the tile waves of one frame do not lose more than the ~5% that the
+  // halved weight traffic was measured to gain on B200.  The choice depends
+  // on (n, c, h, w) -- never on t -- so streamed and whole-sequence calls run
+  // identical arithmetic.
+  UmmaConfig two = one;
+  two.sub = 2;
+  two.nt = largest_nt(128);
+  if (two.nt) {
+    two.n_ntiles = c_out / two.nt;
+    if (finish_config(ks, two) && two.nbuf == 2 &&
+        20 * frame_cost(two, n, h, w, sm_count) <= 21 * frame_cost(one, n, h, w, sm_count))
+      *cfg = two;
+  }
+  // Temporal split: when even kt CTAs per tile fit one wave, a frame has too
+  // few tiles to occupy the GPU (a one-frame chunk of a latent-resolution
+  // decoder layer), and its time is the length of one tile's K loop.  Each
+  // CTA of a cluster of kt then runs one temporal tap, and the last sums the
+  // partials through distributed shared memory before its epilogue.  Like
+  // the rest, decided from (n, c, h, w), never from t.
+  if (kt >= 2 && kt <= 4) {
+    UmmaConfig sp = *cfg;
+    sp.split = kt;
+    const long long tiles = static_cast<long long>(n) * ((h + kTH - 1) / kTH) *
+                            ((w + sp.sub * kTW - 1) / (sp.sub * kTW)) * sp.n_ntiles;
+    if (finish_config(ks, sp) && tiles * kt <= static_cast<long long>(sm_count) * sp.ctas_per_sm)
+      *cfg = sp;
+  }
+  return true;
 }
 
 int umma_tile_w() { return kTW; }
+int umma_halo_box_w(int kc, int sub, int kw) { return halo_cols(kc, sub, kw); }
+int umma_halo_box_c(int kc) { return uses_sw128(kc) ? 64 : 8; }
 int umma_tile_h() { return kTH; }
 
 template <int KC, int KS>
 cudaError_t set_smem_attr() {
-  return cudaFuncSetAttribute(conv_umma_kernel<KC, KS>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  cudaError_t e = cudaFuncSetAttribute(conv_umma_kernel<KC, KS, 1>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(conv_umma_kernel<KC, KS, 2>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  return e;
 }
 
 cudaError_t umma_prepare() {
@@ -441,32 +737,80 @@ cudaError_t umma_prepare() {
   return e;
 }
 
-size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols) {
-  size_t smem = umma_smem_bytes(kc, nt, ks, ks, na, nb);
+size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols, int sub,
+                        int split) {
+  size_t smem = umma_smem_bytes(kc, nt, ks, ks, na, nb, sub, split);
   // A CTA that holds more than half of tensor memory must have its SM to
   // itself; asking for more than half the shared memory guarantees that.
   if (tmem_cols > 256 && smem < 116 * 1024) smem = 116 * 1024;
   return smem;
 }
 
+namespace {
+using UmmaKernel = void (*)(const CUtensorMap, const CUtensorMap, UmmaArgs);
+
+UmmaKernel umma_kernel_for(int kc, int ks, int sub) {
+#define CC3D_PICK(KC_, KS_)                                                              \
+  if (kc == KC_ && ks == KS_)                                                            \
+    return sub == 2 ? conv_umma_kernel<KC_, KS_, 2> : conv_umma_kernel<KC_, KS_, 1>;
+  CC3D_PICK(64, 3)
+  CC3D_PICK(32, 3)
+  CC3D_PICK(96, 3)
+  CC3D_PICK(64, 1)
+  CC3D_PICK(32, 1)
+  CC3D_PICK(96, 1)
+#undef CC3D_PICK
+  return nullptr;
+}
+
+cudaLaunchConfig_t umma_launch_config(unsigned grid, size_t smem, int split, cudaStream_t stream,
+                                      cudaLaunchAttribute *attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  attr->id = cudaLaunchAttributeClusterDimension;
+  attr->val.clusterDim.x = static_cast<unsigned>(split);
+  attr->val.clusterDim.y = 1;
+  attr->val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = split > 1 ? 1 : 0;
+  return cfg;
+}
+}  // namespace
+
+int umma_max_clusters(const UmmaConfig &c, int ks) {
+  if (c.split <= 1) return 0;
+  UmmaKernel k = umma_kernel_for(c.kc, ks, c.sub);
+  if (!k) return 0;
+  const size_t smem =
+      umma_launch_smem(c.kc, c.nt, ks, c.na, c.nb, c.tmem_cols, c.sub, c.split);
+  cudaLaunchAttribute attr;
+  const cudaLaunchConfig_t cfg =
+      umma_launch_config(static_cast<unsigned>(c.split), smem, c.split, nullptr, &attr);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void *>(k), &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
 cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_cache,
                              const UmmaArgs &args, int kc, unsigned grid, cudaStream_t stream) {
   if (args.kh != args.kw || (args.kh != 1 && args.kh != 3)) return cudaErrorInvalidValue;
-  const size_t smem = umma_launch_smem(kc, args.nt, args.kh, args.na, args.nb, args.tmem_cols);
-  if (smem > 227 * 1024) return cudaErrorInvalidValue;
-#define CC3D_LAUNCH(KC_, KS_)                                                              \
-  if (kc == KC_ && args.kh == KS_) {                                                       \
-    conv_umma_kernel<KC_, KS_><<<grid, kThreads, smem, stream>>>(map_x, map_cache, args); \
-    return cudaGetLastError();                                                             \
-  }
-  CC3D_LAUNCH(64, 3)
-  CC3D_LAUNCH(32, 3)
-  CC3D_LAUNCH(96, 3)
-  CC3D_LAUNCH(64, 1)
-  CC3D_LAUNCH(32, 1)
-  CC3D_LAUNCH(96, 1)
-#undef CC3D_LAUNCH
-  return cudaErrorInvalidValue;
+  const size_t smem = umma_launch_smem(kc, args.nt, args.kh, args.na, args.nb, args.tmem_cols,
+                                       args.sub, args.split);
+  if (smem > 227 * 1024 || (args.sub != 1 && args.sub != 2) || args.nbuf < 1 || args.nbuf > 2)
+    return cudaErrorInvalidValue;
+  if (args.split != 1 && (args.split != args.kt || args.split > 4 || grid % args.split != 0))
+    return cudaErrorInvalidValue;
+  UmmaKernel k = umma_kernel_for(kc, args.kh, args.sub);
+  if (!k) return cudaErrorInvalidValue;
+  cudaLaunchAttribute attr;
+  const cudaLaunchConfig_t cfg = umma_launch_config(grid, smem, args.split, stream, &attr);
+  return cudaLaunchKernelEx(&cfg, k, map_x, map_cache, args);
 }
 
 }  // namespace cc3d

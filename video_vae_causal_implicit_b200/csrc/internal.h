@@ -27,13 +27,33 @@ struct UmmaArgs {
   int tmem_cols;
   int epi;                        // 0 bias, 1 bias + residual, 2 bias + RMS + SiLU
   int has_cache;
+  int sub;                        // MMA sub-tiles (8 x 16 px) per CTA tile, side by side: 1 or 2
+  int nbuf;                       // accumulator buffers in tensor memory: 1 or 2
+  int split;                      // 1, or kt: CTAs of a cluster that share a tile, one
+                                  // temporal tap each, reduced in the last one
 };
 
-size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb);
+// Tile configuration of the UMMA conv for a problem (chosen from n, c_in,
+// c_out, h, w and the epilogue -- never from t).
+struct UmmaConfig {
+  int kc, nt, n_ntiles, sub, nbuf, split, na, nb, tmem_cols, ctas_per_sm;
+};
+bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
+                        int sm_count, UmmaConfig *cfg);
+// Clusters of cfg.split CTAs that can be resident at once (split > 1), for
+// sizing the grid; 0 when the query fails.
+int umma_max_clusters(const UmmaConfig &cfg, int ks);
+
+size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb, int sub, int split);
 cudaError_t umma_prepare();
 // Dynamic shared memory a launch requests (with the one-CTA-per-SM rule).
-size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols);
+size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols, int sub,
+                        int split);
 int umma_tile_w();
+// TMA box of the A halo: columns (padded for the 128-byte swizzle) and
+// channels (64: swizzled pixel rows; 8: no-swizzle slabs).
+int umma_halo_box_w(int kc, int sub, int kw);
+int umma_halo_box_c(int kc);
 int umma_tile_h();
 cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_cache,
                              const UmmaArgs &args, int kc, unsigned grid, cudaStream_t stream);
@@ -91,8 +111,9 @@ void count_launch();
 
 // Device address of the status word on the current device (null on error).
 int *device_status_word();
-// 5-D bf16 activation tensor map (dims C, W, H, T, N; 8-channel boxes).
+// 5-D bf16 activation tensor map (dims C, W, H, T, N; boxes of box_c = 8
+// plain or 64 swizzled channels).
 bool encode_activation_map(CUtensorMap *m, const void *base, int c, int w, int h, int t, int n,
-                           int box_w, int box_h);
+                           int box_w, int box_h, int box_c);
 
 }  // namespace cc3d

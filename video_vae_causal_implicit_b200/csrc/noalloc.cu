@@ -133,24 +133,13 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
 
   // ---- tiles: the same choice cc3d_plan_create makes --------------------------------
-  const int kc = (d->c_in % 64 == 0) ? 64 : (d->c_in % 96 == 0) ? 96 : 32;
-  int nt = 0;
-  for (int c = 256; c >= 16 && !nt; c -= 16) {
-    if (d->c_out % c) continue;
-    if (d->epi == CC3D_EPI_BIAS_RMS_SILU && c != d->c_out) continue;
-    nt = c;
-  }
-  if (!nt) return CC3D_ERR_UNSUPPORTED;
-  int tmem_cols = 32;
-  while (tmem_cols < 2 * nt) tmem_cols *= 2;
-  const int na = 2;
-  int nb = 8;
-  while (nb > 2 && umma_smem_bytes(kc, nt, d->kh, d->kw, na, nb) > 200 * 1024) --nb;
-  int per_sm = static_cast<int>((228 * 1024) / (umma_launch_smem(kc, nt, d->kh, na, nb,
-                                                                  tmem_cols) + 1024));
-  if (per_sm > 512 / tmem_cols) per_sm = 512 / tmem_cols;
-  if (per_sm > 2) per_sm = 2;
-  if (per_sm < 1) per_sm = 1;
+  UmmaConfig cfg;
+  if (!choose_umma_config(d->n, d->c_in, d->c_out, d->h, d->w, d->kt, d->kh,
+                          d->epi == CC3D_EPI_BIAS_RMS_SILU, n_sm, &cfg))
+    return CC3D_ERR_UNSUPPORTED;
+  const int max_clusters = cfg.split > 1 ? umma_max_clusters(cfg, d->kh) : 0;
+  if (cfg.split > 1 && max_clusters < 1) return CC3D_ERR_CUDA;
+  const int kc = cfg.kc, nt = cfg.nt;
 
   // ---- scratch: re-tiled weights (every call), zero bias when none is given --------
   uint8_t *wimg = scratch;
@@ -163,12 +152,15 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
 
   // ---- the conv -----------------------------------------------------------------------------
   CUtensorMap mx, mc;
-  const int box_w = umma_tile_w() + d->kw - 1, box_h = umma_tile_h() + d->kh - 1;
-  if (!encode_activation_map(&mx, x, d->c_in, d->w, d->h, t, d->n, box_w, box_h))
+  const int tile_w = umma_tile_w() * cfg.sub;
+  const int box_w = umma_halo_box_w(kc, cfg.sub, d->kw), box_h = umma_tile_h() + d->kh - 1;
+  const int box_c = umma_halo_box_c(kc);
+  if (!encode_activation_map(&mx, x, d->c_in, d->w, d->h, t, d->n, box_w, box_h, box_c))
     return CC3D_ERR_CUDA;
   const bool has_cache = cache_in && front > 0;
   if (has_cache) {
-    if (!encode_activation_map(&mc, cache_in, d->c_in, d->w, d->h, front, d->n, box_w, box_h))
+    if (!encode_activation_map(&mc, cache_in, d->c_in, d->w, d->h, front, d->n, box_w, box_h,
+                               box_c))
       return CC3D_ERR_CUDA;
   } else {
     mc = mx;
@@ -184,16 +176,22 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   a.wait_limit_ns = 2000ull * 1000000ull;
   a.n = d->n; a.t = t; a.h = d->h; a.w = d->w; a.c_in = d->c_in; a.c_out = d->c_out;
   a.kt = d->kt; a.kh = d->kh; a.kw = d->kw; a.pad_h = d->pad_h; a.pad_w = d->pad_w;
-  a.nt = nt; a.n_ntiles = d->c_out / nt;
-  a.tiles_w = (d->w + umma_tile_w() - 1) / umma_tile_w();
+  a.nt = nt; a.n_ntiles = cfg.n_ntiles;
+  a.sub = cfg.sub; a.nbuf = cfg.nbuf; a.split = cfg.split;
+  a.tiles_w = (d->w + tile_w - 1) / tile_w;
   a.tiles_h = (d->h + umma_tile_h() - 1) / umma_tile_h();
-  a.na = na; a.nb = nb; a.tmem_cols = tmem_cols;
+  a.na = cfg.na; a.nb = cfg.nb; a.tmem_cols = cfg.tmem_cols;
   a.epi = static_cast<int>(d->epi);
   a.has_cache = has_cache ? 1 : 0;
   const uint64_t tiles = uint64_t(d->n) * t * a.tiles_h * a.tiles_w * a.n_ntiles;
-  const uint64_t slots = uint64_t(n_sm) * per_sm;
-  e = launch_conv_umma(mx, mc, a, kc, static_cast<unsigned>(tiles < slots ? tiles : slots),
-                       stream);
+  uint64_t grid;
+  if (cfg.split > 1) {
+    grid = (tiles < uint64_t(max_clusters) ? tiles : uint64_t(max_clusters)) * cfg.split;
+  } else {
+    const uint64_t slots = uint64_t(n_sm) * cfg.ctas_per_sm;
+    grid = tiles < slots ? tiles : slots;
+  }
+  e = launch_conv_umma(mx, mc, a, kc, static_cast<unsigned>(grid), stream);
   count_launch();
   if (e == cudaSuccess && cache_out && front > 0)
     e = launch_cache_update(cache_in, x, cache_out, d->n, t, front, in_frame, stream);
