@@ -51,14 +51,53 @@ def test_split_with_cache_every_tap_from_a_real_frame():
     assert_close_bf16(ncthw_np(y), ref, "split with cache")
 
 
-def test_split_rms_epilogue_after_the_fold():
-    """RMS_norm + SiLU needs the whole summed row: the leader folds the
-    partials into its accumulator before both epilogue passes."""
+def test_rms_epilogue_small_frame_runs_unsplit():
+    """RMS_norm + SiLU needs whole rows in one CTA: a small frame with this
+    epilogue keeps one CTA per tile."""
     c, t, h, w = 192, 3, 18, 9
     g = synth.uniform((c,), 0.5, 1.5, 62)
     case, plan, x, y = _run(1, c, c, t, h, w, seed=63, epi=cc3d.EPI_BIAS_RMS_SILU,
                             gamma=to_dev(g))
-    assert plan.stats().k_split == 3
+    assert plan.stats().k_split == 1
     conv = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], case["b"].double().numpy())
     ref = oracle.rms_norm(conv, g.double().numpy(), silu=True)
-    assert_close_bf16(ncthw_np(y), ref, "split rms epilogue")
+    assert_close_bf16(ncthw_np(y), ref, "small-frame rms epilogue")
+
+
+def test_split_residual_epilogue_and_cuda_graph_replay():
+    """Residual epilogue on the split path, called eagerly and from a CUDA
+    graph of the same calls (one-frame chunks carrying the cache): same bytes."""
+    n, cin, cout, t, h, w = 1, 64, 96, 3, 21, 18
+    case = synth.conv_case(cin, cout, t, h, w, n=n, seed_base=64)
+    plan = cc3d.Plan(to_dev(case["w"]), to_dev(case["b"]), n=n, h=h, w=w, max_t=t,
+                     epi=cc3d.EPI_BIAS_RESIDUAL)
+    assert plan.stats().k_split == 3
+    x = to_dev(synth.ndhwc(case["x"]))
+    res = to_dev(synth.ndhwc(synth.normal((n, cout, t, h, w), 65)))
+    xs = [x[:, s:s + 1].contiguous() for s in range(t)]
+    rs = [res[:, s:s + 1].contiguous() for s in range(t)]
+    caches = [torch.empty((n, 2, h, w, cin), dtype=torch.bfloat16, device="cuda")
+              for _ in range(2)]
+
+    def run(ys):
+        cache = None
+        for s in range(t):
+            plan.forward(xs[s], ys[s], cache_in=cache, cache_out=caches[s % 2], residual=rs[s])
+            cache = caches[s % 2]
+
+    eager = [torch.empty((n, 1, h, w, cout), dtype=torch.bfloat16, device="cuda")
+             for _ in range(t)]
+    run(eager)
+    cc3d.sync_status()
+    graphed = [torch.full_like(e, float("nan")) for e in eager]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run(graphed)
+    g.replay()
+    torch.cuda.synchronize()
+    cc3d.sync_status()
+    for a, b in zip(eager, graphed):
+        assert torch.equal(a.cpu(), b.cpu())
+    ref = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], case["b"].double().numpy())
+    ref = ref + ncthw_np(res)
+    assert_close_bf16(ncthw_np(torch.cat(eager, dim=1)), ref, "split residual")

@@ -32,10 +32,11 @@
 //
 // Temporal split.  When a frame has too few tiles to occupy the GPU, the
 // kernel runs as clusters of kt CTAs that all take the same tile: CTA r
-// multiplies temporal tap r only, the senders (r < kt - 1) stage their fp32
-// partial sums in their own shared memory, and the last CTA reads them
-// through distributed shared memory, adds them to its own accumulator in a
-// fixed order and runs the epilogue.
+// multiplies temporal tap r only.  The senders (r < kt - 1) write their fp32
+// partial sums, 16 accumulator columns at a time, straight into receive
+// slots in the last CTA's shared memory (st.async, counted as transaction
+// bytes on its mbarrier); the last CTA adds them to its own accumulator in
+// a fixed order and runs the epilogue on the sums.
 //
 // Warp roles (192 threads): warp 0 issues the loads, warp 1 owns tensor
 // memory and issues tcgen05.mma from one thread, warps 2..5 run the
@@ -65,13 +66,19 @@ constexpr int kEpiWarps = 4;
 // Bound of the drain waits at exit (loads / MMAs already issued finish in
 // microseconds; this only guards against a broken pipeline).
 constexpr unsigned long long kDrainLimitNs = 100ull * 1000000ull;
-// Temporal split: partial sums cross from the sender CTAs to the leader CTA
-// of the cluster in rounds of kXC accumulator columns.  Each epilogue warp of
-// the leader owns kXSlots receive slots, each holding one kXC-column piece
-// (32 lanes x kXC fp32 = kXPieceBytes) per sender.
+// Temporal split: the kXC-column chunks of a tile's accumulator meet in one
+// CTA of the cluster (the owner, the last rank); the other CTAs send their
+// partial sums of each chunk there, and the owner adds them and runs the
+// epilogue for those columns.  Each epilogue warp of each CTA has
+// kXSlots receive slots, each holding one kXC-column piece (32 lanes x kXC
+// fp32 = kXPieceBytes) per sending rank.
 constexpr int kXC = 16;
 constexpr int kXSlots = 2;
 constexpr uint32_t kXPieceBytes = 32u * kXC * 4u;
+// x_ready[warp][slot] and x_free[warp][owner rank][slot]
+__host__ __device__ constexpr int x_bar_count(int split) {
+  return kEpiWarps * kXSlots * (1 + split);
+}
 __host__ __device__ constexpr uint32_t x_bytes(int split) {
   return split > 1 ? kEpiWarps * kXSlots * static_cast<uint32_t>(split - 1) * kXPieceBytes : 0u;
 }
@@ -114,7 +121,7 @@ __host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw
   L.bar_off = round_up(L.x_off + x_bytes(split), 64u);
   // full_a, empty_a, full_b, empty_b, acc_full[2], acc_empty[2], drain,
   // (split: x_ready[4][2], x_free[4][2]), tmem slot
-  L.total = L.bar_off + 8u * (2 * na + 2 * nb + 5 + (split > 1 ? 4 * kEpiWarps : 0)) + 16u;
+  L.total = L.bar_off + 8u * (2 * na + 2 * nb + 5 + (split > 1 ? x_bar_count(split) : 0)) + 16u;
   return L;
 }
 
@@ -158,23 +165,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *acc_empty = acc_full + 2;    // [2]
   uint64_t *drain = acc_empty + 2;       // MMA completion before TMEM is freed
   const bool split = p.split > 1;
-  // split: x_ready[q][slot] (leader: its own arrival plus the senders'
-  // bytes) and x_free[q][slot] (each sender: one arrival from the leader)
+  // split: x_ready[q][slot] (as owner: its own arrival, one arrival per
+  // other rank, and the bytes they store) and x_free[q][o][slot] (as sender
+  // to owner rank o: one arrival from o once it has read the slot)
   uint64_t *x_ready = drain + 1;
   uint64_t *x_free = x_ready + (split ? kEpiWarps * kXSlots : 0);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(x_free + (split ? kEpiWarps * kXSlots : 0));
+  uint32_t *tmem_slot =
+      reinterpret_cast<uint32_t *>(x_ready + (split ? x_bar_count(p.split) : 0));
 
   // Cluster geometry.  Without a split every CTA is its own cluster.  With
   // one, the CTAs of a cluster walk the same tiles; CTA `rank` multiplies
-  // temporal tap kt = rank only, and the last CTA (tap kt - 1: the current
-  // frame, never a causal zero frame) sums the partial results and runs the
-  // epilogue.
+  // temporal tap kt = rank only, and the partial results meet chunk by chunk
+  // in the chunk's owner, which adds them in a fixed order (tap kt-1 -- the
+  // current frame, never a causal zero frame -- then kt-2 .. 0) and runs the
+  // epilogue for those columns.
   const int rank = split ? static_cast<int>(cluster_ctarank()) : 0;
   const int cid = split ? static_cast<int>(blockIdx.x) / p.split : static_cast<int>(blockIdx.x);
   const int ncl = split ? static_cast<int>(gridDim.x) / p.split : static_cast<int>(gridDim.x);
   const int kt_lo = split ? rank : 0;
   const int n_kt = split ? 1 : p.kt;
-  const int leader = p.split - 1;
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -199,11 +208,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[i], kEpiWarps);
     }
     mbar_init(drain, 1);
-    if (split)
-      for (int i = 0; i < kEpiWarps * kXSlots; ++i) {
-        mbar_init(&x_ready[i], 1);
-        mbar_init(&x_free[i], 1);
-      }
+    if (split) {
+      for (int i = 0; i < kEpiWarps * kXSlots; ++i) mbar_init(&x_ready[i], p.split);
+      for (int i = 0; i < kEpiWarps * p.split * kXSlots; ++i) mbar_init(&x_free[i], 1);
+    }
     fence_mbar_init();
     prefetch_tmap(&map_x);
     if (p.has_cache) prefetch_tmap(&map_cache);
@@ -368,8 +376,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int m = q * 32 + lane;
     const int r = m / kTW, c = m % kTW;
     int it = 0;
-    uint32_t xk = 0;  // exchange rounds of this warp so far (split)
-    // the leader's receive slots of this warp: [slot][sender][quad of 4
+    // split: chunks of each owner rank exchanged by this warp so far
+    uint32_t xc0 = 0, xc1 = 0, xc2 = 0, xc3 = 0;
+    // this warp's receive slots: [slot][sending rank index][quad of 4
     // columns][lane][4 fp32]; x_lane(slot, sender) is this lane's quad 0
     const int n_send = p.split - 1;
     auto x_lane = [&](uint32_t slot, int sender) -> uint32_t {
@@ -388,115 +397,159 @@ __global__ void __launch_bounds__(kThreads, 1)
       got = __shfl_sync(0xffffffffu, got, 0);
       if (!got) break;
       tc_fence_after();
-      if (split && rank != leader) {
-        // ---- sender: hand this CTA's partial sums to the leader, kXC
-        // columns per round, written straight into the leader's receive slot
-        // with st.async (the leader's x_ready counts the bytes).  A tile
-        // whose only frame is a causal zero frame has no partial (its MMAs
-        // were skipped): its rounds send nothing but still take their turn.
-        const bool zero = !p.has_cache && tc0.t + rank - (p.kt - 1) < 0;
+      if (split) {
+        // ---- the partial sums of the cluster meet in the owner CTA ----
+        uint32_t live = 0;  // ranks whose tap is not a causal zero frame
+        for (int rr = 0; rr < p.split; ++rr)
+          if (p.has_cache || tc0.t + rr - (p.kt - 1) >= 0) live |= 1u << rr;
+        const bool own_live = (live >> rank) & 1u;
+        const int n0 = tc0.ntile * p.nt;
+        const int chunks_per_sub = p.nt / kXC;
         bool xok = true;
         for (int sbt = 0; sbt < SUB && xok; ++sbt) {
           const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                  static_cast<uint32_t>((buf * SUB + sbt) * p.nt);
-          for (int j0 = 0; j0 < p.nt; j0 += kXC, ++xk) {
+          const int h = tc0.h0 + r, w = tc0.w0 + sbt * kTW + c;
+          const bool valid = (h < p.h) && (w < p.w);
+          const size_t pix = ((static_cast<size_t>(tc0.n) * p.t + tc0.t) * p.h + h) * p.w + w;
+          for (int jc = 0; jc < chunks_per_sub; ++jc) {
+            const int j0 = jc * kXC;
+            // the last CTA (tap kt-1, the current frame) owns every chunk:
+            // the senders then run ahead of it by the receive slots
+            const int owner = p.split - 1;
+            uint32_t k;  // (counters in registers: no indexed local array)
+            if (owner == 0) k = xc0++;
+            else if (owner == 1) k = xc1++;
+            else if (owner == 2) k = xc2++;
+            else k = xc3++;
+            const uint32_t slot = k % kXSlots, ph = (k / kXSlots) & 1u;
             uint32_t raw[kXC];
-            if (!zero) {
+            if (owner != rank) {
+              // sender: this chunk's partial goes to its owner's slot
+              if (own_live) {
+                __syncwarp();
+                tmem_ld16_nowait(taddr + j0, raw);
+                tmem_wait_ld();
+                tmem_regs_after_wait<kXC>(raw);
+              }
+              uint32_t free_ok = 0;
+              if (lane == 0)
+                free_ok = mbar_wait_bounded_cluster(&x_free[(q * p.split + owner) * kXSlots + slot],
+                                                    ph ^ 1u, p.wait_limit_ns, p.status, 7)
+                              ? 1u
+                              : 0u;
+              free_ok = __shfl_sync(0xffffffffu, free_ok, 0);
+              if (!free_ok) {
+                xok = false;
+                break;
+              }
+              const uint32_t bar =
+                  mapa_shared(smem_u32(&x_ready[q * kXSlots + slot]), static_cast<uint32_t>(owner));
+              if (own_live) {
+                const int sidx = rank < owner ? rank : rank - 1;
+                const uint32_t dst = mapa_shared(x_lane(slot, sidx), static_cast<uint32_t>(owner));
+#pragma unroll
+                for (int u = 0; u < kXC / 4; ++u) st_async_v4(dst + u * 512u, raw + 4 * u, bar);
+              }
+              // every rank arrives once per chunk, live or not, so that no
+              // rank's barrier phases run ahead of another's
+              __syncwarp();
+              if (lane == 0) mbar_arrive_remote_relaxed(bar);
+              continue;
+            }
+            // owner: add the partials in a fixed order, then the epilogue
+            uint4 res[2];
+            if (p.epi == 1 && valid) {
+              const uint4 *rr = reinterpret_cast<const uint4 *>(p.residual + pix * p.c_out + n0 + j0);
+              res[0] = rr[0];
+              res[1] = rr[1];
+            }
+            if (own_live) {
               __syncwarp();
               tmem_ld16_nowait(taddr + j0, raw);
-              tmem_wait_ld();
-              tmem_regs_after_wait<kXC>(raw);
             }
-            if (sbt == SUB - 1 && j0 + kXC >= p.nt) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&acc_empty[buf]);
-            }
-            const uint32_t slot = xk % kXSlots, ph = (xk / kXSlots) & 1u;
-            uint32_t free_ok = 0;
-            if (lane == 0)
-              free_ok = mbar_wait_bounded_cluster(&x_free[q * kXSlots + slot], ph ^ 1u,
-                                                  p.wait_limit_ns, p.status, 7)
-                            ? 1u
-                            : 0u;
-            free_ok = __shfl_sync(0xffffffffu, free_ok, 0);
-            if (!free_ok) {
-              xok = false;
-              break;
-            }
-            if (!zero) {
-              const uint32_t dst = mapa_shared(x_lane(slot, rank), static_cast<uint32_t>(leader));
-              const uint32_t bar = mapa_shared(smem_u32(&x_ready[q * kXSlots + slot]),
-                                               static_cast<uint32_t>(leader));
-#pragma unroll
-              for (int u = 0; u < kXC / 4; ++u) st_async_v4(dst + u * 512u, raw + 4 * u, bar);
-            }
-          }
-        }
-        if (!xok) break;
-        continue;
-      }
-      if (split) {
-        // ---- leader: fold the senders' partial sums into this accumulator,
-        // in a fixed order (own tap, then taps kt-2 .. 0), so that every call
-        // over the same frames gives the same bits.
-        int n_live = 0;  // senders whose tap is not a causal zero frame
-        for (int sr = 0; sr < n_send; ++sr)
-          n_live += (!p.has_cache && tc0.t + sr - (p.kt - 1) < 0) ? 0 : 1;
-        bool xok = true;
-        for (int sbt = 0; sbt < SUB && xok; ++sbt) {
-          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                 static_cast<uint32_t>((buf * SUB + sbt) * p.nt);
-          for (int j0 = 0; j0 < p.nt; j0 += kXC, ++xk) {
-            const uint32_t slot = xk % kXSlots, ph = (xk / kXSlots) & 1u;
-            uint32_t raw[kXC];
-            __syncwarp();
-            tmem_ld16_nowait(taddr + j0, raw);
             uint32_t ready = 0;
             if (lane == 0) {
               mbar_arrive_expect_tx(&x_ready[q * kXSlots + slot],
-                                    static_cast<uint32_t>(n_live) * kXPieceBytes);
+                                    static_cast<uint32_t>(__popc(live & ~(1u << rank))) *
+                                        kXPieceBytes);
               ready = mbar_wait_bounded_cluster(&x_ready[q * kXSlots + slot], ph, p.wait_limit_ns,
                                                 p.status, 8)
                           ? 1u
                           : 0u;
             }
             ready = __shfl_sync(0xffffffffu, ready, 0);
-            tmem_wait_ld();
-            tmem_regs_after_wait<kXC>(raw);
+            if (own_live) {
+              tmem_wait_ld();
+              tmem_regs_after_wait<kXC>(raw);
+            }
             if (!ready) {
               xok = false;
               break;
             }
-            for (int src_rank = leader - 1; src_rank >= 0; --src_rank) {
-              if (!p.has_cache && tc0.t + src_rank - (p.kt - 1) < 0) continue;  // no partial
-              const uint32_t src = x_lane(slot, src_rank);
+            float v[kXC];
+            bool first = true;
+            for (int src_rank = p.split - 1; src_rank >= 0; --src_rank) {
+              if (!((live >> src_rank) & 1u)) continue;  // no partial: a causal zero frame
+              float t16[kXC];
+              if (src_rank == rank) {
 #pragma unroll
-              for (int u = 0; u < kXC / 4; ++u) {
-                float4 f;
-                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                             : "=f"(f.x), "=f"(f.y), "=f"(f.z), "=f"(f.w)
-                             : "r"(src + u * 512u)
-                             : "memory");
-                raw[4 * u] = __float_as_uint(__uint_as_float(raw[4 * u]) + f.x);
-                raw[4 * u + 1] = __float_as_uint(__uint_as_float(raw[4 * u + 1]) + f.y);
-                raw[4 * u + 2] = __float_as_uint(__uint_as_float(raw[4 * u + 2]) + f.z);
-                raw[4 * u + 3] = __float_as_uint(__uint_as_float(raw[4 * u + 3]) + f.w);
+                for (int i = 0; i < kXC; ++i) t16[i] = __uint_as_float(raw[i]);
+              } else {
+                const uint32_t src = x_lane(slot, src_rank < rank ? src_rank : src_rank - 1);
+#pragma unroll
+                for (int u = 0; u < kXC / 4; ++u)
+                  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                               : "=f"(t16[4 * u]), "=f"(t16[4 * u + 1]), "=f"(t16[4 * u + 2]),
+                                 "=f"(t16[4 * u + 3])
+                               : "r"(src + u * 512u)
+                               : "memory");
               }
+#pragma unroll
+              for (int i = 0; i < kXC; ++i) v[i] = first ? t16[i] : v[i] + t16[i];
+              first = false;
             }
             // the slot's values are in registers: the senders may refill it
             __syncwarp();
             if (lane == 0)
-              for (int dst_rank = 0; dst_rank < leader; ++dst_rank)
-                mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&x_free[q * kXSlots + slot]),
-                                                       static_cast<uint32_t>(dst_rank)));
-            __syncwarp();
-            tmem_st16(taddr + j0, raw);
+              for (int dst_rank = 0; dst_rank < p.split; ++dst_rank)
+                if (dst_rank != rank)
+                  mbar_arrive_remote_relaxed(
+                      mapa_shared(smem_u32(&x_free[(q * p.split + rank) * kXSlots + slot]),
+                                  static_cast<uint32_t>(dst_rank)));
+#pragma unroll
+            for (int i = 0; i < kXC; ++i) v[i] += p.bias[n0 + j0 + i];
+            if (p.epi == 1 && valid) {
+              const __nv_bfloat16 *rb0 = reinterpret_cast<const __nv_bfloat16 *>(&res[0]);
+              const __nv_bfloat16 *rb1 = reinterpret_cast<const __nv_bfloat16 *>(&res[1]);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                v[i] += __bfloat162float(rb0[i]);
+                v[8 + i] += __bfloat162float(rb1[i]);
+              }
+            }
+            if (valid) {
+              uint4 o0, o1;
+              o0.x = pack_bf16x2(v[0], v[1]);
+              o0.y = pack_bf16x2(v[2], v[3]);
+              o0.z = pack_bf16x2(v[4], v[5]);
+              o0.w = pack_bf16x2(v[6], v[7]);
+              o1.x = pack_bf16x2(v[8], v[9]);
+              o1.y = pack_bf16x2(v[10], v[11]);
+              o1.z = pack_bf16x2(v[12], v[13]);
+              o1.w = pack_bf16x2(v[14], v[15]);
+              uint4 *dst = reinterpret_cast<uint4 *>(p.y + pix * p.c_out + n0 + j0);
+              dst[0] = o0;
+              dst[1] = o1;
+            }
           }
         }
+        // every tensor-memory read of this tile is done
+        tc_fence_before();
         __syncwarp();
-        tmem_wait_st();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
         if (!xok) break;
+        continue;
       }
       for (int sbt = 0; sbt < SUB; ++sbt) {
         const int h = tc0.h0 + r, w = tc0.w0 + sbt * kTW + c;
@@ -697,10 +750,11 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
   // Temporal split: when even kt CTAs per tile fit one wave, a frame has too
   // few tiles to occupy the GPU (a one-frame chunk of a latent-resolution
   // decoder layer), and its time is the length of one tile's K loop.  Each
-  // CTA of a cluster of kt then runs one temporal tap, and the last sums the
-  // partials through distributed shared memory before its epilogue.  Like
-  // the rest, decided from (n, c, h, w), never from t.
-  if (kt >= 2 && kt <= 4) {
+  // CTA of a cluster of kt then runs one temporal tap, and the partial sums
+  // meet through distributed shared memory, each chunk of columns in one of
+  // the CTAs.  Not with the RMS epilogue, which needs whole rows in one CTA.
+  // Like the rest, decided from (n, c, h, w), never from t.
+  if (kt >= 2 && kt <= 4 && !rms_epi && cfg->sub == 1) {
     UmmaConfig sp = *cfg;
     sp.split = kt;
     const long long tiles = static_cast<long long>(n) * ((h + kTH - 1) / kTH) *
@@ -804,7 +858,8 @@ cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_ca
                                        args.sub, args.split);
   if (smem > 227 * 1024 || (args.sub != 1 && args.sub != 2) || args.nbuf < 1 || args.nbuf > 2)
     return cudaErrorInvalidValue;
-  if (args.split != 1 && (args.split != args.kt || args.split > 4 || grid % args.split != 0))
+  if (args.split != 1 && (args.split != args.kt || args.split > 4 || grid % args.split != 0 ||
+                          args.epi == 2 || args.sub != 1))
     return cudaErrorInvalidValue;
   UmmaKernel k = umma_kernel_for(kc, args.kh, args.sub);
   if (!k) return cudaErrorInvalidValue;
