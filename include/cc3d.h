@@ -120,6 +120,8 @@ typedef struct {
   int k_split;             /* CTAs sharing one output tile, one temporal tap
                               each, summed in one of them: 1, or kt for
                               frames too small to occupy the GPU            */
+  int mma_ctas;            /* CTAs (SMs) per tensor-core MMA: 1, or 2 for a
+                              CTA pair issuing 2-SM MMAs (M = 256)          */
 } cc3d_stats;
 
 typedef struct cc3d_plan cc3d_plan;

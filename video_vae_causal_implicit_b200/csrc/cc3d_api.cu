@@ -153,6 +153,21 @@ bool encode_activation_map(CUtensorMap *m, const void *base, int c, int w, int h
   return encode_act_map(m, base, c, w, h, t, n, box_w, box_h, box_c);
 }
 
+// 2-D bf16 tensor map over a weight image of `rows` rows of 64 channels
+// (128 bytes): boxes of box_rows rows, 128-byte swizzled.
+bool encode_weight_map(CUtensorMap *m, const void *img, long long rows, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn || rows < 1 || box_rows < 1 || box_rows > 256) return false;
+  cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(img), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace cc3d
 
 using namespace cc3d;
@@ -163,6 +178,8 @@ struct cc3d_plan {
   int device;
   // UMMA
   int kc, nt, n_ntiles, na, nb, tmem_cols, sm_count, ctas_per_sm, sub, nbuf, split, max_clusters;
+  int pair;
+  CUtensorMap map_w;  // pair: the weight image as 128-byte swizzled rows
   uint8_t *wimg;
   // fp32 / thin
   void *wraw;
@@ -282,6 +299,7 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
   std::memset(&p->st, 0, sizeof(p->st));
   p->st.variant = variant;
   p->st.k_split = 1;
+  p->st.mma_ctas = 1;
   const int taps = desc->kt * desc->kh * desc->kw;
   cudaError_t e = cudaSuccess;
   if ((s = copy_vec(&p->bias, desc->bias, desc->c_out, true)) != CC3D_OK) goto fail;
@@ -350,9 +368,9 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
       }
       p->kc = cfg.kc; p->nt = cfg.nt; p->n_ntiles = cfg.n_ntiles; p->sub = cfg.sub;
       p->nbuf = cfg.nbuf; p->na = cfg.na; p->nb = cfg.nb; p->tmem_cols = cfg.tmem_cols;
-      p->ctas_per_sm = cfg.ctas_per_sm; p->split = cfg.split;
+      p->ctas_per_sm = cfg.ctas_per_sm; p->split = cfg.split; p->pair = cfg.pair;
       p->max_clusters = 0;
-      if (cfg.split > 1) {
+      if (cfg.split > 1 || cfg.pair) {
         p->max_clusters = umma_max_clusters(cfg, desc->kh);
         if (p->max_clusters < 1) { s = CC3D_ERR_CUDA; goto fail; }
       }
@@ -362,12 +380,19 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
     p->st.n_tile = p->nt;
     p->st.k_chunk = p->kc;
     p->st.k_split = p->split;
+    p->st.mma_ctas = p->pair ? 2 : 1;
     const size_t bytes = sizeof(__nv_bfloat16) * desc->c_out * desc->c_in * taps;
     if (cudaMalloc(&p->wimg, bytes) != cudaSuccess) { s = CC3D_ERR_OOM; goto fail; }
     e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(desc->weight), p->wimg,
-                           desc->c_out, desc->c_in, taps, p->nt, p->kc, 0);
+                           desc->c_out, desc->c_in, taps, p->nt, p->kc, p->pair, 0);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
+    if (p->pair && !encode_weight_map(&p->map_w, p->wimg,
+                                      static_cast<long long>(desc->c_out) * taps * (desc->c_in / 64),
+                                      p->nt / 2)) {
+      s = CC3D_ERR_CUDA;
+      goto fail;
+    }
   }
   *out = p;
   return CC3D_OK;
@@ -493,7 +518,9 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
   } else {
     CUtensorMap mx, mc;
     const int tile_w = umma_tile_w() * p->sub;
-    const int box_w = umma_halo_box_w(p->kc, p->sub, d.kw), box_h = umma_tile_h() + d.kh - 1;
+    // (a pair's CTA loads the halo of its own 8-column half)
+    const int box_w = umma_halo_box_w(p->kc, p->pair ? 1 : p->sub, d.kw);
+    const int box_h = umma_tile_h() + d.kh - 1;
     const int box_c = umma_halo_box_c(p->kc);
     if (!encode_act_map(&mx, x, d.c_in, d.w, d.h, t, d.n, box_w, box_h, box_c))
       return reject(CC3D_ERR_CUDA);
@@ -515,7 +542,7 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
     a.n = d.n; a.t = t; a.h = d.h; a.w = d.w; a.c_in = d.c_in; a.c_out = d.c_out;
     a.kt = d.kt; a.kh = d.kh; a.kw = d.kw; a.pad_h = d.pad_h; a.pad_w = d.pad_w;
     a.nt = p->nt; a.n_ntiles = p->n_ntiles;
-    a.sub = p->sub; a.nbuf = p->nbuf; a.split = p->split;
+    a.sub = p->sub; a.nbuf = p->nbuf; a.split = p->split; a.pair = p->pair;
     a.tiles_w = (d.w + tile_w - 1) / tile_w;
     a.tiles_h = (d.h + umma_tile_h() - 1) / umma_tile_h();
     a.na = p->na; a.nb = p->nb; a.tmem_cols = p->tmem_cols;
@@ -523,15 +550,17 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
     a.has_cache = (cache_in && front > 0) ? 1 : 0;
     tiles = static_cast<uint64_t>(d.n) * t * a.tiles_h * a.tiles_w * a.n_ntiles;
     uint64_t grid;
-    if (p->split > 1) {
-      // one cluster of `split` CTAs per tile, at most as many as fit at once
+    if (p->split > 1 || p->pair) {
+      // one cluster (of `split` CTAs, or a pair) per tile, at most as many as
+      // fit at once
       const uint64_t clusters = static_cast<uint64_t>(p->max_clusters);
-      grid = (tiles < clusters ? tiles : clusters) * p->split;
+      grid = (tiles < clusters ? tiles : clusters) * (p->pair ? 2 : p->split);
     } else {
       const uint64_t slots = static_cast<uint64_t>(p->sm_count) * p->ctas_per_sm;
       grid = tiles < slots ? tiles : slots;
     }
-    e = launch_conv_umma(mx, mc, a, p->kc, static_cast<unsigned>(grid), stream);
+    e = launch_conv_umma(mx, mc, p->pair ? p->map_w : mx, a, p->kc, static_cast<unsigned>(grid),
+                         stream);
     count_launch();
   }
   if (e == cudaSuccess && cache_out && front > 0)

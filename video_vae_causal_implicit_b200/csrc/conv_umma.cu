@@ -102,7 +102,7 @@ __host__ __device__ inline int halo_cols(int kc, int sub, int kw) {
 }
 
 __host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw, int na, int nb,
-                                                  int sub, int split) {
+                                                  int sub, int split, bool pair = false) {
   SmemLayout L;
   const uint32_t hh = kTH + kh - 1, hw = static_cast<uint32_t>(halo_cols(kc, sub, kw));
   if (uses_sw128(kc)) {
@@ -112,7 +112,8 @@ __host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw
     L.slab = round_up(hh * hw * 16u, 128u);
     L.a_stage = (kc / 8) * L.slab;
   }
-  L.b_stage = static_cast<uint32_t>(nt) * kc * 2u;
+  // (a CTA pair: this CTA's half of the N rows, 128-byte swizzled rows)
+  L.b_stage = static_cast<uint32_t>(pair ? nt / 2 : nt) * kc * 2u;
   L.na = na;
   L.nb = nb;
   L.a_off = 0;
@@ -146,16 +147,18 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, const UmmaArgs &p) {
   return c;
 }
 
-template <int KC, int KS, int SUB>
+template <int KC, int KS, int SUB, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     conv_umma_kernel(const __grid_constant__ CUtensorMap map_x,
-                     const __grid_constant__ CUtensorMap map_cache, UmmaArgs p) {
+                     const __grid_constant__ CUtensorMap map_cache,
+                     const __grid_constant__ CUtensorMap map_w, UmmaArgs p) {
+  static_assert(!PAIR || (SUB == 1 && uses_sw128(KC)), "CTA pairs take 64-channel chunks");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // Align the dynamic shared window to 1 KiB ourselves (the attribute is a
   // request, not a guarantee).
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const SmemLayout L = make_layout(KC, p.nt, KS, KS, p.na, p.nb, SUB, p.split);
+  const SmemLayout L = make_layout(KC, p.nt, KS, KS, p.na, p.nb, SUB, p.split, PAIR);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
   uint64_t *full_a = bars;
   uint64_t *empty_a = full_a + L.na;
@@ -179,9 +182,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   // in the chunk's owner, which adds them in a fixed order (tap kt-1 -- the
   // current frame, never a causal zero frame -- then kt-2 .. 0) and runs the
   // epilogue for those columns.
-  const int rank = split ? static_cast<int>(cluster_ctarank()) : 0;
-  const int cid = split ? static_cast<int>(blockIdx.x) / p.split : static_cast<int>(blockIdx.x);
-  const int ncl = split ? static_cast<int>(gridDim.x) / p.split : static_cast<int>(gridDim.x);
+  //
+  // With PAIR, a cluster of two CTAs (on one SM pair) takes a 16 x 16 pixel
+  // tile: CTA `rank` holds the 8 x 16 half at columns 8 * rank and half of
+  // each weight stage's N rows, and the leader (rank 0) issues M = 256
+  // tcgen05 MMAs over both CTAs' shared memory into both CTAs' tensor memory.
+  const int csize = PAIR ? 2 : p.split;
+  const int rank = (split || PAIR) ? static_cast<int>(cluster_ctarank()) : 0;
+  const int cid = static_cast<int>(blockIdx.x) / csize;
+  const int ncl = static_cast<int>(gridDim.x) / csize;
+  const bool pair_leader = !PAIR || rank == 0;
   const int kt_lo = split ? rank : 0;
   const int n_kt = split ? 1 : p.kt;
 
@@ -205,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], kEpiWarps);
+      mbar_init(&acc_empty[i], PAIR ? 2 * kEpiWarps : kEpiWarps);  // (pair: both CTAs)
     }
     mbar_init(drain, 1);
     if (split) {
@@ -215,15 +225,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     prefetch_tmap(&map_x);
     if (p.has_cache) prefetch_tmap(&map_cache);
+    if (PAIR) prefetch_tmap(&map_w);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, p.tmem_cols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, p.tmem_cols);  // same columns in both CTAs
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, p.tmem_cols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  // (with a split, no CTA may arrive on a peer's barriers before the peer
+  // (in a cluster, no CTA may arrive on a peer's barriers before the peer
   // has initialised them)
-  if (split)
+  if (split || PAIR)
     cluster_sync();
   else
     __syncthreads();
@@ -236,6 +252,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------ producer ------------------------------------
     if (lane == 0) {
       const uint32_t a_tx = kSw ? L.a_stage : (KC / 8) * (16u * halo_w * (kTH + KS - 1));
+      // PAIR: both CTAs' loads complete on the leader's full barriers, which
+      // the leader arms for the bytes of both halves
+      const uint32_t lead_full_a = PAIR ? mapa_shared(smem_u32(full_a), 0u) : 0u;
+      const uint32_t lead_full_b = PAIR ? mapa_shared(smem_u32(full_b), 0u) : 0u;
       int sa = 0, sb = 0;
       uint32_t pa = 0, pb = 0;
       // stages issued at least once, and the phase parity of their last issue
@@ -253,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full_a[sa], a_tx);
+          if (pair_leader) mbar_arrive_expect_tx(&full_a[sa], PAIR ? 2u * a_tx : a_tx);
           a_used |= 1u << sa;
           a_par = (a_par & ~(1u << sa)) | (pa << sa);
           const int tau = tc0.t + kt - (p.kt - 1);
@@ -261,7 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const CUtensorMap *map = from_cache ? &map_cache : &map_x;
           const int tcoord = from_cache ? tau + (p.kt - 1) : tau;
           const uint32_t dst = smem_base + L.a_off + sa * L.a_stage;
-          if constexpr (kSw) {
+          if constexpr (PAIR) {
+            tma_load_5d_pair(dst, map, lead_full_a + 8u * sa, cc * KC,
+                             tc0.w0 + kTW * rank - KS / 2, tc0.h0 - KS / 2, tcoord, tc0.n);
+          } else if constexpr (kSw) {
             tma_load_5d(dst, map, &full_a[sa], cc * KC, tc0.w0 - KS / 2, tc0.h0 - KS / 2, tcoord,
                         tc0.n);
           } else {
@@ -277,18 +300,31 @@ __global__ void __launch_bounds__(kThreads, 1)
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(&full_b[sb], L.b_stage);
+            if (pair_leader) mbar_arrive_expect_tx(&full_b[sb], PAIR ? 2u * L.b_stage : L.b_stage);
             b_used |= 1u << sb;
             b_par = (b_par & ~(1u << sb)) | (pb << sb);
             const size_t stage_idx = static_cast<size_t>(kt * KS * KS + ts) * n_cc + cc;
-            bulk_load(smem_base + L.b_off + sb * L.b_stage, wsrc + stage_idx * L.b_stage,
-                      L.b_stage, &full_b[sb]);
+            if constexpr (PAIR) {
+              // rows of the weight image [ntile][tap][cchunk][NT][64]: this
+              // CTA's half of the stage's N rows
+              const int row = static_cast<int>(
+                  ((static_cast<size_t>(tc0.ntile) * p.kt * KS * KS * n_cc + stage_idx) * p.nt) +
+                  rank * (p.nt / 2));
+              tma_load_2d_pair(smem_base + L.b_off + sb * L.b_stage, &map_w, lead_full_b + 8u * sb,
+                               0, row);
+            } else {
+              bulk_load(smem_base + L.b_off + sb * L.b_stage, wsrc + stage_idx * L.b_stage,
+                        L.b_stage, &full_b[sb]);
+            }
             if (++sb == L.nb) { sb = 0; pb ^= 1; }
           }
         }
       }
       // Drain: every load this thread issued lands before the CTA may exit
       // (after a timeout elsewhere the consumer may not have waited for it).
+      // A pair's leader drains for both CTAs: their loads complete on its
+      // barriers, and the follower waits at the final cluster barrier.
+      if (!pair_leader) a_used = b_used = 0;
       for (int i = 0; i < L.na; ++i)
         if (a_used >> i & 1u)
           mbar_wait_bounded(&full_a[i], a_par >> i & 1u, kDrainLimitNs, nullptr, 0);
@@ -298,8 +334,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ----------------------------------
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kM, p.nt);
+    // (a pair's follower issues nothing: the leader's MMAs cover both CTAs)
+    if (lane == 0 && pair_leader) {
+      const uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * kM : kM, p.nt);
       const uint32_t b_lbo = static_cast<uint32_t>(p.nt) * 16u;
       // Descriptors of stage 0; other stages, taps, sub-tiles and K steps
       // only move the start address (low 14 bits, 16-byte units), so they
@@ -309,9 +346,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t adesc0 =
           kSw ? smem_desc_sw128(smem_base + L.a_off, halo_w * 128u)
               : smem_desc_noswizzle(smem_base + L.a_off, L.slab, halo_w * 16u);
-      const uint64_t bdesc0 = smem_desc_noswizzle(smem_base + L.b_off, b_lbo, 128u);
+      // B: [NT][KC/8][8] no-swizzle core matrices, or (pair) this CTA's
+      // NT/2 rows of 128 swizzled bytes
+      const uint64_t bdesc0 = PAIR ? smem_desc_sw128(smem_base + L.b_off, 1024u)
+                                   : smem_desc_noswizzle(smem_base + L.b_off, b_lbo, 128u);
       const uint32_t astep16 = kSw ? 2u : 2u * (L.slab >> 4);
-      const uint32_t bstep16 = 2u * (b_lbo >> 4);
+      const uint32_t bstep16 = PAIR ? 2u : 2u * (b_lbo >> 4);
       const uint32_t pix16 = kSw ? 8u : 1u;
       int sa = 0, sb = 0;
       uint32_t pa = 0, pb = 0;
@@ -319,8 +359,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = cid; tile < n_tiles && ok; tile += ncl, ++it) {
         const int buf = it % p.nbuf;
         const uint32_t use_par = static_cast<uint32_t>((it / p.nbuf) & 1);
-        // wait until the epilogue has drained this accumulator buffer
-        if (!mbar_wait_bounded(&acc_empty[buf], use_par ^ 1, p.wait_limit_ns, p.status, 6)) {
+        // wait until the epilogue (of both CTAs of a pair) has drained this
+        // accumulator buffer
+        if (!(PAIR ? mbar_wait_bounded_cluster(&acc_empty[buf], use_par ^ 1, p.wait_limit_ns,
+                                               p.status, 6)
+                   : mbar_wait_bounded(&acc_empty[buf], use_par ^ 1, p.wait_limit_ns, p.status,
+                                       6))) {
           ok = false;
           break;
         }
@@ -353,21 +397,32 @@ __global__ void __launch_bounds__(kThreads, 1)
               // every sub-tile (8 pixels further along the halo row) reuses
               // this weight stage
 #pragma unroll
-              for (int sbt = 0; sbt < SUB; ++sbt)
-                umma_bf16(d_tmem + sbt * p.nt, a_tap + sbt * kTW * pix16 + j * astep16,
-                          b_st + j * bstep16, idesc, accumulate);
+              for (int sbt = 0; sbt < SUB; ++sbt) {
+                if constexpr (PAIR)
+                  umma_bf16_pair(d_tmem, a_tap + j * astep16, b_st + j * bstep16, idesc,
+                                 accumulate);
+                else
+                  umma_bf16(d_tmem + sbt * p.nt, a_tap + sbt * kTW * pix16 + j * astep16,
+                            b_st + j * bstep16, idesc, accumulate);
+              }
               accumulate = 1;
             }
-            umma_commit(&empty_b[sb]);  // frees the B stage when these MMAs finish
+            // frees the B stage (in both CTAs of a pair) when these MMAs finish
+            if constexpr (PAIR) umma_commit_pair(&empty_b[sb], 3);
+            else umma_commit(&empty_b[sb]);
             if (++sb == L.nb) { sb = 0; pb ^= 1; }
           }
-          umma_commit(&empty_a[sa]);
+          if constexpr (PAIR) umma_commit_pair(&empty_a[sa], 3);
+          else umma_commit(&empty_a[sa]);
           if (++sa == L.na) { sa = 0; pa ^= 1; }
         }
-        umma_commit(&acc_full[buf]);  // accumulator ready for the epilogue
+        // accumulator ready for the epilogue(s)
+        if constexpr (PAIR) umma_commit_pair(&acc_full[buf], 3);
+        else umma_commit(&acc_full[buf]);
       }
       // Drain: all MMAs issued here are complete before tensor memory is freed.
-      umma_commit(drain);
+      if constexpr (PAIR) umma_commit_pair(drain, 1);
+      else umma_commit(drain);
       mbar_wait_bounded(drain, 0, kDrainLimitNs, nullptr, 0);
     }
   } else {
@@ -552,7 +607,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       for (int sbt = 0; sbt < SUB; ++sbt) {
-        const int h = tc0.h0 + r, w = tc0.w0 + sbt * kTW + c;
+        // (a pair's CTA holds the 8 columns at 8 * rank of the 16-wide tile)
+        const int h = tc0.h0 + r, w = tc0.w0 + (PAIR ? rank : sbt) * kTW + c;
         const bool valid = (h < p.h) && (w < p.w);
         const bool last_sub = sbt == SUB - 1;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
@@ -608,10 +664,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           tmem_regs_after_wait<48>(raw);
           if (last_sub && j0 + 48 >= p.nt) {
-            // last read of this accumulator buffer: hand it back to the MMA warp
+            // last read of this accumulator buffer: hand it back to the MMA
+            // warp (a pair's follower: to the leader's)
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            if (lane == 0) {
+              if (PAIR && rank != 0)
+                mbar_arrive_remote(mapa_shared(smem_u32(&acc_empty[buf]), 0u));
+              else
+                mbar_arrive(&acc_empty[buf]);
+            }
           }
 #pragma unroll
           for (int u = 0; u < 3; ++u) {
@@ -658,56 +720,79 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  // no CTA leaves while a peer may still read its staging or arrive on its
-  // barriers
-  if (split) cluster_sync();
+  // no CTA leaves while a peer may still write its shared or tensor memory
+  // or arrive on its barriers
+  if (split || PAIR) cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, p.tmem_cols);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, p.tmem_cols);
+    else
+      tmem_dealloc(tmem_base, p.tmem_cols);
   }
 }
 
 }  // namespace
 
-size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb, int sub, int split) {
-  return make_layout(kc, nt, kh, kw, na, nb, sub, split).total + 1024;  // + alignment slack
+size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb, int sub, int split,
+                       int pair) {
+  // (a pair's CTA holds one 8 x 16 MMA tile: sub counts tile widths)
+  return make_layout(kc, nt, kh, kw, na, nb, pair ? 1 : sub, split, pair != 0).total +
+         1024;  // + alignment slack
 }
 
 namespace {
-// Buffers, pipeline depths and residency of one (sub, nt) tile shape.
+// Buffers, pipeline depths and residency of one tile shape.
 bool finish_config(int ks, UmmaConfig &c) {
-  c.nbuf = (2 * c.sub * c.nt <= 512) ? 2 : 1;  // double-buffered accumulators when they fit
+  const int cta_sub = c.pair ? 1 : c.sub;  // MMA tiles whose accumulators one CTA holds
+  c.nbuf = (2 * cta_sub * c.nt <= 512) ? 2 : 1;  // double-buffered accumulators when they fit
   c.tmem_cols = 32;
-  while (c.tmem_cols < c.nbuf * c.sub * c.nt) c.tmem_cols *= 2;
+  while (c.tmem_cols < c.nbuf * cta_sub * c.nt) c.tmem_cols *= 2;
   if (c.tmem_cols > 512) return false;
   c.na = 2;
   c.nb = 8;
   // (a split's exchange staging gets room of its own above the usual budget)
   const size_t budget = (c.split > 1 ? 216 : 200) * 1024;
-  while (c.nb > 2 && umma_smem_bytes(c.kc, c.nt, ks, ks, c.na, c.nb, c.sub, c.split) > budget)
+  while (c.nb > 2 &&
+         umma_smem_bytes(c.kc, c.nt, ks, ks, c.na, c.nb, c.sub, c.split, c.pair) > budget)
     --c.nb;
   int per_sm = static_cast<int>(
       (228 * 1024) /
-      (umma_launch_smem(c.kc, c.nt, ks, c.na, c.nb, c.tmem_cols, c.sub, c.split) + 1024));
+      (umma_launch_smem(c.kc, c.nt, ks, c.na, c.nb, c.tmem_cols, c.sub, c.split, c.pair) +
+       1024));
   if (per_sm > 512 / c.tmem_cols) per_sm = 512 / c.tmem_cols;
   if (per_sm > 2) per_sm = 2;
+  if (c.pair) per_sm = 1;
   c.ctas_per_sm = per_sm < 1 ? 1 : per_sm;
   return true;
 }
 
-// Relative time of one frame of n images: whole waves of CTA tiles, each
-// wave as long as one tile's MMAs -- sub MMAs of 128 x nt x 16 per K step,
-// at the issue times measured on B200 (48 cycles up to N = 64, 56 up to
-// N = 96, N / 2 beyond) -- times the CTAs that share an SM's tensor core
-// once the tiles outnumber the SMs.
+// Cycles one SM spends on one 128-pixel x nt x 16 MMA step, from the two
+// limits measured on B200: the tensor pipe's issue time (48 cycles up to
+// N = 64, 56 up to 96, N / 2 beyond) and shared-memory traffic at ~120
+// bytes per cycle -- the MMA's operand reads (A: 4 KiB; B: nt x 32 bytes,
+// or half of it on a CTA pair) plus the TMA writes of the weights (a stage
+// is written once per CTA and shared by its sub-tiles) and of the halo.
+long long mma_cycles(const UmmaConfig &c) {
+  const long long math = c.nt <= 64 ? 48 : c.nt <= 96 ? 56 : c.nt / 2;
+  const long long b_rows = c.pair ? c.nt / 2 : c.nt;
+  const long long b_read = 32 * b_rows;
+  const long long b_write = 32 * b_rows / (c.pair ? 1 : c.sub);
+  const long long bytes = 4096 + b_read + b_write + 1000;
+  const long long smem = (bytes + 119) / 120;
+  return math > smem ? math : smem;
+}
+
+// Relative time of one frame of n images: whole waves of tiles over the
+// GPU (SMs, or SM pairs for a pair), each as long as one tile's MMA steps.
 long long frame_cost(const UmmaConfig &c, int n, int h, int w, int sm_count) {
   const long long tiles = static_cast<long long>(n) * ((h + kTH - 1) / kTH) *
                           ((w + c.sub * kTW - 1) / (c.sub * kTW)) * c.n_ntiles;
-  const long long slots = static_cast<long long>(sm_count) * c.ctas_per_sm;
-  const long long cyc = c.nt <= 64 ? 48 : c.nt <= 96 ? 56 : c.nt / 2;
-  const long long share = tiles > sm_count ? c.ctas_per_sm : 1;
-  return (tiles + slots - 1) / slots * share * c.sub * cyc;
+  const long long slots = c.pair ? sm_count / 2 : static_cast<long long>(sm_count) * c.ctas_per_sm;
+  const long long share = (!c.pair && tiles > sm_count) ? c.ctas_per_sm : 1;
+  const long long steps = c.pair ? 1 : c.sub;  // MMA steps per SM per K step
+  return (tiles + slots - 1) / slots * share * steps * mma_cycles(c);
 }
 }  // namespace
 
@@ -721,46 +806,67 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
       if (c_out % nt == 0 && (!rms_epi || nt == c_out)) return nt;
     return 0;
   };
+  // Every choice below depends on (n, c, h, w) -- never on t -- so streamed
+  // and whole-sequence calls run identical arithmetic.
   UmmaConfig one;
   one.kc = (c_in % 64 == 0) ? 64 : (c_in % 96 == 0) ? 96 : 32;
   one.sub = 1;
   one.split = 1;
+  one.pair = 0;
   one.nt = largest_nt(256);
   if (!one.nt) return false;
   one.n_ntiles = c_out / one.nt;
   if (!finish_config(ks, one)) return false;
   *cfg = one;
+  const long long tiles1 = static_cast<long long>(n) * ((h + kTH - 1) / kTH) *
+                           ((w + kTW - 1) / kTW) * one.n_ntiles;
+  // Temporal split: when even kt CTAs per tile fit one wave, a frame has too
+  // few tiles to occupy the GPU (a one-frame chunk of a latent-resolution
+  // decoder layer), and its time is the length of one tile's K loop.  Each
+  // CTA of a cluster of kt then runs one temporal tap, and the partial sums
+  // meet through distributed shared memory in the last CTA.  Not with the
+  // RMS epilogue, which needs whole rows in one CTA.
+  if (kt >= 2 && kt <= 4 && !rms_epi) {
+    UmmaConfig sp = one;
+    sp.split = kt;
+    if (finish_config(ks, sp) && tiles1 * kt <= static_cast<long long>(sm_count) * sp.ctas_per_sm) {
+      *cfg = sp;
+      return true;
+    }
+  }
+  long long best = frame_cost(one, n, h, w, sm_count);
   // Two sub-tiles (a 16 x 16 pixel CTA tile, two 8 x 16 MMA tiles) share
-  // every weight stage, halving the weight bytes that each MMA waits for.
-  // Only with N <= 128, where both sub-tiles still fit two accumulator
-  // buffers (a single buffer stalls the MMAs behind the epilogue), and only
-  // when the tile waves of one frame do not lose more than the ~5% that the
-  // halved weight traffic was measured to gain on B200.  The choice depends
-  // on (n, c, h, w) -- never on t -- so streamed and whole-sequence calls run
-  // identical arithmetic.
+  // every weight stage, halving the weight bytes written per MMA.  Only with
+  // N <= 128, where both sub-tiles still fit two accumulator buffers (a
+  // single buffer stalls the MMAs behind the epilogue).
   UmmaConfig two = one;
   two.sub = 2;
   two.nt = largest_nt(128);
   if (two.nt) {
     two.n_ntiles = c_out / two.nt;
-    if (finish_config(ks, two) && two.nbuf == 2 &&
-        20 * frame_cost(two, n, h, w, sm_count) <= 21 * frame_cost(one, n, h, w, sm_count))
-      *cfg = two;
+    if (finish_config(ks, two) && two.nbuf == 2) {
+      const long long cost = frame_cost(two, n, h, w, sm_count);
+      if (cost < best) {
+        best = cost;
+        *cfg = two;
+      }
+    }
   }
-  // Temporal split: when even kt CTAs per tile fit one wave, a frame has too
-  // few tiles to occupy the GPU (a one-frame chunk of a latent-resolution
-  // decoder layer), and its time is the length of one tile's K loop.  Each
-  // CTA of a cluster of kt then runs one temporal tap, and the partial sums
-  // meet through distributed shared memory, each chunk of columns in one of
-  // the CTAs.  Not with the RMS epilogue, which needs whole rows in one CTA.
-  // Like the rest, decided from (n, c, h, w), never from t.
-  if (kt >= 2 && kt <= 4 && !rms_epi && cfg->sub == 1) {
-    UmmaConfig sp = *cfg;
-    sp.split = kt;
-    const long long tiles = static_cast<long long>(n) * ((h + kTH - 1) / kTH) *
-                            ((w + sp.sub * kTW - 1) / (sp.sub * kTW)) * sp.n_ntiles;
-    if (finish_config(ks, sp) && tiles * kt <= static_cast<long long>(sm_count) * sp.ctas_per_sm)
-      *cfg = sp;
+  // A CTA pair (2-SM MMAs, M = 256): each SM holds half of every weight
+  // stage, which cuts the shared-memory traffic per MMA enough to reach the
+  // tensor pipe's own rate.  64-channel chunks (the 128-byte swizzled halo
+  // and weight rows).
+  if (one.kc == 64) {
+    UmmaConfig pr = one;
+    pr.pair = 1;
+    pr.sub = 2;  // the tile is two MMA tiles wide
+    if (finish_config(ks, pr) && pr.nbuf == 2) {
+      const long long cost = frame_cost(pr, n, h, w, sm_count);
+      if (cost <= best) {
+        best = cost;
+        *cfg = pr;
+      }
+    }
   }
   return true;
 }
@@ -772,10 +878,13 @@ int umma_tile_h() { return kTH; }
 
 template <int KC, int KS>
 cudaError_t set_smem_attr() {
-  cudaError_t e = cudaFuncSetAttribute(conv_umma_kernel<KC, KS, 1>,
+  cudaError_t e = cudaFuncSetAttribute(conv_umma_kernel<KC, KS, 1, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(conv_umma_kernel<KC, KS, 2>,
+    e = cudaFuncSetAttribute(conv_umma_kernel<KC, KS, 2, false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e == cudaSuccess && uses_sw128(KC))
+    e = cudaFuncSetAttribute(conv_umma_kernel<KC, KS, 1, uses_sw128(KC)>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   return e;
 }
@@ -792,8 +901,8 @@ cudaError_t umma_prepare() {
 }
 
 size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols, int sub,
-                        int split) {
-  size_t smem = umma_smem_bytes(kc, nt, ks, ks, na, nb, sub, split);
+                        int split, int pair) {
+  size_t smem = umma_smem_bytes(kc, nt, ks, ks, na, nb, sub, split, pair);
   // A CTA that holds more than half of tensor memory must have its SM to
   // itself; asking for more than half the shared memory guarantees that.
   if (tmem_cols > 256 && smem < 116 * 1024) smem = 116 * 1024;
@@ -801,12 +910,15 @@ size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols, i
 }
 
 namespace {
-using UmmaKernel = void (*)(const CUtensorMap, const CUtensorMap, UmmaArgs);
+using UmmaKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, UmmaArgs);
 
-UmmaKernel umma_kernel_for(int kc, int ks, int sub) {
-#define CC3D_PICK(KC_, KS_)                                                              \
-  if (kc == KC_ && ks == KS_)                                                            \
-    return sub == 2 ? conv_umma_kernel<KC_, KS_, 2> : conv_umma_kernel<KC_, KS_, 1>;
+UmmaKernel umma_kernel_for(int kc, int ks, int sub, int pair) {
+#define CC3D_PICK(KC_, KS_)                                                         \
+  if (kc == KC_ && ks == KS_) {                                                     \
+    if (pair) return uses_sw128(KC_) ? conv_umma_kernel<KC_, KS_, 1, uses_sw128(KC_)> : nullptr; \
+    return sub == 2 ? conv_umma_kernel<KC_, KS_, 2, false>                          \
+                    : conv_umma_kernel<KC_, KS_, 1, false>;                         \
+  }
   CC3D_PICK(64, 3)
   CC3D_PICK(32, 3)
   CC3D_PICK(96, 3)
@@ -817,7 +929,7 @@ UmmaKernel umma_kernel_for(int kc, int ks, int sub) {
   return nullptr;
 }
 
-cudaLaunchConfig_t umma_launch_config(unsigned grid, size_t smem, int split, cudaStream_t stream,
+cudaLaunchConfig_t umma_launch_config(unsigned grid, size_t smem, int csize, cudaStream_t stream,
                                       cudaLaunchAttribute *attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
@@ -825,24 +937,25 @@ cudaLaunchConfig_t umma_launch_config(unsigned grid, size_t smem, int split, cud
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   attr->id = cudaLaunchAttributeClusterDimension;
-  attr->val.clusterDim.x = static_cast<unsigned>(split);
+  attr->val.clusterDim.x = static_cast<unsigned>(csize);
   attr->val.clusterDim.y = 1;
   attr->val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = split > 1 ? 1 : 0;
+  cfg.numAttrs = csize > 1 ? 1 : 0;
   return cfg;
 }
 }  // namespace
 
 int umma_max_clusters(const UmmaConfig &c, int ks) {
-  if (c.split <= 1) return 0;
-  UmmaKernel k = umma_kernel_for(c.kc, ks, c.sub);
+  const int csize = c.pair ? 2 : c.split;
+  if (csize <= 1) return 0;
+  UmmaKernel k = umma_kernel_for(c.kc, ks, c.sub, c.pair);
   if (!k) return 0;
   const size_t smem =
-      umma_launch_smem(c.kc, c.nt, ks, c.na, c.nb, c.tmem_cols, c.sub, c.split);
+      umma_launch_smem(c.kc, c.nt, ks, c.na, c.nb, c.tmem_cols, c.sub, c.split, c.pair);
   cudaLaunchAttribute attr;
   const cudaLaunchConfig_t cfg =
-      umma_launch_config(static_cast<unsigned>(c.split), smem, c.split, nullptr, &attr);
+      umma_launch_config(static_cast<unsigned>(csize), smem, csize, nullptr, &attr);
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void *>(k), &cfg) != cudaSuccess) {
     (void)cudaGetLastError();
@@ -852,20 +965,24 @@ int umma_max_clusters(const UmmaConfig &c, int ks) {
 }
 
 cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_cache,
-                             const UmmaArgs &args, int kc, unsigned grid, cudaStream_t stream) {
+                             const CUtensorMap &map_w, const UmmaArgs &args, int kc,
+                             unsigned grid, cudaStream_t stream) {
   if (args.kh != args.kw || (args.kh != 1 && args.kh != 3)) return cudaErrorInvalidValue;
   const size_t smem = umma_launch_smem(kc, args.nt, args.kh, args.na, args.nb, args.tmem_cols,
-                                       args.sub, args.split);
+                                       args.sub, args.split, args.pair);
   if (smem > 227 * 1024 || (args.sub != 1 && args.sub != 2) || args.nbuf < 1 || args.nbuf > 2)
     return cudaErrorInvalidValue;
   if (args.split != 1 && (args.split != args.kt || args.split > 4 || grid % args.split != 0 ||
-                          args.epi == 2 || args.sub != 1))
+                          args.epi == 2 || args.sub != 1 || args.pair))
     return cudaErrorInvalidValue;
-  UmmaKernel k = umma_kernel_for(kc, args.kh, args.sub);
+  if (args.pair && (kc != 64 || args.sub != 2 || grid % 2 != 0 || args.nt % 16 != 0))
+    return cudaErrorInvalidValue;
+  UmmaKernel k = umma_kernel_for(kc, args.kh, args.sub, args.pair);
   if (!k) return cudaErrorInvalidValue;
   cudaLaunchAttribute attr;
-  const cudaLaunchConfig_t cfg = umma_launch_config(grid, smem, args.split, stream, &attr);
-  return cudaLaunchKernelEx(&cfg, k, map_x, map_cache, args);
+  const cudaLaunchConfig_t cfg =
+      umma_launch_config(grid, smem, args.pair ? 2 : args.split, stream, &attr);
+  return cudaLaunchKernelEx(&cfg, k, map_x, map_cache, map_w, args);
 }
 
 }  // namespace cc3d

@@ -31,12 +31,14 @@ struct UmmaArgs {
   int nbuf;                       // accumulator buffers in tensor memory: 1 or 2
   int split;                      // 1, or kt: CTAs of a cluster that share a tile, one
                                   // temporal tap each, reduced in the last one
+  int pair;                       // 1: a cluster of 2 CTAs runs 2-SM MMAs on a 16 x 16 px
+                                  // tile (sub is then 2: the tile width in MMA tiles)
 };
 
 // Tile configuration of the UMMA conv for a problem (chosen from n, c_in,
 // c_out, h, w and the epilogue -- never from t).
 struct UmmaConfig {
-  int kc, nt, n_ntiles, sub, nbuf, split, na, nb, tmem_cols, ctas_per_sm;
+  int kc, nt, n_ntiles, sub, nbuf, split, pair, na, nb, tmem_cols, ctas_per_sm;
 };
 bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
                         int sm_count, UmmaConfig *cfg);
@@ -44,24 +46,30 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
 // sizing the grid; 0 when the query fails.
 int umma_max_clusters(const UmmaConfig &cfg, int ks);
 
-size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb, int sub, int split);
+size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb, int sub, int split,
+                       int pair);
 cudaError_t umma_prepare();
 // Dynamic shared memory a launch requests (with the one-CTA-per-SM rule).
 size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols, int sub,
-                        int split);
+                        int split, int pair);
 int umma_tile_w();
 // TMA box of the A halo: columns (padded for the 128-byte swizzle) and
 // channels (64: swizzled pixel rows; 8: no-swizzle slabs).
 int umma_halo_box_w(int kc, int sub, int kw);
 int umma_halo_box_c(int kc);
 int umma_tile_h();
+// map_w: the weights' tensor map (plain-rows image) for pair launches; any
+// valid map otherwise (unused).
 cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_cache,
-                             const UmmaArgs &args, int kc, unsigned grid, cudaStream_t stream);
+                             const CUtensorMap &map_w, const UmmaArgs &args, int kc,
+                             unsigned grid, cudaStream_t stream);
 
 // Weight re-tiling for the UMMA kernel (plan time):
 // W[c_out][c_in][kt][kh][kw] (bf16) -> image[ntile][tap][cchunk][kc/8][nt][8].
+// rows: 0 = [ntile][tap][cchunk][kc/8][nt][8] (no-swizzle stage images for
+// a bulk copy), 1 = [ntile][tap][cchunk][nt][kc] (plain rows for a tensor map)
 cudaError_t launch_repack_umma(const __nv_bfloat16 *w, uint8_t *img, int c_out, int c_in,
-                               int taps, int nt, int kc, cudaStream_t stream);
+                               int taps, int nt, int kc, int rows, cudaStream_t stream);
 
 // Thin first-layer conv (c_in small): weights to [tap*c_in padded to kpad][c_out]
 // image and the kernel itself.
@@ -115,5 +123,8 @@ int *device_status_word();
 // plain or 64 swizzled channels).
 bool encode_activation_map(CUtensorMap *m, const void *base, int c, int w, int h, int t, int n,
                            int box_w, int box_h, int box_c);
+// 2-D tensor map over a plain-rows weight image (rows of 64 bf16), boxes of
+// box_rows rows, 128-byte swizzled.
+bool encode_weight_map(CUtensorMap *m, const void *img, long long rows, int box_rows);
 
 }  // namespace cc3d

@@ -23,19 +23,30 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 }
 
 __global__ void repack_umma_kernel(const __nv_bfloat16 *__restrict__ w, __nv_bfloat16 *img,
-                                   int c_out, int c_in, int taps, int nt, int kc) {
+                                   int c_out, int c_in, int taps, int nt, int kc, int rows) {
   const long long total = static_cast<long long>(c_out) * c_in * taps;
   const int n_cc = c_in / kc;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    // image order: ntile, tap, cchunk, slab (kc/8), row (nt), element (8)
+    // image order: ntile, tap, cchunk, then within the stage either
+    // slab (kc/8), row (nt), element (8)  -- no-swizzle core matrices -- or
+    // (rows) row (nt), channel (kc)       -- plain rows for a tensor map
     long long r = i;
-    const int e = r % 8;
-    r /= 8;
-    const int nl = r % nt;
-    r /= nt;
-    const int s = r % (kc / 8);
-    r /= (kc / 8);
+    int e, nl, s;
+    if (rows) {
+      e = r % kc;
+      r /= kc;
+      nl = r % nt;
+      r /= nt;
+      s = 0;
+    } else {
+      e = r % 8;
+      r /= 8;
+      nl = r % nt;
+      r /= nt;
+      s = r % (kc / 8);
+      r /= (kc / 8);
+    }
     const int cc = r % n_cc;
     r /= n_cc;
     const int tap = r % taps;
@@ -319,10 +330,10 @@ int grid_for(long long work, int block) {
 }  // namespace
 
 cudaError_t launch_repack_umma(const __nv_bfloat16 *w, uint8_t *img, int c_out, int c_in,
-                               int taps, int nt, int kc, cudaStream_t stream) {
+                               int taps, int nt, int kc, int rows, cudaStream_t stream) {
   const long long total = static_cast<long long>(c_out) * c_in * taps;
   repack_umma_kernel<<<grid_for(total, 256), 256, 0, stream>>>(
-      w, reinterpret_cast<__nv_bfloat16 *>(img), c_out, c_in, taps, nt, kc);
+      w, reinterpret_cast<__nv_bfloat16 *>(img), c_out, c_in, taps, nt, kc, rows);
   count_launch();
   return cudaGetLastError();
 }

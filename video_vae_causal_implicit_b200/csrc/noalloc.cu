@@ -137,23 +137,25 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   if (!choose_umma_config(d->n, d->c_in, d->c_out, d->h, d->w, d->kt, d->kh,
                           d->epi == CC3D_EPI_BIAS_RMS_SILU, n_sm, &cfg))
     return CC3D_ERR_UNSUPPORTED;
-  const int max_clusters = cfg.split > 1 ? umma_max_clusters(cfg, d->kh) : 0;
-  if (cfg.split > 1 && max_clusters < 1) return CC3D_ERR_CUDA;
+  const bool clustered = cfg.split > 1 || cfg.pair;
+  const int max_clusters = clustered ? umma_max_clusters(cfg, d->kh) : 0;
+  if (clustered && max_clusters < 1) return CC3D_ERR_CUDA;
   const int kc = cfg.kc, nt = cfg.nt;
 
   // ---- scratch: re-tiled weights (every call), zero bias when none is given --------
   uint8_t *wimg = scratch;
   float *zero_bias = reinterpret_cast<float *>(scratch + kNoAllocWeightBytes);
   cudaError_t e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(d->weight), wimg,
-                                     d->c_out, d->c_in, taps, nt, kc, stream);
+                                     d->c_out, d->c_in, taps, nt, kc, cfg.pair, stream);
   if (e == cudaSuccess && !d->bias)
     e = cudaMemsetAsync(zero_bias, 0, sizeof(float) * d->c_out, stream);
   if (e != cudaSuccess) return CC3D_ERR_CUDA;
 
   // ---- the conv -----------------------------------------------------------------------------
-  CUtensorMap mx, mc;
+  CUtensorMap mx, mc, mw;
   const int tile_w = umma_tile_w() * cfg.sub;
-  const int box_w = umma_halo_box_w(kc, cfg.sub, d->kw), box_h = umma_tile_h() + d->kh - 1;
+  const int box_w = umma_halo_box_w(kc, cfg.pair ? 1 : cfg.sub, d->kw);
+  const int box_h = umma_tile_h() + d->kh - 1;
   const int box_c = umma_halo_box_c(kc);
   if (!encode_activation_map(&mx, x, d->c_in, d->w, d->h, t, d->n, box_w, box_h, box_c))
     return CC3D_ERR_CUDA;
@@ -164,6 +166,13 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
       return CC3D_ERR_CUDA;
   } else {
     mc = mx;
+  }
+  if (cfg.pair) {
+    if (!encode_weight_map(&mw, wimg, static_cast<long long>(d->c_out) * taps * (d->c_in / 64),
+                           nt / 2))
+      return CC3D_ERR_CUDA;
+  } else {
+    mw = mx;
   }
   UmmaArgs a;
   a.wimg = wimg;
@@ -177,7 +186,7 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   a.n = d->n; a.t = t; a.h = d->h; a.w = d->w; a.c_in = d->c_in; a.c_out = d->c_out;
   a.kt = d->kt; a.kh = d->kh; a.kw = d->kw; a.pad_h = d->pad_h; a.pad_w = d->pad_w;
   a.nt = nt; a.n_ntiles = cfg.n_ntiles;
-  a.sub = cfg.sub; a.nbuf = cfg.nbuf; a.split = cfg.split;
+  a.sub = cfg.sub; a.nbuf = cfg.nbuf; a.split = cfg.split; a.pair = cfg.pair;
   a.tiles_w = (d->w + tile_w - 1) / tile_w;
   a.tiles_h = (d->h + umma_tile_h() - 1) / umma_tile_h();
   a.na = cfg.na; a.nb = cfg.nb; a.tmem_cols = cfg.tmem_cols;
@@ -185,13 +194,14 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   a.has_cache = has_cache ? 1 : 0;
   const uint64_t tiles = uint64_t(d->n) * t * a.tiles_h * a.tiles_w * a.n_ntiles;
   uint64_t grid;
-  if (cfg.split > 1) {
-    grid = (tiles < uint64_t(max_clusters) ? tiles : uint64_t(max_clusters)) * cfg.split;
+  if (clustered) {
+    grid = (tiles < uint64_t(max_clusters) ? tiles : uint64_t(max_clusters)) *
+           (cfg.pair ? 2 : cfg.split);
   } else {
     const uint64_t slots = uint64_t(n_sm) * cfg.ctas_per_sm;
     grid = tiles < slots ? tiles : slots;
   }
-  e = launch_conv_umma(mx, mc, a, kc, static_cast<unsigned>(grid), stream);
+  e = launch_conv_umma(mx, mc, mw, a, kc, static_cast<unsigned>(grid), stream);
   count_launch();
   if (e == cudaSuccess && cache_out && front > 0)
     e = launch_cache_update(cache_in, x, cache_out, d->n, t, front, in_frame, stream);
