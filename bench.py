@@ -48,7 +48,7 @@ C4 = dict(c=192, t=9, h=240, w=416)
 # DRAM bytes (read + write) per launch of the conv kernel on this workload,
 # from one ncu capture of the current kernel (profiles/ holds the summaries
 # and commands); None until captured.
-NCU_TRAFFIC = {"whole": None, "chunk": None}
+NCU_TRAFFIC = {"whole": 14.03e6, "chunk": 10.09e6}
 
 
 def conv_flop(n, cin, cout, t, h, w, taps=27):
