@@ -40,11 +40,14 @@ def _p(t):
 
 def test_noalloc_matches_planned_conv_on_two_calls_in_a_row():
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    # call 1: 384 -> 384 with a bias and a cache; call 2: different weights,
-    # no bias (the scratch's zero bias must be cleared), 96 -> 192.
+    # call 1: 384 -> 384 with a bias and a cache (the temporal split); call 2:
+    # different weights, no bias (the scratch's zero bias must be cleared),
+    # 96 -> 192; call 3: a frame large enough for the CTA pair, whose weights
+    # the scratch holds as plain rows behind a tensor map.
     cases = [
         dict(cin=384, cout=384, t=2, h=30, w=52, bias=True, cache=True, seed=1),
         dict(cin=96, cout=192, t=3, h=21, w=17, bias=False, cache=False, seed=2),
+        dict(cin=64, cout=64, t=2, h=96, w=96, bias=True, cache=True, seed=3),
     ]
     outs = []
     for cs in cases:
@@ -57,6 +60,8 @@ def test_noalloc_matches_planned_conv_on_two_calls_in_a_row():
                  if cs["cache"] else None)
         kw = dict(h=cs["h"], w=cs["w"], max_t=cs["t"])
         plan = cc3d.Plan(w, b, **kw)
+        if cs["seed"] == 3:
+            assert plan.stats().mma_ctas == 2
         y_ref = torch.empty((1, cs["t"], cs["h"], cs["w"], cs["cout"]), dtype=torch.bfloat16,
                             device="cuda")
         plan.forward(x, y_ref, cache_in=cache)
