@@ -279,6 +279,41 @@ def main():
     cc3d.sync_status()
     whole_ms = statistics.mean(whole_l)
     chunk_ms = statistics.mean(chunk_l)
+    plan_stats = plan.stats()
+
+    # For context (not the timed step): the same layer planned for one-frame
+    # calls only (max_t = 1), which takes the temporal split; its 5 chunks
+    # as one graph.  Its outputs are not bit-identical to the whole-sequence
+    # plan's, so the step above uses one plan for both.
+    plan_s = cc3d.Plan(case["w"].to(dev), case["b"].to(dev), h=H, w=W, max_t=1)
+    ys_s = [torch.empty_like(ys[0]) for _ in range(T)]
+    smarks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(T + 1)]
+
+    def stream_only():
+        s = torch.cuda.current_stream()
+        smarks[0].record(s)
+        cache = None
+        for k in range(T):
+            plan_s.forward(xs[k], ys_s[k], t=1, cache_in=cache, cache_out=caches[k % 2])
+            cache = caches[k % 2]
+            smarks[1 + k].record(s)
+
+    stream_only()
+    sgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(sgraph):
+        stream_only()
+    s_chunks = []
+    for k in range(args.warmup + args.steps):
+        flush_l2(k)
+        sgraph.replay()
+        torch.cuda.synchronize()
+        if k >= args.warmup:
+            s_chunks.extend(smarks[i].elapsed_time(smarks[i + 1]) for i in range(T))
+    cc3d.sync_status()
+    stream_plan_ms = statistics.mean(s_chunks)
+    stream_plan_split = plan_s.stats().k_split
+    del sgraph
+    plan_s.close()
     ms_local = sum(step_ms) / len(step_ms)
     ms = max_over_ranks(ms_local)
     value = world * flop_step / (ms * 1e-3) / 1e12
@@ -420,7 +455,16 @@ def main():
                              "one_frame_chunk": {"ms": chunk_ms, "gflop": flop_chunk / 1e9,
                                                  "tflops": flop_chunk / chunk_ms / 1e9,
                                                  "frac": flop_chunk / chunk_ms / 1e9 / peaks["bf16_tflops"],
-                                                 "traffic": NCU_TRAFFIC["chunk"]}}},
+                                                 "traffic": NCU_TRAFFIC["chunk"]},
+                             "plan": {"k_split": plan_stats.k_split,
+                                      "mma_ctas": plan_stats.mma_ctas,
+                                      "n_tile": plan_stats.n_tile},
+                             "one_frame_chunk_streaming_plan": {
+                                 "ms": stream_plan_ms, "tflops": flop_chunk / stream_plan_ms / 1e9,
+                                 "frac": flop_chunk / stream_plan_ms / 1e9 / peaks["bf16_tflops"],
+                                 "k_split": stream_plan_split,
+                                 "note": "the layer planned for one-frame calls (max_t = 1): "
+                                         "temporal split; context only, not in the timed step"}}},
             "resblock": resblock,
             "e2e": e2e,
             "gpu_launches": launches,

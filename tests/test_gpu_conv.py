@@ -108,11 +108,26 @@ def test_config2_whole_and_streaming_bitwise_and_oracle():
     both against the full fp64 oracle."""
     case = synth.conv_case(384, 384, 5, 30, 52)
     plan, x, y = run_conv(case)
-    assert plan.stats().k_split == 3  # 28 tiles a frame: one temporal tap per CTA
+    # a plan for 5-frame calls: one CTA per tile (the temporal split would
+    # take 4 rounds of clusters for 140 tiles)
+    assert plan.stats().k_split == 1
     ys = _stream_chunks(plan, x, 1, 384)
     assert torch.equal(ys.cpu(), y.cpu()), "streaming != whole sequence"
     ref = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], _bias64(case["b"]))
     assert_close_bf16(ncthw_np(y), ref, "config 2")
+
+
+def test_config2_streaming_plan_splits_and_matches_oracle():
+    """A plan made for one-frame calls (max_t = 1) of the config-2 layer
+    takes the temporal split (28 tiles a frame); its streamed chunks carry
+    the cache and match the oracle."""
+    case = synth.conv_case(384, 384, 5, 30, 52)
+    x = to_dev(synth.ndhwc(case["x"]))
+    plan = cc3d.Plan(to_dev(case["w"]), to_dev(case["b"]), h=30, w=52, max_t=1)
+    assert plan.stats().k_split == 3
+    ys = _stream_chunks(plan, x, 1, 384)
+    ref = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], _bias64(case["b"]))
+    assert_close_bf16(ncthw_np(ys), ref, "config 2, streaming plan")
 
 
 @pytest.mark.parametrize("chunk", [2, 3])

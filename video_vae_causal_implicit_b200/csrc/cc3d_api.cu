@@ -356,13 +356,15 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
     if (cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, p->device) !=
         cudaSuccess)
       p->sm_count = 148;
-    // Tile configuration (N split, sub-tiles, pipeline depths): a function
-    // of (n, c_in, c_out, h, w, epilogue), never of t, so a streamed
-    // sequence and a whole-sequence call run identical arithmetic.
+    // Tile configuration (N split, sub-tiles, CTA pair, temporal split,
+    // pipeline depths): a function of (n, c_in, c_out, h, w, epilogue,
+    // max_t), never of a call's t, so a streamed sequence and a
+    // whole-sequence call of one plan run identical arithmetic.
     {
       UmmaConfig cfg;
       if (!choose_umma_config(desc->n, desc->c_in, desc->c_out, desc->h, desc->w, desc->kt,
-                              desc->kh, desc->epi == CC3D_EPI_BIAS_RMS_SILU, p->sm_count, &cfg)) {
+                              desc->kh, desc->epi == CC3D_EPI_BIAS_RMS_SILU, desc->max_t,
+                              p->sm_count, &cfg)) {
         s = CC3D_ERR_UNSUPPORTED;
         goto fail;
       }

@@ -147,6 +147,20 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, const UmmaArgs &p) {
   return c;
 }
 
+// 16 consecutive fp32 parameters (bias / gamma / beta) of 16-byte-aligned
+// rows as four 16-byte loads; every lane of a warp reads the same address.
+__device__ __forceinline__ void ld_param16(const float *src, float (&v)[16]) {
+  const float4 *s4 = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float4 f = __ldg(s4 + u);
+    v[4 * u] = f.x;
+    v[4 * u + 1] = f.y;
+    v[4 * u + 2] = f.z;
+    v[4 * u + 3] = f.w;
+  }
+}
+
 template <int KC, int KS, int SUB, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     conv_umma_kernel(const __grid_constant__ CUtensorMap map_x,
@@ -572,8 +586,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                   mbar_arrive_remote_relaxed(
                       mapa_shared(smem_u32(&x_free[(q * p.split + rank) * kXSlots + slot]),
                                   static_cast<uint32_t>(dst_rank)));
+            {
+              float bv[16];
+              ld_param16(p.bias + n0 + j0, bv);
 #pragma unroll
-            for (int i = 0; i < kXC; ++i) v[i] += p.bias[n0 + j0 + i];
+              for (int i = 0; i < kXC; ++i) v[i] += bv[i];
+            }
             if (p.epi == 1 && valid) {
               const __nv_bfloat16 *rb0 = reinterpret_cast<const __nv_bfloat16 *>(&res[0]);
               const __nv_bfloat16 *rb1 = reinterpret_cast<const __nv_bfloat16 *>(&res[1]);
@@ -633,9 +651,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int u = 0; u < 3; ++u) {
               if (u >= nld) continue;
+              float bv[16];
+              ld_param16(p.bias + n0 + j0 + 16 * u, bv);
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                const float hv = __uint_as_float(raw[16 * u + i]) + p.bias[n0 + j0 + 16 * u + i];
+                const float hv = __uint_as_float(raw[16 * u + i]) + bv[i];
                 ss = fmaf(hv, hv, ss);
               }
             }
@@ -680,8 +700,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (u >= nld) continue;
             const int j = j0 + 16 * u;
             float v[16];
+            {
+              float bv[16];
+              ld_param16(p.bias + n0 + j, bv);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(raw[16 * u + i]) + p.bias[n0 + j + i];
+              for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(raw[16 * u + i]) + bv[i];
+            }
             if (p.epi == 1 && valid) {
               const __nv_bfloat16 *rb0 = reinterpret_cast<const __nv_bfloat16 *>(&res[2 * u]);
               const __nv_bfloat16 *rb1 = reinterpret_cast<const __nv_bfloat16 *>(&res[2 * u + 1]);
@@ -691,10 +715,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 v[8 + i] += __bfloat162float(rb1[i]);
               }
             } else if (p.epi == 2) {
+              float gv[16], be[16];
+              ld_param16(p.gamma + n0 + j, gv);
+              if (p.beta) {
+                ld_param16(p.beta + n0 + j, be);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) be[i] = 0.f;
+              }
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                float a = v[i] * inv * p.gamma[n0 + j + i];
-                if (p.beta) a += p.beta[n0 + j + i];
+                float a = v[i] * inv * gv[i];
+                a += be[i];
                 v[i] = silu_fast(a);
               }
             }
@@ -784,8 +816,9 @@ long long mma_cycles(const UmmaConfig &c) {
   return math > smem ? math : smem;
 }
 
-// Relative time of one frame of n images: whole waves of tiles over the
-// GPU (SMs, or SM pairs for a pair), each as long as one tile's MMA steps.
+// Relative time of one frame of n images (or of n frames): whole waves of
+// tiles over the GPU (SMs, or SM pairs for a pair), each as long as one
+// tile's MMA steps.
 long long frame_cost(const UmmaConfig &c, int n, int h, int w, int sm_count) {
   const long long tiles = static_cast<long long>(n) * ((h + kTH - 1) / kTH) *
                           ((w + c.sub * kTW - 1) / (c.sub * kTW)) * c.n_ntiles;
@@ -797,7 +830,7 @@ long long frame_cost(const UmmaConfig &c, int n, int h, int w, int sm_count) {
 }  // namespace
 
 bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
-                        int sm_count, UmmaConfig *cfg) {
+                        int max_t, int sm_count, UmmaConfig *cfg) {
   // N tile: the largest split of c_out that is a multiple of 16 and at most
   // `cap` (256 is the tcgen05 N limit); the RMS epilogue needs the whole row
   // in one CTA.
@@ -806,8 +839,9 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
       if (c_out % nt == 0 && (!rms_epi || nt == c_out)) return nt;
     return 0;
   };
-  // Every choice below depends on (n, c, h, w) -- never on t -- so streamed
-  // and whole-sequence calls run identical arithmetic.
+  // Every choice below depends on (n, c, h, w, epilogue) and the plan's
+  // max_t -- never on a call's t -- so streamed and whole-sequence calls of
+  // one plan run identical arithmetic.
   UmmaConfig one;
   one.kc = (c_in % 64 == 0) ? 64 : (c_in % 96 == 0) ? 96 : 32;
   one.sub = 1;
@@ -825,16 +859,29 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
   // decoder layer), and its time is the length of one tile's K loop.  Each
   // CTA of a cluster of kt then runs one temporal tap, and the partial sums
   // meet through distributed shared memory in the last CTA.  Not with the
-  // RMS epilogue, which needs whole rows in one CTA.
+  // RMS epilogue, which needs whole rows in one CTA.  Taken only if it also
+  // wins for the plan's largest call (max_t frames): there the split's
+  // clusters (about 9/10 of sm_count / kt fit at once) take whole rounds of
+  // one-tap work plus the exchange (measured at ~0.4 of a tap's MMAs),
+  // against rounds of kt taps over all SMs.
   if (kt >= 2 && kt <= 4 && !rms_epi) {
     UmmaConfig sp = one;
     sp.split = kt;
-    if (finish_config(ks, sp) && tiles1 * kt <= static_cast<long long>(sm_count) * sp.ctas_per_sm) {
+    const long long calls_tiles = tiles1 * (max_t > 0 ? max_t : 1);
+    const long long clusters = sm_count * 9 / (10 * kt);
+    const long long slots = static_cast<long long>(sm_count) * one.ctas_per_sm;
+    const long long cost_one = (calls_tiles + slots - 1) / slots * kt * 10;
+    const long long cost_split = clusters > 0 ? (calls_tiles + clusters - 1) / clusters * 14 : 0;
+    if (clusters > 0 && finish_config(ks, sp) &&
+        tiles1 * kt <= static_cast<long long>(sm_count) * sp.ctas_per_sm && cost_split < cost_one) {
       *cfg = sp;
       return true;
     }
   }
-  long long best = frame_cost(one, n, h, w, sm_count);
+  // the tile shapes are compared on the plan's largest call: max_t frames
+  // of n images tile like n * max_t images
+  const int nt_frames = n * (max_t > 0 ? max_t : 1);
+  long long best = frame_cost(one, nt_frames, h, w, sm_count);
   // Two sub-tiles (a 16 x 16 pixel CTA tile, two 8 x 16 MMA tiles) share
   // every weight stage, halving the weight bytes written per MMA.  Only with
   // N <= 128, where both sub-tiles still fit two accumulator buffers (a
@@ -845,7 +892,7 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
   if (two.nt) {
     two.n_ntiles = c_out / two.nt;
     if (finish_config(ks, two) && two.nbuf == 2) {
-      const long long cost = frame_cost(two, n, h, w, sm_count);
+      const long long cost = frame_cost(two, nt_frames, h, w, sm_count);
       if (cost < best) {
         best = cost;
         *cfg = two;
@@ -861,7 +908,7 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
     pr.pair = 1;
     pr.sub = 2;  // the tile is two MMA tiles wide
     if (finish_config(ks, pr) && pr.nbuf == 2) {
-      const long long cost = frame_cost(pr, n, h, w, sm_count);
+      const long long cost = frame_cost(pr, nt_frames, h, w, sm_count);
       if (cost <= best) {
         best = cost;
         *cfg = pr;

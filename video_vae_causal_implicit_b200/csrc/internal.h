@@ -35,13 +35,13 @@ struct UmmaArgs {
                                   // tile (sub is then 2: the tile width in MMA tiles)
 };
 
-// Tile configuration of the UMMA conv for a problem (chosen from n, c_in,
-// c_out, h, w and the epilogue -- never from t).
+// Tile configuration of the UMMA conv for a plan (chosen from n, c_in, c_out,
+// h, w, the epilogue and the plan's max_t -- never from a call's t).
 struct UmmaConfig {
   int kc, nt, n_ntiles, sub, nbuf, split, pair, na, nb, tmem_cols, ctas_per_sm;
 };
 bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
-                        int sm_count, UmmaConfig *cfg);
+                        int max_t, int sm_count, UmmaConfig *cfg);
 // Clusters of cfg.split CTAs that can be resident at once (split > 1), for
 // sizing the grid; 0 when the query fails.
 int umma_max_clusters(const UmmaConfig &cfg, int ks);

@@ -135,7 +135,7 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   // ---- tiles: the same choice cc3d_plan_create makes --------------------------------
   UmmaConfig cfg;
   if (!choose_umma_config(d->n, d->c_in, d->c_out, d->h, d->w, d->kt, d->kh,
-                          d->epi == CC3D_EPI_BIAS_RMS_SILU, n_sm, &cfg))
+                          d->epi == CC3D_EPI_BIAS_RMS_SILU, d->max_t, n_sm, &cfg))
     return CC3D_ERR_UNSUPPORTED;
   const bool clustered = cfg.split > 1 || cfg.pair;
   const int max_clusters = clustered ? umma_max_clusters(cfg, d->kh) : 0;
