@@ -4,7 +4,10 @@
 
 Cases (seeded synthetic inputs, generated on the device):
   c2      384 -> 384 causal conv, whole sequence, x[1,384,5,30,52]
-  c2s     the same as 5 one-frame chunks with a 2-frame cache
+  c2s     the same as 5 one-frame chunks with a 2-frame cache, planned for
+          one-frame calls (max_t = 1: the temporal split)
+  c2c     the 5 one-frame chunks with the whole-sequence plan (max_t = 5), as
+          in the benchmark step
   c3a     3 -> 96 causal conv on x[1,3,17,480,832]
   c3b     96 -> 96 causal conv on x[1,96,17,480,832]
   c4      the residual block on x[1,192,9,240,416]
@@ -28,7 +31,7 @@ def _rand(shape, dev, seed=0):
 
 
 def build_case(name, dev):
-    if name in ("c2", "c2s"):
+    if name in ("c2", "c2s", "c2c"):
         c, T, H, W = 384, 5, 30, 52
     elif name == "c3a":
         c, T, H, W = 3, 17, 480, 832
@@ -54,8 +57,8 @@ def build_case(name, dev):
     cout = 96 if name == "c3a" else c
     wt = synth.kaiming_uniform(cout, c, (3, 3, 3), 1).to(dev)
     b = synth.uniform((cout,), -0.1, 0.1, 2).to(dev)
-    if name == "c2s":
-        plan = cc3d.Plan(wt, b, h=H, w=W, max_t=1)
+    if name in ("c2s", "c2c"):
+        plan = cc3d.Plan(wt, b, h=H, w=W, max_t=1 if name == "c2s" else T)
         ys = [torch.empty((1, 1, H, W, cout), dtype=torch.bfloat16, device=dev) for _ in range(T)]
         cb = [torch.empty((1, 2, H, W, c), dtype=torch.bfloat16, device=dev) for _ in range(2)]
 
