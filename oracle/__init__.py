@@ -71,6 +71,10 @@ def _load():
             lib.orc_causal_conv3d.argtypes = [T, T, i, i, i, i, i, T, i, i, i, i, i, i, dp, dp]
             lib.orc_causal_conv3d_points.argtypes = [T, T, i, i, i, i, i, T, i, i, i, i, i, i, dp,
                                                      i, ip, dp]
+            lib.orc_causal_conv3d_s.argtypes = [T, T, i, i, i, i, i, T, i, i, i, i, i, i, i, dp,
+                                                dp]
+            lib.orc_causal_conv3d_points_s.argtypes = [T, T, i, i, i, i, i, T, i, i, i, i, i, i, i,
+                                                       dp, i, ip, dp]
             lib.orc_rms_norm.argtypes = [T, i, i, i, i, i, dp, dp, i, dp]
             lib.orc_resblock.argtypes = [T, T, T, i, i, i, i, i, T, dp, dp, T, dp, dp, i, dp, dp, dp]
             lib.orc_resblock_points.argtypes = [T, T, T, i, i, i, i, i, T, dp, dp, T, dp, dp, i,
@@ -79,8 +83,9 @@ def _load():
             lib.orc_round_bf16.restype = ctypes.c_double
             lib.orc_silu.argtypes = [ctypes.c_double]
             lib.orc_silu.restype = ctypes.c_double
-            for name in ("orc_causal_conv3d", "orc_causal_conv3d_points", "orc_rms_norm",
-                         "orc_resblock", "orc_resblock_points"):
+            for name in ("orc_causal_conv3d", "orc_causal_conv3d_points", "orc_causal_conv3d_s",
+                         "orc_causal_conv3d_points_s", "orc_rms_norm", "orc_resblock",
+                         "orc_resblock_points"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -149,11 +154,11 @@ def _shape5(a):
     return tuple(int(s) for s in a.shape)
 
 
-def causal_conv3d(x, weight, bias=None, cache=None, pad=(1, 1)):
+def causal_conv3d(x, weight, bias=None, cache=None, pad=(1, 1), stride_t=1):
     """y[n,co,t,h,w] = b[co] + sum_{ci,kt,kh,kw} W[co,ci,kt,kh,kw] *
-    xt[n,ci,t+kt,h+kh-pad_h,w+kw-pad_w], xt = concat(cache or zeros, x) on t.
-    x: [N,Cin,T,H,W]; weight: [Cout,Cin,KT,KH,KW]; cache: [N,Cin,KT-1,H,W]
-    or None.  Returns float64 [N,Cout,T,H,W]."""
+    xt[n,ci,s*t+kt,h+kh-pad_h,w+kw-pad_w], xt = concat(cache or zeros, x) on
+    t, s = stride_t.  x: [N,Cin,T,H,W]; weight: [Cout,Cin,KT,KH,KW]; cache:
+    [N,Cin,KT-1,H,W] or None.  Returns float64 [N,Cout,(T-1)//s+1,H,W]."""
     lib = _load()
     keep = []
     N, Cin, T, H, W = _shape5(x)
@@ -162,12 +167,13 @@ def causal_conv3d(x, weight, bias=None, cache=None, pad=(1, 1)):
     if cache is not None:
         assert _shape5(cache) == (N, Cin, KT - 1, H, W)
     tx, tc, tw = _view(x, keep), _view(cache, keep), _view(weight, keep)
-    y = np.empty((N, Cout, T, H, W), dtype=np.float64)
-    rc = lib.orc_causal_conv3d(_ptr(tx), _ptr(tc), N, Cin, T, H, W, _ptr(tw), Cout, KT, KH, KW,
-                               pad[0], pad[1], _dvec(bias, keep),
-                               y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    Tout = (T - 1) // stride_t + 1
+    y = np.empty((N, Cout, Tout, H, W), dtype=np.float64)
+    rc = lib.orc_causal_conv3d_s(_ptr(tx), _ptr(tc), N, Cin, T, H, W, _ptr(tw), Cout, KT, KH, KW,
+                                 pad[0], pad[1], stride_t, _dvec(bias, keep),
+                                 y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
     if rc != 0:
-        raise ValueError(f"orc_causal_conv3d failed ({rc})")
+        raise ValueError(f"orc_causal_conv3d_s failed ({rc})")
     return y
 
 
@@ -177,9 +183,9 @@ def _pts(points, keep):
     return p.shape[0], p.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
 
 
-def causal_conv3d_points(x, weight, bias, cache, points, pad=(1, 1)):
-    """The causal Conv3D at the output voxels in ``points`` (rows n,t,h,w).
-    Returns float64 [P, Cout]."""
+def causal_conv3d_points(x, weight, bias, cache, points, pad=(1, 1), stride_t=1):
+    """The causal Conv3D (temporal stride stride_t) at the output voxels in
+    ``points`` (rows n,t,h,w; t an output frame).  Returns float64 [P, Cout]."""
     lib = _load()
     keep = []
     N, Cin, T, H, W = _shape5(x)
@@ -187,11 +193,11 @@ def causal_conv3d_points(x, weight, bias, cache, points, pad=(1, 1)):
     tx, tc, tw = _view(x, keep), _view(cache, keep), _view(weight, keep)
     P, pp = _pts(points, keep)
     y = np.empty((P, Cout), dtype=np.float64)
-    rc = lib.orc_causal_conv3d_points(_ptr(tx), _ptr(tc), N, Cin, T, H, W, _ptr(tw), Cout, KT, KH,
-                                      KW, pad[0], pad[1], _dvec(bias, keep), P, pp,
-                                      y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    rc = lib.orc_causal_conv3d_points_s(_ptr(tx), _ptr(tc), N, Cin, T, H, W, _ptr(tw), Cout, KT,
+                                        KH, KW, pad[0], pad[1], stride_t, _dvec(bias, keep), P,
+                                        pp, y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
     if rc != 0:
-        raise ValueError(f"orc_causal_conv3d_points failed ({rc})")
+        raise ValueError(f"orc_causal_conv3d_points_s failed ({rc})")
     return y
 
 

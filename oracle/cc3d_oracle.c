@@ -14,7 +14,10 @@
  *     §10.3 "WanCausalConv3d": standard Conv3D y = b + sum W.x over
  *     (c_in, kt, kh, kw); spatial padding symmetric; the time axis padded
  *     only on the past side with 2*T_pad frames, or fed from cache_x, the
- *     last frames of the previous chunk, concatenated in front of t);
+ *     last frames of the previous chunk, concatenated in front of t), also
+ *     with a temporal stride s (same page, §10.5: the downsample path's
+ *     time_conv is a CausalConv3d with stride (2,1,1)): output frame t reads
+ *     the padded sequence at s*t + kt, and ceil(T / s) frames come out;
  *   - bias added once, after every tap has been summed ("cache-aware video
  *     decoder lowering" summary, section on turning Conv3D into batched
  *     Conv2D);
@@ -101,12 +104,13 @@ double orc_round_bf16(double v) {
  * this chunk, oldest first) or is zero when there is no cache. */
 static double conv_at(const orc_tensor *x, const orc_tensor *cache, int Cin,
                       int H, int W, const orc_tensor *wt, int KT, int KH,
-                      int KW, int pad_h, int pad_w, const double *bias, int n,
-                      int co, int t, int h, int w) {
+                      int KW, int pad_h, int pad_w, int stride_t,
+                      const double *bias, int n, int co, int t, int h, int w) {
   double acc = 0.0;
   for (int ci = 0; ci < Cin; ++ci)
     for (int kt = 0; kt < KT; ++kt) {
-      int tau = t + kt - (KT - 1);
+      /* padded frame stride_t * t + kt, i.e. input frame tau */
+      int tau = stride_t * t + kt - (KT - 1);
       if (tau < 0 && cache == NULL) continue; /* zero frame */
       for (int kh = 0; kh < KH; ++kh) {
         int hh = h + kh - pad_h;
@@ -124,43 +128,57 @@ static double conv_at(const orc_tensor *x, const orc_tensor *cache, int Cin,
   return acc;
 }
 
-/* Full causal Conv3D.  y is contiguous [N][Cout][T][H][W].
- * Output spatial size equals input size (stride 1, pad = (k - 1) / 2 is
- * what the callers use; any pad_h, pad_w in [0, k) is accepted and the
- * output keeps H x W). Returns 0, or -1 on a bad argument. */
-int orc_causal_conv3d(const orc_tensor *x, const orc_tensor *cache, int N,
-                      int Cin, int T, int H, int W, const orc_tensor *wt,
-                      int Cout, int KT, int KH, int KW, int pad_h, int pad_w,
-                      const double *bias, double *y) {
+/* Full causal Conv3D with temporal stride stride_t (>= 1).  T is the input
+ * frame count; y is contiguous [N][Cout][Tout][H][W] with
+ * Tout = (T - 1) / stride_t + 1.  Output spatial size equals input size
+ * (pad = (k - 1) / 2 is what the callers use; any pad_h, pad_w in [0, k) is
+ * accepted and the output keeps H x W).  Returns 0, or -1 on a bad
+ * argument. */
+int orc_causal_conv3d_s(const orc_tensor *x, const orc_tensor *cache, int N,
+                        int Cin, int T, int H, int W, const orc_tensor *wt,
+                        int Cout, int KT, int KH, int KW, int pad_h, int pad_w,
+                        int stride_t, const double *bias, double *y) {
   if (!x || !wt || !y || N < 1 || Cin < 1 || Cout < 1 || T < 1 || H < 1 ||
-      W < 1 || KT < 1 || KH < 1 || KW < 1)
+      W < 1 || KT < 1 || KH < 1 || KW < 1 || stride_t < 1)
     return -1;
-  long long total = (long long)N * Cout * T * H;
+  const int Tout = (T - 1) / stride_t + 1;
+  long long total = (long long)N * Cout * Tout * H;
 #pragma omp parallel for schedule(dynamic, 1)
   for (long long idx = 0; idx < total; ++idx) {
     int h = (int)(idx % H);
-    int t = (int)((idx / H) % T);
-    int co = (int)((idx / ((long long)H * T)) % Cout);
-    int n = (int)(idx / ((long long)H * T * Cout));
+    int t = (int)((idx / H) % Tout);
+    int co = (int)((idx / ((long long)H * Tout)) % Cout);
+    int n = (int)(idx / ((long long)H * Tout * Cout));
     for (int w = 0; w < W; ++w)
-      y[(((long long)n * Cout + co) * T + t) * H * W + (long long)h * W + w] =
-          conv_at(x, cache, Cin, H, W, wt, KT, KH, KW, pad_h, pad_w, bias, n,
-                  co, t, h, w);
+      y[(((long long)n * Cout + co) * Tout + t) * H * W + (long long)h * W +
+        w] = conv_at(x, cache, Cin, H, W, wt, KT, KH, KW, pad_h, pad_w,
+                     stride_t, bias, n, co, t, h, w);
   }
   return 0;
 }
 
-/* The causal Conv3D at P chosen output voxels: pts holds P rows (n, t, h, w);
- * y is [P][Cout]. */
-int orc_causal_conv3d_points(const orc_tensor *x, const orc_tensor *cache,
-                             int N, int Cin, int T, int H, int W,
-                             const orc_tensor *wt, int Cout, int KT, int KH,
-                             int KW, int pad_h, int pad_w, const double *bias,
-                             int P, const int *pts, double *y) {
-  if (!x || !wt || !y || !pts || P < 0) return -1;
+/* The same with stride 1 (Tout = T). */
+int orc_causal_conv3d(const orc_tensor *x, const orc_tensor *cache, int N,
+                      int Cin, int T, int H, int W, const orc_tensor *wt,
+                      int Cout, int KT, int KH, int KW, int pad_h, int pad_w,
+                      const double *bias, double *y) {
+  return orc_causal_conv3d_s(x, cache, N, Cin, T, H, W, wt, Cout, KT, KH, KW,
+                             pad_h, pad_w, 1, bias, y);
+}
+
+/* The causal Conv3D (temporal stride stride_t) at P chosen output voxels:
+ * pts holds P rows (n, t, h, w), t an output frame; y is [P][Cout]. */
+int orc_causal_conv3d_points_s(const orc_tensor *x, const orc_tensor *cache,
+                               int N, int Cin, int T, int H, int W,
+                               const orc_tensor *wt, int Cout, int KT, int KH,
+                               int KW, int pad_h, int pad_w, int stride_t,
+                               const double *bias, int P, const int *pts,
+                               double *y) {
+  if (!x || !wt || !y || !pts || P < 0 || stride_t < 1) return -1;
+  const int Tout = (T - 1) / stride_t + 1;
   for (int p = 0; p < P; ++p) {
     const int *q = pts + 4 * p;
-    if (q[0] < 0 || q[0] >= N || q[1] < 0 || q[1] >= T || q[2] < 0 ||
+    if (q[0] < 0 || q[0] >= N || q[1] < 0 || q[1] >= Tout || q[2] < 0 ||
         q[2] >= H || q[3] < 0 || q[3] >= W)
       return -1;
   }
@@ -168,10 +186,19 @@ int orc_causal_conv3d_points(const orc_tensor *x, const orc_tensor *cache,
   for (long long pc = 0; pc < (long long)P * Cout; ++pc) {
     int p = (int)(pc / Cout), co = (int)(pc % Cout);
     const int *q = pts + 4 * p;
-    y[pc] = conv_at(x, cache, Cin, H, W, wt, KT, KH, KW, pad_h, pad_w, bias,
-                    q[0], co, q[1], q[2], q[3]);
+    y[pc] = conv_at(x, cache, Cin, H, W, wt, KT, KH, KW, pad_h, pad_w,
+                    stride_t, bias, q[0], co, q[1], q[2], q[3]);
   }
   return 0;
+}
+
+int orc_causal_conv3d_points(const orc_tensor *x, const orc_tensor *cache,
+                             int N, int Cin, int T, int H, int W,
+                             const orc_tensor *wt, int Cout, int KT, int KH,
+                             int KW, int pad_h, int pad_w, const double *bias,
+                             int P, const int *pts, double *y) {
+  return orc_causal_conv3d_points_s(x, cache, N, Cin, T, H, W, wt, Cout, KT,
+                                    KH, KW, pad_h, pad_w, 1, bias, P, pts, y);
 }
 
 /* SiLU(z) = z * sigmoid(z) = z / (1 + e^-z). */

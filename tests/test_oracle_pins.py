@@ -34,8 +34,9 @@ def rnd(shape, seed, scale=1.0):
     return g.standard_normal(shape) * scale
 
 
-def torch_causal_conv3d(x, w, b, cache=None, pad=(1, 1)):
-    """Library special case: F.pad + conv3d in float64."""
+def torch_causal_conv3d(x, w, b, cache=None, pad=(1, 1), stride_t=1):
+    """Library special case: F.pad + conv3d (temporal stride stride_t) in
+    float64."""
     x = torch.from_numpy(np.ascontiguousarray(x))
     w = torch.from_numpy(np.ascontiguousarray(w))
     kt = w.shape[2]
@@ -45,7 +46,7 @@ def torch_causal_conv3d(x, w, b, cache=None, pad=(1, 1)):
     else:
         xt = F.pad(x, (pad[1], pad[1], pad[0], pad[0], kt - 1, 0))
     bb = torch.from_numpy(np.asarray(b)) if b is not None else None
-    return F.conv3d(xt, w, bb).numpy()
+    return F.conv3d(xt, w, bb, stride=(stride_t, 1, 1)).numpy()
 
 
 def numpy_padded_correlation(x, w, b, cache=None):
@@ -188,6 +189,64 @@ def test_streaming_equals_whole_sequence_bitwise(chunk):
         prev = cache if cache is not None else np.zeros((1, 3, 2, 4, 5))
         cache = np.ascontiguousarray(np.concatenate([prev, xc], axis=2)[:, :, -2:])
     np.testing.assert_array_equal(np.concatenate(outs, axis=2), whole)
+
+
+# ---- temporal stride (the downsample path's time_conv, stride (2,1,1)) ----------
+
+@pytest.mark.parametrize("T,k,cached", [(6, (3, 3, 3), False), (7, (3, 1, 1), False),
+                                        (5, (3, 1, 1), True), (4, (1, 3, 3), False)])
+def test_strided_conv_matches_torch_fp64(T, k, cached):
+    x = rnd((2, 3, T, 4, 5), 40)
+    w = rnd((4, 3) + k, 41, 0.3)
+    b = rnd((4,), 42, 0.1)
+    cache = rnd((2, 3, k[0] - 1, 4, 5), 43) if cached else None
+    pad = (k[1] // 2, k[2] // 2)
+    y = oracle.causal_conv3d(x, w, b, cache=cache, pad=pad, stride_t=2)
+    assert y.shape[2] == (T + 1) // 2
+    ref = torch_causal_conv3d(x, w, b, cache=cache, pad=pad, stride_t=2)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_strided_conv_is_unit_stride_at_even_frames_bitwise():
+    """Output frame t of the stride-2 conv reads the same padded frames
+    2t .. 2t+kt-1 as output frame 2t of the unit-stride conv."""
+    x = rnd((1, 4, 9, 5, 4), 44)
+    w = rnd((3, 4, 3, 3, 3), 45, 0.3)
+    b = rnd((3,), 46, 0.1)
+    for cache in (None, rnd((1, 4, 2, 5, 4), 47)):
+        y2 = oracle.causal_conv3d(x, w, b, cache=cache, stride_t=2)
+        y1 = oracle.causal_conv3d(x, w, b, cache=cache)
+        np.testing.assert_array_equal(y2, y1[:, :, ::2])
+
+
+@pytest.mark.parametrize("chunk", [2, 4])
+def test_strided_streaming_even_chunks_equals_whole_bitwise(chunk):
+    """Chunks of an even number of frames, carrying the last 2 input frames,
+    give the whole-sequence stride-2 output."""
+    T = 8
+    x = rnd((1, 3, T, 4, 5), 48)
+    w = rnd((4, 3, 3, 1, 1), 49, 0.3)
+    b = rnd((4,), 50, 0.1)
+    whole = oracle.causal_conv3d(x, w, b, pad=(0, 0), stride_t=2)
+    cache = None
+    outs = []
+    for s0 in range(0, T, chunk):
+        xc = x[:, :, s0:s0 + chunk]
+        outs.append(oracle.causal_conv3d(xc, w, b, cache=cache, pad=(0, 0), stride_t=2))
+        prev = cache if cache is not None else np.zeros((1, 3, 2, 4, 5))
+        cache = np.ascontiguousarray(np.concatenate([prev, xc], axis=2)[:, :, -2:])
+    np.testing.assert_array_equal(np.concatenate(outs, axis=2), whole)
+
+
+def test_strided_points_equal_full_bitwise():
+    x = rnd((1, 3, 7, 4, 5), 51)
+    w = rnd((2, 3, 3, 3, 3), 52, 0.3)
+    b = rnd((2,), 53, 0.1)
+    full = oracle.causal_conv3d(x, w, b, stride_t=2)
+    pts = [(0, t, h, ww) for t in range(4) for h in range(4) for ww in (0, 4)]
+    got = oracle.causal_conv3d_points(x, w, b, None, pts, stride_t=2)
+    for p, (n, t, h, ww) in enumerate(pts):
+        np.testing.assert_array_equal(got[p], full[n, :, t, h, ww])
 
 
 def test_zero_cache_equals_no_cache_bitwise():
