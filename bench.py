@@ -13,8 +13,10 @@ every timed step and the flush is outside the timed events.
 The same JSON line carries the residual block (x[1, 192, 9, 240, 416]:
 RMS_norm+SiLU -> conv -> RMS_norm+SiLU (fused) -> conv + x (fused)) as
 ``resblock`` with its latency, and with ``--sweep`` the encoder convs
-(3 -> 96, 96 -> 96 at 17 x 480 x 832) and the streaming channel/resolution
-sweep (21 one-frame chunks, CUDA-graph captured).
+(3 -> 96, 96 -> 96 at 17 x 480 x 832), the downsample path's time_conv
+(kernel (3, 1, 1), stride 2 in time, at 192 and 384 channels) and the
+streaming channel/resolution sweep (21 one-frame chunks, CUDA-graph
+captured).
 
 Multi-GPU: the path runs as independent replicas (one process per GPU, no
 data-path collective); ``value`` is the FLOP all ranks processed divided by
@@ -530,6 +532,21 @@ def run_sweep(args, dev, stream, peaks, flush_l2):
     out["cfg3b_96to96_17x480x832"] = {"ms": ms, "tflops": fl / ms / 1e9,
                                       "frac": fl / ms / 1e9 / peaks["bf16_tflops"]}
     del p96, x96, y96
+    # the downsample path's time_conv: kernel (3, 1, 1), temporal stride 2,
+    # whole sequence (17 -> 9 frames at 192 channels, 9 -> 5 at 384)
+    for (cc, T, H, W) in ((192, 17, 120, 208), (384, 9, 60, 104)):
+        xs = torch.randn((1, T, H, W, cc), generator=g, device=dev).to(torch.bfloat16)
+        ws = synth.kaiming_uniform(cc, cc, (3, 1, 1), 1).to(dev)
+        bs = synth.uniform((cc,), -0.1, 0.1, 2).to(dev)
+        ps = cc3d.Plan(ws, bs, h=H, w=W, max_t=T, stride_t=2)
+        t_out = (T - 1) // 2 + 1
+        ys = torch.empty((1, t_out, H, W, cc), dtype=torch.bfloat16, device=dev)
+        ms = timed(lambda: ps.forward(xs, ys), flush=True)
+        fl = conv_flop(1, cc, cc, t_out, H, W, taps=3)
+        out[f"time_conv_s2_c{cc}_{T}x{H}x{W}"] = {
+            "ms": ms, "tflops": fl / ms / 1e9, "frac": fl / ms / 1e9 / peaks["bf16_tflops"],
+            "tile": [ps.stats().mma_ctas, ps.stats().tile_w, ps.stats().k_split]}
+        del ps, xs, ys
     # config 5: C x resolution, 21 one-frame chunks, graph-captured
     for cc in (96, 192, 384):
         for (H, W) in ((90, 160), (180, 320), (360, 640)):

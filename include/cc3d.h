@@ -64,7 +64,8 @@ extern "C" {
 typedef enum {
   CC3D_OK = 0,
   CC3D_ERR_INVALID_ARG = 1,  /* null pointer, bad size, t out of [1, max_t] */
-  CC3D_ERR_UNSUPPORTED = 2,  /* stride/dilation/groups != 1, channel counts or
+  CC3D_ERR_UNSUPPORTED = 2,  /* spatial stride, dilation or groups != 1, a temporal
+                                stride other than 1 or 2, channel counts or
                                 kernel sizes no kernel covers, no sm_100 GPU */
   CC3D_ERR_ALIGNMENT = 3,    /* pointer not 16-byte aligned */
   CC3D_ERR_ALIAS = 4,        /* cache_out overlaps cache_in, x or y */
@@ -97,7 +98,15 @@ typedef struct {
   int n, c_in, c_out, h, w, max_t;   /* max_t: largest frame count per call  */
   int kt, kh, kw;                    /* kernel size; causal front pad = kt-1 */
   int pad_h, pad_w;                  /* spatial zero padding (kh/2, kw/2)    */
-  int stride_t, stride_h, stride_w;  /* must be 1                            */
+  int stride_t;        /* temporal stride: 1, or 2 (the downsample path's
+                          time_conv; bf16 tensor-core descriptors only).
+                          Output frame t reads input frames
+                          stride_t*t + kt - (kt-1); a call of t input frames
+                          writes (t-1)/stride_t + 1 output frames (y and
+                          residual have that many).  Streamed chunks of a
+                          multiple of stride_t frames give the whole
+                          sequence's outputs.                               */
+  int stride_h, stride_w;            /* must be 1                            */
   int dil_t, dil_h, dil_w;           /* must be 1                            */
   int groups;                        /* must be 1                            */
   cc3d_dtype dtype;

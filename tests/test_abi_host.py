@@ -66,12 +66,22 @@ def _desc(**kw):
     return d
 
 
-@pytest.mark.parametrize("field,value", [("stride_t", 2), ("stride_h", 2), ("groups", 2),
+@pytest.mark.parametrize("field,value", [("stride_t", 3), ("stride_h", 2), ("groups", 2),
                                          ("dil_t", 2), ("kh", 2), ("pad_h", 0), ("c_out", 40),
                                          ("c_in", 20), ("kt", 5)])
 def test_unsupported_descriptors_refused(lib, field, value):
     out = ctypes.c_void_p()
     assert cc3d.cc3d_plan_create(_desc(**{field: value}), out) == cc3d.ERR_UNSUPPORTED
+    assert not out.value
+
+
+@pytest.mark.parametrize("kw", [dict(dtype=cc3d.FP32), dict(c_in=3),
+                                dict(c_in=3, kh=1, kw=1, pad_h=0, pad_w=0)])
+def test_temporal_stride_only_on_the_tensor_core_path(lib, kw):
+    """Stride 2 in time is a bf16 tensor-core descriptor; the fp32 and the
+    thin (c_in <= 8) variants refuse it before any device query."""
+    out = ctypes.c_void_p()
+    assert cc3d.cc3d_plan_create(_desc(stride_t=2, **kw), out) == cc3d.ERR_UNSUPPORTED
     assert not out.value
 
 

@@ -232,8 +232,9 @@ cc3d_status check_desc(const cc3d_desc *d, int *variant) {
   if (d->n < 1 || d->c_in < 1 || d->c_out < 1 || d->h < 1 || d->w < 1 || d->max_t < 1)
     return CC3D_ERR_INVALID_ARG;
   if (d->kt < 1 || d->kh < 1 || d->kw < 1) return CC3D_ERR_INVALID_ARG;
-  if (d->stride_t != 1 || d->stride_h != 1 || d->stride_w != 1 || d->dil_t != 1 ||
-      d->dil_h != 1 || d->dil_w != 1 || d->groups != 1)
+  // temporal stride 2: the downsample path's time_conv (tensor-core path)
+  if (d->stride_t < 1 || d->stride_t > 2 || d->stride_h != 1 || d->stride_w != 1 ||
+      d->dil_t != 1 || d->dil_h != 1 || d->dil_w != 1 || d->groups != 1)
     return CC3D_ERR_UNSUPPORTED;
   if (d->kh % 2 == 0 || d->kw % 2 == 0 || d->pad_h != d->kh / 2 || d->pad_w != d->kw / 2)
     return CC3D_ERR_UNSUPPORTED;
@@ -241,7 +242,7 @@ cc3d_status check_desc(const cc3d_desc *d, int *variant) {
   if (d->epi < CC3D_EPI_BIAS || d->epi > CC3D_EPI_BIAS_RMS_SILU) return CC3D_ERR_INVALID_ARG;
   if (d->epi == CC3D_EPI_BIAS_RMS_SILU && !d->gamma) return CC3D_ERR_INVALID_ARG;
   if (d->dtype == CC3D_FP32) {
-    if (d->epi != CC3D_EPI_BIAS) return CC3D_ERR_UNSUPPORTED;
+    if (d->epi != CC3D_EPI_BIAS || d->stride_t != 1) return CC3D_ERR_UNSUPPORTED;
     *variant = CC3D_VARIANT_FP32;
     return CC3D_OK;
   }
@@ -249,7 +250,8 @@ cc3d_status check_desc(const cc3d_desc *d, int *variant) {
   if (d->c_out % 16 != 0) return CC3D_ERR_UNSUPPORTED;
   if (d->c_in <= 8) {
     // thin path: whole K gathered per pixel, one N tile, bias epilogue
-    if (d->epi != CC3D_EPI_BIAS || d->c_out > 256) return CC3D_ERR_UNSUPPORTED;
+    if (d->epi != CC3D_EPI_BIAS || d->c_out > 256 || d->stride_t != 1)
+      return CC3D_ERR_UNSUPPORTED;
     if (d->kt * d->kh * d->kw * d->c_in > 256) return CC3D_ERR_UNSUPPORTED;
     *variant = CC3D_VARIANT_THIN;
     return CC3D_OK;
@@ -362,8 +364,10 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
     // whole-sequence call of one plan run identical arithmetic.
     {
       UmmaConfig cfg;
+      // (the largest call's output frames)
+      const int max_out = (desc->max_t - 1) / desc->stride_t + 1;
       if (!choose_umma_config(desc->n, desc->c_in, desc->c_out, desc->h, desc->w, desc->kt,
-                              desc->kh, desc->epi == CC3D_EPI_BIAS_RMS_SILU, desc->max_t,
+                              desc->kh, desc->epi == CC3D_EPI_BIAS_RMS_SILU, max_out,
                               p->sm_count, &cfg)) {
         s = CC3D_ERR_UNSUPPORTED;
         goto fail;
@@ -442,9 +446,10 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
     return reject(CC3D_ERR_ALIGNMENT);
   const size_t esz = d.dtype == CC3D_FP32 ? 4 : 2;
   const int front = d.kt - 1;
+  const int t_out = (t - 1) / d.stride_t + 1;  // frames of y (and of residual)
   const size_t in_frame = static_cast<size_t>(d.h) * d.w * d.c_in * esz;
   const size_t out_frame = static_cast<size_t>(d.h) * d.w * d.c_out * esz;
-  const size_t x_bytes = in_frame * d.n * t, y_bytes = out_frame * d.n * t;
+  const size_t x_bytes = in_frame * d.n * t, y_bytes = out_frame * d.n * t_out;
   const size_t c_bytes = in_frame * d.n * front;
   const size_t nc_bytes = out_frame * d.n * 2;
   if (overlaps(cache_out, c_bytes, cache_in, c_bytes) || overlaps(cache_out, c_bytes, x, x_bytes) ||
@@ -541,8 +546,9 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
     a.y = static_cast<__nv_bfloat16 *>(y);
     a.status = status;
     a.wait_limit_ns = wait_limit_ns();
-    a.n = d.n; a.t = t; a.h = d.h; a.w = d.w; a.c_in = d.c_in; a.c_out = d.c_out;
+    a.n = d.n; a.t = t_out; a.h = d.h; a.w = d.w; a.c_in = d.c_in; a.c_out = d.c_out;
     a.kt = d.kt; a.kh = d.kh; a.kw = d.kw; a.pad_h = d.pad_h; a.pad_w = d.pad_w;
+    a.stride_t = d.stride_t;
     a.nt = p->nt; a.n_ntiles = p->n_ntiles;
     a.sub = p->sub; a.nbuf = p->nbuf; a.split = p->split; a.pair = p->pair;
     a.tiles_w = (d.w + tile_w - 1) / tile_w;
@@ -550,7 +556,7 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
     a.na = p->na; a.nb = p->nb; a.tmem_cols = p->tmem_cols;
     a.epi = static_cast<int>(d.epi);
     a.has_cache = (cache_in && front > 0) ? 1 : 0;
-    tiles = static_cast<uint64_t>(d.n) * t * a.tiles_h * a.tiles_w * a.n_ntiles;
+    tiles = static_cast<uint64_t>(d.n) * t_out * a.tiles_h * a.tiles_w * a.n_ntiles;
     uint64_t grid;
     if (p->split > 1 || p->pair) {
       // one cluster (of `split` CTAs, or a pair) per tile, at most as many as
@@ -568,7 +574,7 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
   if (e == cudaSuccess && cache_out && front > 0)
     e = launch_cache_update(cache_in, x, cache_out, d.n, t, front, in_frame, stream);
   if (e == cudaSuccess && next_cache_out)
-    e = launch_cache_update(next_cache_in, y, next_cache_out, d.n, t, 2, out_frame, stream);
+    e = launch_cache_update(next_cache_in, y, next_cache_out, d.n, t_out, 2, out_frame, stream);
   if (e != cudaSuccess) return reject(from_cuda(e));
   std::lock_guard<std::mutex> lk(p->mu);
   p->st.calls++;

@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int kt = kt_lo + ia / n_cc, cc = ia % n_cc;
           // A frame before the chunk with no cache is all zeros: its stage
           // (and its taps' weights) is skipped here and by the MMA issuer.
-          if (tc0.t + kt - (p.kt - 1) < 0 && !p.has_cache) continue;
+          if (p.stride_t * tc0.t + kt - (p.kt - 1) < 0 && !p.has_cache) continue;
           if (!mbar_wait_bounded(&empty_a[sa], pa ^ 1, p.wait_limit_ns, p.status, 1)) {
             ok = false;
             break;
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (pair_leader) mbar_arrive_expect_tx(&full_a[sa], PAIR ? 2u * a_tx : a_tx);
           a_used |= 1u << sa;
           a_par = (a_par & ~(1u << sa)) | (pa << sa);
-          const int tau = tc0.t + kt - (p.kt - 1);
+          const int tau = p.stride_t * tc0.t + kt - (p.kt - 1);  // input frame
           const bool from_cache = tau < 0;  // (zero frames were skipped above)
           const CUtensorMap *map = from_cache ? &map_cache : &map_x;
           const int tcoord = from_cache ? tau + (p.kt - 1) : tau;
@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ia = 0; ia < n_a && ok; ++ia) {
           // the same zero-frame stages the producer skipped; adding their
           // exact zeros would not change the accumulator
-          if (tcm.t + kt_lo + ia / n_cc - (p.kt - 1) < 0 && !p.has_cache) continue;
+          if (p.stride_t * tcm.t + kt_lo + ia / n_cc - (p.kt - 1) < 0 && !p.has_cache) continue;
           if (!mbar_wait_bounded(&full_a[sa], pa, p.wait_limit_ns, p.status, 3)) {
             ok = false;
             break;
@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- the partial sums of the cluster meet in the owner CTA ----
         uint32_t live = 0;  // ranks whose tap is not a causal zero frame
         for (int rr = 0; rr < p.split; ++rr)
-          if (p.has_cache || tc0.t + rr - (p.kt - 1) >= 0) live |= 1u << rr;
+          if (p.has_cache || p.stride_t * tc0.t + rr - (p.kt - 1) >= 0) live |= 1u << rr;
         const bool own_live = (live >> rank) & 1u;
         const int n0 = tc0.ntile * p.nt;
         const int chunks_per_sub = p.nt / kXC;

@@ -20,8 +20,9 @@ struct UmmaArgs {
   __nv_bfloat16 *y;               // [n][t][h][w][c_out]
   int *status;                    // device status word
   unsigned long long wait_limit_ns;
-  int n, t, h, w, c_in, c_out;
+  int n, t, h, w, c_in, c_out;    // t: output frames of this call
   int kt, kh, kw, pad_h, pad_w;
+  int stride_t;                   // output frame t reads input frames stride_t * t + kt - (kt - 1)
   int nt, n_ntiles, tiles_w, tiles_h;
   int na, nb;                     // pipeline depths (A halo stages, B weight stages)
   int tmem_cols;

@@ -97,8 +97,9 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   if ((d->epi == CC3D_EPI_BIAS_RESIDUAL) != (residual != nullptr)) return CC3D_ERR_INVALID_ARG;
   if (d->epi != CC3D_EPI_BIAS_RMS_SILU && (next_cache_in || next_cache_out))
     return CC3D_ERR_INVALID_ARG;
-  if (d->stride_t != 1 || d->stride_h != 1 || d->stride_w != 1 || d->dil_t != 1 ||
-      d->dil_h != 1 || d->dil_w != 1 || d->groups != 1 || d->dtype != CC3D_BF16)
+  if (d->stride_t < 1 || d->stride_t > 2 || d->stride_h != 1 || d->stride_w != 1 ||
+      d->dil_t != 1 || d->dil_h != 1 || d->dil_w != 1 || d->groups != 1 ||
+      d->dtype != CC3D_BF16)
     return CC3D_ERR_UNSUPPORTED;
   if (d->kh != d->kw || (d->kh != 1 && d->kh != 3) || d->kt > 3 || d->pad_h != d->kh / 2 ||
       d->pad_w != d->kw / 2)
@@ -117,7 +118,8 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   const int front = d->kt - 1;
   const size_t in_frame = size_t(d->h) * d->w * d->c_in * 2;
   const size_t out_frame = size_t(d->h) * d->w * d->c_out * 2;
-  const size_t xb = in_frame * d->n * t, yb = out_frame * d->n * t;
+  const int t_out = (t - 1) / d->stride_t + 1;  // frames of y
+  const size_t xb = in_frame * d->n * t, yb = out_frame * d->n * t_out;
   const size_t cb = in_frame * d->n * front, ncb = out_frame * d->n * 2;
   if (overlap(cache_out, cb, cache_in, cb) || overlap(cache_out, cb, x, xb) ||
       overlap(cache_out, cb, y, yb) || overlap(next_cache_out, ncb, next_cache_in, ncb) ||
@@ -135,7 +137,8 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   // ---- tiles: the same choice cc3d_plan_create makes --------------------------------
   UmmaConfig cfg;
   if (!choose_umma_config(d->n, d->c_in, d->c_out, d->h, d->w, d->kt, d->kh,
-                          d->epi == CC3D_EPI_BIAS_RMS_SILU, d->max_t, n_sm, &cfg))
+                          d->epi == CC3D_EPI_BIAS_RMS_SILU, (d->max_t - 1) / d->stride_t + 1,
+                          n_sm, &cfg))
     return CC3D_ERR_UNSUPPORTED;
   const bool clustered = cfg.split > 1 || cfg.pair;
   const int max_clusters = clustered ? umma_max_clusters(cfg, d->kh) : 0;
@@ -183,7 +186,8 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   a.y = static_cast<__nv_bfloat16 *>(y);
   a.status = status;
   a.wait_limit_ns = 2000ull * 1000000ull;
-  a.n = d->n; a.t = t; a.h = d->h; a.w = d->w; a.c_in = d->c_in; a.c_out = d->c_out;
+  a.n = d->n; a.t = t_out; a.stride_t = d->stride_t;
+  a.h = d->h; a.w = d->w; a.c_in = d->c_in; a.c_out = d->c_out;
   a.kt = d->kt; a.kh = d->kh; a.kw = d->kw; a.pad_h = d->pad_h; a.pad_w = d->pad_w;
   a.nt = nt; a.n_ntiles = cfg.n_ntiles;
   a.sub = cfg.sub; a.nbuf = cfg.nbuf; a.split = cfg.split; a.pair = cfg.pair;
@@ -192,7 +196,7 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   a.na = cfg.na; a.nb = cfg.nb; a.tmem_cols = cfg.tmem_cols;
   a.epi = static_cast<int>(d->epi);
   a.has_cache = has_cache ? 1 : 0;
-  const uint64_t tiles = uint64_t(d->n) * t * a.tiles_h * a.tiles_w * a.n_ntiles;
+  const uint64_t tiles = uint64_t(d->n) * t_out * a.tiles_h * a.tiles_w * a.n_ntiles;
   uint64_t grid;
   if (clustered) {
     grid = (tiles < uint64_t(max_clusters) ? tiles : uint64_t(max_clusters)) *
@@ -206,6 +210,6 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   if (e == cudaSuccess && cache_out && front > 0)
     e = launch_cache_update(cache_in, x, cache_out, d->n, t, front, in_frame, stream);
   if (e == cudaSuccess && next_cache_out)
-    e = launch_cache_update(next_cache_in, y, next_cache_out, d->n, t, 2, out_frame, stream);
+    e = launch_cache_update(next_cache_in, y, next_cache_out, d->n, t_out, 2, out_frame, stream);
   return e == cudaSuccess ? CC3D_OK : CC3D_ERR_CUDA;
 }
