@@ -549,6 +549,7 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
     a.n = d.n; a.t = t_out; a.h = d.h; a.w = d.w; a.c_in = d.c_in; a.c_out = d.c_out;
     a.kt = d.kt; a.kh = d.kh; a.kw = d.kw; a.pad_h = d.pad_h; a.pad_w = d.pad_w;
     a.stride_t = d.stride_t;
+    a.vec32 = (reinterpret_cast<uintptr_t>(y) & 31u) == 0 ? 1 : 0;
     a.nt = p->nt; a.n_ntiles = p->n_ntiles;
     a.sub = p->sub; a.nbuf = p->nbuf; a.split = p->split; a.pair = p->pair;
     a.tiles_w = (d.w + tile_w - 1) / tile_w;

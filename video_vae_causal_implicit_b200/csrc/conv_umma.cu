@@ -84,9 +84,15 @@ __host__ __device__ constexpr uint32_t x_bytes(int split) {
 }
 
 struct SmemLayout {
-  uint32_t a_off, a_stage, slab, b_off, b_stage, x_off, bar_off, total;
+  uint32_t a_off, a_stage, slab, b_off, b_stage, x_off, bar_off, p_off, total;
   int na, nb;
 };
+
+// Epilogue parameters staged in shared memory: bias[c_out] (and, for the
+// RMS epilogue, gamma[c_out], beta[c_out]).
+__host__ __device__ constexpr int param_floats(int c_out, int epi) {
+  return c_out * (epi == 2 ? 3 : 1);
+}
 
 __host__ __device__ inline uint32_t round_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
@@ -102,7 +108,7 @@ __host__ __device__ inline int halo_cols(int kc, int sub, int kw) {
 }
 
 __host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw, int na, int nb,
-                                                  int sub, int split, bool pair = false) {
+                                                  int sub, int split, bool pair, int params) {
   SmemLayout L;
   const uint32_t hh = kTH + kh - 1, hw = static_cast<uint32_t>(halo_cols(kc, sub, kw));
   if (uses_sw128(kc)) {
@@ -122,7 +128,9 @@ __host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw
   L.bar_off = round_up(L.x_off + x_bytes(split), 64u);
   // full_a, empty_a, full_b, empty_b, acc_full[2], acc_empty[2], drain,
   // (split: x_ready[4][2], x_free[4][2]), tmem slot
-  L.total = L.bar_off + 8u * (2 * na + 2 * nb + 5 + (split > 1 ? x_bar_count(split) : 0)) + 16u;
+  L.p_off = round_up(
+      L.bar_off + 8u * (2 * na + 2 * nb + 5 + (split > 1 ? x_bar_count(split) : 0)) + 16u, 16u);
+  L.total = L.p_off + 4u * static_cast<uint32_t>(params);
   return L;
 }
 
@@ -147,17 +155,29 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, const UmmaArgs &p) {
   return c;
 }
 
-// 16 consecutive fp32 parameters (bias / gamma / beta) of 16-byte-aligned
-// rows as four 16-byte loads; every lane of a warp reads the same address.
-__device__ __forceinline__ void ld_param16(const float *src, float (&v)[16]) {
-  const float4 *s4 = reinterpret_cast<const float4 *>(src);
+// 16 consecutive fp32 parameters (bias / gamma / beta, staged in shared
+// memory at the 16-byte-aligned address `src`) as four 16-byte loads; every
+// lane of a warp reads the same address (a broadcast).  Volatile, so that
+// the compiler issues them where they are used instead of hoisting every
+// group's parameters into registers at once.
+__device__ __forceinline__ void ld_param16(uint32_t src, float (&v)[16]) {
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const float4 f = __ldg(s4 + u);
-    v[4 * u] = f.x;
-    v[4 * u + 1] = f.y;
-    v[4 * u + 2] = f.z;
-    v[4 * u + 3] = f.w;
+  for (int u = 0; u < 4; ++u)
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v[4 * u]), "=f"(v[4 * u + 1]), "=f"(v[4 * u + 2]), "=f"(v[4 * u + 3])
+                 : "r"(src + 16u * u));
+}
+
+// 16 bf16 values (two 16-byte halves) to global memory: one 256-bit store
+// when the destination is 32-byte aligned, else two 128-bit stores.
+__device__ __forceinline__ void store_bf16x16(__nv_bfloat16 *dst, const uint4 &lo, const uint4 &hi,
+                                              int vec32) {
+  if (vec32) {
+    st_global_v8(dst, lo, hi);
+  } else {
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+    d[0] = lo;
+    d[1] = hi;
   }
 }
 
@@ -172,7 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // request, not a guarantee).
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const SmemLayout L = make_layout(KC, p.nt, KS, KS, p.na, p.nb, SUB, p.split, PAIR);
+  const SmemLayout L =
+      make_layout(KC, p.nt, KS, KS, p.na, p.nb, SUB, p.split, PAIR, param_floats(p.c_out, p.epi));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
   uint64_t *full_a = bars;
   uint64_t *empty_a = full_a + L.na;
@@ -450,6 +471,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // this warp's receive slots: [slot][sending rank index][quad of 4
     // columns][lane][4 fp32]; x_lane(slot, sender) is this lane's quad 0
     const int n_send = p.split - 1;
+    // bias (and gamma, beta) of every output channel, staged once: the
+    // per-column reads below are then shared-memory broadcasts
+    float *sp = reinterpret_cast<float *>(smem + L.p_off);
+    for (int i = static_cast<int>(threadIdx.x) - 64; i < p.c_out; i += 32 * kEpiWarps) {
+      sp[i] = p.bias[i];
+      if (p.epi == 2) {
+        sp[p.c_out + i] = p.gamma[i];
+        sp[2 * p.c_out + i] = p.beta ? p.beta[i] : 0.f;
+      }
+    }
+    named_barrier_sync(1, 32 * kEpiWarps);  // (the epilogue warps only)
+    // (shared addresses of the three vectors)
+    const uint32_t s_bias = smem_u32(sp), s_gamma = s_bias + 4u * static_cast<uint32_t>(p.c_out),
+                   s_beta = s_gamma + 4u * static_cast<uint32_t>(p.c_out);
     auto x_lane = [&](uint32_t slot, int sender) -> uint32_t {
       return smem_base + L.x_off +
              ((static_cast<uint32_t>(q) * kXSlots + slot) * static_cast<uint32_t>(n_send) +
@@ -588,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   static_cast<uint32_t>(dst_rank)));
             {
               float bv[16];
-              ld_param16(p.bias + n0 + j0, bv);
+              ld_param16(s_bias + 4u * static_cast<uint32_t>(n0 + j0), bv);
 #pragma unroll
               for (int i = 0; i < kXC; ++i) v[i] += bv[i];
             }
@@ -611,9 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               o1.y = pack_bf16x2(v[10], v[11]);
               o1.z = pack_bf16x2(v[12], v[13]);
               o1.w = pack_bf16x2(v[14], v[15]);
-              uint4 *dst = reinterpret_cast<uint4 *>(p.y + pix * p.c_out + n0 + j0);
-              dst[0] = o0;
-              dst[1] = o1;
+              store_bf16x16(p.y + pix * p.c_out + n0 + j0, o0, o1, p.vec32);
             }
           }
         }
@@ -652,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int u = 0; u < 3; ++u) {
               if (u >= nld) continue;
               float bv[16];
-              ld_param16(p.bias + n0 + j0 + 16 * u, bv);
+              ld_param16(s_bias + 4u * static_cast<uint32_t>(n0 + j0 + 16 * u), bv);
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const float hv = __uint_as_float(raw[16 * u + i]) + bv[i];
@@ -662,30 +695,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           inv = sqrtf(static_cast<float>(p.c_out)) / fmaxf(sqrtf(ss), 1e-12f);
         }
-        // pass 2: bias (+ residual | RMS scale + SiLU) -> bf16 -> global
-        for (int j0 = 0; j0 < p.nt; j0 += 48) {
-          const int nld = (p.nt - j0) >= 48 ? 3 : (p.nt - j0) / 16;
-          uint4 res[6];
-          if (p.epi == 1 && valid) {
-            // residual loads first, so their latency overlaps the TMEM reads
+        // pass 2: bias (+ residual | RMS scale + SiLU) -> bf16 -> global, in
+        // groups of 32 columns; the next group's tensor-memory loads are in
+        // flight while this group is converted and stored
+        const int n_groups = (p.nt + 31) / 32;
+        auto load_group = [&](int j0, uint32_t(&dst)[32]) {
+          const int nld = (p.nt - j0) >= 32 ? 2 : 1;
+          __syncwarp();
 #pragma unroll
-            for (int u = 0; u < 3; ++u)
+          for (int u = 0; u < 2; ++u)
+            if (u < nld) tmem_ld16_nowait(taddr + j0 + 16 * u, dst + 16 * u);
+        };
+        uint32_t raw[32];
+        load_group(0, raw);
+        tmem_wait_ld();
+        tmem_regs_after_wait<32>(raw);
+        for (int g = 0; g < n_groups; ++g) {
+          const int j0 = 32 * g;
+          const int nld = (p.nt - j0) >= 32 ? 2 : 1;
+          const bool more = g + 1 < n_groups;
+          uint4 res[4];
+          if (p.epi == 1 && valid) {
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
               if (u < nld) {
                 const uint4 *rr = reinterpret_cast<const uint4 *>(rrow + j0 + 16 * u);
                 res[2 * u] = rr[0];
                 res[2 * u + 1] = rr[1];
               }
           }
-          uint32_t raw[48];
-          __syncwarp();
-#pragma unroll
-          for (int u = 0; u < 3; ++u)
-            if (u < nld) tmem_ld16_nowait(taddr + j0 + 16 * u, raw + 16 * u);
-          tmem_wait_ld();
-          tmem_regs_after_wait<48>(raw);
-          if (last_sub && j0 + 48 >= p.nt) {
-            // last read of this accumulator buffer: hand it back to the MMA
-            // warp (a pair's follower: to the leader's)
+          uint32_t nxt[32];
+          if (more) {
+            load_group(j0 + 32, nxt);
+          } else if (last_sub) {
+            // every read of this accumulator buffer has completed: hand it
+            // back to the MMA warp (a pair's follower: to the leader's)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -696,13 +740,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
 #pragma unroll
-          for (int u = 0; u < 3; ++u) {
+          for (int u = 0; u < 2; ++u) {
             if (u >= nld) continue;
             const int j = j0 + 16 * u;
             float v[16];
             {
               float bv[16];
-              ld_param16(p.bias + n0 + j, bv);
+              ld_param16(s_bias + 4u * static_cast<uint32_t>(n0 + j), bv);
 #pragma unroll
               for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(raw[16 * u + i]) + bv[i];
             }
@@ -716,13 +760,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             } else if (p.epi == 2) {
               float gv[16], be[16];
-              ld_param16(p.gamma + n0 + j, gv);
-              if (p.beta) {
-                ld_param16(p.beta + n0 + j, be);
-              } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) be[i] = 0.f;
-              }
+              ld_param16(s_gamma + 4u * static_cast<uint32_t>(n0 + j), gv);
+              ld_param16(s_beta + 4u * static_cast<uint32_t>(n0 + j), be);
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 float a = v[i] * inv * gv[i];
@@ -740,10 +779,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               o1.y = pack_bf16x2(v[10], v[11]);
               o1.z = pack_bf16x2(v[12], v[13]);
               o1.w = pack_bf16x2(v[14], v[15]);
-              uint4 *dst = reinterpret_cast<uint4 *>(yrow + j);
-              dst[0] = o0;
-              dst[1] = o1;
+              store_bf16x16(yrow + j, o0, o1, p.vec32);
             }
+          }
+          if (more) {
+            tmem_wait_ld();
+            tmem_regs_after_wait<32>(nxt);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) raw[i] = nxt[i];
           }
         }
       }  // sub-tiles
@@ -768,9 +811,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb, int sub, int split,
-                       int pair) {
+                       int pair, int params) {
   // (a pair's CTA holds one 8 x 16 MMA tile: sub counts tile widths)
-  return make_layout(kc, nt, kh, kw, na, nb, pair ? 1 : sub, split, pair != 0).total +
+  return make_layout(kc, nt, kh, kw, na, nb, pair ? 1 : sub, split, pair != 0, params).total +
          1024;  // + alignment slack
 }
 
@@ -782,17 +825,24 @@ bool finish_config(int ks, UmmaConfig &c) {
   c.tmem_cols = 32;
   while (c.tmem_cols < c.nbuf * cta_sub * c.nt) c.tmem_cols *= 2;
   if (c.tmem_cols > 512) return false;
-  c.na = 2;
+  // A 3 x 3 halo stage feeds nine weight stages, so two of them keep the
+  // tensor pipe busy; with a 1 x 1 spatial kernel every weight stage needs
+  // a halo stage of its own, and both rings are as deep as the budget allows
+  // (two would leave the MMAs waiting on each load's round trip).
   c.nb = 8;
-  // (a split's exchange staging gets room of its own above the usual budget)
-  const size_t budget = (c.split > 1 ? 216 : 200) * 1024;
-  while (c.nb > 2 &&
-         umma_smem_bytes(c.kc, c.nt, ks, ks, c.na, c.nb, c.sub, c.split, c.pair) > budget)
+  c.na = ks == 1 ? c.nb : 2;
+  // (a split's exchange staging gets room of its own above the usual
+  // budget, and so do the staged epilogue parameters)
+  const size_t budget = (c.split > 1 ? 216 : 200) * 1024 + 4 * static_cast<size_t>(c.params);
+  while (c.nb > 2 && umma_smem_bytes(c.kc, c.nt, ks, ks, c.na, c.nb, c.sub, c.split, c.pair,
+                                     c.params) > budget) {
     --c.nb;
-  int per_sm = static_cast<int>(
-      (228 * 1024) /
-      (umma_launch_smem(c.kc, c.nt, ks, c.na, c.nb, c.tmem_cols, c.sub, c.split, c.pair) +
-       1024));
+    if (ks == 1) c.na = c.nb;
+  }
+  const size_t smem =
+      umma_launch_smem(c.kc, c.nt, ks, c.na, c.nb, c.tmem_cols, c.sub, c.split, c.pair, c.params);
+  if (smem > 227 * 1024) return false;
+  int per_sm = static_cast<int>((228 * 1024) / (smem + 1024));
   if (per_sm > 512 / c.tmem_cols) per_sm = 512 / c.tmem_cols;
   if (per_sm > 2) per_sm = 2;
   if (c.pair) per_sm = 1;
@@ -850,6 +900,7 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
   one.nt = largest_nt(256);
   if (!one.nt) return false;
   one.n_ntiles = c_out / one.nt;
+  one.params = param_floats(c_out, rms_epi ? 2 : 0);
   if (!finish_config(ks, one)) return false;
   *cfg = one;
   const long long tiles1 = static_cast<long long>(n) * ((h + kTH - 1) / kTH) *
@@ -948,8 +999,8 @@ cudaError_t umma_prepare() {
 }
 
 size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols, int sub,
-                        int split, int pair) {
-  size_t smem = umma_smem_bytes(kc, nt, ks, ks, na, nb, sub, split, pair);
+                        int split, int pair, int params) {
+  size_t smem = umma_smem_bytes(kc, nt, ks, ks, na, nb, sub, split, pair, params);
   // A CTA that holds more than half of tensor memory must have its SM to
   // itself; asking for more than half the shared memory guarantees that.
   if (tmem_cols > 256 && smem < 116 * 1024) smem = 116 * 1024;
@@ -999,7 +1050,7 @@ int umma_max_clusters(const UmmaConfig &c, int ks) {
   UmmaKernel k = umma_kernel_for(c.kc, ks, c.sub, c.pair);
   if (!k) return 0;
   const size_t smem =
-      umma_launch_smem(c.kc, c.nt, ks, c.na, c.nb, c.tmem_cols, c.sub, c.split, c.pair);
+      umma_launch_smem(c.kc, c.nt, ks, c.na, c.nb, c.tmem_cols, c.sub, c.split, c.pair, c.params);
   cudaLaunchAttribute attr;
   const cudaLaunchConfig_t cfg =
       umma_launch_config(static_cast<unsigned>(csize), smem, csize, nullptr, &attr);
@@ -1015,8 +1066,9 @@ cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_ca
                              const CUtensorMap &map_w, const UmmaArgs &args, int kc,
                              unsigned grid, cudaStream_t stream) {
   if (args.kh != args.kw || (args.kh != 1 && args.kh != 3)) return cudaErrorInvalidValue;
-  const size_t smem = umma_launch_smem(kc, args.nt, args.kh, args.na, args.nb, args.tmem_cols,
-                                       args.sub, args.split, args.pair);
+  const size_t smem =
+      umma_launch_smem(kc, args.nt, args.kh, args.na, args.nb, args.tmem_cols, args.sub,
+                       args.split, args.pair, param_floats(args.c_out, args.epi));
   if (smem > 227 * 1024 || (args.sub != 1 && args.sub != 2) || args.nbuf < 1 || args.nbuf > 2)
     return cudaErrorInvalidValue;
   if (args.split != 1 && (args.split != args.kt || args.split > 4 || grid % args.split != 0 ||

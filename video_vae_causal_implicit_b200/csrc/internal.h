@@ -34,12 +34,14 @@ struct UmmaArgs {
                                   // temporal tap each, reduced in the last one
   int pair;                       // 1: a cluster of 2 CTAs runs 2-SM MMAs on a 16 x 16 px
                                   // tile (sub is then 2: the tile width in MMA tiles)
+  int vec32;                      // 1: y and residual are 32-byte aligned (256-bit stores)
 };
 
 // Tile configuration of the UMMA conv for a plan (chosen from n, c_in, c_out,
 // h, w, the epilogue and the plan's max_t -- never from a call's t).
 struct UmmaConfig {
   int kc, nt, n_ntiles, sub, nbuf, split, pair, na, nb, tmem_cols, ctas_per_sm;
+  int params;  // epilogue parameters staged in shared memory (floats)
 };
 bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
                         int max_t, int sm_count, UmmaConfig *cfg);
@@ -48,11 +50,11 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
 int umma_max_clusters(const UmmaConfig &cfg, int ks);
 
 size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb, int sub, int split,
-                       int pair);
+                       int pair, int params);
 cudaError_t umma_prepare();
 // Dynamic shared memory a launch requests (with the one-CTA-per-SM rule).
 size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols, int sub,
-                        int split, int pair);
+                        int split, int pair, int params);
 int umma_tile_w();
 // TMA box of the A halo: columns (padded for the 128-byte swizzle) and
 // channels (64: swizzled pixel rows; 8: no-swizzle slabs).

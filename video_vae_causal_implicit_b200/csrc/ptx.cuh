@@ -295,6 +295,19 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 32 bytes (eight 32-bit words of lo, hi) to a 32-byte-aligned global address.
+__device__ __forceinline__ void st_global_v8(void *dst, const uint4 &lo, const uint4 &hi) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(lo.x),
+               "r"(lo.y), "r"(lo.z), "r"(lo.w), "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
+               : "memory");
+}
+
+// Barrier `id` (not 0, which __syncthreads uses) over `count` threads of
+// whole warps of the block.
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // After tmem_wait_ld(): ties each register to a point after the wait, so the
 // compiler cannot move a use of a loaded value above the wait.
 template <int N>

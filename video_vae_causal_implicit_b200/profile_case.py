@@ -13,6 +13,9 @@ Cases (seeded synthetic inputs, generated on the device):
   c4      the residual block on x[1,192,9,240,416]
   c4s     the residual block on a 3-frame slice x[1,192,3,240,416]
   c5big   384 -> 384, one frame of 360 x 640 with a 2-frame cache
+  tc192   the downsample path's time_conv: 192 -> 192, kernel (3, 1, 1),
+          stride 2 in time, x[1,192,17,120,208] (9 output frames)
+  tc384   the same at 384 channels on x[1,384,9,60,104] (5 output frames)
 Prints nothing but a final "ok"; timing comes from the profiler.
 """
 from __future__ import annotations
@@ -41,6 +44,10 @@ def build_case(name, dev):
         c, T, H, W = 192, (9 if name == "c4" else 3), 240, 416
     elif name == "c5big":
         c, T, H, W = 384, 1, 360, 640
+    elif name == "tc192":
+        c, T, H, W = 192, 17, 120, 208
+    elif name == "tc384":
+        c, T, H, W = 384, 9, 60, 104
     else:
         raise SystemExit(f"unknown case {name}")
     x = _rand((1, T, H, W, c), dev)
@@ -54,6 +61,12 @@ def build_case(name, dev):
         blk = cc3d.Block(w1, b1, g1, w2, b2, g2, h=H, w=W, max_t=T)
         y = torch.empty_like(x)
         return lambda: blk.forward(x, y), [blk]
+    if name in ("tc192", "tc384"):
+        wt = synth.kaiming_uniform(c, c, (3, 1, 1), 1).to(dev)
+        b = synth.uniform((c,), -0.1, 0.1, 2).to(dev)
+        plan = cc3d.Plan(wt, b, h=H, w=W, max_t=T, stride_t=2)
+        y = torch.empty((1, (T - 1) // 2 + 1, H, W, c), dtype=torch.bfloat16, device=dev)
+        return (lambda: plan.forward(x, y)), [plan]
     cout = 96 if name == "c3a" else c
     wt = synth.kaiming_uniform(cout, c, (3, 3, 3), 1).to(dev)
     b = synth.uniform((cout,), -0.1, 0.1, 2).to(dev)
