@@ -131,6 +131,9 @@ typedef struct {
                               frames too small to occupy the GPU            */
   int mma_ctas;            /* CTAs (SMs) per tensor-core MMA: 1, or 2 for a
                               CTA pair issuing 2-SM MMAs (M = 256)          */
+  int w_resident;          /* 1: the weights stay in shared memory for the
+                              whole launch (short K, one N tile), 0: they
+                              stream through a ring, once per tile          */
 } cc3d_stats;
 
 typedef struct cc3d_plan cc3d_plan;

@@ -164,6 +164,8 @@ def test_stride2_time_conv_full_size_sampled():
     n, c, t, h, w, k = 1, 192, 17, 120, 208, (3, 1, 1)
     case = synth.conv_case(c, c, t, h, w, n=n, k=k, seed_base=98)
     plan = _plan(case, n, h, w, t)
+    st = plan.stats()
+    assert (st.mma_ctas, st.w_resident) == (2, 1), "expected the pair with resident weights"
     x = to_dev(synth.ndhwc(case["x"]))
     y = torch.empty((n, t_out(t), h, w, c), dtype=torch.bfloat16, device="cuda")
     plan.forward(x, y)

@@ -81,6 +81,31 @@ def test_noalloc_matches_planned_conv_on_two_calls_in_a_row():
     torch.cuda.synchronize()
 
 
+def test_noalloc_matches_planned_time_conv_with_resident_weights():
+    """Temporal stride 2 with kernel (3, 1, 1): the CTA pair with every
+    weight stage resident in shared memory, as the planned call."""
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    c, t, h, w = 192, 17, 30, 52
+    case = synth.conv_case(c, c, t, h, w, k=(3, 1, 1), seed_base=4)
+    x = to_dev(synth.ndhwc(case["x"]))
+    wt, b = to_dev(case["w"]), to_dev(case["b"])
+    kw = dict(h=h, w=w, max_t=t)
+    plan = cc3d.Plan(wt, b, stride_t=2, **kw)
+    st = plan.stats()
+    assert (st.w_resident, st.mma_ctas) == (1, 2)
+    t_out = (t - 1) // 2 + 1
+    y_ref = torch.empty((1, t_out, h, w, c), dtype=torch.bfloat16, device="cuda")
+    plan.forward(x, y_ref)
+    y = torch.full_like(y_ref, float("nan"))
+    d = _desc_for(kw, wt, b)
+    d.stride_t = 2
+    res = cc3d.cc3d_forward_noalloc(d, _p(x), t, None, _p(y), None, None, None, None, stream)
+    assert res == cc3d.OK, cc3d.cc3d_status_string(res)
+    cc3d.sync_status()
+    assert torch.equal(y.cpu(), y_ref.cpu())
+    plan.close()
+
+
 def test_noalloc_refuses_weights_beyond_its_scratch():
     big = torch.empty((512, 512, 3, 3, 3), dtype=torch.bfloat16, device="cuda")  # 14 MB
     d = _desc_for(dict(h=8, w=8, max_t=1), big, None)

@@ -178,7 +178,7 @@ struct cc3d_plan {
   int device;
   // UMMA
   int kc, nt, n_ntiles, na, nb, tmem_cols, sm_count, ctas_per_sm, sub, nbuf, split, max_clusters;
-  int pair;
+  int pair, b_resident;
   CUtensorMap map_w;  // pair: the weight image as 128-byte swizzled rows
   uint8_t *wimg;
   // fp32 / thin
@@ -375,6 +375,7 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
       p->kc = cfg.kc; p->nt = cfg.nt; p->n_ntiles = cfg.n_ntiles; p->sub = cfg.sub;
       p->nbuf = cfg.nbuf; p->na = cfg.na; p->nb = cfg.nb; p->tmem_cols = cfg.tmem_cols;
       p->ctas_per_sm = cfg.ctas_per_sm; p->split = cfg.split; p->pair = cfg.pair;
+      p->b_resident = cfg.b_resident;
       p->max_clusters = 0;
       if (cfg.split > 1 || cfg.pair) {
         p->max_clusters = umma_max_clusters(cfg, desc->kh);
@@ -387,6 +388,7 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
     p->st.k_chunk = p->kc;
     p->st.k_split = p->split;
     p->st.mma_ctas = p->pair ? 2 : 1;
+    p->st.w_resident = p->b_resident;
     const size_t bytes = sizeof(__nv_bfloat16) * desc->c_out * desc->c_in * taps;
     if (cudaMalloc(&p->wimg, bytes) != cudaSuccess) { s = CC3D_ERR_OOM; goto fail; }
     e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(desc->weight), p->wimg,
@@ -550,6 +552,7 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
     a.kt = d.kt; a.kh = d.kh; a.kw = d.kw; a.pad_h = d.pad_h; a.pad_w = d.pad_w;
     a.stride_t = d.stride_t;
     a.vec32 = (reinterpret_cast<uintptr_t>(y) & 31u) == 0 ? 1 : 0;
+    a.b_resident = p->b_resident;
     a.nt = p->nt; a.n_ntiles = p->n_ntiles;
     a.sub = p->sub; a.nbuf = p->nbuf; a.split = p->split; a.pair = p->pair;
     a.tiles_w = (d.w + tile_w - 1) / tile_w;

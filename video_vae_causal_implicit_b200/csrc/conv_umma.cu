@@ -295,10 +295,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pa = 0, pb = 0;
       // stages issued at least once, and the phase parity of their last issue
       uint32_t a_used = 0, a_par = 0, b_used = 0, b_par = 0;
+      // weight stage `stage_idx` (tap-major, then channel chunk) of N tile
+      // `ntile` into B slot `slot`: the whole stage, or this CTA's half of
+      // its N rows on a pair
+      auto load_b = [&](int slot, size_t stage_idx, int ntile) {
+        if (pair_leader)
+          mbar_arrive_expect_tx(&full_b[slot], PAIR ? 2u * L.b_stage : L.b_stage);
+        if constexpr (PAIR) {
+          // rows of the weight image [ntile][tap][cchunk][NT][64]
+          const int row = static_cast<int>(
+              ((static_cast<size_t>(ntile) * p.kt * KS * KS * n_cc + stage_idx) * p.nt) +
+              rank * (p.nt / 2));
+          tma_load_2d_pair(smem_base + L.b_off + slot * L.b_stage, &map_w,
+                           lead_full_b + 8u * slot, 0, row);
+        } else {
+          const uint8_t *wsrc =
+              p.wimg + static_cast<size_t>(ntile) * p.kt * KS * KS * n_cc * L.b_stage;
+          bulk_load(smem_base + L.b_off + slot * L.b_stage, wsrc + stage_idx * L.b_stage,
+                    L.b_stage, &full_b[slot]);
+        }
+      };
+      if (KS == 1 && p.b_resident) {
+        // one N tile and every weight stage in a slot of its own: loaded
+        // once here, read in place by the MMAs of every tile
+        for (int st = 0; st < L.nb; ++st) load_b(st, static_cast<size_t>(st), 0);
+        b_used = L.nb >= 32 ? 0xffffffffu : (1u << L.nb) - 1u;
+      }
       for (int tile = cid; tile < n_tiles && ok; tile += ncl) {
         const TileCoord tc0 = decode_tile(tile, p);
-        const uint8_t *wsrc =
-            p.wimg + static_cast<size_t>(tc0.ntile) * p.kt * KS * KS * n_cc * L.b_stage;
         for (int ia = 0; ia < n_a && ok; ++ia) {
           const int kt = kt_lo + ia / n_cc, cc = ia % n_cc;
           // A frame before the chunk with no cache is all zeros: its stage
@@ -329,28 +353,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                           tc0.h0 - KS / 2, tcoord, tc0.n);
           }
           if (++sa == L.na) { sa = 0; pa ^= 1; }
+          if (KS == 1 && p.b_resident) continue;
 #pragma unroll 1
           for (int ts = 0; ts < KS * KS; ++ts) {
             if (!mbar_wait_bounded(&empty_b[sb], pb ^ 1, p.wait_limit_ns, p.status, 2)) {
               ok = false;
               break;
             }
-            if (pair_leader) mbar_arrive_expect_tx(&full_b[sb], PAIR ? 2u * L.b_stage : L.b_stage);
             b_used |= 1u << sb;
             b_par = (b_par & ~(1u << sb)) | (pb << sb);
-            const size_t stage_idx = static_cast<size_t>(kt * KS * KS + ts) * n_cc + cc;
-            if constexpr (PAIR) {
-              // rows of the weight image [ntile][tap][cchunk][NT][64]: this
-              // CTA's half of the stage's N rows
-              const int row = static_cast<int>(
-                  ((static_cast<size_t>(tc0.ntile) * p.kt * KS * KS * n_cc + stage_idx) * p.nt) +
-                  rank * (p.nt / 2));
-              tma_load_2d_pair(smem_base + L.b_off + sb * L.b_stage, &map_w, lead_full_b + 8u * sb,
-                               0, row);
-            } else {
-              bulk_load(smem_base + L.b_off + sb * L.b_stage, wsrc + stage_idx * L.b_stage,
-                        L.b_stage, &full_b[sb]);
-            }
+            load_b(sb, static_cast<size_t>(kt * KS * KS + ts) * n_cc + cc, tc0.ntile);
             if (++sb == L.nb) { sb = 0; pb ^= 1; }
           }
         }
@@ -418,15 +430,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint64_t a_st = adesc0 + ((sa * L.a_stage) >> 4);
-#pragma unroll
-          for (int ts = 0; ts < KS * KS; ++ts) {
-            if (!mbar_wait_bounded(&full_b[sb], pb, p.wait_limit_ns, p.status, 4)) {
-              ok = false;
-              break;
-            }
+          // the MMAs of weight slot `slot` (phase parity `par`) with spatial tap `ts`
+          auto issue_b = [&](int slot, uint32_t par, int ts) -> bool {
+            if (!mbar_wait_bounded(&full_b[slot], par, p.wait_limit_ns, p.status, 4)) return false;
             tc_fence_after();
             const uint64_t a_tap = a_st + ((ts / KS) * halo_w + (ts % KS)) * pix16;
-            const uint64_t b_st = bdesc0 + ((sb * L.b_stage) >> 4);
+            const uint64_t b_st = bdesc0 + ((static_cast<uint32_t>(slot) * L.b_stage) >> 4);
 #pragma unroll
             for (int j = 0; j < KC / 16; ++j) {
               // every sub-tile (8 pixels further along the halo row) reuses
@@ -442,10 +451,27 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               accumulate = 1;
             }
-            // frees the B stage (in both CTAs of a pair) when these MMAs finish
-            if constexpr (PAIR) umma_commit_pair(&empty_b[sb], 3);
-            else umma_commit(&empty_b[sb]);
-            if (++sb == L.nb) { sb = 0; pb ^= 1; }
+            return true;
+          };
+          if (KS == 1 && p.b_resident) {
+            // resident weights: stage (kt, cc) sits in slot kt * n_cc + cc,
+            // loaded once (its first phase stays complete) and never freed
+            if (!issue_b(kt_lo * n_cc + ia, 0u, 0)) {
+              ok = false;
+              break;
+            }
+          } else {
+#pragma unroll
+            for (int ts = 0; ts < KS * KS; ++ts) {
+              if (!issue_b(sb, pb, ts)) {
+                ok = false;
+                break;
+              }
+              // frees the B stage (in both CTAs of a pair) when these MMAs finish
+              if constexpr (PAIR) umma_commit_pair(&empty_b[sb], 3);
+              else umma_commit(&empty_b[sb]);
+              if (++sb == L.nb) { sb = 0; pb ^= 1; }
+            }
           }
           if constexpr (PAIR) umma_commit_pair(&empty_a[sa], 3);
           else umma_commit(&empty_a[sa]);
@@ -819,7 +845,7 @@ size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb, int sub, 
 
 namespace {
 // Buffers, pipeline depths and residency of one tile shape.
-bool finish_config(int ks, UmmaConfig &c) {
+bool finish_config(int ks, int kt, int c_in, UmmaConfig &c) {
   const int cta_sub = c.pair ? 1 : c.sub;  // MMA tiles whose accumulators one CTA holds
   c.nbuf = (2 * cta_sub * c.nt <= 512) ? 2 : 1;  // double-buffered accumulators when they fit
   c.tmem_cols = 32;
@@ -838,6 +864,24 @@ bool finish_config(int ks, UmmaConfig &c) {
                                      c.params) > budget) {
     --c.nb;
     if (ks == 1) c.na = c.nb;
+  }
+  // A short K (a 1 x 1 spatial kernel) with a single N tile: every weight
+  // stage of the CTA fits in shared memory beside a halo ring of at least
+  // three stages, so the weights are loaded once per launch instead of once
+  // per tile (they were most of the bytes moved into shared memory).
+  c.b_resident = 0;
+  if (ks == 1 && c.split == 1 && c.n_ntiles == 1 && kt * (c_in / c.kc) <= 32) {
+    const int stages = kt * (c_in / c.kc);
+    const size_t budget_r = 216 * 1024 + 4 * static_cast<size_t>(c.params);
+    int na = 8;
+    while (na > 3 && umma_smem_bytes(c.kc, c.nt, 1, 1, na, stages, c.sub, 1, c.pair,
+                                     c.params) > budget_r)
+      --na;
+    if (umma_smem_bytes(c.kc, c.nt, 1, 1, na, stages, c.sub, 1, c.pair, c.params) <= budget_r) {
+      c.b_resident = 1;
+      c.na = na;
+      c.nb = stages;
+    }
   }
   const size_t smem =
       umma_launch_smem(c.kc, c.nt, ks, c.na, c.nb, c.tmem_cols, c.sub, c.split, c.pair, c.params);
@@ -860,7 +904,7 @@ long long mma_cycles(const UmmaConfig &c) {
   const long long math = c.nt <= 64 ? 48 : c.nt <= 96 ? 56 : c.nt / 2;
   const long long b_rows = c.pair ? c.nt / 2 : c.nt;
   const long long b_read = 32 * b_rows;
-  const long long b_write = 32 * b_rows / (c.pair ? 1 : c.sub);
+  const long long b_write = c.b_resident ? 0 : 32 * b_rows / (c.pair ? 1 : c.sub);
   const long long bytes = 4096 + b_read + b_write + 1000;
   const long long smem = (bytes + 119) / 120;
   return math > smem ? math : smem;
@@ -901,7 +945,7 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
   if (!one.nt) return false;
   one.n_ntiles = c_out / one.nt;
   one.params = param_floats(c_out, rms_epi ? 2 : 0);
-  if (!finish_config(ks, one)) return false;
+  if (!finish_config(ks, kt, c_in, one)) return false;
   *cfg = one;
   const long long tiles1 = static_cast<long long>(n) * ((h + kTH - 1) / kTH) *
                            ((w + kTW - 1) / kTW) * one.n_ntiles;
@@ -923,7 +967,7 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
     const long long slots = static_cast<long long>(sm_count) * one.ctas_per_sm;
     const long long cost_one = (calls_tiles + slots - 1) / slots * kt * 10;
     const long long cost_split = clusters > 0 ? (calls_tiles + clusters - 1) / clusters * 14 : 0;
-    if (clusters > 0 && finish_config(ks, sp) &&
+    if (clusters > 0 && finish_config(ks, kt, c_in, sp) &&
         tiles1 * kt <= static_cast<long long>(sm_count) * sp.ctas_per_sm && cost_split < cost_one) {
       *cfg = sp;
       return true;
@@ -942,7 +986,7 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
   two.nt = largest_nt(128);
   if (two.nt) {
     two.n_ntiles = c_out / two.nt;
-    if (finish_config(ks, two) && two.nbuf == 2) {
+    if (finish_config(ks, kt, c_in, two) && two.nbuf == 2) {
       const long long cost = frame_cost(two, nt_frames, h, w, sm_count);
       if (cost < best) {
         best = cost;
@@ -958,7 +1002,7 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
     UmmaConfig pr = one;
     pr.pair = 1;
     pr.sub = 2;  // the tile is two MMA tiles wide
-    if (finish_config(ks, pr) && pr.nbuf == 2) {
+    if (finish_config(ks, kt, c_in, pr) && pr.nbuf == 2) {
       const long long cost = frame_cost(pr, nt_frames, h, w, sm_count);
       if (cost <= best) {
         best = cost;
@@ -1075,6 +1119,9 @@ cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_ca
                           args.epi == 2 || args.sub != 1 || args.pair))
     return cudaErrorInvalidValue;
   if (args.pair && (kc != 64 || args.sub != 2 || grid % 2 != 0 || args.nt % 16 != 0))
+    return cudaErrorInvalidValue;
+  if (args.b_resident && (args.split != 1 || args.n_ntiles != 1 || args.nb > 32 ||
+                          args.nb != args.kt * args.kh * args.kw * (args.c_in / kc)))
     return cudaErrorInvalidValue;
   UmmaKernel k = umma_kernel_for(kc, args.kh, args.sub, args.pair);
   if (!k) return cudaErrorInvalidValue;

@@ -35,13 +35,16 @@ struct UmmaArgs {
   int pair;                       // 1: a cluster of 2 CTAs runs 2-SM MMAs on a 16 x 16 px
                                   // tile (sub is then 2: the tile width in MMA tiles)
   int vec32;                      // 1: y and residual are 32-byte aligned (256-bit stores)
+  int b_resident;                 // 1: one N tile, every weight stage (nb = kt*kh*kw*c_in/KC)
+                                  // in shared memory for the whole launch
 };
 
 // Tile configuration of the UMMA conv for a plan (chosen from n, c_in, c_out,
 // h, w, the epilogue and the plan's max_t -- never from a call's t).
 struct UmmaConfig {
   int kc, nt, n_ntiles, sub, nbuf, split, pair, na, nb, tmem_cols, ctas_per_sm;
-  int params;  // epilogue parameters staged in shared memory (floats)
+  int params;      // epilogue parameters staged in shared memory (floats)
+  int b_resident;  // every weight stage resident in shared memory (nb of them)
 };
 bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
                         int max_t, int sm_count, UmmaConfig *cfg);

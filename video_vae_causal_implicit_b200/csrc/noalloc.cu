@@ -188,6 +188,7 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   a.wait_limit_ns = 2000ull * 1000000ull;
   a.n = d->n; a.t = t_out; a.stride_t = d->stride_t;
   a.vec32 = (reinterpret_cast<uintptr_t>(y) & 31u) == 0 ? 1 : 0;
+  a.b_resident = cfg.b_resident;
   a.h = d->h; a.w = d->w; a.c_in = d->c_in; a.c_out = d->c_out;
   a.kt = d->kt; a.kh = d->kh; a.kw = d->kw; a.pad_h = d->pad_h; a.pad_w = d->pad_w;
   a.nt = nt; a.n_ntiles = cfg.n_ntiles;
