@@ -15,7 +15,8 @@ Functions (each cites the passage it follows in the C source):
   causal_conv3d         -- §10.3 WanCausalConv3d, bias once
   causal_conv3d_points  -- the same definition at chosen output voxels
   rms_norm              -- §10.2 WanRMS_norm (+ optional SiLU, §10.4)
-  resblock              -- §10.4 WanResidualBlock, identity shortcut
+  resblock              -- §10.4 WanResidualBlock: identity shortcut, or the
+                           1x1x1 conv_shortcut when C_in != C_out
   resblock_points       -- the same definition at chosen output voxels
   round_bf16            -- bfloat16 round-to-nearest-even of one double
 """
@@ -79,13 +80,17 @@ def _load():
             lib.orc_resblock.argtypes = [T, T, T, i, i, i, i, i, T, dp, dp, T, dp, dp, i, dp, dp, dp]
             lib.orc_resblock_points.argtypes = [T, T, T, i, i, i, i, i, T, dp, dp, T, dp, dp, i,
                                                 i, ip, dp]
+            lib.orc_resblock2.argtypes = [T, T, T, i, i, i, i, i, i, T, dp, dp, T, dp, dp, T, dp,
+                                          i, i, dp, dp, dp]
+            lib.orc_resblock2_points.argtypes = [T, T, T, i, i, i, i, i, i, T, dp, dp, T, dp, dp,
+                                                 T, dp, i, i, i, ip, dp]
             lib.orc_round_bf16.argtypes = [ctypes.c_double]
             lib.orc_round_bf16.restype = ctypes.c_double
             lib.orc_silu.argtypes = [ctypes.c_double]
             lib.orc_silu.restype = ctypes.c_double
             for name in ("orc_causal_conv3d", "orc_causal_conv3d_points", "orc_causal_conv3d_s",
                          "orc_causal_conv3d_points_s", "orc_rms_norm", "orc_resblock",
-                         "orc_resblock_points"):
+                         "orc_resblock_points", "orc_resblock2", "orc_resblock2_points"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -216,46 +221,54 @@ def rms_norm(x, gamma, beta=None, silu=False):
 
 
 def resblock(x, w1, b1, g1, w2, b2, g2, cache1=None, cache2=None, round_bf16=True,
-             return_acts=False):
-    """WanResidualBlock (identity shortcut).  Returns y float64 [N,C,T,H,W]
-    (and a0, a1 when return_acts)."""
+             return_acts=False, w_sc=None, b_sc=None, round_h1=False):
+    """WanResidualBlock from C_in = x's channels to C_out = w1's output
+    channels.  The shortcut is x itself (w_sc None, C_in == C_out) or the
+    1x1x1 conv_shortcut w_sc [C_out, C_in, 1, 1, 1] + b_sc.  round_bf16
+    rounds a0 and a1 to bf16; round_h1 also rounds conv1's output before
+    its RMS_norm.  Returns y float64 [N, C_out, T, H, W] (and a0, a1 when
+    return_acts)."""
     lib = _load()
     keep = []
-    N, C, T, H, W = _shape5(x)
+    N, Cin, T, H, W = _shape5(x)
+    Cout = _shape5(w1)[0]
     tx, t1, t2 = _view(x, keep), _view(cache1, keep), _view(cache2, keep)
-    tw1, tw2 = _view(w1, keep), _view(w2, keep)
-    y = np.empty((N, C, T, H, W), dtype=np.float64)
-    a0 = np.empty_like(y) if return_acts else None
-    a1 = np.empty_like(y) if return_acts else None
+    tw1, tw2, tsc = _view(w1, keep), _view(w2, keep), _view(w_sc, keep)
+    y = np.empty((N, Cout, T, H, W), dtype=np.float64)
+    a0 = np.empty((N, Cin, T, H, W), dtype=np.float64) if return_acts else None
+    a1 = np.empty((N, Cout, T, H, W), dtype=np.float64) if return_acts else None
     dp = ctypes.POINTER(ctypes.c_double)
-    rc = lib.orc_resblock(_ptr(tx), _ptr(t1), _ptr(t2), N, C, T, H, W,
-                          _ptr(tw1), _dvec(b1, keep), _dvec(g1, keep),
-                          _ptr(tw2), _dvec(b2, keep), _dvec(g2, keep),
-                          1 if round_bf16 else 0, y.ctypes.data_as(dp),
-                          a0.ctypes.data_as(dp) if a0 is not None else None,
-                          a1.ctypes.data_as(dp) if a1 is not None else None)
+    rc = lib.orc_resblock2(_ptr(tx), _ptr(t1), _ptr(t2), N, Cin, Cout, T, H, W,
+                           _ptr(tw1), _dvec(b1, keep), _dvec(g1, keep),
+                           _ptr(tw2), _dvec(b2, keep), _dvec(g2, keep),
+                           _ptr(tsc), _dvec(b_sc, keep),
+                           1 if round_bf16 else 0, 1 if round_h1 else 0, y.ctypes.data_as(dp),
+                           a0.ctypes.data_as(dp) if a0 is not None else None,
+                           a1.ctypes.data_as(dp) if a1 is not None else None)
     if rc != 0:
-        raise ValueError(f"orc_resblock failed ({rc})")
+        raise ValueError(f"orc_resblock2 failed ({rc})")
     return (y, a0, a1) if return_acts else y
 
 
 def resblock_points(x, w1, b1, g1, w2, b2, g2, points, cache1=None, cache2=None,
-                    round_bf16=True):
-    """The residual block at chosen output voxels.  Returns float64 [P, C]."""
+                    round_bf16=True, w_sc=None, b_sc=None, round_h1=False):
+    """The residual block at chosen output voxels.  Returns float64 [P, C_out]."""
     lib = _load()
     keep = []
-    N, C, T, H, W = _shape5(x)
+    N, Cin, T, H, W = _shape5(x)
+    Cout = _shape5(w1)[0]
     tx, t1, t2 = _view(x, keep), _view(cache1, keep), _view(cache2, keep)
-    tw1, tw2 = _view(w1, keep), _view(w2, keep)
+    tw1, tw2, tsc = _view(w1, keep), _view(w2, keep), _view(w_sc, keep)
     P, pp = _pts(points, keep)
-    y = np.empty((P, C), dtype=np.float64)
-    rc = lib.orc_resblock_points(_ptr(tx), _ptr(t1), _ptr(t2), N, C, T, H, W,
-                                 _ptr(tw1), _dvec(b1, keep), _dvec(g1, keep),
-                                 _ptr(tw2), _dvec(b2, keep), _dvec(g2, keep),
-                                 1 if round_bf16 else 0, P, pp,
-                                 y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    y = np.empty((P, Cout), dtype=np.float64)
+    rc = lib.orc_resblock2_points(_ptr(tx), _ptr(t1), _ptr(t2), N, Cin, Cout, T, H, W,
+                                  _ptr(tw1), _dvec(b1, keep), _dvec(g1, keep),
+                                  _ptr(tw2), _dvec(b2, keep), _dvec(g2, keep),
+                                  _ptr(tsc), _dvec(b_sc, keep),
+                                  1 if round_bf16 else 0, 1 if round_h1 else 0, P, pp,
+                                  y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
     if rc != 0:
-        raise ValueError(f"orc_resblock_points failed ({rc})")
+        raise ValueError(f"orc_resblock2_points failed ({rc})")
     return y
 
 

@@ -260,56 +260,83 @@ static orc_tensor contiguous_ncthw(const double *d, int C, int T, int H,
   return t;
 }
 
-/* WanResidualBlock with C_in == C_out (identity shortcut), 3x3x3 convs,
- * spatial pad 1, causal front pad 2:
- *   a0 = SiLU(RMS(x; g1))            [rounded to bf16 if round_bf16]
- *   a1 = SiLU(RMS(conv1(a0) ; g2))   [rounded to bf16 if round_bf16]
- *   y  = conv2(a1) + x
+/* WanResidualBlock, 3x3x3 convs, spatial pad 1, causal front pad 2, from
+ * C_in to C_out channels:
+ *   a0 = SiLU(RMS(x; g1))               C_in channels  [bf16 if round_bf16]
+ *   h1 = conv1(a0) + b1                 C_out channels [bf16 if round_h1]
+ *   a1 = SiLU(RMS(h1; g2))              C_out channels [bf16 if round_bf16]
+ *   y  = conv2(a1) + b2 + s,   s = x                      (C_in == C_out, wsc NULL)
+ *                              s = conv_1x1x1(x; wsc) + bsc  (the conv_shortcut)
  * conv1 and conv2 take their causal history from cache1 / cache2 (the two
- * a0 / a1 frames before this chunk; NULL = zero frames).
+ * a0 / a1 frames before this chunk; NULL = zero frames); the shortcut reads
+ * the current frame only.  wsc is [C_out][C_in][1][1][1].
  * y, and the optional a0_out / a1_out, are contiguous [N][C][T][H][W]. */
+int orc_resblock2(const orc_tensor *x, const orc_tensor *cache1,
+                  const orc_tensor *cache2, int N, int Cin, int Cout, int T,
+                  int H, int W, const orc_tensor *w1, const double *b1,
+                  const double *g1, const orc_tensor *w2, const double *b2,
+                  const double *g2, const orc_tensor *wsc, const double *bsc,
+                  int round_bf16, int round_h1, double *y, double *a0_out,
+                  double *a1_out) {
+  if (!x || !w1 || !w2 || !g1 || !g2 || !y) return -1;
+  if (!wsc && Cin != Cout) return -1;
+  const long long vox = (long long)N * T * H * W;
+  double *a0 = (double *)malloc(sizeof(double) * vox * Cin);
+  double *h1 = (double *)malloc(sizeof(double) * vox * Cout);
+  double *a1 = (double *)malloc(sizeof(double) * vox * Cout);
+  if (!a0 || !h1 || !a1) {
+    free(a0); free(h1); free(a1);
+    return -2;
+  }
+  int rc = orc_rms_norm(x, N, Cin, T, H, W, g1, NULL, 1, a0);
+  if (round_bf16)
+    for (long long i = 0; i < vox * Cin; ++i) a0[i] = orc_round_bf16(a0[i]);
+  orc_tensor ta0 = contiguous_ncthw(a0, Cin, T, H, W);
+  if (!rc)
+    rc = orc_causal_conv3d(&ta0, cache1, N, Cin, T, H, W, w1, Cout, 3, 3, 3, 1,
+                           1, b1, h1);
+  if (round_h1)
+    for (long long i = 0; i < vox * Cout; ++i) h1[i] = orc_round_bf16(h1[i]);
+  orc_tensor th1 = contiguous_ncthw(h1, Cout, T, H, W);
+  if (!rc) rc = orc_rms_norm(&th1, N, Cout, T, H, W, g2, NULL, 1, a1);
+  if (round_bf16)
+    for (long long i = 0; i < vox * Cout; ++i) a1[i] = orc_round_bf16(a1[i]);
+  orc_tensor ta1 = contiguous_ncthw(a1, Cout, T, H, W);
+  if (!rc)
+    rc = orc_causal_conv3d(&ta1, cache2, N, Cout, T, H, W, w2, Cout, 3, 3, 3,
+                           1, 1, b2, y);
+  if (!rc) {
+    for (int n = 0; n < N; ++n)
+      for (int c = 0; c < Cout; ++c)
+        for (int t = 0; t < T; ++t)
+          for (int h = 0; h < H; ++h)
+            for (int w = 0; w < W; ++w) {
+              double sc;
+              if (wsc) {
+                sc = bsc ? bsc[c] : 0.0;
+                for (int ci = 0; ci < Cin; ++ci)
+                  sc += orc_get(wsc, c, ci, 0, 0, 0) * orc_get(x, n, ci, t, h, w);
+              } else {
+                sc = orc_get(x, n, c, t, h, w);
+              }
+              y[(((long long)n * Cout + c) * T + t) * H * W + (long long)h * W +
+                w] += sc;
+            }
+    if (a0_out) memcpy(a0_out, a0, sizeof(double) * vox * Cin);
+    if (a1_out) memcpy(a1_out, a1, sizeof(double) * vox * Cout);
+  }
+  free(a0); free(h1); free(a1);
+  return rc;
+}
+
+/* The identity-shortcut block (C_in == C_out == C). */
 int orc_resblock(const orc_tensor *x, const orc_tensor *cache1,
                  const orc_tensor *cache2, int N, int C, int T, int H, int W,
                  const orc_tensor *w1, const double *b1, const double *g1,
                  const orc_tensor *w2, const double *b2, const double *g2,
                  int round_bf16, double *y, double *a0_out, double *a1_out) {
-  if (!x || !w1 || !w2 || !g1 || !g2 || !y) return -1;
-  long long nel = (long long)N * C * T * H * W;
-  double *a0 = (double *)malloc(sizeof(double) * nel);
-  double *h1 = (double *)malloc(sizeof(double) * nel);
-  double *a1 = (double *)malloc(sizeof(double) * nel);
-  if (!a0 || !h1 || !a1) {
-    free(a0); free(h1); free(a1);
-    return -2;
-  }
-  int rc = orc_rms_norm(x, N, C, T, H, W, g1, NULL, 1, a0);
-  if (round_bf16)
-    for (long long i = 0; i < nel; ++i) a0[i] = orc_round_bf16(a0[i]);
-  orc_tensor ta0 = contiguous_ncthw(a0, C, T, H, W);
-  if (!rc)
-    rc = orc_causal_conv3d(&ta0, cache1, N, C, T, H, W, w1, C, 3, 3, 3, 1, 1,
-                           b1, h1);
-  orc_tensor th1 = contiguous_ncthw(h1, C, T, H, W);
-  if (!rc) rc = orc_rms_norm(&th1, N, C, T, H, W, g2, NULL, 1, a1);
-  if (round_bf16)
-    for (long long i = 0; i < nel; ++i) a1[i] = orc_round_bf16(a1[i]);
-  orc_tensor ta1 = contiguous_ncthw(a1, C, T, H, W);
-  if (!rc)
-    rc = orc_causal_conv3d(&ta1, cache2, N, C, T, H, W, w2, C, 3, 3, 3, 1, 1,
-                           b2, y);
-  if (!rc) {
-    for (int n = 0; n < N; ++n)
-      for (int c = 0; c < C; ++c)
-        for (int t = 0; t < T; ++t)
-          for (int h = 0; h < H; ++h)
-            for (int w = 0; w < W; ++w)
-              y[(((long long)n * C + c) * T + t) * H * W + (long long)h * W +
-                w] += orc_get(x, n, c, t, h, w);
-    if (a0_out) memcpy(a0_out, a0, sizeof(double) * nel);
-    if (a1_out) memcpy(a1_out, a1, sizeof(double) * nel);
-  }
-  free(a0); free(h1); free(a1);
-  return rc;
+  return orc_resblock2(x, cache1, cache2, N, C, C, T, H, W, w1, b1, g1, w2, b2,
+                       g2, NULL, NULL, round_bf16, 0, y, a0_out, a1_out);
 }
 
 /* a0 = SiLU(RMS(x[n, :, t, h, w]; g1)) at one voxel, optionally rounded. */
@@ -325,22 +352,26 @@ static void block_a0_at(const orc_tensor *x, int C, const double *g1,
 }
 
 /* The residual block at P chosen output voxels (pts rows are n, t, h, w);
- * y is [P][C].  Same definition as orc_resblock, evaluated only on the
+ * y is [P][C_out].  Same definition as orc_resblock2, evaluated only on the
  * receptive field of each requested voxel: a0 on a 5x5x5 window, a1 on the
  * 3x3x3 window, then y. */
-int orc_resblock_points(const orc_tensor *x, const orc_tensor *cache1,
-                        const orc_tensor *cache2, int N, int C, int T, int H,
-                        int W, const orc_tensor *w1, const double *b1,
-                        const double *g1, const orc_tensor *w2,
-                        const double *b2, const double *g2, int round_bf16,
-                        int P, const int *pts, double *y) {
+int orc_resblock2_points(const orc_tensor *x, const orc_tensor *cache1,
+                         const orc_tensor *cache2, int N, int Cin, int Cout,
+                         int T, int H, int W, const orc_tensor *w1,
+                         const double *b1, const double *g1,
+                         const orc_tensor *w2, const double *b2,
+                         const double *g2, const orc_tensor *wsc,
+                         const double *bsc, int round_bf16, int round_h1,
+                         int P, const int *pts, double *y) {
   if (!x || !w1 || !w2 || !g1 || !g2 || !y || !pts || P < 0) return -1;
+  if (!wsc && Cin != Cout) return -1;
   for (int p = 0; p < P; ++p) {
     const int *q = pts + 4 * p;
     if (q[0] < 0 || q[0] >= N || q[1] < 0 || q[1] >= T || q[2] < 0 ||
         q[2] >= H || q[3] < 0 || q[3] >= W)
       return -1;
   }
+  const int Cmax = Cin > Cout ? Cin : Cout;
   int fail = 0;
 #pragma omp parallel for schedule(dynamic, 1)
   for (int p = 0; p < P; ++p) {
@@ -349,12 +380,12 @@ int orc_resblock_points(const orc_tensor *x, const orc_tensor *cache1,
     /* a0 window: frames t0-4..t0, rows h0-2..h0+2, cols w0-2..w0+2.
      * present[] marks voxels that exist (frame >= 0 or taken from cache1,
      * row/col inside the image). */
-    double *a0w = (double *)calloc((size_t)125 * C, sizeof(double));
+    double *a0w = (double *)calloc((size_t)125 * Cin, sizeof(double));
     char present0[125];
-    double *a1w = (double *)calloc((size_t)27 * C, sizeof(double));
+    double *a1w = (double *)calloc((size_t)27 * Cout, sizeof(double));
     char present1[27];
-    double *v = (double *)malloc(sizeof(double) * 2 * C);
-    double *hv = v + C;
+    double *v = (double *)malloc(sizeof(double) * 2 * Cmax);
+    double *hv = v + Cmax;
     if (!a0w || !a1w || !v) {
       free(a0w); free(a1w); free(v);
 #pragma omp atomic write
@@ -366,14 +397,14 @@ int orc_resblock_points(const orc_tensor *x, const orc_tensor *cache1,
         for (int dw = 0; dw < 5; ++dw) {
           int i = (dt * 5 + dh) * 5 + dw;
           int tt = t0 - 4 + dt, hh = h0 - 2 + dh, ww = w0 - 2 + dw;
-          double *o = a0w + (size_t)i * C;
+          double *o = a0w + (size_t)i * Cin;
           present0[i] = 0;
           if (hh < 0 || hh >= H || ww < 0 || ww >= W) continue;
           if (tt >= 0) {
-            block_a0_at(x, C, g1, round_bf16, n, tt, hh, ww, v, o);
+            block_a0_at(x, Cin, g1, round_bf16, n, tt, hh, ww, v, o);
             present0[i] = 1;
           } else if (tt >= -2 && cache1) {
-            for (int c = 0; c < C; ++c) o[c] = orc_get(cache1, n, c, tt + 2, hh, ww);
+            for (int c = 0; c < Cin; ++c) o[c] = orc_get(cache1, n, c, tt + 2, hh, ww);
             present0[i] = 1;
           }
         }
@@ -383,21 +414,21 @@ int orc_resblock_points(const orc_tensor *x, const orc_tensor *cache1,
         for (int dw = 0; dw < 3; ++dw) {
           int i = (dt * 3 + dh) * 3 + dw;
           int tt = t0 - 2 + dt, hh = h0 - 1 + dh, ww = w0 - 1 + dw;
-          double *o = a1w + (size_t)i * C;
+          double *o = a1w + (size_t)i * Cout;
           present1[i] = 0;
           if (hh < 0 || hh >= H || ww < 0 || ww >= W) continue;
           if (tt < 0) {
             if (tt >= -2 && cache2) {
-              for (int c = 0; c < C; ++c) o[c] = orc_get(cache2, n, c, tt + 2, hh, ww);
+              for (int c = 0; c < Cout; ++c) o[c] = orc_get(cache2, n, c, tt + 2, hh, ww);
               present1[i] = 1;
             }
             continue;
           }
           /* h1 = conv1(a0) at (tt, hh, ww): window offset of a0 index is
            * (tt - (t0-4)) + kt - 2 etc. */
-          for (int co = 0; co < C; ++co) {
+          for (int co = 0; co < Cout; ++co) {
             double acc = 0.0;
-            for (int ci = 0; ci < C; ++ci)
+            for (int ci = 0; ci < Cin; ++ci)
               for (int kt = 0; kt < 3; ++kt)
                 for (int kh = 0; kh < 3; ++kh)
                   for (int kw = 0; kw < 3; ++kw) {
@@ -406,31 +437,50 @@ int orc_resblock_points(const orc_tensor *x, const orc_tensor *cache1,
                     int iw = (ww + kw - 1) - (w0 - 2);
                     int j = (it * 5 + ih) * 5 + iw;
                     if (!present0[j]) continue;
-                    acc += orc_get(w1, co, ci, kt, kh, kw) * a0w[(size_t)j * C + ci];
+                    acc += orc_get(w1, co, ci, kt, kh, kw) * a0w[(size_t)j * Cin + ci];
                   }
             hv[co] = acc + (b1 ? b1[co] : 0.0);
+            if (round_h1) hv[co] = orc_round_bf16(hv[co]);
           }
-          rms_vec(hv, C, g2, NULL, o);
-          for (int c = 0; c < C; ++c) {
+          rms_vec(hv, Cout, g2, NULL, o);
+          for (int c = 0; c < Cout; ++c) {
             o[c] = orc_silu(o[c]);
             if (round_bf16) o[c] = orc_round_bf16(o[c]);
           }
           present1[i] = 1;
         }
-    for (int co = 0; co < C; ++co) {
+    for (int co = 0; co < Cout; ++co) {
       double acc = 0.0;
-      for (int ci = 0; ci < C; ++ci)
+      for (int ci = 0; ci < Cout; ++ci)
         for (int kt = 0; kt < 3; ++kt)
           for (int kh = 0; kh < 3; ++kh)
             for (int kw = 0; kw < 3; ++kw) {
               int j = (kt * 3 + kh) * 3 + kw;
               if (!present1[j]) continue;
-              acc += orc_get(w2, co, ci, kt, kh, kw) * a1w[(size_t)j * C + ci];
+              acc += orc_get(w2, co, ci, kt, kh, kw) * a1w[(size_t)j * Cout + ci];
             }
       acc += b2 ? b2[co] : 0.0;
-      y[(size_t)p * C + co] = acc + orc_get(x, n, co, t0, h0, w0);
+      double sc;
+      if (wsc) {
+        sc = bsc ? bsc[co] : 0.0;
+        for (int ci = 0; ci < Cin; ++ci)
+          sc += orc_get(wsc, co, ci, 0, 0, 0) * orc_get(x, n, ci, t0, h0, w0);
+      } else {
+        sc = orc_get(x, n, co, t0, h0, w0);
+      }
+      y[(size_t)p * Cout + co] = acc + sc;
     }
     free(a0w); free(a1w); free(v);
   }
   return fail ? -2 : 0;
+}
+
+int orc_resblock_points(const orc_tensor *x, const orc_tensor *cache1,
+                        const orc_tensor *cache2, int N, int C, int T, int H,
+                        int W, const orc_tensor *w1, const double *b1,
+                        const double *g1, const orc_tensor *w2,
+                        const double *b2, const double *g2, int round_bf16,
+                        int P, const int *pts, double *y) {
+  return orc_resblock2_points(x, cache1, cache2, N, C, C, T, H, W, w1, b1, g1,
+                              w2, b2, g2, NULL, NULL, round_bf16, 0, P, pts, y);
 }

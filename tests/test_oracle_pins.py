@@ -431,6 +431,96 @@ def test_block_streaming_equals_whole():
     np.testing.assert_array_equal(np.concatenate(outs, axis=2), whole)
 
 
+# ---- channel-changing block: the 1x1x1 conv_shortcut ---------------------------
+
+def _block_sc(Cin=6, Cout=10, T=4, H=5, W=5, seed=20):
+    c = synth.block_case(Cin, T, H, W, seed_base=seed)
+    return {
+        "x": c["x"],
+        "w1": synth.kaiming_uniform(Cout, Cin, (3, 3, 3), seed + 31),
+        "b1": synth.uniform((Cout,), -0.1, 0.1, seed + 32),
+        "g1": c["g1"],
+        "w2": synth.kaiming_uniform(Cout, Cout, (3, 3, 3), seed + 33),
+        "b2": synth.uniform((Cout,), -0.1, 0.1, seed + 34),
+        "g2": synth.uniform((Cout,), 0.5, 1.5, seed + 35),
+        "wsc": synth.kaiming_uniform(Cout, Cin, (1, 1, 1), seed + 36),
+        "bsc": synth.uniform((Cout,), -0.1, 0.1, seed + 37),
+    }
+
+
+def _sc_args(c):
+    return (c["x"], c["w1"], _np(c["b1"]), _np(c["g1"]), c["w2"], _np(c["b2"]), _np(c["g2"]))
+
+
+def test_shortcut_block_matches_torch_composition():
+    """C_in != C_out: y = conv2(a1) + b2 + conv_1x1x1(x; wsc) + bsc, rebuilt
+    with torch fp64 ops (normalize * sqrt(C) * gamma, silu, conv3d); with
+    round_h1 conv1's output is rounded to bf16 before its RMS_norm."""
+    c = _block_sc()
+    x = c["x"].double()
+
+    def rs(v, g):
+        C = v.shape[1]
+        return F.silu(F.normalize(v, dim=1) * math.sqrt(C) * g.double()[None, :, None, None, None])
+
+    for round_h1 in (False, True):
+        y, a0, a1 = oracle.resblock(*_sc_args(c), return_acts=True, w_sc=c["wsc"],
+                                    b_sc=_np(c["bsc"]), round_h1=round_h1)
+        a0_ref = rs(x, c["g1"]).float().to(torch.bfloat16).double()
+        np.testing.assert_allclose(a0, a0_ref.numpy(), rtol=2 ** -7, atol=1e-30)
+        h1 = torch_causal_conv3d(a0, _np(c["w1"]), _np(c["b1"]))
+        if round_h1:
+            h1 = oracle.round_bf16_array(h1)
+        a1_ref = rs(torch.from_numpy(h1), c["g2"]).numpy()
+        np.testing.assert_allclose(a1, oracle.round_bf16_array(a1_ref), rtol=0, atol=0)
+        sc = F.conv3d(x, c["wsc"].double(), c["bsc"].double()).numpy()
+        y_ref = torch_causal_conv3d(a1, _np(c["w2"]), _np(c["b2"])) + sc
+        np.testing.assert_allclose(y, y_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_identity_shortcut_weights_give_the_identity_block_bitwise():
+    """C_in == C_out with wsc = I and bsc = 0 is the identity shortcut."""
+    c = _block_small(C=6, seed=21)
+    eye = torch.eye(6, dtype=torch.float64).reshape(6, 6, 1, 1, 1)
+    args = (c["x"], c["w1"], _np(c["b1"]), _np(c["g1"]), c["w2"], _np(c["b2"]), _np(c["g2"]))
+    y_id = oracle.resblock(*args)
+    y_sc = oracle.resblock(*args, w_sc=eye, b_sc=np.zeros(6))
+    np.testing.assert_array_equal(y_sc, y_id)
+
+
+def test_shortcut_block_points_equal_full_bitwise():
+    c = _block_sc(seed=22)
+    cache1 = synth.normal((1, 6, 2, 5, 5), 92)
+    cache2 = synth.normal((1, 10, 2, 5, 5), 93)
+    kw = dict(w_sc=c["wsc"], b_sc=_np(c["bsc"]))
+    for c1, c2, rh in ((None, None, False), (cache1, cache2, True)):
+        y = oracle.resblock(*_sc_args(c), cache1=c1, cache2=c2, round_h1=rh, **kw)
+        pts = np.array([[0, 0, 0, 0], [0, 3, 4, 4], [0, 1, 2, 3], [0, 2, 0, 4]])
+        yp = oracle.resblock_points(*_sc_args(c), pts, cache1=c1, cache2=c2, round_h1=rh, **kw)
+        for k, (n, t, h, w) in enumerate(pts):
+            np.testing.assert_array_equal(yp[k], y[n, :, t, h, w])
+
+
+def test_shortcut_block_streaming_equals_whole():
+    Cin, Cout, T, H, W = 4, 6, 4, 4, 4
+    c = _block_sc(Cin, Cout, T, H, W, seed=23)
+    x = _np(c["x"])
+    rest = _sc_args(c)[1:]
+    kw = dict(w_sc=c["wsc"], b_sc=_np(c["bsc"]))
+    whole, a0, a1 = oracle.resblock(x, *rest, return_acts=True, **kw)
+    outs, c1, c2 = [], None, None
+    for s in range(T):
+        xc = np.ascontiguousarray(x[:, :, s:s + 1])
+        outs.append(oracle.resblock(xc, *rest, cache1=c1, cache2=c2, **kw))
+        pad0 = np.zeros((1, Cin, 1, H, W))
+        pad1 = np.zeros((1, Cout, 1, H, W))
+        c1 = np.ascontiguousarray(a0[:, :, s - 1:s + 1]) if s >= 1 else np.concatenate(
+            [pad0, a0[:, :, :1]], axis=2)
+        c2 = np.ascontiguousarray(a1[:, :, s - 1:s + 1]) if s >= 1 else np.concatenate(
+            [pad1, a1[:, :, :1]], axis=2)
+    np.testing.assert_array_equal(np.concatenate(outs, axis=2), whole)
+
+
 # ---- hand-worked example --------------------------------------------------------
 
 def _read_golden(name):
