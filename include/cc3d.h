@@ -24,10 +24,11 @@
  *   a[v,c] = SiLU( x[v,c] / max(||x[v,:]||_2, 1e-12) * sqrt(C) * gamma[c]
  *                  (+ beta[c]) ),  computed in fp32, rounded once to bf16.
  *
- * Residual block (§10.4 WanResidualBlock, C_in == C_out, identity
- * shortcut, dropout = identity at inference):
+ * Residual block (§10.4 WanResidualBlock, dropout = identity at inference):
  *   a0 = RMS_SiLU(x; g1);  a1 = RMS_SiLU(conv1(a0) + b1; g2);
- *   y  = conv2(a1) + b2 + x.
+ *   y  = conv2(a1) + b2 + s,
+ * s = x (identity shortcut, C_in == C_out), or s = conv_shortcut(x) + b_sc,
+ * the block's 1x1x1 causal conv, when the channel count changes.
  *
  * Layout
  * ------
@@ -178,19 +179,36 @@ cc3d_status rmsnorm_silu(const void *x, const float *gamma, const float *beta,
                          int n, int t, int h, int w, int c, void *y,
                          const void *cache_in, void *cache_out, void *stream);
 
-/* Residual block with c channels (§10.4).  Weights w1, w2 are device
- * [c][c][3][3][3] bf16; b1, b2, g1, g2 device [c] fp32.  All are copied.
- * The block owns two activation buffers of max_t frames (a0, a1).
- * c % 32 == 0 and 32 <= c <= 256. */
+/* Residual block with c channels and the identity shortcut (§10.4):
+ * cc3d_block_create2(n, c, c, ..., w_sc = b_sc = NULL, out). */
 cc3d_status cc3d_block_create(int n, int c, int h, int w, int max_t,
                               const void *w1, const float *b1, const float *g1,
                               const void *w2, const float *b2, const float *g2,
                               cc3d_block **out);
+
+/* Residual block from c_in to c_out channels (§10.4).  Device arguments,
+ * all copied: w1 [c_out][c_in][3][3][3] and w2 [c_out][c_out][3][3][3] bf16;
+ * g1 [c_in], b1, g2, b2 [c_out] fp32 (b1, b2 nullable); w_sc
+ * [c_out][c_in][1][1][1] bf16 and b_sc [c_out] fp32 (nullable): the
+ * conv_shortcut, required when c_in != c_out (NULL: identity shortcut).
+ * The shortcut runs inside conv2 as extra K steps of the same accumulator
+ * (the shortcut's bias is added to b2); for c_out > 256 conv1 writes its
+ * biased output and a separate RMS_norm + SiLU pass follows.
+ * c_in, c_out multiples of 32 in [32, 1024], else CC3D_ERR_UNSUPPORTED;
+ * CC3D_ERR_INVALID_ARG for a NULL weight or gamma, or c_in != c_out without
+ * w_sc.  The block owns its activation buffers (max_t frames each). */
+cc3d_status cc3d_block_create2(int n, int c_in, int c_out, int h, int w,
+                               int max_t, const void *w1, const float *b1,
+                               const float *g1, const void *w2,
+                               const float *b2, const float *g2,
+                               const void *w_sc, const float *b_sc,
+                               cc3d_block **out);
 cc3d_status cc3d_block_destroy(cc3d_block *block);
 
-/* y = block(x) for a chunk of t frames.  cache1_* is conv1's history (a0
- * frames), cache2_* conv2's (a1 frames); *_in nullable (zeros), *_out
- * nullable.  All [n][2][h][w][c] bf16. */
+/* y = block(x) for a chunk of t frames: x [n][t][h][w][c_in], y
+ * [n][t][h][w][c_out].  cache1_* is conv1's history (a0 frames,
+ * [n][2][h][w][c_in]), cache2_* conv2's (a1 frames, [n][2][h][w][c_out]);
+ * *_in nullable (zeros), *_out nullable.  All bf16. */
 cc3d_status cc3d_resblock_forward(cc3d_block *block, const void *x, int t,
                                   const void *cache1_in, const void *cache2_in,
                                   void *y, void *cache1_out, void *cache2_out,

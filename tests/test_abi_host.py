@@ -31,7 +31,8 @@ def declared_functions():
 def test_header_declares_the_abi():
     names = declared_functions()
     for need in ("cc3d_plan_create", "cc3d_plan_destroy", "cc3d_forward", "rmsnorm_silu",
-                 "cc3d_block_create", "cc3d_block_destroy", "cc3d_resblock_forward",
+                 "cc3d_block_create", "cc3d_block_create2", "cc3d_block_destroy",
+                 "cc3d_resblock_forward",
                  "cc3d_sync_status", "cc3d_get_stats", "cc3d_status_string",
                  "cc3d_launch_count"):
         assert need in names
@@ -126,6 +127,24 @@ def test_forward_and_block_null_handles(lib):
     p = ctypes.c_void_p(0x1000)
     assert cc3d.cc3d_block_create(1, 40, 8, 8, 2, p, p, p, p, p, p, out) == cc3d.ERR_UNSUPPORTED
     assert cc3d.cc3d_block_create(1, 64, 8, 8, 0, p, p, p, p, p, p, out) == cc3d.ERR_INVALID_ARG
+
+
+def test_channel_changing_block_validation(lib):
+    out = ctypes.c_void_p()
+    p = ctypes.c_void_p(0x1000)
+    # c_in != c_out needs the conv_shortcut; a shortcut bias needs its weights
+    assert cc3d.cc3d_block_create2(1, 64, 128, 8, 8, 2, p, p, p, p, p, p, None, None, out) == \
+        cc3d.ERR_INVALID_ARG
+    assert cc3d.cc3d_block_create2(1, 64, 64, 8, 8, 2, p, p, p, p, p, p, None, p, out) == \
+        cc3d.ERR_INVALID_ARG
+    assert cc3d.cc3d_block_create2(1, 64, 128, 8, 8, 2, p, p, None, p, p, p, p, p, out) == \
+        cc3d.ERR_INVALID_ARG
+    # channel counts no kernel covers
+    assert cc3d.cc3d_block_create2(1, 48, 64, 8, 8, 2, p, p, p, p, p, p, p, p, out) == \
+        cc3d.ERR_UNSUPPORTED
+    assert cc3d.cc3d_block_create2(1, 64, 2048, 8, 8, 2, p, p, p, p, p, p, p, p, out) == \
+        cc3d.ERR_UNSUPPORTED
+    assert not out.value
 
 
 def test_no_gpu_means_unsupported_not_a_fallback(lib):

@@ -1,0 +1,134 @@
+"""GPU parity of the channel-changing residual block (C_in != C_out) and of
+blocks wider than 256 channels, against the fp64 oracle.
+
+The block's 1x1x1 conv_shortcut runs inside conv2 as extra K steps of the
+same accumulator (its channel chunks past C_in are zero-filled by TMA, so
+96 input channels take two 64-channel chunks); blocks with C_out > 256 run
+conv1 with the bias epilogue and a separate RMS_norm + SiLU pass, whose
+input is conv1's bf16 output (the oracle's round_h1)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.parity import assert_close_bf16, gather_points, ncthw_np, to_dev
+from video_vae_causal_implicit_b200 import cc3d, synth
+
+
+pytestmark = pytest.mark.gpu
+
+
+def block_sc_case(c_in, c_out, t, h, w, *, n=1, seed=0, shortcut=True):
+    c = synth.block_case(c_in, t, h, w, n=n, seed_base=seed)
+    case = {
+        "x": c["x"],
+        "w1": synth.kaiming_uniform(c_out, c_in, (3, 3, 3), seed + 31),
+        "b1": synth.uniform((c_out,), -0.1, 0.1, seed + 32),
+        "g1": c["g1"],
+        "w2": synth.kaiming_uniform(c_out, c_out, (3, 3, 3), seed + 33),
+        "b2": synth.uniform((c_out,), -0.1, 0.1, seed + 34),
+        "g2": synth.uniform((c_out,), 0.5, 1.5, seed + 35),
+    }
+    if shortcut:
+        case["wsc"] = synth.kaiming_uniform(c_out, c_in, (1, 1, 1), seed + 36)
+        case["bsc"] = synth.uniform((c_out,), -0.1, 0.1, seed + 37)
+    return case
+
+
+def _block(case, n, h, w, t):
+    d = {k: to_dev(v) for k, v in case.items() if k != "x"}
+    return cc3d.Block(d["w1"], d["b1"], d["g1"], d["w2"], d["b2"], d["g2"], n=n, h=h, w=w,
+                      max_t=t, w_sc=d.get("wsc"), b_sc=d.get("bsc"))
+
+
+def _oracle_args(case):
+    a = {k: (v.double().numpy() if k in ("b1", "g1", "b2", "g2", "bsc") else v)
+         for k, v in case.items()}
+    return (a["w1"], a["b1"], a["g1"], a["w2"], a["b2"], a["g2"]), dict(
+        w_sc=a.get("wsc"), b_sc=a.get("bsc"))
+
+
+CASES = [
+    # (n, c_in, c_out, t, h, w): 96 -> 192 (shortcut in two 64-channel
+    # chunks, the second half zero-filled), 192 -> 96 (96-channel chunks),
+    # 64 -> 128 on frames large enough for the CTA pair, 192 -> 384 (RMS
+    # after conv1 in its own pass; two N tiles of 192)
+    (1, 96, 192, 3, 20, 24),
+    (1, 192, 96, 3, 18, 20),
+    (4, 64, 128, 2, 32, 48),
+    (1, 192, 384, 2, 12, 16),
+]
+
+
+@pytest.mark.parametrize("n,cin,cout,t,h,w", CASES)
+def test_channel_changing_block_matches_oracle(n, cin, cout, t, h, w):
+    case = block_sc_case(cin, cout, t, h, w, n=n, seed=cin + cout)
+    blk = _block(case, n, h, w, t)
+    x = to_dev(synth.ndhwc(case["x"]))
+    y = torch.empty((n, t, h, w, cout), dtype=torch.bfloat16, device="cuda")
+    blk.forward(x, y)
+    cc3d.sync_status()
+    args, kw = _oracle_args(case)
+    ref = oracle.resblock(synth.ncthw_view(x.cpu()), *args, round_h1=cout > 256, **kw)
+    assert_close_bf16(ncthw_np(y), ref, f"block {cin}->{cout} n{n} {t}x{h}x{w}")
+
+
+def test_wide_identity_block_matches_oracle():
+    """384 channels, identity shortcut: conv1's RMS_norm runs as its own pass."""
+    n, c, t, h, w = 1, 384, 2, 10, 14
+    case = block_sc_case(c, c, t, h, w, seed=5, shortcut=False)
+    blk = _block(case, n, h, w, t)
+    x = to_dev(synth.ndhwc(case["x"]))
+    y = torch.empty_like(x)
+    blk.forward(x, y)
+    cc3d.sync_status()
+    args, _ = _oracle_args(case)
+    ref = oracle.resblock(synth.ncthw_view(x.cpu()), *args, round_h1=True)
+    assert_close_bf16(ncthw_np(y), ref, "wide identity block")
+
+
+@pytest.mark.parametrize("cin,cout", [(96, 192), (192, 384)])
+def test_channel_changing_block_streaming_is_bitwise_whole(cin, cout):
+    """One-frame chunks with conv1's (a0, C_in channels) and conv2's (a1,
+    C_out channels) 2-frame caches reproduce the whole-sequence block."""
+    n, t, h, w = 1, 3, 14, 18
+    case = block_sc_case(cin, cout, t, h, w, seed=7)
+    blk = _block(case, n, h, w, t)
+    x = to_dev(synth.ndhwc(case["x"]))
+    y = torch.empty((n, t, h, w, cout), dtype=torch.bfloat16, device="cuda")
+    blk.forward(x, y)
+
+    def mk(c):
+        return [torch.empty((n, 2, h, w, c), dtype=torch.bfloat16, device="cuda") for _ in (0, 1)]
+
+    c1, c2 = mk(cin), mk(cout)
+    c1_in = c2_in = None
+    ys = []
+    for s in range(t):
+        yc = torch.empty((n, 1, h, w, cout), dtype=torch.bfloat16, device="cuda")
+        blk.forward(x[:, s:s + 1].contiguous(), yc, cache1_in=c1_in, cache2_in=c2_in,
+                    cache1_out=c1[s % 2], cache2_out=c2[s % 2])
+        c1_in, c2_in = c1[s % 2], c2[s % 2]
+        ys.append(yc)
+    cc3d.sync_status()
+    assert torch.equal(torch.cat(ys, dim=1).cpu(), y.cpu())
+
+
+def test_encoder_96_to_192_block_full_size_sampled():
+    """The encoder's first channel-changing block at its full shape,
+    x[1, 96, 17, 240, 416]: whole first and last output frames would cost
+    the oracle minutes, so seeded voxels are checked instead."""
+    n, cin, cout, t, h, w = 1, 96, 192, 17, 240, 416
+    case = block_sc_case(cin, cout, t, h, w, seed=9)
+    blk = _block(case, n, h, w, t)
+    x = to_dev(synth.ndhwc(case["x"]))
+    y = torch.empty((n, t, h, w, cout), dtype=torch.bfloat16, device="cuda")
+    blk.forward(x, y)
+    cc3d.sync_status()
+    pts = synth.sample_points(n, t, h, w, 160, 10).numpy()
+    pts = np.concatenate([pts, np.array([[0, 0, 0, 0], [0, t - 1, h - 1, w - 1],
+                                         [0, 0, h - 1, 0], [0, t - 1, 0, w - 1]],
+                                        dtype=np.int32)])
+    args, kw = _oracle_args(case)
+    ref = oracle.resblock_points(synth.ncthw_view(x.cpu()), *args, pts, **kw)
+    assert_close_bf16(gather_points(y.cpu(), pts), ref, "96->192 block sampled")

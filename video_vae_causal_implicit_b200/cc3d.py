@@ -59,6 +59,8 @@ SIGNATURES = {
     "rmsnorm_silu": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP]),
     "cc3d_block_create": (_I, [_I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP,
                                ctypes.POINTER(_VP)]),
+    "cc3d_block_create2": (_I, [_I, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                ctypes.POINTER(_VP)]),
     "cc3d_block_destroy": (_I, [_VP]),
     "cc3d_resblock_forward": (_I, [_VP, _VP, _I, _VP, _VP, _VP, _VP, _VP, _VP]),
     "cc3d_sync_status": (_I, [_VP]),
@@ -114,6 +116,11 @@ def rmsnorm_silu(x, gamma, beta, n, t, h, w, c, y, cache_in, cache_out, stream):
 
 def cc3d_block_create(n, c, h, w, max_t, w1, b1, g1, w2, b2, g2, out):
     return lib().cc3d_block_create(n, c, h, w, max_t, w1, b1, g1, w2, b2, g2, ctypes.byref(out))
+
+
+def cc3d_block_create2(n, c_in, c_out, h, w, max_t, w1, b1, g1, w2, b2, g2, w_sc, b_sc, out):
+    return lib().cc3d_block_create2(n, c_in, c_out, h, w, max_t, w1, b1, g1, w2, b2, g2, w_sc,
+                                    b_sc, ctypes.byref(out))
 
 
 def cc3d_block_destroy(block):
@@ -213,16 +220,18 @@ class Plan:
 
 
 class Block:
-    """Residual block (C_in == C_out, 3x3x3 convs)."""
+    """Residual block, 3x3x3 convs, from C_in = w1.shape[1] to C_out =
+    w1.shape[0] channels; w_sc [C_out, C_in, 1, 1, 1] (+ b_sc) is the
+    1x1x1 conv_shortcut (None: the identity shortcut, C_in == C_out)."""
 
-    def __init__(self, w1, b1, g1, w2, b2, g2, *, n=1, h, w, max_t):
-        c = int(w1.shape[0])
-        self.c = c
-        self._keep = [t.contiguous() for t in (w1, b1, g1, w2, b2, g2)]
+    def __init__(self, w1, b1, g1, w2, b2, g2, *, n=1, h, w, max_t, w_sc=None, b_sc=None):
+        self.c_out, self.c_in = int(w1.shape[0]), int(w1.shape[1])
+        self.c = self.c_out
+        keep = [None if t is None else t.contiguous() for t in (w1, b1, g1, w2, b2, g2, w_sc, b_sc)]
         self.handle = ctypes.c_void_p()
-        check(cc3d_block_create(n, c, h, w, max_t, *(_ptr(t) for t in self._keep), self.handle),
-              "cc3d_block_create")
-        self._keep = None
+        check(cc3d_block_create2(n, self.c_in, self.c_out, h, w, max_t,
+                                 *(_ptr(t) for t in keep), self.handle),
+              "cc3d_block_create2")
 
     def forward(self, x, y, t=None, cache1_in=None, cache2_in=None, cache1_out=None,
                 cache2_out=None, stream=None):

@@ -16,6 +16,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "cc3d.h"
 #include "internal.h"
@@ -179,6 +180,7 @@ struct cc3d_plan {
   // UMMA
   int kc, nt, n_ntiles, na, nb, tmem_cols, sm_count, ctas_per_sm, sub, nbuf, split, max_clusters;
   int pair, b_resident;
+  int c_sc, n_cc_sc;  // the residual block's fused 1x1x1 conv_shortcut (0: none)
   CUtensorMap map_w;  // pair: the weight image as 128-byte swizzled rows
   uint8_t *wimg;
   // fp32 / thin
@@ -190,10 +192,12 @@ struct cc3d_plan {
 };
 
 struct cc3d_block {
-  int n, c, h, w, max_t;
+  int n, c_in, c_out, h, w, max_t;
+  int fused_rms;    // conv1 applies RMS_norm + SiLU in its epilogue (c_out <= 256)
+  int shortcut;     // conv2 carries the 1x1x1 conv_shortcut of x (else y += x)
   cc3d_plan *conv1, *conv2;
-  float *g1;
-  __nv_bfloat16 *a0, *a1;
+  float *g1, *g2;   // g2: the stand-alone RMS_norm after conv1 when not fused
+  __nv_bfloat16 *a0, *a1, *h1;  // h1: conv1's output before that RMS_norm
 };
 
 namespace {
@@ -267,6 +271,11 @@ cc3d_status check_desc(const cc3d_desc *d, int *variant) {
 
 }  // namespace
 
+namespace {
+cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
+                             const float *b_sc, cc3d_plan **out);
+}  // namespace
+
 extern "C" {
 
 const char *cc3d_status_string(cc3d_status s) {
@@ -287,10 +296,28 @@ const char *cc3d_status_string(cc3d_status s) {
 uint64_t cc3d_launch_count(void) { return g_launches.load(); }
 
 cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
+  return plan_create_impl(desc, 0, nullptr, nullptr, out);
+}
+
+}  // extern "C"
+
+namespace {
+
+// A plan, optionally with the residual block's 1x1x1 conv_shortcut fused in
+// (c_sc > 0: w_sc [c_out][c_sc] bf16 and b_sc [c_out] fp32, device): its
+// channel chunks become extra K stages of the same accumulator, its bias is
+// added to the conv's.  Only for bf16 3x3x3 stride-1 convs with the bias
+// epilogue (the block's conv2).
+cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
+                             const float *b_sc, cc3d_plan **out) {
   if (!out) return CC3D_ERR_INVALID_ARG;
   int variant = 0;
   cc3d_status s = check_desc(desc, &variant);
   if (s != CC3D_OK) return s;
+  if (c_sc < 0 || (c_sc > 0 && !w_sc)) return CC3D_ERR_INVALID_ARG;
+  if (c_sc > 0 && (variant != CC3D_VARIANT_UMMA || desc->kh != 3 || desc->kw != 3 ||
+                   desc->stride_t != 1 || desc->epi != CC3D_EPI_BIAS || c_sc % 16 != 0))
+    return CC3D_ERR_UNSUPPORTED;
   if (!is_sm100()) return CC3D_ERR_UNSUPPORTED;
   cc3d_plan *p = new cc3d_plan();
   p->d = *desc;
@@ -305,6 +332,17 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
   const int taps = desc->kt * desc->kh * desc->kw;
   cudaError_t e = cudaSuccess;
   if ((s = copy_vec(&p->bias, desc->bias, desc->c_out, true)) != CC3D_OK) goto fail;
+  if (c_sc > 0 && b_sc) {
+    // one bias: the conv's plus the shortcut's
+    std::vector<float> hb(desc->c_out), hs(desc->c_out);
+    e = cudaMemcpy(hb.data(), p->bias, sizeof(float) * desc->c_out, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(hs.data(), b_sc, sizeof(float) * desc->c_out, cudaMemcpyDeviceToHost);
+    for (int i = 0; i < desc->c_out; ++i) hb[i] += hs[i];
+    if (e == cudaSuccess)
+      e = cudaMemcpy(p->bias, hb.data(), sizeof(float) * desc->c_out, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
+  }
   if ((s = copy_vec(&p->gamma, desc->gamma, desc->c_out, false)) != CC3D_OK) goto fail;
   if ((s = copy_vec(&p->beta, desc->beta, desc->c_out, false)) != CC3D_OK) goto fail;
   if (variant == CC3D_VARIANT_THIN) {
@@ -367,7 +405,7 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
       // (the largest call's output frames)
       const int max_out = (desc->max_t - 1) / desc->stride_t + 1;
       if (!choose_umma_config(desc->n, desc->c_in, desc->c_out, desc->h, desc->w, desc->kt,
-                              desc->kh, desc->epi == CC3D_EPI_BIAS_RMS_SILU, max_out,
+                              desc->kh, desc->epi == CC3D_EPI_BIAS_RMS_SILU, c_sc > 0, max_out,
                               p->sm_count, &cfg)) {
         s = CC3D_ERR_UNSUPPORTED;
         goto fail;
@@ -389,15 +427,23 @@ cc3d_status cc3d_plan_create(const cc3d_desc *desc, cc3d_plan **out) {
     p->st.k_split = p->split;
     p->st.mma_ctas = p->pair ? 2 : 1;
     p->st.w_resident = p->b_resident;
-    const size_t bytes = sizeof(__nv_bfloat16) * desc->c_out * desc->c_in * taps;
+    // weight image: per N tile, the conv's taps * c_in / kc stages, then the
+    // shortcut's ceil(c_sc / kc) (its channels past c_sc zero)
+    p->c_sc = c_sc;
+    p->n_cc_sc = c_sc > 0 ? (c_sc + p->kc - 1) / p->kc : 0;
+    const int conv_stages = taps * (desc->c_in / p->kc);
+    const int stages = conv_stages + p->n_cc_sc;
+    const size_t bytes = sizeof(__nv_bfloat16) * desc->c_out * stages * p->kc;
     if (cudaMalloc(&p->wimg, bytes) != cudaSuccess) { s = CC3D_ERR_OOM; goto fail; }
     e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(desc->weight), p->wimg,
-                           desc->c_out, desc->c_in, taps, p->nt, p->kc, p->pair, 0);
+                           desc->c_out, desc->c_in, taps, p->nt, p->kc, p->pair, stages, 0, 0);
+    if (e == cudaSuccess && c_sc > 0)
+      e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(w_sc), p->wimg, desc->c_out, c_sc,
+                             1, p->nt, p->kc, p->pair, stages, conv_stages, 0);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
     if (p->pair && !encode_weight_map(&p->map_w, p->wimg,
-                                      static_cast<long long>(desc->c_out) * taps * (desc->c_in / 64),
-                                      p->nt / 2)) {
+                                      static_cast<long long>(desc->c_out) * stages, p->nt / 2)) {
       s = CC3D_ERR_CUDA;
       goto fail;
     }
@@ -408,6 +454,10 @@ fail:
   free_plan(p);
   return s;
 }
+
+}  // namespace
+
+extern "C" {
 
 cc3d_status cc3d_plan_destroy(cc3d_plan *plan) {
   if (!plan) return CC3D_ERR_INVALID_ARG;
@@ -421,9 +471,11 @@ cc3d_status cc3d_get_stats(const cc3d_plan *plan, cc3d_stats *out) {
   return CC3D_OK;
 }
 
-cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_in, void *y,
-                         void *cache_out, const void *residual, const void *next_cache_in,
-                         void *next_cache_out, void *stream_v) {
+// cc3d_forward, plus the input of a fused conv_shortcut (x_sc: [n][t][h][w]
+// [c_sc] bf16, required exactly when the plan has one).
+static cc3d_status forward_impl(cc3d_plan *p, const void *x, int t, const void *cache_in, void *y,
+                                void *cache_out, const void *residual, const void *next_cache_in,
+                                void *next_cache_out, const void *x_sc, void *stream_v) {
   if (!p) return CC3D_ERR_INVALID_ARG;
   const cc3d_desc &d = p->d;
   auto reject = [&](cc3d_status s) {
@@ -436,6 +488,8 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
     return reject(CC3D_ERR_INVALID_ARG);
   if (d.epi != CC3D_EPI_BIAS_RMS_SILU && (next_cache_in || next_cache_out))
     return reject(CC3D_ERR_INVALID_ARG);
+  if ((p->c_sc > 0) != (x_sc != nullptr)) return reject(CC3D_ERR_INVALID_ARG);
+  if (!aligned16(x_sc)) return reject(CC3D_ERR_ALIGNMENT);
   // The thin path reads x and the caches with 2-byte loads (or TMA when they
   // happen to be 16-byte aligned), so a chunk of a 3-channel video may start
   // anywhere on a bf16 boundary; everything else needs 16 bytes.
@@ -458,7 +512,8 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
       overlaps(cache_out, c_bytes, y, y_bytes) ||
       overlaps(next_cache_out, nc_bytes, next_cache_in, nc_bytes) ||
       overlaps(next_cache_out, nc_bytes, y, y_bytes) ||
-      overlaps(next_cache_out, nc_bytes, x, x_bytes) || overlaps(y, y_bytes, x, x_bytes))
+      overlaps(next_cache_out, nc_bytes, x, x_bytes) || overlaps(y, y_bytes, x, x_bytes) ||
+      overlaps(y, y_bytes, x_sc, static_cast<size_t>(d.h) * d.w * p->c_sc * 2 * d.n * t))
     return reject(CC3D_ERR_ALIAS);
   int dev = -1;
   cudaGetDevice(&dev);
@@ -539,6 +594,9 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
     } else {
       mc = mx;
     }
+    CUtensorMap msc = mx;  // the conv_shortcut's input: same boxes, c_sc channels
+    if (p->c_sc > 0 && !encode_act_map(&msc, x_sc, p->c_sc, d.w, d.h, t, d.n, box_w, box_h, box_c))
+      return reject(CC3D_ERR_CUDA);
     UmmaArgs a;
     a.wimg = p->wimg;
     a.bias = p->bias;
@@ -553,6 +611,8 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
     a.stride_t = d.stride_t;
     a.vec32 = (reinterpret_cast<uintptr_t>(y) & 31u) == 0 ? 1 : 0;
     a.b_resident = p->b_resident;
+    a.c_sc = p->c_sc;
+    a.n_cc_sc = p->n_cc_sc;
     a.nt = p->nt; a.n_ntiles = p->n_ntiles;
     a.sub = p->sub; a.nbuf = p->nbuf; a.split = p->split; a.pair = p->pair;
     a.tiles_w = (d.w + tile_w - 1) / tile_w;
@@ -571,8 +631,8 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
       const uint64_t slots = static_cast<uint64_t>(p->sm_count) * p->ctas_per_sm;
       grid = tiles < slots ? tiles : slots;
     }
-    e = launch_conv_umma(mx, mc, p->pair ? p->map_w : mx, a, p->kc, static_cast<unsigned>(grid),
-                         stream);
+    e = launch_conv_umma(mx, mc, p->pair ? p->map_w : mx, msc, a, p->kc,
+                         static_cast<unsigned>(grid), stream);
     count_launch();
   }
   if (e == cudaSuccess && cache_out && front > 0)
@@ -584,6 +644,14 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
   p->st.calls++;
   p->st.tiles += tiles;
   return CC3D_OK;
+}
+
+cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_in, void *y,
+                         void *cache_out, const void *residual, const void *next_cache_in,
+                         void *next_cache_out, void *stream_v) {
+  if (p && p->c_sc > 0) return CC3D_ERR_INVALID_ARG;  // (a block-internal plan)
+  return forward_impl(p, x, t, cache_in, y, cache_out, residual, next_cache_in, next_cache_out,
+                      nullptr, stream_v);
 }
 
 cc3d_status rmsnorm_silu(const void *x, const float *gamma, const float *beta, int n, int t,
@@ -607,33 +675,50 @@ cc3d_status rmsnorm_silu(const void *x, const float *gamma, const float *beta, i
   return from_cuda(e);
 }
 
-cc3d_status cc3d_block_create(int n, int c, int h, int w, int max_t, const void *w1,
-                              const float *b1, const float *g1, const void *w2, const float *b2,
-                              const float *g2, cc3d_block **out) {
+cc3d_status cc3d_block_create2(int n, int c_in, int c_out, int h, int w, int max_t,
+                               const void *w1, const float *b1, const float *g1, const void *w2,
+                               const float *b2, const float *g2, const void *w_sc,
+                               const float *b_sc, cc3d_block **out) {
   if (!out || !w1 || !w2 || !g1 || !g2 || n < 1 || h < 1 || w < 1 || max_t < 1)
     return CC3D_ERR_INVALID_ARG;
-  if (c < 32 || c > 256 || c % 32 != 0) return CC3D_ERR_UNSUPPORTED;
+  if (!w_sc && (c_in != c_out || b_sc)) return CC3D_ERR_INVALID_ARG;
+  if (c_in < 32 || c_in > 1024 || c_in % 32 != 0 || c_out < 32 || c_out > 1024 ||
+      c_out % 32 != 0)
+    return CC3D_ERR_UNSUPPORTED;
   cc3d_desc d;
   std::memset(&d, 0, sizeof d);
-  d.n = n; d.c_in = c; d.c_out = c; d.h = h; d.w = w; d.max_t = max_t;
+  d.n = n; d.h = h; d.w = w; d.max_t = max_t;
   d.kt = d.kh = d.kw = 3; d.pad_h = d.pad_w = 1;
   d.stride_t = d.stride_h = d.stride_w = 1; d.dil_t = d.dil_h = d.dil_w = 1; d.groups = 1;
   d.dtype = CC3D_BF16;
   cc3d_block *b = new cc3d_block();
   std::memset(b, 0, sizeof *b);
-  b->n = n; b->c = c; b->h = h; b->w = w; b->max_t = max_t;
+  b->n = n; b->c_in = c_in; b->c_out = c_out; b->h = h; b->w = w; b->max_t = max_t;
+  // The RMS epilogue needs a whole C_out row in one N tile (tcgen05's N is
+  // at most 256); wider blocks run conv1 with the bias epilogue and the
+  // stand-alone RMS_norm + SiLU after it.
+  b->fused_rms = c_out <= 256;
+  b->shortcut = w_sc != nullptr;
   cc3d_status s;
-  d.weight = w1; d.bias = b1; d.epi = CC3D_EPI_BIAS_RMS_SILU; d.gamma = g2; d.beta = nullptr;
+  const size_t vox = static_cast<size_t>(n) * max_t * h * w;
+  d.c_in = c_in; d.c_out = c_out;
+  d.weight = w1; d.bias = b1;
+  d.epi = b->fused_rms ? CC3D_EPI_BIAS_RMS_SILU : CC3D_EPI_BIAS;
+  d.gamma = b->fused_rms ? g2 : nullptr;
+  d.beta = nullptr;
   if ((s = cc3d_plan_create(&d, &b->conv1)) != CC3D_OK) goto fail;
-  d.weight = w2; d.bias = b2; d.epi = CC3D_EPI_BIAS_RESIDUAL; d.gamma = nullptr;
-  if ((s = cc3d_plan_create(&d, &b->conv2)) != CC3D_OK) goto fail;
-  if ((s = copy_vec(&b->g1, g1, c, false)) != CC3D_OK) goto fail;
-  {
-    const size_t bytes = sizeof(__nv_bfloat16) * static_cast<size_t>(n) * max_t * h * w * c;
-    if (cudaMalloc(&b->a0, bytes) != cudaSuccess || cudaMalloc(&b->a1, bytes) != cudaSuccess) {
-      s = CC3D_ERR_OOM;
-      goto fail;
-    }
+  d.c_in = c_out;
+  d.weight = w2; d.bias = b2; d.gamma = nullptr;
+  d.epi = b->shortcut ? CC3D_EPI_BIAS : CC3D_EPI_BIAS_RESIDUAL;
+  if ((s = plan_create_impl(&d, b->shortcut ? c_in : 0, w_sc, b_sc, &b->conv2)) != CC3D_OK)
+    goto fail;
+  if ((s = copy_vec(&b->g1, g1, c_in, false)) != CC3D_OK) goto fail;
+  if (!b->fused_rms && (s = copy_vec(&b->g2, g2, c_out, false)) != CC3D_OK) goto fail;
+  if (cudaMalloc(&b->a0, vox * c_in * 2) != cudaSuccess ||
+      cudaMalloc(&b->a1, vox * c_out * 2) != cudaSuccess ||
+      (!b->fused_rms && cudaMalloc(&b->h1, vox * c_out * 2) != cudaSuccess)) {
+    s = CC3D_ERR_OOM;
+    goto fail;
   }
   *out = b;
   return CC3D_OK;
@@ -642,13 +727,21 @@ fail:
   return s;
 }
 
+cc3d_status cc3d_block_create(int n, int c, int h, int w, int max_t, const void *w1,
+                              const float *b1, const float *g1, const void *w2, const float *b2,
+                              const float *g2, cc3d_block **out) {
+  return cc3d_block_create2(n, c, c, h, w, max_t, w1, b1, g1, w2, b2, g2, nullptr, nullptr, out);
+}
+
 cc3d_status cc3d_block_destroy(cc3d_block *b) {
   if (!b) return CC3D_ERR_INVALID_ARG;
   if (b->conv1) cc3d_plan_destroy(b->conv1);
   if (b->conv2) cc3d_plan_destroy(b->conv2);
   cudaFree(b->g1);
+  cudaFree(b->g2);
   cudaFree(b->a0);
   cudaFree(b->a1);
+  cudaFree(b->h1);
   delete b;
   return CC3D_OK;
 }
@@ -657,24 +750,37 @@ cc3d_status cc3d_resblock_forward(cc3d_block *b, const void *x, int t, const voi
                                   const void *cache2_in, void *y, void *cache1_out,
                                   void *cache2_out, void *stream) {
   if (!b || !x || !y || t < 1 || t > b->max_t) return CC3D_ERR_INVALID_ARG;
-  const size_t frame = static_cast<size_t>(b->h) * b->w * b->c * 2;
-  const size_t xb = frame * b->n * t, cb = frame * b->n * 2;
-  if (overlaps(x, xb, y, xb)) return CC3D_ERR_ALIAS;
-  if (overlaps(cache1_out, cb, cache1_in, cb) || overlaps(cache2_out, cb, cache2_in, cb) ||
-      overlaps(cache1_out, cb, x, xb) || overlaps(cache1_out, cb, y, xb) ||
-      overlaps(cache2_out, cb, x, xb) || overlaps(cache2_out, cb, y, xb) ||
-      overlaps(cache1_out, cb, cache2_out, cb) || overlaps(cache1_out, cb, cache2_in, cb) ||
-      overlaps(cache2_out, cb, cache1_in, cb))
+  const size_t fin = static_cast<size_t>(b->h) * b->w * b->c_in * 2;
+  const size_t fout = static_cast<size_t>(b->h) * b->w * b->c_out * 2;
+  const size_t xb = fin * b->n * t, yb = fout * b->n * t;
+  const size_t c1 = fin * b->n * 2, c2 = fout * b->n * 2;  // cache1: a0 frames, cache2: a1
+  if (overlaps(x, xb, y, yb)) return CC3D_ERR_ALIAS;
+  if (overlaps(cache1_out, c1, cache1_in, c1) || overlaps(cache2_out, c2, cache2_in, c2) ||
+      overlaps(cache1_out, c1, x, xb) || overlaps(cache1_out, c1, y, yb) ||
+      overlaps(cache2_out, c2, x, xb) || overlaps(cache2_out, c2, y, yb) ||
+      overlaps(cache1_out, c1, cache2_out, c2) || overlaps(cache1_out, c1, cache2_in, c2) ||
+      overlaps(cache2_out, c2, cache1_in, c1))
     return CC3D_ERR_ALIAS;
   // a0 = SiLU(RMS(x; g1)); conv1's cache is a0's history.
-  cc3d_status s = rmsnorm_silu(x, b->g1, nullptr, b->n, t, b->h, b->w, b->c, b->a0, cache1_in,
+  cc3d_status s = rmsnorm_silu(x, b->g1, nullptr, b->n, t, b->h, b->w, b->c_in, b->a0, cache1_in,
                                cache1_out, stream);
   if (s != CC3D_OK) return s;
-  // a1 = SiLU(RMS(conv1(a0) + b1; g2)), fused epilogue; conv2's cache is a1's history.
-  s = cc3d_forward(b->conv1, b->a0, t, cache1_in, b->a1, nullptr, nullptr, cache2_in, cache2_out,
-                   stream);
+  // a1 = SiLU(RMS(conv1(a0) + b1; g2)); conv2's cache is a1's history.
+  if (b->fused_rms) {
+    s = cc3d_forward(b->conv1, b->a0, t, cache1_in, b->a1, nullptr, nullptr, cache2_in,
+                     cache2_out, stream);
+  } else {
+    s = cc3d_forward(b->conv1, b->a0, t, cache1_in, b->h1, nullptr, nullptr, nullptr, nullptr,
+                     stream);
+    if (s == CC3D_OK)
+      s = rmsnorm_silu(b->h1, b->g2, nullptr, b->n, t, b->h, b->w, b->c_out, b->a1, cache2_in,
+                       cache2_out, stream);
+  }
   if (s != CC3D_OK) return s;
-  // y = conv2(a1) + b2 + x, fused epilogue.
+  // y = conv2(a1) + b2 + (x | conv_shortcut(x) + b_sc), fused in conv2.
+  if (b->shortcut)
+    return forward_impl(b->conv2, b->a1, t, cache2_in, y, nullptr, nullptr, nullptr, nullptr, x,
+                        stream);
   return cc3d_forward(b->conv2, b->a1, t, cache2_in, y, nullptr, x, nullptr, nullptr, stream);
 }
 

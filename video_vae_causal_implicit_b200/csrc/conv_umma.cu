@@ -185,7 +185,8 @@ template <int KC, int KS, int SUB, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     conv_umma_kernel(const __grid_constant__ CUtensorMap map_x,
                      const __grid_constant__ CUtensorMap map_cache,
-                     const __grid_constant__ CUtensorMap map_w, UmmaArgs p) {
+                     const __grid_constant__ CUtensorMap map_w,
+                     const __grid_constant__ CUtensorMap map_sc, UmmaArgs p) {
   static_assert(!PAIR || (SUB == 1 && uses_sw128(KC)), "CTA pairs take 64-channel chunks");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // Align the dynamic shared window to 1 KiB ourselves (the attribute is a
@@ -235,6 +236,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int n_cc = p.c_in / KC;   // channel chunks
   const int n_a = n_kt * n_cc;    // A stages per tile (of this CTA)
+  // weight stages of the conv per N tile, and the shortcut's chunks after them
+  const int n_conv_stages = p.kt * KS * KS * n_cc;
+  const int n_sc = (p.c_sc > 0 && !split) ? p.n_cc_sc : 0;
+  const int stages_per_ntile = n_conv_stages + (p.c_sc > 0 ? p.n_cc_sc : 0);  // weight image
   constexpr bool kSw = uses_sw128(KC);
   const uint32_t halo_w = static_cast<uint32_t>(halo_cols(KC, SUB, KS));
   const int n_tiles = p.n * p.t * p.tiles_h * p.tiles_w * p.n_ntiles;
@@ -304,15 +309,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (PAIR) {
           // rows of the weight image [ntile][tap][cchunk][NT][64]
           const int row = static_cast<int>(
-              ((static_cast<size_t>(ntile) * p.kt * KS * KS * n_cc + stage_idx) * p.nt) +
+              ((static_cast<size_t>(ntile) * stages_per_ntile + stage_idx) * p.nt) +
               rank * (p.nt / 2));
           tma_load_2d_pair(smem_base + L.b_off + slot * L.b_stage, &map_w,
                            lead_full_b + 8u * slot, 0, row);
         } else {
           const uint8_t *wsrc =
-              p.wimg + static_cast<size_t>(ntile) * p.kt * KS * KS * n_cc * L.b_stage;
+              p.wimg + static_cast<size_t>(ntile) * stages_per_ntile * L.b_stage;
           bulk_load(smem_base + L.b_off + slot * L.b_stage, wsrc + stage_idx * L.b_stage,
                     L.b_stage, &full_b[slot]);
+        }
+      };
+      // the tile's halo of channels c0 .. c0+KC-1 of frame `tcoord` of `map`
+      // into A slot `slot` (this CTA's half of the tile on a pair)
+      auto load_a = [&](const CUtensorMap *map, int slot, int c0, int tcoord,
+                        const TileCoord &tc) {
+        const uint32_t dst = smem_base + L.a_off + slot * L.a_stage;
+        if constexpr (PAIR) {
+          tma_load_5d_pair(dst, map, lead_full_a + 8u * slot, c0, tc.w0 + kTW * rank - KS / 2,
+                           tc.h0 - KS / 2, tcoord, tc.n);
+        } else if constexpr (kSw) {
+          tma_load_5d(dst, map, &full_a[slot], c0, tc.w0 - KS / 2, tc.h0 - KS / 2, tcoord, tc.n);
+        } else {
+#pragma unroll
+          for (int s = 0; s < KC / 8; ++s)
+            tma_load_5d(dst + s * L.slab, map, &full_a[slot], c0 + s * 8, tc.w0 - KS / 2,
+                        tc.h0 - KS / 2, tcoord, tc.n);
         }
       };
       if (KS == 1 && p.b_resident) {
@@ -337,21 +359,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           a_par = (a_par & ~(1u << sa)) | (pa << sa);
           const int tau = p.stride_t * tc0.t + kt - (p.kt - 1);  // input frame
           const bool from_cache = tau < 0;  // (zero frames were skipped above)
-          const CUtensorMap *map = from_cache ? &map_cache : &map_x;
-          const int tcoord = from_cache ? tau + (p.kt - 1) : tau;
-          const uint32_t dst = smem_base + L.a_off + sa * L.a_stage;
-          if constexpr (PAIR) {
-            tma_load_5d_pair(dst, map, lead_full_a + 8u * sa, cc * KC,
-                             tc0.w0 + kTW * rank - KS / 2, tc0.h0 - KS / 2, tcoord, tc0.n);
-          } else if constexpr (kSw) {
-            tma_load_5d(dst, map, &full_a[sa], cc * KC, tc0.w0 - KS / 2, tc0.h0 - KS / 2, tcoord,
-                        tc0.n);
-          } else {
-#pragma unroll
-            for (int s = 0; s < KC / 8; ++s)
-              tma_load_5d(dst + s * L.slab, map, &full_a[sa], cc * KC + s * 8, tc0.w0 - KS / 2,
-                          tc0.h0 - KS / 2, tcoord, tc0.n);
-          }
+          load_a(from_cache ? &map_cache : &map_x, sa, cc * KC, from_cache ? tau + (p.kt - 1) : tau,
+                 tc0);
           if (++sa == L.na) { sa = 0; pa ^= 1; }
           if (KS == 1 && p.b_resident) continue;
 #pragma unroll 1
@@ -365,6 +374,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             load_b(sb, static_cast<size_t>(kt * KS * KS + ts) * n_cc + cc, tc0.ntile);
             if (++sb == L.nb) { sb = 0; pb ^= 1; }
           }
+        }
+        // the residual block's 1x1x1 conv_shortcut: each channel chunk of
+        // the block input at the output frame (a halo like the conv's, read
+        // at its centre tap) against one weight stage stored after the
+        // conv's, into the same accumulator
+        for (int c2 = 0; c2 < n_sc && ok; ++c2) {
+          if (!mbar_wait_bounded(&empty_a[sa], pa ^ 1, p.wait_limit_ns, p.status, 1)) {
+            ok = false;
+            break;
+          }
+          if (pair_leader) mbar_arrive_expect_tx(&full_a[sa], PAIR ? 2u * a_tx : a_tx);
+          a_used |= 1u << sa;
+          a_par = (a_par & ~(1u << sa)) | (pa << sa);
+          load_a(&map_sc, sa, c2 * KC, tc0.t, tc0);
+          if (++sa == L.na) { sa = 0; pa ^= 1; }
+          if (!mbar_wait_bounded(&empty_b[sb], pb ^ 1, p.wait_limit_ns, p.status, 2)) {
+            ok = false;
+            break;
+          }
+          b_used |= 1u << sb;
+          b_par = (b_par & ~(1u << sb)) | (pb << sb);
+          load_b(sb, static_cast<size_t>(n_conv_stages + c2), tc0.ntile);
+          if (++sb == L.nb) { sb = 0; pb ^= 1; }
         }
       }
       // Drain: every load this thread issued lands before the CTA may exit
@@ -420,6 +452,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_tmem = tmem_base + buf * SUB * p.nt;
         const TileCoord tcm = decode_tile(tile, p);
         uint32_t accumulate = 0;
+        // the MMAs of weight slot `slot` (phase parity `par`) against the
+        // halo at `a_st` seen through spatial tap `ts`
+        auto issue_b = [&](uint64_t a_st, int slot, uint32_t par, int ts) -> bool {
+          if (!mbar_wait_bounded(&full_b[slot], par, p.wait_limit_ns, p.status, 4)) return false;
+          tc_fence_after();
+          const uint64_t a_tap = a_st + ((ts / KS) * halo_w + (ts % KS)) * pix16;
+          const uint64_t b_st = bdesc0 + ((static_cast<uint32_t>(slot) * L.b_stage) >> 4);
+#pragma unroll
+          for (int j = 0; j < KC / 16; ++j) {
+            // every sub-tile (8 pixels further along the halo row) reuses
+            // this weight stage
+#pragma unroll
+            for (int sbt = 0; sbt < SUB; ++sbt) {
+              if constexpr (PAIR)
+                umma_bf16_pair(d_tmem, a_tap + j * astep16, b_st + j * bstep16, idesc,
+                               accumulate);
+              else
+                umma_bf16(d_tmem + sbt * p.nt, a_tap + sbt * kTW * pix16 + j * astep16,
+                          b_st + j * bstep16, idesc, accumulate);
+            }
+            accumulate = 1;
+          }
+          return true;
+        };
         for (int ia = 0; ia < n_a && ok; ++ia) {
           // the same zero-frame stages the producer skipped; adding their
           // exact zeros would not change the accumulator
@@ -430,40 +486,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint64_t a_st = adesc0 + ((sa * L.a_stage) >> 4);
-          // the MMAs of weight slot `slot` (phase parity `par`) with spatial tap `ts`
-          auto issue_b = [&](int slot, uint32_t par, int ts) -> bool {
-            if (!mbar_wait_bounded(&full_b[slot], par, p.wait_limit_ns, p.status, 4)) return false;
-            tc_fence_after();
-            const uint64_t a_tap = a_st + ((ts / KS) * halo_w + (ts % KS)) * pix16;
-            const uint64_t b_st = bdesc0 + ((static_cast<uint32_t>(slot) * L.b_stage) >> 4);
-#pragma unroll
-            for (int j = 0; j < KC / 16; ++j) {
-              // every sub-tile (8 pixels further along the halo row) reuses
-              // this weight stage
-#pragma unroll
-              for (int sbt = 0; sbt < SUB; ++sbt) {
-                if constexpr (PAIR)
-                  umma_bf16_pair(d_tmem, a_tap + j * astep16, b_st + j * bstep16, idesc,
-                                 accumulate);
-                else
-                  umma_bf16(d_tmem + sbt * p.nt, a_tap + sbt * kTW * pix16 + j * astep16,
-                            b_st + j * bstep16, idesc, accumulate);
-              }
-              accumulate = 1;
-            }
-            return true;
-          };
           if (KS == 1 && p.b_resident) {
             // resident weights: stage (kt, cc) sits in slot kt * n_cc + cc,
             // loaded once (its first phase stays complete) and never freed
-            if (!issue_b(kt_lo * n_cc + ia, 0u, 0)) {
+            if (!issue_b(a_st, kt_lo * n_cc + ia, 0u, 0)) {
               ok = false;
               break;
             }
           } else {
 #pragma unroll
             for (int ts = 0; ts < KS * KS; ++ts) {
-              if (!issue_b(sb, pb, ts)) {
+              if (!issue_b(a_st, sb, pb, ts)) {
                 ok = false;
                 break;
               }
@@ -475,6 +508,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if constexpr (PAIR) umma_commit_pair(&empty_a[sa], 3);
           else umma_commit(&empty_a[sa]);
+          if (++sa == L.na) { sa = 0; pa ^= 1; }
+        }
+        // the conv_shortcut's chunks: the centre tap of each halo
+        for (int c2 = 0; c2 < n_sc && ok; ++c2) {
+          if (!mbar_wait_bounded(&full_a[sa], pa, p.wait_limit_ns, p.status, 3)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (!issue_b(adesc0 + ((sa * L.a_stage) >> 4), sb, pb, (KS / 2) * KS + KS / 2)) {
+            ok = false;
+            break;
+          }
+          if constexpr (PAIR) {
+            umma_commit_pair(&empty_b[sb], 3);
+            umma_commit_pair(&empty_a[sa], 3);
+          } else {
+            umma_commit(&empty_b[sb]);
+            umma_commit(&empty_a[sa]);
+          }
+          if (++sb == L.nb) { sb = 0; pb ^= 1; }
           if (++sa == L.na) { sa = 0; pa ^= 1; }
         }
         // accumulator ready for the epilogue(s)
@@ -924,7 +978,7 @@ long long frame_cost(const UmmaConfig &c, int n, int h, int w, int sm_count) {
 }  // namespace
 
 bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
-                        int max_t, int sm_count, UmmaConfig *cfg) {
+                        bool shortcut, int max_t, int sm_count, UmmaConfig *cfg) {
   // N tile: the largest split of c_out that is a multiple of 16 and at most
   // `cap` (256 is the tcgen05 N limit); the RMS epilogue needs the whole row
   // in one CTA.
@@ -959,7 +1013,7 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
   // clusters (about 9/10 of sm_count / kt fit at once) take whole rounds of
   // one-tap work plus the exchange (measured at ~0.4 of a tap's MMAs),
   // against rounds of kt taps over all SMs.
-  if (kt >= 2 && kt <= 4 && !rms_epi) {
+  if (kt >= 2 && kt <= 4 && !rms_epi && !shortcut) {
     UmmaConfig sp = one;
     sp.split = kt;
     const long long calls_tiles = tiles1 * (max_t > 0 ? max_t : 1);
@@ -1052,7 +1106,8 @@ size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols, i
 }
 
 namespace {
-using UmmaKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, UmmaArgs);
+using UmmaKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                            const CUtensorMap, UmmaArgs);
 
 UmmaKernel umma_kernel_for(int kc, int ks, int sub, int pair) {
 #define CC3D_PICK(KC_, KS_)                                                         \
@@ -1107,8 +1162,8 @@ int umma_max_clusters(const UmmaConfig &c, int ks) {
 }
 
 cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_cache,
-                             const CUtensorMap &map_w, const UmmaArgs &args, int kc,
-                             unsigned grid, cudaStream_t stream) {
+                             const CUtensorMap &map_w, const CUtensorMap &map_sc,
+                             const UmmaArgs &args, int kc, unsigned grid, cudaStream_t stream) {
   if (args.kh != args.kw || (args.kh != 1 && args.kh != 3)) return cudaErrorInvalidValue;
   const size_t smem =
       umma_launch_smem(kc, args.nt, args.kh, args.na, args.nb, args.tmem_cols, args.sub,
@@ -1123,12 +1178,16 @@ cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_ca
   if (args.b_resident && (args.split != 1 || args.n_ntiles != 1 || args.nb > 32 ||
                           args.nb != args.kt * args.kh * args.kw * (args.c_in / kc)))
     return cudaErrorInvalidValue;
+  if (args.c_sc < 0 ||
+      (args.c_sc > 0 && (args.split != 1 || args.b_resident || args.c_sc % 8 != 0 ||
+                         args.n_cc_sc != (args.c_sc + kc - 1) / kc)))
+    return cudaErrorInvalidValue;
   UmmaKernel k = umma_kernel_for(kc, args.kh, args.sub, args.pair);
   if (!k) return cudaErrorInvalidValue;
   cudaLaunchAttribute attr;
   const cudaLaunchConfig_t cfg =
       umma_launch_config(grid, smem, args.pair ? 2 : args.split, stream, &attr);
-  return cudaLaunchKernelEx(&cfg, k, map_x, map_cache, map_w, args);
+  return cudaLaunchKernelEx(&cfg, k, map_x, map_cache, map_w, map_sc, args);
 }
 
 }  // namespace cc3d

@@ -37,6 +37,9 @@ struct UmmaArgs {
   int vec32;                      // 1: y and residual are 32-byte aligned (256-bit stores)
   int b_resident;                 // 1: one N tile, every weight stage (nb = kt*kh*kw*c_in/KC)
                                   // in shared memory for the whole launch
+  int c_sc;                       // > 0: the residual block's 1x1x1 conv_shortcut of a
+                                  // c_sc-channel input (map_sc), summed into the accumulator
+  int n_cc_sc;                    // its channel chunks, ceil(c_sc / KC) (tail zero-filled)
 };
 
 // Tile configuration of the UMMA conv for a plan (chosen from n, c_in, c_out,
@@ -46,8 +49,9 @@ struct UmmaConfig {
   int params;      // epilogue parameters staged in shared memory (floats)
   int b_resident;  // every weight stage resident in shared memory (nb of them)
 };
+// shortcut: the plan carries a fused conv_shortcut (no temporal split).
 bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
-                        int max_t, int sm_count, UmmaConfig *cfg);
+                        bool shortcut, int max_t, int sm_count, UmmaConfig *cfg);
 // Clusters of cfg.split CTAs that can be resident at once (split > 1), for
 // sizing the grid; 0 when the query fails.
 int umma_max_clusters(const UmmaConfig &cfg, int ks);
@@ -64,18 +68,23 @@ int umma_tile_w();
 int umma_halo_box_w(int kc, int sub, int kw);
 int umma_halo_box_c(int kc);
 int umma_tile_h();
-// map_w: the weights' tensor map (plain-rows image) for pair launches; any
-// valid map otherwise (unused).
+// map_w: the weights' tensor map (plain-rows image) for pair launches;
+// map_sc: the conv_shortcut's input (c_sc > 0).  Unused maps may be any
+// valid map.
 cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_cache,
-                             const CUtensorMap &map_w, const UmmaArgs &args, int kc,
-                             unsigned grid, cudaStream_t stream);
+                             const CUtensorMap &map_w, const CUtensorMap &map_sc,
+                             const UmmaArgs &args, int kc, unsigned grid, cudaStream_t stream);
 
 // Weight re-tiling for the UMMA kernel (plan time):
 // W[c_out][c_in][kt][kh][kw] (bf16) -> image[ntile][tap][cchunk][kc/8][nt][8].
 // rows: 0 = [ntile][tap][cchunk][kc/8][nt][8] (no-swizzle stage images for
 // a bulk copy), 1 = [ntile][tap][cchunk][nt][kc] (plain rows for a tensor map)
+// stages_per_ntile / stage0: the image holds stages_per_ntile stages per N
+// tile and this weight fills stages stage0 .. stage0 + taps*ceil(c_in/kc) - 1
+// of each (channels past c_in are zero).
 cudaError_t launch_repack_umma(const __nv_bfloat16 *w, uint8_t *img, int c_out, int c_in,
-                               int taps, int nt, int kc, int rows, cudaStream_t stream);
+                               int taps, int nt, int kc, int rows, int stages_per_ntile,
+                               int stage0, cudaStream_t stream);
 
 // Thin first-layer conv (c_in small): weights to [tap*c_in padded to kpad][c_out]
 // image and the kernel itself.

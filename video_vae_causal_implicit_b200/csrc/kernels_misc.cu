@@ -23,9 +23,11 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 }
 
 __global__ void repack_umma_kernel(const __nv_bfloat16 *__restrict__ w, __nv_bfloat16 *img,
-                                   int c_out, int c_in, int taps, int nt, int kc, int rows) {
-  const long long total = static_cast<long long>(c_out) * c_in * taps;
-  const int n_cc = c_in / kc;
+                                   int c_out, int c_in, int taps, int nt, int kc, int rows,
+                                   int stages_per_ntile, int stage0) {
+  const int n_cc = (c_in + kc - 1) / kc;  // channels past c_in are zero
+  const long long total = static_cast<long long>(c_out) * n_cc * kc * taps;
+  const long long stage_elems = static_cast<long long>(nt) * kc;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     // image order: ntile, tap, cchunk, then within the stage either
@@ -53,7 +55,12 @@ __global__ void repack_umma_kernel(const __nv_bfloat16 *__restrict__ w, __nv_bfl
     const int ntile = static_cast<int>(r / taps);
     const int co = ntile * nt + nl;
     const int ci = cc * kc + s * 8 + e;
-    img[i] = w[(static_cast<long long>(co) * c_in + ci) * taps + tap];
+    const long long dst =
+        (static_cast<long long>(ntile) * stages_per_ntile + stage0 + tap * n_cc + cc) *
+            stage_elems +
+        i % stage_elems;
+    img[dst] = ci < c_in ? w[(static_cast<long long>(co) * c_in + ci) * taps + tap]
+                         : __float2bfloat16(0.f);
   }
 }
 
@@ -330,10 +337,12 @@ int grid_for(long long work, int block) {
 }  // namespace
 
 cudaError_t launch_repack_umma(const __nv_bfloat16 *w, uint8_t *img, int c_out, int c_in,
-                               int taps, int nt, int kc, int rows, cudaStream_t stream) {
-  const long long total = static_cast<long long>(c_out) * c_in * taps;
+                               int taps, int nt, int kc, int rows, int stages_per_ntile,
+                               int stage0, cudaStream_t stream) {
+  const long long total = static_cast<long long>(c_out) * ((c_in + kc - 1) / kc) * kc * taps;
   repack_umma_kernel<<<grid_for(total, 256), 256, 0, stream>>>(
-      w, reinterpret_cast<__nv_bfloat16 *>(img), c_out, c_in, taps, nt, kc, rows);
+      w, reinterpret_cast<__nv_bfloat16 *>(img), c_out, c_in, taps, nt, kc, rows,
+      stages_per_ntile, stage0);
   count_launch();
   return cudaGetLastError();
 }

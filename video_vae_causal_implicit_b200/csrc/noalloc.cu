@@ -137,8 +137,8 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   // ---- tiles: the same choice cc3d_plan_create makes --------------------------------
   UmmaConfig cfg;
   if (!choose_umma_config(d->n, d->c_in, d->c_out, d->h, d->w, d->kt, d->kh,
-                          d->epi == CC3D_EPI_BIAS_RMS_SILU, (d->max_t - 1) / d->stride_t + 1,
-                          n_sm, &cfg))
+                          d->epi == CC3D_EPI_BIAS_RMS_SILU, false,
+                          (d->max_t - 1) / d->stride_t + 1, n_sm, &cfg))
     return CC3D_ERR_UNSUPPORTED;
   const bool clustered = cfg.split > 1 || cfg.pair;
   const int max_clusters = clustered ? umma_max_clusters(cfg, d->kh) : 0;
@@ -149,7 +149,8 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   uint8_t *wimg = scratch;
   float *zero_bias = reinterpret_cast<float *>(scratch + kNoAllocWeightBytes);
   cudaError_t e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(d->weight), wimg,
-                                     d->c_out, d->c_in, taps, nt, kc, cfg.pair, stream);
+                                     d->c_out, d->c_in, taps, nt, kc, cfg.pair,
+                                     taps * (d->c_in / kc), 0, stream);
   if (e == cudaSuccess && !d->bias)
     e = cudaMemsetAsync(zero_bias, 0, sizeof(float) * d->c_out, stream);
   if (e != cudaSuccess) return CC3D_ERR_CUDA;
@@ -189,6 +190,8 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   a.n = d->n; a.t = t_out; a.stride_t = d->stride_t;
   a.vec32 = (reinterpret_cast<uintptr_t>(y) & 31u) == 0 ? 1 : 0;
   a.b_resident = cfg.b_resident;
+  a.c_sc = 0;
+  a.n_cc_sc = 0;
   a.h = d->h; a.w = d->w; a.c_in = d->c_in; a.c_out = d->c_out;
   a.kt = d->kt; a.kh = d->kh; a.kw = d->kw; a.pad_h = d->pad_h; a.pad_w = d->pad_w;
   a.nt = nt; a.n_ntiles = cfg.n_ntiles;
@@ -207,7 +210,7 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
     const uint64_t slots = uint64_t(n_sm) * cfg.ctas_per_sm;
     grid = tiles < slots ? tiles : slots;
   }
-  e = launch_conv_umma(mx, mc, mw, a, kc, static_cast<unsigned>(grid), stream);
+  e = launch_conv_umma(mx, mc, mw, mx, a, kc, static_cast<unsigned>(grid), stream);
   count_launch();
   if (e == cudaSuccess && cache_out && front > 0)
     e = launch_cache_update(cache_in, x, cache_out, d->n, t, front, in_frame, stream);
