@@ -14,9 +14,10 @@ The same JSON line carries the residual block (x[1, 192, 9, 240, 416]:
 RMS_norm+SiLU -> conv -> RMS_norm+SiLU (fused) -> conv + x (fused)) as
 ``resblock`` with its latency, and with ``--sweep`` the encoder convs
 (3 -> 96, 96 -> 96 at 17 x 480 x 832), the downsample path's time_conv
-(kernel (3, 1, 1), stride 2 in time, at 192 and 384 channels) and the
-streaming channel/resolution sweep (21 one-frame chunks, CUDA-graph
-captured).
+(kernel (3, 1, 1), stride 2 in time, at 192 and 384 channels), the
+encoder's channel-changing residual blocks (96 -> 192, 192 -> 384) and a
+384-channel block, and the streaming channel/resolution sweep (21
+one-frame chunks, CUDA-graph captured).
 
 Multi-GPU: the path runs as independent replicas (one process per GPU, no
 data-path collective); ``value`` is the FLOP all ranks processed divided by
@@ -547,6 +548,28 @@ def run_sweep(args, dev, stream, peaks, flush_l2):
             "ms": ms, "tflops": fl / ms / 1e9, "frac": fl / ms / 1e9 / peaks["bf16_tflops"],
             "tile": [ps.stats().mma_ctas, ps.stats().tile_w, ps.stats().k_split]}
         del ps, xs, ys
+    # the encoder's other residual blocks (§8(f) NEXT-2): the two that change
+    # the channel count (the 1x1x1 conv_shortcut fused into conv2) and a
+    # 384-channel one (RMS_norm after conv1 in its own pass), whole sequence
+    for (ci, co, T, H, W) in ((96, 192, 17, 240, 416), (192, 384, 9, 120, 208),
+                              (384, 384, 5, 60, 104)):
+        xb = torch.randn((1, T, H, W, ci), generator=g, device=dev).to(torch.bfloat16)
+        wts = dict(w1=synth.kaiming_uniform(co, ci, (3, 3, 3), 11),
+                   b1=synth.uniform((co,), -0.1, 0.1, 12), g1=synth.uniform((ci,), 0.5, 1.5, 13),
+                   w2=synth.kaiming_uniform(co, co, (3, 3, 3), 14),
+                   b2=synth.uniform((co,), -0.1, 0.1, 15), g2=synth.uniform((co,), 0.5, 1.5, 16))
+        if ci != co:
+            wts["w_sc"] = synth.kaiming_uniform(co, ci, (1, 1, 1), 17)
+            wts["b_sc"] = synth.uniform((co,), -0.1, 0.1, 18)
+        wts = {k: v.to(dev) for k, v in wts.items()}
+        blk = cc3d.Block(**wts, h=H, w=W, max_t=T)
+        yb = torch.empty((1, T, H, W, co), dtype=torch.bfloat16, device=dev)
+        ms = timed(lambda: blk.forward(xb, yb), flush=True)
+        fl = conv_flop(1, ci, co, T, H, W) + conv_flop(1, co, co, T, H, W) + (
+            conv_flop(1, ci, co, T, H, W, taps=1) if ci != co else 0)
+        out[f"block_{ci}to{co}_{T}x{H}x{W}"] = {
+            "ms": ms, "tflops": fl / ms / 1e9, "frac": fl / ms / 1e9 / peaks["bf16_tflops"]}
+        del blk, xb, yb
     # config 5: C x resolution, 21 one-frame chunks, graph-captured
     for cc in (96, 192, 384):
         for (H, W) in ((90, 160), (180, 320), (360, 640)):
