@@ -18,6 +18,8 @@ Functions (each cites the passage it follows in the C source):
   resblock              -- §10.4 WanResidualBlock: identity shortcut, or the
                            1x1x1 conv_shortcut when C_in != C_out
   resblock_points       -- the same definition at chosen output voxels
+  conv2d_frames         -- §10.5 the downsample path's per-frame ZeroPad2d +
+                           stride-2 Conv2d
   round_bf16            -- bfloat16 round-to-nearest-even of one double
 """
 from __future__ import annotations
@@ -84,13 +86,16 @@ def _load():
                                           i, i, dp, dp, dp]
             lib.orc_resblock2_points.argtypes = [T, T, T, i, i, i, i, i, i, T, dp, dp, T, dp, dp,
                                                  T, dp, i, i, i, ip, dp]
+            lib.orc_conv2d_frames.argtypes = [T, i, i, i, i, i, T, i, i, i, i, i, i, i, i, i,
+                                              dp, dp]
             lib.orc_round_bf16.argtypes = [ctypes.c_double]
             lib.orc_round_bf16.restype = ctypes.c_double
             lib.orc_silu.argtypes = [ctypes.c_double]
             lib.orc_silu.restype = ctypes.c_double
             for name in ("orc_causal_conv3d", "orc_causal_conv3d_points", "orc_causal_conv3d_s",
                          "orc_causal_conv3d_points_s", "orc_rms_norm", "orc_resblock",
-                         "orc_resblock_points", "orc_resblock2", "orc_resblock2_points"):
+                         "orc_resblock_points", "orc_resblock2", "orc_resblock2_points",
+                         "orc_conv2d_frames"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -269,6 +274,30 @@ def resblock_points(x, w1, b1, g1, w2, b2, g2, points, cache1=None, cache2=None,
                                   y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
     if rc != 0:
         raise ValueError(f"orc_resblock2_points failed ({rc})")
+    return y
+
+
+def conv2d_frames(x, weight, bias=None, stride=(2, 2), pad=(0, 1, 0, 1)):
+    """Per-frame ZeroPad2d(pad = (left, right, top, bottom)) + Conv2d with
+    `stride` (the downsample path's spatial step).  x: [N, Cin, T, H, W];
+    weight: [Cout, Cin, KH, KW].  Returns float64 [N, Cout, T, Ho, Wo],
+    Ho = (H + top + bottom - KH) // stride[0] + 1 (likewise Wo)."""
+    lib = _load()
+    keep = []
+    N, Cin, T, H, W = _shape5(x)
+    Cout, Cin2, KH, KW = (int(s) for s in weight.shape)
+    assert Cin2 == Cin
+    l, r, t, b = pad
+    Ho = (H + t + b - KH) // stride[0] + 1
+    Wo = (W + l + r - KW) // stride[1] + 1
+    w5 = weight.reshape(Cout, Cin, 1, KH, KW)
+    tx, tw = _view(x, keep), _view(w5, keep)
+    y = np.empty((N, Cout, T, Ho, Wo), dtype=np.float64)
+    rc = lib.orc_conv2d_frames(_ptr(tx), N, Cin, T, H, W, _ptr(tw), Cout, KH, KW, stride[0],
+                               stride[1], l, r, t, b, _dvec(bias, keep),
+                               y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc != 0:
+        raise ValueError(f"orc_conv2d_frames failed ({rc})")
     return y
 
 

@@ -201,6 +201,53 @@ int orc_causal_conv3d_points(const orc_tensor *x, const orc_tensor *cache,
                                     KH, KW, pad_h, pad_w, 1, bias, P, pts, y);
 }
 
+/* The downsample path's spatial step ("Cosmos3 Wan VAE" page, section 10.5,
+ * WanResample in downsample mode): every frame on its own goes through
+ * ZeroPad2d(pad_l, pad_r, pad_t, pad_b) and a KH x KW Conv2d with stride
+ * (sh, sw), bias once:
+ *   y[n,co,t,i,j] = b[co] + sum_{ci,kh,kw} W[co,ci,0,kh,kw] *
+ *                   xp[n,ci,t, sh*i + kh, sw*j + kw],
+ *   xp[.., r, c] = x[.., r - pad_t, c - pad_l] inside the frame, else 0.
+ * wt is [Cout][Cin][1][KH][KW]; y is contiguous [N][Cout][T][Ho][Wo] with
+ * Ho = (H + pad_t + pad_b - KH) / sh + 1 and Wo likewise.  Returns 0, or -1
+ * on a bad argument. */
+int orc_conv2d_frames(const orc_tensor *x, int N, int Cin, int T, int H,
+                      int W, const orc_tensor *wt, int Cout, int KH, int KW,
+                      int sh, int sw, int pad_l, int pad_r, int pad_t,
+                      int pad_b, const double *bias, double *y) {
+  if (!x || !wt || !y || N < 1 || Cin < 1 || Cout < 1 || T < 1 || H < 1 ||
+      W < 1 || KH < 1 || KW < 1 || sh < 1 || sw < 1 || pad_l < 0 ||
+      pad_r < 0 || pad_t < 0 || pad_b < 0)
+    return -1;
+  if (H + pad_t + pad_b < KH || W + pad_l + pad_r < KW) return -1;
+  const int Ho = (H + pad_t + pad_b - KH) / sh + 1;
+  const int Wo = (W + pad_l + pad_r - KW) / sw + 1;
+  const long long total = (long long)N * Cout * T * Ho;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long long idx = 0; idx < total; ++idx) {
+    const int i = (int)(idx % Ho);
+    const int t = (int)((idx / Ho) % T);
+    const int co = (int)((idx / ((long long)Ho * T)) % Cout);
+    const int n = (int)(idx / ((long long)Ho * T * Cout));
+    for (int j = 0; j < Wo; ++j) {
+      double acc = 0.0;
+      for (int ci = 0; ci < Cin; ++ci)
+        for (int kh = 0; kh < KH; ++kh) {
+          const int r = sh * i + kh - pad_t; /* row of the unpadded frame */
+          if (r < 0 || r >= H) continue;
+          for (int kw = 0; kw < KW; ++kw) {
+            const int c = sw * j + kw - pad_l;
+            if (c < 0 || c >= W) continue;
+            acc += orc_get(wt, co, ci, 0, kh, kw) * orc_get(x, n, ci, t, r, c);
+          }
+        }
+      if (bias) acc += bias[co];
+      y[(((long long)n * Cout + co) * T + t) * Ho * Wo + (long long)i * Wo + j] = acc;
+    }
+  }
+  return 0;
+}
+
 /* SiLU(z) = z * sigmoid(z) = z / (1 + e^-z). */
 double orc_silu(double z) { return z / (1.0 + exp(-z)); }
 

@@ -521,6 +521,67 @@ def test_shortcut_block_streaming_equals_whole():
     np.testing.assert_array_equal(np.concatenate(outs, axis=2), whole)
 
 
+# ---- the downsample path's per-frame stride-2 Conv2d ----------------------------
+
+def torch_conv2d_frames(x, w, b, stride, pad):
+    """Library special case: frames to the batch, F.pad, F.conv2d (fp64)."""
+    x = torch.from_numpy(np.ascontiguousarray(x))
+    N, C, T, H, W = x.shape
+    xf = x.permute(0, 2, 1, 3, 4).reshape(N * T, C, H, W)
+    yf = F.conv2d(F.pad(xf, pad), torch.from_numpy(w), torch.from_numpy(b), stride=stride)
+    Co, Ho, Wo = yf.shape[1:]
+    return yf.reshape(N, T, Co, Ho, Wo).permute(0, 2, 1, 3, 4).numpy()
+
+
+@pytest.mark.parametrize("stride,pad", [((2, 2), (0, 1, 0, 1)), ((2, 2), (1, 1, 1, 1)),
+                                        ((2, 2), (1, 0, 1, 0)), ((1, 1), (1, 1, 1, 1))])
+def test_conv2d_frames_matches_torch(stride, pad):
+    x = rnd((2, 3, 3, 9, 10), 60)
+    w = rnd((5, 3, 3, 3), 61, 0.3)
+    b = rnd((5,), 62)
+    y = oracle.conv2d_frames(x, w, b, stride=stride, pad=pad)
+    ref = torch_conv2d_frames(x, w, b, stride, pad)
+    assert y.shape == ref.shape
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_conv2d_frames_stride1_is_the_kt1_causal_conv_bitwise():
+    x = rnd((1, 4, 3, 6, 7), 63)
+    w = rnd((2, 4, 3, 3), 64)
+    b = rnd((2,), 65)
+    y = oracle.conv2d_frames(x, w, b, stride=(1, 1), pad=(1, 1, 1, 1))
+    ref = oracle.causal_conv3d(x, w.reshape(2, 4, 1, 3, 3), b, pad=(1, 1))
+    np.testing.assert_array_equal(y, ref)
+
+
+def test_conv2d_frames_impulse_pins_stride_and_padding_side():
+    """A one-hot input reaches output (i, j) through tap (kh, kw) exactly
+    when 2i + kh - top = h0 and 2j + kw - left = w0."""
+    C, T, H, W = 2, 2, 8, 9
+    h0, w0, ci0, t0 = 4, 5, 1, 1
+    x = np.zeros((1, C, T, H, W))
+    x[0, ci0, t0, h0, w0] = 1.0
+    w = rnd((3, C, 3, 3), 66)
+    for pad in ((0, 1, 0, 1), (1, 0, 1, 0)):
+        left, _, top, _ = pad
+        y = oracle.conv2d_frames(x, w, None, stride=(2, 2), pad=pad)
+        want = np.zeros_like(y)
+        for i in range(y.shape[3]):
+            for j in range(y.shape[4]):
+                for kh in range(3):
+                    for kw in range(3):
+                        if 2 * i + kh - top == h0 and 2 * j + kw - left == w0:
+                            want[0, :, t0, i, j] += w[:, ci0, kh, kw]
+        np.testing.assert_array_equal(y, want)
+
+
+def test_conv2d_frames_halves_the_pages_frame():
+    """ZeroPad2d(0, 1, 0, 1) + 3x3 stride 2 maps 480 x 832 to 240 x 416."""
+    y = oracle.conv2d_frames(np.ones((1, 1, 1, 480, 832)), np.ones((1, 1, 3, 3)), None)
+    assert y.shape == (1, 1, 1, 240, 416)
+    assert y[0, 0, 0, 0, 0] == 9.0 and y[0, 0, 0, -1, -1] == 4.0
+
+
 # ---- hand-worked example --------------------------------------------------------
 
 def _read_golden(name):
