@@ -1,0 +1,127 @@
+"""Host logic of the tensor-core conv's planner (choose_umma_config), no
+GPU: a small C++ probe links libcc3d.so and reports the plan chosen for a
+grid of shapes; the tests check the invariants every plan must satisfy
+(shared and tensor memory within the SM's, N tiles that divide C_out, the
+temporal split and resident weights only where they are valid) and the
+choices the design rests on (the latent-resolution layer unsplit for
+5-frame calls and split for 1-frame calls, the residual block on CTA
+pairs, the time_conv with resident weights)."""
+import itertools
+import os
+import shutil
+import subprocess
+
+import pytest
+
+from video_vae_causal_implicit_b200 import cc3d
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(ROOT, "video_vae_causal_implicit_b200", "csrc")
+FIELDS = ("ok", "kc", "nt", "n_ntiles", "sub", "nbuf", "split", "pair", "na", "nb", "tmem_cols",
+          "ctas_per_sm", "params", "b_resident", "smem")
+SMEM_MAX = 227 * 1024
+
+
+def _cuda_include():
+    for cand in (os.environ.get("CUDA_HOME"), "/usr/local/cuda"):
+        if cand and os.path.exists(os.path.join(cand, "include", "cuda.h")):
+            return os.path.join(cand, "include")
+    return None
+
+
+@pytest.fixture(scope="module")
+def probe(tmp_path_factory):
+    if not os.path.exists(cc3d.LIB_PATH):
+        pytest.skip("libcc3d.so is not built")
+    inc = _cuda_include()
+    if inc is None or shutil.which("g++") is None:
+        pytest.skip("needs g++ and the CUDA headers")
+    exe = str(tmp_path_factory.mktemp("plan") / "plan_probe")
+    libdir = os.path.dirname(cc3d.LIB_PATH)
+    subprocess.run(["g++", "-O1", "-std=c++17", "-I", CSRC, "-I", os.path.join(ROOT, "include"),
+                    "-I", inc, os.path.join(HERE, "plan", "plan_probe.cpp"), "-o", exe,
+                    "-L", libdir, "-lcc3d", "-Wl,-rpath," + libdir], check=True)
+
+    def run(cases):
+        text = "\n".join(" ".join(str(int(v)) for v in c) for c in cases) + "\n"
+        out = subprocess.run([exe], input=text, capture_output=True, text=True, check=True).stdout
+        return [dict(zip(FIELDS, map(int, line.split()))) for line in out.splitlines()]
+    return run
+
+
+def case(n=1, ci=64, co=64, h=30, w=52, kt=3, ks=3, rms=False, sc=False, mt=1, sms=148):
+    return (n, ci, co, h, w, kt, ks, rms, sc, mt, sms)
+
+
+GRID = [case(n=n, ci=ci, co=co, h=h, w=w, kt=kt, ks=ks, rms=rms, sc=sc, mt=mt)
+        for (ci, co), (h, w), (kt, ks), rms, sc, n, mt in itertools.product(
+            [(32, 48), (64, 64), (96, 96), (96, 192), (192, 192), (192, 384), (384, 384)],
+            [(9, 17), (30, 52), (120, 208), (240, 416)],
+            [(3, 3), (3, 1), (1, 1)],
+            [False, True], [False, True], [1, 4], [1, 5])
+        if not (rms and co > 256) and not (sc and ks != 3) and not (sc and rms)]
+
+
+def test_every_plan_fits_the_sm(probe):
+    for c, p in zip(GRID, probe(GRID)):
+        n, ci, co, h, w, kt, ks, rms, sc, mt, sms = c
+        assert p["ok"] == 1, c
+        assert p["smem"] <= SMEM_MAX, (c, p)
+        assert 32 <= p["tmem_cols"] <= 512 and p["tmem_cols"] & (p["tmem_cols"] - 1) == 0, (c, p)
+        cta_sub = 1 if p["pair"] else p["sub"]
+        assert p["tmem_cols"] >= p["nbuf"] * cta_sub * p["nt"], (c, p)
+        assert co % p["nt"] == 0 and p["nt"] <= 256 and p["nt"] % 16 == 0, (c, p)
+        assert p["n_ntiles"] * p["nt"] == co, (c, p)
+        assert ci % p["kc"] == 0 and p["kc"] in (32, 64, 96), (c, p)
+        if rms:
+            assert p["nt"] == co, (c, p)  # the RMS epilogue needs the whole row
+        assert p["params"] == co * (3 if rms else 1), (c, p)
+        assert 1 <= p["ctas_per_sm"] <= 2, (c, p)
+
+
+def test_split_pair_and_resident_only_where_valid(probe):
+    for c, p in zip(GRID, probe(GRID)):
+        n, ci, co, h, w, kt, ks, rms, sc, mt, sms = c
+        assert p["split"] in (1, kt), (c, p)
+        if p["split"] > 1:
+            assert not rms and not sc and p["sub"] == 1 and not p["pair"], (c, p)
+        if p["pair"]:
+            assert p["kc"] == 64 and p["sub"] == 2 and p["ctas_per_sm"] == 1, (c, p)
+        if p["b_resident"]:
+            assert ks == 1 and p["n_ntiles"] == 1 and p["split"] == 1 and not sc, (c, p)
+            assert p["nb"] == kt * ci // p["kc"] and p["na"] >= 3, (c, p)
+        else:
+            assert 2 <= p["na"] <= 8 and 2 <= p["nb"] <= 8, (c, p)
+            if ks == 3:
+                assert p["na"] == 2, (c, p)
+
+
+def test_plan_is_a_function_of_the_problem(probe):
+    """Asking twice gives the same plan (no hidden state), and the plan
+    depends on the largest call (max_t), not on anything per call."""
+    a = probe(GRID[:64])
+    b = probe(GRID[:64])
+    assert a == b
+
+
+def test_the_documented_choices(probe):
+    c2_whole, c2_chunks, c4, tc192, tc384, blk_sc = probe([
+        case(ci=384, co=384, h=30, w=52, mt=5),
+        case(ci=384, co=384, h=30, w=52, mt=1),
+        case(ci=192, co=192, h=240, w=416, rms=True, mt=9),
+        case(ci=192, co=192, h=120, w=208, ks=1, mt=9),
+        case(ci=384, co=384, h=60, w=104, ks=1, mt=5),
+        case(ci=192, co=192, h=240, w=416, sc=True, mt=17),
+    ])
+    # the latent-resolution layer: unsplit for its 5-frame call, temporal
+    # split when planned for one-frame calls only
+    assert (c2_whole["split"], c2_whole["pair"], c2_whole["nt"]) == (1, 0, 192)
+    assert c2_chunks["split"] == 3
+    # the residual block's convs run on CTA pairs
+    assert (c4["pair"], c4["nt"]) == (1, 192)
+    # the 192-channel time_conv keeps its weights resident; 384 channels do not fit
+    assert (tc192["pair"], tc192["b_resident"], tc192["nb"]) == (1, 1, 9)
+    assert tc384["b_resident"] == 0
+    # a conv carrying the conv_shortcut is never split
+    assert blk_sc["split"] == 1
