@@ -21,6 +21,9 @@ Functions (each cites the passage it follows in the C source):
   conv2d_frames         -- §10.5 the downsample path's per-frame ZeroPad2d +
                            stride-2 Conv2d
   round_bf16            -- bfloat16 round-to-nearest-even of one double
+  round_e4m3 / quantize_e4m3 / causal_conv3d_fp8
+                        -- FP8 E4M3 quantiser and the causal conv on E4M3
+                           operands with per-tensor / per-channel scales
 """
 from __future__ import annotations
 
@@ -88,6 +91,8 @@ def _load():
                                                  T, dp, i, i, i, ip, dp]
             lib.orc_conv2d_frames.argtypes = [T, i, i, i, i, i, T, i, i, i, i, i, i, i, i, i,
                                               dp, dp]
+            lib.orc_round_e4m3.argtypes = [ctypes.c_double]
+            lib.orc_round_e4m3.restype = ctypes.c_double
             lib.orc_round_bf16.argtypes = [ctypes.c_double]
             lib.orc_round_bf16.restype = ctypes.c_double
             lib.orc_silu.argtypes = [ctypes.c_double]
@@ -298,6 +303,43 @@ def conv2d_frames(x, weight, bias=None, stride=(2, 2), pad=(0, 1, 0, 1)):
                                y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
     if rc != 0:
         raise ValueError(f"orc_conv2d_frames failed ({rc})")
+    return y
+
+
+def round_e4m3(v: float) -> float:
+    """FP8 E4M3 (e4m3fn) round-to-nearest-even of one double, clamped to
+    +-448."""
+    return _load().orc_round_e4m3(float(v))
+
+
+def quantize_e4m3(a, scale):
+    """E4M3 codes of a / scale, returned as their float64 values (so that
+    a ~= scale * quantize_e4m3(a, scale)); scale broadcasts against a.
+    Loops over round_e4m3: meant for the small arrays of the tests."""
+    lib = _load()
+    v = np.asarray(a, dtype=np.float64) / np.asarray(scale, dtype=np.float64)
+    out = np.empty_like(v)
+    flat_in, flat_out = v.reshape(-1), out.reshape(-1)
+    for k in range(flat_in.size):
+        flat_out[k] = lib.orc_round_e4m3(float(flat_in[k]))
+    return out
+
+
+def causal_conv3d_fp8(x, weight, bias, s_x, s_w, cache=None, pad=(1, 1)):
+    """The causal Conv3D on E4M3 operands: x is quantised with the
+    per-tensor scale s_x (cache too), weight with the per-output-channel
+    scales s_w [Cout]; y = s_x * s_w[co] * conv(q_x, q_w) + b[co], the
+    contraction exact in float64.  Returns float64 [N, Cout, T, H, W]."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(weight, dtype=np.float64)
+    s_w = np.asarray(s_w, dtype=np.float64).reshape(-1)
+    qx = quantize_e4m3(x, s_x)
+    qw = quantize_e4m3(w, s_w.reshape(-1, 1, 1, 1, 1))
+    qc = quantize_e4m3(np.asarray(cache, dtype=np.float64), s_x) if cache is not None else None
+    y = causal_conv3d(qx, qw, None, cache=qc, pad=pad)
+    y *= float(s_x) * s_w.reshape(1, -1, 1, 1, 1)
+    if bias is not None:
+        y += np.asarray(bias, dtype=np.float64).reshape(1, -1, 1, 1, 1)
     return y
 
 

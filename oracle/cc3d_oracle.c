@@ -97,6 +97,28 @@ double orc_round_bf16(double v) {
   return v < 0 ? -r : r;
 }
 
+/* FP8 E4M3 ("e4m3fn": 4 exponent bits, bias 7, 3 mantissa bits, no
+ * infinities, largest finite 448 = 1.75 * 2^8, smallest subnormal 2^-9):
+ * v clamped to [-448, 448], then rounded to the nearest E4M3 value, ties to
+ * the even mantissa.  The quantiser of a low-precision conv (the pages name
+ * INT8 / NVFP4 conv quantisation without giving one; this is the FP8 form
+ * the tensor cores take). */
+double orc_round_e4m3(double v) {
+  if (v != v || v == 0.0) return v;
+  double a = fabs(v);
+  if (a > 448.0) a = 448.0;
+  double r;
+  if (a < ldexp(1.0, -6)) {
+    /* subnormal range: a fixed grid of spacing 2^-9 */
+    r = ldexp(nearbyint(ldexp(a, 9)), -9);
+  } else {
+    int e;
+    double m = frexp(a, &e);            /* a = m * 2^e, m in [0.5, 1) */
+    r = ldexp(nearbyint(ldexp(m, 4)), e - 4);  /* 4 significant bits, RNE */
+  }
+  return v < 0 ? -r : r;
+}
+
 /* One output of the causal Conv3D, straight from the definition.
  * Input frame for output frame t and temporal tap kt is
  * tau = t + kt - (KT - 1): KT - 1 frames of causal front padding.  A frame

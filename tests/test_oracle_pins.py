@@ -582,6 +582,74 @@ def test_conv2d_frames_halves_the_pages_frame():
     assert y[0, 0, 0, 0, 0] == 9.0 and y[0, 0, 0, -1, -1] == 4.0
 
 
+# ---- FP8 E4M3 quantiser and the conv on E4M3 operands --------------------------
+
+def _e4m3_values():
+    codes = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn)
+    v = codes.to(torch.float64).numpy()
+    return v[np.isfinite(v)]
+
+
+def test_e4m3_fixes_every_e4m3_value():
+    vals = _e4m3_values()
+    assert len(vals) == 254 and vals.max() == 448.0 and vals.min() == -448.0
+    got = np.array([oracle.round_e4m3(v) for v in vals])
+    np.testing.assert_array_equal(got, vals)
+
+
+def test_e4m3_matches_torch_cast_on_values_and_midpoints():
+    """Single rounding from float32: every E4M3 value, every midpoint
+    between neighbours (the ties), and seeded values across the range."""
+    pos = np.unique(np.abs(_e4m3_values()))
+    mids = (pos[:-1] + pos[1:]) / 2
+    g = np.random.default_rng(70)
+    rand = np.concatenate([g.uniform(-460, 460, 3000), g.standard_normal(3000) * 0.01,
+                           g.standard_normal(3000)])
+    v32 = torch.from_numpy(np.concatenate([pos, -pos, mids, -mids, rand])).float()
+    ref = v32.to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.round_e4m3(float(v)) for v in v32.double().numpy()])
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_e4m3_special_cases():
+    assert oracle.round_e4m3(1.0625) == 1.0      # tie -> even mantissa
+    assert oracle.round_e4m3(1.1875) == 1.25     # tie -> even mantissa
+    assert oracle.round_e4m3(2.0 ** -10) == 0.0  # half the smallest subnormal
+    assert oracle.round_e4m3(3 * 2.0 ** -11) == 2.0 ** -9
+    assert oracle.round_e4m3(500.0) == 448.0 and oracle.round_e4m3(-1e9) == -448.0  # clamp
+    assert oracle.round_e4m3(-1.3) == -oracle.round_e4m3(1.3)
+
+
+def test_fp8_conv_on_representable_operands_is_the_plain_conv():
+    """Unit scales and operands already in E4M3: quantisation is exact, so
+    the FP8 conv is the plain conv bit for bit."""
+    vals = _e4m3_values()
+    g = np.random.default_rng(71)
+    small = vals[np.abs(vals) <= 4]
+    x = g.choice(small, size=(1, 3, 3, 5, 6))
+    w = g.choice(small, size=(4, 3, 3, 3, 3))
+    b = rnd((4,), 72)
+    y = oracle.causal_conv3d_fp8(x, w, b, 1.0, np.ones(4))
+    np.testing.assert_array_equal(y, oracle.causal_conv3d(x, w, b))
+
+
+def test_fp8_conv_scales_multiply_the_contraction():
+    """y = s_x * s_w[co] * conv(q_x, q_w) + b equals the conv of the
+    dequantised operands, and stays close to the unquantised conv."""
+    g = np.random.default_rng(73)
+    x = g.standard_normal((1, 4, 3, 5, 5))
+    w = g.standard_normal((3, 4, 3, 3, 3)) * 0.2
+    b = rnd((3,), 74)
+    s_x = np.abs(x).max() / 448
+    s_w = np.abs(w).reshape(3, -1).max(axis=1) / 448
+    y = oracle.causal_conv3d_fp8(x, w, b, s_x, s_w)
+    xd = s_x * oracle.quantize_e4m3(x, s_x)
+    wd = s_w.reshape(-1, 1, 1, 1, 1) * oracle.quantize_e4m3(w, s_w.reshape(-1, 1, 1, 1, 1))
+    np.testing.assert_allclose(y, oracle.causal_conv3d(xd, wd, b), rtol=1e-12, atol=1e-12)
+    ref = oracle.causal_conv3d(x, w, b)
+    assert np.abs(y - ref).max() < 0.1 * np.abs(ref).max()
+
+
 # ---- hand-worked example --------------------------------------------------------
 
 def _read_golden(name):
