@@ -142,8 +142,9 @@ typedef struct cc3d_block cc3d_block;
 
 /* Validate desc, pick a kernel, copy and re-tile the weights (and bias,
  * gamma, beta) into plan-owned device memory.  Synchronous.  Returns
- * CC3D_ERR_UNSUPPORTED for stride/dilation/groups != 1, even kernel sizes,
- * or channel counts no kernel covers.  bf16 covers c_out % 16 == 0 with
+ * CC3D_ERR_UNSUPPORTED for dilation/groups != 1, spatial strides != 1, a
+ * temporal stride other than 1 (or 2 on the bf16 c_in % 32 == 0 path),
+ * even kernel sizes, or channel counts no kernel covers.  bf16 covers c_out % 16 == 0 with
  * either c_in % 32 == 0 (kh == kw in {1, 3}, kt <= 3; N tiles of at most
  * 256 channels) or c_in <= 8 (the thin first-layer path: bias epilogue,
  * c_out <= 256, kt*kh*kw*c_in <= 256); fp32 covers any channel count with
@@ -155,10 +156,11 @@ cc3d_status cc3d_plan_destroy(cc3d_plan *plan);
  *   x         [n][t][h][w][c_in]       input chunk
  *   cache_in  [n][kt-1][h][w][c_in]    frames before the chunk, oldest
  *                                      first; NULL = zero frames
- *   y         [n][t][h][w][c_out]      output
+ *   y         [n][t'][h][w][c_out]     output, t' = (t-1)/stride_t + 1
+ *                                      (t' = t at temporal stride 1)
  *   cache_out [n][kt-1][h][w][c_in]    nullable: the last kt-1 frames of
  *                                      concat(cache_in, x), for the next call
- *   residual  [n][t][h][w][c_out]      EPI_BIAS_RESIDUAL only, else NULL
+ *   residual  [n][t'][h][w][c_out]     EPI_BIAS_RESIDUAL only, else NULL
  *   next_cache_in / next_cache_out     EPI_BIAS_RMS_SILU only, nullable:
  *                                      [n][2][h][w][c_out]; next_cache_out
  *                                      receives the last 2 frames of
