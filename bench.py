@@ -14,7 +14,8 @@ The same JSON line carries the residual block (x[1, 192, 9, 240, 416]:
 RMS_norm+SiLU -> conv -> RMS_norm+SiLU (fused) -> conv + x (fused)) as
 ``resblock`` with its latency, and with ``--sweep`` the encoder convs
 (3 -> 96, 96 -> 96 at 17 x 480 x 832), the downsample path's time_conv
-(kernel (3, 1, 1), stride 2 in time, at 192 and 384 channels), the
+(kernel (3, 1, 1), stride 2 in time, at 192 and 384 channels) and its
+per-frame 3x3 stride-2 conv (96 channels, 480 x 832 -> 240 x 416), the
 encoder's channel-changing residual blocks (96 -> 192, 192 -> 384) and a
 384-channel block, and the streaming channel/resolution sweep (21
 one-frame chunks, CUDA-graph captured).
@@ -548,6 +549,21 @@ def run_sweep(args, dev, stream, peaks, flush_l2):
             "ms": ms, "tflops": fl / ms / 1e9, "frac": fl / ms / 1e9 / peaks["bf16_tflops"],
             "tile": [ps.stats().mma_ctas, ps.stats().tile_w, ps.stats().k_split]}
         del ps, xs, ys
+    # the downsample path's spatial step: ZeroPad2d(0, 1, 0, 1) + 3x3 stride 2
+    # per frame, 96 channels, 17 x 480 x 832 -> 17 x 240 x 416
+    T, H, W, cc = 17, 480, 832, 96
+    xs = torch.randn((1, T, H, W, cc), generator=g, device=dev).to(torch.bfloat16)
+    ws = synth.kaiming_uniform(cc, cc, (1, 3, 3), 1).to(dev)
+    bs = synth.uniform((cc,), -0.1, 0.1, 2).to(dev)
+    ps = cc3d.Plan(ws, bs, h=H, w=W, max_t=T, pad=(0, 0), stride_hw=2)
+    ys = torch.empty((1, T, H // 2, W // 2, cc), dtype=torch.bfloat16, device=dev)
+    ms = timed(lambda: ps.forward(xs, ys), flush=True)
+    fl = conv_flop(1, cc, cc, T, H // 2, W // 2, taps=9)
+    byts = xs.numel() * 2 + ys.numel() * 2
+    out[f"downsample_s2_c{cc}_{T}x{H}x{W}"] = {
+        "ms": ms, "tflops": fl / ms / 1e9, "frac": fl / ms / 1e9 / peaks["bf16_tflops"],
+        "hbm_gbs": byts / ms / 1e6, "hbm_frac": byts / ms / 1e6 / peaks["hbm_gbs"]}
+    del ps, xs, ys
     # the encoder's other residual blocks (§8(f) NEXT-2): the two that change
     # the channel count (the 1x1x1 conv_shortcut fused into conv2) and a
     # 384-channel one (RMS_norm after conv1 in its own pass), whole sequence

@@ -107,7 +107,13 @@ typedef struct {
                           residual have that many).  Streamed chunks of a
                           multiple of stride_t frames give the whole
                           sequence's outputs.                               */
-  int stride_h, stride_w;            /* must be 1                            */
+  int stride_h, stride_w;  /* 1, or both 2: the downsample path's spatial
+                              step (§10.5): each frame zero-padded by one
+                              row and column after it, then a 3x3 conv with
+                              stride 2 -- kt = 1, kh = kw = 3, pad_h = pad_w
+                              = 0, h and w even, bf16 with c_in % 32 == 0,
+                              bias or residual epilogue.  y (and residual)
+                              are [n][t][h/2][w/2][c_out].                  */
   int dil_t, dil_h, dil_w;           /* must be 1                            */
   int groups;                        /* must be 1                            */
   cc3d_dtype dtype;
@@ -142,9 +148,9 @@ typedef struct cc3d_block cc3d_block;
 
 /* Validate desc, pick a kernel, copy and re-tile the weights (and bias,
  * gamma, beta) into plan-owned device memory.  Synchronous.  Returns
- * CC3D_ERR_UNSUPPORTED for dilation/groups != 1, spatial strides != 1, a
- * temporal stride other than 1 (or 2 on the bf16 c_in % 32 == 0 path),
- * even kernel sizes, or channel counts no kernel covers.  bf16 covers c_out % 16 == 0 with
+ * CC3D_ERR_UNSUPPORTED for dilation/groups != 1, strides other than those
+ * stride_t / stride_h / stride_w document, even kernel sizes, or channel
+ * counts no kernel covers.  bf16 covers c_out % 16 == 0 with
  * either c_in % 32 == 0 (kh == kw in {1, 3}, kt <= 3; N tiles of at most
  * 256 channels) or c_in <= 8 (the thin first-layer path: bias epilogue,
  * c_out <= 256, kt*kh*kw*c_in <= 256); fp32 covers any channel count with

@@ -173,14 +173,14 @@ class Plan:
     device (bf16, or fp32 for dtype=FP32); bias/gamma/beta fp32 [C_out]."""
 
     def __init__(self, weight, bias=None, *, n=1, h, w, max_t, epi=EPI_BIAS, gamma=None,
-                 beta=None, dtype=BF16, pad=None, stride_t=1):
+                 beta=None, dtype=BF16, pad=None, stride_t=1, stride_hw=1):
         co, ci, kt, kh, kw = (int(s) for s in weight.shape)
         d = Desc()
         d.n, d.c_in, d.c_out, d.h, d.w, d.max_t = n, ci, co, h, w, max_t
         d.kt, d.kh, d.kw = kt, kh, kw
         d.pad_h, d.pad_w = pad if pad is not None else (kh // 2, kw // 2)
         d.stride_t = stride_t
-        d.stride_h = d.stride_w = 1
+        d.stride_h = d.stride_w = stride_hw
         d.dil_t = d.dil_h = d.dil_w = 1
         d.groups = 1
         d.dtype = dtype

@@ -109,6 +109,28 @@ bool encode_act_map(CUtensorMap *m, const void *base, int c, int w, int h, int t
   return r == CUDA_SUCCESS;
 }
 
+// The same map walking every other pixel in W and H (element strides 2):
+// a box of box_c channels x box_w x box_h pixels of the stride-2 lattice
+// that starts at the box's first pixel.
+bool encode_act_map_s2(CUtensorMap *m, const void *base, int c, int w, int h, int t, int n,
+                       int box_w, int box_h, int box_c) {
+  if (box_c != 8 && box_c != 64) return false;
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[5] = {(cuuint64_t)c, (cuuint64_t)w, (cuuint64_t)h, (cuuint64_t)t,
+                        (cuuint64_t)n};
+  cuuint64_t strides[4] = {(cuuint64_t)c * 2, (cuuint64_t)c * 2 * w, (cuuint64_t)c * 2 * w * h,
+                           (cuuint64_t)c * 2 * w * h * t};
+  // (the box counts traversed elements: 2 * box pixels at stride 2)
+  cuuint32_t box[5] = {(cuuint32_t)box_c, 2u * (cuuint32_t)box_w, 2u * (cuuint32_t)box_h, 1, 1};
+  cuuint32_t estr[5] = {1, 2, 2, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  box_c == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // 4-D bf16 tensor map over an NDHWC buffer with few channels: dims
 // (W*C, H, T, N), a box of `row` elements x `box_h` rows x 1 x 1.
 bool encode_thin_map(CUtensorMap *m, const void *base, int c, int w, int h, int t, int n,
@@ -181,6 +203,7 @@ struct cc3d_plan {
   int kc, nt, n_ntiles, na, nb, tmem_cols, sm_count, ctas_per_sm, sub, nbuf, split, max_clusters;
   int pair, b_resident;
   int c_sc, n_cc_sc;  // the residual block's fused 1x1x1 conv_shortcut (0: none)
+  int s2;             // stride 2 in H and W (the downsample path's per-frame conv)
   CUtensorMap map_w;  // pair: the weight image as 128-byte swizzled rows
   uint8_t *wimg;
   // fp32 / thin
@@ -236,12 +259,23 @@ cc3d_status check_desc(const cc3d_desc *d, int *variant) {
   if (d->n < 1 || d->c_in < 1 || d->c_out < 1 || d->h < 1 || d->w < 1 || d->max_t < 1)
     return CC3D_ERR_INVALID_ARG;
   if (d->kt < 1 || d->kh < 1 || d->kw < 1) return CC3D_ERR_INVALID_ARG;
-  // temporal stride 2: the downsample path's time_conv (tensor-core path)
-  if (d->stride_t < 1 || d->stride_t > 2 || d->stride_h != 1 || d->stride_w != 1 ||
+  // temporal stride 2: the downsample path's time_conv; spatial stride 2:
+  // its per-frame 3x3 conv (both on the tensor-core path)
+  const bool s2 = d->stride_h == 2 && d->stride_w == 2;
+  if (d->stride_t < 1 || d->stride_t > 2 || !(s2 || (d->stride_h == 1 && d->stride_w == 1)) ||
       d->dil_t != 1 || d->dil_h != 1 || d->dil_w != 1 || d->groups != 1)
     return CC3D_ERR_UNSUPPORTED;
-  if (d->kh % 2 == 0 || d->kw % 2 == 0 || d->pad_h != d->kh / 2 || d->pad_w != d->kw / 2)
+  if (s2) {
+    // ZeroPad2d(0, 1, 0, 1) + 3x3 stride 2 on each frame (pad_h = pad_w = 0:
+    // no zero rows or columns before the frame, one after): H/2 x W/2 out
+    if (d->kt != 1 || d->kh != 3 || d->kw != 3 || d->pad_h != 0 || d->pad_w != 0 ||
+        d->stride_t != 1 || d->h % 2 != 0 || d->w % 2 != 0 || d->dtype != CC3D_BF16 ||
+        d->c_in % 32 != 0 || d->epi == CC3D_EPI_BIAS_RMS_SILU)
+      return CC3D_ERR_UNSUPPORTED;
+  } else if (d->kh % 2 == 0 || d->kw % 2 == 0 || d->pad_h != d->kh / 2 ||
+             d->pad_w != d->kw / 2) {
     return CC3D_ERR_UNSUPPORTED;
+  }
   if (d->kt > 3 || d->kh > 3 || d->kw > 3) return CC3D_ERR_UNSUPPORTED;
   if (d->epi < CC3D_EPI_BIAS || d->epi > CC3D_EPI_BIAS_RMS_SILU) return CC3D_ERR_INVALID_ARG;
   if (d->epi == CC3D_EPI_BIAS_RMS_SILU && !d->gamma) return CC3D_ERR_INVALID_ARG;
@@ -316,7 +350,8 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
   if (s != CC3D_OK) return s;
   if (c_sc < 0 || (c_sc > 0 && !w_sc)) return CC3D_ERR_INVALID_ARG;
   if (c_sc > 0 && (variant != CC3D_VARIANT_UMMA || desc->kh != 3 || desc->kw != 3 ||
-                   desc->stride_t != 1 || desc->epi != CC3D_EPI_BIAS || c_sc % 16 != 0))
+                   desc->stride_t != 1 || desc->stride_h != 1 || desc->epi != CC3D_EPI_BIAS ||
+                   c_sc % 16 != 0))
     return CC3D_ERR_UNSUPPORTED;
   if (!is_sm100()) return CC3D_ERR_UNSUPPORTED;
   cc3d_plan *p = new cc3d_plan();
@@ -404,8 +439,12 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
       UmmaConfig cfg;
       // (the largest call's output frames)
       const int max_out = (desc->max_t - 1) / desc->stride_t + 1;
-      if (!choose_umma_config(desc->n, desc->c_in, desc->c_out, desc->h, desc->w, desc->kt,
-                              desc->kh, desc->epi == CC3D_EPI_BIAS_RMS_SILU, c_sc > 0, max_out,
+      // spatial stride 2 runs as nine 1x1 taps over the output frame
+      p->s2 = desc->stride_h == 2 ? 1 : 0;
+      const int kt_eff = p->s2 ? 9 : desc->kt, ks_eff = p->s2 ? 1 : desc->kh;
+      const int h_out = desc->h / desc->stride_h, w_out = desc->w / desc->stride_w;
+      if (!choose_umma_config(desc->n, desc->c_in, desc->c_out, h_out, w_out, kt_eff, ks_eff,
+                              desc->epi == CC3D_EPI_BIAS_RMS_SILU, c_sc > 0, max_out,
                               p->sm_count, &cfg)) {
         s = CC3D_ERR_UNSUPPORTED;
         goto fail;
@@ -416,7 +455,7 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
       p->b_resident = cfg.b_resident;
       p->max_clusters = 0;
       if (cfg.split > 1 || cfg.pair) {
-        p->max_clusters = umma_max_clusters(cfg, desc->kh);
+        p->max_clusters = umma_max_clusters(cfg, ks_eff);
         if (p->max_clusters < 1) { s = CC3D_ERR_CUDA; goto fail; }
       }
     }
@@ -504,7 +543,8 @@ static cc3d_status forward_impl(cc3d_plan *p, const void *x, int t, const void *
   const int front = d.kt - 1;
   const int t_out = (t - 1) / d.stride_t + 1;  // frames of y (and of residual)
   const size_t in_frame = static_cast<size_t>(d.h) * d.w * d.c_in * esz;
-  const size_t out_frame = static_cast<size_t>(d.h) * d.w * d.c_out * esz;
+  const size_t out_frame =
+      static_cast<size_t>(d.h / d.stride_h) * (d.w / d.stride_w) * d.c_out * esz;
   const size_t x_bytes = in_frame * d.n * t, y_bytes = out_frame * d.n * t_out;
   const size_t c_bytes = in_frame * d.n * front;
   const size_t nc_bytes = out_frame * d.n * 2;
@@ -582,11 +622,15 @@ static cc3d_status forward_impl(cc3d_plan *p, const void *x, int t, const void *
   } else {
     CUtensorMap mx, mc;
     const int tile_w = umma_tile_w() * p->sub;
+    // the kernel's spatial kernel: kh x kw, or 1 x 1 taps for stride 2
+    const int ks = p->s2 ? 1 : d.kh;
+    const int h_out = d.h / d.stride_h, w_out = d.w / d.stride_w;
     // (a pair's CTA loads the halo of its own 8-column half)
-    const int box_w = umma_halo_box_w(p->kc, p->pair ? 1 : p->sub, d.kw);
-    const int box_h = umma_tile_h() + d.kh - 1;
+    const int box_w = umma_halo_box_w(p->kc, p->pair ? 1 : p->sub, ks);
+    const int box_h = umma_tile_h() + ks - 1;
     const int box_c = umma_halo_box_c(p->kc);
-    if (!encode_act_map(&mx, x, d.c_in, d.w, d.h, t, d.n, box_w, box_h, box_c))
+    if (!(p->s2 ? encode_act_map_s2(&mx, x, d.c_in, d.w, d.h, t, d.n, box_w, box_h, box_c)
+                : encode_act_map(&mx, x, d.c_in, d.w, d.h, t, d.n, box_w, box_h, box_c)))
       return reject(CC3D_ERR_CUDA);
     if (cache_in && front > 0) {
       if (!encode_act_map(&mc, cache_in, d.c_in, d.w, d.h, front, d.n, box_w, box_h, box_c))
@@ -606,17 +650,18 @@ static cc3d_status forward_impl(cc3d_plan *p, const void *x, int t, const void *
     a.y = static_cast<__nv_bfloat16 *>(y);
     a.status = status;
     a.wait_limit_ns = wait_limit_ns();
-    a.n = d.n; a.t = t_out; a.h = d.h; a.w = d.w; a.c_in = d.c_in; a.c_out = d.c_out;
-    a.kt = d.kt; a.kh = d.kh; a.kw = d.kw; a.pad_h = d.pad_h; a.pad_w = d.pad_w;
+    a.n = d.n; a.t = t_out; a.h = h_out; a.w = w_out; a.c_in = d.c_in; a.c_out = d.c_out;
+    a.kt = p->s2 ? 9 : d.kt; a.kh = ks; a.kw = ks; a.pad_h = d.pad_h; a.pad_w = d.pad_w;
     a.stride_t = d.stride_t;
+    a.s2 = p->s2;
     a.vec32 = (reinterpret_cast<uintptr_t>(y) & 31u) == 0 ? 1 : 0;
     a.b_resident = p->b_resident;
     a.c_sc = p->c_sc;
     a.n_cc_sc = p->n_cc_sc;
     a.nt = p->nt; a.n_ntiles = p->n_ntiles;
     a.sub = p->sub; a.nbuf = p->nbuf; a.split = p->split; a.pair = p->pair;
-    a.tiles_w = (d.w + tile_w - 1) / tile_w;
-    a.tiles_h = (d.h + umma_tile_h() - 1) / umma_tile_h();
+    a.tiles_w = (w_out + tile_w - 1) / tile_w;
+    a.tiles_h = (h_out + umma_tile_h() - 1) / umma_tile_h();
     a.na = p->na; a.nb = p->nb; a.tmem_cols = p->tmem_cols;
     a.epi = static_cast<int>(d.epi);
     a.has_cache = (cache_in && front > 0) ? 1 : 0;

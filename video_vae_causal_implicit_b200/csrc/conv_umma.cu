@@ -320,22 +320,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     L.b_stage, &full_b[slot]);
         }
       };
+      // channels c0 .. c0+KC-1 of the box of `map` that starts at column
+      // wc, row hc of frame `tcoord` of image `n`, into A slot `slot`
+      auto load_a_at = [&](const CUtensorMap *map, int slot, int c0, int wc, int hc, int tcoord,
+                           int n) {
+        const uint32_t dst = smem_base + L.a_off + slot * L.a_stage;
+        if constexpr (PAIR) {
+          tma_load_5d_pair(dst, map, lead_full_a + 8u * slot, c0, wc, hc, tcoord, n);
+        } else if constexpr (kSw) {
+          tma_load_5d(dst, map, &full_a[slot], c0, wc, hc, tcoord, n);
+        } else {
+#pragma unroll
+          for (int s = 0; s < KC / 8; ++s)
+            tma_load_5d(dst + s * L.slab, map, &full_a[slot], c0 + s * 8, wc, hc, tcoord, n);
+        }
+      };
       // the tile's halo of channels c0 .. c0+KC-1 of frame `tcoord` of `map`
       // into A slot `slot` (this CTA's half of the tile on a pair)
       auto load_a = [&](const CUtensorMap *map, int slot, int c0, int tcoord,
                         const TileCoord &tc) {
-        const uint32_t dst = smem_base + L.a_off + slot * L.a_stage;
-        if constexpr (PAIR) {
-          tma_load_5d_pair(dst, map, lead_full_a + 8u * slot, c0, tc.w0 + kTW * rank - KS / 2,
-                           tc.h0 - KS / 2, tcoord, tc.n);
-        } else if constexpr (kSw) {
-          tma_load_5d(dst, map, &full_a[slot], c0, tc.w0 - KS / 2, tc.h0 - KS / 2, tcoord, tc.n);
-        } else {
-#pragma unroll
-          for (int s = 0; s < KC / 8; ++s)
-            tma_load_5d(dst + s * L.slab, map, &full_a[slot], c0 + s * 8, tc.w0 - KS / 2,
-                        tc.h0 - KS / 2, tcoord, tc.n);
-        }
+        load_a_at(map, slot, c0, tc.w0 + kTW * rank - KS / 2, tc.h0 - KS / 2, tcoord, tc.n);
       };
       if (KS == 1 && p.b_resident) {
         // one N tile and every weight stage in a slot of its own: loaded
@@ -349,7 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int kt = kt_lo + ia / n_cc, cc = ia % n_cc;
           // A frame before the chunk with no cache is all zeros: its stage
           // (and its taps' weights) is skipped here and by the MMA issuer.
-          if (p.stride_t * tc0.t + kt - (p.kt - 1) < 0 && !p.has_cache) continue;
+          if (!(KS == 1 && p.s2) && p.stride_t * tc0.t + kt - (p.kt - 1) < 0 && !p.has_cache)
+            continue;
           if (!mbar_wait_bounded(&empty_a[sa], pa ^ 1, p.wait_limit_ns, p.status, 1)) {
             ok = false;
             break;
@@ -357,10 +362,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (pair_leader) mbar_arrive_expect_tx(&full_a[sa], PAIR ? 2u * a_tx : a_tx);
           a_used |= 1u << sa;
           a_par = (a_par & ~(1u << sa)) | (pa << sa);
-          const int tau = p.stride_t * tc0.t + kt - (p.kt - 1);  // input frame
-          const bool from_cache = tau < 0;  // (zero frames were skipped above)
-          load_a(from_cache ? &map_cache : &map_x, sa, cc * KC, from_cache ? tau + (p.kt - 1) : tau,
-                 tc0);
+          if (KS == 1 && p.s2) {
+            // stride 2 in H and W: stage `kt` is spatial tap (kh, kw) =
+            // (kt / 3, kt % 3); the map walks every other pixel, so the box
+            // of output pixel (h, w) starts at input (2h + kh, 2w + kw)
+            load_a_at(&map_x, sa, cc * KC, 2 * (tc0.w0 + kTW * rank) + kt % 3 - p.pad_w,
+                      2 * tc0.h0 + kt / 3 - p.pad_h, tc0.t, tc0.n);
+          } else {
+            const int tau = p.stride_t * tc0.t + kt - (p.kt - 1);  // input frame
+            const bool from_cache = tau < 0;  // (zero frames were skipped above)
+            load_a(from_cache ? &map_cache : &map_x, sa, cc * KC,
+                   from_cache ? tau + (p.kt - 1) : tau, tc0);
+          }
           if (++sa == L.na) { sa = 0; pa ^= 1; }
           if (KS == 1 && p.b_resident) continue;
 #pragma unroll 1
@@ -479,7 +492,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ia = 0; ia < n_a && ok; ++ia) {
           // the same zero-frame stages the producer skipped; adding their
           // exact zeros would not change the accumulator
-          if (p.stride_t * tcm.t + kt_lo + ia / n_cc - (p.kt - 1) < 0 && !p.has_cache) continue;
+          if (!(KS == 1 && p.s2) && p.stride_t * tcm.t + kt_lo + ia / n_cc - (p.kt - 1) < 0 &&
+              !p.has_cache)
+            continue;
           if (!mbar_wait_bounded(&full_a[sa], pa, p.wait_limit_ns, p.status, 3)) {
             ok = false;
             break;

@@ -40,6 +40,10 @@ struct UmmaArgs {
   int c_sc;                       // > 0: the residual block's 1x1x1 conv_shortcut of a
                                   // c_sc-channel input (map_sc), summed into the accumulator
   int n_cc_sc;                    // its channel chunks, ceil(c_sc / KC) (tail zero-filled)
+  int s2;                         // 1: stride 2 in H and W (the downsample path's 3x3 conv
+                                  // per frame): kt = 9 spatial taps of a 1x1 kernel, each
+                                  // read through a map that walks every other pixel; h, w
+                                  // are the output frame's
 };
 
 // Tile configuration of the UMMA conv for a plan (chosen from n, c_in, c_out,

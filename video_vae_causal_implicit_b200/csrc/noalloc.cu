@@ -191,6 +191,7 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   a.vec32 = (reinterpret_cast<uintptr_t>(y) & 31u) == 0 ? 1 : 0;
   a.b_resident = cfg.b_resident;
   a.c_sc = 0;
+  a.s2 = 0;
   a.n_cc_sc = 0;
   a.h = d->h; a.w = d->w; a.c_in = d->c_in; a.c_out = d->c_out;
   a.kt = d->kt; a.kh = d->kh; a.kw = d->kw; a.pad_h = d->pad_h; a.pad_w = d->pad_w;
