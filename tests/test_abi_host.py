@@ -86,6 +86,21 @@ def test_temporal_stride_only_on_the_tensor_core_path(lib, kw):
     assert not out.value
 
 
+@pytest.mark.parametrize("kw", [dict(pad_h=1, pad_w=1), dict(kt=3), dict(h=9), dict(w=7),
+                                dict(stride_t=2), dict(dtype=cc3d.FP32), dict(c_in=3),
+                                dict(epi=cc3d.EPI_BIAS_RMS_SILU, gamma=0x2000),
+                                dict(stride_w=1)])
+def test_spatial_stride_two_only_for_the_downsample_conv(lib, kw):
+    """Stride 2 in H and W is the downsample path's 3x3 conv (kt = 1, no
+    leading pad, even frame, bf16 tensor-core channels, no RMS epilogue);
+    anything else with it is refused before any device query."""
+    base = dict(kt=1, kh=3, kw=3, pad_h=0, pad_w=0, stride_h=2, stride_w=2, h=8, w=8)
+    base.update(kw)
+    out = ctypes.c_void_p()
+    assert cc3d.cc3d_plan_create(_desc(**base), out) == cc3d.ERR_UNSUPPORTED
+    assert not out.value
+
+
 @pytest.mark.parametrize("field,value", [("n", 0), ("h", 0), ("max_t", 0), ("epi", 7)])
 def test_invalid_descriptors_refused(lib, field, value):
     out = ctypes.c_void_p()
