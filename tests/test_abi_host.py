@@ -171,3 +171,22 @@ def test_no_gpu_means_unsupported_not_a_fallback(lib):
     out = ctypes.c_void_p()
     assert cc3d.cc3d_plan_create(_desc(), out) == cc3d.ERR_UNSUPPORTED
     assert cc3d.cc3d_launch_count() == 0
+
+def test_noalloc_validation_before_any_device_work(lib):
+    """cc3d_forward_noalloc refuses bad calls on the host, before touching
+    its scratch or the GPU (so these run without one)."""
+    p = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    f = cc3d.cc3d_forward_noalloc
+    assert f(_desc(), None, 1, None, p, None, None, None, None, None) == cc3d.ERR_INVALID_ARG
+    assert f(_desc(), p, 5, None, p, None, None, None, None, None) == cc3d.ERR_INVALID_ARG  # t > max_t
+    assert f(_desc(epi=cc3d.EPI_BIAS_RESIDUAL), p, 1, None, p, None, None, None, None,
+             None) == cc3d.ERR_INVALID_ARG  # residual epilogue without a residual
+    assert f(_desc(stride_h=2, stride_w=2), p, 1, None, p, None, None, None, None, None) == \
+        cc3d.ERR_UNSUPPORTED
+    assert f(_desc(c_in=48), p, 1, None, p, None, None, None, None, None) == cc3d.ERR_UNSUPPORTED
+    assert f(_desc(dtype=cc3d.FP32), p, 1, None, p, None, None, None, None, None) == \
+        cc3d.ERR_UNSUPPORTED
+    assert f(_desc(c_in=1024, c_out=1024), p, 1, None, p, None, None, None, None, None) == \
+        cc3d.ERR_TOO_LARGE  # 56 MB of weights against an 8 MiB scratch
+    assert f(_desc(), odd, 1, None, p, None, None, None, None, None) == cc3d.ERR_ALIGNMENT
