@@ -16,6 +16,10 @@ Cases (seeded synthetic inputs, generated on the device):
   tc192   the downsample path's time_conv: 192 -> 192, kernel (3, 1, 1),
           stride 2 in time, x[1,192,17,120,208] (9 output frames)
   tc384   the same at 384 channels on x[1,384,9,60,104] (5 output frames)
+  ds96    the downsample path's per-frame ZeroPad2d(0,1,0,1) + 3x3 stride-2
+          conv, 96 channels, x[1,96,17,480,832] -> 240 x 416
+  blk96   the encoder's channel-changing block 96 -> 192 (conv_shortcut fused
+          into conv2) on x[1,96,17,240,416]
 Prints nothing but a final "ok"; timing comes from the profiler.
 """
 from __future__ import annotations
@@ -48,6 +52,10 @@ def build_case(name, dev):
         c, T, H, W = 192, 17, 120, 208
     elif name == "tc384":
         c, T, H, W = 384, 9, 60, 104
+    elif name == "ds96":
+        c, T, H, W = 96, 17, 480, 832
+    elif name == "blk96":
+        c, T, H, W = 96, 17, 240, 416
     else:
         raise SystemExit(f"unknown case {name}")
     x = _rand((1, T, H, W, c), dev)
@@ -61,6 +69,23 @@ def build_case(name, dev):
         blk = cc3d.Block(w1, b1, g1, w2, b2, g2, h=H, w=W, max_t=T)
         y = torch.empty_like(x)
         return lambda: blk.forward(x, y), [blk]
+    if name == "ds96":
+        wt = synth.kaiming_uniform(c, c, (1, 3, 3), 1).to(dev)
+        b = synth.uniform((c,), -0.1, 0.1, 2).to(dev)
+        plan = cc3d.Plan(wt, b, h=H, w=W, max_t=T, pad=(0, 0), stride_hw=2)
+        y = torch.empty((1, T, H // 2, W // 2, c), dtype=torch.bfloat16, device=dev)
+        return (lambda: plan.forward(x, y)), [plan]
+    if name == "blk96":
+        co = 192
+        wts = dict(w1=synth.kaiming_uniform(co, c, (3, 3, 3), 1),
+                   b1=synth.uniform((co,), -0.1, 0.1, 2), g1=synth.uniform((c,), 0.5, 1.5, 3),
+                   w2=synth.kaiming_uniform(co, co, (3, 3, 3), 4),
+                   b2=synth.uniform((co,), -0.1, 0.1, 5), g2=synth.uniform((co,), 0.5, 1.5, 6),
+                   w_sc=synth.kaiming_uniform(co, c, (1, 1, 1), 7),
+                   b_sc=synth.uniform((co,), -0.1, 0.1, 8))
+        blk = cc3d.Block(**{k: v.to(dev) for k, v in wts.items()}, h=H, w=W, max_t=T)
+        y = torch.empty((1, T, H, W, co), dtype=torch.bfloat16, device=dev)
+        return (lambda: blk.forward(x, y)), [blk]
     if name in ("tc192", "tc384"):
         wt = synth.kaiming_uniform(c, c, (3, 1, 1), 1).to(dev)
         b = synth.uniform((c,), -0.1, 0.1, 2).to(dev)
