@@ -1,0 +1,31 @@
+"""The sampled-parity helper used by the full-size GPU tests, checked on
+the CPU: fed the oracle's own whole-sequence output it passes, and a
+single wrong voxel at a sampled pixel makes it fail."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.sampled import check_frames, sample_frame_points
+from video_vae_causal_implicit_b200 import synth
+
+
+def _case():
+    case = synth.conv_case(6, 5, 6, 7, 9, seed_base=40)
+    x = synth.ndhwc(case["x"])
+    y = oracle.causal_conv3d(synth.ncthw_view(x), case["w"], case["b"].double().numpy())
+    y = torch.from_numpy(y).permute(0, 2, 3, 4, 1).contiguous()  # NDHWC, float64
+    return x, y, case
+
+
+def test_helper_accepts_the_oracle_output():
+    x, y, case = _case()
+    check_frames(x, y, case["w"], case["b"], [0, 1, 2, 5], 6, 7, "helper")
+
+
+def test_helper_rejects_a_wrong_voxel():
+    x, y, case = _case()
+    hw = sample_frame_points(7, 9, 6, 7 + 2)  # the pixels frame index 2 samples
+    y[0, 2, hw[-1, 0], hw[-1, 1], 3] += 10.0
+    with pytest.raises(AssertionError):
+        check_frames(x, y, case["w"], case["b"], [0, 1, 2, 5], 6, 7, "helper")
