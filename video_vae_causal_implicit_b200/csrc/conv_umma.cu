@@ -339,7 +339,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // into A slot `slot` (this CTA's half of the tile on a pair)
       auto load_a = [&](const CUtensorMap *map, int slot, int c0, int tcoord,
                         const TileCoord &tc) {
-        load_a_at(map, slot, c0, tc.w0 + kTW * rank - KS / 2, tc.h0 - KS / 2, tcoord, tc.n);
+        // (only a pair's CTAs hold different columns: a temporal split's
+        // CTAs all load the whole tile)
+        load_a_at(map, slot, c0, tc.w0 + (PAIR ? kTW * rank : 0) - KS / 2, tc.h0 - KS / 2, tcoord,
+                  tc.n);
       };
       if (KS == 1 && p.b_resident) {
         // one N tile and every weight stage in a slot of its own: loaded
@@ -366,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // stride 2 in H and W: stage `kt` is spatial tap (kh, kw) =
             // (kt / 3, kt % 3); the map walks every other pixel, so the box
             // of output pixel (h, w) starts at input (2h + kh, 2w + kw)
-            load_a_at(&map_x, sa, cc * KC, 2 * (tc0.w0 + kTW * rank) + kt % 3 - p.pad_w,
+            load_a_at(&map_x, sa, cc * KC, 2 * (tc0.w0 + (PAIR ? kTW * rank : 0)) + kt % 3 - p.pad_w,
                       2 * tc0.h0 + kt / 3 - p.pad_h, tc0.t, tc0.n);
           } else {
             const int tau = p.stride_t * tc0.t + kt - (p.kt - 1);  // input frame
