@@ -231,13 +231,15 @@ def rms_norm(x, gamma, beta=None, silu=False):
 
 
 def resblock(x, w1, b1, g1, w2, b2, g2, cache1=None, cache2=None, round_bf16=True,
-             return_acts=False, w_sc=None, b_sc=None, round_h1=False):
+             return_acts=False, w_sc=None, b_sc=None, round_h1=True):
     """WanResidualBlock from C_in = x's channels to C_out = w1's output
     channels.  The shortcut is x itself (w_sc None, C_in == C_out) or the
     1x1x1 conv_shortcut w_sc [C_out, C_in, 1, 1, 1] + b_sc.  round_bf16
-    rounds a0 and a1 to bf16; round_h1 also rounds conv1's output before
-    its RMS_norm.  Returns y float64 [N, C_out, T, H, W] (and a0, a1 when
-    return_acts)."""
+    rounds a0 and a1 to bf16; round_h1 rounds conv1's output h1 to bf16
+    before its RMS_norm.  Both are on by default: in every block the page's
+    module hands a0, h1 and a1 on as bf16 activations ("Cosmos3 Wan VAE",
+    §10.4 WanResidualBlock, run in bf16).  Returns y float64
+    [N, C_out, T, H, W] (and a0, a1 when return_acts)."""
     lib = _load()
     keep = []
     N, Cin, T, H, W = _shape5(x)
@@ -261,7 +263,7 @@ def resblock(x, w1, b1, g1, w2, b2, g2, cache1=None, cache2=None, round_bf16=Tru
 
 
 def resblock_points(x, w1, b1, g1, w2, b2, g2, points, cache1=None, cache2=None,
-                    round_bf16=True, w_sc=None, b_sc=None, round_h1=False):
+                    round_bf16=True, w_sc=None, b_sc=None, round_h1=True):
     """The residual block at chosen output voxels.  Returns float64 [P, C_out]."""
     lib = _load()
     keep = []

@@ -110,7 +110,8 @@ def _failures(mod):
     w1, w2, wsc = _rnd((6, 4, 3, 3, 3), 8, 0.2), _rnd((6, 6, 3, 3, 3), 9, 0.2), _rnd((6, 4, 1, 1, 1), 10)
     b1, b2, bsc = _rnd((6,), 11), _rnd((6,), 12), _rnd((6,), 13)
     g1, g2 = np.abs(_rnd((4,), 14)) + 0.5, np.abs(_rnd((6,), 15)) + 0.5
-    y = mod.resblock(xb, w1, b1, g1, w2, b2, g2, round_bf16=False, w_sc=wsc, b_sc=bsc)
+    y = mod.resblock(xb, w1, b1, g1, w2, b2, g2, round_bf16=False, round_h1=False, w_sc=wsc,
+                     b_sc=bsc)
     a0 = _rs(torch.from_numpy(xb), torch.from_numpy(g1)).numpy()
     a1 = _rs(torch.from_numpy(_torch_conv(a0, w1, b1)), torch.from_numpy(g2)).numpy()
     ref = _torch_conv(a1, w2, b2) + F.conv3d(torch.from_numpy(xb), torch.from_numpy(wsc),

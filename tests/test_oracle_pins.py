@@ -384,7 +384,9 @@ def test_block_is_composition_of_pinned_parts():
     # double->float->bf16 can double-round; compare with tolerance of 1 bf16 ulp
     np.testing.assert_allclose(a0, a0_ref.numpy(), rtol=2 ** -7, atol=1e-30)
     a0t = torch.from_numpy(a0)
-    h1 = torch.from_numpy(torch_causal_conv3d(a0t.numpy(), _np(c["w1"]), _np(c["b1"])))
+    # conv1's output h1 is a bf16 activation (the default reading)
+    h1 = torch.from_numpy(oracle.round_bf16_array(
+        torch_causal_conv3d(a0t.numpy(), _np(c["w1"]), _np(c["b1"]))))
     a1_ref = rs(h1, c["g2"]).numpy()
     np.testing.assert_allclose(a1, oracle.round_bf16_array(a1_ref), rtol=0, atol=0)
     y_ref = torch_causal_conv3d(a1, _np(c["w2"]), _np(c["b2"])) + x.numpy()

@@ -768,7 +768,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const __nv_bfloat16 *rrow = p.residual ? p.residual + pix * p.c_out + n0 : nullptr;
         float inv = 1.0f;
         if (p.epi == 2) {
-          // pass 1: sum of squares of the biased row (three loads in flight)
+          // pass 1: sum of squares of the biased row h1 (three loads in
+          // flight).  h1 is a bf16 activation, as it is when conv1 writes it
+          // out for a separate RMS_norm: it is rounded before it is used.
           float ss = 0.f;
           for (int j0 = 0; j0 < p.nt; j0 += 48) {
             const int nld = (p.nt - j0) >= 48 ? 3 : (p.nt - j0) / 16;
@@ -786,7 +788,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               ld_param16(s_bias + 4u * static_cast<uint32_t>(n0 + j0 + 16 * u), bv);
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                const float hv = __uint_as_float(raw[16 * u + i]) + bv[i];
+                const float hv = round_to_bf16(__uint_as_float(raw[16 * u + i]) + bv[i]);
                 ss = fmaf(hv, hv, ss);
               }
             }
@@ -862,7 +864,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               ld_param16(s_beta + 4u * static_cast<uint32_t>(n0 + j), be);
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                float a = v[i] * inv * gv[i];
+                float a = round_to_bf16(v[i]) * inv * gv[i];
                 a += be[i];
                 v[i] = silu_fast(a);
               }

@@ -366,6 +366,13 @@ __device__ __forceinline__ float silu_fast(float a) {
   return fmaf(h, t, h);
 }
 
+// v rounded to the nearest bf16 (ties to even), returned as fp32.
+__device__ __forceinline__ float round_to_bf16(float v) {
+  uint16_t h;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(v));
+  return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
