@@ -83,8 +83,10 @@ typedef enum { CC3D_BF16 = 0, CC3D_FP32 = 1 } cc3d_dtype;
 typedef enum {
   CC3D_EPI_BIAS = 0,          /* y = conv + b                                  */
   CC3D_EPI_BIAS_RESIDUAL = 1, /* y = conv + b + residual                       */
-  CC3D_EPI_BIAS_RMS_SILU = 2  /* y = SiLU(RMS(conv + b; gamma) (+ beta)),
-                                 needs c_out <= 256 so one CTA owns a row      */
+  CC3D_EPI_BIAS_RMS_SILU = 2  /* y = SiLU(RMS(h; gamma) (+ beta)), h = conv + b
+                                 rounded to bf16 first (the block's conv1
+                                 output is a bf16 activation); needs
+                                 c_out <= 256 so one CTA owns a row          */
 } cc3d_epilogue;
 
 /* Kernel that served a call (the plan's route counters). */
@@ -133,9 +135,8 @@ typedef struct {
   int tile_h, tile_w;      /* output tile (rows x cols of one frame)         */
   int n_tile;              /* output channels per CTA                        */
   int k_chunk;             /* input channels per pipeline stage              */
-  int k_split;             /* CTAs sharing one output tile, one temporal tap
-                              each, summed in one of them: 1, or kt for
-                              frames too small to occupy the GPU            */
+  int k_split;             /* always 1: every output sums all of its taps in
+                              one accumulator of one CTA (no split-K)       */
   int mma_ctas;            /* CTAs (SMs) per tensor-core MMA: 1, or 2 for a
                               CTA pair issuing 2-SM MMAs (M = 256)          */
   int w_resident;          /* 1: the weights stay in shared memory for the
@@ -166,6 +167,8 @@ cc3d_status cc3d_plan_destroy(cc3d_plan *plan);
  *                                      (t' = t at temporal stride 1)
  *   cache_out [n][kt-1][h][w][c_in]    nullable: the last kt-1 frames of
  *                                      concat(cache_in, x), for the next call
+ *                                      (written by the conv kernel itself on
+ *                                      the tensor-core path: no extra launch)
  *   residual  [n][t'][h][w][c_out]     EPI_BIAS_RESIDUAL only, else NULL
  *   next_cache_in / next_cache_out     EPI_BIAS_RMS_SILU only, nullable:
  *                                      [n][2][h][w][c_out]; next_cache_out
@@ -181,7 +184,8 @@ cc3d_status cc3d_forward(cc3d_plan *plan, const void *x, int t,
 /* Stand-alone channel RMS_norm + SiLU (§10.2, §10.4), bf16 in / bf16 out.
  *   x, y      [n][t][h][w][c]; gamma [c] fp32; beta [c] fp32 nullable
  *   cache_in / cache_out  nullable, [n][2][h][w][c]: cache_out receives the
- *             last 2 frames of concat(cache_in (or zeros), y).
+ *             last 2 frames of concat(cache_in (or zeros), y), written by
+ *             the same kernel.
  * c must be a multiple of 8 and at most 1024. */
 cc3d_status rmsnorm_silu(const void *x, const float *gamma, const float *beta,
                          int n, int t, int h, int w, int c, void *y,
@@ -201,7 +205,8 @@ cc3d_status cc3d_block_create(int n, int c, int h, int w, int max_t,
  * conv_shortcut, required when c_in != c_out (NULL: identity shortcut).
  * The shortcut runs inside conv2 as extra K steps of the same accumulator
  * (the shortcut's bias is added to b2); for c_out > 256 conv1 writes its
- * biased output and a separate RMS_norm + SiLU pass follows.
+ * biased output (bf16) and a separate RMS_norm + SiLU pass follows.  In
+ * every block conv1's output is rounded to bf16 before its RMS_norm.
  * c_in, c_out multiples of 32 in [32, 1024], else CC3D_ERR_UNSUPPORTED;
  * CC3D_ERR_INVALID_ARG for a NULL weight or gamma, or c_in != c_out without
  * w_sc.  The block owns its activation buffers (max_t frames each). */

@@ -108,26 +108,24 @@ def test_config2_whole_and_streaming_bitwise_and_oracle():
     both against the full fp64 oracle."""
     case = synth.conv_case(384, 384, 5, 30, 52)
     plan, x, y = run_conv(case)
-    # a plan for 5-frame calls: one CTA per tile (the temporal split would
-    # take 4 rounds of clusters for 140 tiles)
-    assert plan.stats().k_split == 1
+    assert plan.stats().k_split == 1  # every output sums all taps in one accumulator
     ys = _stream_chunks(plan, x, 1, 384)
     assert torch.equal(ys.cpu(), y.cpu()), "streaming != whole sequence"
     ref = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], _bias64(case["b"]))
     assert_close_bf16(ncthw_np(y), ref, "config 2")
 
 
-def test_config2_streaming_plan_splits_and_matches_oracle():
-    """A plan made for one-frame calls (max_t = 1) of the config-2 layer
-    takes the temporal split (28 tiles a frame); its streamed chunks carry
-    the cache and match the oracle."""
+def test_config2_streaming_plan_is_bitwise_the_whole_sequence_plan():
+    """The config-2 layer planned for one-frame calls only (max_t = 1) may
+    pick another tile shape than the plan for 5-frame calls; every output
+    still sums its taps into one accumulator in the same order, so its
+    streamed chunks give the whole-sequence plan's bytes."""
     case = synth.conv_case(384, 384, 5, 30, 52)
-    x = to_dev(synth.ndhwc(case["x"]))
-    plan = cc3d.Plan(to_dev(case["w"]), to_dev(case["b"]), h=30, w=52, max_t=1)
-    assert plan.stats().k_split == 3
-    ys = _stream_chunks(plan, x, 1, 384)
-    ref = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], _bias64(case["b"]))
-    assert_close_bf16(ncthw_np(ys), ref, "config 2, streaming plan")
+    plan5, x, y = run_conv(case)
+    plan1 = cc3d.Plan(to_dev(case["w"]), to_dev(case["b"]), h=30, w=52, max_t=1)
+    assert plan1.stats().k_split == 1
+    ys = _stream_chunks(plan1, x, 1, 384)
+    assert torch.equal(ys.cpu(), y.cpu()), "streaming-only plan != whole-sequence plan"
 
 
 @pytest.mark.parametrize("chunk", [2, 3])
@@ -207,7 +205,8 @@ def test_rms_silu_epilogue():
     plan.forward(x, y)
     cc3d.sync_status()
     h1 = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], _bias64(case["b"]))
-    ref = oracle.rms_norm(h1, g.double().numpy(), silu=True)
+    # the conv's output is rounded to bf16 before its RMS_norm (the block's h1)
+    ref = oracle.rms_norm(oracle.round_bf16_array(h1), g.double().numpy(), silu=True)
     assert_close_bf16(ncthw_np(y), ref, "rms+silu epilogue")
 
 

@@ -2,7 +2,8 @@
 kernels is bounded.  A child process runs with a 1 microsecond wait limit
 (CC3D_WAIT_LIMIT_US=1), so the pipelines' first real waits run out; the
 kernels must record the timeout, drain their own in-flight copies and
-MMAs, free tensor memory and return.  The host then sees CC3D_ERR_TIMEOUT
+MMAs, free tensor memory and return.  The limit governs every entry point,
+cc3d_forward_noalloc included.  The host then sees CC3D_ERR_TIMEOUT
 from cc3d_sync_status (once: reading clears it) and the CUDA context stays
 usable."""
 import json
@@ -22,14 +23,28 @@ sys.path.insert(0, %r)
 from video_vae_causal_implicit_b200 import cc3d, synth
 dev = torch.device('cuda', 0)
 out = {}
-# tensor-core conv, several tiles per SM
-case = synth.conv_case(384, 384, 2, 30, 52)
+# tensor-core conv, one CTA per tile (not a CTA pair: a pair's drain at
+# exit covers the loads its leader armed, which a 1 us limit can outrun)
+case = synth.conv_case(96, 96, 2, 30, 52)
 plan = cc3d.Plan(case['w'].to(dev), case['b'].to(dev), h=30, w=52, max_t=2)
+assert plan.stats().mma_ctas == 1
 x = synth.ndhwc(case['x']).to(dev)
-y = torch.empty((1, 2, 30, 52, 384), dtype=torch.bfloat16, device=dev)
-plan.forward(x, y)
+y = torch.empty((1, 2, 30, 52, 96), dtype=torch.bfloat16, device=dev)
+cache_out = torch.empty((1, 2, 30, 52, 96), dtype=torch.bfloat16, device=dev)
+plan.forward(x, y, cache_out=cache_out)
 out['umma_first'] = cc3d.cc3d_sync_status(cc3d._stream())
 out['umma_second'] = cc3d.cc3d_sync_status(cc3d._stream())
+# the same conv through the entry point without device allocation
+d = plan.desc
+wkeep = case['w'].to(dev)
+d.weight = wkeep.data_ptr()
+bkeep = case['b'].to(dev)
+d.bias = bkeep.data_ptr()
+import ctypes
+out['noalloc_call'] = cc3d.cc3d_forward_noalloc(d, ctypes.c_void_p(x.data_ptr()), 2, None,
+                                                ctypes.c_void_p(y.data_ptr()), None, None, None,
+                                                None, cc3d._stream())
+out['noalloc_first'] = cc3d.cc3d_sync_status(cc3d._stream())
 # thin first-layer conv
 c3 = synth.conv_case(3, 96, 3, 48, 64, x_dist='uniform')
 p3 = cc3d.Plan(c3['w'].to(dev), c3['b'].to(dev), h=48, w=64, max_t=3)
@@ -55,5 +70,7 @@ def test_bounded_waits_report_timeout_and_leave_context_usable():
     TIMEOUT, OK = 7, 0
     assert res["umma_first"] == TIMEOUT
     assert res["umma_second"] == OK          # reading the status clears it
+    assert res["noalloc_call"] == OK         # the limit reaches this entry point too
+    assert res["noalloc_first"] == TIMEOUT
     assert res["thin_first"] == TIMEOUT
     assert res["torch_after"] == float(sum(range(1024)) * 2)

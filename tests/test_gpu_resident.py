@@ -101,5 +101,6 @@ def test_resident_rms_epilogue_on_a_pair():
     cc3d.sync_status()
     conv = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], case["b"].double().numpy(),
                                 pad=(0, 0))
-    ref = oracle.rms_norm(conv, g.double().numpy(), be.double().numpy(), silu=True)
+    ref = oracle.rms_norm(oracle.round_bf16_array(conv), g.double().numpy(),
+                          be.double().numpy(), silu=True)
     assert_close_bf16(ncthw_np(y), ref, "resident rms epilogue")

@@ -1,10 +1,9 @@
 """Host logic of the tensor-core conv's planner (choose_umma_config), no
 GPU: a small C++ probe links libcc3d.so and reports the plan chosen for a
 grid of shapes; the tests check the invariants every plan must satisfy
-(shared and tensor memory within the SM's, N tiles that divide C_out, the
-temporal split and resident weights only where they are valid) and the
-choices the design rests on (the latent-resolution layer unsplit for
-5-frame calls and split for 1-frame calls, the residual block on CTA
+(shared and tensor memory within the SM's, N tiles that divide C_out,
+weight slots of whole kernel rows, resident weights only where they are
+valid) and the choices the design rests on (the residual block on CTA
 pairs, the time_conv with resident weights)."""
 import itertools
 import os
@@ -18,7 +17,7 @@ from video_vae_causal_implicit_b200 import cc3d
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(ROOT, "video_vae_causal_implicit_b200", "csrc")
-FIELDS = ("ok", "kc", "nt", "n_ntiles", "sub", "nbuf", "split", "pair", "na", "nb", "tmem_cols",
+FIELDS = ("ok", "kc", "nt", "n_ntiles", "sub", "nbuf", "g_taps", "pair", "na", "nb", "tmem_cols",
           "ctas_per_sm", "params", "b_resident", "smem")
 SMEM_MAX = 227 * 1024
 
@@ -50,22 +49,22 @@ def probe(tmp_path_factory):
     return run
 
 
-def case(n=1, ci=64, co=64, h=30, w=52, kt=3, ks=3, rms=False, sc=False, mt=1, sms=148):
-    return (n, ci, co, h, w, kt, ks, rms, sc, mt, sms)
+def case(n=1, ci=64, co=64, h=30, w=52, kt=3, ks=3, rms=False, mt=1, sms=148):
+    return (n, ci, co, h, w, kt, ks, rms, mt, sms)
 
 
-GRID = [case(n=n, ci=ci, co=co, h=h, w=w, kt=kt, ks=ks, rms=rms, sc=sc, mt=mt)
-        for (ci, co), (h, w), (kt, ks), rms, sc, n, mt in itertools.product(
+GRID = [case(n=n, ci=ci, co=co, h=h, w=w, kt=kt, ks=ks, rms=rms, mt=mt)
+        for (ci, co), (h, w), (kt, ks), rms, n, mt in itertools.product(
             [(32, 48), (64, 64), (96, 96), (96, 192), (192, 192), (192, 384), (384, 384)],
             [(9, 17), (30, 52), (120, 208), (240, 416)],
             [(3, 3), (3, 1), (1, 1)],
-            [False, True], [False, True], [1, 4], [1, 5])
-        if not (rms and co > 256) and not (sc and ks != 3) and not (sc and rms)]
+            [False, True], [1, 4], [1, 5])
+        if not (rms and co > 256)]
 
 
 def test_every_plan_fits_the_sm(probe):
     for c, p in zip(GRID, probe(GRID)):
-        n, ci, co, h, w, kt, ks, rms, sc, mt, sms = c
+        n, ci, co, h, w, kt, ks, rms, mt, sms = c
         assert p["ok"] == 1, c
         assert p["smem"] <= SMEM_MAX, (c, p)
         assert 32 <= p["tmem_cols"] <= 512 and p["tmem_cols"] & (p["tmem_cols"] - 1) == 0, (c, p)
@@ -80,21 +79,24 @@ def test_every_plan_fits_the_sm(probe):
         assert 1 <= p["ctas_per_sm"] <= 2, (c, p)
 
 
-def test_split_pair_and_resident_only_where_valid(probe):
+def test_slots_pair_and_resident_only_where_valid(probe):
     for c, p in zip(GRID, probe(GRID)):
-        n, ci, co, h, w, kt, ks, rms, sc, mt, sms = c
-        assert p["split"] in (1, kt), (c, p)
-        if p["split"] > 1:
-            assert not rms and not sc and p["sub"] == 1 and not p["pair"], (c, p)
+        n, ci, co, h, w, kt, ks, rms, mt, sms = c
+        # a weight slot holds one tap, or one whole kernel row of taps
+        assert p["g_taps"] in (1, ks), (c, p)
         if p["pair"]:
             assert p["kc"] == 64 and p["sub"] == 2 and p["ctas_per_sm"] == 1, (c, p)
         if p["b_resident"]:
-            assert ks == 1 and p["n_ntiles"] == 1 and p["split"] == 1 and not sc, (c, p)
+            assert ks == 1 and p["n_ntiles"] == 1 and p["g_taps"] == 1, (c, p)
             assert p["nb"] == kt * ci // p["kc"] and p["na"] >= 3, (c, p)
         else:
             assert 2 <= p["na"] <= 8 and 2 <= p["nb"] <= 8, (c, p)
             if ks == 3:
                 assert p["na"] == 2, (c, p)
+                # kernel-row slots wherever two of them fit beside the two
+                # halo stages: every 64-channel-chunk plan up to N = 192
+                if p["kc"] == 64 and p["nt"] <= 192:
+                    assert p["g_taps"] == 3, (c, p)
 
 
 def test_plan_is_a_function_of_the_problem(probe):
@@ -113,28 +115,22 @@ def test_downsample_conv_plans(probe):
                  [(64, 64), (96, 96), (64, 128), (192, 192)],
                  [(10, 12), (15, 26), (48, 80), (240, 416)], [1, 2], [1, 17])]
     for c, p in zip(cases, probe(cases)):
-        assert p["ok"] == 1 and p["smem"] <= SMEM_MAX and p["split"] == 1, (c, p)
+        assert p["ok"] == 1 and p["smem"] <= SMEM_MAX and p["g_taps"] == 1, (c, p)
         if p["b_resident"]:
             assert p["nb"] == 9 * c[1] // p["kc"] and p["na"] >= 3, (c, p)
 
 
 def test_the_documented_choices(probe):
-    c2_whole, c2_chunks, c4, tc192, tc384, blk_sc = probe([
-        case(ci=384, co=384, h=30, w=52, mt=5),
-        case(ci=384, co=384, h=30, w=52, mt=1),
+    c4, tc192, tc384, c2 = probe([
         case(ci=192, co=192, h=240, w=416, rms=True, mt=9),
         case(ci=192, co=192, h=120, w=208, ks=1, mt=9),
         case(ci=384, co=384, h=60, w=104, ks=1, mt=5),
-        case(ci=192, co=192, h=240, w=416, sc=True, mt=17),
+        case(ci=384, co=384, h=30, w=52, mt=5),
     ])
-    # the latent-resolution layer: unsplit for its 5-frame call, temporal
-    # split when planned for one-frame calls only
-    assert (c2_whole["split"], c2_whole["pair"], c2_whole["nt"]) == (1, 0, 192)
-    assert c2_chunks["split"] == 3
-    # the residual block's convs run on CTA pairs
-    assert (c4["pair"], c4["nt"]) == (1, 192)
+    # the residual block's convs run on CTA pairs with kernel-row weight slots
+    assert (c4["pair"], c4["nt"], c4["g_taps"]) == (1, 192, 3)
     # the 192-channel time_conv keeps its weights resident; 384 channels do not fit
     assert (tc192["pair"], tc192["b_resident"], tc192["nb"]) == (1, 1, 9)
     assert tc384["b_resident"] == 0
-    # a conv carrying the conv_shortcut is never split
-    assert blk_sc["split"] == 1
+    # the latent-resolution layer: kernel-row weight slots
+    assert c2["g_taps"] == 3

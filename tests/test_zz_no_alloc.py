@@ -11,6 +11,7 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 from tests.parity import assert_close_bf16, ncthw_np, to_dev
 from video_vae_causal_implicit_b200 import cc3d, synth
 
@@ -40,10 +41,10 @@ def _p(t):
 
 def test_noalloc_matches_planned_conv_on_two_calls_in_a_row():
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    # call 1: 384 -> 384 with a bias and a cache (the temporal split); call 2:
-    # different weights, no bias (the scratch's zero bias must be cleared),
-    # 96 -> 192; call 3: a frame large enough for the CTA pair, whose weights
-    # the scratch holds as plain rows behind a tensor map.
+    # call 1: 384 -> 384 with a bias and a cache (a small frame, two N
+    # tiles); call 2: different weights, no bias (the scratch's zero bias
+    # must be cleared), 96 -> 192; call 3: a frame large enough for the CTA
+    # pair, whose weights the scratch holds as plain rows behind a tensor map.
     cases = [
         dict(cin=384, cout=384, t=2, h=30, w=52, bias=True, cache=True, seed=1),
         dict(cin=96, cout=192, t=3, h=21, w=17, bias=False, cache=False, seed=2),
@@ -73,9 +74,13 @@ def test_noalloc_matches_planned_conv_on_two_calls_in_a_row():
                                        None, None, stream)
         assert st == cc3d.OK, cc3d.cc3d_status_string(st)
         cc3d.sync_status()
-        assert_close_bf16(ncthw_np(y), ncthw_np(y_ref), f"noalloc call {cs}")
         assert torch.equal(y.cpu(), y_ref.cpu())  # same kernel and tiles: same bytes
         assert torch.equal(cache_out[:, -2:].cpu(), x[:, -2:].cpu())
+        ref = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"],
+                                   case["b"].double().numpy() if cs["bias"] else None,
+                                   cache=synth.ncthw_view(cache.cpu()) if cache is not None
+                                   else None)
+        assert_close_bf16(ncthw_np(y), ref, f"noalloc call {cs} vs oracle")
         outs.append(y)
         plan.close()
     torch.cuda.synchronize()
@@ -103,6 +108,56 @@ def test_noalloc_matches_planned_time_conv_with_resident_weights():
     assert res == cc3d.OK, cc3d.cc3d_status_string(res)
     cc3d.sync_status()
     assert torch.equal(y.cpu(), y_ref.cpu())
+    plan.close()
+
+
+def test_noalloc_residual_and_rms_epilogues():
+    """The residual epilogue, and the RMS_norm + SiLU epilogue with the
+    output's two-frame history (next_cache_out after a carried
+    next_cache_in), against the planned call and the oracle."""
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    n, c, h, w = 1, 64, 20, 36
+    # residual: 2 frames
+    case = synth.conv_case(c, c, 2, h, w, seed_base=5)
+    x, wt, b = to_dev(synth.ndhwc(case["x"])), to_dev(case["w"]), to_dev(case["b"])
+    res = to_dev(synth.ndhwc(synth.normal((n, c, 2, h, w), 51)))
+    kw = dict(h=h, w=w, max_t=2, epi=cc3d.EPI_BIAS_RESIDUAL)
+    plan = cc3d.Plan(wt, b, **kw)
+    y_ref = torch.empty_like(res)
+    plan.forward(x, y_ref, residual=res)
+    y = torch.full_like(res, float("nan"))
+    st = cc3d.cc3d_forward_noalloc(_desc_for(kw, wt, b), _p(x), 2, None, _p(y), None, _p(res),
+                                   None, None, stream)
+    assert st == cc3d.OK, cc3d.cc3d_status_string(st)
+    cc3d.sync_status()
+    assert torch.equal(y.cpu(), y_ref.cpu())
+    ref = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], case["b"].double().numpy())
+    assert_close_bf16(ncthw_np(y), ref + ncthw_np(res), "noalloc residual vs oracle")
+    plan.close()
+    # RMS + SiLU: one-frame call carrying next_cache_in
+    case = synth.conv_case(c, c, 1, h, w, seed_base=6)
+    x, wt, b = to_dev(synth.ndhwc(case["x"])), to_dev(case["w"]), to_dev(case["b"])
+    g = to_dev(synth.uniform((c,), 0.5, 1.5, 52))
+    nc_in = to_dev(synth.ndhwc(synth.normal((n, c, 2, h, w), 53)))
+    kw = dict(h=h, w=w, max_t=1, epi=cc3d.EPI_BIAS_RMS_SILU)
+    plan = cc3d.Plan(wt, b, gamma=g, **kw)
+    y_ref = torch.empty((n, 1, h, w, c), dtype=torch.bfloat16, device="cuda")
+    nc_ref = torch.empty_like(nc_in)
+    plan.forward(x, y_ref, next_cache_in=nc_in, next_cache_out=nc_ref)
+    y = torch.full_like(y_ref, float("nan"))
+    nc = torch.full_like(nc_in, float("nan"))
+    st = cc3d.cc3d_forward_noalloc(_desc_for(kw, wt, b, g), _p(x), 1, None, _p(y), None, None,
+                                   _p(nc_in), _p(nc), stream)
+    assert st == cc3d.OK, cc3d.cc3d_status_string(st)
+    cc3d.sync_status()
+    assert torch.equal(y.cpu(), y_ref.cpu())
+    assert torch.equal(nc.cpu(), nc_ref.cpu())
+    assert torch.equal(nc[:, :1].cpu(), nc_in[:, 1:].cpu())
+    assert torch.equal(nc[:, 1:].cpu(), y.cpu())
+    conv = oracle.round_bf16_array(
+        oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], case["b"].double().numpy()))
+    ref = oracle.rms_norm(conv, synth.uniform((c,), 0.5, 1.5, 52).double().numpy(), silu=True)
+    assert_close_bf16(ncthw_np(y), ref, "noalloc rms vs oracle")
     plan.close()
 
 

@@ -30,18 +30,6 @@ namespace {
 
 std::atomic<uint64_t> g_launches{0};
 
-// Bound of every device-side wait, read once per process from
-// CC3D_WAIT_LIMIT_US (microseconds; default 2 s).
-unsigned long long wait_limit_ns() {
-  static unsigned long long v = [] {
-    const char *s = std::getenv("CC3D_WAIT_LIMIT_US");
-    unsigned long long us = s ? std::strtoull(s, nullptr, 10) : 0ull;
-    if (us == 0) us = 2000000ull;
-    return us * 1000ull;
-  }();
-  return v;
-}
-
 std::mutex g_mu;
 int *g_status_ptr[64] = {nullptr};
 
@@ -169,6 +157,96 @@ bool encode_store_map(CUtensorMap *m, const void *base, int c, int w, int h, int
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+// Bound of every device-side wait, read once per process from
+// CC3D_WAIT_LIMIT_US (microseconds; default 2 s).
+unsigned long long wait_limit_ns() {
+  static unsigned long long v = [] {
+    const char *s = std::getenv("CC3D_WAIT_LIMIT_US");
+    unsigned long long us = s ? std::strtoull(s, nullptr, 10) : 0ull;
+    if (us == 0) us = 2000000ull;
+    return us * 1000ull;
+  }();
+  return v;
+}
+
+cudaError_t run_umma_layer(const UmmaLayer &L, const UmmaCall &c, int *status,
+                           cudaStream_t stream, uint64_t *tiles_out) {
+  const UmmaConfig &cfg = L.cfg;
+  CUtensorMap mx, mc;
+  const int front = L.kt - 1;  // frames of the causal cache (0 for the stride-2 spatial conv)
+  const int tile_w = umma_tile_w() * cfg.sub;
+  // the kernel's spatial kernel: kh x kw, or 1 x 1 taps for stride 2
+  const int ks = L.s2 ? 1 : L.kh;
+  const int h_out = L.s2 ? L.h / 2 : L.h, w_out = L.s2 ? L.w / 2 : L.w;
+  const int t_out = (c.t - 1) / L.stride_t + 1;
+  // (a pair's CTA loads the halo of its own 8-column half)
+  const int box_w = umma_halo_box_w(cfg.kc, cfg.pair ? 1 : cfg.sub, ks);
+  const int box_h = umma_tile_h() + ks - 1;
+  const int box_c = umma_halo_box_c(cfg.kc);
+  if (!(L.s2 ? encode_act_map_s2(&mx, c.x, L.c_in, L.w, L.h, c.t, L.n, box_w, box_h, box_c)
+             : encode_act_map(&mx, c.x, L.c_in, L.w, L.h, c.t, L.n, box_w, box_h, box_c)))
+    return cudaErrorInvalidValue;
+  const bool has_cache = c.cache_in && front > 0;
+  if (has_cache) {
+    if (!encode_act_map(&mc, c.cache_in, L.c_in, L.w, L.h, front, L.n, box_w, box_h, box_c))
+      return cudaErrorInvalidValue;
+  } else {
+    mc = mx;
+  }
+  CUtensorMap msc = mx;  // the conv_shortcut's input: same boxes, c_sc channels
+  if (L.c_sc > 0 && !encode_act_map(&msc, c.x_sc, L.c_sc, L.w, L.h, c.t, L.n, box_w, box_h, box_c))
+    return cudaErrorInvalidValue;
+  UmmaArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.wimg = L.wimg;
+  a.bias = L.bias;
+  a.gamma = L.gamma;
+  a.beta = L.beta;
+  a.residual = static_cast<const __nv_bfloat16 *>(c.residual);
+  a.y = static_cast<__nv_bfloat16 *>(c.y);
+  a.status = status;
+  a.wait_limit_ns = wait_limit_ns();
+  a.n = L.n; a.t = t_out; a.h = h_out; a.w = w_out; a.c_in = L.c_in; a.c_out = L.c_out;
+  a.kt = L.s2 ? 9 : L.kt; a.kh = ks; a.kw = ks; a.pad_h = L.pad_h; a.pad_w = L.pad_w;
+  a.stride_t = L.stride_t;
+  a.s2 = L.s2;
+  a.vec32 = (reinterpret_cast<uintptr_t>(c.y) & 31u) == 0 ? 1 : 0;
+  a.b_resident = cfg.b_resident;
+  a.c_sc = L.c_sc;
+  a.n_cc_sc = L.n_cc_sc;
+  a.nt = cfg.nt; a.n_ntiles = cfg.n_ntiles;
+  a.sub = cfg.sub; a.nbuf = cfg.nbuf; a.g_taps = cfg.g_taps; a.pair = cfg.pair;
+  a.tiles_w = (w_out + tile_w - 1) / tile_w;
+  a.tiles_h = (h_out + umma_tile_h() - 1) / umma_tile_h();
+  a.na = cfg.na; a.nb = cfg.nb; a.tmem_cols = cfg.tmem_cols;
+  a.epi = L.epi;
+  a.has_cache = has_cache ? 1 : 0;
+  // the frame caches, written by the kernel's epilogue
+  a.x_in = static_cast<const __nv_bfloat16 *>(c.x);
+  a.t_in = c.t;
+  a.cache_frames = front;
+  a.cache_in = static_cast<const __nv_bfloat16 *>(has_cache ? c.cache_in : nullptr);
+  a.cache_out = front > 0 ? static_cast<__nv_bfloat16 *>(c.cache_out) : nullptr;
+  a.ncache_in = static_cast<const __nv_bfloat16 *>(c.ncache_in);
+  a.ncache_out = static_cast<__nv_bfloat16 *>(c.ncache_out);
+  a.nc_vec32 = (reinterpret_cast<uintptr_t>(c.ncache_out) & 31u) == 0 ? 1 : 0;
+  const uint64_t tiles = static_cast<uint64_t>(L.n) * t_out * a.tiles_h * a.tiles_w * a.n_ntiles;
+  uint64_t grid;
+  if (cfg.pair) {
+    // one pair per tile, at most as many pairs as fit at once
+    const uint64_t clusters = static_cast<uint64_t>(L.max_clusters);
+    grid = (tiles < clusters ? tiles : clusters) * 2;
+  } else {
+    const uint64_t slots = static_cast<uint64_t>(L.sm_count) * cfg.ctas_per_sm;
+    grid = tiles < slots ? tiles : slots;
+  }
+  *tiles_out = tiles;
+  const cudaError_t e = launch_conv_umma(mx, mc, cfg.pair ? *L.map_w : mx, msc, a, cfg.kc,
+                                         static_cast<unsigned>(grid), stream);
+  count_launch();
+  return e;
+}
+
 int *device_status_word() { return status_ptr(); }
 
 bool encode_activation_map(CUtensorMap *m, const void *base, int c, int w, int h, int t, int n,
@@ -199,16 +277,14 @@ struct cc3d_plan {
   cc3d_desc d;
   int variant;
   int device;
-  // UMMA
-  int kc, nt, n_ntiles, na, nb, tmem_cols, sm_count, ctas_per_sm, sub, nbuf, split, max_clusters;
-  int pair, b_resident;
-  int c_sc, n_cc_sc;  // the residual block's fused 1x1x1 conv_shortcut (0: none)
-  int s2;             // stride 2 in H and W (the downsample path's per-frame conv)
+  // UMMA: the layer as the shared launcher sees it
+  UmmaLayer layer;
   CUtensorMap map_w;  // pair: the weight image as 128-byte swizzled rows
   uint8_t *wimg;
+  int c_sc;           // the residual block's fused 1x1x1 conv_shortcut (0: none)
   // fp32 / thin
   void *wraw;
-  int kpad, thin_spec;
+  int kpad, thin_spec, nt, tmem_cols, sm_count, ctas_per_sm;
   float *bias, *gamma, *beta;
   cc3d_stats st;
   std::mutex mu;
@@ -392,7 +468,6 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
                        ? 1
                        : 0;
     p->nt = desc->c_out;
-    p->n_ntiles = 1;
     int cols = 32;
     while (cols < 2 * desc->c_out) cols *= 2;
     p->tmem_cols = cols;
@@ -428,63 +503,68 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
     e = umma_prepare();
     if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
     if (!status_ptr()) { s = CC3D_ERR_CUDA; goto fail; }
-    if (cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, p->device) !=
-        cudaSuccess)
-      p->sm_count = 148;
-    // Tile configuration (N split, sub-tiles, CTA pair, temporal split,
-    // pipeline depths): a function of (n, c_in, c_out, h, w, epilogue,
-    // max_t), never of a call's t, so a streamed sequence and a
-    // whole-sequence call of one plan run identical arithmetic.
     {
-      UmmaConfig cfg;
-      // (the largest call's output frames)
-      const int max_out = (desc->max_t - 1) / desc->stride_t + 1;
+      UmmaLayer &L = p->layer;
+      std::memset(&L, 0, sizeof L);
+      if (cudaDeviceGetAttribute(&L.sm_count, cudaDevAttrMultiProcessorCount, p->device) !=
+          cudaSuccess)
+        L.sm_count = 148;
+      L.n = desc->n; L.c_in = desc->c_in; L.c_out = desc->c_out; L.h = desc->h; L.w = desc->w;
+      L.kt = desc->kt; L.kh = desc->kh; L.kw = desc->kw;
+      L.pad_h = desc->pad_h; L.pad_w = desc->pad_w;
+      L.stride_t = desc->stride_t;
       // spatial stride 2 runs as nine 1x1 taps over the output frame
-      p->s2 = desc->stride_h == 2 ? 1 : 0;
-      const int kt_eff = p->s2 ? 9 : desc->kt, ks_eff = p->s2 ? 1 : desc->kh;
+      L.s2 = desc->stride_h == 2 ? 1 : 0;
+      L.epi = static_cast<int>(desc->epi);
+      // Tile configuration (N split, sub-tiles, CTA pair, weight grouping,
+      // pipeline depths): a function of (n, c_in, c_out, h, w, epilogue,
+      // max_t), never of a call's t.
+      UmmaConfig &cfg = L.cfg;
+      const int max_out = (desc->max_t - 1) / desc->stride_t + 1;  // largest call's frames
+      const int kt_eff = L.s2 ? 9 : desc->kt, ks_eff = L.s2 ? 1 : desc->kh;
       const int h_out = desc->h / desc->stride_h, w_out = desc->w / desc->stride_w;
       if (!choose_umma_config(desc->n, desc->c_in, desc->c_out, h_out, w_out, kt_eff, ks_eff,
-                              desc->epi == CC3D_EPI_BIAS_RMS_SILU, c_sc > 0, max_out,
-                              p->sm_count, &cfg)) {
+                              desc->epi == CC3D_EPI_BIAS_RMS_SILU, max_out, L.sm_count, &cfg)) {
         s = CC3D_ERR_UNSUPPORTED;
         goto fail;
       }
-      p->kc = cfg.kc; p->nt = cfg.nt; p->n_ntiles = cfg.n_ntiles; p->sub = cfg.sub;
-      p->nbuf = cfg.nbuf; p->na = cfg.na; p->nb = cfg.nb; p->tmem_cols = cfg.tmem_cols;
-      p->ctas_per_sm = cfg.ctas_per_sm; p->split = cfg.split; p->pair = cfg.pair;
-      p->b_resident = cfg.b_resident;
-      p->max_clusters = 0;
-      if (cfg.split > 1 || cfg.pair) {
-        p->max_clusters = umma_max_clusters(cfg, ks_eff);
-        if (p->max_clusters < 1) { s = CC3D_ERR_CUDA; goto fail; }
+      if (cfg.pair) {
+        L.max_clusters = umma_max_clusters(cfg, ks_eff);
+        if (L.max_clusters < 1) { s = CC3D_ERR_CUDA; goto fail; }
       }
-    }
-    p->st.tile_h = umma_tile_h();
-    p->st.tile_w = umma_tile_w() * p->sub;
-    p->st.n_tile = p->nt;
-    p->st.k_chunk = p->kc;
-    p->st.k_split = p->split;
-    p->st.mma_ctas = p->pair ? 2 : 1;
-    p->st.w_resident = p->b_resident;
-    // weight image: per N tile, the conv's taps * c_in / kc stages, then the
-    // shortcut's ceil(c_sc / kc) (its channels past c_sc zero)
-    p->c_sc = c_sc;
-    p->n_cc_sc = c_sc > 0 ? (c_sc + p->kc - 1) / p->kc : 0;
-    const int conv_stages = taps * (desc->c_in / p->kc);
-    const int stages = conv_stages + p->n_cc_sc;
-    const size_t bytes = sizeof(__nv_bfloat16) * desc->c_out * stages * p->kc;
-    if (cudaMalloc(&p->wimg, bytes) != cudaSuccess) { s = CC3D_ERR_OOM; goto fail; }
-    e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(desc->weight), p->wimg,
-                           desc->c_out, desc->c_in, taps, p->nt, p->kc, p->pair, stages, 0, 0);
-    if (e == cudaSuccess && c_sc > 0)
-      e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(w_sc), p->wimg, desc->c_out, c_sc,
-                             1, p->nt, p->kc, p->pair, stages, conv_stages, 0);
-    if (e == cudaSuccess) e = cudaDeviceSynchronize();
-    if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
-    if (p->pair && !encode_weight_map(&p->map_w, p->wimg,
-                                      static_cast<long long>(desc->c_out) * stages, p->nt / 2)) {
-      s = CC3D_ERR_CUDA;
-      goto fail;
+      p->st.tile_h = umma_tile_h();
+      p->st.tile_w = umma_tile_w() * cfg.sub;
+      p->st.n_tile = cfg.nt;
+      p->st.k_chunk = cfg.kc;
+      p->st.k_split = 1;
+      p->st.mma_ctas = cfg.pair ? 2 : 1;
+      p->st.w_resident = cfg.b_resident;
+      // weight image: per N tile, the conv's taps * c_in / kc stages, then the
+      // shortcut's ceil(c_sc / kc) (its channels past c_sc zero)
+      p->c_sc = c_sc;
+      L.c_sc = c_sc;
+      L.n_cc_sc = c_sc > 0 ? (c_sc + cfg.kc - 1) / cfg.kc : 0;
+      const int conv_stages = taps * (desc->c_in / cfg.kc);
+      const int stages = conv_stages + L.n_cc_sc;
+      const size_t bytes = sizeof(__nv_bfloat16) * desc->c_out * stages * cfg.kc;
+      if (cudaMalloc(&p->wimg, bytes) != cudaSuccess) { s = CC3D_ERR_OOM; goto fail; }
+      e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(desc->weight), p->wimg,
+                             desc->c_out, desc->c_in, taps, cfg.nt, cfg.kc, cfg.pair, stages, 0, 0);
+      if (e == cudaSuccess && c_sc > 0)
+        e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(w_sc), p->wimg, desc->c_out,
+                               c_sc, 1, cfg.nt, cfg.kc, cfg.pair, stages, conv_stages, 0);
+      if (e == cudaSuccess) e = cudaDeviceSynchronize();
+      if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
+      if (cfg.pair && !encode_weight_map(&p->map_w, p->wimg,
+                                         static_cast<long long>(desc->c_out) * stages, cfg.nt / 2)) {
+        s = CC3D_ERR_CUDA;
+        goto fail;
+      }
+      L.wimg = p->wimg;
+      L.map_w = &p->map_w;
+      L.bias = p->bias;
+      L.gamma = p->gamma;
+      L.beta = p->beta;
     }
   }
   *out = p;
@@ -620,65 +700,16 @@ static cc3d_status forward_impl(cc3d_plan *p, const void *x, int t, const void *
     e = launch_conv_thin(mx, mc, my_map, a, static_cast<unsigned>(tiles < slots ? tiles : slots),
                          stream);
   } else {
-    CUtensorMap mx, mc;
-    const int tile_w = umma_tile_w() * p->sub;
-    // the kernel's spatial kernel: kh x kw, or 1 x 1 taps for stride 2
-    const int ks = p->s2 ? 1 : d.kh;
-    const int h_out = d.h / d.stride_h, w_out = d.w / d.stride_w;
-    // (a pair's CTA loads the halo of its own 8-column half)
-    const int box_w = umma_halo_box_w(p->kc, p->pair ? 1 : p->sub, ks);
-    const int box_h = umma_tile_h() + ks - 1;
-    const int box_c = umma_halo_box_c(p->kc);
-    if (!(p->s2 ? encode_act_map_s2(&mx, x, d.c_in, d.w, d.h, t, d.n, box_w, box_h, box_c)
-                : encode_act_map(&mx, x, d.c_in, d.w, d.h, t, d.n, box_w, box_h, box_c)))
-      return reject(CC3D_ERR_CUDA);
-    if (cache_in && front > 0) {
-      if (!encode_act_map(&mc, cache_in, d.c_in, d.w, d.h, front, d.n, box_w, box_h, box_c))
-        return reject(CC3D_ERR_CUDA);
-    } else {
-      mc = mx;
-    }
-    CUtensorMap msc = mx;  // the conv_shortcut's input: same boxes, c_sc channels
-    if (p->c_sc > 0 && !encode_act_map(&msc, x_sc, p->c_sc, d.w, d.h, t, d.n, box_w, box_h, box_c))
-      return reject(CC3D_ERR_CUDA);
-    UmmaArgs a;
-    a.wimg = p->wimg;
-    a.bias = p->bias;
-    a.gamma = p->gamma;
-    a.beta = p->beta;
-    a.residual = static_cast<const __nv_bfloat16 *>(residual);
-    a.y = static_cast<__nv_bfloat16 *>(y);
-    a.status = status;
-    a.wait_limit_ns = wait_limit_ns();
-    a.n = d.n; a.t = t_out; a.h = h_out; a.w = w_out; a.c_in = d.c_in; a.c_out = d.c_out;
-    a.kt = p->s2 ? 9 : d.kt; a.kh = ks; a.kw = ks; a.pad_h = d.pad_h; a.pad_w = d.pad_w;
-    a.stride_t = d.stride_t;
-    a.s2 = p->s2;
-    a.vec32 = (reinterpret_cast<uintptr_t>(y) & 31u) == 0 ? 1 : 0;
-    a.b_resident = p->b_resident;
-    a.c_sc = p->c_sc;
-    a.n_cc_sc = p->n_cc_sc;
-    a.nt = p->nt; a.n_ntiles = p->n_ntiles;
-    a.sub = p->sub; a.nbuf = p->nbuf; a.split = p->split; a.pair = p->pair;
-    a.tiles_w = (w_out + tile_w - 1) / tile_w;
-    a.tiles_h = (h_out + umma_tile_h() - 1) / umma_tile_h();
-    a.na = p->na; a.nb = p->nb; a.tmem_cols = p->tmem_cols;
-    a.epi = static_cast<int>(d.epi);
-    a.has_cache = (cache_in && front > 0) ? 1 : 0;
-    tiles = static_cast<uint64_t>(d.n) * t_out * a.tiles_h * a.tiles_w * a.n_ntiles;
-    uint64_t grid;
-    if (p->split > 1 || p->pair) {
-      // one cluster (of `split` CTAs, or a pair) per tile, at most as many as
-      // fit at once
-      const uint64_t clusters = static_cast<uint64_t>(p->max_clusters);
-      grid = (tiles < clusters ? tiles : clusters) * (p->pair ? 2 : p->split);
-    } else {
-      const uint64_t slots = static_cast<uint64_t>(p->sm_count) * p->ctas_per_sm;
-      grid = tiles < slots ? tiles : slots;
-    }
-    e = launch_conv_umma(mx, mc, p->pair ? p->map_w : mx, msc, a, p->kc,
-                         static_cast<unsigned>(grid), stream);
-    count_launch();
+    UmmaCall c;
+    c.x = x; c.t = t; c.cache_in = cache_in; c.y = y; c.cache_out = cache_out;
+    c.residual = residual; c.ncache_in = next_cache_in; c.ncache_out = next_cache_out;
+    c.x_sc = x_sc;
+    e = run_umma_layer(p->layer, c, status, stream, &tiles);
+  }
+  // (the tensor-core conv writes both caches itself)
+  if (p->variant == CC3D_VARIANT_UMMA) {
+    cache_out = nullptr;
+    next_cache_out = nullptr;
   }
   if (e == cudaSuccess && cache_out && front > 0)
     e = launch_cache_update(cache_in, x, cache_out, d.n, t, front, in_frame, stream);
@@ -712,11 +743,11 @@ cc3d_status rmsnorm_silu(const void *x, const float *gamma, const float *beta, i
       overlaps(cache_out, cb, x, xb))
     return CC3D_ERR_ALIAS;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
-  const long long voxels = static_cast<long long>(n) * t * h * w;
-  cudaError_t e = launch_rmsnorm_silu(static_cast<const __nv_bfloat16 *>(x), gamma, beta, voxels,
-                                      c, static_cast<__nv_bfloat16 *>(y), stream);
-  if (e == cudaSuccess && cache_out)
-    e = launch_cache_update(cache_in, y, cache_out, n, t, 2, frame, stream);
+  // one kernel: the normalised activation and its 2-frame cache
+  const cudaError_t e = launch_rmsnorm_silu(
+      static_cast<const __nv_bfloat16 *>(x), gamma, beta, n, t, static_cast<long long>(h) * w, c,
+      static_cast<__nv_bfloat16 *>(y), static_cast<const __nv_bfloat16 *>(cache_in),
+      static_cast<__nv_bfloat16 *>(cache_out), stream);
   return from_cuda(e);
 }
 

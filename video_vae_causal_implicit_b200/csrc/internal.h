@@ -30,8 +30,8 @@ struct UmmaArgs {
   int has_cache;
   int sub;                        // MMA sub-tiles (8 x 16 px) per CTA tile, side by side: 1 or 2
   int nbuf;                       // accumulator buffers in tensor memory: 1 or 2
-  int split;                      // 1, or kt: CTAs of a cluster that share a tile, one
-                                  // temporal tap each, reduced in the last one
+  int g_taps;                     // weight stages (spatial taps) per weight slot: 1, or kw
+                                  // (one kernel row)
   int pair;                       // 1: a cluster of 2 CTAs runs 2-SM MMAs on a 16 x 16 px
                                   // tile (sub is then 2: the tile width in MMA tiles)
   int vec32;                      // 1: y and residual are 32-byte aligned (256-bit stores)
@@ -44,28 +44,39 @@ struct UmmaArgs {
                                   // per frame): kt = 9 spatial taps of a 1x1 kernel, each
                                   // read through a map that walks every other pixel; h, w
                                   // are the output frame's
+  // Frame caches written by the epilogue (null: not written).
+  //   cache_out [n][cache_frames][h][w][c_in] = the last cache_frames frames of
+  //   concat(cache_in or zeros, x_in), x_in having t_in frames;
+  //   ncache_out [n][2][h][w][c_out] = the last two frames of concat(ncache_in
+  //   or zeros, y) (the RMS epilogue's output history).
+  const __nv_bfloat16 *x_in;
+  const __nv_bfloat16 *cache_in;
+  __nv_bfloat16 *cache_out;
+  int cache_frames, t_in;
+  const __nv_bfloat16 *ncache_in;
+  __nv_bfloat16 *ncache_out;
+  int nc_vec32;                   // 1: ncache_out is 32-byte aligned (256-bit stores)
 };
 
 // Tile configuration of the UMMA conv for a plan (chosen from n, c_in, c_out,
 // h, w, the epilogue and the plan's max_t -- never from a call's t).
 struct UmmaConfig {
-  int kc, nt, n_ntiles, sub, nbuf, split, pair, na, nb, tmem_cols, ctas_per_sm;
+  int kc, nt, n_ntiles, sub, nbuf, g_taps, pair, na, nb, tmem_cols, ctas_per_sm;
   int params;      // epilogue parameters staged in shared memory (floats)
   int b_resident;  // every weight stage resident in shared memory (nb of them)
 };
-// shortcut: the plan carries a fused conv_shortcut (no temporal split).
 bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
-                        bool shortcut, int max_t, int sm_count, UmmaConfig *cfg);
-// Clusters of cfg.split CTAs that can be resident at once (split > 1), for
-// sizing the grid; 0 when the query fails.
+                        int max_t, int sm_count, UmmaConfig *cfg);
+// CTA pairs that can be resident at once (cfg.pair), for sizing the grid;
+// 0 when the query fails.
 int umma_max_clusters(const UmmaConfig &cfg, int ks);
 
-size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb, int sub, int split,
+size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb, int sub, int g_taps,
                        int pair, int params);
 cudaError_t umma_prepare();
 // Dynamic shared memory a launch requests (with the one-CTA-per-SM rule).
 size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols, int sub,
-                        int split, int pair, int params);
+                        int g_taps, int pair, int params);
 int umma_tile_w();
 // TMA box of the A halo: columns (padded for the 128-byte swizzle) and
 // channels (64: swizzled pixel rows; 8: no-swizzle slabs).
@@ -129,9 +140,49 @@ cudaError_t launch_conv_fp32(const Fp32Args &a, cudaStream_t stream);
 cudaError_t launch_cache_update(const void *cache_in, const void *src, void *cache_out, int n,
                                 int t, int frames, size_t frame_bytes, cudaStream_t stream);
 
-// RMS_norm + SiLU over channels, bf16 in/out.
+// RMS_norm + SiLU over channels of n x t frames of hw pixels, bf16 in/out;
+// cache_out (null: not written) = the last two frames of concat(cache_in or
+// zeros, y), written by the same kernel.
 cudaError_t launch_rmsnorm_silu(const __nv_bfloat16 *x, const float *gamma, const float *beta,
-                                long long voxels, int c, __nv_bfloat16 *y, cudaStream_t stream);
+                                int n, int t, long long hw, int c, __nv_bfloat16 *y,
+                                const __nv_bfloat16 *cache_in, __nv_bfloat16 *cache_out,
+                                cudaStream_t stream);
+
+// One tensor-core conv layer as planned: its tile configuration, geometry
+// and device-resident operands (the plan's, or the no-allocation scratch).
+struct UmmaLayer {
+  UmmaConfig cfg;
+  int n, c_in, c_out, h, w;        // input frame geometry
+  int kt, kh, kw, pad_h, pad_w;    // kernel as declared (kt, kh, kw of the descriptor)
+  int stride_t, s2;                // temporal stride; s2: stride 2 in H and W
+  int epi;                         // 0 bias, 1 bias + residual, 2 bias + RMS + SiLU
+  int c_sc, n_cc_sc;               // fused 1x1x1 conv_shortcut (0: none)
+  int sm_count, max_clusters;      // grid sizing (max_clusters: CTA pairs)
+  const uint8_t *wimg;             // re-tiled weights
+  const CUtensorMap *map_w;        // the weights as 128-byte swizzled rows (pairs)
+  const float *bias, *gamma, *beta;
+};
+// The pointers of one call (device; null where absent).  t: input frames.
+struct UmmaCall {
+  const void *x;
+  int t;
+  const void *cache_in;
+  void *y;
+  void *cache_out;
+  const void *residual;
+  const void *ncache_in;
+  void *ncache_out;
+  const void *x_sc;
+};
+// Encodes the call's tensor maps and launches the conv (one kernel, which
+// also writes cache_out and ncache_out).  Arguments are assumed validated.
+// *tiles: output tiles of the launch.
+cudaError_t run_umma_layer(const UmmaLayer &L, const UmmaCall &c, int *status,
+                           cudaStream_t stream, uint64_t *tiles);
+
+// Bound of every device-side wait in nanoseconds (CC3D_WAIT_LIMIT_US, else
+// 2 s), read once per process.
+unsigned long long wait_limit_ns();
 
 // Host-side launch counter (all kernels of this library).
 void count_launch();

@@ -131,20 +131,51 @@ __global__ void copy_frames2_kernel(const uint8_t *__restrict__ cache_in,
   }
 }
 
+// The frame cache of an RMS_norm + SiLU pass over t frames of hw pixels:
+// cache_out [n][2][hw][c] = the last two frames of concat(cache_in or
+// zeros, y).  The thread that writes a voxel's output (chunk `g` of 8
+// channels) also writes it to the cache when its frame is one of the last
+// two, and with a single frame copies cache_in's second frame into the
+// first cache frame.
+struct RmsCache {
+  const __nv_bfloat16 *in;  // [n][2][hw][c] or null (zeros)
+  __nv_bfloat16 *out;       // [n][2][hw][c] or null (not written)
+  long long hw;             // pixels per frame
+  int t;                    // frames of the call
+};
+
+__device__ __forceinline__ void rms_cache_store(const RmsCache &k, long long v, int c, int g,
+                                                const uint4 &w) {
+  const long long per_img = k.hw * k.t;
+  const long long img = v / per_img, rem = v - img * per_img;
+  const int tt = static_cast<int>(rem / k.hw);
+  const long long pix = rem - static_cast<long long>(tt) * k.hw;
+  const int f = tt - (k.t - 2);  // frame of the cache this output lands in
+  if (f < 0) return;
+  __stcs(reinterpret_cast<uint4 *>(k.out + ((img * 2 + f) * k.hw + pix) * c) + g, w);
+  if (k.t == 1) {
+    const uint4 prev = k.in ? __ldcs(reinterpret_cast<const uint4 *>(
+                                         k.in + ((img * 2 + 1) * k.hw + pix) * c) + g)
+                            : make_uint4(0, 0, 0, 0);
+    __stcs(reinterpret_cast<uint4 *>(k.out + (img * 2 * k.hw + pix) * c) + g, prev);
+  }
+}
+
 // Lane-mapped RMS_norm + SiLU for channel counts whose 8-channel groups
 // split evenly over a power-of-two number of lanes: LPV lanes share a voxel,
 // each lane owning GPL groups (GPL = c / 8 / LPV, e.g. C = 192: 8 lanes x 3
 // groups, four voxels per warp).  A warp's loads cover 32 * GPL consecutive
 // 16-byte chunks (fully coalesced, every lane busy); UNR warp passes are
-// loaded before any is used.  The sum of squares is reduced with a fixed
+// loaded before any is used, and four CTAs per SM keep enough bytes in
+// flight to stream at HBM speed.  The sum of squares is reduced with a fixed
 // xor butterfly over the LPV lanes, so the result does not depend on
 // scheduling.
 template <int GPL, int UNR>
-__global__ void __launch_bounds__(256, 2)
+__global__ void __launch_bounds__(256, 4)
     rmsnorm_silu_lanes_kernel(const __nv_bfloat16 *__restrict__ x,
                               const float *__restrict__ gamma, const float *__restrict__ beta,
                               long long voxels, int c, int lpv,
-                              __nv_bfloat16 *__restrict__ y) {
+                              __nv_bfloat16 *__restrict__ y, RmsCache cache) {
   const int lane = threadIdx.x % 32;
   const int vpw = 32 / lpv;                 // voxels per warp pass
   const int sub = lane % lpv, vloc = lane / lpv;
@@ -199,6 +230,7 @@ __global__ void __launch_bounds__(256, 2)
         w.z = pack2(o[4], o[5]);
         w.w = pack2(o[6], o[7]);
         __stcs(reinterpret_cast<uint4 *>(y + v * c) + g, w);
+        if (cache.out) rms_cache_store(cache, v, c, g, w);
       }
     }
     (void)groups;
@@ -215,7 +247,7 @@ template <int CPT>
 __global__ void __launch_bounds__(256)
     rmsnorm_silu_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ gamma,
                         const float *__restrict__ beta, long long voxels, int c,
-                        __nv_bfloat16 *__restrict__ y) {
+                        __nv_bfloat16 *__restrict__ y, RmsCache cache) {
   __shared__ float partial[256 * CPT];
   __shared__ float inv_s[256 * CPT];
   const int groups = c / 8;
@@ -275,6 +307,7 @@ __global__ void __launch_bounds__(256)
         w.z = pack2(o[4], o[5]);
         w.w = pack2(o[6], o[7]);
         __stcs(dst + idx, w);
+        if (cache.out) rms_cache_store(cache, v0 + v, c, g, w);
       }
     }
     __syncthreads();  // partial / inv_s are rewritten by the next pass
@@ -374,9 +407,17 @@ cudaError_t launch_cache_update(const void *cache_in, const void *src, void *cac
 }
 
 cudaError_t launch_rmsnorm_silu(const __nv_bfloat16 *x, const float *gamma, const float *beta,
-                                long long voxels, int c, __nv_bfloat16 *y, cudaStream_t stream) {
+                                int n, int t, long long hw, int c, __nv_bfloat16 *y,
+                                const __nv_bfloat16 *cache_in, __nv_bfloat16 *cache_out,
+                                cudaStream_t stream) {
   const int groups = c / 8;
-  if (groups < 1) return cudaErrorInvalidValue;
+  if (groups < 1 || n < 1 || t < 1 || hw < 1) return cudaErrorInvalidValue;
+  const long long voxels = static_cast<long long>(n) * t * hw;
+  RmsCache cache;
+  cache.in = cache_in;
+  cache.out = cache_out;
+  cache.hw = hw;
+  cache.t = t;
   // lanes per voxel: the largest power of two (<= 32) dividing the groups
   int lpv = 1;
   while (lpv < 32 && groups % (lpv * 2) == 0) lpv *= 2;
@@ -386,14 +427,14 @@ cudaError_t launch_rmsnorm_silu(const __nv_bfloat16 *x, const float *gamma, cons
     const long long per_warp = static_cast<long long>(32 / lpv) * kUnr;
     long long warps = (voxels + per_warp - 1) / per_warp;
     long long g = (warps * 32 + 255) / 256;
-    if (g > 148LL * 8) g = 148LL * 8;
+    if (g > 148LL * 16) g = 148LL * 16;
     if (g < 1) g = 1;
     const int grid = static_cast<int>(g);
     switch (gpl) {
-      case 1: rmsnorm_silu_lanes_kernel<1, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y); break;
-      case 2: rmsnorm_silu_lanes_kernel<2, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y); break;
-      case 3: rmsnorm_silu_lanes_kernel<3, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y); break;
-      default: rmsnorm_silu_lanes_kernel<4, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y); break;
+      case 1: rmsnorm_silu_lanes_kernel<1, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache); break;
+      case 2: rmsnorm_silu_lanes_kernel<2, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache); break;
+      case 3: rmsnorm_silu_lanes_kernel<3, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache); break;
+      default: rmsnorm_silu_lanes_kernel<4, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache); break;
     }
   } else {
     constexpr int kCpt = 12;  // 16-byte chunks per thread and pass
@@ -403,7 +444,7 @@ cudaError_t launch_rmsnorm_silu(const __nv_bfloat16 *x, const float *gamma, cons
     if (g > 148LL * 8) g = 148LL * 8;
     if (g < 1) g = 1;
     rmsnorm_silu_kernel<kCpt><<<static_cast<int>(g), 256, 0, stream>>>(x, gamma, beta, voxels,
-                                                                       c, y);
+                                                                       c, y, cache);
   }
   count_launch();
   return cudaGetLastError();

@@ -23,6 +23,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 
 #include "cc3d.h"
@@ -135,14 +136,17 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
 
   // ---- tiles: the same choice cc3d_plan_create makes --------------------------------
-  UmmaConfig cfg;
+  UmmaLayer L;
+  std::memset(&L, 0, sizeof L);
   if (!choose_umma_config(d->n, d->c_in, d->c_out, d->h, d->w, d->kt, d->kh,
-                          d->epi == CC3D_EPI_BIAS_RMS_SILU, false,
-                          (d->max_t - 1) / d->stride_t + 1, n_sm, &cfg))
+                          d->epi == CC3D_EPI_BIAS_RMS_SILU, (d->max_t - 1) / d->stride_t + 1, n_sm,
+                          &L.cfg))
     return CC3D_ERR_UNSUPPORTED;
-  const bool clustered = cfg.split > 1 || cfg.pair;
-  const int max_clusters = clustered ? umma_max_clusters(cfg, d->kh) : 0;
-  if (clustered && max_clusters < 1) return CC3D_ERR_CUDA;
+  const UmmaConfig &cfg = L.cfg;
+  if (cfg.pair) {
+    L.max_clusters = umma_max_clusters(cfg, d->kh);
+    if (L.max_clusters < 1) return CC3D_ERR_CUDA;
+  }
   const int kc = cfg.kc, nt = cfg.nt;
 
   // ---- scratch: re-tiled weights (every call), zero bias when none is given --------
@@ -154,68 +158,29 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   if (e == cudaSuccess && !d->bias)
     e = cudaMemsetAsync(zero_bias, 0, sizeof(float) * d->c_out, stream);
   if (e != cudaSuccess) return CC3D_ERR_CUDA;
-
-  // ---- the conv -----------------------------------------------------------------------------
-  CUtensorMap mx, mc, mw;
-  const int tile_w = umma_tile_w() * cfg.sub;
-  const int box_w = umma_halo_box_w(kc, cfg.pair ? 1 : cfg.sub, d->kw);
-  const int box_h = umma_tile_h() + d->kh - 1;
-  const int box_c = umma_halo_box_c(kc);
-  if (!encode_activation_map(&mx, x, d->c_in, d->w, d->h, t, d->n, box_w, box_h, box_c))
+  CUtensorMap mw;
+  if (cfg.pair && !encode_weight_map(&mw, wimg,
+                                     static_cast<long long>(d->c_out) * taps * (d->c_in / 64),
+                                     nt / 2))
     return CC3D_ERR_CUDA;
-  const bool has_cache = cache_in && front > 0;
-  if (has_cache) {
-    if (!encode_activation_map(&mc, cache_in, d->c_in, d->w, d->h, front, d->n, box_w, box_h,
-                               box_c))
-      return CC3D_ERR_CUDA;
-  } else {
-    mc = mx;
-  }
-  if (cfg.pair) {
-    if (!encode_weight_map(&mw, wimg, static_cast<long long>(d->c_out) * taps * (d->c_in / 64),
-                           nt / 2))
-      return CC3D_ERR_CUDA;
-  } else {
-    mw = mx;
-  }
-  UmmaArgs a;
-  a.wimg = wimg;
-  a.bias = d->bias ? d->bias : zero_bias;
-  a.gamma = d->gamma;
-  a.beta = d->beta;
-  a.residual = static_cast<const __nv_bfloat16 *>(residual);
-  a.y = static_cast<__nv_bfloat16 *>(y);
-  a.status = status;
-  a.wait_limit_ns = 2000ull * 1000000ull;
-  a.n = d->n; a.t = t_out; a.stride_t = d->stride_t;
-  a.vec32 = (reinterpret_cast<uintptr_t>(y) & 31u) == 0 ? 1 : 0;
-  a.b_resident = cfg.b_resident;
-  a.c_sc = 0;
-  a.s2 = 0;
-  a.n_cc_sc = 0;
-  a.h = d->h; a.w = d->w; a.c_in = d->c_in; a.c_out = d->c_out;
-  a.kt = d->kt; a.kh = d->kh; a.kw = d->kw; a.pad_h = d->pad_h; a.pad_w = d->pad_w;
-  a.nt = nt; a.n_ntiles = cfg.n_ntiles;
-  a.sub = cfg.sub; a.nbuf = cfg.nbuf; a.split = cfg.split; a.pair = cfg.pair;
-  a.tiles_w = (d->w + tile_w - 1) / tile_w;
-  a.tiles_h = (d->h + umma_tile_h() - 1) / umma_tile_h();
-  a.na = cfg.na; a.nb = cfg.nb; a.tmem_cols = cfg.tmem_cols;
-  a.epi = static_cast<int>(d->epi);
-  a.has_cache = has_cache ? 1 : 0;
-  const uint64_t tiles = uint64_t(d->n) * t_out * a.tiles_h * a.tiles_w * a.n_ntiles;
-  uint64_t grid;
-  if (clustered) {
-    grid = (tiles < uint64_t(max_clusters) ? tiles : uint64_t(max_clusters)) *
-           (cfg.pair ? 2 : cfg.split);
-  } else {
-    const uint64_t slots = uint64_t(n_sm) * cfg.ctas_per_sm;
-    grid = tiles < slots ? tiles : slots;
-  }
-  e = launch_conv_umma(mx, mc, mw, mx, a, kc, static_cast<unsigned>(grid), stream);
-  count_launch();
-  if (e == cudaSuccess && cache_out && front > 0)
-    e = launch_cache_update(cache_in, x, cache_out, d->n, t, front, in_frame, stream);
-  if (e == cudaSuccess && next_cache_out)
-    e = launch_cache_update(next_cache_in, y, next_cache_out, d->n, t_out, 2, out_frame, stream);
+
+  // ---- the conv (one kernel, which also writes cache_out and next_cache_out) ---------
+  L.n = d->n; L.c_in = d->c_in; L.c_out = d->c_out; L.h = d->h; L.w = d->w;
+  L.kt = d->kt; L.kh = d->kh; L.kw = d->kw; L.pad_h = d->pad_h; L.pad_w = d->pad_w;
+  L.stride_t = d->stride_t;
+  L.s2 = 0;
+  L.epi = static_cast<int>(d->epi);
+  L.sm_count = n_sm;
+  L.wimg = wimg;
+  L.map_w = &mw;
+  L.bias = d->bias ? d->bias : zero_bias;
+  L.gamma = d->gamma;
+  L.beta = d->beta;
+  UmmaCall c;
+  c.x = x; c.t = t; c.cache_in = cache_in; c.y = y; c.cache_out = cache_out;
+  c.residual = residual; c.ncache_in = next_cache_in; c.ncache_out = next_cache_out;
+  c.x_sc = nullptr;
+  uint64_t tiles = 0;
+  e = run_umma_layer(L, c, status, stream, &tiles);
   return e == cudaSuccess ? CC3D_OK : CC3D_ERR_CUDA;
 }
