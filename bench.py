@@ -1,6 +1,6 @@
 """Benchmark of the causal Conv3D hot path (libcc3d.so) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cc3d|reference] [--sweep]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cc3d|reference] [--sweep|--no-sweep]
 
 Workload (one "step"): the decoder latent-resolution causal conv,
 bf16, C_in = C_out = 384 on x[1, 384, 5, 30, 52], 3x3x3, run once over the
@@ -12,13 +12,14 @@ every timed step and the flush is outside the timed events.
 
 The same JSON line carries the residual block (x[1, 192, 9, 240, 416]:
 RMS_norm+SiLU -> conv -> RMS_norm+SiLU (fused) -> conv + x (fused)) as
-``resblock`` with its latency, and with ``--sweep`` the encoder convs
-(3 -> 96, 96 -> 96 at 17 x 480 x 832), the downsample path's time_conv
-(kernel (3, 1, 1), stride 2 in time, at 192 and 384 channels) and its
-per-frame 3x3 stride-2 conv (96 channels, 480 x 832 -> 240 x 416), the
-encoder's channel-changing residual blocks (96 -> 192, 192 -> 384) and a
-384-channel block, and the streaming channel/resolution sweep (21
-one-frame chunks, CUDA-graph captured).
+``resblock`` with its latency, and as ``sweep`` the encoder convs (3 -> 96,
+96 -> 96 at 17 x 480 x 832), the downsample path's time_conv (kernel
+(3, 1, 1), stride 2 in time, at 192 and 384 channels) and its per-frame
+3x3 stride-2 conv (96 channels, 480 x 832 -> 240 x 416), and the
+384-channel rows of the streaming channel/resolution sweep (21 one-frame
+chunks, CUDA-graph captured).  ``--sweep`` adds the sweep's 96- and
+192-channel rows and the encoder's residual blocks (96 -> 192, 192 -> 384
+and a 384-channel one); ``--no-sweep`` drops the sweep.
 
 Multi-GPU: the path runs as independent replicas (one process per GPU, no
 data-path collective); ``value`` is the FLOP all ranks processed divided by
@@ -186,7 +187,10 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cc3d", choices=["cc3d", "reference"])
-    ap.add_argument("--sweep", action="store_true", help="also time configs 3 and 5")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every sweep row (C = 96 and 192 of config 5, the encoder blocks) "
+                         "besides the default ones")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the sweep rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -286,9 +290,10 @@ def main():
     plan_stats = plan.stats()
 
     # For context (not the timed step): the same layer planned for one-frame
-    # calls only (max_t = 1), which takes the temporal split; its 5 chunks
-    # as one graph.  Its outputs are not bit-identical to the whole-sequence
-    # plan's, so the step above uses one plan for both.
+    # calls only (max_t = 1); its 5 chunks as one graph.  Whatever tile shape
+    # that plan picks, every output sums its taps in one accumulator in the
+    # same order, so its bytes equal the whole-sequence plan's (the tests
+    # check it).
     plan_s = cc3d.Plan(case["w"].to(dev), case["b"].to(dev), h=H, w=W, max_t=1)
     ys_s = [torch.empty_like(ys[0]) for _ in range(T)]
     smarks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(T + 1)]
@@ -315,7 +320,7 @@ def main():
             s_chunks.extend(smarks[i].elapsed_time(smarks[i + 1]) for i in range(T))
     cc3d.sync_status()
     stream_plan_ms = statistics.mean(s_chunks)
-    stream_plan_split = plan_s.stats().k_split
+    stream_plan_stats = plan_s.stats()
     del sgraph
     plan_s.close()
     ms_local = sum(step_ms) / len(step_ms)
@@ -330,6 +335,13 @@ def main():
     traffic_avg = None
     if NCU_TRAFFIC["whole"] is not None and NCU_TRAFFIC["chunk"] is not None:
         traffic_avg = (NCU_TRAFFIC["whole"] + T * NCU_TRAFFIC["chunk"]) / (T + 1)
+    # FLOP the MMAs execute: a tap that reads a causal zero frame of a call
+    # without a cache is skipped (output frame t of the whole sequence runs
+    # min(t + 1, 3) of its 3 temporal taps; the first chunk, which has no
+    # cache, runs 1 of 3; the later chunks multiply their cache frames)
+    exec_whole = flop_whole * sum(min(t + 1, 3) for t in range(T)) / (3 * T)
+    exec_step = exec_whole + flop_chunk * (1 / 3 + (T - 1))
+    executed = (exec_step / (T + 1)) / (avg_launch_ms * 1e-3) / 1e12
 
     # --- end to end through the public API with host buffers ---
     x_host = x.cpu().pin_memory()
@@ -422,7 +434,8 @@ def main():
     del conv1, conv2, a0, a1
     del blk, xb, yb
 
-    sweep = run_sweep(args, dev, stream, peaks, flush_l2) if args.sweep else None
+    sweep = None if args.no_sweep else run_sweep(args, dev, stream, peaks, flush_l2,
+                                                  full=args.sweep)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -450,6 +463,12 @@ def main():
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["bf16_tflops"], "traffic": traffic_avg,
                          "kernel": "conv_umma_kernel, average over the 6 launches of a step",
+                         "executed_tflops": executed,
+                         "executed_frac": executed / peaks["bf16_tflops"],
+                         "executed_note": "FLOP of the MMAs run: the taps that read causal zero "
+                                          "frames of a call without a cache are skipped "
+                                          f"({exec_step / 1e9:.1f} of {flop_step / 1e9:.1f} "
+                                          "GFLOP per step)",
                          "peak_basis": "burst bf16 (" + peaks["source"] + ")",
                          "per_launch": {
                              "whole_sequence": {"ms": whole_ms, "gflop": flop_whole / 1e9,
@@ -466,9 +485,11 @@ def main():
                              "one_frame_chunk_streaming_plan": {
                                  "ms": stream_plan_ms, "tflops": flop_chunk / stream_plan_ms / 1e9,
                                  "frac": flop_chunk / stream_plan_ms / 1e9 / peaks["bf16_tflops"],
-                                 "k_split": stream_plan_split,
-                                 "note": "the layer planned for one-frame calls (max_t = 1): "
-                                         "temporal split; context only, not in the timed step"}}},
+                                 "n_tile": stream_plan_stats.n_tile,
+                                 "mma_ctas": stream_plan_stats.mma_ctas,
+                                 "note": "the layer planned for one-frame calls (max_t = 1); "
+                                         "same bytes as the step's plan; context only, not in "
+                                         "the timed step"}}},
             "resblock": resblock,
             "e2e": e2e,
             "gpu_launches": launches,
@@ -482,8 +503,10 @@ def main():
     return 0
 
 
-def run_sweep(args, dev, stream, peaks, flush_l2):
-    """Configs 3 (encoder full-res convs) and 5 (streaming sweep)."""
+def run_sweep(args, dev, stream, peaks, flush_l2, full=False):
+    """Config 3 (encoder full-res convs), the downsample path's convs and the
+    384-channel rows of config 5 (streaming sweep); with `full` also config
+    5's 96- and 192-channel rows and the encoder's residual blocks."""
     import torch
 
     from video_vae_causal_implicit_b200 import cc3d, synth
@@ -567,8 +590,8 @@ def run_sweep(args, dev, stream, peaks, flush_l2):
     # the encoder's other residual blocks (§8(f) NEXT-2): the two that change
     # the channel count (the 1x1x1 conv_shortcut fused into conv2) and a
     # 384-channel one (RMS_norm after conv1 in its own pass), whole sequence
-    for (ci, co, T, H, W) in ((96, 192, 17, 240, 416), (192, 384, 9, 120, 208),
-                              (384, 384, 5, 60, 104)):
+    for (ci, co, T, H, W) in (((96, 192, 17, 240, 416), (192, 384, 9, 120, 208),
+                               (384, 384, 5, 60, 104)) if full else ()):
         xb = torch.randn((1, T, H, W, ci), generator=g, device=dev).to(torch.bfloat16)
         wts = dict(w1=synth.kaiming_uniform(co, ci, (3, 3, 3), 11),
                    b1=synth.uniform((co,), -0.1, 0.1, 12), g1=synth.uniform((ci,), 0.5, 1.5, 13),
@@ -587,7 +610,7 @@ def run_sweep(args, dev, stream, peaks, flush_l2):
             "ms": ms, "tflops": fl / ms / 1e9, "frac": fl / ms / 1e9 / peaks["bf16_tflops"]}
         del blk, xb, yb
     # config 5: C x resolution, 21 one-frame chunks, graph-captured
-    for cc in (96, 192, 384):
+    for cc in ((96, 192, 384) if full else (384,)):
         for (H, W) in ((90, 160), (180, 320), (360, 640)):
             T = 21
             x5 = torch.randn((1, T, H, W, cc), generator=g, device=dev).to(torch.bfloat16)

@@ -83,10 +83,14 @@ typedef enum { CC3D_BF16 = 0, CC3D_FP32 = 1 } cc3d_dtype;
 typedef enum {
   CC3D_EPI_BIAS = 0,          /* y = conv + b                                  */
   CC3D_EPI_BIAS_RESIDUAL = 1, /* y = conv + b + residual                       */
-  CC3D_EPI_BIAS_RMS_SILU = 2  /* y = SiLU(RMS(h; gamma) (+ beta)), h = conv + b
+  CC3D_EPI_BIAS_RMS_SILU = 2, /* y = SiLU(RMS(h; gamma) (+ beta)), h = conv + b
                                  rounded to bf16 first (the block's conv1
-                                 output is a bf16 activation); needs
-                                 c_out <= 256 so one CTA owns a row          */
+                                 output is a bf16 activation); one CTA owns
+                                 each whole row: c_out <= 256, or up to 512
+                                 in steps of 32 (two MMAs per K step)      */
+  CC3D_EPI_BIAS_RMS = 3       /* y = RMS(h; gamma) (+ beta), the same without
+                                 SiLU: the WanRMS_norm after the downsample
+                                 path's convs (§10.5)                        */
 } cc3d_epilogue;
 
 /* Kernel that served a call (the plan's route counters). */
@@ -123,7 +127,7 @@ typedef struct {
                           dtype; copied (and re-tiled) at create             */
   const float *bias;   /* device [c_out] fp32, nullable (= 0); copied        */
   cc3d_epilogue epi;
-  const float *gamma;  /* device [c_out] fp32, EPI_BIAS_RMS_SILU only; copied */
+  const float *gamma;  /* device [c_out] fp32, RMS epilogues only; copied    */
   const float *beta;   /* device [c_out] fp32, nullable; copied               */
 } cc3d_desc;
 
@@ -170,7 +174,7 @@ cc3d_status cc3d_plan_destroy(cc3d_plan *plan);
  *                                      (written by the conv kernel itself on
  *                                      the tensor-core path: no extra launch)
  *   residual  [n][t'][h][w][c_out]     EPI_BIAS_RESIDUAL only, else NULL
- *   next_cache_in / next_cache_out     EPI_BIAS_RMS_SILU only, nullable:
+ *   next_cache_in / next_cache_out     RMS epilogues only, nullable:
  *                                      [n][2][h][w][c_out]; next_cache_out
  *                                      receives the last 2 frames of
  *                                      concat(next_cache_in, y) -- the cache
@@ -191,6 +195,14 @@ cc3d_status rmsnorm_silu(const void *x, const float *gamma, const float *beta,
                          int n, int t, int h, int w, int c, void *y,
                          const void *cache_in, void *cache_out, void *stream);
 
+/* Stand-alone channel RMS_norm without SiLU (§10.2 WanRMS_norm; the norms
+ * around the downsample path's convs, §10.5), bf16 in / bf16 out:
+ *   y[v,c] = x[v,c] / max(||x[v,:]||_2, 1e-12) * sqrt(C) * gamma[c] (+ beta[c]).
+ * Arguments, layout, caches and errors as for rmsnorm_silu. */
+cc3d_status rms_norm(const void *x, const float *gamma, const float *beta, int n,
+                     int t, int h, int w, int c, void *y, const void *cache_in,
+                     void *cache_out, void *stream);
+
 /* Residual block with c channels and the identity shortcut (§10.4):
  * cc3d_block_create2(n, c, c, ..., w_sc = b_sc = NULL, out). */
 cc3d_status cc3d_block_create(int n, int c, int h, int w, int max_t,
@@ -204,9 +216,10 @@ cc3d_status cc3d_block_create(int n, int c, int h, int w, int max_t,
  * [c_out][c_in][1][1][1] bf16 and b_sc [c_out] fp32 (nullable): the
  * conv_shortcut, required when c_in != c_out (NULL: identity shortcut).
  * The shortcut runs inside conv2 as extra K steps of the same accumulator
- * (the shortcut's bias is added to b2); for c_out > 256 conv1 writes its
- * biased output (bf16) and a separate RMS_norm + SiLU pass follows.  In
- * every block conv1's output is rounded to bf16 before its RMS_norm.
+ * (the shortcut's bias is added to b2); conv1's epilogue applies the
+ * RMS_norm + SiLU (up to c_out = 512; wider blocks write conv1's biased
+ * output and run a separate RMS_norm + SiLU pass).  In every block conv1's
+ * output is rounded to bf16 before its RMS_norm.
  * c_in, c_out multiples of 32 in [32, 1024], else CC3D_ERR_UNSUPPORTED;
  * CC3D_ERR_INVALID_ARG for a NULL weight or gamma, or c_in != c_out without
  * w_sc.  The block owns its activation buffers (max_t frames each). */

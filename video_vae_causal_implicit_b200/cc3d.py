@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(PKG, "libcc3d.so")
 (OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_ALIAS, ERR_OOM, ERR_CUDA, ERR_TIMEOUT,
  ERR_TOO_LARGE) = range(9)
 BF16, FP32 = 0, 1
-EPI_BIAS, EPI_BIAS_RESIDUAL, EPI_BIAS_RMS_SILU = 0, 1, 2
+EPI_BIAS, EPI_BIAS_RESIDUAL, EPI_BIAS_RMS_SILU, EPI_BIAS_RMS = 0, 1, 2, 3
 VARIANT_NONE, VARIANT_UMMA, VARIANT_THIN, VARIANT_FP32 = 0, 1, 2, 3
 
 _STATUS_NAMES = {0: "CC3D_OK", 1: "CC3D_ERR_INVALID_ARG", 2: "CC3D_ERR_UNSUPPORTED",
@@ -57,6 +57,7 @@ SIGNATURES = {
     "cc3d_plan_destroy": (_I, [_VP]),
     "cc3d_forward": (_I, [_VP, _VP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "rmsnorm_silu": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP]),
+    "rms_norm": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP]),
     "cc3d_block_create": (_I, [_I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP,
                                ctypes.POINTER(_VP)]),
     "cc3d_block_create2": (_I, [_I, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
@@ -112,6 +113,10 @@ def cc3d_forward(plan, x, t, cache_in, y, cache_out, residual, next_cache_in, ne
 
 def rmsnorm_silu(x, gamma, beta, n, t, h, w, c, y, cache_in, cache_out, stream):
     return lib().rmsnorm_silu(x, gamma, beta, n, t, h, w, c, y, cache_in, cache_out, stream)
+
+
+def rms_norm(x, gamma, beta, n, t, h, w, c, y, cache_in, cache_out, stream):
+    return lib().rms_norm(x, gamma, beta, n, t, h, w, c, y, cache_in, cache_out, stream)
 
 
 def cc3d_block_create(n, c, h, w, max_t, w1, b1, g1, w2, b2, g2, out):
@@ -257,6 +262,14 @@ def rms_silu(x, gamma, y, beta=None, cache_in=None, cache_out=None, stream=None)
     n, t, h, w, c = (int(s) for s in x.shape)
     check(rmsnorm_silu(_ptr(x), _ptr(gamma), _ptr(beta), n, t, h, w, c, _ptr(y), _ptr(cache_in),
                        _ptr(cache_out), _stream(stream)), "rmsnorm_silu")
+    return y
+
+
+def rms(x, gamma, y, beta=None, cache_in=None, cache_out=None, stream=None):
+    """The RMS_norm alone (no SiLU)."""
+    n, t, h, w, c = (int(s) for s in x.shape)
+    check(rms_norm(_ptr(x), _ptr(gamma), _ptr(beta), n, t, h, w, c, _ptr(y), _ptr(cache_in),
+                   _ptr(cache_out), _stream(stream)), "rms_norm")
     return y
 
 

@@ -214,7 +214,7 @@ cudaError_t run_umma_layer(const UmmaLayer &L, const UmmaCall &c, int *status,
   a.b_resident = cfg.b_resident;
   a.c_sc = L.c_sc;
   a.n_cc_sc = L.n_cc_sc;
-  a.nt = cfg.nt; a.n_ntiles = cfg.n_ntiles;
+  a.nt = cfg.nt; a.n_ntiles = cfg.n_ntiles; a.nh = cfg.nh;
   a.sub = cfg.sub; a.nbuf = cfg.nbuf; a.g_taps = cfg.g_taps; a.pair = cfg.pair;
   a.tiles_w = (w_out + tile_w - 1) / tile_w;
   a.tiles_h = (h_out + umma_tile_h() - 1) / umma_tile_h();
@@ -346,15 +346,16 @@ cc3d_status check_desc(const cc3d_desc *d, int *variant) {
     // no zero rows or columns before the frame, one after): H/2 x W/2 out
     if (d->kt != 1 || d->kh != 3 || d->kw != 3 || d->pad_h != 0 || d->pad_w != 0 ||
         d->stride_t != 1 || d->h % 2 != 0 || d->w % 2 != 0 || d->dtype != CC3D_BF16 ||
-        d->c_in % 32 != 0 || d->epi == CC3D_EPI_BIAS_RMS_SILU)
+        d->c_in % 32 != 0)
       return CC3D_ERR_UNSUPPORTED;
   } else if (d->kh % 2 == 0 || d->kw % 2 == 0 || d->pad_h != d->kh / 2 ||
              d->pad_w != d->kw / 2) {
     return CC3D_ERR_UNSUPPORTED;
   }
   if (d->kt > 3 || d->kh > 3 || d->kw > 3) return CC3D_ERR_UNSUPPORTED;
-  if (d->epi < CC3D_EPI_BIAS || d->epi > CC3D_EPI_BIAS_RMS_SILU) return CC3D_ERR_INVALID_ARG;
-  if (d->epi == CC3D_EPI_BIAS_RMS_SILU && !d->gamma) return CC3D_ERR_INVALID_ARG;
+  if (d->epi < CC3D_EPI_BIAS || d->epi > CC3D_EPI_BIAS_RMS) return CC3D_ERR_INVALID_ARG;
+  const bool rms = d->epi == CC3D_EPI_BIAS_RMS_SILU || d->epi == CC3D_EPI_BIAS_RMS;
+  if (rms && !d->gamma) return CC3D_ERR_INVALID_ARG;
   if (d->dtype == CC3D_FP32) {
     if (d->epi != CC3D_EPI_BIAS || d->stride_t != 1) return CC3D_ERR_UNSUPPORTED;
     *variant = CC3D_VARIANT_FP32;
@@ -372,7 +373,9 @@ cc3d_status check_desc(const cc3d_desc *d, int *variant) {
   }
   if (d->c_in % 32 == 0) {
     if (d->kh != d->kw) return CC3D_ERR_UNSUPPORTED;
-    if (d->epi == CC3D_EPI_BIAS_RMS_SILU && d->c_out > 256) return CC3D_ERR_UNSUPPORTED;
+    // one CTA owns each RMS row: up to 256 channels, or 512 as two MMAs
+    if (rms && d->c_out > 256 && (d->c_out > 512 || d->c_out % 32 != 0))
+      return CC3D_ERR_UNSUPPORTED;
     *variant = CC3D_VARIANT_UMMA;
     return CC3D_OK;
   }
@@ -524,7 +527,9 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
       const int kt_eff = L.s2 ? 9 : desc->kt, ks_eff = L.s2 ? 1 : desc->kh;
       const int h_out = desc->h / desc->stride_h, w_out = desc->w / desc->stride_w;
       if (!choose_umma_config(desc->n, desc->c_in, desc->c_out, h_out, w_out, kt_eff, ks_eff,
-                              desc->epi == CC3D_EPI_BIAS_RMS_SILU, max_out, L.sm_count, &cfg)) {
+                              desc->epi == CC3D_EPI_BIAS_RMS_SILU ||
+                                  desc->epi == CC3D_EPI_BIAS_RMS,
+                              max_out, L.sm_count, &cfg)) {
         s = CC3D_ERR_UNSUPPORTED;
         goto fail;
       }
@@ -555,8 +560,10 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
                                c_sc, 1, cfg.nt, cfg.kc, cfg.pair, stages, conv_stages, 0);
       if (e == cudaSuccess) e = cudaDeviceSynchronize();
       if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
+      // (a pair's CTA loads half of each MMA N-subtile's rows per box)
       if (cfg.pair && !encode_weight_map(&p->map_w, p->wimg,
-                                         static_cast<long long>(desc->c_out) * stages, cfg.nt / 2)) {
+                                         static_cast<long long>(desc->c_out) * stages,
+                                         cfg.nt / cfg.nh / 2)) {
         s = CC3D_ERR_CUDA;
         goto fail;
       }
@@ -605,7 +612,8 @@ static cc3d_status forward_impl(cc3d_plan *p, const void *x, int t, const void *
   if (!x || !y || t < 1 || t > d.max_t) return reject(CC3D_ERR_INVALID_ARG);
   if ((d.epi == CC3D_EPI_BIAS_RESIDUAL) != (residual != nullptr))
     return reject(CC3D_ERR_INVALID_ARG);
-  if (d.epi != CC3D_EPI_BIAS_RMS_SILU && (next_cache_in || next_cache_out))
+  if (d.epi != CC3D_EPI_BIAS_RMS_SILU && d.epi != CC3D_EPI_BIAS_RMS &&
+      (next_cache_in || next_cache_out))
     return reject(CC3D_ERR_INVALID_ARG);
   if ((p->c_sc > 0) != (x_sc != nullptr)) return reject(CC3D_ERR_INVALID_ARG);
   if (!aligned16(x_sc)) return reject(CC3D_ERR_ALIGNMENT);
@@ -730,9 +738,13 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
                       nullptr, stream_v);
 }
 
-cc3d_status rmsnorm_silu(const void *x, const float *gamma, const float *beta, int n, int t,
-                         int h, int w, int c, void *y, const void *cache_in, void *cache_out,
-                         void *stream_v) {
+}  // extern "C"
+
+namespace {
+// RMS_norm over channels (+ SiLU when `silu`), with its 2-frame cache.
+cc3d_status rms_pass(const void *x, const float *gamma, const float *beta, int n, int t, int h,
+                     int w, int c, void *y, const void *cache_in, void *cache_out, bool silu,
+                     void *stream_v) {
   if (!x || !gamma || !y || n < 1 || t < 1 || h < 1 || w < 1 || c < 8) return CC3D_ERR_INVALID_ARG;
   if (c % 8 != 0 || c > 1024) return CC3D_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(y) || !aligned16(cache_in) || !aligned16(cache_out))
@@ -747,8 +759,22 @@ cc3d_status rmsnorm_silu(const void *x, const float *gamma, const float *beta, i
   const cudaError_t e = launch_rmsnorm_silu(
       static_cast<const __nv_bfloat16 *>(x), gamma, beta, n, t, static_cast<long long>(h) * w, c,
       static_cast<__nv_bfloat16 *>(y), static_cast<const __nv_bfloat16 *>(cache_in),
-      static_cast<__nv_bfloat16 *>(cache_out), stream);
+      static_cast<__nv_bfloat16 *>(cache_out), silu, stream);
   return from_cuda(e);
+}
+}  // namespace
+
+extern "C" {
+
+cc3d_status rmsnorm_silu(const void *x, const float *gamma, const float *beta, int n, int t,
+                         int h, int w, int c, void *y, const void *cache_in, void *cache_out,
+                         void *stream) {
+  return rms_pass(x, gamma, beta, n, t, h, w, c, y, cache_in, cache_out, true, stream);
+}
+
+cc3d_status rms_norm(const void *x, const float *gamma, const float *beta, int n, int t, int h,
+                     int w, int c, void *y, const void *cache_in, void *cache_out, void *stream) {
+  return rms_pass(x, gamma, beta, n, t, h, w, c, y, cache_in, cache_out, false, stream);
 }
 
 cc3d_status cc3d_block_create2(int n, int c_in, int c_out, int h, int w, int max_t,
@@ -773,7 +799,7 @@ cc3d_status cc3d_block_create2(int n, int c_in, int c_out, int h, int w, int max
   // The RMS epilogue needs a whole C_out row in one N tile (tcgen05's N is
   // at most 256); wider blocks run conv1 with the bias epilogue and the
   // stand-alone RMS_norm + SiLU after it.
-  b->fused_rms = c_out <= 256;
+  b->fused_rms = c_out <= 256 || (c_out <= 512 && c_out % 32 == 0);
   b->shortcut = w_sc != nullptr;
   cc3d_status s;
   const size_t vox = static_cast<size_t>(n) * max_t * h * w;

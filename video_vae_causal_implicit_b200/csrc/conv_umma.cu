@@ -76,10 +76,13 @@ struct SmemLayout {
   int na, nb;
 };
 
+// RMS_norm epilogues: 2 with SiLU after it, 3 without.
+__host__ __device__ constexpr bool rms_epilogue(int epi) { return epi == 2 || epi == 3; }
+
 // Epilogue parameters staged in shared memory: bias[c_out] (and, for the
-// RMS epilogue, gamma[c_out], beta[c_out]).
+// RMS epilogues, gamma[c_out], beta[c_out]).
 __host__ __device__ constexpr int param_floats(int c_out, int epi) {
-  return c_out * (epi == 2 ? 3 : 1);
+  return c_out * (rms_epilogue(epi) ? 3 : 1);
 }
 
 __host__ __device__ inline uint32_t round_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
@@ -125,6 +128,12 @@ __host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw
 
 struct TileCoord {
   int ntile, n, t, h0, w0;
+};
+
+// A compile-time int for generic lambdas.
+template <int V>
+struct IntConst {
+  static constexpr int value = V;
 };
 
 // Tile order: N tile fastest (CTAs sharing an input halo run together),
@@ -301,11 +310,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto load_b = [&](int slot, int part, size_t stage_idx, int ntile) {
         const uint32_t dst = smem_base + L.b_off + slot * L.b_slot + part * L.b_stage;
         if constexpr (PAIR) {
-          // rows of the weight image [ntile][tap][cchunk][NT][64]
-          const int row = static_cast<int>(
-              ((static_cast<size_t>(ntile) * stages_per_ntile + stage_idx) * p.nt) +
-              rank * (p.nt / 2));
-          tma_load_2d_pair(dst, &map_w, lead_full_b + 8u * slot, 0, row);
+          // rows of the weight image [ntile][tap][cchunk][NT][64]: for each
+          // of the nh MMA N-subtiles, this CTA's half of its rows
+          const int nm = p.nt / p.nh;
+          const int row0 = static_cast<int>(
+              (static_cast<size_t>(ntile) * stages_per_ntile + stage_idx) * p.nt);
+          for (int hh = 0; hh < p.nh; ++hh)
+            tma_load_2d_pair(dst + static_cast<uint32_t>(hh * (nm / 2)) * 128u, &map_w,
+                             lead_full_b + 8u * slot, 0, row0 + hh * nm + rank * (nm / 2));
         } else {
           const uint8_t *wsrc =
               p.wimg + static_cast<size_t>(ntile) * stages_per_ntile * L.b_stage;
@@ -435,7 +447,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------ MMA issuer ----------------------------------
     // (a pair's follower issues nothing: the leader's MMAs cover both CTAs)
     if (lane == 0 && pair_leader) {
-      const uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * kM : kM, p.nt);
+      // nh MMAs of N = nt / nh each cover the tile's nt columns
+      const int nm = p.nt / p.nh;
+      const uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * kM : kM, nm);
+      // B start of N-subtile 1 relative to 0: nm rows of 16 bytes in each
+      // core-matrix slab, or (pair) nm / 2 rows of 128 swizzled bytes
+      const uint32_t bhalf16 = PAIR ? static_cast<uint32_t>(nm / 2) * 8u : static_cast<uint32_t>(nm);
       const uint32_t b_lbo = static_cast<uint32_t>(p.nt) * 16u;
       // Descriptors of stage 0; other stages, taps, sub-tiles and K steps
       // only move the start address (low 14 bits, 16-byte units), so they
@@ -478,23 +495,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         // halo at `a_st` seen through spatial tap `ts`.  The operands were
         // written by TMA and handed over by the full barriers, whose
         // completion the tensor core's reads observe without a fence.
+        // (the issuing thread is the throughput limit of the big convs:
+        // the loops below unroll completely, with the N-subtile count
+        // resolved once per stage)
         auto mma_stage = [&](uint64_t a_st, uint64_t b_st, int ts) {
           const uint64_t a_tap = a_st + ((ts / KS) * halo_w + (ts % KS)) * pix16;
+          auto issue = [&](auto nh_c) {
+            constexpr int NH = decltype(nh_c)::value;
 #pragma unroll
-          for (int j = 0; j < KC / 16; ++j) {
-            // every sub-tile (8 pixels further along the halo row) reuses
-            // this weight stage
+            for (int j = 0; j < KC / 16; ++j) {
+              // every sub-tile (8 pixels further along the halo row) and
+              // every N-subtile reuses this weight stage
 #pragma unroll
-            for (int sbt = 0; sbt < SUB; ++sbt) {
-              if constexpr (PAIR)
-                umma_bf16_pair(d_tmem, a_tap + j * astep16, b_st + j * bstep16, idesc,
-                               accumulate);
-              else
-                umma_bf16(d_tmem + sbt * p.nt, a_tap + sbt * kTW * pix16 + j * astep16,
-                          b_st + j * bstep16, idesc, accumulate);
+              for (int sbt = 0; sbt < SUB; ++sbt) {
+#pragma unroll
+                for (int hh = 0; hh < NH; ++hh) {
+                  if constexpr (PAIR)
+                    umma_bf16_pair(d_tmem + hh * nm, a_tap + j * astep16,
+                                   b_st + j * bstep16 + hh * bhalf16, idesc, accumulate);
+                  else
+                    umma_bf16(d_tmem + sbt * p.nt + hh * nm,
+                              a_tap + sbt * kTW * pix16 + j * astep16,
+                              b_st + j * bstep16 + hh * bhalf16, idesc, accumulate);
+                }
+              }
+              accumulate = 1;
             }
-            accumulate = 1;
-          }
+          };
+          if (p.nh == 2) issue(IntConst<2>{});
+          else issue(IntConst<1>{});
         };
         // arrive on `bar` (in both CTAs of a pair) once the MMAs issued so
         // far have completed
@@ -527,8 +556,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
               }
               const uint64_t b_slot = bdesc0 + static_cast<uint32_t>(sb) * bslot16;
-              for (int u = 0; u < g_taps; ++u)
-                mma_stage(a_st, b_slot + static_cast<uint32_t>(u) * bstage16, g * g_taps + u);
+              if (g_taps == KS) {
+                // one kernel row: taps (g, 0 .. KS-1)
+#pragma unroll
+                for (int u = 0; u < KS; ++u)
+                  mma_stage(a_st, b_slot + static_cast<uint32_t>(u) * bstage16, g * KS + u);
+              } else {
+                mma_stage(a_st, b_slot, g);
+              }
               // frees the weight slot (in both CTAs of a pair) once these
               // MMAs have read it
               release(&empty_b[sb]);
@@ -572,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *sp = reinterpret_cast<float *>(smem + L.p_off);
     for (int i = static_cast<int>(threadIdx.x) - 64; i < p.c_out; i += 32 * kEpiWarps) {
       sp[i] = p.bias[i];
-      if (p.epi == 2) {
+      if (rms_epilogue(p.epi)) {
         sp[p.c_out + i] = p.gamma[i];
         sp[2 * p.c_out + i] = p.beta ? p.beta[i] : 0.f;
       }
@@ -584,10 +619,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     // elements of one input frame and one output frame
     const size_t in_frame = static_cast<size_t>(p.h) * p.w * p.c_in;
     const size_t out_frame = static_cast<size_t>(p.h) * p.w * p.c_out;
+    // The call's frame caches, written by the last output frame's tiles:
+    // plain copies of the tile's pixels (each N tile takes its share of the
+    // channels), made while the tile's MMAs run.
+    auto copy_caches = [&](const TileCoord &tc) {
+      for (int sbt = 0; sbt < SUB; ++sbt) {
+        const int h = tc.h0 + r, w = tc.w0 + (PAIR ? rank : sbt) * kTW + c;
+        if (h >= p.h || w >= p.w) continue;
+        const size_t pix_img = static_cast<size_t>(h) * p.w + w;
+        const int cf = p.cache_frames;
+        if (p.cache_out && cf > 0) {
+          // cache_out[f] = concat(cache_in or zeros, x)[t_in + f]
+          const int q_all = p.c_in / 8;
+          const int q0 = tc.ntile * q_all / p.n_ntiles;
+          const int q1 = (tc.ntile + 1) * q_all / p.n_ntiles;
+          for (int f = 0; f < cf; ++f) {
+            const int src_f = p.t_in + f;  // index into the concatenation
+            const __nv_bfloat16 *src = nullptr;
+            if (src_f >= cf)
+              src = p.x_in + (static_cast<size_t>(tc.n) * p.t_in + (src_f - cf)) * in_frame;
+            else if (p.cache_in)
+              src = p.cache_in + (static_cast<size_t>(tc.n) * cf + src_f) * in_frame;
+            __nv_bfloat16 *dst = p.cache_out + (static_cast<size_t>(tc.n) * cf + f) * in_frame;
+            copy_pixel_chunks(src ? src + pix_img * p.c_in : nullptr, dst + pix_img * p.c_in, q0,
+                              q1);
+          }
+        }
+        if (p.ncache_out && p.t < 2) {
+          // one output frame: next_cache_out[0] = next_cache_in[1] (or
+          // zeros); frame 1 is this tile's output, stored with it
+          const int n0 = tc.ntile * p.nt;
+          const __nv_bfloat16 *src =
+              p.ncache_in ? p.ncache_in + (static_cast<size_t>(tc.n) * 2 + 1) * out_frame +
+                                pix_img * p.c_out
+                          : nullptr;
+          __nv_bfloat16 *dst =
+              p.ncache_out + static_cast<size_t>(tc.n) * 2 * out_frame + pix_img * p.c_out;
+          copy_pixel_chunks(src, dst, n0 / 8, (n0 + p.nt) / 8);
+        }
+      }
+    };
     for (int tile = cid; tile < n_tiles; tile += ncl, ++it) {
       const int buf = it % p.nbuf;
       const uint32_t use_par = static_cast<uint32_t>((it / p.nbuf) & 1);
       const TileCoord tc0 = decode_tile(tile, p);
+      if (tc0.t == p.t - 1) copy_caches(tc0);
       uint32_t got = 0;
       if (lane == 0)
         got = mbar_wait_bounded(&acc_full[buf], use_par, p.wait_limit_ns, p.status, 5) ? 1u : 0u;
@@ -614,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 pix_img * p.c_out + n0
                           : nullptr;
         float inv = 1.0f;
-        if (p.epi == 2) {
+        if (rms_epilogue(p.epi)) {
           // pass 1: sum of squares of the biased row h1 (three loads in
           // flight).  h1 is a bf16 activation, as it is when conv1 writes it
           // out for a separate RMS_norm: it is rounded before it is used.
@@ -705,7 +781,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 v[i] += __bfloat162float(rb0[i]);
                 v[8 + i] += __bfloat162float(rb1[i]);
               }
-            } else if (p.epi == 2) {
+            } else if (rms_epilogue(p.epi)) {
               float gv[16], be[16];
               ld_param16(s_gamma + 4u * static_cast<uint32_t>(n0 + j), gv);
               ld_param16(s_beta + 4u * static_cast<uint32_t>(n0 + j), be);
@@ -713,7 +789,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int i = 0; i < 16; ++i) {
                 float a = round_to_bf16(v[i]) * inv * gv[i];
                 a += be[i];
-                v[i] = silu_fast(a);
+                v[i] = p.epi == 2 ? silu_fast(a) : a;
               }
             }
             if (valid) {
@@ -735,40 +811,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_regs_after_wait<32>(nxt);
 #pragma unroll
             for (int i = 0; i < 32; ++i) raw[i] = nxt[i];
-          }
-        }
-        // ---- the call's frame caches, written by the last output frame's
-        // tiles: plain copies of this tile's pixels, each N tile taking its
-        // share of the channels ----
-        if (valid && tc0.t == p.t - 1) {
-          const int cf = p.cache_frames;
-          if (p.cache_out && cf > 0) {
-            // cache_out[f] = concat(cache_in or zeros, x)[t_in + f]
-            const int q_all = p.c_in / 8;
-            const int q0 = tc0.ntile * q_all / p.n_ntiles;
-            const int q1 = (tc0.ntile + 1) * q_all / p.n_ntiles;
-            for (int f = 0; f < cf; ++f) {
-              const int src_f = p.t_in + f;  // index into the concatenation
-              const __nv_bfloat16 *src = nullptr;
-              if (src_f >= cf)
-                src = p.x_in + (static_cast<size_t>(tc0.n) * p.t_in + (src_f - cf)) * in_frame;
-              else if (p.cache_in)
-                src = p.cache_in + (static_cast<size_t>(tc0.n) * cf + src_f) * in_frame;
-              __nv_bfloat16 *dst = p.cache_out + (static_cast<size_t>(tc0.n) * cf + f) * in_frame;
-              copy_pixel_chunks(src ? src + pix_img * p.c_in : nullptr, dst + pix_img * p.c_in,
-                                q0, q1);
-            }
-          }
-          if (p.ncache_out && p.t < 2) {
-            // one output frame: next_cache_out[0] = next_cache_in[1] (or
-            // zeros); frame 1 is this tile's output, stored above
-            const __nv_bfloat16 *src =
-                p.ncache_in ? p.ncache_in + (static_cast<size_t>(tc0.n) * 2 + 1) * out_frame +
-                                  pix_img * p.c_out
-                            : nullptr;
-            __nv_bfloat16 *dst =
-                p.ncache_out + static_cast<size_t>(tc0.n) * 2 * out_frame + pix_img * p.c_out;
-            copy_pixel_chunks(src, dst, n0 / 8, (n0 + p.nt) / 8);
           }
         }
       }  // sub-tiles
@@ -904,6 +946,11 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
       if (c_out % nt == 0 && (!rms_epi || nt == c_out)) return nt;
     return 0;
   };
+  // An RMS row wider than one MMA (c_out up to 512): the CTA tile takes the
+  // whole row as two MMAs of N = c_out / 2 per K step into adjacent tensor
+  // memory columns (one accumulator buffer: 2 x c_out columns do not fit).
+  const bool wide_rms = rms_epi && c_out > 256;
+  if (wide_rms && (c_out > 512 || c_out % 32 != 0)) return false;
   // Every choice below depends on (n, c, h, w, epilogue) and the plan's
   // max_t -- never on a call's t.  Whatever the shape, every output sums
   // its taps into one fp32 accumulator in the same order: the shapes differ
@@ -912,7 +959,8 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
   one.kc = (c_in % 64 == 0) ? 64 : (c_in % 96 == 0) ? 96 : 32;
   one.sub = 1;
   one.pair = 0;
-  one.nt = largest_nt(256);
+  one.nh = wide_rms ? 2 : 1;
+  one.nt = wide_rms ? c_out : largest_nt(256);
   if (!one.nt) return false;
   one.n_ntiles = c_out / one.nt;
   one.params = param_floats(c_out, rms_epi ? 2 : 0);
@@ -928,7 +976,7 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
   // single buffer stalls the MMAs behind the epilogue).
   UmmaConfig two = one;
   two.sub = 2;
-  two.nt = largest_nt(128);
+  two.nt = wide_rms ? 0 : largest_nt(128);
   if (two.nt) {
     two.n_ntiles = c_out / two.nt;
     if (finish_config(ks, kt, c_in, two) && two.nbuf == 2) {
@@ -947,7 +995,8 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
     UmmaConfig pr = one;
     pr.pair = 1;
     pr.sub = 2;  // the tile is two MMA tiles wide
-    if (finish_config(ks, kt, c_in, pr) && pr.nbuf == 2) {
+    // (a wide RMS row has one accumulator buffer whatever the shape)
+    if (finish_config(ks, kt, c_in, pr) && (pr.nbuf == 2 || wide_rms)) {
       const long long cost = frame_cost(pr, nt_frames, h, w, sm_count);
       if (cost <= best) {
         best = cost;
@@ -1063,6 +1112,11 @@ cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_ca
     return cudaErrorInvalidValue;
   if (args.pair && (kc != 64 || args.sub != 2 || grid % 2 != 0 || args.nt % 16 != 0))
     return cudaErrorInvalidValue;
+  // nh MMA N-subtiles: each a valid MMA N (a multiple of 16, at most 256;
+  // on a pair each CTA's half of it whole 8-row swizzle atoms)
+  if (args.nh < 1 || args.nh > 2 || args.nt % args.nh != 0 || (args.nt / args.nh) % 16 != 0 ||
+      args.nt / args.nh > 256 || (args.pair && (args.nt / args.nh) % 16 != 0))
+    return cudaErrorInvalidValue;
   if (args.b_resident && (args.n_ntiles != 1 || args.g_taps != 1 ||
                           args.nb != args.kt * args.kh * args.kw * (args.c_in / kc)))
     return cudaErrorInvalidValue;
@@ -1073,7 +1127,7 @@ cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_ca
   // the frame caches the epilogue writes: whole 16-byte chunks per pixel
   if ((args.cache_out && (args.cache_frames < 1 || args.c_in % 8 != 0 || !args.x_in ||
                           args.t_in < 1 || args.s2)) ||
-      (args.ncache_out && (args.epi != 2 || args.nt % 8 != 0)))
+      (args.ncache_out && (!rms_epilogue(args.epi) || args.nt % 8 != 0)))
     return cudaErrorInvalidValue;
   UmmaKernel k = umma_kernel_for(kc, args.kh, args.sub, args.pair);
   if (!k) return cudaErrorInvalidValue;

@@ -24,9 +24,12 @@ struct UmmaArgs {
   int kt, kh, kw, pad_h, pad_w;
   int stride_t;                   // output frame t reads input frames stride_t * t + kt - (kt - 1)
   int nt, n_ntiles, tiles_w, tiles_h;
+  int nh;                         // MMAs of N = nt / nh that cover the tile's nt columns
+                                  // (2: an RMS row wider than one MMA, e.g. 384 channels)
   int na, nb;                     // pipeline depths (A halo stages, B weight stages)
   int tmem_cols;
-  int epi;                        // 0 bias, 1 bias + residual, 2 bias + RMS + SiLU
+  int epi;                        // 0 bias, 1 bias + residual, 2 bias + RMS + SiLU,
+                                  // 3 bias + RMS
   int has_cache;
   int sub;                        // MMA sub-tiles (8 x 16 px) per CTA tile, side by side: 1 or 2
   int nbuf;                       // accumulator buffers in tensor memory: 1 or 2
@@ -61,7 +64,7 @@ struct UmmaArgs {
 // Tile configuration of the UMMA conv for a plan (chosen from n, c_in, c_out,
 // h, w, the epilogue and the plan's max_t -- never from a call's t).
 struct UmmaConfig {
-  int kc, nt, n_ntiles, sub, nbuf, g_taps, pair, na, nb, tmem_cols, ctas_per_sm;
+  int kc, nt, n_ntiles, nh, sub, nbuf, g_taps, pair, na, nb, tmem_cols, ctas_per_sm;
   int params;      // epilogue parameters staged in shared memory (floats)
   int b_resident;  // every weight stage resident in shared memory (nb of them)
 };
@@ -143,10 +146,11 @@ cudaError_t launch_cache_update(const void *cache_in, const void *src, void *cac
 // RMS_norm + SiLU over channels of n x t frames of hw pixels, bf16 in/out;
 // cache_out (null: not written) = the last two frames of concat(cache_in or
 // zeros, y), written by the same kernel.
+// silu: apply SiLU after the RMS_norm (else the RMS_norm alone).
 cudaError_t launch_rmsnorm_silu(const __nv_bfloat16 *x, const float *gamma, const float *beta,
                                 int n, int t, long long hw, int c, __nv_bfloat16 *y,
                                 const __nv_bfloat16 *cache_in, __nv_bfloat16 *cache_out,
-                                cudaStream_t stream);
+                                bool silu, cudaStream_t stream);
 
 // One tensor-core conv layer as planned: its tile configuration, geometry
 // and device-resident operands (the plan's, or the no-allocation scratch).
@@ -155,7 +159,7 @@ struct UmmaLayer {
   int n, c_in, c_out, h, w;        // input frame geometry
   int kt, kh, kw, pad_h, pad_w;    // kernel as declared (kt, kh, kw of the descriptor)
   int stride_t, s2;                // temporal stride; s2: stride 2 in H and W
-  int epi;                         // 0 bias, 1 bias + residual, 2 bias + RMS + SiLU
+  int epi;                         // 0 bias, 1 bias + residual, 2 bias + RMS + SiLU, 3 bias + RMS
   int c_sc, n_cc_sc;               // fused 1x1x1 conv_shortcut (0: none)
   int sm_count, max_clusters;      // grid sizing (max_clusters: CTA pairs)
   const uint8_t *wimg;             // re-tiled weights

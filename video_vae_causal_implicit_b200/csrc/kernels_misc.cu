@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(256, 4)
     rmsnorm_silu_lanes_kernel(const __nv_bfloat16 *__restrict__ x,
                               const float *__restrict__ gamma, const float *__restrict__ beta,
                               long long voxels, int c, int lpv,
-                              __nv_bfloat16 *__restrict__ y, RmsCache cache) {
+                              __nv_bfloat16 *__restrict__ y, RmsCache cache, bool silu) {
   const int lane = threadIdx.x % 32;
   const int vpw = 32 / lpv;                 // voxels per warp pass
   const int sub = lane % lpv, vloc = lane / lpv;
@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(256, 4)
         for (int e = 0; e < 8; ++e) {
           float a = __bfloat162float(b[e]) * inv * gm[e];
           if (beta) a += __ldg(beta + g * 8 + e);
-          o[e] = silu_fast(a);
+          o[e] = silu ? silu_fast(a) : a;
         }
         uint4 w;
         w.x = pack2(o[0], o[1]);
@@ -247,7 +247,7 @@ template <int CPT>
 __global__ void __launch_bounds__(256)
     rmsnorm_silu_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ gamma,
                         const float *__restrict__ beta, long long voxels, int c,
-                        __nv_bfloat16 *__restrict__ y, RmsCache cache) {
+                        __nv_bfloat16 *__restrict__ y, RmsCache cache, bool silu) {
   __shared__ float partial[256 * CPT];
   __shared__ float inv_s[256 * CPT];
   const int groups = c / 8;
@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(256)
         for (int e = 0; e < 8; ++e) {
           float a = __bfloat162float(b[e]) * inv * gm[e];
           if (beta) a += __ldg(beta + g * 8 + e);
-          o[e] = silu_fast(a);
+          o[e] = silu ? silu_fast(a) : a;
         }
         uint4 w;
         w.x = pack2(o[0], o[1]);
@@ -409,7 +409,7 @@ cudaError_t launch_cache_update(const void *cache_in, const void *src, void *cac
 cudaError_t launch_rmsnorm_silu(const __nv_bfloat16 *x, const float *gamma, const float *beta,
                                 int n, int t, long long hw, int c, __nv_bfloat16 *y,
                                 const __nv_bfloat16 *cache_in, __nv_bfloat16 *cache_out,
-                                cudaStream_t stream) {
+                                bool silu, cudaStream_t stream) {
   const int groups = c / 8;
   if (groups < 1 || n < 1 || t < 1 || hw < 1) return cudaErrorInvalidValue;
   const long long voxels = static_cast<long long>(n) * t * hw;
@@ -431,10 +431,10 @@ cudaError_t launch_rmsnorm_silu(const __nv_bfloat16 *x, const float *gamma, cons
     if (g < 1) g = 1;
     const int grid = static_cast<int>(g);
     switch (gpl) {
-      case 1: rmsnorm_silu_lanes_kernel<1, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache); break;
-      case 2: rmsnorm_silu_lanes_kernel<2, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache); break;
-      case 3: rmsnorm_silu_lanes_kernel<3, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache); break;
-      default: rmsnorm_silu_lanes_kernel<4, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache); break;
+      case 1: rmsnorm_silu_lanes_kernel<1, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache, silu); break;
+      case 2: rmsnorm_silu_lanes_kernel<2, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache, silu); break;
+      case 3: rmsnorm_silu_lanes_kernel<3, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache, silu); break;
+      default: rmsnorm_silu_lanes_kernel<4, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache, silu); break;
     }
   } else {
     constexpr int kCpt = 12;  // 16-byte chunks per thread and pass
@@ -444,7 +444,7 @@ cudaError_t launch_rmsnorm_silu(const __nv_bfloat16 *x, const float *gamma, cons
     if (g > 148LL * 8) g = 148LL * 8;
     if (g < 1) g = 1;
     rmsnorm_silu_kernel<kCpt><<<static_cast<int>(g), 256, 0, stream>>>(x, gamma, beta, voxels,
-                                                                       c, y, cache);
+                                                                       c, y, cache, silu);
   }
   count_launch();
   return cudaGetLastError();

@@ -93,10 +93,11 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   if (d->n < 1 || d->c_in < 1 || d->c_out < 1 || d->h < 1 || d->w < 1 || d->max_t < 1 ||
       d->kt < 1 || d->kh < 1 || d->kw < 1 || t < 1 || t > d->max_t)
     return CC3D_ERR_INVALID_ARG;
-  if (d->epi < CC3D_EPI_BIAS || d->epi > CC3D_EPI_BIAS_RMS_SILU) return CC3D_ERR_INVALID_ARG;
-  if (d->epi == CC3D_EPI_BIAS_RMS_SILU && !d->gamma) return CC3D_ERR_INVALID_ARG;
+  if (d->epi < CC3D_EPI_BIAS || d->epi > CC3D_EPI_BIAS_RMS) return CC3D_ERR_INVALID_ARG;
+  const bool rms = d->epi == CC3D_EPI_BIAS_RMS_SILU || d->epi == CC3D_EPI_BIAS_RMS;
+  if (rms && !d->gamma) return CC3D_ERR_INVALID_ARG;
   if ((d->epi == CC3D_EPI_BIAS_RESIDUAL) != (residual != nullptr)) return CC3D_ERR_INVALID_ARG;
-  if (d->epi != CC3D_EPI_BIAS_RMS_SILU && (next_cache_in || next_cache_out))
+  if (!rms && (next_cache_in || next_cache_out))
     return CC3D_ERR_INVALID_ARG;
   if (d->stride_t < 1 || d->stride_t > 2 || d->stride_h != 1 || d->stride_w != 1 ||
       d->dil_t != 1 || d->dil_h != 1 || d->dil_w != 1 || d->groups != 1 ||
@@ -106,7 +107,8 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
       d->pad_w != d->kw / 2)
     return CC3D_ERR_UNSUPPORTED;
   if (d->c_in % 32 != 0 || d->c_out % 16 != 0) return CC3D_ERR_UNSUPPORTED;
-  if (d->epi == CC3D_EPI_BIAS_RMS_SILU && d->c_out > 256) return CC3D_ERR_UNSUPPORTED;
+  if (rms && d->c_out > 256 && (d->c_out > 512 || d->c_out % 32 != 0))
+    return CC3D_ERR_UNSUPPORTED;
   const int taps = d->kt * d->kh * d->kw;
   const size_t wbytes = size_t(2) * d->c_out * d->c_in * taps;
   if (wbytes > kNoAllocWeightBytes || size_t(4) * d->c_out > kNoAllocBiasBytes)
@@ -139,7 +141,7 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   UmmaLayer L;
   std::memset(&L, 0, sizeof L);
   if (!choose_umma_config(d->n, d->c_in, d->c_out, d->h, d->w, d->kt, d->kh,
-                          d->epi == CC3D_EPI_BIAS_RMS_SILU, (d->max_t - 1) / d->stride_t + 1, n_sm,
+                          rms, (d->max_t - 1) / d->stride_t + 1, n_sm,
                           &L.cfg))
     return CC3D_ERR_UNSUPPORTED;
   const UmmaConfig &cfg = L.cfg;
@@ -161,7 +163,7 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   CUtensorMap mw;
   if (cfg.pair && !encode_weight_map(&mw, wimg,
                                      static_cast<long long>(d->c_out) * taps * (d->c_in / 64),
-                                     nt / 2))
+                                     nt / cfg.nh / 2))
     return CC3D_ERR_CUDA;
 
   // ---- the conv (one kernel, which also writes cache_out and next_cache_out) ---------
