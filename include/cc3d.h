@@ -77,7 +77,13 @@ typedef enum {
                                 fixed scratch                              */
 } cc3d_status;
 
-typedef enum { CC3D_BF16 = 0, CC3D_FP32 = 1 } cc3d_dtype;
+/* CC3D_FP8_E4M3: FP8 operands ("Cosmos3 Wan VAE", §9 names low-precision
+ * conv quantisation without fixing one; this is the E4M3 form the tensor
+ * cores take).  x and the caches are E4M3 codes (one byte per element, see
+ * cc3d_quantize_e4m3) standing for x_scale * code; the weights are given in
+ * bf16 and quantised at plan time to w / w_scale[c_out]; y (and residual)
+ * stay bf16:  y = x_scale * w_scale[co] * conv(q_x, q_w) + b[co]. */
+typedef enum { CC3D_BF16 = 0, CC3D_FP32 = 1, CC3D_FP8_E4M3 = 2 } cc3d_dtype;
 
 /* Epilogue fused into the conv (§10.4: bias, residual add, next RMS+SiLU). */
 typedef enum {
@@ -129,6 +135,10 @@ typedef struct {
   cc3d_epilogue epi;
   const float *gamma;  /* device [c_out] fp32, RMS epilogues only; copied    */
   const float *beta;   /* device [c_out] fp32, nullable; copied               */
+  const float *w_scale; /* CC3D_FP8_E4M3 only: device [c_out] fp32 per-output-
+                           channel weight scales (> 0); copied               */
+  float x_scale;        /* CC3D_FP8_E4M3 only: the activation scale (> 0) of x
+                           and the caches                                   */
 } cc3d_desc;
 
 typedef struct {
@@ -155,7 +165,9 @@ typedef struct cc3d_block cc3d_block;
  * gamma, beta) into plan-owned device memory.  Synchronous.  Returns
  * CC3D_ERR_UNSUPPORTED for dilation/groups != 1, strides other than those
  * stride_t / stride_h / stride_w document, even kernel sizes, or channel
- * counts no kernel covers.  bf16 covers c_out % 16 == 0 with
+ * counts no kernel covers.  FP8 E4M3 covers c_in % 128 == 0, c_out % 16 ==
+ * 0, kh == kw in {1, 3}, kt <= 3, temporal stride 1 or 2, bias or residual
+ * epilogue.  bf16 covers c_out % 16 == 0 with
  * either c_in % 32 == 0 (kh == kw in {1, 3}, kt <= 3; N tiles of at most
  * 256 channels) or c_in <= 8 (the thin first-layer path: bias epilogue,
  * c_out <= 256, kt*kh*kw*c_in <= 256); fp32 covers any channel count with
@@ -184,6 +196,14 @@ cc3d_status cc3d_forward(cc3d_plan *plan, const void *x, int t,
                          const void *cache_in, void *y, void *cache_out,
                          const void *residual, const void *next_cache_in,
                          void *next_cache_out, void *stream);
+
+/* FP8 E4M3 codes of bf16 values: q[i] = E4M3(x[i] / scale), the quotient
+ * an IEEE fp32 division, rounded to nearest even and saturated to +-448
+ * (the activation side of a CC3D_FP8_E4M3 plan).  x (device, 16-byte
+ * aligned) holds `count` bf16 values, q (device, 8-byte aligned) receives
+ * `count` bytes; count % 8 == 0, scale > 0, else CC3D_ERR_INVALID_ARG. */
+cc3d_status cc3d_quantize_e4m3(const void *x, size_t count, float scale, void *q,
+                               void *stream);
 
 /* Stand-alone channel RMS_norm + SiLU (§10.2, §10.4), bf16 in / bf16 out.
  *   x, y      [n][t][h][w][c]; gamma [c] fp32; beta [c] fp32 nullable

@@ -93,6 +93,8 @@ def _load():
                                               dp, dp]
             lib.orc_round_e4m3.argtypes = [ctypes.c_double]
             lib.orc_round_e4m3.restype = ctypes.c_double
+            lib.orc_round_e4m3_array.argtypes = [dp, ctypes.c_longlong]
+            lib.orc_round_e4m3_array.restype = None
             lib.orc_round_bf16.argtypes = [ctypes.c_double]
             lib.orc_round_bf16.restype = ctypes.c_double
             lib.orc_silu.argtypes = [ctypes.c_double]
@@ -314,31 +316,41 @@ def round_e4m3(v: float) -> float:
     return _load().orc_round_e4m3(float(v))
 
 
-def quantize_e4m3(a, scale):
+def quantize_e4m3(a, scale, quotient="f64"):
     """E4M3 codes of a / scale, returned as their float64 values (so that
     a ~= scale * quantize_e4m3(a, scale)); scale broadcasts against a.
-    Loops over round_e4m3: meant for the small arrays of the tests."""
+    quotient "f64" divides in float64; "f32" divides the float32 values of
+    a and scale in float32 (one correctly rounded IEEE division), the
+    precision in which a GPU kernel that quantises in fp32 takes the same
+    rounding decision.  Each code is round_e4m3 of its quotient."""
     lib = _load()
-    v = np.asarray(a, dtype=np.float64) / np.asarray(scale, dtype=np.float64)
-    out = np.empty_like(v)
-    flat_in, flat_out = v.reshape(-1), out.reshape(-1)
-    for k in range(flat_in.size):
-        flat_out[k] = lib.orc_round_e4m3(float(flat_in[k]))
+    if quotient == "f32":
+        v = (np.asarray(a, dtype=np.float32) / np.asarray(scale, dtype=np.float32)).astype(
+            np.float64)
+    elif quotient == "f64":
+        v = np.asarray(a, dtype=np.float64) / np.asarray(scale, dtype=np.float64)
+    else:
+        raise ValueError(quotient)
+    out = np.ascontiguousarray(v, dtype=np.float64).copy()
+    lib.orc_round_e4m3_array(out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), out.size)
     return out
 
 
-def causal_conv3d_fp8(x, weight, bias, s_x, s_w, cache=None, pad=(1, 1)):
+def causal_conv3d_fp8(x, weight, bias, s_x, s_w, cache=None, pad=(1, 1), quotient="f64",
+                      stride_t=1):
     """The causal Conv3D on E4M3 operands: x is quantised with the
     per-tensor scale s_x (cache too), weight with the per-output-channel
     scales s_w [Cout]; y = s_x * s_w[co] * conv(q_x, q_w) + b[co], the
-    contraction exact in float64.  Returns float64 [N, Cout, T, H, W]."""
+    contraction exact in float64.  quotient: as for quantize_e4m3.
+    Returns float64 [N, Cout, (T-1)//stride_t+1, H, W]."""
     x = np.asarray(x, dtype=np.float64)
     w = np.asarray(weight, dtype=np.float64)
     s_w = np.asarray(s_w, dtype=np.float64).reshape(-1)
-    qx = quantize_e4m3(x, s_x)
-    qw = quantize_e4m3(w, s_w.reshape(-1, 1, 1, 1, 1))
-    qc = quantize_e4m3(np.asarray(cache, dtype=np.float64), s_x) if cache is not None else None
-    y = causal_conv3d(qx, qw, None, cache=qc, pad=pad)
+    qx = quantize_e4m3(x, s_x, quotient)
+    qw = quantize_e4m3(w, s_w.reshape(-1, 1, 1, 1, 1), quotient)
+    qc = (quantize_e4m3(np.asarray(cache, dtype=np.float64), s_x, quotient)
+          if cache is not None else None)
+    y = causal_conv3d(qx, qw, None, cache=qc, pad=pad, stride_t=stride_t)
     y *= float(s_x) * s_w.reshape(1, -1, 1, 1, 1)
     if bias is not None:
         y += np.asarray(bias, dtype=np.float64).reshape(1, -1, 1, 1, 1)

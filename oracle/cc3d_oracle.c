@@ -119,6 +119,11 @@ double orc_round_e4m3(double v) {
   return v < 0 ? -r : r;
 }
 
+/* orc_round_e4m3 over an array, in place. */
+void orc_round_e4m3_array(double *v, long long count) {
+  for (long long i = 0; i < count; ++i) v[i] = orc_round_e4m3(v[i]);
+}
+
 /* One output of the causal Conv3D, straight from the definition.
  * Input frame for output frame t and temporal tap kt is
  * tau = t + kt - (KT - 1): KT - 1 frames of causal front padding.  A frame

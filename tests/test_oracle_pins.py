@@ -622,6 +622,23 @@ def test_e4m3_special_cases():
     assert oracle.round_e4m3(-1.3) == -oracle.round_e4m3(1.3)
 
 
+def test_e4m3_quantiser_with_f32_quotient_matches_torch():
+    """quotient="f32": the float32 division x / s followed by one rounding to
+    E4M3 equals torch's float32 division and float8_e4m3fn cast (saturated
+    to +-448 first), code for code, across scales and values; the f64
+    quotient gives the same codes away from rounding boundaries."""
+    g = np.random.default_rng(73)
+    x = np.concatenate([g.standard_normal(4000) * 3, g.uniform(-2000, 2000, 1000),
+                        g.standard_normal(1000) * 1e-3]).astype(np.float32)
+    for s in (0.0137, 0.5, 1.0, 3.7, 448.0 / 7.3):
+        got = oracle.quantize_e4m3(x, s, quotient="f32")
+        q = (torch.from_numpy(x) / torch.tensor(s, dtype=torch.float32)).clamp(-448, 448)
+        ref = q.to(torch.float8_e4m3fn).to(torch.float64).numpy()
+        np.testing.assert_array_equal(got, ref)
+        got64 = oracle.quantize_e4m3(x, s, quotient="f64")
+        assert np.mean(got64 == got) > 0.99
+
+
 def test_fp8_conv_on_representable_operands_is_the_plain_conv():
     """Unit scales and operands already in E4M3: quantisation is exact, so
     the FP8 conv is the plain conv bit for bit."""

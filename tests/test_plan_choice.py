@@ -17,8 +17,8 @@ from video_vae_causal_implicit_b200 import cc3d
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(ROOT, "video_vae_causal_implicit_b200", "csrc")
-FIELDS = ("ok", "kc", "nt", "n_ntiles", "sub", "nbuf", "g_taps", "pair", "na", "nb", "tmem_cols",
-          "ctas_per_sm", "params", "b_resident", "smem")
+FIELDS = ("ok", "kc", "nt", "n_ntiles", "nh", "sub", "nbuf", "g_taps", "pair", "na", "nb",
+          "tmem_cols", "ctas_per_sm", "params", "b_resident", "smem")
 SMEM_MAX = 227 * 1024
 
 
@@ -49,8 +49,8 @@ def probe(tmp_path_factory):
     return run
 
 
-def case(n=1, ci=64, co=64, h=30, w=52, kt=3, ks=3, rms=False, mt=1, sms=148):
-    return (n, ci, co, h, w, kt, ks, rms, mt, sms)
+def case(n=1, ci=64, co=64, h=30, w=52, kt=3, ks=3, rms=False, mt=1, sms=148, f8=False):
+    return (n, ci, co, h, w, kt, ks, rms, mt, sms, f8)
 
 
 GRID = [case(n=n, ci=ci, co=co, h=h, w=w, kt=kt, ks=ks, rms=rms, mt=mt)
@@ -59,29 +59,31 @@ GRID = [case(n=n, ci=ci, co=co, h=h, w=w, kt=kt, ks=ks, rms=rms, mt=mt)
             [(9, 17), (30, 52), (120, 208), (240, 416)],
             [(3, 3), (3, 1), (1, 1)],
             [False, True], [1, 4], [1, 5])
-        if not (rms and co > 256)]
+        ]
 
 
 def test_every_plan_fits_the_sm(probe):
     for c, p in zip(GRID, probe(GRID)):
-        n, ci, co, h, w, kt, ks, rms, mt, sms = c
+        n, ci, co, h, w, kt, ks, rms, mt, sms, f8 = c
         assert p["ok"] == 1, c
         assert p["smem"] <= SMEM_MAX, (c, p)
         assert 32 <= p["tmem_cols"] <= 512 and p["tmem_cols"] & (p["tmem_cols"] - 1) == 0, (c, p)
         cta_sub = 1 if p["pair"] else p["sub"]
         assert p["tmem_cols"] >= p["nbuf"] * cta_sub * p["nt"], (c, p)
-        assert co % p["nt"] == 0 and p["nt"] <= 256 and p["nt"] % 16 == 0, (c, p)
+        assert co % p["nt"] == 0 and p["nt"] % 16 == 0, (c, p)
         assert p["n_ntiles"] * p["nt"] == co, (c, p)
         assert ci % p["kc"] == 0 and p["kc"] in (32, 64, 96), (c, p)
         if rms:
             assert p["nt"] == co, (c, p)  # the RMS epilogue needs the whole row
+            assert p["nh"] == (2 if co > 256 else 1), (c, p)
         assert p["params"] == co * (3 if rms else 1), (c, p)
+        assert p["nt"] // p["nh"] <= 256, (c, p)
         assert 1 <= p["ctas_per_sm"] <= 2, (c, p)
 
 
 def test_slots_pair_and_resident_only_where_valid(probe):
     for c, p in zip(GRID, probe(GRID)):
-        n, ci, co, h, w, kt, ks, rms, mt, sms = c
+        n, ci, co, h, w, kt, ks, rms, mt, sms, f8 = c
         # a weight slot holds one tap, or one whole kernel row of taps
         assert p["g_taps"] in (1, ks), (c, p)
         if p["pair"]:
@@ -118,6 +120,20 @@ def test_downsample_conv_plans(probe):
         assert p["ok"] == 1 and p["smem"] <= SMEM_MAX and p["g_taps"] == 1, (c, p)
         if p["b_resident"]:
             assert p["nb"] == 9 * c[1] // p["kc"] and p["na"] >= 3, (c, p)
+
+
+def test_fp8_plans(probe):
+    """FP8 E4M3 operands: 128-channel chunks (one 128-byte swizzled row per
+    pixel), on every tile shape that takes them, within the SM."""
+    cases = [case(n=n, ci=ci, co=co, h=h, w=w, ks=ks, mt=mt, f8=True)
+             for (ci, co), (h, w), ks, n, mt in itertools.product(
+                 [(128, 128), (384, 384), (256, 512)], [(16, 20), (30, 52), (120, 208)],
+                 [3, 1], [1, 2], [1, 5])]
+    for c, p in zip(cases, probe(cases)):
+        assert p["ok"] == 1 and p["kc"] == 128 and p["smem"] <= SMEM_MAX, (c, p)
+    # channel counts that are not whole 128-channel chunks have no FP8 plan
+    bad = probe([case(ci=96, co=96, f8=True), case(ci=192, co=192, f8=True)])
+    assert [p["ok"] for p in bad] == [0, 0]
 
 
 def test_the_documented_choices(probe):

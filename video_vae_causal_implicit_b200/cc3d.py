@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(PKG, "libcc3d.so")
 
 (OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_ALIAS, ERR_OOM, ERR_CUDA, ERR_TIMEOUT,
  ERR_TOO_LARGE) = range(9)
-BF16, FP32 = 0, 1
+BF16, FP32, FP8_E4M3 = 0, 1, 2
 EPI_BIAS, EPI_BIAS_RESIDUAL, EPI_BIAS_RMS_SILU, EPI_BIAS_RMS = 0, 1, 2, 3
 VARIANT_NONE, VARIANT_UMMA, VARIANT_THIN, VARIANT_FP32 = 0, 1, 2, 3
 
@@ -39,7 +39,8 @@ class Desc(ctypes.Structure):
         "n", "c_in", "c_out", "h", "w", "max_t", "kt", "kh", "kw", "pad_h", "pad_w",
         "stride_t", "stride_h", "stride_w", "dil_t", "dil_h", "dil_w", "groups", "dtype")] + [
         ("weight", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("epi", ctypes.c_int),
-        ("gamma", ctypes.c_void_p), ("beta", ctypes.c_void_p)]
+        ("gamma", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("w_scale", ctypes.c_void_p),
+        ("x_scale", ctypes.c_float)]
 
 
 class Stats(ctypes.Structure):
@@ -58,6 +59,7 @@ SIGNATURES = {
     "cc3d_forward": (_I, [_VP, _VP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "rmsnorm_silu": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP]),
     "rms_norm": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP]),
+    "cc3d_quantize_e4m3": (_I, [_VP, ctypes.c_size_t, ctypes.c_float, _VP, _VP]),
     "cc3d_block_create": (_I, [_I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP,
                                ctypes.POINTER(_VP)]),
     "cc3d_block_create2": (_I, [_I, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
@@ -178,7 +180,8 @@ class Plan:
     device (bf16, or fp32 for dtype=FP32); bias/gamma/beta fp32 [C_out]."""
 
     def __init__(self, weight, bias=None, *, n=1, h, w, max_t, epi=EPI_BIAS, gamma=None,
-                 beta=None, dtype=BF16, pad=None, stride_t=1, stride_hw=1):
+                 beta=None, dtype=BF16, pad=None, stride_t=1, stride_hw=1, w_scale=None,
+                 x_scale=0.0):
         co, ci, kt, kh, kw = (int(s) for s in weight.shape)
         d = Desc()
         d.n, d.c_in, d.c_out, d.h, d.w, d.max_t = n, ci, co, h, w, max_t
@@ -195,6 +198,8 @@ class Plan:
         d.epi = epi
         d.gamma = gamma.data_ptr() if gamma is not None else None
         d.beta = beta.data_ptr() if beta is not None else None
+        d.w_scale = w_scale.data_ptr() if w_scale is not None else None
+        d.x_scale = float(x_scale)
         self.desc = d
         self.handle = ctypes.c_void_p()
         check(cc3d_plan_create(d, self.handle), "cc3d_plan_create")
@@ -271,6 +276,13 @@ def rms(x, gamma, y, beta=None, cache_in=None, cache_out=None, stream=None):
     check(rms_norm(_ptr(x), _ptr(gamma), _ptr(beta), n, t, h, w, c, _ptr(y), _ptr(cache_in),
                    _ptr(cache_out), _stream(stream)), "rms_norm")
     return y
+
+
+def quantize_e4m3(x, scale, q, stream=None):
+    """q (uint8, same element count as the bf16 tensor x) = E4M3(x / scale)."""
+    check(lib().cc3d_quantize_e4m3(_ptr(x), x.numel(), float(scale), _ptr(q), _stream(stream)),
+          "cc3d_quantize_e4m3")
+    return q
 
 
 def sync_status(stream=None):

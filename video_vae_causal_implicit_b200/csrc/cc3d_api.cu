@@ -76,23 +76,27 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
-// 5-D bf16 tensor map over an NDHWC buffer: dims (C, W, H, T, N), a box of
-// box_c channels x box_w x box_h x 1 x 1, zero fill out of bounds; 64-channel
-// boxes (128-byte pixel rows) land 128-byte swizzled, 8-channel boxes plain.
+// 5-D tensor map over an NDHWC buffer of bf16 (esz 2) or FP8 E4M3 bytes
+// (esz 1): dims (C, W, H, T, N), a box of box_c channels x box_w x box_h x
+// 1 x 1, zero fill out of bounds.  Boxes of 128-byte pixel rows (64 bf16 or
+// 128 E4M3 channels) land 128-byte swizzled, 8-channel bf16 boxes plain.
 bool encode_act_map(CUtensorMap *m, const void *base, int c, int w, int h, int t, int n,
-                    int box_w, int box_h, int box_c) {
-  if (box_c != 8 && box_c != 64) return false;
+                    int box_w, int box_h, int box_c, int esz = 2) {
+  const bool sw = box_c * esz == 128;
+  if (!(esz == 2 && (box_c == 8 || box_c == 64)) && !(esz == 1 && box_c == 128)) return false;
   auto fn = encode_fn();
   if (!fn) return false;
+  const cuuint64_t e = static_cast<cuuint64_t>(esz);
   cuuint64_t dims[5] = {(cuuint64_t)c, (cuuint64_t)w, (cuuint64_t)h, (cuuint64_t)t,
                         (cuuint64_t)n};
-  cuuint64_t strides[4] = {(cuuint64_t)c * 2, (cuuint64_t)c * 2 * w, (cuuint64_t)c * 2 * w * h,
-                           (cuuint64_t)c * 2 * w * h * t};
+  cuuint64_t strides[4] = {(cuuint64_t)c * e, (cuuint64_t)c * e * w, (cuuint64_t)c * e * w * h,
+                           (cuuint64_t)c * e * w * h * t};
   cuuint32_t box[5] = {(cuuint32_t)box_c, (cuuint32_t)box_w, (cuuint32_t)box_h, 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  box_c == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+  CUresult r = fn(m, esz == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                  5, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  sw ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -183,12 +187,13 @@ cudaError_t run_umma_layer(const UmmaLayer &L, const UmmaCall &c, int *status,
   const int box_w = umma_halo_box_w(cfg.kc, cfg.pair ? 1 : cfg.sub, ks);
   const int box_h = umma_tile_h() + ks - 1;
   const int box_c = umma_halo_box_c(cfg.kc);
+  const int esz = L.e4m3 ? 1 : 2;  // bytes per input element
   if (!(L.s2 ? encode_act_map_s2(&mx, c.x, L.c_in, L.w, L.h, c.t, L.n, box_w, box_h, box_c)
-             : encode_act_map(&mx, c.x, L.c_in, L.w, L.h, c.t, L.n, box_w, box_h, box_c)))
+             : encode_act_map(&mx, c.x, L.c_in, L.w, L.h, c.t, L.n, box_w, box_h, box_c, esz)))
     return cudaErrorInvalidValue;
   const bool has_cache = c.cache_in && front > 0;
   if (has_cache) {
-    if (!encode_act_map(&mc, c.cache_in, L.c_in, L.w, L.h, front, L.n, box_w, box_h, box_c))
+    if (!encode_act_map(&mc, c.cache_in, L.c_in, L.w, L.h, front, L.n, box_w, box_h, box_c, esz))
       return cudaErrorInvalidValue;
   } else {
     mc = mx;
@@ -222,11 +227,13 @@ cudaError_t run_umma_layer(const UmmaLayer &L, const UmmaCall &c, int *status,
   a.epi = L.epi;
   a.has_cache = has_cache ? 1 : 0;
   // the frame caches, written by the kernel's epilogue
-  a.x_in = static_cast<const __nv_bfloat16 *>(c.x);
+  a.x_in = static_cast<const uint8_t *>(c.x);
   a.t_in = c.t;
   a.cache_frames = front;
-  a.cache_in = static_cast<const __nv_bfloat16 *>(has_cache ? c.cache_in : nullptr);
-  a.cache_out = front > 0 ? static_cast<__nv_bfloat16 *>(c.cache_out) : nullptr;
+  a.cache_in = static_cast<const uint8_t *>(has_cache ? c.cache_in : nullptr);
+  a.cache_out = front > 0 ? static_cast<uint8_t *>(c.cache_out) : nullptr;
+  a.in_esz = esz;
+  a.oscale = L.e4m3 ? L.oscale : nullptr;
   a.ncache_in = static_cast<const __nv_bfloat16 *>(c.ncache_in);
   a.ncache_out = static_cast<__nv_bfloat16 *>(c.ncache_out);
   a.nc_vec32 = (reinterpret_cast<uintptr_t>(c.ncache_out) & 31u) == 0 ? 1 : 0;
@@ -254,17 +261,19 @@ bool encode_activation_map(CUtensorMap *m, const void *base, int c, int w, int h
   return encode_act_map(m, base, c, w, h, t, n, box_w, box_h, box_c);
 }
 
-// 2-D bf16 tensor map over a weight image of `rows` rows of 64 channels
-// (128 bytes): boxes of box_rows rows, 128-byte swizzled.
-bool encode_weight_map(CUtensorMap *m, const void *img, long long rows, int box_rows) {
+// 2-D tensor map over a weight image of `rows` rows of 128 bytes (64 bf16
+// or 128 E4M3 channels): boxes of box_rows rows, 128-byte swizzled.
+bool encode_weight_map(CUtensorMap *m, const void *img, long long rows, int box_rows, bool e4m3) {
   auto fn = encode_fn();
   if (!fn || rows < 1 || box_rows < 1 || box_rows > 256) return false;
-  cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows)};
+  const cuuint64_t per_row = e4m3 ? 128 : 64;
+  cuuint64_t dims[2] = {per_row, static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {128};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(per_row), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(img), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = fn(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void *>(img), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -286,6 +295,7 @@ struct cc3d_plan {
   void *wraw;
   int kpad, thin_spec, nt, tmem_cols, sm_count, ctas_per_sm;
   float *bias, *gamma, *beta;
+  float *oscale;  // FP8: s_x * s_w[c] per output channel
   cc3d_stats st;
   std::mutex mu;
 };
@@ -314,6 +324,7 @@ void free_plan(cc3d_plan *p) {
   cudaFree(p->bias);
   cudaFree(p->gamma);
   cudaFree(p->beta);
+  cudaFree(p->oscale);
   delete p;
 }
 
@@ -359,6 +370,15 @@ cc3d_status check_desc(const cc3d_desc *d, int *variant) {
   if (d->dtype == CC3D_FP32) {
     if (d->epi != CC3D_EPI_BIAS || d->stride_t != 1) return CC3D_ERR_UNSUPPORTED;
     *variant = CC3D_VARIANT_FP32;
+    return CC3D_OK;
+  }
+  if (d->dtype == CC3D_FP8_E4M3) {
+    // FP8 operands on the tensor-core path: 128-channel chunks, per-channel
+    // weight scales and one activation scale, bias or residual epilogue
+    if (!d->w_scale || !(d->x_scale > 0.f)) return CC3D_ERR_INVALID_ARG;
+    if (d->c_in % 128 != 0 || d->c_out % 16 != 0 || d->kh != d->kw || s2 || rms)
+      return CC3D_ERR_UNSUPPORTED;
+    *variant = CC3D_VARIANT_UMMA;
     return CC3D_OK;
   }
   if (d->dtype != CC3D_BF16) return CC3D_ERR_INVALID_ARG;
@@ -523,13 +543,15 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
       // pipeline depths): a function of (n, c_in, c_out, h, w, epilogue,
       // max_t), never of a call's t.
       UmmaConfig &cfg = L.cfg;
+      const bool e4m3 = desc->dtype == CC3D_FP8_E4M3;
+      L.e4m3 = e4m3 ? 1 : 0;
       const int max_out = (desc->max_t - 1) / desc->stride_t + 1;  // largest call's frames
       const int kt_eff = L.s2 ? 9 : desc->kt, ks_eff = L.s2 ? 1 : desc->kh;
       const int h_out = desc->h / desc->stride_h, w_out = desc->w / desc->stride_w;
       if (!choose_umma_config(desc->n, desc->c_in, desc->c_out, h_out, w_out, kt_eff, ks_eff,
                               desc->epi == CC3D_EPI_BIAS_RMS_SILU ||
                                   desc->epi == CC3D_EPI_BIAS_RMS,
-                              max_out, L.sm_count, &cfg)) {
+                              max_out, L.sm_count, &cfg, e4m3)) {
         s = CC3D_ERR_UNSUPPORTED;
         goto fail;
       }
@@ -551,10 +573,22 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
       L.n_cc_sc = c_sc > 0 ? (c_sc + cfg.kc - 1) / cfg.kc : 0;
       const int conv_stages = taps * (desc->c_in / cfg.kc);
       const int stages = conv_stages + L.n_cc_sc;
-      const size_t bytes = sizeof(__nv_bfloat16) * desc->c_out * stages * cfg.kc;
+      // (a stage row is 128 bytes: 64 bf16 or 128 E4M3 channels per 64 / 128)
+      const size_t bytes =
+          static_cast<size_t>(desc->c_out) * stages * cfg.kc * (e4m3 ? 1 : sizeof(__nv_bfloat16));
       if (cudaMalloc(&p->wimg, bytes) != cudaSuccess) { s = CC3D_ERR_OOM; goto fail; }
-      e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(desc->weight), p->wimg,
-                             desc->c_out, desc->c_in, taps, cfg.nt, cfg.kc, cfg.pair, stages, 0, 0);
+      if (e4m3) {
+        // E4M3 weights, quantised here with the per-channel scales; the
+        // epilogue multiplies by s_x * s_w[c]
+        if ((s = copy_vec(&p->oscale, desc->w_scale, desc->c_out, false)) != CC3D_OK) goto fail;
+        e = launch_repack_umma_e4m3(static_cast<const __nv_bfloat16 *>(desc->weight), p->oscale,
+                                    p->wimg, desc->c_out, desc->c_in, taps, cfg.nt, cfg.pair, 0);
+        if (e == cudaSuccess) e = launch_scale_vector(p->oscale, desc->c_out, desc->x_scale, 0);
+      } else {
+        e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(desc->weight), p->wimg,
+                               desc->c_out, desc->c_in, taps, cfg.nt, cfg.kc, cfg.pair, stages, 0,
+                               0);
+      }
       if (e == cudaSuccess && c_sc > 0)
         e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(w_sc), p->wimg, desc->c_out,
                                c_sc, 1, cfg.nt, cfg.kc, cfg.pair, stages, conv_stages, 0);
@@ -563,7 +597,7 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
       // (a pair's CTA loads half of each MMA N-subtile's rows per box)
       if (cfg.pair && !encode_weight_map(&p->map_w, p->wimg,
                                          static_cast<long long>(desc->c_out) * stages,
-                                         cfg.nt / cfg.nh / 2)) {
+                                         cfg.nt / cfg.nh / 2, e4m3)) {
         s = CC3D_ERR_CUDA;
         goto fail;
       }
@@ -572,6 +606,7 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
       L.bias = p->bias;
       L.gamma = p->gamma;
       L.beta = p->beta;
+      L.oscale = p->oscale;
     }
   }
   *out = p;
@@ -627,10 +662,12 @@ static cc3d_status forward_impl(cc3d_plan *p, const void *x, int t, const void *
   if (!in_ok(x) || !aligned16(y) || !in_ok(cache_in) || !in_ok(cache_out) ||
       !aligned16(residual) || !aligned16(next_cache_in) || !aligned16(next_cache_out))
     return reject(CC3D_ERR_ALIGNMENT);
+  // bytes per element of x / caches and of y: fp32, bf16, or E4M3 in -> bf16 out
   const size_t esz = d.dtype == CC3D_FP32 ? 4 : 2;
+  const size_t in_esz = d.dtype == CC3D_FP8_E4M3 ? 1 : esz;
   const int front = d.kt - 1;
   const int t_out = (t - 1) / d.stride_t + 1;  // frames of y (and of residual)
-  const size_t in_frame = static_cast<size_t>(d.h) * d.w * d.c_in * esz;
+  const size_t in_frame = static_cast<size_t>(d.h) * d.w * d.c_in * in_esz;
   const size_t out_frame =
       static_cast<size_t>(d.h / d.stride_h) * (d.w / d.stride_w) * d.c_out * esz;
   const size_t x_bytes = in_frame * d.n * t, y_bytes = out_frame * d.n * t_out;
@@ -775,6 +812,16 @@ cc3d_status rmsnorm_silu(const void *x, const float *gamma, const float *beta, i
 cc3d_status rms_norm(const void *x, const float *gamma, const float *beta, int n, int t, int h,
                      int w, int c, void *y, const void *cache_in, void *cache_out, void *stream) {
   return rms_pass(x, gamma, beta, n, t, h, w, c, y, cache_in, cache_out, false, stream);
+}
+
+cc3d_status cc3d_quantize_e4m3(const void *x, size_t count, float scale, void *q, void *stream) {
+  if (!x || !q || count % 8 != 0 || !(scale > 0.f)) return CC3D_ERR_INVALID_ARG;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(q) & 7u) != 0) return CC3D_ERR_ALIGNMENT;
+  if (overlaps(x, count * 2, q, count)) return CC3D_ERR_ALIAS;
+  if (count == 0) return CC3D_OK;
+  return from_cuda(launch_quantize_e4m3(static_cast<const __nv_bfloat16 *>(x), count, scale,
+                                        static_cast<uint8_t *>(q),
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 cc3d_status cc3d_block_create2(int n, int c_in, int c_out, int h, int w, int max_t,

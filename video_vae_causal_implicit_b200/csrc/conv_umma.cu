@@ -80,10 +80,16 @@ struct SmemLayout {
 __host__ __device__ constexpr bool rms_epilogue(int epi) { return epi == 2 || epi == 3; }
 
 // Epilogue parameters staged in shared memory: bias[c_out] (and, for the
-// RMS epilogues, gamma[c_out], beta[c_out]).
-__host__ __device__ constexpr int param_floats(int c_out, int epi) {
-  return c_out * (rms_epilogue(epi) ? 3 : 1);
+// RMS epilogues, gamma[c_out], beta[c_out]; for FP8 operands the output
+// scale[c_out] = s_x * s_w[c_out]).
+__host__ __device__ constexpr int param_floats(int c_out, int epi, bool scaled) {
+  return c_out * ((rms_epilogue(epi) ? 3 : 1) + (scaled ? 1 : 0));
 }
+
+// A channel chunk of 128 means FP8 E4M3 operands: 128 one-byte channels
+// per 128-byte pixel row, the same bytes as a 64-channel bf16 chunk.
+__host__ __device__ constexpr bool is_e4m3(int kc) { return kc == 128; }
+__host__ __device__ constexpr int kc_bytes(int kc) { return is_e4m3(kc) ? kc : 2 * kc; }
 
 __host__ __device__ inline uint32_t round_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
@@ -92,7 +98,7 @@ __host__ __device__ inline uint32_t round_up(uint32_t v, uint32_t a) { return (v
 // image row of the halo spans whole 1024-byte swizzle atoms.  Other chunk
 // widths use 8-channel no-swizzle slabs (16-byte rows, 8 boxes for 64
 // channels: many more TMA requests per stage).
-__host__ __device__ constexpr bool uses_sw128(int kc) { return kc == 64; }
+__host__ __device__ constexpr bool uses_sw128(int kc) { return kc == 64 || kc == 128; }
 __host__ __device__ inline int halo_cols(int kc, int sub, int kw) {
   const int hw = kTW * sub + kw - 1;
   return uses_sw128(kc) ? (hw + 7) / 8 * 8 : hw;
@@ -112,7 +118,7 @@ __host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw
   }
   // (a CTA pair: this CTA's half of the N rows, 128-byte swizzled rows, so
   // a stage is a multiple of 1024 bytes as the swizzle atoms require)
-  L.b_stage = static_cast<uint32_t>(pair ? nt / 2 : nt) * kc * 2u;
+  L.b_stage = static_cast<uint32_t>(pair ? nt / 2 : nt) * static_cast<uint32_t>(kc_bytes(kc));
   L.b_slot = static_cast<uint32_t>(g_taps) * L.b_stage;
   L.na = na;
   L.nb = nb;
@@ -179,10 +185,10 @@ __device__ __forceinline__ void store_bf16x16(__nv_bfloat16 *dst, const uint4 &l
   }
 }
 
-// One pixel's 16-byte chunks [q0, q1) (8 bf16 channels each) from `src`
-// (null: zeros) to `dst`; both point at the pixel's first channel.
-__device__ __forceinline__ void copy_pixel_chunks(const __nv_bfloat16 *src, __nv_bfloat16 *dst,
-                                                  int q0, int q1) {
+// One pixel's 16-byte chunks [q0, q1) from `src` (null: zeros) to `dst`;
+// both point at the pixel's first byte.
+__device__ __forceinline__ void copy_pixel_chunks(const uint8_t *src, uint8_t *dst, int q0,
+                                                  int q1) {
   const uint4 *s = reinterpret_cast<const uint4 *>(src);
   uint4 *d = reinterpret_cast<uint4 *>(dst);
   int q = q0;
@@ -202,14 +208,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap map_cache,
                      const __grid_constant__ CUtensorMap map_w,
                      const __grid_constant__ CUtensorMap map_sc, UmmaArgs p) {
-  static_assert(!PAIR || (SUB == 1 && uses_sw128(KC)), "CTA pairs take 64-channel chunks");
+  static_assert(!PAIR || (SUB == 1 && uses_sw128(KC)), "CTA pairs take 128-byte chunks");
+  // K steps of one stage: 16 bf16 or 32 E4M3 elements (32 bytes) each
+  constexpr int kSteps = kc_bytes(KC) / 32;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // Align the dynamic shared window to 1 KiB ourselves (the attribute is a
   // request, not a guarantee).
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const SmemLayout L = make_layout(KC, p.nt, KS, KS, p.na, p.nb, SUB, p.g_taps, PAIR,
-                                   param_floats(p.c_out, p.epi));
+                                   param_floats(p.c_out, p.epi, p.oscale != nullptr));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
   uint64_t *full_a = bars;
   uint64_t *empty_a = full_a + L.na;
@@ -449,7 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && pair_leader) {
       // nh MMAs of N = nt / nh each cover the tile's nt columns
       const int nm = p.nt / p.nh;
-      const uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * kM : kM, nm);
+      const uint32_t idesc = is_e4m3(KC) ? idesc_e4m3_f32(PAIR ? 2 * kM : kM, nm)
+                                         : idesc_bf16_f32(PAIR ? 2 * kM : kM, nm);
       // B start of N-subtile 1 relative to 0: nm rows of 16 bytes in each
       // core-matrix slab, or (pair) nm / 2 rows of 128 swizzled bytes
       const uint32_t bhalf16 = PAIR ? static_cast<uint32_t>(nm / 2) * 8u : static_cast<uint32_t>(nm);
@@ -503,20 +512,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           auto issue = [&](auto nh_c) {
             constexpr int NH = decltype(nh_c)::value;
 #pragma unroll
-            for (int j = 0; j < KC / 16; ++j) {
+            for (int j = 0; j < kSteps; ++j) {
               // every sub-tile (8 pixels further along the halo row) and
               // every N-subtile reuses this weight stage
 #pragma unroll
               for (int sbt = 0; sbt < SUB; ++sbt) {
 #pragma unroll
                 for (int hh = 0; hh < NH; ++hh) {
-                  if constexpr (PAIR)
-                    umma_bf16_pair(d_tmem + hh * nm, a_tap + j * astep16,
-                                   b_st + j * bstep16 + hh * bhalf16, idesc, accumulate);
-                  else
-                    umma_bf16(d_tmem + sbt * p.nt + hh * nm,
-                              a_tap + sbt * kTW * pix16 + j * astep16,
-                              b_st + j * bstep16 + hh * bhalf16, idesc, accumulate);
+                  const uint32_t d = d_tmem + (PAIR ? 0 : sbt * p.nt) + hh * nm;
+                  const uint64_t a = a_tap + (PAIR ? 0 : sbt * kTW * pix16) + j * astep16;
+                  const uint64_t b = b_st + j * bstep16 + hh * bhalf16;
+                  if constexpr (PAIR && is_e4m3(KC)) umma_e4m3_pair(d, a, b, idesc, accumulate);
+                  else if constexpr (PAIR) umma_bf16_pair(d, a, b, idesc, accumulate);
+                  else if constexpr (is_e4m3(KC)) umma_e4m3(d, a, b, idesc, accumulate);
+                  else umma_bf16(d, a, b, idesc, accumulate);
                 }
               }
               accumulate = 1;
@@ -605,17 +614,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // bias (and gamma, beta) of every output channel, staged once: the
     // per-column reads below are then shared-memory broadcasts
     float *sp = reinterpret_cast<float *>(smem + L.p_off);
+    const int scale_at = rms_epilogue(p.epi) ? 3 * p.c_out : p.c_out;  // (FP8 output scale)
     for (int i = static_cast<int>(threadIdx.x) - 64; i < p.c_out; i += 32 * kEpiWarps) {
       sp[i] = p.bias[i];
       if (rms_epilogue(p.epi)) {
         sp[p.c_out + i] = p.gamma[i];
         sp[2 * p.c_out + i] = p.beta ? p.beta[i] : 0.f;
       }
+      if (p.oscale) sp[scale_at + i] = p.oscale[i];
     }
     named_barrier_sync(1, 32 * kEpiWarps);  // (the epilogue warps only)
     // (shared addresses of the three vectors)
     const uint32_t s_bias = smem_u32(sp), s_gamma = s_bias + 4u * static_cast<uint32_t>(p.c_out),
-                   s_beta = s_gamma + 4u * static_cast<uint32_t>(p.c_out);
+                   s_beta = s_gamma + 4u * static_cast<uint32_t>(p.c_out),
+                   s_scale = s_bias + 4u * static_cast<uint32_t>(scale_at);
     // elements of one input frame and one output frame
     const size_t in_frame = static_cast<size_t>(p.h) * p.w * p.c_in;
     const size_t out_frame = static_cast<size_t>(p.h) * p.w * p.c_out;
@@ -629,20 +641,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const size_t pix_img = static_cast<size_t>(h) * p.w + w;
         const int cf = p.cache_frames;
         if (p.cache_out && cf > 0) {
-          // cache_out[f] = concat(cache_in or zeros, x)[t_in + f]
-          const int q_all = p.c_in / 8;
+          // cache_out[f] = concat(cache_in or zeros, x)[t_in + f]  (bytes:
+          // in_esz per input element)
+          const size_t pix_bytes = static_cast<size_t>(p.c_in) * p.in_esz;
+          const size_t frame_bytes = in_frame * p.in_esz;
+          const int q_all = static_cast<int>(pix_bytes / 16);
           const int q0 = tc.ntile * q_all / p.n_ntiles;
           const int q1 = (tc.ntile + 1) * q_all / p.n_ntiles;
           for (int f = 0; f < cf; ++f) {
             const int src_f = p.t_in + f;  // index into the concatenation
-            const __nv_bfloat16 *src = nullptr;
+            const uint8_t *src = nullptr;
             if (src_f >= cf)
-              src = p.x_in + (static_cast<size_t>(tc.n) * p.t_in + (src_f - cf)) * in_frame;
+              src = p.x_in + (static_cast<size_t>(tc.n) * p.t_in + (src_f - cf)) * frame_bytes;
             else if (p.cache_in)
-              src = p.cache_in + (static_cast<size_t>(tc.n) * cf + src_f) * in_frame;
-            __nv_bfloat16 *dst = p.cache_out + (static_cast<size_t>(tc.n) * cf + f) * in_frame;
-            copy_pixel_chunks(src ? src + pix_img * p.c_in : nullptr, dst + pix_img * p.c_in, q0,
-                              q1);
+              src = p.cache_in + (static_cast<size_t>(tc.n) * cf + src_f) * frame_bytes;
+            uint8_t *dst = p.cache_out + (static_cast<size_t>(tc.n) * cf + f) * frame_bytes;
+            copy_pixel_chunks(src ? src + pix_img * pix_bytes : nullptr, dst + pix_img * pix_bytes,
+                              q0, q1);
           }
         }
         if (p.ncache_out && p.t < 2) {
@@ -655,7 +670,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                           : nullptr;
           __nv_bfloat16 *dst =
               p.ncache_out + static_cast<size_t>(tc.n) * 2 * out_frame + pix_img * p.c_out;
-          copy_pixel_chunks(src, dst, n0 / 8, (n0 + p.nt) / 8);
+          copy_pixel_chunks(reinterpret_cast<const uint8_t *>(src), reinterpret_cast<uint8_t *>(dst),
+                            n0 / 8, (n0 + p.nt) / 8);
         }
       }
     };
@@ -770,8 +786,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             {
               float bv[16];
               ld_param16(s_bias + 4u * static_cast<uint32_t>(n0 + j), bv);
+              if (p.oscale) {
+                // FP8 operands: the accumulator times s_x * s_w[c], then bias
+                float sv[16];
+                ld_param16(s_scale + 4u * static_cast<uint32_t>(n0 + j), sv);
 #pragma unroll
-              for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(raw[16 * u + i]) + bv[i];
+                for (int i = 0; i < 16; ++i) v[i] = fmaf(__uint_as_float(raw[16 * u + i]), sv[i], bv[i]);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(raw[16 * u + i]) + bv[i];
+              }
             }
             if (p.epi == 1 && valid) {
               const __nv_bfloat16 *rb0 = reinterpret_cast<const __nv_bfloat16 *>(&res[2 * u]);
@@ -937,7 +961,7 @@ long long frame_cost(const UmmaConfig &c, int n, int h, int w, int sm_count) {
 }  // namespace
 
 bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
-                        int max_t, int sm_count, UmmaConfig *cfg) {
+                        int max_t, int sm_count, UmmaConfig *cfg, bool e4m3) {
   // N tile: the largest split of c_out that is a multiple of 16 and at most
   // `cap` (256 is the tcgen05 N limit); the RMS epilogue needs the whole row
   // in one CTA.
@@ -956,14 +980,16 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
   // its taps into one fp32 accumulator in the same order: the shapes differ
   // in which CTA computes which outputs, not in how.
   UmmaConfig one;
-  one.kc = (c_in % 64 == 0) ? 64 : (c_in % 96 == 0) ? 96 : 32;
+  // channel chunk: 128 E4M3 channels, or 64 / 96 / 32 bf16 channels
+  if (e4m3 && c_in % 128 != 0) return false;
+  one.kc = e4m3 ? 128 : (c_in % 64 == 0) ? 64 : (c_in % 96 == 0) ? 96 : 32;
   one.sub = 1;
   one.pair = 0;
   one.nh = wide_rms ? 2 : 1;
   one.nt = wide_rms ? c_out : largest_nt(256);
   if (!one.nt) return false;
   one.n_ntiles = c_out / one.nt;
-  one.params = param_floats(c_out, rms_epi ? 2 : 0);
+  one.params = param_floats(c_out, rms_epi ? 2 : 0, e4m3);
   if (!finish_config(ks, kt, c_in, one)) return false;
   *cfg = one;
   // the tile shapes are compared on the plan's largest call: max_t frames
@@ -989,9 +1015,9 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
   }
   // A CTA pair (2-SM MMAs, M = 256): each SM holds half of every weight
   // stage, which cuts the shared-memory traffic per MMA enough to reach the
-  // tensor pipe's own rate.  64-channel chunks (the 128-byte swizzled halo
+  // tensor pipe's own rate.  128-byte chunks (the 128-byte swizzled halo
   // and weight rows).
-  if (one.kc == 64) {
+  if (uses_sw128(one.kc)) {
     UmmaConfig pr = one;
     pr.pair = 1;
     pr.sub = 2;  // the tile is two MMA tiles wide
@@ -1009,7 +1035,7 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
 
 int umma_tile_w() { return kTW; }
 int umma_halo_box_w(int kc, int sub, int kw) { return halo_cols(kc, sub, kw); }
-int umma_halo_box_c(int kc) { return uses_sw128(kc) ? 64 : 8; }
+int umma_halo_box_c(int kc) { return is_e4m3(kc) ? 128 : uses_sw128(kc) ? 64 : 8; }
 int umma_tile_h() { return kTH; }
 
 template <int KC, int KS>
@@ -1033,6 +1059,8 @@ cudaError_t umma_prepare() {
   if (e == cudaSuccess) e = set_smem_attr<64, 1>();
   if (e == cudaSuccess) e = set_smem_attr<32, 1>();
   if (e == cudaSuccess) e = set_smem_attr<96, 1>();
+  if (e == cudaSuccess) e = set_smem_attr<128, 3>();
+  if (e == cudaSuccess) e = set_smem_attr<128, 1>();
   return e;
 }
 
@@ -1062,6 +1090,8 @@ UmmaKernel umma_kernel_for(int kc, int ks, int sub, int pair) {
   CC3D_PICK(64, 1)
   CC3D_PICK(32, 1)
   CC3D_PICK(96, 1)
+  CC3D_PICK(128, 3)
+  CC3D_PICK(128, 1)
 #undef CC3D_PICK
   return nullptr;
 }
@@ -1106,11 +1136,12 @@ cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_ca
   if (args.g_taps != 1 && args.g_taps != args.kw) return cudaErrorInvalidValue;
   const size_t smem =
       umma_launch_smem(kc, args.nt, args.kh, args.na, args.nb, args.tmem_cols, args.sub,
-                       args.g_taps, args.pair, param_floats(args.c_out, args.epi));
+                       args.g_taps, args.pair,
+                       param_floats(args.c_out, args.epi, args.oscale != nullptr));
   if (smem > kSmemLimit || (args.sub != 1 && args.sub != 2) || args.nbuf < 1 || args.nbuf > 2 ||
       args.na < 1 || args.na > 32 || args.nb < 1 || args.nb > 32)
     return cudaErrorInvalidValue;
-  if (args.pair && (kc != 64 || args.sub != 2 || grid % 2 != 0 || args.nt % 16 != 0))
+  if (args.pair && (!uses_sw128(kc) || args.sub != 2 || grid % 2 != 0 || args.nt % 16 != 0))
     return cudaErrorInvalidValue;
   // nh MMA N-subtiles: each a valid MMA N (a multiple of 16, at most 256;
   // on a pair each CTA's half of it whole 8-row swizzle atoms)
@@ -1124,9 +1155,14 @@ cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_ca
       (args.c_sc > 0 && (args.b_resident || args.c_sc % 8 != 0 ||
                          args.n_cc_sc != (args.c_sc + kc - 1) / kc)))
     return cudaErrorInvalidValue;
+  // FP8 operands (128-channel chunks) come with their output scale and a
+  // bias or residual epilogue
+  if (is_e4m3(kc) != (args.oscale != nullptr) || (is_e4m3(kc) && rms_epilogue(args.epi)) ||
+      (args.in_esz != (is_e4m3(kc) ? 1 : 2)))
+    return cudaErrorInvalidValue;
   // the frame caches the epilogue writes: whole 16-byte chunks per pixel
-  if ((args.cache_out && (args.cache_frames < 1 || args.c_in % 8 != 0 || !args.x_in ||
-                          args.t_in < 1 || args.s2)) ||
+  if ((args.cache_out && (args.cache_frames < 1 || (args.c_in * args.in_esz) % 16 != 0 ||
+                          !args.x_in || args.t_in < 1 || args.s2)) ||
       (args.ncache_out && (!rms_epilogue(args.epi) || args.nt % 8 != 0)))
     return cudaErrorInvalidValue;
   UmmaKernel k = umma_kernel_for(kc, args.kh, args.sub, args.pair);

@@ -52,10 +52,12 @@ struct UmmaArgs {
   //   concat(cache_in or zeros, x_in), x_in having t_in frames;
   //   ncache_out [n][2][h][w][c_out] = the last two frames of concat(ncache_in
   //   or zeros, y) (the RMS epilogue's output history).
-  const __nv_bfloat16 *x_in;
-  const __nv_bfloat16 *cache_in;
-  __nv_bfloat16 *cache_out;
+  const uint8_t *x_in;
+  const uint8_t *cache_in;
+  uint8_t *cache_out;
   int cache_frames, t_in;
+  int in_esz;                     // bytes per input element: 2 (bf16) or 1 (FP8 E4M3)
+  const float *oscale;            // FP8 operands: [c_out] output scale s_x * s_w[c] (else null)
   const __nv_bfloat16 *ncache_in;
   __nv_bfloat16 *ncache_out;
   int nc_vec32;                   // 1: ncache_out is 32-byte aligned (256-bit stores)
@@ -68,8 +70,9 @@ struct UmmaConfig {
   int params;      // epilogue parameters staged in shared memory (floats)
   int b_resident;  // every weight stage resident in shared memory (nb of them)
 };
+// e4m3: FP8 E4M3 operands (128-channel chunks; c_in % 128 == 0).
 bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
-                        int max_t, int sm_count, UmmaConfig *cfg);
+                        int max_t, int sm_count, UmmaConfig *cfg, bool e4m3 = false);
 // CTA pairs that can be resident at once (cfg.pair), for sizing the grid;
 // 0 when the query fails.
 int umma_max_clusters(const UmmaConfig &cfg, int ks);
@@ -103,6 +106,20 @@ cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_ca
 cudaError_t launch_repack_umma(const __nv_bfloat16 *w, uint8_t *img, int c_out, int c_in,
                                int taps, int nt, int kc, int rows, int stages_per_ntile,
                                int stage0, cudaStream_t stream);
+
+// The same image for FP8 E4M3 weights (128-channel chunks, one byte per
+// channel): W[c_out][c_in][taps] / w_scale[c_out] rounded to E4M3 in fp32
+// (saturated to +-448); rows as for launch_repack_umma, one stage per
+// (tap, chunk), stages_per_ntile = taps * c_in / 128.
+cudaError_t launch_repack_umma_e4m3(const __nv_bfloat16 *w, const float *w_scale, uint8_t *img,
+                                    int c_out, int c_in, int taps, int nt, int rows,
+                                    cudaStream_t stream);
+// v[i] *= s for i < count (device vector).
+cudaError_t launch_scale_vector(float *v, int count, float s, cudaStream_t stream);
+// q[i] = E4M3(x[i] / scale) for i < count: bf16 in, one byte out, the
+// quotient in fp32, rounded to nearest even and saturated to +-448.
+cudaError_t launch_quantize_e4m3(const __nv_bfloat16 *x, size_t count, float scale, uint8_t *q,
+                                 cudaStream_t stream);
 
 // Thin first-layer conv (c_in small): weights to [tap*c_in padded to kpad][c_out]
 // image and the kernel itself.
@@ -162,6 +179,8 @@ struct UmmaLayer {
   int epi;                         // 0 bias, 1 bias + residual, 2 bias + RMS + SiLU, 3 bias + RMS
   int c_sc, n_cc_sc;               // fused 1x1x1 conv_shortcut (0: none)
   int sm_count, max_clusters;      // grid sizing (max_clusters: CTA pairs)
+  int e4m3;                        // FP8 E4M3 operands (x, caches, weights)
+  const float *oscale;             // e4m3: [c_out] output scale s_x * s_w[c]
   const uint8_t *wimg;             // re-tiled weights
   const CUtensorMap *map_w;        // the weights as 128-byte swizzled rows (pairs)
   const float *bias, *gamma, *beta;
@@ -197,8 +216,9 @@ int *device_status_word();
 // plain or 64 swizzled channels).
 bool encode_activation_map(CUtensorMap *m, const void *base, int c, int w, int h, int t, int n,
                            int box_w, int box_h, int box_c);
-// 2-D tensor map over a plain-rows weight image (rows of 64 bf16), boxes of
-// box_rows rows, 128-byte swizzled.
-bool encode_weight_map(CUtensorMap *m, const void *img, long long rows, int box_rows);
+// 2-D tensor map over a plain-rows weight image (rows of 128 bytes: 64 bf16,
+// or 128 E4M3 codes), boxes of box_rows rows, 128-byte swizzled.
+bool encode_weight_map(CUtensorMap *m, const void *img, long long rows, int box_rows,
+                       bool e4m3 = false);
 
 }  // namespace cc3d

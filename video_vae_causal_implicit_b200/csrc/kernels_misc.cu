@@ -64,6 +64,74 @@ __global__ void repack_umma_kernel(const __nv_bfloat16 *__restrict__ w, __nv_bfl
   }
 }
 
+// The FP8 E4M3 weight image: 128 one-byte channels per chunk, laid out like
+// repack_umma_kernel's (rows: [ntile][tap][cchunk][NT][128]; else no-swizzle
+// core matrices [ntile][tap][cchunk][8][NT][16]), each weight divided by its
+// output channel's scale in fp32 (an IEEE division) and rounded to E4M3.
+__global__ void repack_umma_e4m3_kernel(const __nv_bfloat16 *__restrict__ w,
+                                        const float *__restrict__ w_scale, uint8_t *img,
+                                        int c_out, int c_in, int taps, int nt, int rows) {
+  constexpr int kc = 128;
+  const int n_cc = c_in / kc;
+  const long long total = static_cast<long long>(c_out) * n_cc * kc * taps;
+  const long long stage_elems = static_cast<long long>(nt) * kc;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    long long r = i;
+    int e, nl, s;
+    if (rows) {
+      e = r % kc;
+      r /= kc;
+      nl = r % nt;
+      r /= nt;
+      s = 0;
+    } else {
+      e = r % 16;
+      r /= 16;
+      nl = r % nt;
+      r /= nt;
+      s = r % (kc / 16);
+      r /= (kc / 16);
+    }
+    const int cc = r % n_cc;
+    r /= n_cc;
+    const int tap = r % taps;
+    const int ntile = static_cast<int>(r / taps);
+    const int co = ntile * nt + nl;
+    const int ci = cc * kc + s * 16 + e;
+    const float q = __fdiv_rn(__bfloat162float(w[(static_cast<long long>(co) * c_in + ci) * taps + tap]),
+                              w_scale[co]);
+    const long long dst =
+        (static_cast<long long>(ntile) * taps * n_cc + tap * n_cc + cc) * stage_elems +
+        i % stage_elems;
+    img[dst] = static_cast<uint8_t>(pack_e4m3x2(q, 0.f) & 0xFFu);
+  }
+}
+
+__global__ void scale_vector_kernel(float *v, int count, float s) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < count) v[i] *= s;
+}
+
+// q = E4M3(x / scale), 8 elements per thread (16 bytes in, 8 out).
+__global__ void quantize_e4m3_kernel(const __nv_bfloat16 *__restrict__ x, long long groups,
+                                     float scale, uint8_t *__restrict__ q) {
+  for (long long g = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; g < groups;
+       g += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4 raw = __ldcs(reinterpret_cast<const uint4 *>(x) + g);
+    const __nv_bfloat16 *b = reinterpret_cast<const __nv_bfloat16 *>(&raw);
+    uint16_t h[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      h[k] = pack_e4m3x2(__fdiv_rn(__bfloat162float(b[2 * k]), scale),
+                         __fdiv_rn(__bfloat162float(b[2 * k + 1]), scale));
+    uint2 out;
+    out.x = static_cast<uint32_t>(h[0]) | (static_cast<uint32_t>(h[1]) << 16);
+    out.y = static_cast<uint32_t>(h[2]) | (static_cast<uint32_t>(h[3]) << 16);
+    __stcs(reinterpret_cast<uint2 *>(q) + g, out);
+  }
+}
+
 // out[b][i] = concat(cache_in[b] (frames), src[b] (t))[t + i], i < frames.
 // 16-byte path: each thread moves U chunks per pass, all loads issued before
 // the stores, so enough bytes are in flight to stream at HBM speed.
@@ -376,6 +444,35 @@ cudaError_t launch_repack_umma(const __nv_bfloat16 *w, uint8_t *img, int c_out, 
   repack_umma_kernel<<<grid_for(total, 256), 256, 0, stream>>>(
       w, reinterpret_cast<__nv_bfloat16 *>(img), c_out, c_in, taps, nt, kc, rows,
       stages_per_ntile, stage0);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_repack_umma_e4m3(const __nv_bfloat16 *w, const float *w_scale, uint8_t *img,
+                                    int c_out, int c_in, int taps, int nt, int rows,
+                                    cudaStream_t stream) {
+  if (c_in % 128 != 0 || nt < 1 || c_out % nt != 0) return cudaErrorInvalidValue;
+  const long long total = static_cast<long long>(c_out) * c_in * taps;
+  repack_umma_e4m3_kernel<<<grid_for(total, 256), 256, 0, stream>>>(w, w_scale, img, c_out, c_in,
+                                                                     taps, nt, rows);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scale_vector(float *v, int count, float s, cudaStream_t stream) {
+  scale_vector_kernel<<<(count + 255) / 256, 256, 0, stream>>>(v, count, s);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_e4m3(const __nv_bfloat16 *x, size_t count, float scale, uint8_t *q,
+                                 cudaStream_t stream) {
+  if (count % 8 != 0) return cudaErrorInvalidValue;
+  const long long groups = static_cast<long long>(count / 8);
+  long long g = (groups + 255) / 256;
+  if (g > 148LL * 16) g = 148LL * 16;
+  if (g < 1) g = 1;
+  quantize_e4m3_kernel<<<static_cast<int>(g), 256, 0, stream>>>(x, groups, scale, q);
   count_launch();
   return cudaGetLastError();
 }
