@@ -587,11 +587,99 @@ def run_sweep(args, dev, stream, peaks, flush_l2, full=False):
         "ms": ms, "tflops": fl / ms / 1e9, "frac": fl / ms / 1e9 / peaks["bf16_tflops"],
         "hbm_gbs": byts / ms / 1e6, "hbm_frac": byts / ms / 1e6 / peaks["hbm_gbs"]}
     del ps, xs, ys
+    # the downsample path as the page draws it: WanRMS_norm, the stride-2
+    # conv, WanRMS_norm (the second one in the conv's epilogue)
+    T, H, W, cc = 17, 480, 832, 96
+    xs = torch.randn((1, T, H, W, cc), generator=g, device=dev).to(torch.bfloat16)
+    ga = synth.uniform((cc,), 0.5, 1.5, 3).to(dev)
+    gb = synth.uniform((cc,), 0.5, 1.5, 4).to(dev)
+    ps = cc3d.Plan(ws, bs, h=H, w=W, max_t=T, pad=(0, 0), stride_hw=2, epi=cc3d.EPI_BIAS_RMS,
+                   gamma=gb)
+    xa = torch.empty_like(xs)
+    ys = torch.empty((1, T, H // 2, W // 2, cc), dtype=torch.bfloat16, device=dev)
+
+    def down_path():
+        cc3d.rms(xs, ga, xa)
+        ps.forward(xa, ys)
+
+    ms = timed(down_path, flush=True)
+    byts = 3 * xs.numel() * 2 + ys.numel() * 2  # norm r/w, conv r, conv w
+    out[f"downsample_path_rms_s2conv_rms_c{cc}_{T}x{H}x{W}"] = {
+        "ms": ms, "hbm_gbs": byts / ms / 1e6, "hbm_frac": byts / ms / 1e6 / peaks["hbm_gbs"],
+        "tflops": fl / ms / 1e9}
+    del ps, xs, ys, xa
+    # FP8 (E4M3) operands: the config-2 step (whole sequence + 5 one-frame
+    # chunks) and config 5's largest 384-channel row, against the fp8 peak
+    # (the measured bf16 peak x the nominal fp8 / bf16 ratio of 2)
+    fp8_peak = 2 * peaks["bf16_tflops"]
+    c2, T2, H2, W2 = C2["c"], C2["t"], C2["h"], C2["w"]
+    case = synth.conv_case(c2, c2, T2, H2, W2)
+    w8 = case["w"].to(dev)
+    s_w = (w8.float().abs().reshape(c2, -1).amax(dim=1) / 448.0).contiguous()
+    xb = synth.ndhwc(case["x"]).to(dev)
+    s_x = float(xb.float().abs().max()) / 448.0
+    p8 = cc3d.Plan(w8, case["b"].to(dev), h=H2, w=W2, max_t=T2, dtype=cc3d.FP8_E4M3,
+                   w_scale=s_w, x_scale=s_x)
+    xq = torch.empty(xb.shape, dtype=torch.uint8, device=dev)
+    cc3d.quantize_e4m3(xb, s_x, xq)
+    y8 = torch.empty((1, T2, H2, W2, c2), dtype=torch.bfloat16, device=dev)
+    xq1 = [xq[:, k:k + 1].contiguous() for k in range(T2)]
+    y81 = [torch.empty((1, 1, H2, W2, c2), dtype=torch.bfloat16, device=dev) for _ in range(T2)]
+    c8 = [torch.empty((1, 2, H2, W2, c2), dtype=torch.uint8, device=dev) for _ in range(2)]
+
+    def fp8_step():
+        p8.forward(xq, y8)
+        cache = None
+        for k in range(T2):
+            p8.forward(xq1[k], y81[k], t=1, cache_in=cache, cache_out=c8[k % 2])
+            cache = c8[k % 2]
+
+    fp8_step()
+    gr8 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr8):
+        fp8_step()
+    ms = timed(gr8.replay, flush=True)
+    fl = 2 * conv_flop(1, c2, c2, T2, H2, W2)
+    out["fp8_cfg2_step_whole_plus_5_chunks"] = {
+        "ms": ms, "tflops": fl / ms / 1e9, "frac_of_fp8_peak": fl / ms / 1e9 / fp8_peak,
+        "fp8_peak_basis": "2 x bf16 (" + peaks["source"] + ")"}
+    del gr8, p8, xq, y8, xq1, y81, c8
+    H5, W5 = 360, 640
+    x5 = torch.randn((1, 21, H5, W5, 384), generator=g, device=dev).to(torch.bfloat16)
+    w5 = synth.kaiming_uniform(384, 384, (3, 3, 3), 1).to(dev)
+    s_w5 = (w5.float().abs().reshape(384, -1).amax(dim=1) / 448.0).contiguous()
+    s_x5 = float(x5.float().abs().max()) / 448.0
+    x5q = torch.empty(x5.shape, dtype=torch.uint8, device=dev)
+    cc3d.quantize_e4m3(x5, s_x5, x5q)
+    del x5
+    p5 = cc3d.Plan(w5, synth.uniform((384,), -0.1, 0.1, 2).to(dev), h=H5, w=W5, max_t=1,
+                   dtype=cc3d.FP8_E4M3, w_scale=s_w5, x_scale=s_x5)
+    y5 = torch.empty((1, 21, H5, W5, 384), dtype=torch.bfloat16, device=dev)
+    xs5 = [x5q[:, k:k + 1] for k in range(21)]
+    ys5 = [y5[:, k:k + 1] for k in range(21)]
+    cb5 = [torch.empty((1, 2, H5, W5, 384), dtype=torch.uint8, device=dev) for _ in range(2)]
+
+    def run5():
+        cache = None
+        for k in range(21):
+            p5.forward(xs5[k], ys5[k], t=1, cache_in=cache, cache_out=cb5[k % 2])
+            cache = cb5[k % 2]
+
+    run5()
+    gr5 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr5):
+        run5()
+    ms = timed(gr5.replay, flush=True)
+    fl = conv_flop(1, 384, 384, 21, H5, W5)
+    out["fp8_cfg5_c384_360x640_21x1frame"] = {
+        "ms": ms, "tflops": fl / ms / 1e9, "frac_of_fp8_peak": fl / ms / 1e9 / fp8_peak}
+    del gr5, p5, x5q, y5, cb5
     # the encoder's other residual blocks (§8(f) NEXT-2): the two that change
     # the channel count (the 1x1x1 conv_shortcut fused into conv2) and a
-    # 384-channel one (RMS_norm after conv1 in its own pass), whole sequence
+    # 384-channel one (conv1's RMS_norm + SiLU fused into its epilogue as two
+    # N = 192 MMAs per K step), whole sequence; the 384-channel one always
     for (ci, co, T, H, W) in (((96, 192, 17, 240, 416), (192, 384, 9, 120, 208),
-                               (384, 384, 5, 60, 104)) if full else ()):
+                               (384, 384, 5, 60, 104)) if full else ((384, 384, 5, 60, 104),)):
         xb = torch.randn((1, T, H, W, ci), generator=g, device=dev).to(torch.bfloat16)
         wts = dict(w1=synth.kaiming_uniform(co, ci, (3, 3, 3), 11),
                    b1=synth.uniform((co,), -0.1, 0.1, 12), g1=synth.uniform((ci,), 0.5, 1.5, 13),

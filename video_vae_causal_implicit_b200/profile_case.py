@@ -5,7 +5,7 @@
 Cases (seeded synthetic inputs, generated on the device):
   c2      384 -> 384 causal conv, whole sequence, x[1,384,5,30,52]
   c2s     the same as 5 one-frame chunks with a 2-frame cache, planned for
-          one-frame calls (max_t = 1: the temporal split)
+          one-frame calls (max_t = 1)
   c2c     the 5 one-frame chunks with the whole-sequence plan (max_t = 5), as
           in the benchmark step
   c3a     3 -> 96 causal conv on x[1,3,17,480,832]
@@ -20,6 +20,9 @@ Cases (seeded synthetic inputs, generated on the device):
           conv, 96 channels, x[1,96,17,480,832] -> 240 x 416
   blk96   the encoder's channel-changing block 96 -> 192 (conv_shortcut fused
           into conv2) on x[1,96,17,240,416]
+  blk384  a 384-channel residual block on x[1,384,5,60,104] (conv1's RMS_norm
+          + SiLU in its epilogue, two N = 192 MMAs per K step)
+  c2f8    the 384 -> 384 conv of c2 on FP8 E4M3 operands
 Prints nothing but a final "ok"; timing comes from the profiler.
 """
 from __future__ import annotations
@@ -56,6 +59,10 @@ def build_case(name, dev):
         c, T, H, W = 96, 17, 480, 832
     elif name == "blk96":
         c, T, H, W = 96, 17, 240, 416
+    elif name == "blk384":
+        c, T, H, W = 384, 5, 60, 104
+    elif name == "c2f8":
+        c, T, H, W = 384, 5, 30, 52
     else:
         raise SystemExit(f"unknown case {name}")
     x = _rand((1, T, H, W, c), dev)
@@ -86,6 +93,24 @@ def build_case(name, dev):
         blk = cc3d.Block(**{k: v.to(dev) for k, v in wts.items()}, h=H, w=W, max_t=T)
         y = torch.empty((1, T, H, W, co), dtype=torch.bfloat16, device=dev)
         return (lambda: blk.forward(x, y)), [blk]
+    if name == "blk384":
+        wts = dict(w1=synth.kaiming_uniform(c, c, (3, 3, 3), 1),
+                   b1=synth.uniform((c,), -0.1, 0.1, 2), g1=synth.uniform((c,), 0.5, 1.5, 3),
+                   w2=synth.kaiming_uniform(c, c, (3, 3, 3), 4),
+                   b2=synth.uniform((c,), -0.1, 0.1, 5), g2=synth.uniform((c,), 0.5, 1.5, 6))
+        blk = cc3d.Block(**{k: v.to(dev) for k, v in wts.items()}, h=H, w=W, max_t=T)
+        y = torch.empty_like(x)
+        return (lambda: blk.forward(x, y)), [blk]
+    if name == "c2f8":
+        wt = synth.kaiming_uniform(c, c, (3, 3, 3), 1).to(dev)
+        s_w = (wt.float().abs().reshape(c, -1).amax(dim=1) / 448.0).contiguous()
+        s_x = float(x.float().abs().max()) / 448.0
+        plan = cc3d.Plan(wt, synth.uniform((c,), -0.1, 0.1, 2).to(dev), h=H, w=W, max_t=T,
+                         dtype=cc3d.FP8_E4M3, w_scale=s_w, x_scale=s_x)
+        xq = torch.empty(x.shape, dtype=torch.uint8, device=dev)
+        cc3d.quantize_e4m3(x, s_x, xq)
+        y = torch.empty_like(x)
+        return (lambda: plan.forward(xq, y)), [plan, xq]
     if name in ("tc192", "tc384"):
         wt = synth.kaiming_uniform(c, c, (3, 1, 1), 1).to(dev)
         b = synth.uniform((c,), -0.1, 0.1, 2).to(dev)
