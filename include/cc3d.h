@@ -156,6 +156,11 @@ typedef struct {
   int w_resident;          /* 1: the weights stay in shared memory for the
                               whole launch (short K, one N tile), 0: they
                               stream through a ring, once per tile          */
+  int row_ctas;            /* CTAs that share one output pixel's channels: 1,
+                              or 2 when an RMS row wider than 256 channels
+                              is split over a cluster of two CTAs (each one
+                              half, the row's sum of squares exchanged
+                              between them through shared memory)          */
 } cc3d_stats;
 
 typedef struct cc3d_plan cc3d_plan;

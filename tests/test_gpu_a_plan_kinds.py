@@ -19,7 +19,8 @@ pytestmark = pytest.mark.gpu
 def _shape(plan):
     st = plan.stats()
     return dict(variant=st.variant, mma_ctas=st.mma_ctas, tile_w=st.tile_w,
-                resident=st.w_resident, n_tile=st.n_tile, k_split=st.k_split)
+                resident=st.w_resident, n_tile=st.n_tile, k_split=st.k_split,
+                row_ctas=st.row_ctas)
 
 
 def _conv(n, cin, cout, t, h, w, k=(3, 3, 3), seed=0, stride_t=1, cache=False, **plan_kw):
@@ -87,6 +88,26 @@ def test_rms_epilogue_with_next_cache():
         oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], case["b"].double().numpy()))
     ref = oracle.rms_norm(conv, g.double().numpy(), silu=True)
     assert_close_bf16(ncthw_np(y), ref, "rms epilogue")
+
+
+def test_rms_row_split_over_a_cluster():
+    """A 320-channel RMS row: each CTA of a cluster takes 160 channels of
+    the same pixels, and the two swap each row's partial sum of squares."""
+    n, cin, cout, t, h, w = 1, 64, 320, 2, 16, 20
+    g = synth.uniform((cout,), 0.5, 1.5, 10)
+    case = synth.conv_case(cin, cout, t, h, w, n=n, seed_base=11)
+    plan = cc3d.Plan(to_dev(case["w"]), to_dev(case["b"]), n=n, h=h, w=w, max_t=t,
+                     epi=cc3d.EPI_BIAS_RMS_SILU, gamma=to_dev(g))
+    got = _shape(plan)
+    assert (got["row_ctas"], got["n_tile"], got["mma_ctas"]) == (2, 160, 1), got
+    x = to_dev(synth.ndhwc(case["x"]))
+    y = torch.empty((n, t, h, w, cout), dtype=torch.bfloat16, device="cuda")
+    plan.forward(x, y)
+    cc3d.sync_status()
+    conv = oracle.round_bf16_array(
+        oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], case["b"].double().numpy()))
+    ref = oracle.rms_norm(conv, g.double().numpy(), silu=True)
+    assert_close_bf16(ncthw_np(y), ref, "rms row split over a cluster")
 
 
 def test_thin_first_layer():

@@ -1,14 +1,17 @@
 """GPU parity of the RMS_norm epilogues on rows wider than one MMA (up to
-512 channels: the CTA tile holds the whole row as two MMAs of half the
-width per K step), of the RMS_norm epilogue without SiLU, of the
+512 channels: the two CTAs of a cluster each hold one half of the row for
+the same pixels and swap each row's partial sum of squares), of the RMS_norm
+epilogue without SiLU, of the
 stand-alone RMS_norm without SiLU, and of the downsample path they make
 up ("Cosmos3 Wan VAE", §10.5: WanRMS_norm, then ZeroPad2d + 3x3 stride-2
 Conv2d per frame, then WanRMS_norm).  References round a conv's output to
 bf16 before its RMS_norm, as the block's reading does."""
+import numpy as np
 import pytest
 import torch
 
 import oracle
+from tests import sampled
 from tests.parity import assert_close_bf16, ncthw_np, to_dev
 from video_vae_causal_implicit_b200 import cc3d, synth
 
@@ -20,27 +23,29 @@ def _rms_ref(conv, g, beta=None, silu=True):
                            None if beta is None else beta.double().numpy(), silu=silu)
 
 
-# (n, c_in, c_out, t, h, w, epi, mma_ctas)
+# (n, c_in, c_out, t, h, w, epi)
 WIDE = [
-    (1, 384, 384, 2, 16, 20, cc3d.EPI_BIAS_RMS_SILU, 2),
-    (1, 96, 384, 2, 16, 20, cc3d.EPI_BIAS_RMS_SILU, 1),
-    (2, 32, 320, 2, 12, 16, cc3d.EPI_BIAS_RMS_SILU, None),
-    (1, 384, 384, 3, 10, 14, cc3d.EPI_BIAS_RMS, 2),
-    (1, 64, 64, 2, 17, 20, cc3d.EPI_BIAS_RMS, None),
+    (1, 384, 384, 2, 16, 20, cc3d.EPI_BIAS_RMS_SILU),
+    (1, 96, 384, 2, 16, 20, cc3d.EPI_BIAS_RMS_SILU),
+    (2, 32, 320, 2, 12, 16, cc3d.EPI_BIAS_RMS_SILU),
+    (1, 64, 512, 2, 9, 17, cc3d.EPI_BIAS_RMS_SILU),
+    (1, 384, 384, 3, 10, 14, cc3d.EPI_BIAS_RMS),
+    (1, 64, 64, 2, 17, 20, cc3d.EPI_BIAS_RMS),
 ]
 
 
-@pytest.mark.parametrize("n,cin,cout,t,h,w,epi,ctas", WIDE)
-def test_rms_epilogues_match_oracle(n, cin, cout, t, h, w, epi, ctas):
+@pytest.mark.parametrize("n,cin,cout,t,h,w,epi", WIDE)
+def test_rms_epilogues_match_oracle(n, cin, cout, t, h, w, epi):
     case = synth.conv_case(cin, cout, t, h, w, n=n, seed_base=cin + cout + epi)
     g = synth.uniform((cout,), 0.5, 1.5, 70)
     be = synth.uniform((cout,), -0.2, 0.2, 71)
     plan = cc3d.Plan(to_dev(case["w"]), to_dev(case["b"]), n=n, h=h, w=w, max_t=t, epi=epi,
                      gamma=to_dev(g), beta=to_dev(be))
     st = plan.stats()
-    assert st.n_tile == cout, "one CTA tile owns the whole row"
-    if ctas is not None:
-        assert st.mma_ctas == ctas
+    # rows up to 256 channels: one CTA owns the whole row; wider: each CTA
+    # of a cluster one half
+    assert st.row_ctas == (2 if cout > 256 else 1)
+    assert st.n_tile * st.row_ctas == cout
     x = to_dev(synth.ndhwc(case["x"]))
     y = torch.empty((n, t, h, w, cout), dtype=torch.bfloat16, device="cuda")
     nc_in = to_dev(synth.ndhwc(synth.normal((n, cout, 2, h, w), 72)))
@@ -51,6 +56,41 @@ def test_rms_epilogues_match_oracle(n, cin, cout, t, h, w, epi, ctas):
     conv = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], case["b"].double().numpy())
     ref = _rms_ref(conv, g, be, silu=epi == cc3d.EPI_BIAS_RMS_SILU)
     assert_close_bf16(ncthw_np(y), ref, f"rms epilogue {cin}->{cout} epi{epi}")
+
+
+def test_wide_rms_many_tiles_per_cluster():
+    """The block's 384-channel shape, [1, 384, 5, 60, 104]: each cluster
+    takes several M tiles in turn, so both exchange slots and both phases of
+    their barriers are reused; checked at seeded voxels of every frame plus
+    every border pixel of the last frame, against the oracle's conv at those
+    voxels (all channels), rounded to bf16 and RMS-normalised."""
+    n, c, t, h, w = 1, 384, 5, 60, 104
+    case = synth.conv_case(c, c, t, h, w, n=n, seed_base=84)
+    g = synth.uniform((c,), 0.5, 1.5, 85)
+    plan = cc3d.Plan(to_dev(case["w"]), to_dev(case["b"]), n=n, h=h, w=w, max_t=t,
+                     epi=cc3d.EPI_BIAS_RMS_SILU, gamma=to_dev(g))
+    assert plan.stats().row_ctas == 2
+    x = to_dev(synth.ndhwc(case["x"]))
+    y = torch.empty((n, t, h, w, c), dtype=torch.bfloat16, device="cuda")
+    plan.forward(x, y)
+    cc3d.sync_status()
+    vox = sampled.random_voxels(t, h, w, 400, 86)
+    vox[t - 1] = np.concatenate([vox.get(t - 1, np.zeros((0, 2), np.int32)),
+                                 sampled.border_pixels(h, w)])
+    got, ref = [], []
+    for f, hw in sorted(vox.items()):
+        s = max(0, f - 2)
+        pts = np.concatenate([np.zeros((len(hw), 1), np.int32),
+                              np.full((len(hw), 1), f - s, np.int32), hw], axis=1)
+        conv = oracle.causal_conv3d_points(synth.ncthw_view(x[:1, s:f + 1].cpu()), case["w"],
+                                           case["b"].double().numpy(), None, pts)
+        # [P, C] -> [1, C, 1, 1, P]: the RMS_norm over channels of each voxel
+        conv5 = np.ascontiguousarray(conv.T.reshape(1, c, 1, 1, -1))
+        ref.append(_rms_ref(conv5, g).reshape(c, -1).T)
+        ih = torch.as_tensor(hw[:, 0], dtype=torch.long, device="cuda")
+        iw = torch.as_tensor(hw[:, 1], dtype=torch.long, device="cuda")
+        got.append(y[0, f][ih, iw].double().cpu().numpy())
+    assert_close_bf16(np.concatenate(got), np.concatenate(ref), "wide rms, block shape")
 
 
 def test_wide_rms_streaming_is_bitwise_whole():

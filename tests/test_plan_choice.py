@@ -17,8 +17,8 @@ from video_vae_causal_implicit_b200 import cc3d
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(ROOT, "video_vae_causal_implicit_b200", "csrc")
-FIELDS = ("ok", "kc", "nt", "n_ntiles", "nh", "sub", "nbuf", "g_taps", "pair", "na", "nb",
-          "tmem_cols", "ctas_per_sm", "params", "b_resident", "smem")
+FIELDS = ("ok", "kc", "nt", "n_ntiles", "sub", "nbuf", "g_taps", "pair", "na", "nb",
+          "tmem_cols", "ctas_per_sm", "params", "b_resident", "xs", "smem")
 SMEM_MAX = 227 * 1024
 
 
@@ -73,11 +73,17 @@ def test_every_plan_fits_the_sm(probe):
         assert co % p["nt"] == 0 and p["nt"] % 16 == 0, (c, p)
         assert p["n_ntiles"] * p["nt"] == co, (c, p)
         assert ci % p["kc"] == 0 and p["kc"] in (32, 64, 96), (c, p)
-        if rms:
-            assert p["nt"] == co, (c, p)  # the RMS epilogue needs the whole row
-            assert p["nh"] == (2 if co > 256 else 1), (c, p)
+        if rms and co <= 256:
+            assert p["nt"] == co and p["xs"] == 0, (c, p)  # the whole row
+        elif rms:
+            # a row wider than one MMA: its halves on the two CTAs of a
+            # cluster, each with two accumulator buffers
+            assert (p["xs"], p["nt"], p["n_ntiles"]) == (2, co // 2, 2), (c, p)
+            assert p["pair"] == 0 and p["sub"] == 1 and p["nbuf"] == 2, (c, p)
+        else:
+            assert p["xs"] == 0, (c, p)
         assert p["params"] == co * (3 if rms else 1), (c, p)
-        assert p["nt"] // p["nh"] <= 256, (c, p)
+        assert p["nt"] <= 256, (c, p)
         assert 1 <= p["ctas_per_sm"] <= 2, (c, p)
 
 

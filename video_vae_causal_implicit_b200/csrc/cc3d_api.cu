@@ -219,7 +219,7 @@ cudaError_t run_umma_layer(const UmmaLayer &L, const UmmaCall &c, int *status,
   a.b_resident = cfg.b_resident;
   a.c_sc = L.c_sc;
   a.n_cc_sc = L.n_cc_sc;
-  a.nt = cfg.nt; a.n_ntiles = cfg.n_ntiles; a.nh = cfg.nh;
+  a.nt = cfg.nt; a.n_ntiles = cfg.n_ntiles;
   a.sub = cfg.sub; a.nbuf = cfg.nbuf; a.g_taps = cfg.g_taps; a.pair = cfg.pair;
   a.tiles_w = (w_out + tile_w - 1) / tile_w;
   a.tiles_h = (h_out + umma_tile_h() - 1) / umma_tile_h();
@@ -237,12 +237,15 @@ cudaError_t run_umma_layer(const UmmaLayer &L, const UmmaCall &c, int *status,
   a.ncache_in = static_cast<const __nv_bfloat16 *>(c.ncache_in);
   a.ncache_out = static_cast<__nv_bfloat16 *>(c.ncache_out);
   a.nc_vec32 = (reinterpret_cast<uintptr_t>(c.ncache_out) & 31u) == 0 ? 1 : 0;
+  a.xs = cfg.xs;
   const uint64_t tiles = static_cast<uint64_t>(L.n) * t_out * a.tiles_h * a.tiles_w * a.n_ntiles;
   uint64_t grid;
-  if (cfg.pair) {
-    // one pair per tile, at most as many pairs as fit at once
+  if (cfg.pair || cfg.xs == 2) {
+    // one cluster per tile (pair) or per M tile (xs: its two N tiles), at
+    // most as many clusters as fit at once
+    const uint64_t need = cfg.pair ? tiles : tiles / 2;
     const uint64_t clusters = static_cast<uint64_t>(L.max_clusters);
-    grid = (tiles < clusters ? tiles : clusters) * 2;
+    grid = (need < clusters ? need : clusters) * 2;
   } else {
     const uint64_t slots = static_cast<uint64_t>(L.sm_count) * cfg.ctas_per_sm;
     grid = tiles < slots ? tiles : slots;
@@ -463,6 +466,7 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
   p->st.variant = variant;
   p->st.k_split = 1;
   p->st.mma_ctas = 1;
+  p->st.row_ctas = 1;
   const int taps = desc->kt * desc->kh * desc->kw;
   cudaError_t e = cudaSuccess;
   if ((s = copy_vec(&p->bias, desc->bias, desc->c_out, true)) != CC3D_OK) goto fail;
@@ -555,7 +559,7 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
         s = CC3D_ERR_UNSUPPORTED;
         goto fail;
       }
-      if (cfg.pair) {
+      if (cfg.pair || cfg.xs == 2) {
         L.max_clusters = umma_max_clusters(cfg, ks_eff);
         if (L.max_clusters < 1) { s = CC3D_ERR_CUDA; goto fail; }
       }
@@ -565,6 +569,7 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
       p->st.k_chunk = cfg.kc;
       p->st.k_split = 1;
       p->st.mma_ctas = cfg.pair ? 2 : 1;
+      p->st.row_ctas = cfg.xs == 2 ? 2 : 1;
       p->st.w_resident = cfg.b_resident;
       // weight image: per N tile, the conv's taps * c_in / kc stages, then the
       // shortcut's ceil(c_sc / kc) (its channels past c_sc zero)
@@ -597,7 +602,7 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
       // (a pair's CTA loads half of each MMA N-subtile's rows per box)
       if (cfg.pair && !encode_weight_map(&p->map_w, p->wimg,
                                          static_cast<long long>(desc->c_out) * stages,
-                                         cfg.nt / cfg.nh / 2, e4m3)) {
+                                         cfg.nt / 2, e4m3)) {
         s = CC3D_ERR_CUDA;
         goto fail;
       }

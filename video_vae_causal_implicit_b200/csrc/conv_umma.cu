@@ -72,9 +72,14 @@ constexpr size_t kSmemLimit = 227 * 1024;
 constexpr unsigned long long kDrainLimitNs = 100ull * 1000000ull;
 
 struct SmemLayout {
-  uint32_t a_off, a_stage, slab, b_off, b_stage, b_slot, bar_off, p_off, total;
+  uint32_t a_off, a_stage, slab, b_off, b_stage, b_slot, x_off, bar_off, p_off, total;
   int na, nb;
 };
+
+// A row split over the two CTAs of a cluster (xs = 2): each epilogue warp
+// receives its 32 rows' partial sums of squares from the peer into one of
+// two slots (tile parity).
+constexpr uint32_t kXsBytes = 2u * 4u * 32u * 4u;
 
 // RMS_norm epilogues: 2 with SiLU after it, 3 without.
 __host__ __device__ constexpr bool rms_epilogue(int epi) { return epi == 2 || epi == 3; }
@@ -104,9 +109,11 @@ __host__ __device__ inline int halo_cols(int kc, int sub, int kw) {
   return uses_sw128(kc) ? (hw + 7) / 8 * 8 : hw;
 }
 
-// g_taps: weight stages (taps) per B slot.
+// g_taps: weight stages (taps) per B slot; xs: 2 when a row is split over
+// the two CTAs of a cluster.
 __host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw, int na, int nb,
-                                                  int sub, int g_taps, bool pair, int params) {
+                                                  int sub, int g_taps, bool pair, int params,
+                                                  int xs) {
   SmemLayout L;
   const uint32_t hh = kTH + kh - 1, hw = static_cast<uint32_t>(halo_cols(kc, sub, kw));
   if (uses_sw128(kc)) {
@@ -124,22 +131,17 @@ __host__ __device__ inline SmemLayout make_layout(int kc, int nt, int kh, int kw
   L.nb = nb;
   L.a_off = 0;
   L.b_off = round_up(L.a_off + na * L.a_stage, 1024u);
-  L.bar_off = round_up(L.b_off + nb * L.b_slot, 64u);
+  L.x_off = round_up(L.b_off + nb * L.b_slot, 128u);
+  L.bar_off = round_up(L.x_off + (xs == 2 ? kXsBytes : 0u), 64u);
   // full_a, empty_a, full_b, empty_b, acc_full[2], acc_empty[2], drain,
-  // tmem slot
-  L.p_off = round_up(L.bar_off + 8u * (2 * na + 2 * nb + 5) + 16u, 16u);
+  // (xs: x_full[2][4]), tmem slot
+  L.p_off = round_up(L.bar_off + 8u * (2 * na + 2 * nb + 5 + (xs == 2 ? 8 : 0)) + 16u, 16u);
   L.total = L.p_off + 4u * static_cast<uint32_t>(params);
   return L;
 }
 
 struct TileCoord {
   int ntile, n, t, h0, w0;
-};
-
-// A compile-time int for generic lambdas.
-template <int V>
-struct IntConst {
-  static constexpr int value = V;
 };
 
 // Tile order: N tile fastest (CTAs sharing an input halo run together),
@@ -217,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const SmemLayout L = make_layout(KC, p.nt, KS, KS, p.na, p.nb, SUB, p.g_taps, PAIR,
-                                   param_floats(p.c_out, p.epi, p.oscale != nullptr));
+                                   param_floats(p.c_out, p.epi, p.oscale != nullptr), p.xs);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
   uint64_t *full_a = bars;
   uint64_t *empty_a = full_a + L.na;
@@ -226,16 +228,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *acc_full = empty_b + L.nb;   // [2]
   uint64_t *acc_empty = acc_full + 2;    // [2]
   uint64_t *drain = acc_empty + 2;       // MMA completion before TMEM is freed
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  uint64_t *x_full = drain + 1;          // xs: [tile parity][epilogue warp]
+  const bool xs = p.xs == 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(x_full + (xs ? 8 : 0));
 
   // With PAIR, a cluster of two CTAs (on one SM pair) takes a 16 x 16 pixel
   // tile: CTA `rank` holds the 8 x 16 half at columns 8 * rank and half of
   // each weight stage's N rows, and the leader (rank 0) issues M = 256
   // tcgen05 MMAs over both CTAs' shared memory into both CTAs' tensor memory.
-  const int csize = PAIR ? 2 : 1;
-  const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
+  // With xs, a cluster of two CTAs takes the same pixels: CTA `rank` the
+  // output channels of N tile `rank` (its half of an RMS row).
+  const int csize = PAIR ? 2 : (xs ? 2 : 1);
+  const int rank = (PAIR || xs) ? static_cast<int>(cluster_ctarank()) : 0;
   const int cid = static_cast<int>(blockIdx.x) / csize;
   const int ncl = static_cast<int>(gridDim.x) / csize;
+  // this CTA's tiles: tile_first, tile_first + tile_step, ...  (xs: the
+  // M tiles of its cluster, each at N tile `rank`)
+  const int tile_first = xs ? cid * 2 + rank : cid;
+  const int tile_step = xs ? ncl * 2 : ncl;
   const bool pair_leader = !PAIR || rank == 0;
 
   const int warp = threadIdx.x / 32;
@@ -274,6 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[i], PAIR ? 2 * kEpiWarps : kEpiWarps);  // (pair: both CTAs)
     }
     mbar_init(drain, 1);
+    if (xs)
+      for (int i = 0; i < 8; ++i) mbar_init(&x_full[i], 32);  // (the peer warp's lanes)
     fence_mbar_init();
     prefetch_tmap(&map_x);
     if (p.has_cache) prefetch_tmap(&map_cache);
@@ -289,9 +301,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   tc_fence_before();
-  // (in a pair, no CTA may arrive on its peer's barriers before the peer
+  // (in a cluster, no CTA may arrive on its peer's barriers before the peer
   // has initialised them)
-  if (PAIR)
+  if (PAIR || xs)
     cluster_sync();
   else
     __syncthreads();
@@ -318,14 +330,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto load_b = [&](int slot, int part, size_t stage_idx, int ntile) {
         const uint32_t dst = smem_base + L.b_off + slot * L.b_slot + part * L.b_stage;
         if constexpr (PAIR) {
-          // rows of the weight image [ntile][tap][cchunk][NT][64]: for each
-          // of the nh MMA N-subtiles, this CTA's half of its rows
-          const int nm = p.nt / p.nh;
+          // rows of the weight image [ntile][tap][cchunk][NT][64]: this
+          // CTA's half of the stage's rows
           const int row0 = static_cast<int>(
               (static_cast<size_t>(ntile) * stages_per_ntile + stage_idx) * p.nt);
-          for (int hh = 0; hh < p.nh; ++hh)
-            tma_load_2d_pair(dst + static_cast<uint32_t>(hh * (nm / 2)) * 128u, &map_w,
-                             lead_full_b + 8u * slot, 0, row0 + hh * nm + rank * (nm / 2));
+          tma_load_2d_pair(dst, &map_w, lead_full_b + 8u * slot, 0, row0 + rank * (p.nt / 2));
         } else {
           const uint8_t *wsrc =
               p.wimg + static_cast<size_t>(ntile) * stages_per_ntile * L.b_stage;
@@ -379,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           load_b(st, 0, static_cast<size_t>(st), 0);
         }
       }
-      for (int tile = cid; tile < n_tiles && ok; tile += ncl) {
+      for (int tile = tile_first; tile < n_tiles && ok; tile += tile_step) {
         const TileCoord tc0 = decode_tile(tile, p);
         for (int ia = 0; ia < n_a && ok; ++ia) {
           const int kt = ia / n_cc, cc = ia % n_cc;
@@ -455,13 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------ MMA issuer ----------------------------------
     // (a pair's follower issues nothing: the leader's MMAs cover both CTAs)
     if (lane == 0 && pair_leader) {
-      // nh MMAs of N = nt / nh each cover the tile's nt columns
-      const int nm = p.nt / p.nh;
-      const uint32_t idesc = is_e4m3(KC) ? idesc_e4m3_f32(PAIR ? 2 * kM : kM, nm)
-                                         : idesc_bf16_f32(PAIR ? 2 * kM : kM, nm);
-      // B start of N-subtile 1 relative to 0: nm rows of 16 bytes in each
-      // core-matrix slab, or (pair) nm / 2 rows of 128 swizzled bytes
-      const uint32_t bhalf16 = PAIR ? static_cast<uint32_t>(nm / 2) * 8u : static_cast<uint32_t>(nm);
+      const uint32_t idesc = is_e4m3(KC) ? idesc_e4m3_f32(PAIR ? 2 * kM : kM, p.nt)
+                                         : idesc_bf16_f32(PAIR ? 2 * kM : kM, p.nt);
       const uint32_t b_lbo = static_cast<uint32_t>(p.nt) * 16u;
       // Descriptors of stage 0; other stages, taps, sub-tiles and K steps
       // only move the start address (low 14 bits, 16-byte units), so they
@@ -482,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int sa = 0, sb = 0;
       uint32_t pa = 0, pb = 0;
       int it = 0;
-      for (int tile = cid; tile < n_tiles && ok; tile += ncl, ++it) {
+      for (int tile = tile_first; tile < n_tiles && ok; tile += tile_step, ++it) {
         const int buf = it % p.nbuf;
         const uint32_t use_par = static_cast<uint32_t>((it / p.nbuf) & 1);
         // wait until the epilogue (of both CTAs of a pair) has drained this
@@ -505,34 +509,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         // written by TMA and handed over by the full barriers, whose
         // completion the tensor core's reads observe without a fence.
         // (the issuing thread is the throughput limit of the big convs:
-        // the loops below unroll completely, with the N-subtile count
-        // resolved once per stage)
+        // the loops below unroll completely)
         auto mma_stage = [&](uint64_t a_st, uint64_t b_st, int ts) {
           const uint64_t a_tap = a_st + ((ts / KS) * halo_w + (ts % KS)) * pix16;
-          auto issue = [&](auto nh_c) {
-            constexpr int NH = decltype(nh_c)::value;
 #pragma unroll
-            for (int j = 0; j < kSteps; ++j) {
-              // every sub-tile (8 pixels further along the halo row) and
-              // every N-subtile reuses this weight stage
+          for (int j = 0; j < kSteps; ++j) {
+            // every sub-tile (8 pixels further along the halo row) reuses
+            // this weight stage
 #pragma unroll
-              for (int sbt = 0; sbt < SUB; ++sbt) {
-#pragma unroll
-                for (int hh = 0; hh < NH; ++hh) {
-                  const uint32_t d = d_tmem + (PAIR ? 0 : sbt * p.nt) + hh * nm;
-                  const uint64_t a = a_tap + (PAIR ? 0 : sbt * kTW * pix16) + j * astep16;
-                  const uint64_t b = b_st + j * bstep16 + hh * bhalf16;
-                  if constexpr (PAIR && is_e4m3(KC)) umma_e4m3_pair(d, a, b, idesc, accumulate);
-                  else if constexpr (PAIR) umma_bf16_pair(d, a, b, idesc, accumulate);
-                  else if constexpr (is_e4m3(KC)) umma_e4m3(d, a, b, idesc, accumulate);
-                  else umma_bf16(d, a, b, idesc, accumulate);
-                }
-              }
-              accumulate = 1;
+            for (int sbt = 0; sbt < SUB; ++sbt) {
+              const uint32_t d = d_tmem + (PAIR ? 0 : sbt * p.nt);
+              const uint64_t a = a_tap + (PAIR ? 0 : sbt * kTW * pix16) + j * astep16;
+              const uint64_t b = b_st + j * bstep16;
+              if constexpr (PAIR && is_e4m3(KC)) umma_e4m3_pair(d, a, b, idesc, accumulate);
+              else if constexpr (PAIR) umma_bf16_pair(d, a, b, idesc, accumulate);
+              else if constexpr (is_e4m3(KC)) umma_e4m3(d, a, b, idesc, accumulate);
+              else umma_bf16(d, a, b, idesc, accumulate);
             }
-          };
-          if (p.nh == 2) issue(IntConst<2>{});
-          else issue(IntConst<1>{});
+            accumulate = 1;
+          }
         };
         // arrive on `bar` (in both CTAs of a pair) once the MMAs issued so
         // far have completed
@@ -611,6 +606,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int m = q * 32 + lane;
     const int r = m / kTW, c = m % kTW;
     int it = 0;
+    // xs: the peer's partial sums of squares, [tile parity][quarter][lane]
+    const float *xbuf = reinterpret_cast<const float *>(smem + L.x_off);
+    const uint32_t xbuf_u32 = smem_u32(xbuf);
+    bool epi_ok = true;
     // bias (and gamma, beta) of every output channel, staged once: the
     // per-column reads below are then shared-memory broadcasts
     float *sp = reinterpret_cast<float *>(smem + L.p_off);
@@ -675,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     };
-    for (int tile = cid; tile < n_tiles; tile += ncl, ++it) {
+    for (int tile = tile_first; tile < n_tiles; tile += tile_step, ++it) {
       const int buf = it % p.nbuf;
       const uint32_t use_par = static_cast<uint32_t>((it / p.nbuf) & 1);
       const TileCoord tc0 = decode_tile(tile, p);
@@ -731,6 +730,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ss = fmaf(hv, hv, ss);
               }
             }
+          }
+          if (xs) {
+            // the row's other half is the peer CTA's: swap partial sums
+            // through its shared memory (slot: tile parity, this warp's
+            // quarter, this lane's row) and add them in rank order, so that
+            // both CTAs compute the same norm
+            const int slot = ((it & 1) * 4 + q);
+            const uint32_t peer = static_cast<uint32_t>(rank ^ 1);
+            st_cluster_b32(mapa_shared(xbuf_u32 + 4u * static_cast<uint32_t>(slot * 32 + lane), peer),
+                           __float_as_uint(ss));
+            mbar_arrive_remote(mapa_shared(smem_u32(&x_full[slot]), peer));
+            uint32_t got_x = 0;
+            if (lane == 0)
+              got_x = mbar_wait_bounded_cluster(&x_full[slot], static_cast<uint32_t>((it >> 1) & 1),
+                                                p.wait_limit_ns, p.status, 7)
+                          ? 1u
+                          : 0u;
+            got_x = __shfl_sync(0xffffffffu, got_x, 0);
+            if (!got_x) {
+              epi_ok = false;
+              break;
+            }
+            const float other = xbuf[slot * 32 + lane];
+            ss = rank == 0 ? ss + other : other + ss;
           }
           inv = sqrtf(static_cast<float>(p.c_out)) / fmaxf(sqrtf(ss), 1e-12f);
         }
@@ -838,6 +861,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }  // sub-tiles
+      if (!epi_ok) break;
     }
   }
 
@@ -845,7 +869,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   // no CTA leaves while its peer may still write its shared or tensor memory
   // or arrive on its barriers
-  if (PAIR) cluster_sync();
+  if (PAIR || xs) cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -859,9 +883,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb, int sub, int g_taps,
-                       int pair, int params) {
+                       int pair, int params, int xs) {
   // (a pair's CTA holds one 8 x 16 MMA tile: sub counts tile widths)
-  return make_layout(kc, nt, kh, kw, na, nb, pair ? 1 : sub, g_taps, pair != 0, params).total +
+  return make_layout(kc, nt, kh, kw, na, nb, pair ? 1 : sub, g_taps, pair != 0, params, xs)
+             .total +
          1024;  // + alignment slack
 }
 
@@ -874,7 +899,8 @@ bool finish_config(int ks, int kt, int c_in, UmmaConfig &c) {
   while (c.tmem_cols < c.nbuf * cta_sub * c.nt) c.tmem_cols *= 2;
   if (c.tmem_cols > 512) return false;
   auto smem = [&](int na, int nb, int g) {
-    return umma_launch_smem(c.kc, c.nt, ks, na, nb, c.tmem_cols, c.sub, g, c.pair, c.params);
+    return umma_launch_smem(c.kc, c.nt, ks, na, nb, c.tmem_cols, c.sub, g, c.pair, c.params,
+                            c.xs);
   };
   // A 3 x 3 halo stage feeds nine weight stages, so two of them keep the
   // tensor pipe busy.  Its weights travel as three slots of one kernel row
@@ -970,28 +996,31 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
       if (c_out % nt == 0 && (!rms_epi || nt == c_out)) return nt;
     return 0;
   };
-  // An RMS row wider than one MMA (c_out up to 512): the CTA tile takes the
-  // whole row as two MMAs of N = c_out / 2 per K step into adjacent tensor
-  // memory columns (one accumulator buffer: 2 x c_out columns do not fit).
+  // An RMS row wider than one MMA (257 to 512 channels): the two CTAs of a
+  // cluster each take one half of the row (N = c_out / 2) for the same
+  // pixels, each into two accumulator buffers (a tile's epilogue runs under
+  // the next tile's MMAs), and swap each row's partial sum of squares
+  // through shared memory.
   const bool wide_rms = rms_epi && c_out > 256;
   if (wide_rms && (c_out > 512 || c_out % 32 != 0)) return false;
   // Every choice below depends on (n, c, h, w, epilogue) and the plan's
   // max_t -- never on a call's t.  Whatever the shape, every output sums
   // its taps into one fp32 accumulator in the same order: the shapes differ
   // in which CTA computes which outputs, not in how.
-  UmmaConfig one;
+  UmmaConfig one{};
   // channel chunk: 128 E4M3 channels, or 64 / 96 / 32 bf16 channels
   if (e4m3 && c_in % 128 != 0) return false;
   one.kc = e4m3 ? 128 : (c_in % 64 == 0) ? 64 : (c_in % 96 == 0) ? 96 : 32;
   one.sub = 1;
   one.pair = 0;
-  one.nh = wide_rms ? 2 : 1;
-  one.nt = wide_rms ? c_out : largest_nt(256);
+  one.nt = wide_rms ? c_out / 2 : largest_nt(256);
   if (!one.nt) return false;
   one.n_ntiles = c_out / one.nt;
+  one.xs = wide_rms ? 2 : 0;
   one.params = param_floats(c_out, rms_epi ? 2 : 0, e4m3);
   if (!finish_config(ks, kt, c_in, one)) return false;
   *cfg = one;
+  if (wide_rms) return one.nbuf == 2;
   // the tile shapes are compared on the plan's largest call: max_t frames
   // of n images tile like n * max_t images
   const int nt_frames = n * (max_t > 0 ? max_t : 1);
@@ -1002,7 +1031,7 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
   // single buffer stalls the MMAs behind the epilogue).
   UmmaConfig two = one;
   two.sub = 2;
-  two.nt = wide_rms ? 0 : largest_nt(128);
+  two.nt = largest_nt(128);
   if (two.nt) {
     two.n_ntiles = c_out / two.nt;
     if (finish_config(ks, kt, c_in, two) && two.nbuf == 2) {
@@ -1021,8 +1050,7 @@ bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks
     UmmaConfig pr = one;
     pr.pair = 1;
     pr.sub = 2;  // the tile is two MMA tiles wide
-    // (a wide RMS row has one accumulator buffer whatever the shape)
-    if (finish_config(ks, kt, c_in, pr) && (pr.nbuf == 2 || wide_rms)) {
+    if (finish_config(ks, kt, c_in, pr) && pr.nbuf == 2) {
       const long long cost = frame_cost(pr, nt_frames, h, w, sm_count);
       if (cost <= best) {
         best = cost;
@@ -1065,8 +1093,8 @@ cudaError_t umma_prepare() {
 }
 
 size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols, int sub,
-                        int g_taps, int pair, int params) {
-  size_t smem = umma_smem_bytes(kc, nt, ks, ks, na, nb, sub, g_taps, pair, params);
+                        int g_taps, int pair, int params, int xs) {
+  size_t smem = umma_smem_bytes(kc, nt, ks, ks, na, nb, sub, g_taps, pair, params, xs);
   // A CTA that holds more than half of tensor memory must have its SM to
   // itself; asking for more than half the shared memory guarantees that.
   if (tmem_cols > 256 && smem < 116 * 1024) smem = 116 * 1024;
@@ -1114,11 +1142,11 @@ cudaLaunchConfig_t umma_launch_config(unsigned grid, size_t smem, int csize, cud
 }  // namespace
 
 int umma_max_clusters(const UmmaConfig &c, int ks) {
-  if (!c.pair) return 0;
+  if (!c.pair && c.xs != 2) return 0;
   UmmaKernel k = umma_kernel_for(c.kc, ks, c.sub, c.pair);
   if (!k) return 0;
-  const size_t smem =
-      umma_launch_smem(c.kc, c.nt, ks, c.na, c.nb, c.tmem_cols, c.sub, c.g_taps, c.pair, c.params);
+  const size_t smem = umma_launch_smem(c.kc, c.nt, ks, c.na, c.nb, c.tmem_cols, c.sub, c.g_taps,
+                                       c.pair, c.params, c.xs);
   cudaLaunchAttribute attr;
   const cudaLaunchConfig_t cfg = umma_launch_config(2u, smem, 2, nullptr, &attr);
   int n = 0;
@@ -1137,16 +1165,19 @@ cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_ca
   const size_t smem =
       umma_launch_smem(kc, args.nt, args.kh, args.na, args.nb, args.tmem_cols, args.sub,
                        args.g_taps, args.pair,
-                       param_floats(args.c_out, args.epi, args.oscale != nullptr));
+                       param_floats(args.c_out, args.epi, args.oscale != nullptr), args.xs);
   if (smem > kSmemLimit || (args.sub != 1 && args.sub != 2) || args.nbuf < 1 || args.nbuf > 2 ||
       args.na < 1 || args.na > 32 || args.nb < 1 || args.nb > 32)
     return cudaErrorInvalidValue;
   if (args.pair && (!uses_sw128(kc) || args.sub != 2 || grid % 2 != 0 || args.nt % 16 != 0))
     return cudaErrorInvalidValue;
-  // nh MMA N-subtiles: each a valid MMA N (a multiple of 16, at most 256;
-  // on a pair each CTA's half of it whole 8-row swizzle atoms)
-  if (args.nh < 1 || args.nh > 2 || args.nt % args.nh != 0 || (args.nt / args.nh) % 16 != 0 ||
-      args.nt / args.nh > 256 || (args.pair && (args.nt / args.nh) % 16 != 0))
+  // a valid MMA N: a multiple of 16, at most 256 (on a pair each CTA's half
+  // of it whole 8-row swizzle atoms)
+  if (args.nt % 16 != 0 || args.nt > 256) return cudaErrorInvalidValue;
+  // an RMS row split over a cluster: one MMA tile per CTA, two N tiles (one
+  // per CTA), two accumulator buffers, whole clusters
+  if (args.xs != 0 && (args.xs != 2 || args.pair || args.sub != 1 || args.n_ntiles != 2 ||
+                       !rms_epilogue(args.epi) || grid % 2 != 0))
     return cudaErrorInvalidValue;
   if (args.b_resident && (args.n_ntiles != 1 || args.g_taps != 1 ||
                           args.nb != args.kt * args.kh * args.kw * (args.c_in / kc)))
@@ -1168,7 +1199,8 @@ cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_ca
   UmmaKernel k = umma_kernel_for(kc, args.kh, args.sub, args.pair);
   if (!k) return cudaErrorInvalidValue;
   cudaLaunchAttribute attr;
-  const cudaLaunchConfig_t cfg = umma_launch_config(grid, smem, args.pair ? 2 : 1, stream, &attr);
+  const cudaLaunchConfig_t cfg =
+      umma_launch_config(grid, smem, (args.pair || args.xs == 2) ? 2 : 1, stream, &attr);
   return cudaLaunchKernelEx(&cfg, k, map_x, map_cache, map_w, map_sc, args);
 }
 

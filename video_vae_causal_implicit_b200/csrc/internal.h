@@ -24,8 +24,6 @@ struct UmmaArgs {
   int kt, kh, kw, pad_h, pad_w;
   int stride_t;                   // output frame t reads input frames stride_t * t + kt - (kt - 1)
   int nt, n_ntiles, tiles_w, tiles_h;
-  int nh;                         // MMAs of N = nt / nh that cover the tile's nt columns
-                                  // (2: an RMS row wider than one MMA, e.g. 384 channels)
   int na, nb;                     // pipeline depths (A halo stages, B weight stages)
   int tmem_cols;
   int epi;                        // 0 bias, 1 bias + residual, 2 bias + RMS + SiLU,
@@ -61,28 +59,33 @@ struct UmmaArgs {
   const __nv_bfloat16 *ncache_in;
   __nv_bfloat16 *ncache_out;
   int nc_vec32;                   // 1: ncache_out is 32-byte aligned (256-bit stores)
+  int xs;                         // 2: the two CTAs of a cluster take the same M tiles, CTA
+                                  // `rank` N tile `rank` (n_ntiles == 2): an RMS row split
+                                  // in halves whose partial sums of squares the CTAs swap
+                                  // through shared memory; else 0
 };
 
 // Tile configuration of the UMMA conv for a plan (chosen from n, c_in, c_out,
 // h, w, the epilogue and the plan's max_t -- never from a call's t).
 struct UmmaConfig {
-  int kc, nt, n_ntiles, nh, sub, nbuf, g_taps, pair, na, nb, tmem_cols, ctas_per_sm;
+  int kc, nt, n_ntiles, sub, nbuf, g_taps, pair, na, nb, tmem_cols, ctas_per_sm;
   int params;      // epilogue parameters staged in shared memory (floats)
   int b_resident;  // every weight stage resident in shared memory (nb of them)
+  int xs;          // 2: an RMS row split over the two CTAs of a cluster (UmmaArgs::xs)
 };
 // e4m3: FP8 E4M3 operands (128-channel chunks; c_in % 128 == 0).
 bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
                         int max_t, int sm_count, UmmaConfig *cfg, bool e4m3 = false);
-// CTA pairs that can be resident at once (cfg.pair), for sizing the grid;
-// 0 when the query fails.
+// Clusters of two CTAs that can be resident at once (cfg.pair or cfg.xs),
+// for sizing the grid; 0 when the query fails.
 int umma_max_clusters(const UmmaConfig &cfg, int ks);
 
 size_t umma_smem_bytes(int kc, int nt, int kh, int kw, int na, int nb, int sub, int g_taps,
-                       int pair, int params);
+                       int pair, int params, int xs);
 cudaError_t umma_prepare();
 // Dynamic shared memory a launch requests (with the one-CTA-per-SM rule).
 size_t umma_launch_smem(int kc, int nt, int ks, int na, int nb, int tmem_cols, int sub,
-                        int g_taps, int pair, int params);
+                        int g_taps, int pair, int params, int xs);
 int umma_tile_w();
 // TMA box of the A halo: columns (padded for the 128-byte swizzle) and
 // channels (64: swizzled pixel rows; 8: no-swizzle slabs).

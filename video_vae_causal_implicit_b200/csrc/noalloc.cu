@@ -145,7 +145,7 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
                           &L.cfg))
     return CC3D_ERR_UNSUPPORTED;
   const UmmaConfig &cfg = L.cfg;
-  if (cfg.pair) {
+  if (cfg.pair || cfg.xs == 2) {
     L.max_clusters = umma_max_clusters(cfg, d->kh);
     if (L.max_clusters < 1) return CC3D_ERR_CUDA;
   }
@@ -163,7 +163,7 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   CUtensorMap mw;
   if (cfg.pair && !encode_weight_map(&mw, wimg,
                                      static_cast<long long>(d->c_out) * taps * (d->c_in / 64),
-                                     nt / cfg.nh / 2))
+                                     nt / 2))
     return CC3D_ERR_CUDA;
 
   // ---- the conv (one kernel, which also writes cache_out and next_cache_out) ---------

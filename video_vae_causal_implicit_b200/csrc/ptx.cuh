@@ -156,6 +156,12 @@ __device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, const uint32_
       : "memory");
 }
 
+// A 32-bit store into another CTA's shared memory (ordered before a later
+// release-arrive of the same thread).
+__device__ __forceinline__ void st_cluster_b32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
 // ---- two-SM (CTA pair) forms --------------------------------------------------
 // TMA tiled loads issued by either CTA of a pair into its own shared memory,
 // completing on an mbarrier of the pair's leader CTA (`bar` is a
