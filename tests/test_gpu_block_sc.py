@@ -5,8 +5,9 @@ The block's 1x1x1 conv_shortcut runs inside conv2 as extra K steps of the
 same accumulator (its channel chunks past C_in are zero-filled by TMA, so
 96 input channels take two 64-channel chunks).  In every block conv1's
 output h1 is a bf16 activation before its RMS_norm (the oracle's default
-reading): blocks up to 256 channels round it inside conv1's fused
-epilogue, wider ones write it as bf16 for the RMS_norm + SiLU pass."""
+reading): conv1's fused RMS epilogue rounds it before the sum of squares
+(blocks up to 512 channels; wider ones write it as bf16 for a separate
+RMS_norm + SiLU pass)."""
 import numpy as np
 import pytest
 import torch
@@ -75,7 +76,8 @@ def test_channel_changing_block_matches_oracle(n, cin, cout, t, h, w):
 
 
 def test_wide_identity_block_matches_oracle():
-    """384 channels, identity shortcut: conv1's RMS_norm runs as its own pass."""
+    """384 channels, identity shortcut: conv1's RMS_norm + SiLU in its
+    epilogue, each 192-channel half of a row on one CTA of a cluster."""
     n, c, t, h, w = 1, 384, 2, 10, 14
     case = block_sc_case(c, c, t, h, w, seed=5, shortcut=False)
     blk = _block(case, n, h, w, t)

@@ -229,8 +229,11 @@ def test_sampled_points_config3b_shape():
 
 # ---- thin first layer (C_in <= 8) --------------------------------------------------
 
-@pytest.mark.parametrize("cin,cout,t,h,w", [(3, 96, 3, 20, 13), (3, 32, 2, 17, 9), (1, 16, 2, 9, 8),
-                                            (8, 64, 2, 16, 11)])
+# (w * cin % 8 == 0: the halo by TMA, else staged with plain loads; RGB
+# 3x3x3 takes the kernel-row-shifted A buffer, the others the im2col tile)
+@pytest.mark.parametrize("cin,cout,t,h,w", [(3, 96, 3, 20, 13), (3, 96, 3, 35, 24),
+                                            (3, 32, 2, 17, 9), (1, 16, 2, 9, 8),
+                                            (8, 64, 2, 16, 11), (4, 48, 2, 18, 14)])
 def test_thin_conv_matches_oracle(cin, cout, t, h, w):
     case = synth.conv_case(cin, cout, t, h, w, seed_base=30 + cin, x_dist="uniform")
     plan, x, y = run_conv(case)

@@ -3,7 +3,8 @@ kernels is bounded.  A child process runs with a 1 microsecond wait limit
 (CC3D_WAIT_LIMIT_US=1), so the pipelines' first real waits run out; the
 kernels must record the timeout, drain their own in-flight copies and
 MMAs, free tensor memory and return.  The limit governs every entry point,
-cc3d_forward_noalloc included.  The host then sees CC3D_ERR_TIMEOUT
+cc3d_forward_noalloc included, and every kind of wait, the exchange between
+the two CTAs that share a wide RMS row included.  The host then sees CC3D_ERR_TIMEOUT
 from cc3d_sync_status (once: reading clears it) and the CUDA context stays
 usable."""
 import json
@@ -45,6 +46,17 @@ out['noalloc_call'] = cc3d.cc3d_forward_noalloc(d, ctypes.c_void_p(x.data_ptr())
                                                 ctypes.c_void_p(y.data_ptr()), None, None, None,
                                                 None, cc3d._stream())
 out['noalloc_first'] = cc3d.cc3d_sync_status(cc3d._stream())
+# an RMS row split over a cluster of two CTAs: each runs its own pipeline,
+# and the exchange of the rows' partial sums of squares is bounded too
+cw = synth.conv_case(64, 320, 2, 16, 20)
+gw = synth.uniform((320,), 0.5, 1.5, 3).to(dev)
+pw = cc3d.Plan(cw['w'].to(dev), cw['b'].to(dev), h=16, w=20, max_t=2,
+               epi=cc3d.EPI_BIAS_RMS_SILU, gamma=gw)
+assert pw.stats().row_ctas == 2
+xw = synth.ndhwc(cw['x']).to(dev)
+yw = torch.empty((1, 2, 16, 20, 320), dtype=torch.bfloat16, device=dev)
+pw.forward(xw, yw)
+out['row_split_first'] = cc3d.cc3d_sync_status(cc3d._stream())
 # thin first-layer conv
 c3 = synth.conv_case(3, 96, 3, 48, 64, x_dist='uniform')
 p3 = cc3d.Plan(c3['w'].to(dev), c3['b'].to(dev), h=48, w=64, max_t=3)
@@ -72,5 +84,6 @@ def test_bounded_waits_report_timeout_and_leave_context_usable():
     assert res["umma_second"] == OK          # reading the status clears it
     assert res["noalloc_call"] == OK         # the limit reaches this entry point too
     assert res["noalloc_first"] == TIMEOUT
+    assert res["row_split_first"] == TIMEOUT
     assert res["thin_first"] == TIMEOUT
     assert res["torch_after"] == float(sum(range(1024)) * 2)

@@ -17,11 +17,14 @@
 //              run of (8 + kw - 1) * C_in elements) into a double-buffered
 //              shared buffer -- from the cache when the frame precedes the
 //              chunk; out-of-image and absent-cache reads are TMA zero fill;
-//   warps 0-3  builders: write the 128 x K_pad A tile from the halo as
-//              K-major core matrices (A double buffered).  When the input
-//              cannot be described by a tensor map (unaligned chunk start,
-//              W * C_in not a multiple of 8) they stage the halo themselves
-//              with plain loads;
+//   warps 0-3  builders: write the A operand from the halo as K-major core
+//              matrices (double buffered): in general the 128 x K_pad im2col
+//              tile; for RGB with a 3x3x3 kernel only the (kt, kw, ci) part
+//              of it, one 32-value row per halo row and tile column, which
+//              the MMAs of the three kernel rows kh read at start addresses
+//              kh halo rows apart.  When the input cannot be described by a
+//              tensor map (unaligned chunk start, W * C_in not a multiple of
+//              8) they stage the halo themselves with plain loads;
 //   warp  4    tensor memory owner and MMA issuer (one thread);
 //   warps 6-9  epilogue: tensor memory -> +bias -> bf16 -> global.
 // The weights ([K_pad/8][C_out][8] core matrices) stay in shared memory for
@@ -77,13 +80,19 @@ struct ThinLayout {
       stage_pitch, bar_off, total;
 };
 
+// RGB 3x3x3: the A buffer holds one 32-value row of K for each of the
+// (16 + 2) halo rows and 8 tile columns, as [halo row][4 K groups of 8][8
+// columns][8] bf16 -- 512 bytes per halo row.
+constexpr uint32_t kRgbRowBytes = 4u * 128u;
+
 __host__ __device__ inline ThinLayout thin_layout(const ThinArgs &a) {
   ThinLayout L;
   const HaloGeom g = halo_geom(a);
   L.b_off = 0;
   const uint32_t b_bytes = static_cast<uint32_t>(a.kpad) * a.c_out * 2u;
   L.a_off = rup(b_bytes, 1024u);
-  L.a_bytes = rup(static_cast<uint32_t>(a.kpad) * kM * 2u, 1024u);
+  L.a_bytes = a.spec_rgb333 ? rup(static_cast<uint32_t>(kTH + a.kh - 1) * kRgbRowBytes, 1024u)
+                            : rup(static_cast<uint32_t>(a.kpad) * kM * 2u, 1024u);
   L.halo_off = L.a_off + 2 * L.a_bytes;
   L.halo_bytes = rup(static_cast<uint32_t>(a.kt) * g.kt_stride * 2u, 128u);  // per buffer
   L.koff_off = L.halo_off + kNH * L.halo_bytes;  // int32 halo offset per K index
@@ -126,31 +135,43 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
-// Row of A for C_in = 3 and a 3x3x3 kernel, read from the halo (rows of 40
-// elements, frames 768 elements apart).  K is ordered as nine segments
-// (kt, kh) of ten: k = ((kt * 3 + kh) * 10) + kw * 3 + ci, the tenth element
-// of each segment (the next pixel's first channel) meeting a zero weight,
-// and K 90..95 zero.  A segment is ten consecutive halo elements, so it is
-// read as six aligned 32-bit words and realigned with funnel shifts.
-__device__ __forceinline__ void build_row_rgb333(const uint16_t *hbits, uint8_t *a_row) {
+// One row of the RGB 3x3x3 A buffer: the 27 values of halo row `row` of
+// the three frames at tile column c, k = kt * 9 + kw * 3 + ci, then five
+// zeros.  With kernel row kh at K offset 32 * kh of the weights, output
+// pixel (r, c) meets rows r, r + 1, r + 2 of this buffer in three MMA
+// steps of K = 32.  A frame's nine values are consecutive halo elements
+// (three pixels of three channels): five aligned 32-bit words, realigned
+// with funnel shifts.  `hbits` points at frame 0's first value; frames are
+// 768 elements apart (even), so all three share the realignment.
+__device__ __forceinline__ void build_row_rgb333(const uint16_t *hbits, uint8_t *dst) {
   const uintptr_t e0 = reinterpret_cast<uintptr_t>(hbits);
   const uint32_t *w32 = reinterpret_cast<const uint32_t *>(e0 & ~static_cast<uintptr_t>(3));
   const uint32_t sh = (e0 & 2) ? 16u : 0u;
-  uint32_t pairs[48];
+  uint32_t v[27];  // the 27 values, one per register (low 16 bits)
 #pragma unroll
-  for (int seg = 0; seg < 9; ++seg) {
-    const int off = ((seg / 3) * 768 + (seg % 3) * 40) / 2;  // even element offsets
-    uint32_t w[6];
+  for (int kt = 0; kt < 3; ++kt) {
+    uint32_t w[5];
 #pragma unroll
-    for (int i = 0; i < 6; ++i) w[i] = w32[off + i];
+    for (int i = 0; i < 5; ++i) w[i] = w32[kt * 384 + i];
 #pragma unroll
-    for (int i = 0; i < 5; ++i) pairs[seg * 5 + i] = __funnelshift_r(w[i], w[i + 1], sh);
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t pr = __funnelshift_r(w[i], w[i + 1], sh);  // values 2i, 2i + 1
+      v[kt * 9 + 2 * i] = pr & 0xffffu;
+      v[kt * 9 + 2 * i + 1] = pr >> 16;
+    }
+    v[kt * 9 + 8] = (w[4] >> sh) & 0xffffu;
   }
-  pairs[45] = pairs[46] = pairs[47] = 0u;
+  uint32_t out[16];
 #pragma unroll
-  for (int k8 = 0; k8 < 12; ++k8)
-    *reinterpret_cast<uint4 *>(a_row + k8 * (kM * 16)) =
-        make_uint4(pairs[4 * k8], pairs[4 * k8 + 1], pairs[4 * k8 + 2], pairs[4 * k8 + 3]);
+  for (int q = 0; q < 16; ++q) {
+    const uint32_t lo = 2 * q < 27 ? v[2 * q] : 0u;
+    const uint32_t hi = 2 * q + 1 < 27 ? v[2 * q + 1] : 0u;
+    out[q] = lo | (hi << 16);
+  }
+#pragma unroll
+  for (int k8 = 0; k8 < 4; ++k8)
+    *reinterpret_cast<uint4 *>(dst + k8 * 128) =
+        make_uint4(out[4 * k8], out[4 * k8 + 1], out[4 * k8 + 2], out[4 * k8 + 3]);
 }
 
 __global__ void __launch_bounds__(kThreads, 2)
@@ -295,11 +316,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         ok = false;
         break;
       }
-      uint8_t *a_row = smem + L.a_off + buf * L.a_bytes + (m / 8) * 128 + (m % 8) * 16;
-      const uint16_t *hbits = halo + r * G.row + G.rem + c * p.c_in;
+      uint8_t *a_buf = smem + L.a_off + buf * L.a_bytes;
       if (p.spec_rgb333) {
-        build_row_rgb333(hbits, a_row);
+        // rows (halo row, column) v = m and, for the last two halo rows,
+        // v = 128 + m
+        for (int v = m; v < (kTH + 2) * kTW; v += kBuilders)
+          build_row_rgb333(halo + (v / kTW) * G.row + G.rem + (v % kTW) * 3,
+                           a_buf + (v / kTW) * kRgbRowBytes + (v % kTW) * 16);
       } else {
+        uint8_t *a_row = a_buf + (m / 8) * 128 + (m % 8) * 16;
+        const uint16_t *hbits = halo + r * G.row + G.rem + c * p.c_in;
         // build row m of A (zero where koff is -1)
         for (int k8 = 0; k8 < p.kpad / 8; ++k8) {
           uint32_t packed[4];
@@ -358,8 +384,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ------------------------------ MMA issuer ----------------------------------
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kM, p.c_out);
-      // A: [kpad/8][16 row groups][8 rows][8]: K step 16*128 B, M step 128 B
-      const uint64_t adesc0 = smem_desc_noswizzle(smem_base + L.a_off, kM * 16u, 128u);
+      // A, im2col tile: [kpad/8][16 row groups][8 rows][8], K core matrices
+      // 16 * 128 B apart, M groups 128 B.  RGB 3x3x3: [halo row][4][8][8],
+      // K core matrices 128 B apart, M groups (tile rows) 512 B; the K step
+      // j of 16 (kernel row kh = j / 2) starts kh rows and (j % 2) * 256 B
+      // further on.
+      const uint64_t adesc0 =
+          p.spec_rgb333 ? smem_desc_noswizzle(smem_base + L.a_off, 128u, kRgbRowBytes)
+                        : smem_desc_noswizzle(smem_base + L.a_off, kM * 16u, 128u);
       // B: [kpad/8][c_out][8]: K step c_out*16 B, N step 128 B
       const uint32_t b_lbo = static_cast<uint32_t>(p.c_out) * 16u;
       const uint64_t bdesc0 = smem_desc_noswizzle(smem_base + L.b_off, b_lbo, 128u);
@@ -375,9 +407,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         tc_fence_after();
         const uint64_t a_st = adesc0 + ((buf * L.a_bytes) >> 4);
-        for (int j = 0; j < p.kpad / 16; ++j)
-          umma_bf16(tmem_base + buf * p.c_out, a_st + 2 * j * (kM * 16 / 16),
-                    bdesc0 + 2 * j * (b_lbo >> 4), idesc, j > 0 ? 1u : 0u);
+        for (int j = 0; j < p.kpad / 16; ++j) {
+          const uint32_t a_step = p.spec_rgb333 ? (j / 2) * (kRgbRowBytes / 16) + (j % 2) * 16u
+                                                : 2 * j * (kM * 16 / 16);
+          umma_bf16(tmem_base + buf * p.c_out, a_st + a_step, bdesc0 + 2 * j * (b_lbo >> 4), idesc,
+                    j > 0 ? 1u : 0u);
+        }
         umma_commit(&a_empty[buf]);
         umma_commit(&acc_full[buf]);
       }
@@ -506,8 +541,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 __global__ void repack_thin_kernel(const __nv_bfloat16 *__restrict__ w, __nv_bfloat16 *img,
                                    int c_out, int c_in, int taps, int kpad, int spec) {
   // img[k8][co][e] = W[co][ci][tap] at K index k = k8 * 8 + e; 0 past K.
-  // Generic order: k = tap * c_in + ci.  RGB 3x3x3 order (spec): nine
-  // segments of ten, k = (kt * 3 + kh) * 10 + kw * 3 + ci, the tenth zero.
+  // Generic order: k = tap * c_in + ci.  RGB 3x3x3 order (spec): three
+  // kernel rows of 32, k = kh * 32 + kt * 9 + kw * 3 + ci, 27..31 zero.
   const int total = kpad * c_out;
   const int K = taps * c_in;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
@@ -517,10 +552,10 @@ __global__ void repack_thin_kernel(const __nv_bfloat16 *__restrict__ w, __nv_bfl
     const int k = k8 * 8 + e;
     __nv_bfloat16 v = __float2bfloat16_rn(0.f);
     if (spec) {
-      const int seg = k / 10, j = k % 10;
-      if (seg < 9 && j < 9) {
-        const int tap = seg * 3 + j / 3, ci = j % 3;
-        v = w[(static_cast<size_t>(co) * 3 + ci) * 27 + tap];
+      const int kh = k / 32, j = k % 32;
+      if (j < 27) {
+        const int kt = j / 9, kw = (j % 9) / 3, ci = j % 3;
+        v = w[(static_cast<size_t>(co) * 3 + ci) * 27 + (kt * 3 + kh) * 3 + kw];
       }
     } else if (k < K) {
       const int tap = k / c_in, ci = k % c_in;

@@ -21,7 +21,8 @@ Cases (seeded synthetic inputs, generated on the device):
   blk96   the encoder's channel-changing block 96 -> 192 (conv_shortcut fused
           into conv2) on x[1,96,17,240,416]
   blk384  a 384-channel residual block on x[1,384,5,60,104] (conv1's RMS_norm
-          + SiLU in its epilogue, two N = 192 MMAs per K step)
+          + SiLU in its epilogue, each 192-channel half of a row on one CTA
+          of a two-CTA cluster)
   c2f8    the 384 -> 384 conv of c2 on FP8 E4M3 operands
 Prints nothing but a final "ok"; timing comes from the profiler.
 """
