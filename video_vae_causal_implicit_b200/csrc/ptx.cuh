@@ -40,14 +40,26 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+// A waiting thread is suspended by the hardware until the phase completes
+// or this many nanoseconds pass (then the bounded loops below check the
+// clock and try again): waiting warps do not spin on the issue slots the
+// working warps of the SM need.  A wait limit below four times this
+// shortens it, so that the limit still decides.
+constexpr uint32_t kWaitSuspendHintNs = 20000u;
+
+__device__ __forceinline__ uint32_t suspend_hint(uint64_t limit_ns) {
+  return limit_ns / 4 < kWaitSuspendHintNs ? static_cast<uint32_t>(limit_ns / 4)
+                                           : kWaitSuspendHintNs;
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -57,10 +69,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // wall-clock time has passed; never traps.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   uint64_t limit_ns, int *status, int site) {
-  if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t hint = suspend_hint(limit_ns);
+  if (mbar_try_wait(bar, parity, hint)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity, hint)) return true;
     if (globaltimer_ns() - t0 > limit_ns) {
       if (status) atomicCAS(status, 0, kDevTimeoutBase + site);
       return false;
@@ -113,14 +126,15 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity,
+                                                      uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -129,10 +143,11 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
 __device__ __forceinline__ bool mbar_wait_bounded_cluster(uint64_t *bar, uint32_t parity,
                                                           uint64_t limit_ns, int *status,
                                                           int site) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint32_t hint = suspend_hint(limit_ns);
+  if (mbar_try_wait_cluster(bar, parity, hint)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (mbar_try_wait_cluster(bar, parity, hint)) return true;
     if (globaltimer_ns() - t0 > limit_ns) {
       if (status) atomicCAS(status, 0, kDevTimeoutBase + site);
       return false;
