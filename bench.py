@@ -514,6 +514,11 @@ def run_sweep(args, dev, stream, peaks, flush_l2, full=False):
     reps = max(3, min(args.steps, 10))
 
     def timed(fn, flush=False):
+        # every row starts from an idle GPU (half a second), so that the
+        # power and clock state a heavy row leaves behind does not carry
+        # over into the next one
+        torch.cuda.synchronize()
+        time.sleep(0.5)
         for k in range(2):
             fn()
         torch.cuda.synchronize()
