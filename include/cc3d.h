@@ -91,9 +91,10 @@ typedef enum {
   CC3D_EPI_BIAS_RESIDUAL = 1, /* y = conv + b + residual                       */
   CC3D_EPI_BIAS_RMS_SILU = 2, /* y = SiLU(RMS(h; gamma) (+ beta)), h = conv + b
                                  rounded to bf16 first (the block's conv1
-                                 output is a bf16 activation); one CTA owns
-                                 each whole row: c_out <= 256, or up to 512
-                                 in steps of 32 (two MMAs per K step)      */
+                                 output is a bf16 activation); c_out <= 256
+                                 (one CTA owns each row), or up to 512 in
+                                 steps of 32 (the row's halves on the two
+                                 CTAs of a cluster)                         */
   CC3D_EPI_BIAS_RMS = 3       /* y = RMS(h; gamma) (+ beta), the same without
                                  SiLU: the WanRMS_norm after the downsample
                                  path's convs (§10.5)                        */
@@ -201,6 +202,40 @@ cc3d_status cc3d_forward(cc3d_plan *plan, const void *x, int t,
                          const void *cache_in, void *y, void *cache_out,
                          const void *residual, const void *next_cache_in,
                          void *next_cache_out, void *stream);
+
+/* One call of cc3d_forward_host: x and y in host memory, the rest as in
+ * cc3d_forward (device pointers, same shapes and rules). */
+typedef struct {
+  const void *x_host;     /* [n][t][h][w][c_in] host memory                 */
+  int t;                  /* frames of x, 1 <= t <= max_t                    */
+  const void *cache_in;   /* device, nullable                                */
+  void *cache_out;        /* device, nullable                                */
+  const void *residual;   /* device, EPI_BIAS_RESIDUAL only                  */
+  void *y_host;           /* [n][t'][h][w][c_out] host memory                */
+} cc3d_host_call;
+
+/* cc3d_forward over host buffers, for callers whose video lives in host
+ * memory: `ncalls` calls of one plan run in order, each as upload of x ->
+ * conv -> download of y, overlapped across calls: call i+1's upload and
+ * call i-1's download run while call i's conv runs.  The uploads use a
+ * stream of the plan, the convs run on `stream`, the downloads on a second
+ * stream of the plan; the data pass through three device staging slots of
+ * max_t frames of x and of y that the plan allocates on first use (freed
+ * by cc3d_plan_destroy).  The first upload starts after the work enqueued
+ * on `stream` before the call; on return every copy and conv is enqueued
+ * and `stream` waits for the last download, so work enqueued on `stream`
+ * afterwards, or a synchronize of it, sees every y_host complete.  Host
+ * buffers should be pinned (cudaHostAlloc / cudaHostRegister) for the
+ * copies to overlap; pageable memory works, with the copies serialised.
+ * A call's y_host must not overlap another call's x_host or y_host.  The
+ * calls are validated before anything is enqueued: CC3D_ERR_INVALID_ARG
+ * (null host pointers, ncalls < 1, t out of range, a residual that does
+ * not match the epilogue, an RMS-epilogue plan -- its next caches have no
+ * host form), CC3D_ERR_ALIGNMENT / CC3D_ERR_ALIAS for the device pointers
+ * as in cc3d_forward; CC3D_ERR_OOM when the staging slots cannot be
+ * allocated.  Not safe to call on one plan from two threads at once. */
+cc3d_status cc3d_forward_host(cc3d_plan *plan, const cc3d_host_call *calls, int ncalls,
+                              void *stream);
 
 /* FP8 E4M3 codes of bf16 values: q[i] = E4M3(x[i] / scale), the quotient
  * an IEEE fp32 division, rounded to nearest even and saturated to +-448

@@ -49,6 +49,13 @@ def test_library_exports_every_declared_symbol(lib):
     assert set(declared_functions()) <= set(cc3d.SIGNATURES)
 
 
+def test_forward_host_refuses_bad_calls_on_the_host(lib):
+    # no plan, no calls: refused before any CUDA call
+    assert cc3d.cc3d_forward_host(None, None, 0, None) == cc3d.ERR_INVALID_ARG
+    arr = (cc3d.HostCall * 1)()
+    assert cc3d.cc3d_forward_host(None, arr, 1, None) == cc3d.ERR_INVALID_ARG
+
+
 def test_status_strings(lib):
     for s in range(8):
         assert cc3d.cc3d_status_string(s)

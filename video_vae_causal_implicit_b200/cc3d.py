@@ -51,12 +51,19 @@ class Stats(ctypes.Structure):
                 ("w_resident", ctypes.c_int), ("row_ctas", ctypes.c_int)]
 
 
+class HostCall(ctypes.Structure):
+    _fields_ = [("x_host", ctypes.c_void_p), ("t", ctypes.c_int), ("cache_in", ctypes.c_void_p),
+                ("cache_out", ctypes.c_void_p), ("residual", ctypes.c_void_p),
+                ("y_host", ctypes.c_void_p)]
+
+
 # name -> (restype, argtypes)
 _VP, _I = ctypes.c_void_p, ctypes.c_int
 SIGNATURES = {
     "cc3d_plan_create": (_I, [ctypes.POINTER(Desc), ctypes.POINTER(_VP)]),
     "cc3d_plan_destroy": (_I, [_VP]),
     "cc3d_forward": (_I, [_VP, _VP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "cc3d_forward_host": (_I, [_VP, ctypes.POINTER(HostCall), _I, _VP]),
     "rmsnorm_silu": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP]),
     "rms_norm": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP]),
     "cc3d_quantize_e4m3": (_I, [_VP, ctypes.c_size_t, ctypes.c_float, _VP, _VP]),
@@ -111,6 +118,10 @@ def cc3d_forward(plan, x, t, cache_in, y, cache_out, residual, next_cache_in, ne
                  stream):
     return lib().cc3d_forward(plan, x, t, cache_in, y, cache_out, residual, next_cache_in,
                               next_cache_out, stream)
+
+
+def cc3d_forward_host(plan, calls, ncalls, stream):
+    return lib().cc3d_forward_host(plan, calls, ncalls, stream)
 
 
 def rmsnorm_silu(x, gamma, beta, n, t, h, w, c, y, cache_in, cache_out, stream):
@@ -211,6 +222,21 @@ class Plan:
                            _ptr(residual), _ptr(next_cache_in), _ptr(next_cache_out),
                            _stream(stream)), "cc3d_forward")
         return y
+
+    def forward_host(self, calls, stream=None):
+        """cc3d_forward_host: ``calls`` is a list of dicts with x_host and
+        y_host (host tensors, pinned for overlap) and optionally t,
+        cache_in, cache_out, residual (device tensors)."""
+        arr = (HostCall * len(calls))()
+        for i, c in enumerate(calls):
+            arr[i].x_host = c["x_host"].data_ptr()
+            arr[i].t = int(c.get("t", c["x_host"].shape[1]))
+            for k in ("cache_in", "cache_out", "residual"):
+                v = c.get(k)
+                setattr(arr[i], k, v.data_ptr() if v is not None else None)
+            arr[i].y_host = c["y_host"].data_ptr()
+        check(cc3d_forward_host(self.handle, arr, len(calls), _stream(stream)),
+              "cc3d_forward_host")
 
     def stats(self):
         s = Stats()

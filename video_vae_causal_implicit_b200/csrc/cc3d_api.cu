@@ -301,6 +301,23 @@ struct cc3d_plan {
   float *oscale;  // FP8: s_x * s_w[c] per output channel
   cc3d_stats st;
   std::mutex mu;
+  // cc3d_forward_host: staging slots (x and y of max_t frames each), an
+  // upload and a download stream and their events, created on first use.
+  // Three slots: a call's conv then waits only for the download of the
+  // call three before it, which a long download (a whole sequence's y)
+  // has usually finished by then.
+  static constexpr int kHostSlots = 3;
+  struct HostPipe {
+    void *x[kHostSlots] = {};
+    void *y[kHostSlots] = {};
+    size_t x_frame = 0, y_frame = 0;  // bytes per frame (all n images)
+    cudaStream_t up = nullptr, down = nullptr;
+    cudaEvent_t entry = nullptr;
+    cudaEvent_t up_done[kHostSlots] = {};
+    cudaEvent_t conv_done[kHostSlots] = {};
+    cudaEvent_t down_done[kHostSlots] = {};
+    bool ready = false;
+  } host;
 };
 
 struct cc3d_block {
@@ -320,8 +337,25 @@ cc3d_status from_cuda(cudaError_t e) {
   return CC3D_ERR_CUDA;
 }
 
+void free_host_pipe(cc3d_plan::HostPipe &h) {
+  for (int s = 0; s < cc3d_plan::kHostSlots; ++s) {
+    cudaFree(h.x[s]);
+    cudaFree(h.y[s]);
+    if (h.up_done[s]) cudaEventDestroy(h.up_done[s]);
+    if (h.conv_done[s]) cudaEventDestroy(h.conv_done[s]);
+    if (h.down_done[s]) cudaEventDestroy(h.down_done[s]);
+  }
+  if (h.entry) cudaEventDestroy(h.entry);
+  if (h.up) cudaStreamDestroy(h.up);
+  if (h.down) cudaStreamDestroy(h.down);
+  h = cc3d_plan::HostPipe();
+}
+
 void free_plan(cc3d_plan *p) {
   if (!p) return;
+  if (p->host.up) cudaStreamSynchronize(p->host.up);
+  if (p->host.down) cudaStreamSynchronize(p->host.down);
+  free_host_pipe(p->host);
   cudaFree(p->wimg);
   cudaFree(p->wraw);
   cudaFree(p->bias);
@@ -778,6 +812,104 @@ cc3d_status cc3d_forward(cc3d_plan *p, const void *x, int t, const void *cache_i
   if (p && p->c_sc > 0) return CC3D_ERR_INVALID_ARG;  // (a block-internal plan)
   return forward_impl(p, x, t, cache_in, y, cache_out, residual, next_cache_in, next_cache_out,
                       nullptr, stream_v);
+}
+
+}  // extern "C"
+
+namespace {
+// The staging slots, streams and events of cc3d_forward_host (first use).
+cc3d_status host_pipe_init(cc3d_plan *p) {
+  cc3d_plan::HostPipe &h = p->host;
+  if (h.ready) return CC3D_OK;
+  const cc3d_desc &d = p->d;
+  const size_t esz = d.dtype == CC3D_FP32 ? 4 : 2;
+  const size_t in_esz = d.dtype == CC3D_FP8_E4M3 ? 1 : esz;
+  h.x_frame = static_cast<size_t>(d.n) * d.h * d.w * d.c_in * in_esz;
+  h.y_frame = static_cast<size_t>(d.n) * (d.h / d.stride_h) * (d.w / d.stride_w) * d.c_out * esz;
+  const int max_out = (d.max_t - 1) / d.stride_t + 1;
+  cudaError_t e = cudaSuccess;
+  for (int s = 0; s < cc3d_plan::kHostSlots && e == cudaSuccess; ++s) {
+    e = cudaMalloc(&h.x[s], h.x_frame * d.max_t);
+    if (e == cudaSuccess) e = cudaMalloc(&h.y[s], h.y_frame * max_out);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h.up_done[s], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h.conv_done[s], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h.down_done[s], cudaEventDisableTiming);
+  }
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h.entry, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h.up, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h.down, cudaStreamNonBlocking);
+  if (e != cudaSuccess) {
+    free_host_pipe(h);
+    return from_cuda(e);
+  }
+  h.ready = true;
+  return CC3D_OK;
+}
+}  // namespace
+
+extern "C" {
+
+cc3d_status cc3d_forward_host(cc3d_plan *p, const cc3d_host_call *calls, int ncalls,
+                              void *stream_v) {
+  if (!p || !calls || ncalls < 1 || p->c_sc > 0) return CC3D_ERR_INVALID_ARG;
+  const cc3d_desc &d = p->d;
+  // the next caches of an RMS epilogue have no host form
+  if (d.epi == CC3D_EPI_BIAS_RMS_SILU || d.epi == CC3D_EPI_BIAS_RMS) return CC3D_ERR_INVALID_ARG;
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (dev != p->device) return CC3D_ERR_INVALID_ARG;
+  // everything cc3d_forward would check on these calls, before any enqueue
+  // (x and y are the plan's own staging slots)
+  const bool thin = p->variant == CC3D_VARIANT_THIN;
+  auto in_ok = [&](const void *q) {
+    return thin ? (reinterpret_cast<uintptr_t>(q) & 1u) == 0 : aligned16(q);
+  };
+  const size_t in_esz = d.dtype == CC3D_FP8_E4M3 ? 1 : (d.dtype == CC3D_FP32 ? 4 : 2);
+  const size_t c_bytes = static_cast<size_t>(d.n) * (d.kt - 1) * d.h * d.w * d.c_in * in_esz;
+  for (int i = 0; i < ncalls; ++i) {
+    const cc3d_host_call &c = calls[i];
+    if (!c.x_host || !c.y_host || c.t < 1 || c.t > d.max_t ||
+        (d.epi == CC3D_EPI_BIAS_RESIDUAL) != (c.residual != nullptr))
+      return CC3D_ERR_INVALID_ARG;
+    if (!in_ok(c.cache_in) || !in_ok(c.cache_out) || !aligned16(c.residual))
+      return CC3D_ERR_ALIGNMENT;
+    if (overlaps(c.cache_out, c_bytes, c.cache_in, c_bytes)) return CC3D_ERR_ALIAS;
+  }
+  cc3d_status s = host_pipe_init(p);
+  if (s != CC3D_OK) return s;
+  cc3d_plan::HostPipe &h = p->host;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  // the uploads start after the work already on `stream`
+  cudaError_t e = cudaEventRecord(h.entry, stream);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(h.up, h.entry, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(h.down, h.entry, 0);
+  for (int i = 0; i < ncalls && e == cudaSuccess; ++i) {
+    const cc3d_host_call &c = calls[i];
+    const int sl = i % cc3d_plan::kHostSlots;
+    const bool reused = i >= cc3d_plan::kHostSlots;
+    const int t_out = (c.t - 1) / d.stride_t + 1;
+    // slot sl was last used by call i - kHostSlots: its x is free once that
+    // conv has run, its y once that download has run
+    if (reused) e = cudaStreamWaitEvent(h.up, h.conv_done[sl], 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(h.x[sl], c.x_host, h.x_frame * c.t, cudaMemcpyHostToDevice, h.up);
+    if (e == cudaSuccess) e = cudaEventRecord(h.up_done[sl], h.up);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, h.up_done[sl], 0);
+    if (e == cudaSuccess && reused) e = cudaStreamWaitEvent(stream, h.down_done[sl], 0);
+    if (e != cudaSuccess) break;
+    s = forward_impl(p, h.x[sl], c.t, c.cache_in, h.y[sl], c.cache_out, c.residual, nullptr,
+                     nullptr, nullptr, stream_v);
+    if (s != CC3D_OK) return s;
+    e = cudaEventRecord(h.conv_done[sl], stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h.down, h.conv_done[sl], 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(c.y_host, h.y[sl], h.y_frame * t_out, cudaMemcpyDeviceToHost, h.down);
+    if (e == cudaSuccess) e = cudaEventRecord(h.down_done[sl], h.down);
+  }
+  // `stream` waits for every download (the last one of each slot)
+  for (int sl = 0; sl < cc3d_plan::kHostSlots && sl < ncalls && e == cudaSuccess; ++sl)
+    e = cudaStreamWaitEvent(stream, h.down_done[sl], 0);
+  return from_cuda(e);
 }
 
 }  // extern "C"
