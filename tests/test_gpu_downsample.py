@@ -1,10 +1,11 @@
 """GPU parity of the downsample path's spatial step: each frame through
 ZeroPad2d(0, 1, 0, 1) and a 3x3 conv with stride 2 (H x W -> H/2 x W/2),
-on the tensor-core conv: the nine taps run as separate K stages, each
-loaded through a tensor map that walks every other pixel.  Cases cover
-96-channel (no-swizzle) and 64-channel (swizzled) chunks, one CTA per tile,
-the CTA pair with resident and with streamed weights, two sub-tiles (the
-encoder's full-size layer), and the residual epilogue."""
+on the tensor-core conv: the input's four stride-2 phases are loaded once
+per channel chunk, each through a tensor map that walks every other pixel,
+and the nine taps read them through 2 x 2 shifted views.  Cases cover 96-
+and 32-channel (no-swizzle slab) and 64-channel (swizzled) chunks, one CTA
+per tile, the CTA pair, two sub-tiles (the encoder's full-size layer), and
+the residual epilogue."""
 import pytest
 import torch
 
@@ -32,7 +33,8 @@ CASES = [
     # (n, c_in, c_out, t, h, w, shape): shape = (mma_ctas, tile_w, w_resident)
     (1, 96, 96, 2, 20, 24, (1, 8, 0)),
     (1, 96, 96, 2, 96, 160, (1, 8, 0)),
-    (1, 64, 128, 1, 32, 48, (2, 16, 1)),
+    (1, 64, 128, 1, 32, 48, (2, 16, 0)),
+    (1, 32, 64, 2, 20, 24, (1, 8, 0)),
     (2, 192, 192, 2, 30, 52, (2, 16, 0)),
 ]
 

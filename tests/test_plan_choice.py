@@ -116,16 +116,16 @@ def test_plan_is_a_function_of_the_problem(probe):
 
 
 def test_downsample_conv_plans(probe):
-    """The stride-2 spatial conv plans nine 1x1 taps over the output frame
-    (kt = 9, ks = 1): its plans satisfy the same invariants."""
-    cases = [case(n=n, ci=ci, co=co, h=h, w=w, kt=9, ks=1, mt=mt)
+    """The stride-2 spatial conv plans the input's four stride-2 phases
+    seen through 2 x 2 views over the output frame (kt = 4, ks = 2): one tap
+    per weight slot, weights streamed, within the SM."""
+    cases = [case(n=n, ci=ci, co=co, h=h, w=w, kt=4, ks=2, mt=mt)
              for (ci, co), (h, w), n, mt in itertools.product(
                  [(64, 64), (96, 96), (64, 128), (192, 192)],
                  [(10, 12), (15, 26), (48, 80), (240, 416)], [1, 2], [1, 17])]
     for c, p in zip(cases, probe(cases)):
         assert p["ok"] == 1 and p["smem"] <= SMEM_MAX and p["g_taps"] == 1, (c, p)
-        if p["b_resident"]:
-            assert p["nb"] == 9 * c[1] // p["kc"] and p["na"] >= 3, (c, p)
+        assert p["b_resident"] == 0 and p["na"] == 2 and 2 <= p["nb"] <= 8, (c, p)
 
 
 def test_fp8_plans(probe):

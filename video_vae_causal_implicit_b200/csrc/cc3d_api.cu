@@ -179,8 +179,9 @@ cudaError_t run_umma_layer(const UmmaLayer &L, const UmmaCall &c, int *status,
   CUtensorMap mx, mc;
   const int front = L.kt - 1;  // frames of the causal cache (0 for the stride-2 spatial conv)
   const int tile_w = umma_tile_w() * cfg.sub;
-  // the kernel's spatial kernel: kh x kw, or 1 x 1 taps for stride 2
-  const int ks = L.s2 ? 1 : L.kh;
+  // the kernel's spatial kernel: kh x kw, or for stride 2 the 2 x 2 views
+  // of the input's four stride-2 phases
+  const int ks = L.s2 ? 2 : L.kh;
   const int h_out = L.s2 ? L.h / 2 : L.h, w_out = L.s2 ? L.w / 2 : L.w;
   const int t_out = (c.t - 1) / L.stride_t + 1;
   // (a pair's CTA loads the halo of its own 8-column half)
@@ -212,7 +213,7 @@ cudaError_t run_umma_layer(const UmmaLayer &L, const UmmaCall &c, int *status,
   a.status = status;
   a.wait_limit_ns = wait_limit_ns();
   a.n = L.n; a.t = t_out; a.h = h_out; a.w = w_out; a.c_in = L.c_in; a.c_out = L.c_out;
-  a.kt = L.s2 ? 9 : L.kt; a.kh = ks; a.kw = ks; a.pad_h = L.pad_h; a.pad_w = L.pad_w;
+  a.kt = L.s2 ? 4 : L.kt; a.kh = ks; a.kw = ks; a.pad_h = L.pad_h; a.pad_w = L.pad_w;
   a.stride_t = L.stride_t;
   a.s2 = L.s2;
   a.vec32 = (reinterpret_cast<uintptr_t>(c.y) & 31u) == 0 ? 1 : 0;
@@ -584,7 +585,8 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
       const bool e4m3 = desc->dtype == CC3D_FP8_E4M3;
       L.e4m3 = e4m3 ? 1 : 0;
       const int max_out = (desc->max_t - 1) / desc->stride_t + 1;  // largest call's frames
-      const int kt_eff = L.s2 ? 9 : desc->kt, ks_eff = L.s2 ? 1 : desc->kh;
+      // (the stride-2 conv: four phase stages seen through 2 x 2 views)
+      const int kt_eff = L.s2 ? 4 : desc->kt, ks_eff = L.s2 ? 2 : desc->kh;
       const int h_out = desc->h / desc->stride_h, w_out = desc->w / desc->stride_w;
       if (!choose_umma_config(desc->n, desc->c_in, desc->c_out, h_out, w_out, kt_eff, ks_eff,
                               desc->epi == CC3D_EPI_BIAS_RMS_SILU ||

@@ -146,6 +146,16 @@ struct TileCoord {
 
 // Tile order: N tile fastest (CTAs sharing an input halo run together),
 // then tile column, tile row, frame, batch image.
+// The stride-2 3x3 conv as four phases: output pixel (h, w), tap (kh, kw)
+// reads input (2h + kh, 2w + kw) = phase (kh % 2, kw % 2) of the input --
+// the pixels (2i + kh % 2, 2j + kw % 2) -- at (i, j) = (h + kh / 2,
+// w + kw / 2).  Phase q = 2 * (kh % 2) + kw % 2 serves 4, 2, 2, 1 taps.
+__host__ __device__ constexpr int phase_tap_count(int q) { return q == 0 ? 4 : (q == 3 ? 1 : 2); }
+// The j-th tap of phase q, as kh * 3 + kw.
+__host__ __device__ constexpr int phase_tap(int q, int j) {
+  return ((q >> 1) + 2 * (j / ((q & 1) ? 1 : 2))) * 3 + (q & 1) + 2 * (j % ((q & 1) ? 1 : 2));
+}
+
 __device__ __forceinline__ TileCoord decode_tile(int tile, const UmmaArgs &p) {
   TileCoord c;
   c.ntile = tile % p.n_ntiles;
@@ -254,7 +264,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_cc = p.c_in / KC;   // channel chunks
   const int n_a = p.kt * n_cc;    // A stages per tile
   // weight stages of the conv per N tile, and the shortcut's chunks after them
-  const int n_conv_stages = p.kt * KS * KS * n_cc;
+  // (the stride-2 phase conv: four phase stages against the nine taps'
+  // weight stages)
+  const bool phases = KS == 2 && p.s2;
+  const int n_conv_stages = (phases ? 9 : p.kt * KS * KS) * n_cc;
   const int n_sc = p.c_sc > 0 ? p.n_cc_sc : 0;
   const int stages_per_ntile = n_conv_stages + n_sc;  // weight image
   // weight slots per A stage: one per group of g_taps spatial taps
@@ -264,8 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t halo_w = static_cast<uint32_t>(halo_cols(KC, SUB, KS));
   const int n_tiles = p.n * p.t * p.tiles_h * p.tiles_w * p.n_ntiles;
   // A stage whose input frame lies before a chunk that has no cache reads
-  // only zeros (not for the stride-2 spatial conv, whose kt counts its nine
-  // spatial taps).
+  // only zeros (not for the stride-2 spatial conv, whose kt counts its
+  // phases or taps).
   auto zero_frame = [&](int t, int kt) {
     return !p.s2 && !p.has_cache && p.stride_t * t + kt - (p.kt - 1) < 0;
   };
@@ -399,13 +412,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          if (KS == 1 && p.s2) {
-            // stride 2 in H and W: stage `kt` is spatial tap (kh, kw) =
-            // (kt / 3, kt % 3); the map walks every other pixel, so the box
-            // of output pixel (h, w) starts at input (2h + kh, 2w + kw)
-            load_a_at(&map_x, sa, cc * KC,
-                      2 * (tc0.w0 + (PAIR ? kTW * rank : 0)) + kt % 3 - p.pad_w,
-                      2 * tc0.h0 + kt / 3 - p.pad_h, tc0.t, tc0.n);
+          if (phases) {
+            // stride 2 in H and W, stage `kt` = phase (a, b) = (kt / 2, kt %
+            // 2): the map walks every other pixel from input (2 w0 + b,
+            // 2 h0 + a), a halo one row and column wider than the tile
+            load_a_at(&map_x, sa, cc * KC, 2 * (tc0.w0 + (PAIR ? kTW * rank : 0)) + (kt & 1),
+                      2 * tc0.h0 + (kt >> 1), tc0.t, tc0.n);
           } else {
             const int tau = p.stride_t * tc0.t + kt - (p.kt - 1);  // input frame
             const bool from_cache = tau < 0;  // (zero frames were skipped above)
@@ -414,16 +426,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (++sa == L.na) { sa = 0; pa ^= 1; }
           if (KS == 1 && p.b_resident) continue;
-          // this A stage's weight slots: g_taps consecutive taps each
+          // this A stage's weight slots: g_taps consecutive taps each (a
+          // phase stage: one slot per tap it serves)
+          const int n_w = phases ? phase_tap_count(kt) : n_groups;
 #pragma unroll 1
-          for (int g = 0; g < n_groups; ++g) {
+          for (int g = 0; g < n_w; ++g) {
             if (!mbar_wait_bounded(&empty_b[sb], pb ^ 1, p.wait_limit_ns, p.status, 2)) {
               ok = false;
               break;
             }
             arm_b(sb, g_taps);
             for (int u = 0; u < g_taps; ++u)
-              load_b(sb, u, static_cast<size_t>(kt * KS * KS + g * g_taps + u) * n_cc + cc,
+              load_b(sb, u,
+                     static_cast<size_t>(phases ? phase_tap(kt, g)
+                                                : kt * KS * KS + g * g_taps + u) * n_cc + cc,
                      tc0.ntile);
             if (++sb == L.nb) { sb = 0; pb ^= 1; }
           }
@@ -553,14 +569,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             mma_stage(a_st, bdesc0 + static_cast<uint32_t>(ia) * bslot16, 0);
           } else {
+            const int q = ia / n_cc;  // (a phase stage's phase)
+            const int n_w = phases ? phase_tap_count(q) : n_groups;
 #pragma unroll 1
-            for (int g = 0; g < n_groups; ++g) {
+            for (int g = 0; g < n_w; ++g) {
               if (!mbar_wait_bounded(&full_b[sb], pb, p.wait_limit_ns, p.status, 4)) {
                 ok = false;
                 break;
               }
               const uint64_t b_slot = bdesc0 + static_cast<uint32_t>(sb) * bslot16;
-              if (g_taps == KS) {
+              if (phases) {
+                // tap (kh, kw) reads its phase at (kh / 2, kw / 2): view
+                // (dh, dw) of the 2 x 2 halo
+                const int tap = phase_tap(q, g);
+                mma_stage(a_st, b_slot, ((tap / 3) >> 1) * KS + ((tap % 3) >> 1));
+              } else if (g_taps == KS) {
                 // one kernel row: taps (g, 0 .. KS-1)
 #pragma unroll
                 for (int u = 0; u < KS; ++u)
@@ -916,6 +939,14 @@ bool finish_config(int ks, int kt, int c_in, UmmaConfig &c) {
     c.na = 8;
     const size_t budget = 200 * 1024 + 4 * static_cast<size_t>(c.params);
     while (c.nb > 2 && smem(c.na, c.nb, 1) > budget) c.na = --c.nb;
+  } else if (ks == 2) {
+    // the stride-2 phase conv: a phase halo serves one to four taps, each
+    // tap a weight slot of its own
+    c.g_taps = 1;
+    c.na = 2;
+    c.nb = 8;
+    const size_t budget = 200 * 1024 + 4 * static_cast<size_t>(c.params);
+    while (c.nb > 2 && smem(c.na, c.nb, 1) > budget) --c.nb;
   } else {
     c.na = 2;
     c.g_taps = ks;
@@ -1089,6 +1120,10 @@ cudaError_t umma_prepare() {
   if (e == cudaSuccess) e = set_smem_attr<96, 1>();
   if (e == cudaSuccess) e = set_smem_attr<128, 3>();
   if (e == cudaSuccess) e = set_smem_attr<128, 1>();
+  // (2 x 2 views of a phase halo: the stride-2 conv)
+  if (e == cudaSuccess) e = set_smem_attr<64, 2>();
+  if (e == cudaSuccess) e = set_smem_attr<32, 2>();
+  if (e == cudaSuccess) e = set_smem_attr<96, 2>();
   return e;
 }
 
@@ -1120,6 +1155,9 @@ UmmaKernel umma_kernel_for(int kc, int ks, int sub, int pair) {
   CC3D_PICK(96, 1)
   CC3D_PICK(128, 3)
   CC3D_PICK(128, 1)
+  CC3D_PICK(64, 2)
+  CC3D_PICK(32, 2)
+  CC3D_PICK(96, 2)
 #undef CC3D_PICK
   return nullptr;
 }
@@ -1160,8 +1198,13 @@ int umma_max_clusters(const UmmaConfig &c, int ks) {
 cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_cache,
                              const CUtensorMap &map_w, const CUtensorMap &map_sc,
                              const UmmaArgs &args, int kc, unsigned grid, cudaStream_t stream) {
-  if (args.kh != args.kw || (args.kh != 1 && args.kh != 3)) return cudaErrorInvalidValue;
+  if (args.kh != args.kw || (args.kh != 1 && args.kh != 3 && !(args.kh == 2 && args.s2)))
+    return cudaErrorInvalidValue;
   if (args.g_taps != 1 && args.g_taps != args.kw) return cudaErrorInvalidValue;
+  // the stride-2 phase conv: four phase stages per channel chunk, one tap
+  // per weight slot
+  if (args.kh == 2 && (args.kt != 4 || args.g_taps != 1 || args.b_resident))
+    return cudaErrorInvalidValue;
   const size_t smem =
       umma_launch_smem(kc, args.nt, args.kh, args.na, args.nb, args.tmem_cols, args.sub,
                        args.g_taps, args.pair,

@@ -42,9 +42,11 @@ struct UmmaArgs {
                                   // c_sc-channel input (map_sc), summed into the accumulator
   int n_cc_sc;                    // its channel chunks, ceil(c_sc / KC) (tail zero-filled)
   int s2;                         // 1: stride 2 in H and W (the downsample path's 3x3 conv
-                                  // per frame): kt = 9 spatial taps of a 1x1 kernel, each
-                                  // read through a map that walks every other pixel; h, w
-                                  // are the output frame's
+                                  // per frame): kt = 4 stages per channel chunk, the
+                                  // input's four stride-2 phases, each read through a map
+                                  // that walks every other pixel and seen through 2 x 2
+                                  // views (kh = kw = 2) by the taps it serves; h, w are
+                                  // the output frame's
   // Frame caches written by the epilogue (null: not written).
   //   cache_out [n][cache_frames][h][w][c_in] = the last cache_frames frames of
   //   concat(cache_in or zeros, x_in), x_in having t_in frames;
