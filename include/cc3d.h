@@ -162,6 +162,12 @@ typedef struct {
                               is split over a cluster of two CTAs (each one
                               half, the row's sum of squares exchanged
                               between them through shared memory)          */
+  int one_frame_mma_ctas;  /* mma_ctas of the tiles that calls of one output
+                              frame use: a plan for max_t > 1 keeps a second
+                              tile choice (and weight image) for them when
+                              the best tiles for one frame differ; every
+                              tile shape gives the same bytes              */
+  int one_frame_n_tile;    /* n_tile of those tiles                          */
 } cc3d_stats;
 
 typedef struct cc3d_plan cc3d_plan;

@@ -105,10 +105,14 @@ def _stream_chunks(plan, x, chunk, cin):
 def test_config2_whole_and_streaming_bitwise_and_oracle():
     """Decoder latent-res conv, C 384 -> 384 on [1,384,5,30,52]: whole
     sequence vs 5 one-frame chunks with a 2-frame cache, identical bytes;
-    both against the full fp64 oracle."""
+    both against the full fp64 oracle.  The plan runs its 5-frame calls on
+    one CTA per tile and its one-frame calls on CTA pairs (a second tile
+    choice with its own weight image)."""
     case = synth.conv_case(384, 384, 5, 30, 52)
     plan, x, y = run_conv(case)
-    assert plan.stats().k_split == 1  # every output sums all taps in one accumulator
+    st = plan.stats()
+    assert st.k_split == 1  # every output sums all taps in one accumulator
+    assert (st.mma_ctas, st.one_frame_mma_ctas) == (1, 2)
     ys = _stream_chunks(plan, x, 1, 384)
     assert torch.equal(ys.cpu(), y.cpu()), "streaming != whole sequence"
     ref = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], _bias64(case["b"]))

@@ -48,7 +48,8 @@ class Stats(ctypes.Structure):
                 ("tiles", ctypes.c_uint64), ("variant", ctypes.c_int), ("tile_h", ctypes.c_int),
                 ("tile_w", ctypes.c_int), ("n_tile", ctypes.c_int), ("k_chunk", ctypes.c_int),
                 ("k_split", ctypes.c_int), ("mma_ctas", ctypes.c_int),
-                ("w_resident", ctypes.c_int), ("row_ctas", ctypes.c_int)]
+                ("w_resident", ctypes.c_int), ("row_ctas", ctypes.c_int),
+                ("one_frame_mma_ctas", ctypes.c_int), ("one_frame_n_tile", ctypes.c_int)]
 
 
 class HostCall(ctypes.Structure):

@@ -294,6 +294,14 @@ struct cc3d_plan {
   UmmaLayer layer;
   CUtensorMap map_w;  // pair: the weight image as 128-byte swizzled rows
   uint8_t *wimg;
+  // Calls of one output frame (streamed chunks) run with the tiles chosen
+  // for one frame when those differ from the plan's (chosen for max_t):
+  // their own layer and weight image.  Every tile shape sums each output's
+  // taps in the same order, so both give the same bytes.
+  bool has_layer1;
+  UmmaLayer layer1;
+  CUtensorMap map_w1;
+  uint8_t *wimg1;
   int c_sc;           // the residual block's fused 1x1x1 conv_shortcut (0: none)
   // fp32 / thin
   void *wraw;
@@ -358,6 +366,7 @@ void free_plan(cc3d_plan *p) {
   if (p->host.down) cudaStreamSynchronize(p->host.down);
   free_host_pipe(p->host);
   cudaFree(p->wimg);
+  cudaFree(p->wimg1);
   cudaFree(p->wraw);
   cudaFree(p->bias);
   cudaFree(p->gamma);
@@ -502,6 +511,7 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
   p->st.k_split = 1;
   p->st.mma_ctas = 1;
   p->st.row_ctas = 1;
+  p->st.one_frame_mma_ctas = 1;
   const int taps = desc->kt * desc->kh * desc->kw;
   cudaError_t e = cudaSuccess;
   if ((s = copy_vec(&p->bias, desc->bias, desc->c_out, true)) != CC3D_OK) goto fail;
@@ -547,6 +557,7 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
     p->st.tile_h = umma_tile_h();
     p->st.tile_w = umma_tile_w();
     p->st.n_tile = p->nt;
+    p->st.one_frame_n_tile = p->nt;
     p->st.k_chunk = p->kpad;
     const size_t bytes = sizeof(__nv_bfloat16) * p->kpad * desc->c_out;
     if (cudaMalloc(&p->wraw, bytes) != cudaSuccess) { s = CC3D_ERR_OOM; goto fail; }
@@ -580,7 +591,7 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
       L.epi = static_cast<int>(desc->epi);
       // Tile configuration (N split, sub-tiles, CTA pair, weight grouping,
       // pipeline depths): a function of (n, c_in, c_out, h, w, epilogue,
-      // max_t), never of a call's t.
+      // max_t), and a second one for one-frame calls.
       UmmaConfig &cfg = L.cfg;
       const bool e4m3 = desc->dtype == CC3D_FP8_E4M3;
       L.e4m3 = e4m3 ? 1 : 0;
@@ -595,10 +606,13 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
         s = CC3D_ERR_UNSUPPORTED;
         goto fail;
       }
-      if (cfg.pair || cfg.xs == 2) {
-        L.max_clusters = umma_max_clusters(cfg, ks_eff);
-        if (L.max_clusters < 1) { s = CC3D_ERR_CUDA; goto fail; }
-      }
+      // the tiles for one-frame calls, when they differ
+      UmmaConfig cfg1;
+      const bool rms_epi = desc->epi == CC3D_EPI_BIAS_RMS_SILU || desc->epi == CC3D_EPI_BIAS_RMS;
+      p->has_layer1 = max_out > 1 &&
+                      choose_umma_config(desc->n, desc->c_in, desc->c_out, h_out, w_out, kt_eff,
+                                         ks_eff, rms_epi, 1, L.sm_count, &cfg1, e4m3) &&
+                      std::memcmp(&cfg1, &cfg, sizeof cfg) != 0;
       p->st.tile_h = umma_tile_h();
       p->st.tile_w = umma_tile_w() * cfg.sub;
       p->st.n_tile = cfg.nt;
@@ -607,47 +621,69 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
       p->st.mma_ctas = cfg.pair ? 2 : 1;
       p->st.row_ctas = cfg.xs == 2 ? 2 : 1;
       p->st.w_resident = cfg.b_resident;
-      // weight image: per N tile, the conv's taps * c_in / kc stages, then the
-      // shortcut's ceil(c_sc / kc) (its channels past c_sc zero)
+      p->st.one_frame_mma_ctas = (p->has_layer1 ? cfg1.pair : cfg.pair) ? 2 : 1;
+      p->st.one_frame_n_tile = p->has_layer1 ? cfg1.nt : cfg.nt;
       p->c_sc = c_sc;
       L.c_sc = c_sc;
-      L.n_cc_sc = c_sc > 0 ? (c_sc + cfg.kc - 1) / cfg.kc : 0;
-      const int conv_stages = taps * (desc->c_in / cfg.kc);
-      const int stages = conv_stages + L.n_cc_sc;
-      // (a stage row is 128 bytes: 64 bf16 or 128 E4M3 channels per 64 / 128)
-      const size_t bytes =
-          static_cast<size_t>(desc->c_out) * stages * cfg.kc * (e4m3 ? 1 : sizeof(__nv_bfloat16));
-      if (cudaMalloc(&p->wimg, bytes) != cudaSuccess) { s = CC3D_ERR_OOM; goto fail; }
-      if (e4m3) {
-        // E4M3 weights, quantised here with the per-channel scales; the
-        // epilogue multiplies by s_x * s_w[c]
-        if ((s = copy_vec(&p->oscale, desc->w_scale, desc->c_out, false)) != CC3D_OK) goto fail;
-        e = launch_repack_umma_e4m3(static_cast<const __nv_bfloat16 *>(desc->weight), p->oscale,
-                                    p->wimg, desc->c_out, desc->c_in, taps, cfg.nt, cfg.pair, 0);
-        if (e == cudaSuccess) e = launch_scale_vector(p->oscale, desc->c_out, desc->x_scale, 0);
-      } else {
-        e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(desc->weight), p->wimg,
-                               desc->c_out, desc->c_in, taps, cfg.nt, cfg.kc, cfg.pair, stages, 0,
-                               0);
-      }
-      if (e == cudaSuccess && c_sc > 0)
-        e = launch_repack_umma(static_cast<const __nv_bfloat16 *>(w_sc), p->wimg, desc->c_out,
-                               c_sc, 1, cfg.nt, cfg.kc, cfg.pair, stages, conv_stages, 0);
-      if (e == cudaSuccess) e = cudaDeviceSynchronize();
-      if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
-      // (a pair's CTA loads half of each MMA N-subtile's rows per box)
-      if (cfg.pair && !encode_weight_map(&p->map_w, p->wimg,
-                                         static_cast<long long>(desc->c_out) * stages,
-                                         cfg.nt / 2, e4m3)) {
-        s = CC3D_ERR_CUDA;
-        goto fail;
-      }
-      L.wimg = p->wimg;
-      L.map_w = &p->map_w;
       L.bias = p->bias;
       L.gamma = p->gamma;
       L.beta = p->beta;
+      if (e4m3 && (s = copy_vec(&p->oscale, desc->w_scale, desc->c_out, false)) != CC3D_OK)
+        goto fail;
+      if (p->has_layer1) {
+        p->layer1 = L;
+        p->layer1.cfg = cfg1;
+      }
+      // weight image of a layer: per N tile, the conv's taps * c_in / kc
+      // stages, then the shortcut's ceil(c_sc / kc) (its channels past c_sc
+      // zero); pairs read it through a tensor map of 128-byte rows
+      auto build = [&](UmmaLayer &Ly, uint8_t **img, CUtensorMap *map) -> cc3d_status {
+        const UmmaConfig &cf = Ly.cfg;
+        if (cf.pair || cf.xs == 2) {
+          Ly.max_clusters = umma_max_clusters(cf, ks_eff);
+          if (Ly.max_clusters < 1) return CC3D_ERR_CUDA;
+        }
+        Ly.n_cc_sc = c_sc > 0 ? (c_sc + cf.kc - 1) / cf.kc : 0;
+        const int conv_stages = taps * (desc->c_in / cf.kc);
+        const int stages = conv_stages + Ly.n_cc_sc;
+        // (a stage row is 128 bytes: 64 bf16 or 128 E4M3 channels per 64 / 128)
+        const size_t bytes = static_cast<size_t>(desc->c_out) * stages * cf.kc *
+                             (e4m3 ? 1 : sizeof(__nv_bfloat16));
+        if (cudaMalloc(img, bytes) != cudaSuccess) return CC3D_ERR_OOM;
+        cudaError_t err;
+        if (e4m3) {
+          // E4M3 weights, quantised here with the per-channel scales (p->oscale
+          // still holds s_w); the epilogue multiplies by s_x * s_w[c]
+          err = launch_repack_umma_e4m3(static_cast<const __nv_bfloat16 *>(desc->weight),
+                                        p->oscale, *img, desc->c_out, desc->c_in, taps, cf.nt,
+                                        cf.pair, 0);
+        } else {
+          err = launch_repack_umma(static_cast<const __nv_bfloat16 *>(desc->weight), *img,
+                                   desc->c_out, desc->c_in, taps, cf.nt, cf.kc, cf.pair, stages,
+                                   0, 0);
+        }
+        if (err == cudaSuccess && c_sc > 0)
+          err = launch_repack_umma(static_cast<const __nv_bfloat16 *>(w_sc), *img, desc->c_out,
+                                   c_sc, 1, cf.nt, cf.kc, cf.pair, stages, conv_stages, 0);
+        if (err == cudaSuccess) err = cudaDeviceSynchronize();
+        if (err != cudaSuccess) return from_cuda(err);
+        // (a pair's CTA loads half of each weight stage's rows per box)
+        if (cf.pair && !encode_weight_map(map, *img, static_cast<long long>(desc->c_out) * stages,
+                                          cf.nt / 2, e4m3))
+          return CC3D_ERR_CUDA;
+        Ly.wimg = *img;
+        Ly.map_w = map;
+        return CC3D_OK;
+      };
+      if ((s = build(L, &p->wimg, &p->map_w)) != CC3D_OK) goto fail;
+      if (p->has_layer1 && (s = build(p->layer1, &p->wimg1, &p->map_w1)) != CC3D_OK) goto fail;
+      if (e4m3) {
+        e = launch_scale_vector(p->oscale, desc->c_out, desc->x_scale, 0);
+        if (e == cudaSuccess) e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
+      }
       L.oscale = p->oscale;
+      if (p->has_layer1) p->layer1.oscale = p->oscale;
     }
   }
   *out = p;
@@ -790,7 +826,9 @@ static cc3d_status forward_impl(cc3d_plan *p, const void *x, int t, const void *
     c.x = x; c.t = t; c.cache_in = cache_in; c.y = y; c.cache_out = cache_out;
     c.residual = residual; c.ncache_in = next_cache_in; c.ncache_out = next_cache_out;
     c.x_sc = x_sc;
-    e = run_umma_layer(p->layer, c, status, stream, &tiles);
+    const bool one_frame = (t - 1) / d.stride_t + 1 == 1;
+    e = run_umma_layer(p->has_layer1 && one_frame ? p->layer1 : p->layer, c, status, stream,
+                       &tiles);
   }
   // (the tensor-core conv writes both caches itself)
   if (p->variant == CC3D_VARIANT_UMMA) {
