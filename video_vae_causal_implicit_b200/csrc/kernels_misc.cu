@@ -229,17 +229,46 @@ __device__ __forceinline__ void rms_cache_store(const RmsCache &k, long long v, 
   }
 }
 
+// Packed fp32 pairs (the f32x2 forms of sm_100): two lanes of math per
+// instruction.
+__device__ __forceinline__ unsigned long long f2_make(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(unsigned long long v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// two bf16 (low half first) as an fp32 pair
+__device__ __forceinline__ unsigned long long f2_from_bf16x2(uint32_t u) {
+  return f2_make(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+
 // Lane-mapped RMS_norm + SiLU for channel counts whose 8-channel groups
 // split evenly over a power-of-two number of lanes: LPV lanes share a voxel,
 // each lane owning GPL groups (GPL = c / 8 / LPV, e.g. C = 192: 8 lanes x 3
 // groups, four voxels per warp).  A warp's loads cover 32 * GPL consecutive
 // 16-byte chunks (fully coalesced, every lane busy); UNR warp passes are
-// loaded before any is used, and four CTAs per SM keep enough bytes in
-// flight to stream at HBM speed.  The sum of squares is reduced with a fixed
-// xor butterfly over the LPV lanes, so the result does not depend on
-// scheduling.
+// loaded before any is used.  The lane's gamma (and beta) stay in registers
+// for the whole loop, and the arithmetic runs on packed fp32 pairs (the
+// kernel issues about as many instructions as it moves bytes, so halving
+// the multiplies and adds shows), with two CTAs of 128-register threads per
+// SM.  The sum of squares is kept as two pair halves, added, then reduced
+// with a fixed xor butterfly over the LPV lanes, so the result does not
+// depend on scheduling.
 template <int GPL, int UNR>
-__global__ void __launch_bounds__(256, 4)
+__global__ void __launch_bounds__(256, 2)
     rmsnorm_silu_lanes_kernel(const __nv_bfloat16 *__restrict__ x,
                               const float *__restrict__ gamma, const float *__restrict__ beta,
                               long long voxels, int c, int lpv,
@@ -250,7 +279,20 @@ __global__ void __launch_bounds__(256, 4)
   const long long warp0 = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) / 32;
   const long long nwarps = static_cast<long long>(gridDim.x) * blockDim.x / 32;
   const float scale = sqrtf(static_cast<float>(c));
-  const int groups = c / 8;
+  // this lane's groups are the same for every voxel: gamma (and beta) once,
+  // halved for SiLU's h = a / 2 (SiLU(a) = h + h * tanh(h))
+  const float half = silu ? 0.5f : 1.0f;
+  unsigned long long hg[GPL][4], hb[GPL][4];
+#pragma unroll
+  for (int k = 0; k < GPL; ++k) {
+    const int g = sub + k * lpv;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      hg[k][q] = f2_make(half * __ldg(gamma + g * 8 + 2 * q), half * __ldg(gamma + g * 8 + 2 * q + 1));
+      hb[k][q] = beta ? f2_make(half * __ldg(beta + g * 8 + 2 * q), half * __ldg(beta + g * 8 + 2 * q + 1))
+                      : 0ull;
+    }
+  }
   for (long long vb = warp0 * vpw * UNR; vb < voxels; vb += nwarps * vpw * UNR) {
     uint4 raw[UNR][GPL];
 #pragma unroll
@@ -265,43 +307,47 @@ __global__ void __launch_bounds__(256, 4)
 #pragma unroll
     for (int u = 0; u < UNR; ++u) {
       const long long v = vb + u * vpw + vloc;
-      float ss = 0.f;
+      unsigned long long ss2 = 0ull;
 #pragma unroll
       for (int k = 0; k < GPL; ++k) {
-        const __nv_bfloat16 *b = reinterpret_cast<const __nv_bfloat16 *>(&raw[u][k]);
+        const uint32_t w4[4] = {raw[u][k].x, raw[u][k].y, raw[u][k].z, raw[u][k].w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float f = __bfloat162float(b[e]);
-          ss = fmaf(f, f, ss);
+        for (int q = 0; q < 4; ++q) {
+          const unsigned long long f = f2_from_bf16x2(w4[q]);
+          ss2 = f2_fma(f, f, ss2);
         }
       }
+      float s0, s1;
+      f2_split(ss2, s0, s1);
+      float ss = s0 + s1;
       for (int o = lpv / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       const float inv = scale / fmaxf(sqrtf(ss), 1e-12f);
       if (v >= voxels) continue;
+      const unsigned long long inv2 = f2_make(inv, inv);
 #pragma unroll
       for (int k = 0; k < GPL; ++k) {
         const int g = sub + k * lpv;
-        const float4 g0 = __ldg(reinterpret_cast<const float4 *>(gamma + g * 8));
-        const float4 g1 = __ldg(reinterpret_cast<const float4 *>(gamma + g * 8) + 1);
-        const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-        const __nv_bfloat16 *b = reinterpret_cast<const __nv_bfloat16 *>(&raw[u][k]);
-        float o[8];
+        const uint32_t w4[4] = {raw[u][k].x, raw[u][k].y, raw[u][k].z, raw[u][k].w};
+        uint32_t ow[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float a = __bfloat162float(b[e]) * inv * gm[e];
-          if (beta) a += __ldg(beta + g * 8 + e);
-          o[e] = silu ? silu_fast(a) : a;
+        for (int q = 0; q < 4; ++q) {
+          // h = x / rms * gamma (+ beta), halved when SiLU follows
+          const unsigned long long h = f2_fma(f2_mul(f2_from_bf16x2(w4[q]), inv2), hg[k][q], hb[k][q]);
+          float h0, h1;
+          f2_split(h, h0, h1);
+          if (silu) {
+            float t0, t1;
+            asm("tanh.approx.f32 %0, %1;" : "=f"(t0) : "f"(h0));
+            asm("tanh.approx.f32 %0, %1;" : "=f"(t1) : "f"(h1));
+            f2_split(f2_fma(h, f2_make(t0, t1), h), h0, h1);
+          }
+          ow[q] = pack2(h0, h1);
         }
-        uint4 w;
-        w.x = pack2(o[0], o[1]);
-        w.y = pack2(o[2], o[3]);
-        w.z = pack2(o[4], o[5]);
-        w.w = pack2(o[6], o[7]);
+        const uint4 w = make_uint4(ow[0], ow[1], ow[2], ow[3]);
         __stcs(reinterpret_cast<uint4 *>(y + v * c) + g, w);
         if (cache.out) rms_cache_store(cache, v, c, g, w);
       }
     }
-    (void)groups;
   }
 }
 
