@@ -440,7 +440,8 @@ cc3d_status check_desc(const cc3d_desc *d, int *variant) {
   }
   if (d->c_in % 32 == 0) {
     if (d->kh != d->kw) return CC3D_ERR_UNSUPPORTED;
-    // one CTA owns each RMS row: up to 256 channels, or 512 as two MMAs
+    // an RMS row: up to 256 channels on one CTA, or up to 512 (steps of 32)
+    // split over the two CTAs of a cluster
     if (rms && d->c_out > 256 && (d->c_out > 512 || d->c_out % 32 != 0))
       return CC3D_ERR_UNSUPPORTED;
     *variant = CC3D_VARIANT_UMMA;
