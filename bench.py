@@ -442,7 +442,39 @@ def main():
                         "causal zero frames (1/9 of the MMAs at T=9) are not executed",
                 "kernels": breakdown}
     del conv1, conv2, a0, a1
-    del blk, xb, yb
+    # two such blocks in a row: each running its own first norm, or the
+    # first block's conv2 epilogue handing the second block its activation
+    bc2 = synth.block_case(cb, Tb, Hb, Wb, seed_base=100)
+    blk2 = cc3d.Block(*(bc2[k].to(dev) for k in ("w1", "b1", "g1", "w2", "b2", "g2")), h=Hb,
+                      w=Wb, max_t=Tb)
+    y2b, a_hand = torch.empty_like(xb), torch.empty_like(xb)
+    chain = {"unfused": lambda: (blk.forward(xb, yb), blk2.forward(yb, y2b)),
+             "fused": lambda: (blk.forward(xb, yb, g_next=blk2.g1, a0_next=a_hand),
+                               blk2.forward(yb, y2b, a0_in=a_hand))}
+    # (the two forms alternate step by step: run one after the other, the
+    # second would run on a hotter, more power-capped GPU)
+    for fn in chain.values():
+        fn()
+        fn()
+    torch.cuda.synchronize()
+    ev = {name: [] for name in chain}
+    for k in range(args.steps):
+        for name, fn in chain.items():
+            ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ea.record(stream)
+            fn()
+            eb.record(stream)
+            ev[name].append((ea, eb))
+    torch.cuda.synchronize()
+    chain_ms = {name: statistics.median(a.elapsed_time(b) for a, b in pairs)
+                for name, pairs in ev.items()}
+    cc3d.sync_status()
+    resblock["chain2"] = {"workload": "two 192ch blocks in a row, x[1,192,9,240,416]",
+                          "unfused_ms": chain_ms["unfused"], "fused_ms": chain_ms["fused"],
+                          "note": "fused: the first block's conv2 epilogue also writes the "
+                                  "second block's SiLU(RMS_norm(y)), which then skips its "
+                                  "stand-alone norm pass"}
+    del blk, blk2, xb, yb, y2b, a_hand
 
     sweep = None if args.no_sweep else run_sweep(args, dev, stream, peaks, flush_l2,
                                                   full=args.sweep)

@@ -306,6 +306,39 @@ cc3d_status cc3d_resblock_forward(cc3d_block *block, const void *x, int t,
                                   void *y, void *cache1_out, void *cache2_out,
                                   void *stream);
 
+/* cc3d_resblock_forward for chains of blocks, with the next block's first
+ * RMS_norm + SiLU moved into this block's conv2 epilogue (§10.4: in a stage
+ * of residual blocks, block k+1 starts with SiLU(RMS_norm(y_k; g1 of k+1))).
+ * Up to c_out = 256 conv2's epilogue computes it from the accumulator row it
+ * stores as y; wider blocks hand over through a norm pass over y after
+ * conv2 (the whole-row tiles such rows need make conv2 slower than that
+ * pass costs).  Either way the next block skips its own first norm.
+ *   a0_in        nullable; else this block's a0 = SiLU(RMS_norm(x; g1)),
+ *                [n][t][h][w][c_in], as the previous block's call wrote it
+ *                into its a0_next: the block's own first norm is skipped
+ *                (x is still read: residual or conv_shortcut input), and
+ *                cache1_out is written by conv1 from cache1_in and a0_in.
+ *   g_next       nullable: device [c_out] fp32, the next block's g1.  With
+ *                it, conv2's epilogue writes y (unchanged) and also
+ *   a0_next      [n][t][h][w][c_out] = SiLU(RMS_norm(y; g_next)), computed
+ *                from y rounded to bf16, with its history
+ *   a0_next_cache_in / a0_next_cache_out  nullable, [n][2][h][w][c_out]:
+ *                the next block's cache1 (last two frames of
+ *                concat(a0_next_cache_in or zeros, a0_next)).
+ * The result equals cc3d_resblock_forward of each block in turn up to the
+ * rounding order of the fused norm's sum of squares.  a0_next without
+ * g_next, or the reverse, or a0_next_cache_* without them, is
+ * CC3D_ERR_INVALID_ARG; a0_next must not overlap x, y, a0_in or any cache
+ * (CC3D_ERR_ALIAS). */
+cc3d_status cc3d_resblock_forward_fused(cc3d_block *block, const void *x,
+                                        const void *a0_in, int t,
+                                        const void *cache1_in,
+                                        const void *cache2_in, void *y,
+                                        void *cache1_out, void *cache2_out,
+                                        const float *g_next, void *a0_next,
+                                        const void *a0_next_cache_in,
+                                        void *a0_next_cache_out, void *stream);
+
 /* Synchronise `stream` and report (then clear) the device status word:
  * CC3D_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
  * CC3D_ERR_CUDA on a CUDA error, else CC3D_OK. */

@@ -32,7 +32,7 @@ def test_header_declares_the_abi():
     names = declared_functions()
     for need in ("cc3d_plan_create", "cc3d_plan_destroy", "cc3d_forward", "rmsnorm_silu",
                  "cc3d_block_create", "cc3d_block_create2", "cc3d_block_destroy",
-                 "cc3d_resblock_forward",
+                 "cc3d_resblock_forward", "cc3d_resblock_forward_fused",
                  "cc3d_sync_status", "cc3d_get_stats", "cc3d_status_string",
                  "cc3d_launch_count"):
         assert need in names
@@ -143,6 +143,8 @@ def test_forward_and_block_null_handles(lib):
         cc3d.ERR_INVALID_ARG
     assert cc3d.cc3d_resblock_forward(None, None, 1, None, None, None, None, None, None) == \
         cc3d.ERR_INVALID_ARG
+    assert cc3d.cc3d_resblock_forward_fused(None, None, None, 1, None, None, None, None, None,
+                                            None, None, None, None, None) == cc3d.ERR_INVALID_ARG
     assert cc3d.cc3d_plan_destroy(None) == cc3d.ERR_INVALID_ARG
     assert cc3d.cc3d_block_destroy(None) == cc3d.ERR_INVALID_ARG
     out = ctypes.c_void_p()

@@ -74,6 +74,8 @@ SIGNATURES = {
                                 ctypes.POINTER(_VP)]),
     "cc3d_block_destroy": (_I, [_VP]),
     "cc3d_resblock_forward": (_I, [_VP, _VP, _I, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "cc3d_resblock_forward_fused": (_I, [_VP, _VP, _VP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                         _VP, _VP, _VP]),
     "cc3d_sync_status": (_I, [_VP]),
     "cc3d_get_stats": (_I, [_VP, ctypes.POINTER(Stats)]),
     "cc3d_status_string": (ctypes.c_char_p, [_I]),
@@ -149,6 +151,14 @@ def cc3d_block_destroy(block):
 def cc3d_resblock_forward(block, x, t, cache1_in, cache2_in, y, cache1_out, cache2_out, stream):
     return lib().cc3d_resblock_forward(block, x, t, cache1_in, cache2_in, y, cache1_out,
                                        cache2_out, stream)
+
+
+def cc3d_resblock_forward_fused(block, x, a0_in, t, cache1_in, cache2_in, y, cache1_out,
+                                cache2_out, g_next, a0_next, a0_next_cache_in, a0_next_cache_out,
+                                stream):
+    return lib().cc3d_resblock_forward_fused(block, x, a0_in, t, cache1_in, cache2_in, y,
+                                             cache1_out, cache2_out, g_next, a0_next,
+                                             a0_next_cache_in, a0_next_cache_out, stream)
 
 
 def cc3d_sync_status(stream):
@@ -259,23 +269,39 @@ class Plan:
 class Block:
     """Residual block, 3x3x3 convs, from C_in = w1.shape[1] to C_out =
     w1.shape[0] channels; w_sc [C_out, C_in, 1, 1, 1] (+ b_sc) is the
-    1x1x1 conv_shortcut (None: the identity shortcut, C_in == C_out)."""
+    1x1x1 conv_shortcut (None: the identity shortcut, C_in == C_out).
+
+    In a chain of blocks, ``forward(..., g_next=next_block.g1, a0_next=A)``
+    also writes the next block's first activation SiLU(RMS_norm(y; g_next))
+    to A (from this block's conv2 epilogue), and the next block takes it as
+    ``forward(y, ..., a0_in=A)``, skipping its own first norm."""
 
     def __init__(self, w1, b1, g1, w2, b2, g2, *, n=1, h, w, max_t, w_sc=None, b_sc=None):
         self.c_out, self.c_in = int(w1.shape[0]), int(w1.shape[1])
         self.c = self.c_out
         keep = [None if t is None else t.contiguous() for t in (w1, b1, g1, w2, b2, g2, w_sc, b_sc)]
+        self.g1 = keep[2].float().contiguous()  # (the previous block's g_next)
         self.handle = ctypes.c_void_p()
         check(cc3d_block_create2(n, self.c_in, self.c_out, h, w, max_t,
                                  *(_ptr(t) for t in keep), self.handle),
               "cc3d_block_create2")
 
     def forward(self, x, y, t=None, cache1_in=None, cache2_in=None, cache1_out=None,
-                cache2_out=None, stream=None):
+                cache2_out=None, stream=None, a0_in=None, g_next=None, a0_next=None,
+                a0_next_cache_in=None, a0_next_cache_out=None):
         t = int(x.shape[1]) if t is None else t
-        check(cc3d_resblock_forward(self.handle, _ptr(x), t, _ptr(cache1_in), _ptr(cache2_in),
-                                    _ptr(y), _ptr(cache1_out), _ptr(cache2_out), _stream(stream)),
-              "cc3d_resblock_forward")
+        if a0_in is None and g_next is None and a0_next is None:
+            check(cc3d_resblock_forward(self.handle, _ptr(x), t, _ptr(cache1_in),
+                                        _ptr(cache2_in), _ptr(y), _ptr(cache1_out),
+                                        _ptr(cache2_out), _stream(stream)),
+                  "cc3d_resblock_forward")
+            return y
+        check(cc3d_resblock_forward_fused(self.handle, _ptr(x), _ptr(a0_in), t, _ptr(cache1_in),
+                                          _ptr(cache2_in), _ptr(y), _ptr(cache1_out),
+                                          _ptr(cache2_out), _ptr(g_next), _ptr(a0_next),
+                                          _ptr(a0_next_cache_in), _ptr(a0_next_cache_out),
+                                          _stream(stream)),
+              "cc3d_resblock_forward_fused")
         return y
 
     def close(self):

@@ -225,7 +225,7 @@ cudaError_t run_umma_layer(const UmmaLayer &L, const UmmaCall &c, int *status,
   a.tiles_w = (w_out + tile_w - 1) / tile_w;
   a.tiles_h = (h_out + umma_tile_h() - 1) / umma_tile_h();
   a.na = cfg.na; a.nb = cfg.nb; a.tmem_cols = cfg.tmem_cols;
-  a.epi = L.epi;
+  a.epi = c.y2 ? 4 : L.epi;
   a.has_cache = has_cache ? 1 : 0;
   // the frame caches, written by the kernel's epilogue
   a.x_in = static_cast<const uint8_t *>(c.x);
@@ -239,6 +239,12 @@ cudaError_t run_umma_layer(const UmmaLayer &L, const UmmaCall &c, int *status,
   a.ncache_out = static_cast<__nv_bfloat16 *>(c.ncache_out);
   a.nc_vec32 = (reinterpret_cast<uintptr_t>(c.ncache_out) & 31u) == 0 ? 1 : 0;
   a.xs = cfg.xs;
+  a.y2 = static_cast<__nv_bfloat16 *>(c.y2);
+  a.y2_vec32 = (reinterpret_cast<uintptr_t>(c.y2) & 31u) == 0 ? 1 : 0;
+  if (c.y2) {
+    a.gamma = c.gamma2;
+    a.beta = nullptr;
+  }
   const uint64_t tiles = static_cast<uint64_t>(L.n) * t_out * a.tiles_h * a.tiles_w * a.n_ntiles;
   uint64_t grid;
   if (cfg.pair || cfg.xs == 2) {
@@ -299,6 +305,7 @@ struct cc3d_plan {
   // their own layer and weight image.  Every tile shape sums each output's
   // taps in the same order, so both give the same bytes.
   bool has_layer1;
+  bool whole_rows;  // tiles hold whole C_out rows (an RMS epilogue may run)
   UmmaLayer layer1;
   CUtensorMap map_w1;
   uint8_t *wimg1;
@@ -331,7 +338,7 @@ struct cc3d_plan {
 
 struct cc3d_block {
   int n, c_in, c_out, h, w, max_t;
-  int fused_rms;    // conv1 applies RMS_norm + SiLU in its epilogue (c_out <= 256)
+  int fused_rms;    // conv1 applies RMS_norm + SiLU in its epilogue (c_out <= 512)
   int shortcut;     // conv2 carries the 1x1x1 conv_shortcut of x (else y += x)
   cc3d_plan *conv1, *conv2;
   float *g1, *g2;   // g2: the stand-alone RMS_norm after conv1 when not fused
@@ -454,7 +461,7 @@ cc3d_status check_desc(const cc3d_desc *d, int *variant) {
 
 namespace {
 cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
-                             const float *b_sc, cc3d_plan **out);
+                             const float *b_sc, cc3d_plan **out, bool whole_rows = false);
 }  // namespace
 
 extern "C" {
@@ -488,9 +495,11 @@ namespace {
 // (c_sc > 0: w_sc [c_out][c_sc] bf16 and b_sc [c_out] fp32, device): its
 // channel chunks become extra K stages of the same accumulator, its bias is
 // added to the conv's.  Only for bf16 3x3x3 stride-1 convs with the bias
-// epilogue (the block's conv2).
+// epilogue (the block's conv2).  whole_rows: tiles that hold whole C_out
+// rows, as an RMS epilogue needs, although the plan's own epilogue has none
+// (a block's conv2, whose calls may also apply the next block's first norm).
 cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
-                             const float *b_sc, cc3d_plan **out) {
+                             const float *b_sc, cc3d_plan **out, bool whole_rows) {
   if (!out) return CC3D_ERR_INVALID_ARG;
   int variant = 0;
   cc3d_status s = check_desc(desc, &variant);
@@ -600,16 +609,16 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
       // (the stride-2 conv: four phase stages seen through 2 x 2 views)
       const int kt_eff = L.s2 ? 4 : desc->kt, ks_eff = L.s2 ? 2 : desc->kh;
       const int h_out = desc->h / desc->stride_h, w_out = desc->w / desc->stride_w;
+      const bool rms_epi = desc->epi == CC3D_EPI_BIAS_RMS_SILU ||
+                           desc->epi == CC3D_EPI_BIAS_RMS || whole_rows;
+      p->whole_rows = rms_epi;
       if (!choose_umma_config(desc->n, desc->c_in, desc->c_out, h_out, w_out, kt_eff, ks_eff,
-                              desc->epi == CC3D_EPI_BIAS_RMS_SILU ||
-                                  desc->epi == CC3D_EPI_BIAS_RMS,
-                              max_out, L.sm_count, &cfg, e4m3)) {
+                              rms_epi, max_out, L.sm_count, &cfg, e4m3)) {
         s = CC3D_ERR_UNSUPPORTED;
         goto fail;
       }
       // the tiles for one-frame calls, when they differ
       UmmaConfig cfg1;
-      const bool rms_epi = desc->epi == CC3D_EPI_BIAS_RMS_SILU || desc->epi == CC3D_EPI_BIAS_RMS;
       p->has_layer1 = max_out > 1 &&
                       choose_umma_config(desc->n, desc->c_in, desc->c_out, h_out, w_out, kt_eff,
                                          ks_eff, rms_epi, 1, L.sm_count, &cfg1, e4m3) &&
@@ -711,10 +720,13 @@ cc3d_status cc3d_get_stats(const cc3d_plan *plan, cc3d_stats *out) {
 }
 
 // cc3d_forward, plus the input of a fused conv_shortcut (x_sc: [n][t][h][w]
-// [c_sc] bf16, required exactly when the plan has one).
+// [c_sc] bf16, required exactly when the plan has one), plus an optional
+// second output of a bias / residual plan with whole-row tiles: y2 =
+// SiLU(RMS_norm(y; gamma2)) with its 2-frame history in next_cache_*.
 static cc3d_status forward_impl(cc3d_plan *p, const void *x, int t, const void *cache_in, void *y,
                                 void *cache_out, const void *residual, const void *next_cache_in,
-                                void *next_cache_out, const void *x_sc, void *stream_v) {
+                                void *next_cache_out, const void *x_sc, void *stream_v,
+                                void *y2 = nullptr, const float *gamma2 = nullptr) {
   if (!p) return CC3D_ERR_INVALID_ARG;
   const cc3d_desc &d = p->d;
   auto reject = [&](cc3d_status s) {
@@ -725,9 +737,14 @@ static cc3d_status forward_impl(cc3d_plan *p, const void *x, int t, const void *
   if (!x || !y || t < 1 || t > d.max_t) return reject(CC3D_ERR_INVALID_ARG);
   if ((d.epi == CC3D_EPI_BIAS_RESIDUAL) != (residual != nullptr))
     return reject(CC3D_ERR_INVALID_ARG);
-  if (d.epi != CC3D_EPI_BIAS_RMS_SILU && d.epi != CC3D_EPI_BIAS_RMS &&
+  if (d.epi != CC3D_EPI_BIAS_RMS_SILU && d.epi != CC3D_EPI_BIAS_RMS && !y2 &&
       (next_cache_in || next_cache_out))
     return reject(CC3D_ERR_INVALID_ARG);
+  // the second output: a bias or residual plan on tiles with whole rows
+  if (y2 && (!gamma2 || !p->whole_rows || p->variant != CC3D_VARIANT_UMMA ||
+             (d.epi != CC3D_EPI_BIAS && d.epi != CC3D_EPI_BIAS_RESIDUAL)))
+    return reject(CC3D_ERR_INVALID_ARG);
+  if (!aligned16(y2)) return reject(CC3D_ERR_ALIGNMENT);
   if ((p->c_sc > 0) != (x_sc != nullptr)) return reject(CC3D_ERR_INVALID_ARG);
   if (!aligned16(x_sc)) return reject(CC3D_ERR_ALIGNMENT);
   // The thin path reads x and the caches with 2-byte loads (or TMA when they
@@ -756,7 +773,10 @@ static cc3d_status forward_impl(cc3d_plan *p, const void *x, int t, const void *
       overlaps(next_cache_out, nc_bytes, next_cache_in, nc_bytes) ||
       overlaps(next_cache_out, nc_bytes, y, y_bytes) ||
       overlaps(next_cache_out, nc_bytes, x, x_bytes) || overlaps(y, y_bytes, x, x_bytes) ||
-      overlaps(y, y_bytes, x_sc, static_cast<size_t>(d.h) * d.w * p->c_sc * 2 * d.n * t))
+      overlaps(y, y_bytes, x_sc, static_cast<size_t>(d.h) * d.w * p->c_sc * 2 * d.n * t) ||
+      overlaps(y2, y_bytes, y, y_bytes) || overlaps(y2, y_bytes, x, x_bytes) ||
+      overlaps(y2, y_bytes, residual, y_bytes) || overlaps(y2, y_bytes, next_cache_in, nc_bytes) ||
+      overlaps(y2, y_bytes, next_cache_out, nc_bytes) || overlaps(y2, y_bytes, cache_out, c_bytes))
     return reject(CC3D_ERR_ALIAS);
   int dev = -1;
   cudaGetDevice(&dev);
@@ -823,10 +843,12 @@ static cc3d_status forward_impl(cc3d_plan *p, const void *x, int t, const void *
     e = launch_conv_thin(mx, mc, my_map, a, static_cast<unsigned>(tiles < slots ? tiles : slots),
                          stream);
   } else {
-    UmmaCall c;
+    UmmaCall c{};
     c.x = x; c.t = t; c.cache_in = cache_in; c.y = y; c.cache_out = cache_out;
     c.residual = residual; c.ncache_in = next_cache_in; c.ncache_out = next_cache_out;
     c.x_sc = x_sc;
+    c.y2 = y2;
+    c.gamma2 = gamma2;
     const bool one_frame = (t - 1) / d.stride_t + 1 == 1;
     e = run_umma_layer(p->has_layer1 && one_frame ? p->layer1 : p->layer, c, status, stream,
                        &tiles);
@@ -1021,9 +1043,9 @@ cc3d_status cc3d_block_create2(int n, int c_in, int c_out, int h, int w, int max
   cc3d_block *b = new cc3d_block();
   std::memset(b, 0, sizeof *b);
   b->n = n; b->c_in = c_in; b->c_out = c_out; b->h = h; b->w = w; b->max_t = max_t;
-  // The RMS epilogue needs a whole C_out row in one N tile (tcgen05's N is
-  // at most 256); wider blocks run conv1 with the bias epilogue and the
-  // stand-alone RMS_norm + SiLU after it.
+  // conv1's RMS epilogue covers rows up to 512 channels (wider than 256:
+  // split over a cluster); wider blocks run conv1 with the bias epilogue and
+  // the stand-alone RMS_norm + SiLU after it.
   b->fused_rms = c_out <= 256 || (c_out <= 512 && c_out % 32 == 0);
   b->shortcut = w_sc != nullptr;
   cc3d_status s;
@@ -1037,7 +1059,13 @@ cc3d_status cc3d_block_create2(int n, int c_in, int c_out, int h, int w, int max
   d.c_in = c_out;
   d.weight = w2; d.bias = b2; d.gamma = nullptr;
   d.epi = b->shortcut ? CC3D_EPI_BIAS : CC3D_EPI_BIAS_RESIDUAL;
-  if ((s = plan_create_impl(&d, b->shortcut ? c_in : 0, w_sc, b_sc, &b->conv2)) != CC3D_OK)
+  // conv2 on whole-row tiles where that costs nothing (up to 256 channels:
+  // the same tiles), so that in a chain its epilogue can also apply the next
+  // block's first norm.  (Wider rows would need the cluster-split tiles,
+  // whose conv2 runs slower than its own CTA-pair tiles by more than the
+  // stand-alone norm pass costs: there the hand-over is that pass.)
+  if ((s = plan_create_impl(&d, b->shortcut ? c_in : 0, w_sc, b_sc, &b->conv2,
+                            c_out <= 256)) != CC3D_OK)
     goto fail;
   if ((s = copy_vec(&b->g1, g1, c_in, false)) != CC3D_OK) goto fail;
   if (!b->fused_rms && (s = copy_vec(&b->g2, g2, c_out, false)) != CC3D_OK) goto fail;
@@ -1076,39 +1104,75 @@ cc3d_status cc3d_block_destroy(cc3d_block *b) {
 cc3d_status cc3d_resblock_forward(cc3d_block *b, const void *x, int t, const void *cache1_in,
                                   const void *cache2_in, void *y, void *cache1_out,
                                   void *cache2_out, void *stream) {
+  return cc3d_resblock_forward_fused(b, x, nullptr, t, cache1_in, cache2_in, y, cache1_out,
+                                     cache2_out, nullptr, nullptr, nullptr, nullptr, stream);
+}
+
+cc3d_status cc3d_resblock_forward_fused(cc3d_block *b, const void *x, const void *a0_in, int t,
+                                        const void *cache1_in, const void *cache2_in, void *y,
+                                        void *cache1_out, void *cache2_out, const float *g_next,
+                                        void *a0_next, const void *a0_next_cache_in,
+                                        void *a0_next_cache_out, void *stream) {
   if (!b || !x || !y || t < 1 || t > b->max_t) return CC3D_ERR_INVALID_ARG;
+  if ((g_next != nullptr) != (a0_next != nullptr) ||
+      (!g_next && (a0_next_cache_in || a0_next_cache_out)))
+    return CC3D_ERR_INVALID_ARG;
   const size_t fin = static_cast<size_t>(b->h) * b->w * b->c_in * 2;
   const size_t fout = static_cast<size_t>(b->h) * b->w * b->c_out * 2;
   const size_t xb = fin * b->n * t, yb = fout * b->n * t;
   const size_t c1 = fin * b->n * 2, c2 = fout * b->n * 2;  // cache1: a0 frames, cache2: a1
-  if (overlaps(x, xb, y, yb)) return CC3D_ERR_ALIAS;
+  if (overlaps(x, xb, y, yb) || overlaps(a0_in, xb, y, yb)) return CC3D_ERR_ALIAS;
   if (overlaps(cache1_out, c1, cache1_in, c1) || overlaps(cache2_out, c2, cache2_in, c2) ||
       overlaps(cache1_out, c1, x, xb) || overlaps(cache1_out, c1, y, yb) ||
       overlaps(cache2_out, c2, x, xb) || overlaps(cache2_out, c2, y, yb) ||
       overlaps(cache1_out, c1, cache2_out, c2) || overlaps(cache1_out, c1, cache2_in, c2) ||
-      overlaps(cache2_out, c2, cache1_in, c1))
+      overlaps(cache2_out, c2, cache1_in, c1) || overlaps(cache1_out, c1, a0_in, xb))
     return CC3D_ERR_ALIAS;
-  // a0 = SiLU(RMS(x; g1)); conv1's cache is a0's history.
-  cc3d_status s = rmsnorm_silu(x, b->g1, nullptr, b->n, t, b->h, b->w, b->c_in, b->a0, cache1_in,
-                               cache1_out, stream);
-  if (s != CC3D_OK) return s;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(a0_in) || !aligned16(a0_next))
+    return CC3D_ERR_ALIGNMENT;
+  if (overlaps(a0_next, yb, x, xb) || overlaps(a0_next, yb, y, yb) ||
+      overlaps(a0_next, yb, a0_in, xb) ||
+      overlaps(a0_next, yb, cache1_in, c1) || overlaps(a0_next, yb, cache1_out, c1) ||
+      overlaps(a0_next, yb, cache2_in, c2) || overlaps(a0_next, yb, cache2_out, c2) ||
+      overlaps(a0_next_cache_out, c2, cache1_out, c1) ||
+      overlaps(a0_next_cache_out, c2, cache2_out, c2))
+    return CC3D_ERR_ALIAS;
+  cc3d_status s = CC3D_OK;
+  // a0 = SiLU(RMS(x; g1)), unless the previous block's conv2 produced it;
+  // conv1's cache is a0's history (written by the norm pass, or else by
+  // conv1 itself from its cache_in and a0)
+  const void *a0 = a0_in;
+  if (!a0_in) {
+    s = rmsnorm_silu(x, b->g1, nullptr, b->n, t, b->h, b->w, b->c_in, b->a0, cache1_in,
+                     cache1_out, stream);
+    if (s != CC3D_OK) return s;
+    a0 = b->a0;
+  }
+  void *conv1_cache_out = a0_in ? cache1_out : nullptr;
   // a1 = SiLU(RMS(conv1(a0) + b1; g2)); conv2's cache is a1's history.
   if (b->fused_rms) {
-    s = cc3d_forward(b->conv1, b->a0, t, cache1_in, b->a1, nullptr, nullptr, cache2_in,
+    s = cc3d_forward(b->conv1, a0, t, cache1_in, b->a1, conv1_cache_out, nullptr, cache2_in,
                      cache2_out, stream);
   } else {
-    s = cc3d_forward(b->conv1, b->a0, t, cache1_in, b->h1, nullptr, nullptr, nullptr, nullptr,
-                     stream);
+    s = cc3d_forward(b->conv1, a0, t, cache1_in, b->h1, conv1_cache_out, nullptr, nullptr,
+                     nullptr, stream);
     if (s == CC3D_OK)
       s = rmsnorm_silu(b->h1, b->g2, nullptr, b->n, t, b->h, b->w, b->c_out, b->a1, cache2_in,
                        cache2_out, stream);
   }
   if (s != CC3D_OK) return s;
-  // y = conv2(a1) + b2 + (x | conv_shortcut(x) + b_sc), fused in conv2.
-  if (b->shortcut)
-    return forward_impl(b->conv2, b->a1, t, cache2_in, y, nullptr, nullptr, nullptr, nullptr, x,
-                        stream);
-  return cc3d_forward(b->conv2, b->a1, t, cache2_in, y, nullptr, x, nullptr, nullptr, stream);
+  // y = conv2(a1) + b2 + (x | conv_shortcut(x) + b_sc), fused in conv2; with
+  // g_next, the same epilogue also writes the next block's a0 (up to 256
+  // channels; wider, a norm pass over y follows)
+  const bool hand_over_in_epilogue = g_next && b->c_out <= 256;
+  s = forward_impl(b->conv2, b->a1, t, cache2_in, y, nullptr, b->shortcut ? nullptr : x,
+                   hand_over_in_epilogue ? a0_next_cache_in : nullptr,
+                   hand_over_in_epilogue ? a0_next_cache_out : nullptr, b->shortcut ? x : nullptr,
+                   stream, hand_over_in_epilogue ? a0_next : nullptr,
+                   hand_over_in_epilogue ? g_next : nullptr);
+  if (s != CC3D_OK || !g_next || hand_over_in_epilogue) return s;
+  return rmsnorm_silu(y, g_next, nullptr, b->n, t, b->h, b->w, b->c_out, a0_next,
+                      a0_next_cache_in, a0_next_cache_out, stream);
 }
 
 cc3d_status cc3d_sync_status(void *stream) {

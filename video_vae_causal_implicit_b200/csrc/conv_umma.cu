@@ -81,8 +81,25 @@ struct SmemLayout {
 // two slots (tile parity).
 constexpr uint32_t kXsBytes = 2u * 4u * 32u * 4u;
 
-// RMS_norm epilogues: 2 with SiLU after it, 3 without.
-__host__ __device__ constexpr bool rms_epilogue(int epi) { return epi == 2 || epi == 3; }
+// RMS_norm epilogues: 2 with SiLU after it, 3 without, 4 the biased (and,
+// with a residual, summed) output stored as y and, as a second output y2,
+// RMS_norm + SiLU of it (the next residual block's first norm).
+__host__ __device__ constexpr bool rms_epilogue(int epi) { return epi == 2 || epi == 3 || epi == 4; }
+
+// 16 bf16 values at `src` as fp32 (zeros when `valid` is false).
+__device__ __forceinline__ void load_bf16x16(const __nv_bfloat16 *src, bool valid, float (&v)[16]) {
+  uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+  if (valid) {
+    a = reinterpret_cast<const uint4 *>(src)[0];
+    b = reinterpret_cast<const uint4 *>(src)[1];
+  }
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
 
 // Epilogue parameters staged in shared memory: bias[c_out] (and, for the
 // RMS epilogues, gamma[c_out], beta[c_out]; for FP8 operands the output
@@ -697,10 +714,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     };
+    // this thread's pixel rows of the residual for tile `tc` into L2 (its
+    // first reads come from HBM, and the epilogue waits for each of them)
+    auto prefetch_residual = [&](const TileCoord &tc) {
+      for (int sbt = 0; sbt < SUB; ++sbt) {
+        const int h = tc.h0 + r, w = tc.w0 + (PAIR ? rank : sbt) * kTW + c;
+        if (h >= p.h || w >= p.w) continue;
+        const size_t pix = (static_cast<size_t>(tc.n) * p.t + tc.t) * p.h * p.w +
+                           static_cast<size_t>(h) * p.w + w;
+        bulk_prefetch_l2(p.residual + pix * p.c_out + tc.ntile * p.nt,
+                         static_cast<uint32_t>(p.nt) * 2u);
+      }
+    };
     for (int tile = tile_first; tile < n_tiles; tile += tile_step, ++it) {
       const int buf = it % p.nbuf;
       const uint32_t use_par = static_cast<uint32_t>((it / p.nbuf) & 1);
       const TileCoord tc0 = decode_tile(tile, p);
+      if (p.residual) {
+        // this tile's rows (the first tile only) and the next tile's, read
+        // one tile from now
+        if (it == 0) prefetch_residual(tc0);
+        if (tile + tile_step < n_tiles) prefetch_residual(decode_tile(tile + tile_step, p));
+      }
       if (tc0.t == p.t - 1) copy_caches(tc0);
       uint32_t got = 0;
       if (lane == 0)
@@ -722,6 +757,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const size_t pix_img = static_cast<size_t>(h) * p.w + w;  // within a frame
         const size_t pix = (static_cast<size_t>(tc0.n) * p.t + tc0.t) * p.h * p.w + pix_img;
         __nv_bfloat16 *yrow = p.y + pix * p.c_out + n0;
+        // epi 4: the normalised activation goes to y2, the residual sum to y
+        __nv_bfloat16 *outrow = p.epi == 4 ? p.y2 + pix * p.c_out + n0 : yrow;
         const __nv_bfloat16 *rrow = p.residual ? p.residual + pix * p.c_out + n0 : nullptr;
         __nv_bfloat16 *ncrow =
             nc_frame >= 0 ? p.ncache_out + (static_cast<size_t>(tc0.n) * 2 + nc_frame) * out_frame +
@@ -732,6 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // pass 1: sum of squares of the biased row h1 (three loads in
           // flight).  h1 is a bf16 activation, as it is when conv1 writes it
           // out for a separate RMS_norm: it is rounded before it is used.
+          // (epi 4: h1 is the residual sum y, the block output)
           float ss = 0.f;
           for (int j0 = 0; j0 < p.nt; j0 += 48) {
             const int nld = (p.nt - j0) >= 48 ? 3 : (p.nt - j0) / 16;
@@ -747,6 +785,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (u >= nld) continue;
               float bv[16];
               ld_param16(s_bias + 4u * static_cast<uint32_t>(n0 + j0 + 16 * u), bv);
+              if (p.epi == 4 && p.residual) {
+                float rv[16];
+                load_bf16x16(rrow + j0 + 16 * u, valid, rv);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) bv[i] += rv[i];
+              }
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const float hv = round_to_bf16(__uint_as_float(raw[16 * u + i]) + bv[i]);
@@ -800,7 +844,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nld = (p.nt - j0) >= 32 ? 2 : 1;
           const bool more = g + 1 < n_groups;
           uint4 res[4];
-          if (p.epi == 1 && valid) {
+          const bool add_res = (p.epi == 1 || (p.epi == 4 && p.residual)) && valid;
+          if (add_res) {
 #pragma unroll
             for (int u = 0; u < 2; ++u)
               if (u < nld) {
@@ -843,7 +888,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(raw[16 * u + i]) + bv[i];
               }
             }
-            if (p.epi == 1 && valid) {
+            if (add_res) {
               const __nv_bfloat16 *rb0 = reinterpret_cast<const __nv_bfloat16 *>(&res[2 * u]);
               const __nv_bfloat16 *rb1 = reinterpret_cast<const __nv_bfloat16 *>(&res[2 * u + 1]);
 #pragma unroll
@@ -851,7 +896,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 v[i] += __bfloat162float(rb0[i]);
                 v[8 + i] += __bfloat162float(rb1[i]);
               }
-            } else if (rms_epilogue(p.epi)) {
+            }
+            if (p.epi == 4 && valid) {
+              // the block output, before the next block's norm
+              uint4 o0, o1;
+              o0.x = pack_bf16x2(v[0], v[1]);
+              o0.y = pack_bf16x2(v[2], v[3]);
+              o0.z = pack_bf16x2(v[4], v[5]);
+              o0.w = pack_bf16x2(v[6], v[7]);
+              o1.x = pack_bf16x2(v[8], v[9]);
+              o1.y = pack_bf16x2(v[10], v[11]);
+              o1.z = pack_bf16x2(v[12], v[13]);
+              o1.w = pack_bf16x2(v[14], v[15]);
+              store_bf16x16(yrow + j, o0, o1, p.vec32);
+            }
+            if (rms_epilogue(p.epi)) {
               float gv[16], be[16];
               ld_param16(s_gamma + 4u * static_cast<uint32_t>(n0 + j), gv);
               ld_param16(s_beta + 4u * static_cast<uint32_t>(n0 + j), be);
@@ -859,7 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int i = 0; i < 16; ++i) {
                 float a = round_to_bf16(v[i]) * inv * gv[i];
                 a += be[i];
-                v[i] = p.epi == 2 ? silu_fast(a) : a;
+                v[i] = p.epi != 3 ? silu_fast(a) : a;
               }
             }
             if (valid) {
@@ -872,7 +931,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               o1.y = pack_bf16x2(v[10], v[11]);
               o1.z = pack_bf16x2(v[12], v[13]);
               o1.w = pack_bf16x2(v[14], v[15]);
-              store_bf16x16(yrow + j, o0, o1, p.vec32);
+              store_bf16x16(outrow + j, o0, o1, p.epi == 4 ? p.y2_vec32 : p.vec32);
               if (ncrow) store_bf16x16(ncrow + j, o0, o1, p.nc_vec32);
             }
           }
@@ -1228,6 +1287,9 @@ cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_ca
   if (args.c_sc < 0 ||
       (args.c_sc > 0 && (args.b_resident || args.c_sc % 8 != 0 ||
                          args.n_cc_sc != (args.c_sc + kc - 1) / kc)))
+    return cudaErrorInvalidValue;
+  // epi 4 (the residual sum and its next-block norm) needs both outputs
+  if (args.epi < 0 || args.epi > 4 || (args.epi == 4) != (args.y2 != nullptr))
     return cudaErrorInvalidValue;
   // FP8 operands (128-channel chunks) come with their output scale and a
   // bias or residual epilogue

@@ -27,7 +27,8 @@ struct UmmaArgs {
   int na, nb;                     // pipeline depths (A halo stages, B weight stages)
   int tmem_cols;
   int epi;                        // 0 bias, 1 bias + residual, 2 bias + RMS + SiLU,
-                                  // 3 bias + RMS
+                                  // 3 bias + RMS, 4 bias + residual -> y, and RMS + SiLU
+                                  // of that sum -> y2 (the next block's first norm)
   int has_cache;
   int sub;                        // MMA sub-tiles (8 x 16 px) per CTA tile, side by side: 1 or 2
   int nbuf;                       // accumulator buffers in tensor memory: 1 or 2
@@ -61,6 +62,8 @@ struct UmmaArgs {
   const __nv_bfloat16 *ncache_in;
   __nv_bfloat16 *ncache_out;
   int nc_vec32;                   // 1: ncache_out is 32-byte aligned (256-bit stores)
+  __nv_bfloat16 *y2;              // epi 4: [n][t][h][w][c_out], the normalised sum
+  int y2_vec32;                   // 1: y2 is 32-byte aligned
   int xs;                         // 2: the two CTAs of a cluster take the same M tiles, CTA
                                   // `rank` N tile `rank` (n_ntiles == 2): an RMS row split
                                   // in halves whose partial sums of squares the CTAs swap
@@ -201,6 +204,10 @@ struct UmmaCall {
   const void *ncache_in;
   void *ncache_out;
   const void *x_sc;
+  // a residual plan's call that also writes y2 = RMS_norm + SiLU(y; gamma2)
+  // (epilogue 4; the plan's tiles must hold whole rows): null = no y2
+  void *y2;
+  const float *gamma2;
 };
 // Encodes the call's tensor maps and launches the conv (one kernel, which
 // also writes cache_out and ncache_out).  Arguments are assumed validated.

@@ -178,7 +178,7 @@ extern "C" cc3d_status cc3d_forward_noalloc(const cc3d_desc *d, const void *x, i
   L.bias = d->bias ? d->bias : zero_bias;
   L.gamma = d->gamma;
   L.beta = d->beta;
-  UmmaCall c;
+  UmmaCall c{};
   c.x = x; c.t = t; c.cache_in = cache_in; c.y = y; c.cache_out = cache_out;
   c.residual = residual; c.ncache_in = next_cache_in; c.ncache_out = next_cache_out;
   c.x_sc = nullptr;

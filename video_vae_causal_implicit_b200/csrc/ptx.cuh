@@ -82,6 +82,11 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 }
 
 // ---- TMA / bulk copies ---------------------------------------------------------
+// `bytes` (a multiple of 16) at `src` (16-byte aligned) into L2, no completion
+// to wait for: a hint that turns later loads of them into L2 hits.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap *map, uint64_t *bar,
                                             int c0, int c1, int c2, int c3, int c4) {
   asm volatile(
