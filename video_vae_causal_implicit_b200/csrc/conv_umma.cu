@@ -173,6 +173,25 @@ __host__ __device__ constexpr int phase_tap(int q, int j) {
   return ((q >> 1) + 2 * (j / ((q & 1) ? 1 : 2))) * 3 + (q & 1) + 2 * (j % ((q & 1) ? 1 : 2));
 }
 
+// The tiles of one CTA, round by round.  In round k its cluster takes unit
+// (a pixel tile, at each N tile the cluster covers) number k * ncl + slot,
+// counting units from the last one -- the last frames first, because a
+// chunk's first frames skip their causal zero taps and cost less -- and the
+// slot runs over the clusters forwards in even rounds and backwards in odd
+// ones, so that the clusters that drew the cheapest units of one round draw
+// the dearest of the next (a serpentine deal: with a few more units than
+// clusters, the spare ones pair up with cheap ones instead of full ones).
+struct TileOrder {
+  int n_units, ncl, cid, per, rank;
+  __device__ __forceinline__ int rounds() const { return (n_units + ncl - 1) / ncl; }
+  // this CTA's tile in round k, or -1 if its cluster has none that round
+  __device__ __forceinline__ int at(int k) const {
+    const int slot = (k & 1) ? ncl - 1 - cid : cid;
+    const int u = k * ncl + slot;
+    return u < n_units ? (n_units - 1 - u) * per + rank : -1;
+  }
+};
+
 __device__ __forceinline__ TileCoord decode_tile(int tile, const UmmaArgs &p) {
   TileCoord c;
   c.ntile = tile % p.n_ntiles;
@@ -269,10 +288,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int rank = (PAIR || xs) ? static_cast<int>(cluster_ctarank()) : 0;
   const int cid = static_cast<int>(blockIdx.x) / csize;
   const int ncl = static_cast<int>(gridDim.x) / csize;
-  // this CTA's tiles: tile_first, tile_first + tile_step, ...  (xs: the
-  // M tiles of its cluster, each at N tile `rank`)
-  const int tile_first = xs ? cid * 2 + rank : cid;
-  const int tile_step = xs ? ncl * 2 : ncl;
   const bool pair_leader = !PAIR || rank == 0;
 
   const int warp = threadIdx.x / 32;
@@ -293,6 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kSw = uses_sw128(KC);
   const uint32_t halo_w = static_cast<uint32_t>(halo_cols(KC, SUB, KS));
   const int n_tiles = p.n * p.t * p.tiles_h * p.tiles_w * p.n_ntiles;
+  // this CTA's tiles (xs: the M tiles of its cluster, each at N tile `rank`)
+  const TileOrder order{xs ? n_tiles / 2 : n_tiles, ncl, cid, xs ? 2 : 1, xs ? rank : 0};
   // A stage whose input frame lies before a chunk that has no cache reads
   // only zeros (not for the stride-2 spatial conv, whose kt counts its
   // phases or taps).
@@ -418,7 +435,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           load_b(st, 0, static_cast<size_t>(st), 0);
         }
       }
-      for (int tile = tile_first; tile < n_tiles && ok; tile += tile_step) {
+      for (int k = 0; k < order.rounds() && ok; ++k) {
+        const int tile = order.at(k);
+        if (tile < 0) continue;
         const TileCoord tc0 = decode_tile(tile, p);
         for (int ia = 0; ia < n_a && ok; ++ia) {
           const int kt = ia / n_cc, cc = ia % n_cc;
@@ -519,7 +538,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int sa = 0, sb = 0;
       uint32_t pa = 0, pb = 0;
       int it = 0;
-      for (int tile = tile_first; tile < n_tiles && ok; tile += tile_step, ++it) {
+      for (int k = 0; k < order.rounds() && ok; ++k) {
+        const int tile = order.at(k);
+        if (tile < 0) continue;
         const int buf = it % p.nbuf;
         const uint32_t use_par = static_cast<uint32_t>((it / p.nbuf) & 1);
         // wait until the epilogue (of both CTAs of a pair) has drained this
@@ -634,6 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // accumulator ready for the epilogue(s)
         release(&acc_full[buf]);
+        ++it;
       }
       // Drain: all MMAs issued here are complete before tensor memory is freed.
       if constexpr (PAIR) umma_commit_pair(drain, 1);
@@ -726,7 +748,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                          static_cast<uint32_t>(p.nt) * 2u);
       }
     };
-    for (int tile = tile_first; tile < n_tiles; tile += tile_step, ++it) {
+    for (int k = 0; k < order.rounds(); ++k) {
+      const int tile = order.at(k);
+      if (tile < 0) continue;
       const int buf = it % p.nbuf;
       const uint32_t use_par = static_cast<uint32_t>((it / p.nbuf) & 1);
       const TileCoord tc0 = decode_tile(tile, p);
@@ -734,7 +758,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // this tile's rows (the first tile only) and the next tile's, read
         // one tile from now
         if (it == 0) prefetch_residual(tc0);
-        if (tile + tile_step < n_tiles) prefetch_residual(decode_tile(tile + tile_step, p));
+        const int next = order.at(k + 1);
+        if (next >= 0) prefetch_residual(decode_tile(next, p));
       }
       if (tc0.t == p.t - 1) copy_caches(tc0);
       uint32_t got = 0;
@@ -944,6 +969,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }  // sub-tiles
       if (!epi_ok) break;
+      ++it;
     }
   }
 
