@@ -168,6 +168,11 @@ typedef struct {
                               the best tiles for one frame differ; every
                               tile shape gives the same bytes              */
   int one_frame_n_tile;    /* n_tile of those tiles                          */
+  uint64_t second_tile_calls; /* calls that ran on that second tile choice:
+                              every one-frame call, and the longer calls it
+                              finishes sooner (e.g. a call without a cache,
+                              whose first frames skip their causal zero
+                              taps)                                         */
 } cc3d_stats;
 
 typedef struct cc3d_plan cc3d_plan;

@@ -105,18 +105,30 @@ def _stream_chunks(plan, x, chunk, cin):
 def test_config2_whole_and_streaming_bitwise_and_oracle():
     """Decoder latent-res conv, C 384 -> 384 on [1,384,5,30,52]: whole
     sequence vs 5 one-frame chunks with a 2-frame cache, identical bytes;
-    both against the full fp64 oracle.  The plan runs its 5-frame calls on
-    one CTA per tile and its one-frame calls on CTA pairs (a second tile
-    choice with its own weight image)."""
+    both against the full fp64 oracle.  The plan's tiles (for 5-frame calls)
+    are one CTA per tile; its second tile choice, CTA pairs with their own
+    weight image, runs the one-frame calls and also this uncached
+    whole-sequence call, whose cheap first frames balance the pair tiles'
+    second round."""
     case = synth.conv_case(384, 384, 5, 30, 52)
     plan, x, y = run_conv(case)
     st = plan.stats()
     assert st.k_split == 1  # every output sums all taps in one accumulator
     assert (st.mma_ctas, st.one_frame_mma_ctas) == (1, 2)
+    assert st.second_tile_calls == 1  # (run_conv's whole-sequence call)
     ys = _stream_chunks(plan, x, 1, 384)
     assert torch.equal(ys.cpu(), y.cpu()), "streaming != whole sequence"
     ref = oracle.causal_conv3d(synth.ncthw_view(x.cpu()), case["w"], _bias64(case["b"]))
     assert_close_bf16(ncthw_np(y), ref, "config 2")
+    # a 5-frame call with a cache (zeros: the same conv) runs on the plan's
+    # own tiles and gives the same bytes
+    before = plan.stats().second_tile_calls
+    zeros = torch.zeros((1, 2, 30, 52, 384), dtype=torch.bfloat16, device="cuda")
+    y_c = torch.empty_like(y)
+    plan.forward(x, y_c, cache_in=zeros)
+    cc3d.sync_status()
+    assert plan.stats().second_tile_calls == before
+    assert torch.equal(y_c.cpu(), y.cpu()), "own tiles != second tiles"
 
 
 def test_config2_streaming_plan_is_bitwise_the_whole_sequence_plan():

@@ -156,3 +156,56 @@ def test_the_documented_choices(probe):
     assert tc384["b_resident"] == 0
     # the latent-resolution layer: kernel-row weight slots
     assert c2["g_taps"] == 3
+
+
+@pytest.fixture(scope="module")
+def deal(tmp_path_factory):
+    if not os.path.exists(cc3d.LIB_PATH):
+        pytest.skip("libcc3d.so is not built")
+    inc = _cuda_include()
+    if inc is None or shutil.which("g++") is None:
+        pytest.skip("needs g++ and the CUDA headers")
+    exe = str(tmp_path_factory.mktemp("deal") / "deal_probe")
+    libdir = os.path.dirname(cc3d.LIB_PATH)
+    subprocess.run(["g++", "-O1", "-std=c++17", "-I", CSRC, "-I", os.path.join(ROOT, "include"),
+                    "-I", inc, os.path.join(HERE, "plan", "deal_probe.cpp"), "-o", exe,
+                    "-L", libdir, "-lcc3d", "-Wl,-rpath," + libdir], check=True)
+
+    def run(cases):
+        text = "\n".join(" ".join(str(int(v)) for v in c) for c in cases) + "\n"
+        out = subprocess.run([exe], input=text, capture_output=True, text=True, check=True).stdout
+        return [dict(zip(("ok", "plan", "one", "pair_plan", "pair_one"), map(int, line.split())))
+                for line in out.splitlines()]
+    return run
+
+
+def dcase(n=1, ci=384, co=384, h=30, w=52, kt=3, ks=3, rms=False, mt=5, sms=148, t_out=5,
+          cached=True, stride=1):
+    return (n, ci, co, h, w, kt, ks, rms, mt, sms, t_out, cached, stride)
+
+
+def test_call_cost_without_a_cache(deal):
+    """A call without a cache skips its first frames' causal zero taps, so it
+    costs less than the same call with one, and a call whose units all fit
+    one wave costs one unit: all kt taps once some output frame reads no
+    zero frame, one tap for a single uncached frame."""
+    cases = [dcase(t_out=t, cached=c) for t in (1, 2, 3, 5) for c in (False, True)]
+    res = deal(cases)
+    for i in range(0, len(res), 2):
+        unc, cac = res[i], res[i + 1]
+        assert unc["ok"] == cac["ok"] == 1
+        assert unc["plan"] <= cac["plan"] and unc["one"] <= cac["one"], cases[i]
+    one_frame_unc, one_frame_cac = res[0], res[1]
+    # one output frame, one wave: the plan tiles' unit with 1 of 3 taps live
+    assert one_frame_cac["plan"] == 3 * one_frame_unc["plan"]
+
+
+def test_uncached_whole_sequence_takes_the_pair_tiles(deal):
+    """The 384-channel latent layer planned for 5 frames: its own tiles (one
+    CTA per tile, one wave) for a 5-frame call with a cache; for the
+    uncached whole-sequence call, the one-frame tiles (CTA pairs), whose
+    six spare tiles are dealt to clusters that drew cheap first-frame tiles."""
+    unc, cac = deal([dcase(cached=False), dcase(cached=True)])
+    assert (unc["pair_plan"], unc["pair_one"]) == (0, 1)
+    assert unc["one"] < unc["plan"]
+    assert cac["one"] > cac["plan"]

@@ -49,7 +49,8 @@ class Stats(ctypes.Structure):
                 ("tile_w", ctypes.c_int), ("n_tile", ctypes.c_int), ("k_chunk", ctypes.c_int),
                 ("k_split", ctypes.c_int), ("mma_ctas", ctypes.c_int),
                 ("w_resident", ctypes.c_int), ("row_ctas", ctypes.c_int),
-                ("one_frame_mma_ctas", ctypes.c_int), ("one_frame_n_tile", ctypes.c_int)]
+                ("one_frame_mma_ctas", ctypes.c_int), ("one_frame_n_tile", ctypes.c_int),
+                ("second_tile_calls", ctypes.c_uint64)]
 
 
 class HostCall(ctypes.Structure):

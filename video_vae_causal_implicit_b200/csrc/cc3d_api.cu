@@ -305,6 +305,10 @@ struct cc3d_plan {
   // their own layer and weight image.  Every tile shape sums each output's
   // taps in the same order, so both give the same bytes.
   bool has_layer1;
+  // per call shape [output frames][with a cache]: whether layer1 finishes it
+  // sooner (the plan's tiles are chosen for max_t frames with a cache; a
+  // call without one has cheap first frames, which may favour layer1's)
+  std::vector<uint8_t> use_layer1;
   bool whole_rows;  // tiles hold whole C_out rows (an RMS epilogue may run)
   UmmaLayer layer1;
   CUtensorMap map_w1;
@@ -693,7 +697,17 @@ cc3d_status plan_create_impl(const cc3d_desc *desc, int c_sc, const void *w_sc,
         if (e != cudaSuccess) { s = from_cuda(e); goto fail; }
       }
       L.oscale = p->oscale;
-      if (p->has_layer1) p->layer1.oscale = p->oscale;
+      if (p->has_layer1) {
+        p->layer1.oscale = p->oscale;
+        p->use_layer1.assign(2 * static_cast<size_t>(max_out + 1), 1);
+        for (int to = 2; to <= max_out; ++to)
+          for (int cached = 0; cached < 2; ++cached)
+            p->use_layer1[2 * to + cached] =
+                umma_deal_cost(cfg1, desc->n, to, h_out, w_out, desc->kt, desc->stride_t,
+                               cached != 0, L.sm_count) <
+                umma_deal_cost(cfg, desc->n, to, h_out, w_out, desc->kt, desc->stride_t,
+                               cached != 0, L.sm_count);
+      }
     }
   }
   *out = p;
@@ -849,9 +863,13 @@ static cc3d_status forward_impl(cc3d_plan *p, const void *x, int t, const void *
     c.x_sc = x_sc;
     c.y2 = y2;
     c.gamma2 = gamma2;
-    const bool one_frame = (t - 1) / d.stride_t + 1 == 1;
-    e = run_umma_layer(p->has_layer1 && one_frame ? p->layer1 : p->layer, c, status, stream,
-                       &tiles);
+    const bool use1 =
+        p->has_layer1 && p->use_layer1[2 * t_out + (cache_in && front > 0 ? 1 : 0)] != 0;
+    e = run_umma_layer(use1 ? p->layer1 : p->layer, c, status, stream, &tiles);
+    if (e == cudaSuccess && use1) {
+      std::lock_guard<std::mutex> lk(p->mu);
+      p->st.second_tile_calls++;
+    }
   }
   // (the tensor-core conv writes both caches itself)
   if (p->variant == CC3D_VARIANT_UMMA) {

@@ -51,7 +51,9 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
+#include <vector>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -1101,6 +1103,36 @@ long long frame_cost(const UmmaConfig &c, int n, int h, int w, int sm_count) {
   return (tiles + slots - 1) / slots * share * steps * mma_cycles(c);
 }
 }  // namespace
+
+long long umma_deal_cost(const UmmaConfig &c, int n, int t_out, int h, int w, int kt,
+                         int stride_t, bool cached, int sm_count) {
+  const long long tiles_w = (w + c.sub * kTW - 1) / (c.sub * kTW), tiles_h = (h + kTH - 1) / kTH;
+  const long long per_frame = tiles_h * tiles_w * (c.xs == 2 ? c.n_ntiles / 2 : c.n_ntiles);
+  const long long units = static_cast<long long>(n) * t_out * per_frame;
+  const bool clusters = c.pair || c.xs == 2;
+  const long long slots =
+      clusters ? sm_count / 2 : static_cast<long long>(sm_count) * c.ctas_per_sm;
+  const long long workers = std::min(units, slots);
+  if (workers < 1 || per_frame < 1) return 0;
+  // one unit with all kt taps live (two CTAs of a plan with two per SM
+  // share it: each runs at half the rate)
+  const long long share = (!clusters && units > sm_count) ? c.ctas_per_sm : 1;
+  const long long unit = share * (c.pair ? 1 : c.sub) * mma_cycles(c);
+  std::vector<long long> load(static_cast<size_t>(workers), 0);
+  for (long long i = 0; i < units; ++i) {
+    // the kernel's TileOrder: the i-th unit dealt is unit units-1-i, to
+    // worker i % workers in even rounds and from the other end in odd ones
+    const long long k = i / workers, slot = i % workers;
+    const long long wk = (k & 1) ? workers - 1 - slot : slot;
+    const long long t = ((units - 1 - i) / per_frame) % t_out;
+    int live = kt;
+    if (!cached)
+      for (int j = 0; j < kt; ++j)
+        if (stride_t * t + j - (kt - 1) < 0) --live;
+    load[static_cast<size_t>(wk)] += unit * live;
+  }
+  return *std::max_element(load.begin(), load.end());
+}
 
 bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
                         int max_t, int sm_count, UmmaConfig *cfg, bool e4m3) {

@@ -81,6 +81,13 @@ struct UmmaConfig {
 // e4m3: FP8 E4M3 operands (128-channel chunks; c_in % 128 == 0).
 bool choose_umma_config(int n, int c_in, int c_out, int h, int w, int kt, int ks, bool rms_epi,
                         int max_t, int sm_count, UmmaConfig *cfg, bool e4m3 = false);
+// Relative time of a call of t_out output frames of n images (h x w) on the
+// tiles of `cfg`, dealt to the CTAs (or clusters) as the kernel deals them;
+// without a cache (`cached` false) an output frame's temporal taps that read
+// the frames before the chunk are skipped.  kt, stride_t: the temporal
+// kernel size and stride.  For choosing a plan's layer per call.
+long long umma_deal_cost(const UmmaConfig &cfg, int n, int t_out, int h, int w, int kt,
+                         int stride_t, bool cached, int sm_count);
 // Clusters of two CTAs that can be resident at once (cfg.pair or cfg.xs),
 // for sizing the grid; 0 when the query fails.
 int umma_max_clusters(const UmmaConfig &cfg, int ks);
