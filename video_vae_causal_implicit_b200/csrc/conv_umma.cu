@@ -360,6 +360,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t smem_base = smem_u32(smem);
   bool ok = true;
+  // The setup above touched only this CTA's own memories: the next conv of
+  // the stream may start its setup now, on the SMs this launch leaves free.
+  // Before their first access to memory that earlier kernels write (x, the
+  // caches, the residual, y), the producer and the epilogue wait for them;
+  // the plan's constants (weights, bias, gamma) need no wait.
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------ producer ------------------------------------
@@ -437,6 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           load_b(st, 0, static_cast<size_t>(st), 0);
         }
       }
+      griddep_wait();
       for (int k = 0; k < order.rounds() && ok; ++k) {
         const int tile = order.at(k);
         if (tile < 0) continue;
@@ -686,6 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (p.oscale) sp[scale_at + i] = p.oscale[i];
     }
+    griddep_wait();
     named_barrier_sync(1, 32 * kEpiWarps);  // (the epilogue warps only)
     // (shared addresses of the three vectors)
     const uint32_t s_bias = smem_u32(sp), s_gamma = s_bias + 4u * static_cast<uint32_t>(p.c_out),
@@ -1279,19 +1287,31 @@ UmmaKernel umma_kernel_for(int kc, int ks, int sub, int pair) {
   return nullptr;
 }
 
+// attr: room for two attributes.  `overlap`: programmatic stream
+// serialization (the kernel may start while the stream's previous kernel
+// runs; it waits for it before reading what that kernel writes).
 cudaLaunchConfig_t umma_launch_config(unsigned grid, size_t smem, int csize, cudaStream_t stream,
-                                      cudaLaunchAttribute *attr) {
+                                      cudaLaunchAttribute *attr, bool overlap = false) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  attr->id = cudaLaunchAttributeClusterDimension;
-  attr->val.clusterDim.x = static_cast<unsigned>(csize);
-  attr->val.clusterDim.y = 1;
-  attr->val.clusterDim.z = 1;
+  unsigned n = 0;
+  if (csize > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = static_cast<unsigned>(csize);
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (overlap) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = csize > 1 ? 1 : 0;
+  cfg.numAttrs = n;
   return cfg;
 }
 }  // namespace
@@ -1302,8 +1322,8 @@ int umma_max_clusters(const UmmaConfig &c, int ks) {
   if (!k) return 0;
   const size_t smem = umma_launch_smem(c.kc, c.nt, ks, c.na, c.nb, c.tmem_cols, c.sub, c.g_taps,
                                        c.pair, c.params, c.xs);
-  cudaLaunchAttribute attr;
-  const cudaLaunchConfig_t cfg = umma_launch_config(2u, smem, 2, nullptr, &attr);
+  cudaLaunchAttribute attr[2];
+  const cudaLaunchConfig_t cfg = umma_launch_config(2u, smem, 2, nullptr, attr);
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void *>(k), &cfg) != cudaSuccess) {
     (void)cudaGetLastError();
@@ -1361,9 +1381,9 @@ cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_ca
     return cudaErrorInvalidValue;
   UmmaKernel k = umma_kernel_for(kc, args.kh, args.sub, args.pair);
   if (!k) return cudaErrorInvalidValue;
-  cudaLaunchAttribute attr;
+  cudaLaunchAttribute attr[2];
   const cudaLaunchConfig_t cfg =
-      umma_launch_config(grid, smem, (args.pair || args.xs == 2) ? 2 : 1, stream, &attr);
+      umma_launch_config(grid, smem, (args.pair || args.xs == 2) ? 2 : 1, stream, attr, true);
   return cudaLaunchKernelEx(&cfg, k, map_x, map_cache, map_w, map_sc, args);
 }
 

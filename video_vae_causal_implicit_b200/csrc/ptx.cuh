@@ -81,6 +81,16 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   }
 }
 
+// ---- programmatic dependent launch ------------------------------------------------
+// Let the next kernel of the stream start (when it was launched with
+// programmatic stream serialization: on SMs this grid leaves free), and wait
+// until the kernels this grid depends on have completed and their writes are
+// visible.  Both are no-ops for a plainly launched grid.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---- TMA / bulk copies ---------------------------------------------------------
 // `bytes` (a multiple of 16) at `src` (16-byte aligned) into L2, no completion
 // to wait for: a hint that turns later loads of them into L2 hits.

@@ -24,6 +24,9 @@ Cases (seeded synthetic inputs, generated on the device):
           + SiLU in its epilogue, each 192-channel half of a row on one CTA
           of a two-CTA cluster)
   c2f8    the 384 -> 384 conv of c2 on FP8 E4M3 operands
+  c4chain two c4 blocks in a row, the first one's conv2 epilogue also
+          writing the second one's SiLU(RMS_norm(y)) (launches: rmsnorm,
+          conv1, conv2 with the hand-over; conv1, conv2)
 Prints nothing but a final "ok"; timing comes from the profiler.
 """
 from __future__ import annotations
@@ -48,8 +51,8 @@ def build_case(name, dev):
         c, T, H, W = 3, 17, 480, 832
     elif name == "c3b":
         c, T, H, W = 96, 17, 480, 832
-    elif name in ("c4", "c4s"):
-        c, T, H, W = 192, (9 if name == "c4" else 3), 240, 416
+    elif name in ("c4", "c4s", "c4chain"):
+        c, T, H, W = 192, (3 if name == "c4s" else 9), 240, 416
     elif name == "c5big":
         c, T, H, W = 384, 1, 360, 640
     elif name == "tc192":
@@ -77,6 +80,22 @@ def build_case(name, dev):
         blk = cc3d.Block(w1, b1, g1, w2, b2, g2, h=H, w=W, max_t=T)
         y = torch.empty_like(x)
         return lambda: blk.forward(x, y), [blk]
+    if name == "c4chain":
+        blks = []
+        for s in (0, 10):
+            blks.append(cc3d.Block(synth.kaiming_uniform(c, c, (3, 3, 3), 1 + s).to(dev),
+                                   synth.uniform((c,), -0.1, 0.1, 2 + s).to(dev),
+                                   synth.uniform((c,), 0.5, 1.5, 3 + s).to(dev),
+                                   synth.kaiming_uniform(c, c, (3, 3, 3), 4 + s).to(dev),
+                                   synth.uniform((c,), -0.1, 0.1, 5 + s).to(dev),
+                                   synth.uniform((c,), 0.5, 1.5, 6 + s).to(dev),
+                                   h=H, w=W, max_t=T))
+        y0, y1, a1 = torch.empty_like(x), torch.empty_like(x), torch.empty_like(x)
+
+        def run():
+            blks[0].forward(x, y0, g_next=blks[1].g1, a0_next=a1)
+            blks[1].forward(y0, y1, a0_in=a1)
+        return run, blks
     if name == "ds96":
         wt = synth.kaiming_uniform(c, c, (1, 3, 3), 1).to(dev)
         b = synth.uniform((c,), -0.1, 0.1, 2).to(dev)
