@@ -303,6 +303,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool phases = KS == 2 && p.s2;
   const int n_conv_stages = (phases ? 9 : p.kt * KS * KS) * n_cc;
   const int n_sc = p.c_sc > 0 ? p.n_cc_sc : 0;
+  // A 1x1 spatial kernel feeds only kSteps MMAs per halo stage, too few to
+  // hide a stage's barrier wait and commit: with resident weights (no weight
+  // waits at all) `a_grp` consecutive channel chunks of one frame (in
+  // consecutive A slots) share the first slot's full and empty barriers, one
+  // wait and one commit per group.  (With streamed weights the longer groups
+  // keep fewer halos in flight and cost more than they save.)
+  const int a_grp = (KS == 1 && p.b_resident && n_sc == 0)
+                        ? ((n_cc % 3 == 0 && L.na % 3 == 0)   ? 3
+                           : (n_cc % 2 == 0 && L.na % 2 == 0) ? 2
+                                                              : 1)
+                        : 1;
   const int stages_per_ntile = n_conv_stages + n_sc;  // weight image
   // weight slots per A stage: one per group of g_taps spatial taps
   const int g_taps = p.g_taps;
@@ -407,30 +418,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // channels c0 .. c0+KC-1 of the box of `map` that starts at column
       // wc, row hc of frame `tcoord` of image `n`, into A slot `slot`
+      // (completing on the barrier of slot `bar`: the first of its group)
       auto load_a_at = [&](const CUtensorMap *map, int slot, int c0, int wc, int hc, int tcoord,
-                           int n) {
+                           int n, int bar) {
         const uint32_t dst = smem_base + L.a_off + slot * L.a_stage;
         if constexpr (PAIR) {
-          tma_load_5d_pair(dst, map, lead_full_a + 8u * slot, c0, wc, hc, tcoord, n);
+          tma_load_5d_pair(dst, map, lead_full_a + 8u * bar, c0, wc, hc, tcoord, n);
         } else if constexpr (kSw) {
-          tma_load_5d(dst, map, &full_a[slot], c0, wc, hc, tcoord, n);
+          tma_load_5d(dst, map, &full_a[bar], c0, wc, hc, tcoord, n);
         } else {
 #pragma unroll
           for (int s = 0; s < KC / 8; ++s)
-            tma_load_5d(dst + s * L.slab, map, &full_a[slot], c0 + s * 8, wc, hc, tcoord, n);
+            tma_load_5d(dst + s * L.slab, map, &full_a[bar], c0 + s * 8, wc, hc, tcoord, n);
         }
       };
       // the tile's halo of channels c0 .. c0+KC-1 of frame `tcoord` of `map`
       // into A slot `slot` (on a pair, this CTA's 8-column half of the tile)
       auto load_a = [&](const CUtensorMap *map, int slot, int c0, int tcoord,
-                        const TileCoord &tc) {
+                        const TileCoord &tc, int bar) {
         load_a_at(map, slot, c0, tc.w0 + (PAIR ? kTW * rank : 0) - KS / 2, tc.h0 - KS / 2, tcoord,
-                  tc.n);
+                  tc.n, bar);
       };
       // wait for A slot `sa` to be free and arm it
       auto take_a = [&]() -> bool {
         if (!mbar_wait_bounded(&empty_a[sa], pa ^ 1, p.wait_limit_ns, p.status, 1)) return false;
-        if (pair_leader) mbar_arrive_expect_tx(&full_a[sa], PAIR ? 2u * a_tx : a_tx);
+        if (pair_leader)
+          mbar_arrive_expect_tx(&full_a[sa],
+                                (PAIR ? 2u : 1u) * static_cast<uint32_t>(a_grp) * a_tx);
         a_used |= 1u << sa;
         a_par = (a_par & ~(1u << sa)) | (pa << sa);
         return true;
@@ -448,29 +462,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tile = order.at(k);
         if (tile < 0) continue;
         const TileCoord tc0 = decode_tile(tile, p);
-        for (int ia = 0; ia < n_a && ok; ++ia) {
-          const int kt = ia / n_cc, cc = ia % n_cc;
+        for (int ia = 0; ia < n_a && ok; ia += a_grp) {
+          const int kt = ia / n_cc, cc0 = ia % n_cc;
           // A frame before the chunk with no cache is all zeros: its stage
           // (and its taps' weights) is skipped here and by the MMA issuer.
           if (zero_frame(tc0.t, kt)) continue;
+          // the group's a_grp stages (chunks cc0 .. of frame kt) complete on
+          // the barrier of its first slot
           if (!take_a()) {
             ok = false;
             break;
           }
-          if (phases) {
-            // stride 2 in H and W, stage `kt` = phase (a, b) = (kt / 2, kt %
-            // 2): the map walks every other pixel from input (2 w0 + b,
-            // 2 h0 + a), a halo one row and column wider than the tile
-            load_a_at(&map_x, sa, cc * KC, 2 * (tc0.w0 + (PAIR ? kTW * rank : 0)) + (kt & 1),
-                      2 * tc0.h0 + (kt >> 1), tc0.t, tc0.n);
-          } else {
-            const int tau = p.stride_t * tc0.t + kt - (p.kt - 1);  // input frame
-            const bool from_cache = tau < 0;  // (zero frames were skipped above)
-            load_a(from_cache ? &map_cache : &map_x, sa, cc * KC,
-                   from_cache ? tau + (p.kt - 1) : tau, tc0);
+          const int bar = sa;
+          for (int u = 0; u < a_grp; ++u) {
+            if (phases) {
+              // stride 2 in H and W, stage `kt` = phase (a, b) = (kt / 2, kt %
+              // 2): the map walks every other pixel from input (2 w0 + b,
+              // 2 h0 + a), a halo one row and column wider than the tile
+              load_a_at(&map_x, sa + u, cc0 * KC,
+                        2 * (tc0.w0 + (PAIR ? kTW * rank : 0)) + (kt & 1), 2 * tc0.h0 + (kt >> 1),
+                        tc0.t, tc0.n, bar);
+            } else {
+              const int tau = p.stride_t * tc0.t + kt - (p.kt - 1);  // input frame
+              const bool from_cache = tau < 0;  // (zero frames were skipped above)
+              load_a(from_cache ? &map_cache : &map_x, sa + u, (cc0 + u) * KC,
+                     from_cache ? tau + (p.kt - 1) : tau, tc0, bar);
+            }
           }
-          if (++sa == L.na) { sa = 0; pa ^= 1; }
+          sa += a_grp;
+          if (sa == L.na) { sa = 0; pa ^= 1; }
           if (KS == 1 && p.b_resident) continue;
+          for (int u = 0; u < a_grp && ok; ++u) {
+          const int cc = cc0 + u;
           // this A stage's weight slots: g_taps consecutive taps each (a
           // phase stage: one slot per tap it serves)
           const int n_w = phases ? phase_tap_count(kt) : n_groups;
@@ -481,13 +504,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             arm_b(sb, g_taps);
-            for (int u = 0; u < g_taps; ++u)
-              load_b(sb, u,
+            for (int v = 0; v < g_taps; ++v)
+              load_b(sb, v,
                      static_cast<size_t>(phases ? phase_tap(kt, g)
-                                                : kt * KS * KS + g * g_taps + u) * n_cc + cc,
+                                                : kt * KS * KS + g * g_taps + v) * n_cc + cc,
                      tc0.ntile);
             if (++sb == L.nb) { sb = 0; pb ^= 1; }
           }
+          }  // the group's stages
         }
         // the residual block's 1x1x1 conv_shortcut: each channel chunk of
         // the block input at the output frame (a halo like the conv's, read
@@ -498,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          load_a(&map_sc, sa, c2 * KC, tc0.t, tc0);
+          load_a(&map_sc, sa, c2 * KC, tc0.t, tc0, sa);
           if (++sa == L.na) { sa = 0; pa ^= 1; }
           if (!mbar_wait_bounded(&empty_b[sb], pb ^ 1, p.wait_limit_ns, p.status, 2)) {
             ok = false;
@@ -546,6 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t bstage16 = L.b_stage >> 4, bslot16 = L.b_slot >> 4;
       int sa = 0, sb = 0;
       uint32_t pa = 0, pb = 0;
+      uint32_t b_seen = 0;  // resident weight slots already seen loaded
       int it = 0;
       for (int k = 0; k < order.rounds() && ok; ++k) {
         const int tile = order.at(k);
@@ -598,25 +623,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (PAIR) umma_commit_pair(bar, 3);
           else umma_commit(bar);
         };
-        for (int ia = 0; ia < n_a && ok; ++ia) {
+        for (int ia = 0; ia < n_a && ok; ia += a_grp) {
           // the same zero-frame stages the producer skipped; adding their
           // exact zeros would not change the accumulator
           if (zero_frame(tcm.t, ia / n_cc)) continue;
+          // (a group of a_grp stages: one wait, one release)
           if (!mbar_wait_bounded(&full_a[sa], pa, p.wait_limit_ns, p.status, 3)) {
             ok = false;
             break;
           }
-          const uint64_t a_st = adesc0 + ((sa * L.a_stage) >> 4);
+          for (int u = 0; u < a_grp && ok; ++u) {
+          const int is = ia + u;  // this stage: (kt, cc) = (is / n_cc, is % n_cc)
+          const uint64_t a_st = adesc0 + (((sa + u) * L.a_stage) >> 4);
           if (KS == 1 && p.b_resident) {
             // resident weights: stage (kt, cc) sits in slot kt * n_cc + cc,
-            // loaded once (its first phase stays complete) and never freed
-            if (!mbar_wait_bounded(&full_b[ia], 0u, p.wait_limit_ns, p.status, 4)) {
-              ok = false;
-              break;
+            // loaded once (its first phase stays complete) and never freed,
+            // so it is waited for once (a bit per slot: at most 32 slots)
+            if (!(b_seen >> is & 1u)) {
+              if (!mbar_wait_bounded(&full_b[is], 0u, p.wait_limit_ns, p.status, 4)) {
+                ok = false;
+                break;
+              }
+              b_seen |= 1u << is;
             }
-            mma_stage(a_st, bdesc0 + static_cast<uint32_t>(ia) * bslot16, 0);
+            mma_stage(a_st, bdesc0 + static_cast<uint32_t>(is) * bslot16, 0);
           } else {
-            const int q = ia / n_cc;  // (a phase stage's phase)
+            const int q = is / n_cc;  // (a phase stage's phase)
             const int n_w = phases ? phase_tap_count(q) : n_groups;
 #pragma unroll 1
             for (int g = 0; g < n_w; ++g) {
@@ -645,8 +677,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
           }
+          }  // the group's stages
+          if (!ok) break;
           release(&empty_a[sa]);
-          if (++sa == L.na) { sa = 0; pa ^= 1; }
+          sa += a_grp;
+          if (sa == L.na) { sa = 0; pa ^= 1; }
         }
         // the conv_shortcut's chunks: the centre tap of each halo
         for (int c2 = 0; c2 < n_sc && ok; ++c2) {
