@@ -457,7 +457,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           load_b(st, 0, static_cast<size_t>(st), 0);
         }
       }
-      griddep_wait();
+      // the weight slots of a group of A stages (chunks cc0 .. of frame kt)
+      auto load_weights = [&](int kt, int cc0, const TileCoord &tc0) -> bool {
+        for (int u = 0; u < a_grp; ++u) {
+          const int cc = cc0 + u;
+          // this A stage's weight slots: g_taps consecutive taps each (a
+          // phase stage: one slot per tap it serves)
+          const int n_w = phases ? phase_tap_count(kt) : n_groups;
+#pragma unroll 1
+          for (int g = 0; g < n_w; ++g) {
+            if (!mbar_wait_bounded(&empty_b[sb], pb ^ 1, p.wait_limit_ns, p.status, 2))
+              return false;
+            arm_b(sb, g_taps);
+            for (int v = 0; v < g_taps; ++v)
+              load_b(sb, v,
+                     static_cast<size_t>(phases ? phase_tap(kt, g)
+                                                : kt * KS * KS + g * g_taps + v) * n_cc + cc,
+                     tc0.ntile);
+            if (++sb == L.nb) { sb = 0; pb ^= 1; }
+          }
+        }
+        return true;
+      };
+      bool dep_waited = false;  // (griddep_wait issued)
       for (int k = 0; k < order.rounds() && ok; ++k) {
         const int tile = order.at(k);
         if (tile < 0) continue;
@@ -467,6 +489,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           // A frame before the chunk with no cache is all zeros: its stage
           // (and its taps' weights) is skipped here and by the MMA issuer.
           if (zero_frame(tc0.t, kt)) continue;
+          // The first stage's weights (plan constants) go out before the
+          // wait for the previous kernel of the stream when the ring holds
+          // them all without the MMAs freeing a slot; its halo after it.
+          const bool streamed = !(KS == 1 && p.b_resident);
+          const bool early_w =
+              !dep_waited && streamed &&
+              a_grp * (phases ? phase_tap_count(kt) : n_groups) <= L.nb;
+          if (early_w && !load_weights(kt, cc0, tc0)) {
+            ok = false;
+            break;
+          }
+          if (!dep_waited) {
+            griddep_wait();
+            dep_waited = true;
+          }
           // the group's a_grp stages (chunks cc0 .. of frame kt) complete on
           // the barrier of its first slot
           if (!take_a()) {
@@ -491,32 +528,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           sa += a_grp;
           if (sa == L.na) { sa = 0; pa ^= 1; }
-          if (KS == 1 && p.b_resident) continue;
-          for (int u = 0; u < a_grp && ok; ++u) {
-          const int cc = cc0 + u;
-          // this A stage's weight slots: g_taps consecutive taps each (a
-          // phase stage: one slot per tap it serves)
-          const int n_w = phases ? phase_tap_count(kt) : n_groups;
-#pragma unroll 1
-          for (int g = 0; g < n_w; ++g) {
-            if (!mbar_wait_bounded(&empty_b[sb], pb ^ 1, p.wait_limit_ns, p.status, 2)) {
-              ok = false;
-              break;
-            }
-            arm_b(sb, g_taps);
-            for (int v = 0; v < g_taps; ++v)
-              load_b(sb, v,
-                     static_cast<size_t>(phases ? phase_tap(kt, g)
-                                                : kt * KS * KS + g * g_taps + v) * n_cc + cc,
-                     tc0.ntile);
-            if (++sb == L.nb) { sb = 0; pb ^= 1; }
+          if (!streamed || early_w) continue;
+          if (!load_weights(kt, cc0, tc0)) {
+            ok = false;
+            break;
           }
-          }  // the group's stages
         }
         // the residual block's 1x1x1 conv_shortcut: each channel chunk of
         // the block input at the output frame (a halo like the conv's, read
         // at its centre tap) against one weight stage stored after the
         // conv's, into the same accumulator
+        if (n_sc > 0 && !dep_waited) {
+          griddep_wait();
+          dep_waited = true;
+        }
         for (int c2 = 0; c2 < n_sc && ok; ++c2) {
           if (!take_a()) {
             ok = false;
