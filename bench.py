@@ -1,6 +1,7 @@
 """Benchmark of the causal Conv3D hot path (libcc3d.so) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cc3d|reference] [--sweep|--no-sweep]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cc3d|reference]
+                    [--quick-sweep|--no-sweep]
 
 Workload (one "step"): the decoder latent-resolution causal conv,
 bf16, C_in = C_out = 384 on x[1, 384, 5, 30, 52], 3x3x3, run once over the
@@ -15,11 +16,12 @@ RMS_norm+SiLU -> conv -> RMS_norm+SiLU (fused) -> conv + x (fused)) as
 ``resblock`` with its latency, and as ``sweep`` the encoder convs (3 -> 96,
 96 -> 96 at 17 x 480 x 832), the downsample path's time_conv (kernel
 (3, 1, 1), stride 2 in time, at 192 and 384 channels) and its per-frame
-3x3 stride-2 conv (96 channels, 480 x 832 -> 240 x 416), and the
-384-channel rows of the streaming channel/resolution sweep (21 one-frame
-chunks, CUDA-graph captured).  ``--sweep`` adds the sweep's 96- and
-192-channel rows and the encoder's residual blocks (96 -> 192, 192 -> 384
-and a 384-channel one); ``--no-sweep`` drops the sweep.
+3x3 stride-2 conv (96 channels, 480 x 832 -> 240 x 416), all nine rows of
+the streaming channel/resolution sweep (C = 96, 192, 384 at three sizes, 21
+one-frame chunks each, CUDA-graph captured) and the encoder's residual
+blocks (96 -> 192, 192 -> 384 and a 384-channel one).  ``--quick-sweep``
+keeps only the 384-channel rows and the 384-channel block; ``--no-sweep``
+drops the sweep.
 
 Multi-GPU: the path runs as independent replicas (one process per GPU, no
 data-path collective); ``value`` is the FLOP all ranks processed divided by
@@ -188,8 +190,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cc3d", choices=["cc3d", "reference"])
     ap.add_argument("--sweep", action="store_true",
-                    help="time every sweep row (C = 96 and 192 of config 5, the encoder blocks) "
-                         "besides the default ones")
+                    help="(the default) time every sweep row: all nine config 5 rows and the "
+                         "encoder blocks")
+    ap.add_argument("--quick-sweep", action="store_true",
+                    help="time only the 384-channel rows of config 5 and one encoder block")
     ap.add_argument("--no-sweep", action="store_true", help="skip the sweep rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -498,7 +502,7 @@ def main():
     del blk, blk2, xb, yb, y2b, a_hand
 
     sweep = None if args.no_sweep else run_sweep(args, dev, stream, peaks, flush_l2,
-                                                  full=args.sweep)
+                                                  full=not args.quick_sweep)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
