@@ -12,9 +12,9 @@
 // CTA tile is SUB = 1 or 2 such MMA tiles side by side (8 or 16 columns);
 // with two, every weight stage feeds two MMAs.  A CTA pair (cluster of two
 // CTAs on one SM pair) takes a 16 x 16 tile with 2-SM MMAs (M = 256).  The
-// kernel is persistent: one CTA (or pair) per SM walks the tiles
-// round-robin.  The K loop of a tile runs over (kt, channel chunk of KC,
-// kh, kw).
+// kernel is persistent: one CTA (or pair) per SM takes its tiles in rounds,
+// last frame first and serpentine over the clusters (TileOrder).  The K loop
+// of a tile runs over (kt, channel chunk of KC, kh, kw).
 //
 // A operand: for each (kt, channel chunk) the input halo of the tile --
 // (TH + kh - 1) x (SUB * TW + kw - 1) pixels x KC channels -- arrives by TMA
@@ -35,7 +35,8 @@
 //
 // Epilogue.  Four warps read the accumulator from tensor memory and apply
 // bias (once), then the residual add, or RMS_norm over the whole C_out row
-// followed by SiLU, and store bf16.  The same warps write the frame caches
+// followed by SiLU, and store bf16 (or, for a residual block in a chain,
+// store y and also SiLU(RMS_norm(y)) for the next block).  The same warps write the frame caches
 // of the call: the input cache (the last kt-1 frames of concat(cache_in,
 // x)) is copied tile by tile by the tiles of the last output frame, and the
 // RMS epilogue's own output frames go to next_cache_out as they are
@@ -46,7 +47,9 @@
 // epilogue.  Two accumulators live in tensor memory when they fit, so the
 // epilogue of one tile overlaps the MMAs of the next.  Stages are handed
 // over with mbarriers; every wait is bounded and reports through the status
-// word instead of hanging.
+// word instead of hanging.  Launches overlap: after its setup a CTA lets the
+// stream's next conv start (programmatic dependent launch), and it waits for
+// the previous kernel only before touching memory that kernel may write.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
