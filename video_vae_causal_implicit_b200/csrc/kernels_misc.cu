@@ -260,15 +260,17 @@ __device__ __forceinline__ unsigned long long f2_from_bf16x2(uint32_t u) {
 // each lane owning GPL groups (GPL = c / 8 / LPV, e.g. C = 192: 8 lanes x 3
 // groups, four voxels per warp).  A warp's loads cover 32 * GPL consecutive
 // 16-byte chunks (fully coalesced, every lane busy); UNR warp passes are
-// loaded before any is used.  The lane's gamma (and beta) stay in registers
-// for the whole loop, and the arithmetic runs on packed fp32 pairs (the
-// kernel issues about as many instructions as it moves bytes, so halving
-// the multiplies and adds shows), with two CTAs of 128-register threads per
-// SM.  The sum of squares is kept as two pair halves, added, then reduced
-// with a fixed xor butterfly over the LPV lanes, so the result does not
-// depend on scheduling.
-template <int GPL, int UNR>
-__global__ void __launch_bounds__(256, 2)
+// loaded before any is used.  Gamma (and beta, when given) sit in shared
+// memory as pre-halved fp32 pairs, which keeps the thread at 80 registers:
+// three CTAs per SM, 24 warps to cover the loads' latency (with them in
+// registers, two CTAs of 128-register threads).  The arithmetic runs on
+// packed fp32 pairs (the kernel issues about as many instructions as it
+// moves bytes, so halving the multiplies and adds shows).  The sum of
+// squares is kept as two pair halves, added, then reduced with a fixed xor
+// butterfly over the LPV lanes, so the result does not depend on
+// scheduling.
+template <int GPL, int UNR, bool BETA>
+__global__ void __launch_bounds__(256, 3)
     rmsnorm_silu_lanes_kernel(const __nv_bfloat16 *__restrict__ x,
                               const float *__restrict__ gamma, const float *__restrict__ beta,
                               long long voxels, int c, int lpv,
@@ -279,20 +281,16 @@ __global__ void __launch_bounds__(256, 2)
   const long long warp0 = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) / 32;
   const long long nwarps = static_cast<long long>(gridDim.x) * blockDim.x / 32;
   const float scale = sqrtf(static_cast<float>(c));
-  // this lane's groups are the same for every voxel: gamma (and beta) once,
-  // halved for SiLU's h = a / 2 (SiLU(a) = h + h * tanh(h))
+  // gamma (and beta), halved for SiLU's h = a / 2 (SiLU(a) = h + h *
+  // tanh(h)), as fp32 pairs in shared memory: read where they are used, so
+  // that three CTAs fit per SM (kept in registers they cost 24-48 of them)
+  __shared__ unsigned long long s_g[512], s_b[BETA ? 512 : 1];
   const float half = silu ? 0.5f : 1.0f;
-  unsigned long long hg[GPL][4], hb[GPL][4];
-#pragma unroll
-  for (int k = 0; k < GPL; ++k) {
-    const int g = sub + k * lpv;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      hg[k][q] = f2_make(half * __ldg(gamma + g * 8 + 2 * q), half * __ldg(gamma + g * 8 + 2 * q + 1));
-      hb[k][q] = beta ? f2_make(half * __ldg(beta + g * 8 + 2 * q), half * __ldg(beta + g * 8 + 2 * q + 1))
-                      : 0ull;
-    }
+  for (int i = threadIdx.x; i < c / 2; i += blockDim.x) {
+    s_g[i] = f2_make(half * __ldg(gamma + 2 * i), half * __ldg(gamma + 2 * i + 1));
+    if (BETA) s_b[i] = f2_make(half * __ldg(beta + 2 * i), half * __ldg(beta + 2 * i + 1));
   }
+  __syncthreads();
   for (long long vb = warp0 * vpw * UNR; vb < voxels; vb += nwarps * vpw * UNR) {
     uint4 raw[UNR][GPL];
 #pragma unroll
@@ -332,7 +330,8 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           // h = x / rms * gamma (+ beta), halved when SiLU follows
-          const unsigned long long h = f2_fma(f2_mul(f2_from_bf16x2(w4[q]), inv2), hg[k][q], hb[k][q]);
+          const unsigned long long h =
+              f2_fma(f2_mul(f2_from_bf16x2(w4[q]), inv2), s_g[g * 4 + q], BETA ? s_b[g * 4 + q] : 0ull);
           float h0, h1;
           f2_split(h, h0, h1);
           if (silu) {
@@ -574,10 +573,16 @@ cudaError_t launch_rmsnorm_silu(const __nv_bfloat16 *x, const float *gamma, cons
     if (g < 1) g = 1;
     const int grid = static_cast<int>(g);
     switch (gpl) {
-      case 1: rmsnorm_silu_lanes_kernel<1, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache, silu); break;
-      case 2: rmsnorm_silu_lanes_kernel<2, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache, silu); break;
-      case 3: rmsnorm_silu_lanes_kernel<3, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache, silu); break;
-      default: rmsnorm_silu_lanes_kernel<4, kUnr><<<grid, 256, 0, stream>>>(x, gamma, beta, voxels, c, lpv, y, cache, silu); break;
+#define CC3D_RMS_LANES(G)                                                                     \
+  (beta ? rmsnorm_silu_lanes_kernel<G, kUnr, true><<<grid, 256, 0, stream>>>(                  \
+              x, gamma, beta, voxels, c, lpv, y, cache, silu)                                   \
+        : rmsnorm_silu_lanes_kernel<G, kUnr, false><<<grid, 256, 0, stream>>>(                 \
+              x, gamma, beta, voxels, c, lpv, y, cache, silu))
+      case 1: CC3D_RMS_LANES(1); break;
+      case 2: CC3D_RMS_LANES(2); break;
+      case 3: CC3D_RMS_LANES(3); break;
+      default: CC3D_RMS_LANES(4); break;
+#undef CC3D_RMS_LANES
     }
   } else {
     constexpr int kCpt = 12;  // 16-byte chunks per thread and pass
