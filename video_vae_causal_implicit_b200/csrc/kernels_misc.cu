@@ -260,17 +260,18 @@ __device__ __forceinline__ unsigned long long f2_from_bf16x2(uint32_t u) {
 // each lane owning GPL groups (GPL = c / 8 / LPV, e.g. C = 192: 8 lanes x 3
 // groups, four voxels per warp).  A warp's loads cover 32 * GPL consecutive
 // 16-byte chunks (fully coalesced, every lane busy); UNR warp passes are
-// loaded before any is used.  Gamma (and beta, when given) sit in shared
-// memory as pre-halved fp32 pairs, which keeps the thread at 80 registers:
-// three CTAs per SM, 24 warps to cover the loads' latency (with them in
-// registers, two CTAs of 128-register threads).  The arithmetic runs on
+// loaded before any is used (one: more warps cover the loads' latency
+// better than more passes per warp).  Gamma (and beta, when given) sit in
+// shared memory as pre-halved fp32 pairs, which keeps the thread at 64
+// registers: four CTAs per SM, 32 warps (with them in registers and two
+// passes, two CTAs of 128-register threads).  The arithmetic runs on
 // packed fp32 pairs (the kernel issues about as many instructions as it
 // moves bytes, so halving the multiplies and adds shows).  The sum of
 // squares is kept as two pair halves, added, then reduced with a fixed xor
 // butterfly over the LPV lanes, so the result does not depend on
 // scheduling.
 template <int GPL, int UNR, bool BETA>
-__global__ void __launch_bounds__(256, 3)
+__global__ void __launch_bounds__(256, UNR == 1 ? 4 : 3)
     rmsnorm_silu_lanes_kernel(const __nv_bfloat16 *__restrict__ x,
                               const float *__restrict__ gamma, const float *__restrict__ beta,
                               long long voxels, int c, int lpv,
@@ -565,7 +566,7 @@ cudaError_t launch_rmsnorm_silu(const __nv_bfloat16 *x, const float *gamma, cons
   while (lpv < 32 && groups % (lpv * 2) == 0) lpv *= 2;
   const int gpl = groups / lpv;
   if (gpl <= 4) {
-    constexpr int kUnr = 2;
+    constexpr int kUnr = 1;
     const long long per_warp = static_cast<long long>(32 / lpv) * kUnr;
     long long warps = (voxels + per_warp - 1) / per_warp;
     long long g = (warps * 32 + 255) / 256;
