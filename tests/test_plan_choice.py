@@ -90,8 +90,14 @@ def test_every_plan_fits_the_sm(probe):
 def test_slots_pair_and_resident_only_where_valid(probe):
     for c, p in zip(GRID, probe(GRID)):
         n, ci, co, h, w, kt, ks, rms, mt, sms, f8 = c
-        # a weight slot holds one tap, or one whole kernel row of taps
-        assert p["g_taps"] in (1, ks), (c, p)
+        # a weight slot holds one tap, or one whole kernel row of taps, or
+        # (a 1 x 1 kernel with streamed weights) two channel chunks beside a
+        # halo group of two slots
+        if ks == 1 and p["g_taps"] == 2:
+            assert not p["b_resident"] and (ci // p["kc"]) % 2 == 0 and p["na"] % 2 == 0, (c, p)
+            assert p["na"] >= 4 and p["nb"] >= 3, (c, p)
+        else:
+            assert p["g_taps"] in (1, ks), (c, p)
         if p["pair"]:
             assert p["kc"] == 64 and p["sub"] == 2 and p["ctas_per_sm"] == 1, (c, p)
         if p["b_resident"]:

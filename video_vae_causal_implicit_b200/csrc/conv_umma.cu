@@ -312,15 +312,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   // consecutive A slots) share the first slot's full and empty barriers, one
   // wait and one commit per group.  (With streamed weights the longer groups
   // keep fewer halos in flight and cost more than they save.)
+  // With streamed weights the plan may group them the same way: g_taps (2
+  // or 3) consecutive chunks share one weight slot of g_taps stages beside
+  // a group of as many halo slots (b_grouped).
+  const bool b_grouped = KS == 1 && !p.b_resident && n_sc == 0 && p.g_taps > 1;
   const int a_grp = (KS == 1 && p.b_resident && n_sc == 0)
                         ? ((n_cc % 3 == 0 && L.na % 3 == 0)   ? 3
                            : (n_cc % 2 == 0 && L.na % 2 == 0) ? 2
                                                               : 1)
-                        : 1;
+                        : (b_grouped ? p.g_taps : 1);
   const int stages_per_ntile = n_conv_stages + n_sc;  // weight image
   // weight slots per A stage: one per group of g_taps spatial taps
   const int g_taps = p.g_taps;
-  const int n_groups = KS * KS / g_taps;
+  const int n_groups = b_grouped ? 1 : KS * KS / g_taps;
   constexpr bool kSw = uses_sw128(KC);
   const uint32_t halo_w = static_cast<uint32_t>(halo_cols(KC, SUB, KS));
   const int n_tiles = p.n * p.t * p.tiles_h * p.tiles_w * p.n_ntiles;
@@ -462,6 +466,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // the weight slots of a group of A stages (chunks cc0 .. of frame kt)
       auto load_weights = [&](int kt, int cc0, const TileCoord &tc0) -> bool {
+        if (b_grouped) {
+          // one slot: the stages (kt, cc0 .. cc0 + a_grp - 1) of the 1 x 1 kernel
+          if (!mbar_wait_bounded(&empty_b[sb], pb ^ 1, p.wait_limit_ns, p.status, 2)) return false;
+          arm_b(sb, a_grp);
+          for (int v = 0; v < a_grp; ++v)
+            load_b(sb, v, static_cast<size_t>(kt) * n_cc + cc0 + v, tc0.ntile);
+          if (++sb == L.nb) { sb = 0; pb ^= 1; }
+          return true;
+        }
         for (int u = 0; u < a_grp; ++u) {
           const int cc = cc0 + u;
           // this A stage's weight slots: g_taps consecutive taps each (a
@@ -498,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool streamed = !(KS == 1 && p.b_resident);
           const bool early_w =
               !dep_waited && streamed &&
-              a_grp * (phases ? phase_tap_count(kt) : n_groups) <= L.nb;
+              (b_grouped ? 1 : a_grp * (phases ? phase_tap_count(kt) : n_groups)) <= L.nb;
           if (early_w && !load_weights(kt, cc0, tc0)) {
             ok = false;
             break;
@@ -675,6 +688,19 @@ __global__ void __launch_bounds__(kThreads, 1)
               b_seen |= 1u << is;
             }
             mma_stage(a_st, bdesc0 + static_cast<uint32_t>(is) * bslot16, 0);
+          } else if (b_grouped) {
+            // the group's weight slot: stage u of it against halo slot sa + u
+            if (u == 0 && !mbar_wait_bounded(&full_b[sb], pb, p.wait_limit_ns, p.status, 4)) {
+              ok = false;
+              break;
+            }
+            mma_stage(a_st, bdesc0 + static_cast<uint32_t>(sb) * bslot16 +
+                                static_cast<uint32_t>(u) * bstage16,
+                      0);
+            if (u == a_grp - 1) {
+              release(&empty_b[sb]);
+              if (++sb == L.nb) { sb = 0; pb ^= 1; }
+            }
           } else {
             const int q = is / n_cc;  // (a phase stage's phase)
             const int n_w = phases ? phase_tap_count(q) : n_groups;
@@ -1097,6 +1123,22 @@ bool finish_config(int ks, int kt, int c_in, UmmaConfig &c) {
     c.na = 8;
     const size_t budget = 200 * 1024 + 4 * static_cast<size_t>(c.params);
     while (c.nb > 2 && smem(c.na, c.nb, 1) > budget) c.na = --c.nb;
+    // Two channel chunks per weight slot and per halo group (one wait and
+    // one commit per 2 * KC / 16 MMAs instead of per KC / 16) when the
+    // chunks pair up and at least three such slots fit beside two halo
+    // groups (the deepest of these ring shapes that fits).
+    const int n_cc = c_in / c.kc;
+    if (n_cc % 2 == 0) {
+      const int shapes[5][2] = {{8, 4}, {6, 4}, {8, 3}, {6, 3}, {4, 3}};
+      for (const auto &s : shapes) {
+        if (smem(s[0], s[1], 2) <= budget) {
+          c.g_taps = 2;
+          c.na = s[0];
+          c.nb = s[1];
+          break;
+        }
+      }
+    }
   } else if (ks == 2) {
     // the stride-2 phase conv: a phase halo serves one to four taps, each
     // tap a weight slot of its own
@@ -1128,6 +1170,7 @@ bool finish_config(int ks, int kt, int c_in, UmmaConfig &c) {
     while (na > 3 && smem(na, stages, 1) > budget_r) --na;
     if (smem(na, stages, 1) <= budget_r) {
       c.b_resident = 1;
+      c.g_taps = 1;
       c.na = na;
       c.nb = stages;
     }
@@ -1400,7 +1443,12 @@ cudaError_t launch_conv_umma(const CUtensorMap &map_x, const CUtensorMap &map_ca
                              const UmmaArgs &args, int kc, unsigned grid, cudaStream_t stream) {
   if (args.kh != args.kw || (args.kh != 1 && args.kh != 3 && !(args.kh == 2 && args.s2)))
     return cudaErrorInvalidValue;
-  if (args.g_taps != 1 && args.g_taps != args.kw) return cudaErrorInvalidValue;
+  // weight slots: one tap, one kernel row, or (a 1 x 1 kernel with streamed
+  // weights) g_taps channel chunks beside as many halo slots
+  const bool chunk_slots = args.kh == 1 && args.g_taps > 1 && !args.b_resident &&
+                           args.c_sc == 0 && (args.c_in / kc) % args.g_taps == 0 &&
+                           args.na % args.g_taps == 0 && args.g_taps <= 3;
+  if (args.g_taps != 1 && args.g_taps != args.kw && !chunk_slots) return cudaErrorInvalidValue;
   // the stride-2 phase conv: four phase stages per channel chunk, one tap
   // per weight slot
   if (args.kh == 2 && (args.kt != 4 || args.g_taps != 1 || args.b_resident))
