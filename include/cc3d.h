@@ -324,7 +324,7 @@ cc3d_status cc3d_resblock_forward(cc3d_block *block, const void *x, int t,
  *                (x is still read: residual or conv_shortcut input), and
  *                cache1_out is written by conv1 from cache1_in and a0_in.
  *   g_next       nullable: device [c_out] fp32, the next block's g1.  With
- *                it, conv2's epilogue writes y (unchanged) and also
+ *                it, the call writes y (unchanged) and also
  *   a0_next      [n][t][h][w][c_out] = SiLU(RMS_norm(y; g_next)), computed
  *                from y rounded to bf16, with its history
  *   a0_next_cache_in / a0_next_cache_out  nullable, [n][2][h][w][c_out]:
@@ -334,7 +334,8 @@ cc3d_status cc3d_resblock_forward(cc3d_block *block, const void *x, int t,
  * rounding order of the fused norm's sum of squares.  a0_next without
  * g_next, or the reverse, or a0_next_cache_* without them, is
  * CC3D_ERR_INVALID_ARG; a0_next must not overlap x, y, a0_in or any cache
- * (CC3D_ERR_ALIAS). */
+ * (CC3D_ERR_ALIAS); x, y, a0_in and a0_next are 16-byte aligned
+ * (CC3D_ERR_ALIGNMENT).  Every check runs before any launch. */
 cc3d_status cc3d_resblock_forward_fused(cc3d_block *block, const void *x,
                                         const void *a0_in, int t,
                                         const void *cache1_in,
