@@ -334,8 +334,8 @@ cc3d_status cc3d_resblock_forward(cc3d_block *block, const void *x, int t,
  * rounding order of the fused norm's sum of squares.  a0_next without
  * g_next, or the reverse, or a0_next_cache_* without them, is
  * CC3D_ERR_INVALID_ARG; a0_next must not overlap x, y, a0_in or any cache
- * (CC3D_ERR_ALIAS); x, y, a0_in and a0_next are 16-byte aligned
- * (CC3D_ERR_ALIGNMENT).  Every check runs before any launch. */
+ * (CC3D_ERR_ALIAS); every pointer is 16-byte aligned (CC3D_ERR_ALIGNMENT).
+ * These checks run before any launch. */
 cc3d_status cc3d_resblock_forward_fused(cc3d_block *block, const void *x,
                                         const void *a0_in, int t,
                                         const void *cache1_in,

@@ -176,6 +176,13 @@ def test_fused_chain_refusals():
                  nul, nul) == cc3d.ERR_ALIAS
     assert fused(b0.handle, ptr(x), nul, t, nul, nul, ptr(y), nul, nul, ptr(b1.g1), ptr(y), nul,
                  nul, nul) == cc3d.ERR_ALIAS
+    # the hand-over history written over its own input, a cache that is not
+    # 16-byte aligned: refused before anything runs as well
+    hist = torch.empty((n, 2, h, w, 64), dtype=torch.bfloat16, device="cuda")
+    assert fused(b0.handle, ptr(x), nul, t, nul, nul, ptr(y), nul, nul, ptr(b1.g1), ptr(a),
+                 ptr(hist), ptr(hist), nul) == cc3d.ERR_ALIAS
+    assert fused(b0.handle, ptr(x), nul, t, nul, ptr(hist) + 2, ptr(y), nul, nul, ptr(b1.g1),
+                 ptr(a), nul, nul, nul) == cc3d.ERR_ALIGNMENT
     assert cc3d.cc3d_launch_count() == before
     cc3d.sync_status()
     for b in (b0, b1):

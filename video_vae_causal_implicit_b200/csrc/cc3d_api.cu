@@ -1146,14 +1146,19 @@ cc3d_status cc3d_resblock_forward_fused(cc3d_block *b, const void *x, const void
       overlaps(cache1_out, c1, cache2_out, c2) || overlaps(cache1_out, c1, cache2_in, c2) ||
       overlaps(cache2_out, c2, cache1_in, c1) || overlaps(cache1_out, c1, a0_in, xb))
     return CC3D_ERR_ALIAS;
-  if (!aligned16(x) || !aligned16(y) || !aligned16(a0_in) || !aligned16(a0_next))
+  if (!aligned16(x) || !aligned16(y) || !aligned16(a0_in) || !aligned16(a0_next) ||
+      !aligned16(cache1_in) || !aligned16(cache1_out) || !aligned16(cache2_in) ||
+      !aligned16(cache2_out) || !aligned16(a0_next_cache_in) || !aligned16(a0_next_cache_out))
     return CC3D_ERR_ALIGNMENT;
   if (overlaps(a0_next, yb, x, xb) || overlaps(a0_next, yb, y, yb) ||
       overlaps(a0_next, yb, a0_in, xb) ||
       overlaps(a0_next, yb, cache1_in, c1) || overlaps(a0_next, yb, cache1_out, c1) ||
       overlaps(a0_next, yb, cache2_in, c2) || overlaps(a0_next, yb, cache2_out, c2) ||
       overlaps(a0_next_cache_out, c2, cache1_out, c1) ||
-      overlaps(a0_next_cache_out, c2, cache2_out, c2))
+      overlaps(a0_next_cache_out, c2, cache2_out, c2) ||
+      overlaps(a0_next_cache_out, c2, a0_next_cache_in, c2) ||
+      overlaps(a0_next_cache_out, c2, a0_next, yb) || overlaps(a0_next_cache_out, c2, y, yb) ||
+      overlaps(a0_next_cache_out, c2, x, xb))
     return CC3D_ERR_ALIAS;
   cc3d_status s = CC3D_OK;
   // a0 = SiLU(RMS(x; g1)), unless the previous block's conv2 produced it;
