@@ -508,7 +508,8 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        pts = 2048
+        # a bounded sample of the workload: about 10 s of the host cores' time
+        pts = 16384
         rate, dt, fl = oracle_sample_rate(pts)
         cpu = {"value": rate, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
                "kind": "oracle", "seconds": dt,
