@@ -1144,7 +1144,8 @@ cc3d_status cc3d_resblock_forward_fused(cc3d_block *b, const void *x, const void
       overlaps(cache1_out, c1, x, xb) || overlaps(cache1_out, c1, y, yb) ||
       overlaps(cache2_out, c2, x, xb) || overlaps(cache2_out, c2, y, yb) ||
       overlaps(cache1_out, c1, cache2_out, c2) || overlaps(cache1_out, c1, cache2_in, c2) ||
-      overlaps(cache2_out, c2, cache1_in, c1) || overlaps(cache1_out, c1, a0_in, xb))
+      overlaps(cache2_out, c2, cache1_in, c1) || overlaps(cache1_out, c1, a0_in, xb) ||
+      overlaps(cache2_out, c2, a0_in, xb))
     return CC3D_ERR_ALIAS;
   if (!aligned16(x) || !aligned16(y) || !aligned16(a0_in) || !aligned16(a0_next) ||
       !aligned16(cache1_in) || !aligned16(cache1_out) || !aligned16(cache2_in) ||
