@@ -215,3 +215,15 @@ def test_uncached_whole_sequence_takes_the_pair_tiles(deal):
     assert (unc["pair_plan"], unc["pair_one"]) == (0, 1)
     assert unc["one"] < unc["plan"]
     assert cac["one"] > cac["plan"]
+
+
+def test_serpentine_deal_pairs_spare_units_with_cheap_ones(deal):
+    """80 pair units on 74 clusters, dealt last frame first: 48 full units
+    (3 live taps), 16 of frame 1 (2 taps), 16 of frame 0 (1 tap).  The
+    serpentine deal gives the 6 spare frame-0 units to the clusters that
+    drew frame-0 units in the first round, so the makespan is one full unit
+    -- the cost of one cached frame, whose units all run at once.  A plain
+    round-robin deal would give them to clusters with full units (4 taps)."""
+    unc5, cac1 = deal([dcase(cached=False, t_out=5), dcase(cached=True, t_out=1)])
+    assert (unc5["pair_one"], cac1["pair_one"]) == (1, 1)
+    assert unc5["one"] == cac1["one"]
