@@ -610,10 +610,28 @@ def run_sweep(args, dev, stream, peaks, flush_l2, full=False):
             ts.append(a.elapsed_time(b))
         return statistics.median(ts)
 
-    # config 3a: 3 -> 96 at 17 x 480 x 832 (HBM-bound on the output write)
-    T, H, W = 17, 480, 832
     g = torch.Generator(device=dev)
     g.manual_seed(0)
+    # config 1: the fp32 causal conv, 16 -> 16 on x[1,16,5,16,16] (SIMT FFMA;
+    # a launch-latency-bound 17.7 MFLOP, reported in microseconds)
+    c1 = synth.conv_case(16, 16, 5, 16, 16, dtype=torch.float32)
+    p1 = cc3d.Plan(c1["w"].to(dev), c1["b"].to(dev), h=16, w=16, max_t=5, dtype=cc3d.FP32)
+    x1 = synth.ndhwc(c1["x"]).to(dev)
+    y1 = torch.empty((1, 5, 16, 16, 16), dtype=torch.float32, device=dev)
+    # the device time of one call (captured once as a CUDA graph and
+    # replayed: a single call's events would mostly time the host's call
+    # path, which is reported beside it)
+    host_ms = timed(lambda: p1.forward(x1, y1))
+    g1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1):
+        p1.forward(x1, y1)
+    ms = timed(g1.replay)
+    out["cfg1_fp32_16to16_5x16x16"] = {"us": ms * 1e3,
+                                       "gflops": conv_flop(1, 16, 16, 5, 16, 16) / ms / 1e6,
+                                       "us_one_host_call": host_ms * 1e3}
+    del g1, p1, x1, y1
+    # config 3a: 3 -> 96 at 17 x 480 x 832 (HBM-bound on the output write)
+    T, H, W = 17, 480, 832
     x3 = (torch.rand((1, T, H, W, 3), generator=g, device=dev) * 2 - 1).to(torch.bfloat16)
     w3 = synth.kaiming_uniform(96, 3, (3, 3, 3), 1).to(dev)
     b3 = synth.uniform((96,), -0.1, 0.1, 2).to(dev)
